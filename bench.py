@@ -1,0 +1,394 @@
+"""Benchmark of the CARVE chunk-parallel recurrent core on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--mode train|fwd]
+                    [--workload layer_1p3b|long_context|tiny] [--impl carve|reference]
+
+One step = one pass of the whole hot path over one batch: the training-mode
+forward (chunk walk, gate, WY solve, state update, checkpoints) plus the
+backward (reverse chunk walk and the U_b gradient reduction) -- or the
+forward alone with --mode fwd.  Inputs are synthetic (seeded, the
+distributions of chunk_gated_delta_02_b200/inputs.py) and resident in HBM
+when the timed region starts; they are larger than the 126 MB L2.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
+the same shape (independent sequences, no data-path collective) -> weak
+scaling; the time is the max over ranks.
+
+Prints ONE JSON line on rank 0.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+from chunk_gated_delta_02_b200.inputs import (WORKLOADS, make_grad_outputs,  # noqa: E402
+                                              make_inputs)
+
+METRIC = "CARVE chunk fwd / fwd+bwd tokens/s on 1 B200; % of roofline"
+
+
+def peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d["bf16_tflops_sustained"]),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+# Algorithmic work per token per head (K = DK, V = DV, e = element bytes):
+# FLOPs are the chunk contractions at full L x L tiles; bytes are the
+# compulsory tensor traffic (inputs read once, outputs written once).
+def fwd_flops(L, K, V):
+    return 8 * L * K + 8 * K * V + 8 * L * V
+
+
+def bwd_flops(L, K, V):
+    return 24 * L * K + 18 * K * V + 20 * L * V
+
+
+def fwd_bytes(K, V, e):
+    return e * (4 * K + 2 * V + 1)      # q k g bx v w in, o out
+
+
+def bwd_bytes(K, V, e):
+    return e * (8 * K + 3 * V + 2)      # q k g bx v w d_o in, 6 grads out
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        self.rows = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            self.sel = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "200"] + self.sel,
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
+        rows = [r for r in rows if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4)
+                          if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_init():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120),
+            device_id=torch.device("cuda", local))
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample(cfg, mode, seed, threads=None):
+    """Time the fp64 oracle on a bounded sample of the workload: `n` whole
+    (sequence, head) pairs at the full sequence length.  Returns
+    (seconds, pair_tokens, n_pairs, threads)."""
+    from oracle import ref
+    n = threads or max(1, len(os.sched_getaffinity(0)))
+    n = min(n, 16, cfg["B"] * cfg["H"])
+    inp = make_inputs(seed=seed, dtype=torch.bfloat16,
+                      **dict(cfg, B=1, H=n))
+    gro = make_grad_outputs(seed=seed, dtype=torch.bfloat16,
+                            **dict(cfg, B=1, H=n))
+    pairs = [(0, h) for h in range(n)]
+    ref.fwd_batch(inp, cfg["L"], pairs=pairs[:1], threads=1)  # load/build
+    t0 = time.perf_counter()
+    if mode == "fwd":
+        ref.fwd_batch(inp, cfg["L"], pairs=pairs, threads=n)
+    else:
+        ref.bwd_batch(inp, cfg["L"], gro["d_o"], pairs=pairs, threads=n)
+    dt = time.perf_counter() - t0
+    return dt, n * cfg["T"], n, n
+
+
+def run_reference(args, cfg, ws, rank):
+    """The oracle as the reference arm (CPU, host cores)."""
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_sample(cfg, args.mode, 100)
+    secs, ptoks, npairs, thr = 0.0, 0, 0, 0
+    for i in range(args.steps):
+        s, p, npairs, thr = oracle_sample(cfg, args.mode, 200 + i)
+        secs += s
+        ptoks += p
+    value = ptoks / cfg["H"] / secs
+    sample = ("%d (sequence, head) pairs x %d tokens per step, %s, fp64; "
+              "tokens = pair-tokens / H" % (npairs, cfg["T"],
+                                            "fwd+bwd" if args.mode == "train"
+                                            else "fwd"))
+    line = {"impl": "reference", "metric": METRIC, "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": config_dict(args, cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s",
+                    "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(args, cfg):
+    return {"workload": "%s %s" % (args.workload,
+                                   "fwd+bwd" if args.mode == "train" else "fwd"),
+            "B": cfg["B"], "T": cfg["T"], "H": cfg["H"], "DK": cfg["DK"],
+            "DV": cfg["DV"], "L": cfg["L"], "R": cfg["R"],
+            "state": "fp32", "l2": "inputs larger than L2 (no flush needed)",
+            "parallelism": "independent sequences per rank (dp%d)" % args.gpus}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--mode", choices=["train", "fwd"], default="train")
+    ap.add_argument("--workload", default="layer_1p3b", choices=list(WORKLOADS))
+    ap.add_argument("--impl", choices=["carve", "reference"], default="carve")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "carve":
+        ap.error("--warmup must be >= 3")
+    cfg = dict(WORKLOADS[args.workload])
+    ws, rank, local = dist_init() if args.impl == "carve" else (
+        int(os.environ.get("WORLD_SIZE", "1")),
+        int(os.environ.get("RANK", "0")), 0)
+    if args.impl == "reference":
+        run_reference(args, cfg, ws, rank)
+        return
+
+    from chunk_gated_delta_02_b200 import carve
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dtype = torch.bfloat16
+    B, T, H, DK, DV, R, L = (cfg[n] for n in ("B", "T", "H", "DK", "DV", "R",
+                                              "L"))
+    inp = make_inputs(seed=1000 + rank, dtype=dtype, **cfg)
+    gro = make_grad_outputs(seed=1000 + rank, dtype=dtype, **cfg)
+    host = {k: v for k, v in inp.items() if v is not None}
+    host["d_o"] = gro["d_o"]
+    d = {k: v.to(dev) for k, v in host.items()}
+    d.setdefault("S0", None)
+    training = args.mode == "train"
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd(ws_buf=None, o=None):
+        return carve.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["bx"],
+                               d["w"], d["u_down"], d["u_up"], L, d.get("S0"),
+                               None, training=training, workspace=ws_buf, o=o)
+
+    o, S_T, m_T, wsb = fwd()
+    grads = None
+    if training:
+        grads = carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"],
+                                d["w"], d["u_down"], d["u_up"], L, d["d_o"],
+                                wsb)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record(stream)
+        carve.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
+                        d["u_down"], d["u_up"], L, d.get("S0"), None,
+                        training=training, workspace=wsb, o=o,
+                        want_state=False)
+        if ev:
+            ev[1].record(stream)
+        if training:
+            carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
+                            d["u_down"], d["u_up"], L, d["d_o"], wsb,
+                            out=grads)
+        if ev:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert carve.get_status(wsb) == 0, "device status word set"
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+           for _ in range(args.steps)]
+    clocks = ClockSampler(dev) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop() if clocks else None
+    total_ms = t_start.elapsed_time(t_end)
+    total_ms = max_over_ranks(total_ms, ws)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    bwd_ms = (sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+              if training else 0.0)
+    assert carve.get_status(wsb) == 0, "device status word set"
+
+    ms_step = total_ms / args.steps
+    tokens = B * T
+    value = tokens * ws / (ms_step * 1e-3)
+
+    # roofline of the dominant kernel (fwd or bwd), HBM-bound
+    pk = peaks()
+    e = 2
+    fwd_b = fwd_bytes(DK, DV, e) * B * T * H
+    bwd_b = bwd_bytes(DK, DV, e) * B * T * H
+    fwd_f = fwd_flops(L, DK, DV) * B * T * H
+    bwd_f = bwd_flops(L, DK, DV) * B * T * H
+    if training and bwd_ms >= fwd_ms:
+        dom, dom_ms, dom_b, dom_f = "bwd", bwd_ms, bwd_b, bwd_f
+    else:
+        dom, dom_ms, dom_b, dom_f = "fwd", fwd_ms, fwd_b, fwd_f
+    peak = pk["hbm"] if dom == "fwd" else pk["hbm"]
+    achieved = dom_b / (dom_ms * 1e-3) / 1e9
+    roof_t_fwd = max(fwd_f / (pk["bf16"] * 1e12), fwd_b / (pk["hbm"] * 1e9))
+    roof_t_all = max((fwd_f + (bwd_f if training else 0)) / (pk["bf16"] * 1e12),
+                     (fwd_b + (bwd_b if training else 0)) / (pk["hbm"] * 1e9))
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic (seeded; inputs.py distributions)",
+        "config": config_dict(args, cfg),
+        "kernel_path": carve.fwd_path(carve.make_shape(B, T, H, DK, DV, R, L,
+                                                       dtype)),
+        "roofline": {"bound": "hbm", "kernel": "carve_chunk_" + dom,
+                     "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_src": pk["src"] + " hbm_gbs",
+                     "algorithmic_bytes": dom_b, "algorithmic_flops": dom_f,
+                     "ms_per_launch": dom_ms},
+        "step_roofline": {"roofline_ms": roof_t_all * 1e3,
+                          "frac": roof_t_all * 1e3 / ms_step},
+        "fwd": {"ms": fwd_ms, "tokens_per_s": tokens / (fwd_ms * 1e-3),
+                "roofline_ms": roof_t_fwd * 1e3,
+                "frac": roof_t_fwd * 1e3 / fwd_ms},
+        "bwd": {"ms": bwd_ms} if training else None,
+        "gpu_launches": args.steps * (3 if training else 1),
+        "clocks": clk,
+    }
+
+    # end to end through the public API: pinned host inputs -> device, step,
+    # results -> pinned host, all inside the timed region
+    if not args.no_e2e:
+        pin = {k: v.pin_memory() for k, v in host.items()}
+        outs_host = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory()}
+        if training:
+            for k, v in grads.items():
+                if v is not None:
+                    outs_host[k] = torch.empty(v.shape, dtype=v.dtype).pin_memory()
+        h2d = sum(v.numel() * v.element_size() for v in pin.values())
+        d2h = sum(v.numel() * v.element_size() for v in outs_host.values())
+
+        def e2e_step():
+            for k, v in pin.items():
+                d[k].copy_(v, non_blocking=True)
+            step()
+            outs_host["o"].copy_(o, non_blocking=True)
+            if training:
+                for k, v in grads.items():
+                    if v is not None:
+                        outs_host[k].copy_(v, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        a, b = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+        n_e2e = max(3, args.steps // 2)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, ws)
+        line["e2e"] = {"value": tokens * ws / (e2e_ms * 1e-3),
+                       "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        secs, ptoks, npairs, thr = oracle_sample(cfg, args.mode, 7)
+        line["cpu_baseline"] = {
+            "value": ptoks / H / secs, "unit": "tokens/s", "cores": thr,
+            "kind": "oracle",
+            "sample": "%d (sequence, head) pairs x %d tokens, %s, fp64; "
+                      "tokens = pair-tokens / H" % (
+                          npairs, T, "fwd+bwd" if training else "fwd")}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

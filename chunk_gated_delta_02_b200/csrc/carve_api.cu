@@ -1,0 +1,169 @@
+// carve_api.cu -- the C ABI of libcarve: validation, workspace layout and
+// kernel dispatch.  Declared in include/carve.h.
+#include <string.h>
+
+#include "carve_internal.cuh"
+
+using namespace carve;
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+carve_status check_shape(const carve_shape* s) {
+  if (!s) return CARVE_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->T < 0 || s->R < 0 || s->L < 1 ||
+      s->DK < 1 || s->DV < 1)
+    return CARVE_ERR_INVALID_ARG;
+  if (s->dtype != CARVE_BF16 && s->dtype != CARVE_FP32)
+    return CARVE_ERR_INVALID_ARG;
+  if (s->DK % 16 || s->DV % 16 || s->DK > 256 || s->DV > 256)
+    return CARVE_ERR_UNSUPPORTED;
+  if (s->R > kMaxR) return CARVE_ERR_UNSUPPORTED;
+  if (!(s->L <= kMaxBlock || (s->L % kMaxBlock == 0 && s->L <= 256)))
+    return CARVE_ERR_UNSUPPORTED;
+  if (s->T % s->L) return CARVE_ERR_UNSUPPORTED;
+  // all element indices are computed in 64-bit; grid is B*H CTAs
+  if ((long long)s->B * s->H > (1LL << 30)) return CARVE_ERR_UNSUPPORTED;
+  const int C = block_len(s->L);
+  if (generic_bwd_smem_bytes(C, s->DK, s->DV) > 227 * 1024)
+    return CARVE_ERR_UNSUPPORTED;
+  return CARVE_OK;
+}
+
+bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
+bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
+
+}  // namespace
+
+extern "C" {
+
+size_t carve_workspace_bytes(const carve_shape* shape, int training) {
+  if (check_shape(shape) != CARVE_OK) return 0;
+  return ws_layout(*shape, training != 0).total;
+}
+
+const char* carve_status_str(carve_status s) {
+  switch (s) {
+    case CARVE_OK: return "CARVE_OK";
+    case CARVE_ERR_INVALID_ARG: return "CARVE_ERR_INVALID_ARG";
+    case CARVE_ERR_UNSUPPORTED: return "CARVE_ERR_UNSUPPORTED";
+    case CARVE_ERR_WORKSPACE: return "CARVE_ERR_WORKSPACE";
+    case CARVE_ERR_CUDA: return "CARVE_ERR_CUDA";
+    case CARVE_ERR_TIMEOUT: return "CARVE_ERR_TIMEOUT";
+  }
+  return "CARVE_ERR_UNKNOWN";
+}
+
+const char* carve_fwd_path(const carve_shape* shape) {
+  if (check_shape(shape) != CARVE_OK) return nullptr;
+  return "generic";
+}
+
+carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
+                             const void* k, const void* v, const void* g,
+                             const void* b_x, const void* w,
+                             const void* u_down, const void* u_up,
+                             const float* S0, const float* m0, void* o,
+                             float* S_T, float* m_T, void* workspace,
+                             size_t workspace_bytes, int training,
+                             void* stream) {
+  carve_status st = check_shape(shape);
+  if (st != CARVE_OK) return st;
+  const carve_shape& s = *shape;
+  const bool tok = s.T > 0;
+  if (tok && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) ||
+              !ptr_ok(b_x) || !ptr_ok(w) || !ptr_ok(o)))
+    return CARVE_ERR_INVALID_ARG;
+  if (s.R > 0 && (!ptr_ok(u_down) || !ptr_ok(u_up)))
+    return CARVE_ERR_INVALID_ARG;
+  if (!opt_ptr_ok(S0) || !opt_ptr_ok(m0) || !opt_ptr_ok(S_T) ||
+      !opt_ptr_ok(m_T))
+    return CARVE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(s, training != 0);
+  if (!workspace || !aligned16(workspace)) return CARVE_ERR_WORKSPACE;
+  if (workspace_bytes < L.total) return CARVE_ERR_WORKSPACE;
+
+  char* ws = (char*)workspace;
+  FwdArgs a{};
+  a.B = s.B; a.T = s.T; a.H = s.H; a.DK = s.DK; a.DV = s.DV; a.R = s.R;
+  a.L = s.L; a.C = L.C; a.NB = L.NB; a.NC = L.NC;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.bx = b_x; a.w = w;
+  a.u_down = u_down; a.u_up = u_up; a.S0 = S0; a.m0 = m0;
+  a.o = o; a.S_T = S_T; a.m_T = m_T;
+  a.ck_S = training ? (float*)(ws + L.ck_S) : nullptr;
+  a.ck_m = training ? (float*)(ws + L.ck_m) : nullptr;
+  a.scratch = (float*)(ws + L.scratch);
+  a.scratch_per_pair = L.scratch_per_pair;
+  a.hdr = (WsHeader*)ws;
+  cudaError_t e = launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
+                             const void* k, const void* v, const void* g,
+                             const void* b_x, const void* w,
+                             const void* u_down, const void* u_up,
+                             const void* d_o, const float* dS_T,
+                             const float* dm_T, void* workspace,
+                             size_t workspace_bytes, void* dq, void* dk,
+                             void* dv, void* dg, void* db_x, void* dw,
+                             float* du_down, float* du_up, float* dS0,
+                             float* dm0, void* stream) {
+  carve_status st = check_shape(shape);
+  if (st != CARVE_OK) return st;
+  const carve_shape& s = *shape;
+  const bool tok = s.T > 0;
+  if (tok && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) ||
+              !ptr_ok(b_x) || !ptr_ok(w) || !ptr_ok(d_o) || !ptr_ok(dq) ||
+              !ptr_ok(dk) || !ptr_ok(dv) || !ptr_ok(dg) || !ptr_ok(db_x) ||
+              !ptr_ok(dw)))
+    return CARVE_ERR_INVALID_ARG;
+  if (s.R > 0 && (!ptr_ok(u_down) || !ptr_ok(u_up) || !ptr_ok(du_down) ||
+                  !ptr_ok(du_up)))
+    return CARVE_ERR_INVALID_ARG;
+  if (!opt_ptr_ok(dS_T) || !opt_ptr_ok(dm_T) || !opt_ptr_ok(dS0) ||
+      !opt_ptr_ok(dm0))
+    return CARVE_ERR_INVALID_ARG;
+  const WsLayout L = ws_layout(s, true);
+  if (!workspace || !aligned16(workspace)) return CARVE_ERR_WORKSPACE;
+  if (workspace_bytes < L.total) return CARVE_ERR_WORKSPACE;
+
+  char* ws = (char*)workspace;
+  BwdArgs a{};
+  a.B = s.B; a.T = s.T; a.H = s.H; a.DK = s.DK; a.DV = s.DV; a.R = s.R;
+  a.L = s.L; a.C = L.C; a.NB = L.NB; a.NC = L.NC;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.bx = b_x; a.w = w;
+  a.u_down = u_down; a.u_up = u_up; a.d_o = d_o; a.dS_T = dS_T; a.dm_T = dm_T;
+  a.ck_S = (const float*)(ws + L.ck_S);
+  a.ck_m = (const float*)(ws + L.ck_m);
+  a.scratch = (float*)(ws + L.scratch);
+  a.scratch_per_pair = L.scratch_per_pair;
+  a.du = (float*)(ws + L.du);
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbx = db_x; a.dw = dw;
+  a.du_down = du_down; a.du_up = du_up; a.dS0 = dS0; a.dm0 = dm0;
+  a.hdr = (WsHeader*)ws;
+  cudaError_t e = launch_bwd_generic(a, s.dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_get_status(const void* workspace, void* stream) {
+  if (!workspace) return CARVE_ERR_INVALID_ARG;
+  uint32_t word = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost,
+                      st) != cudaSuccess)
+    return CARVE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return CARVE_ERR_CUDA;
+  return (carve_status)word;
+}
+
+carve_status carve_reset_status(void* workspace, void* stream) {
+  if (!workspace) return CARVE_ERR_INVALID_ARG;
+  if (cudaMemsetAsync(workspace, 0, sizeof(uint32_t), (cudaStream_t)stream) !=
+      cudaSuccess)
+    return CARVE_ERR_CUDA;
+  return CARVE_OK;
+}
+
+}  // extern "C"

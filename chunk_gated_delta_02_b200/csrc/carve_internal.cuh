@@ -1,0 +1,124 @@
+// carve_internal.cuh -- shared definitions of libcarve's host and device code.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/carve.h"
+
+namespace carve {
+
+constexpr uint32_t kWsMagic = 0xCA7E0001u;
+constexpr size_t kHeaderBytes = 256;
+constexpr int kMaxR = 64;
+constexpr int kMaxBlock = 64;  // tokens per solver block (C = min(L, 64))
+
+// Device status word at the start of the workspace.
+struct WsHeader {
+  uint32_t status;   // carve_status written by kernels (sticky)
+  uint32_t magic;    // kWsMagic once a training forward wrote checkpoints
+  uint32_t where;    // diagnostic: which wait gave up
+  uint32_t pad[61];
+};
+static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
+
+// Layout of the workspace (byte offsets, 256-aligned).
+struct WsLayout {
+  int C;    // tokens per solver block
+  int NB;   // blocks per sequence
+  int NC;   // chunks per sequence
+  size_t ck_S;         // [B*H][NB+1][DV][DK] fp32 block-start states
+  size_t ck_m;         // [B*H][NC][DV] fp32 chunk gate inputs m_c
+  size_t scratch;      // per-pair fp32 scratch of the generic kernels
+  size_t scratch_per_pair;  // floats
+  size_t du;           // [B*H][R*DV + DK*R] fp32 per-pair U_b gradients
+  size_t total;
+};
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+inline int block_len(int L) { return L < kMaxBlock ? L : kMaxBlock; }
+
+inline size_t generic_fwd_scratch_floats(int C, int DK, int DV) {
+  return 4 * (size_t)C * DK + 4 * (size_t)C * DV + (size_t)DV * DK;
+}
+inline size_t generic_bwd_scratch_floats(int C, int DK, int DV) {
+  return 9 * (size_t)C * DK + 7 * (size_t)C * DV + 2 * (size_t)DV * DK;
+}
+
+inline WsLayout ws_layout(const carve_shape& s, bool training) {
+  WsLayout w{};
+  w.C = block_len(s.L);
+  w.NB = s.T / w.C;
+  w.NC = s.T / s.L;
+  const size_t P = (size_t)s.B * s.H;
+  size_t off = kHeaderBytes;
+  if (training) {
+    w.ck_S = off;
+    off = align256(off + P * (size_t)(w.NB + 1) * s.DV * s.DK * 4);
+    w.ck_m = off;
+    off = align256(off + P * (size_t)(w.NC > 0 ? w.NC : 1) * s.DV * 4);
+  }
+  size_t sc = generic_fwd_scratch_floats(w.C, s.DK, s.DV);
+  if (training) {
+    size_t sb = generic_bwd_scratch_floats(w.C, s.DK, s.DV);
+    sc = sc > sb ? sc : sb;
+  }
+  w.scratch_per_pair = sc;
+  w.scratch = off;
+  off = align256(off + P * sc * 4);
+  if (training) {
+    w.du = off;
+    off = align256(off + P * ((size_t)s.R * s.DV + (size_t)s.DK * s.R) * 4);
+  }
+  w.total = off;
+  return w;
+}
+
+// Element load/store in the I/O dtype, arithmetic in fp32.
+__device__ __forceinline__ float ldf(const float* p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ldf(const __nv_bfloat16* p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void stf(float* p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void stf(__nv_bfloat16* p, size_t i, float x) {
+  p[i] = __float2bfloat16_rn(x);
+}
+
+// Arguments of the forward kernels (pointers already validated).
+struct FwdArgs {
+  int B, T, H, DK, DV, R, L, C, NB, NC;
+  const void *q, *k, *v, *g, *bx, *w, *u_down, *u_up;
+  const float *S0, *m0;
+  void* o;
+  float *S_T, *m_T;
+  float* ck_S;     // NULL unless training
+  float* ck_m;     // NULL unless training
+  float* scratch;  // generic kernels only
+  size_t scratch_per_pair;
+  WsHeader* hdr;
+};
+
+struct BwdArgs {
+  int B, T, H, DK, DV, R, L, C, NB, NC;
+  const void *q, *k, *v, *g, *bx, *w, *u_down, *u_up;
+  const void* d_o;
+  const float *dS_T, *dm_T;
+  const float *ck_S, *ck_m;
+  float* scratch;
+  size_t scratch_per_pair;
+  float* du;  // per-pair partial U_b gradients
+  void *dq, *dk, *dv, *dg, *dbx, *dw;
+  float *du_down, *du_up, *dS0, *dm0;
+  WsHeader* hdr;
+};
+
+// Host launchers (carve_generic.cu).
+cudaError_t launch_fwd_generic(const FwdArgs& a, int dtype, cudaStream_t st);
+cudaError_t launch_bwd_generic(const BwdArgs& a, int dtype, cudaStream_t st);
+size_t generic_fwd_smem_bytes(int C, int DK, int DV);
+size_t generic_bwd_smem_bytes(int C, int DK, int DV);
+
+}  // namespace carve

@@ -1,0 +1,164 @@
+/*
+ * carve.h -- C ABI of libcarve, the B200 (sm_100a) implementation of the
+ * CARVE chunk-parallel recurrent core.
+ *
+ * The operation (one state per (sequence b, head h)); the pages' notation:
+ *
+ *   S_t = S_{t-1} Diag(exp g_t) (I - k_t (b_t (.) k_t)^T) + w_t v_t k_t^T
+ *   o_t = S_{t-1} q_t
+ *   b_{c,t} = sigmoid(b_x,t + U_b m_c),  U_b = U_up U_down  (rank R)
+ *   m_c = (1/L) sum of o_t over chunk c-1 (L tokens); chunk 0 uses m0 (or 0)
+ *
+ * Sources (CARVE: Content-Aware Recurrent with Value Efficiency for
+ * Chunk-Parallel Linear Attention, arXiv 2606.27229, as summarised on
+ * gist.science):
+ *   state S_t in R^{dv x dk} ............ technical summary section 1
+ *   o_t = S_{t-1} q_t, m_c, b_{c,t} ...... section 2.1 (content-aware erase
+ *                                          via output reuse)
+ *   scalar write gate w per head ......... section 2.2
+ *   exponential decay on the key axis .... section 2.3
+ *   erase on the key axis only, solved by
+ *   one WY triangular solve per chunk .... abstract; section 3 (Theorem 11)
+ *   no content signal in chunk 0 ......... section 5 (acknowledged limitation)
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are caller-owned DEVICE memory on the current
+ *     device, contiguous row-major in the layouts given, 16-byte aligned.
+ *   - The library never allocates, frees or synchronises (except
+ *     carve_get_status); work is enqueued on `stream` (a cudaStream_t; NULL
+ *     = legacy default stream) and the call returns immediately.
+ *   - Host-side validation failures return a status and enqueue nothing.
+ *   - "dtype" tensors are bf16 (CARVE_BF16) or fp32 (CARVE_FP32) as given in
+ *     carve_shape.dtype; the state, S0, S_T, m0, m_T and the U_b gradients
+ *     are always fp32.  Arithmetic is fp32 with fp32 accumulation.
+ */
+#ifndef CARVE_H_
+#define CARVE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CARVE_OK = 0,
+  CARVE_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size        */
+  CARVE_ERR_UNSUPPORTED = 2, /* shape outside the supported set (see below) */
+  CARVE_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
+  CARVE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed        */
+  CARVE_ERR_TIMEOUT = 5      /* a device-side bounded wait gave up          */
+} carve_status;
+
+typedef enum { CARVE_BF16 = 0, CARVE_FP32 = 1 } carve_dtype;
+
+/*
+ * Problem shape.  B sequences of T tokens, H heads, key width DK, value
+ * width DV, rank R of U_b, chunk length L.
+ * Supported: B, H >= 1; T >= 0 with T % L == 0; DK, DV multiples of 16 in
+ * [16, 256]; 0 <= R <= 64; L in [1, 64] or a multiple of 64 up to 256.
+ * Anything else returns CARVE_ERR_UNSUPPORTED.
+ */
+typedef struct {
+  int32_t B, T, H, DK, DV, R, L;
+  int32_t dtype; /* carve_dtype */
+} carve_shape;
+
+/*
+ * Bytes of device workspace carve_chunk_fwd / carve_chunk_bwd need for this
+ * shape.  training != 0 adds the per-block state checkpoints and per-chunk
+ * gate inputs that carve_chunk_bwd reads.  Returns 0 for an invalid or
+ * unsupported shape.  The workspace starts with a 256-byte header holding
+ * the device status word (see carve_get_status).
+ */
+size_t carve_workspace_bytes(const carve_shape* shape, int training);
+
+/*
+ * Forward pass over all chunks of all (b, h) pairs.
+ *
+ *   q, k, g, b_x : [B, T, H, DK] dtype   (g is the log-decay, g <= 0)
+ *   v            : [B, T, H, DV] dtype
+ *   w            : [B, T, H]     dtype   scalar write gate per token, head
+ *   u_down       : [H, R, DV]    dtype   U_b = u_up[h] @ u_down[h]
+ *   u_up         : [H, DK, R]    dtype   (may be NULL when R == 0)
+ *   S0           : [B, H, DV, DK] fp32, or NULL for zeros
+ *   m0           : [B, H, DV]     fp32, or NULL for zeros (the pages' rule:
+ *                  chunk 0 gets no content signal); a non-NULL m0 resumes a
+ *                  sequence split at a chunk boundary exactly
+ *   o            : [B, T, H, DV] dtype   (output, overwritten)
+ *   S_T          : [B, H, DV, DK] fp32 final state, or NULL
+ *   m_T          : [B, H, DV]     fp32 mean of the last chunk's outputs
+ *                  (the next call's m0), or NULL
+ *   workspace    : carve_workspace_bytes(shape, training) bytes
+ *   training     : nonzero to keep what carve_chunk_bwd needs in workspace
+ *
+ * Inputs and outputs must not overlap.  Errors: INVALID_ARG, UNSUPPORTED,
+ * WORKSPACE, CUDA (launch failure; the stream is left as CUDA left it).
+ */
+carve_status carve_chunk_fwd(const carve_shape* shape,
+                             const void* q, const void* k, const void* v,
+                             const void* g, const void* b_x, const void* w,
+                             const void* u_down, const void* u_up,
+                             const float* S0, const float* m0,
+                             void* o, float* S_T, float* m_T,
+                             void* workspace, size_t workspace_bytes,
+                             int training, void* stream);
+
+/*
+ * Backward pass: exact reverse mode of carve_chunk_fwd (the gradient also
+ * flows through the content gate into the previous chunk's outputs).
+ *
+ *   q ... u_up   : the same inputs given to the training-mode forward
+ *   workspace    : the workspace of that forward (training != 0), untouched
+ *                  since; it holds the block-start states, the chunk gate
+ *                  inputs and S0 / m0, so S0 and m0 are not passed again
+ *   d_o          : [B, T, H, DV] dtype upstream gradient of o
+ *   dS_T         : [B, H, DV, DK] fp32 upstream gradient of S_T, or NULL (0)
+ *   dm_T         : [B, H, DV] fp32 upstream gradient of m_T, or NULL (0)
+ *   dq, dk, dg, db_x : [B, T, H, DK] dtype (overwritten)
+ *   dv           : [B, T, H, DV] dtype   (overwritten)
+ *   dw           : [B, T, H]     dtype   (overwritten)
+ *   du_down      : [H, R, DV] fp32 summed over the batch (overwritten)
+ *   du_up        : [H, DK, R] fp32 summed over the batch (overwritten)
+ *   dS0          : [B, H, DV, DK] fp32 or NULL;  dm0 : [B, H, DV] fp32 or NULL
+ *
+ * Errors as for carve_chunk_fwd.
+ */
+carve_status carve_chunk_bwd(const carve_shape* shape,
+                             const void* q, const void* k, const void* v,
+                             const void* g, const void* b_x, const void* w,
+                             const void* u_down, const void* u_up,
+                             const void* d_o, const float* dS_T,
+                             const float* dm_T,
+                             void* workspace, size_t workspace_bytes,
+                             void* dq, void* dk, void* dv, void* dg,
+                             void* db_x, void* dw,
+                             float* du_down, float* du_up,
+                             float* dS0, float* dm0, void* stream);
+
+/*
+ * Synchronises `stream`, then reads the device status word that kernels
+ * write into the workspace header (CARVE_OK, or CARVE_ERR_TIMEOUT when a
+ * bounded device-side wait gave up; the kernel then skipped the rest of its
+ * work and left its outputs unspecified).  The word is sticky until
+ * carve_reset_status.
+ */
+carve_status carve_get_status(const void* workspace, void* stream);
+
+/* Enqueue a reset of the workspace status word to CARVE_OK on `stream`. */
+carve_status carve_reset_status(void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* carve_status_str(carve_status status);
+
+/* Name of the kernel family carve_chunk_fwd would use for this shape
+ * ("tc" for the tcgen05 path, "generic" otherwise), or NULL if
+ * unsupported. */
+const char* carve_fwd_path(const carve_shape* shape);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CARVE_H_ */

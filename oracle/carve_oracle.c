@@ -69,7 +69,8 @@ static void content_projection(int DK, int DV, int R, const double* u_down,
  */
 static void token_step(int DK, int DV, double* S, const double* q,
                        const double* k, const double* vv, const double* g,
-                       const double* b, double w, double* o, double* e) {
+                       const double* b, double w, double* o, double* e,
+                       double* alpha) {
   /* o_t = S_{t-1} q_t */
   for (int v = 0; v < DV; ++v) {
     double acc = 0.0;
@@ -77,10 +78,11 @@ static void token_step(int DK, int DV, double* S, const double* q,
     o[v] = acc;
   }
   /* S' = S_{t-1} Diag(exp g_t) ; e = S' k_t */
+  for (int j = 0; j < DK; ++j) alpha[j] = exp(g[j]);
   for (int v = 0; v < DV; ++v) {
     double acc = 0.0;
     for (int j = 0; j < DK; ++j) {
-      S[(size_t)v * DK + j] *= exp(g[j]);
+      S[(size_t)v * DK + j] *= alpha[j];
       acc += S[(size_t)v * DK + j] * k[j];
     }
     e[v] = acc;
@@ -105,7 +107,8 @@ int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
   double* p = (double*)calloc((size_t)DK, sizeof(double));
   double* b = (double*)calloc((size_t)DK, sizeof(double));
   double* e = (double*)calloc((size_t)DV, sizeof(double));
-  if (!S || !m || !msum || !h || !p || !b || !e) return 2;
+  double* alpha = (double*)calloc((size_t)DK, sizeof(double));
+  if (!S || !m || !msum || !h || !p || !b || !e || !alpha) return 2;
   if (S0) memcpy(S, S0, sizeof(double) * (size_t)DV * DK);
   if (m0) memcpy(m, m0, sizeof(double) * (size_t)DV);
 
@@ -118,7 +121,7 @@ int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
       for (int j = 0; j < DK; ++j) b[j] = sigmoid(bx[(size_t)t * DK + j] + p[j]);
       token_step(DK, DV, S, q + (size_t)t * DK, k + (size_t)t * DK,
                  v + (size_t)t * DV, g + (size_t)t * DK, b, w[t],
-                 o + (size_t)t * DV, e);
+                 o + (size_t)t * DV, e, alpha);
       for (int vv = 0; vv < DV; ++vv) msum[vv] += o[(size_t)t * DV + vv];
     }
     /* m_{c+1} = (1/L) sum over chunk c of o_t */
@@ -127,6 +130,7 @@ int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
   if (S_T) memcpy(S_T, S, sizeof(double) * (size_t)DV * DK);
   if (m_T) memcpy(m_T, m, sizeof(double) * (size_t)DV);
   free(S); free(m); free(msum); free(h); free(p); free(b); free(e);
+  free(alpha);
   return 0;
 }
 
@@ -189,7 +193,8 @@ int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
     for (int t = t0; t < t1; ++t) {
       for (int j = 0; j < DK; ++j) b[j] = sigmoid(bx[(size_t)t * DK + j] + p[j]);
       token_step(DK, DV, S, q + (size_t)t * DK, k + (size_t)t * DK,
-                 v + (size_t)t * DV, g + (size_t)t * DK, b, w[t], otmp, e);
+                 v + (size_t)t * DV, g + (size_t)t * DK, b, w[t], otmp, e,
+                 alpha);
       for (int vv = 0; vv < DV; ++vv) msum[vv] += otmp[vv];
     }
     for (int vv = 0; vv < DV; ++vv) m[vv] = msum[vv] / (double)L;
@@ -210,7 +215,8 @@ int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
       memcpy(Stok + (size_t)(t - t0) * SZ, S, sizeof(double) * SZ);
       for (int j = 0; j < DK; ++j) b[j] = sigmoid(bx[(size_t)t * DK + j] + p[j]);
       token_step(DK, DV, S, q + (size_t)t * DK, k + (size_t)t * DK,
-                 v + (size_t)t * DV, g + (size_t)t * DK, b, w[t], otmp, e);
+                 v + (size_t)t * DV, g + (size_t)t * DK, b, w[t], otmp, e,
+                 alpha);
     }
     memset(dp, 0, sizeof(double) * (size_t)DK);
     for (int t = t1 - 1; t >= t0; --t) {

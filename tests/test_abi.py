@@ -1,0 +1,130 @@
+"""The C-ABI library loads and exports what include/carve.h declares, and its
+host-side validation rejects bad calls before touching the GPU.
+
+CPU only: every call below fails validation on the host, so no kernel is
+ever launched (the pointers passed are never dereferenced).
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunk_gated_delta_02_b200 import build as cbuild
+from chunk_gated_delta_02_b200 import carve
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "carve.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    cbuild.build()
+    return carve.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(carve_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declarations_are_exported(lib):
+    names = declared_functions()
+    assert names, "no declarations parsed"
+    for n in names:
+        assert hasattr(lib, n), "missing export " + n
+    assert sorted(carve.EXPORTS) == names
+
+
+def shape(**kw):
+    d = dict(B=2, T=128, H=3, DK=64, DV=64, R=8, L=64, dtype=0)
+    d.update(kw)
+    return carve.Shape(*(d[n] for n in ("B", "T", "H", "DK", "DV", "R", "L",
+                                        "dtype")))
+
+
+def ws_bytes(lib, s, training):
+    return lib.carve_workspace_bytes(ctypes.byref(s), training)
+
+
+def test_workspace_bytes(lib):
+    s = shape()
+    inf, trn = ws_bytes(lib, s, 0), ws_bytes(lib, s, 1)
+    assert inf > 256 and trn > inf
+    # training adds the block-start states: (NB + 1) states per pair
+    P, NB, DV, DK = 2 * 3, 128 // 64, 64, 64
+    assert trn - inf >= P * (NB + 1) * DV * DK * 4
+    for bad in (dict(DK=24), dict(DV=272), dict(L=96), dict(T=100),
+                dict(R=65), dict(B=0), dict(dtype=7), dict(L=0)):
+        assert ws_bytes(lib, shape(**bad), 0) == 0, bad
+    assert ws_bytes(lib, shape(T=0), 0) > 0
+
+
+def test_status_strings_and_path(lib):
+    for code, name in carve.STATUS.items():
+        assert lib.carve_status_str(code).decode() == name
+    assert lib.carve_fwd_path(ctypes.byref(shape())) is not None
+    assert lib.carve_fwd_path(ctypes.byref(shape(DK=24))) is None
+
+
+FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
+MIS = ctypes.c_void_p((1 << 20) + 4)     # misaligned
+
+
+def call_fwd(lib, s, ws=None, nbytes=0, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, bx=FAKE, w=FAKE, ud=FAKE,
+                uu=FAKE, S0=None, m0=None, o=FAKE, S_T=None, m_T=None)
+    args.update(over)
+    return lib.carve_chunk_fwd(
+        ctypes.byref(s) if s is not None else None, args["q"], args["k"],
+        args["v"], args["g"], args["bx"], args["w"], args["ud"], args["uu"],
+        args["S0"], args["m0"], args["o"], args["S_T"], args["m_T"], ws,
+        ctypes.c_size_t(nbytes), 0, None)
+
+
+def test_fwd_validation_returns_before_launch(lib):
+    s = shape()
+    need = ws_bytes(lib, s, 0)
+    assert call_fwd(lib, None) == 1                       # no shape
+    assert call_fwd(lib, shape(DK=24), FAKE, need) == 2   # unsupported
+    assert call_fwd(lib, shape(T=100), FAKE, need) == 2   # T % L != 0
+    assert call_fwd(lib, s, FAKE, need, q=None) == 1      # null input
+    assert call_fwd(lib, s, FAKE, need, v=MIS) == 1       # misaligned
+    assert call_fwd(lib, s, FAKE, need, S_T=MIS) == 1     # misaligned output
+    assert call_fwd(lib, s, None, need) == 3              # no workspace
+    assert call_fwd(lib, s, FAKE, need - 1) == 3          # too small
+    assert call_fwd(lib, s, MIS, need) == 3               # misaligned ws
+
+
+def test_bwd_validation_returns_before_launch(lib):
+    s = shape()
+    need = ws_bytes(lib, s, 1)
+    base = [FAKE] * 8 + [FAKE, None, None]
+    outs = [FAKE] * 8 + [None, None]
+
+    def call(sh, ws, nbytes, ins=base, o=outs):
+        return lib.carve_chunk_bwd(ctypes.byref(sh), *ins, ws,
+                                   ctypes.c_size_t(nbytes), *o, None)
+
+    assert call(shape(L=96), FAKE, need) == 2
+    bad_in = list(base)
+    bad_in[8] = None                                      # d_o missing
+    assert call(s, FAKE, need, ins=bad_in) == 1
+    bad_out = list(outs)
+    bad_out[6] = None                                     # du_down missing
+    assert call(s, FAKE, need, o=bad_out) == 1
+    # inference-sized workspace is too small for the backward (checked
+    # first, so that this call can never reach a launch)
+    assert ws_bytes(lib, s, 0) < need
+    assert call(s, FAKE, ws_bytes(lib, s, 0)) == 3
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 64, 1, 64, dtype=torch.bfloat16)
+    u = torch.zeros(1, 4, 64, dtype=torch.bfloat16)
+    uu = torch.zeros(1, 64, 4, dtype=torch.bfloat16)
+    w = torch.zeros(1, 64, 1, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        carve.chunk_fwd(x, x, x, x, x, w, u, uu, 64)

@@ -20,7 +20,8 @@ MUTANTS = {
     # erase with the wrong sign
     "erase_sign": ("+= -e[v] * (b[j] * k[j])", "+= e[v] * (b[j] * k[j])"),
     # decay applied on the value axis instead of the key axis
-    "decay_on_value_axis": ("*= exp(g[j]);", "*= exp(g[v % DK]);"),
+    "decay_on_value_axis": ("S[(size_t)v * DK + j] *= alpha[j];",
+                            "S[(size_t)v * DK + j] *= alpha[v % DK];"),
     # write gate dropped
     "no_write_gate": ("+ w * vv[v] * k[j]", "+ vv[v] * k[j]"),
     # chunk mean divides by the tokens present instead of L
