@@ -22,7 +22,7 @@ STATUS = {0: "CARVE_OK", 1: "CARVE_ERR_INVALID_ARG", 2: "CARVE_ERR_UNSUPPORTED",
 # Entry points declared in include/carve.h (the ABI test checks the list).
 EXPORTS = ("carve_workspace_bytes", "carve_chunk_fwd", "carve_chunk_bwd",
            "carve_get_status", "carve_reset_status", "carve_status_str",
-           "carve_fwd_path")
+           "carve_fwd_path", "carve_chunk_fwd_noalloc")
 
 
 class Shape(ctypes.Structure):

@@ -138,6 +138,41 @@ carve_status carve_chunk_bwd(const carve_shape* shape,
                              float* dS0, float* dm0, void* stream);
 
 /*
+ * Allocation-free forward (no counterpart in the paper; a convenience of
+ * this library).  For callers that cannot allocate device memory where they
+ * run the recurrence: a plugin whose host framework hands it only input and
+ * output tensors, a stream-ordered section where cudaMalloc's implicit
+ * device-wide synchronisation would stall other streams, or a real-time
+ * loop with a fixed memory budget.
+ *
+ * Same arguments and results as carve_chunk_fwd with training = 0, minus
+ * the workspace: the generic forward kernel keeps its per-(b, h) scratch in
+ * a static device array of CARVE_NOALLOC_SCRATCH_BYTES that is part of the
+ * library's device image (every GPU that loads libcarve holds it until the
+ * process exits).  The call allocates and frees nothing.
+ *   - Needs 256 + B*H*(4*C*DK + 4*C*DV + DV*DK)*4 bytes of that array,
+ *     C = min(L, 64); a larger shape returns CARVE_ERR_WORKSPACE and
+ *     enqueues nothing.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind; the kernel writes every scratch element before reading it, so
+ *     nothing has to be cleared between calls.  Calls whose kernels overlap
+ *     on the GPU (e.g. on two streams) race on the array: serialise them.
+ *   - Always runs the generic CUDA-core kernel, whatever carve_fwd_path says.
+ * Errors as for carve_chunk_fwd.
+ */
+#define CARVE_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+carve_status carve_chunk_fwd_noalloc(const carve_shape* shape,
+                                     const void* q, const void* k,
+                                     const void* v, const void* g,
+                                     const void* b_x, const void* w,
+                                     const void* u_down, const void* u_up,
+                                     const float* S0, const float* m0,
+                                     void* o, float* S_T, float* m_T,
+                                     void* stream);
+
+/*
  * Synchronises `stream`, then reads the device status word that kernels
  * write into the workspace header (CARVE_OK, or CARVE_ERR_TIMEOUT when a
  * bounded device-side wait gave up; the kernel then skipped the rest of its

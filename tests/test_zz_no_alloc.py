@@ -1,0 +1,86 @@
+"""carve_chunk_fwd_noalloc: the forward entry point that allocates nothing.
+
+It exists for callers that cannot call cudaMalloc where they run the
+recurrence (a plugin handed only its input and output tensors by a host
+framework that owns all device memory, a stream-ordered section where
+cudaMalloc's implicit synchronisation would stall other streams, a
+real-time loop with a fixed memory budget).  Its scratch is a static device
+array shared by every call on a device.
+
+The test calls it through the C ABI twice in a row, on different inputs,
+and checks each result against carve_chunk_fwd on the same inputs within
+the parity tolerance (max|delta| / max|ref| <= 1e-2 for bf16 inputs, 1e-4
+for fp32).  The test itself allocates its tensors with torch; the entry
+point under test does not allocate.  This file is collected last.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from chunk_gated_delta_02_b200 import carve
+from chunk_gated_delta_02_b200.inputs import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL = {torch.bfloat16: 1e-2, torch.float32: 1e-4}
+
+
+def _fn():
+    f = carve.lib().carve_chunk_fwd_noalloc
+    f.argtypes = [ctypes.POINTER(carve.Shape)] + [ctypes.c_void_p] * 14
+    f.restype = ctypes.c_int
+    return f
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def noalloc_fwd(d, L):
+    B, T, H, DK = d["q"].shape
+    DV, R = d["v"].shape[-1], d["u_down"].shape[1]
+    shape = carve.make_shape(B, T, H, DK, DV, R, L, d["q"].dtype)
+    o = torch.empty((B, T, H, DV), dtype=d["q"].dtype, device="cuda")
+    S_T = torch.empty((B, H, DV, DK), dtype=torch.float32, device="cuda")
+    m_T = torch.empty((B, H, DV), dtype=torch.float32, device="cuda")
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = _fn()(ctypes.byref(shape), _p(d["q"]), _p(d["k"]), _p(d["v"]),
+               _p(d["g"]), _p(d["bx"]), _p(d["w"]), _p(d["u_down"]),
+               _p(d["u_up"]), _p(d["S0"]), _p(d["m0"]), _p(o), _p(S_T),
+               _p(m_T), stream)
+    assert rc == 0, carve.STATUS.get(rc, rc)
+    return o, S_T, m_T
+
+
+def rel(a, b):
+    a, b = a.double(), b.double()
+    return float((a - b).abs().max() / b.abs().max().clamp_min(1e-30))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_noalloc_matches_workspace_entry_point_twice(dtype):
+    cfg = dict(B=2, H=3, T=192, DK=64, DV=64, R=8)
+    for call, seed in enumerate((31, 32)):
+        inp = make_inputs(seed=seed, dtype=dtype, **cfg)
+        gen = torch.Generator().manual_seed(seed)
+        if call == 1:  # second call: non-zero initial state and mean
+            inp["S0"] = torch.randn((2, 3, 64, 64), generator=gen) * 0.3
+            inp["m0"] = torch.randn((2, 3, 64), generator=gen) * 0.3
+        d = {k: (None if x is None else x.cuda()) for k, x in inp.items()}
+        o, S_T, m_T = noalloc_fwd(d, 64)
+        ro, rS, rm, _ = carve.chunk_fwd(d["q"], d["k"], d["v"], d["g"],
+                                        d["bx"], d["w"], d["u_down"],
+                                        d["u_up"], 64, d["S0"], d["m0"])
+        torch.cuda.synchronize()
+        for name, a, b in (("o", o, ro), ("S_T", S_T, rS), ("m_T", m_T, rm)):
+            assert rel(a, b) <= TOL[dtype], (call, name, rel(a, b))
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch():
+    # host-side size check: returns before any launch (pointers unused)
+    fake = ctypes.c_void_p(1 << 20)
+    shape = carve.make_shape(64, 64, 16, 256, 256, 8, 64, torch.bfloat16)
+    rc = _fn()(ctypes.byref(shape), *([fake] * 8), None, None, fake, None,
+               None, None)
+    assert carve.STATUS[rc] == "CARVE_ERR_WORKSPACE"
