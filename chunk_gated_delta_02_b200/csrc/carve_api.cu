@@ -1,5 +1,6 @@
 // carve_api.cu -- the C ABI of libcarve: validation, workspace layout and
 // kernel dispatch.  Declared in include/carve.h.
+#include <stdlib.h>
 #include <string.h>
 
 #include "carve_internal.cuh"
@@ -32,6 +33,15 @@ carve_status check_shape(const carve_shape* s) {
 }
 
 bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
+
+// Forward kernel family for a valid shape: the tensor-core kernel where it
+// applies, else the generic one.  CARVE_FWD_PATH=generic forces the generic
+// kernel (both are GPU kernels; used to cross-check the two paths).
+bool use_tc_fwd(const carve_shape& s) {
+  const char* env = getenv("CARVE_FWD_PATH");
+  if (env && strcmp(env, "generic") == 0) return false;
+  return tc_fwd_supported(s);
+}
 bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
 
 }  // namespace
@@ -57,7 +67,7 @@ const char* carve_status_str(carve_status s) {
 
 const char* carve_fwd_path(const carve_shape* shape) {
   if (check_shape(shape) != CARVE_OK) return nullptr;
-  return "generic";
+  return use_tc_fwd(*shape) ? "tc" : "generic";
 }
 
 carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
@@ -96,7 +106,9 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   a.scratch = (float*)(ws + L.scratch);
   a.scratch_per_pair = L.scratch_per_pair;
   a.hdr = (WsHeader*)ws;
-  cudaError_t e = launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
+  cudaError_t e = use_tc_fwd(s)
+                      ? launch_fwd_tc(a, (cudaStream_t)stream)
+                      : launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 

@@ -119,6 +119,11 @@ struct BwdArgs {
 cudaError_t launch_fwd_generic(const FwdArgs& a, int dtype, cudaStream_t st);
 cudaError_t launch_bwd_generic(const BwdArgs& a, int dtype, cudaStream_t st);
 size_t generic_fwd_smem_bytes(int C, int DK, int DV);
+
+// Tensor-core forward (carve_tc_fwd.cu): bf16, DK = DV = 128, L % 64 == 0,
+// R <= 32, T > 0.
+bool tc_fwd_supported(const carve_shape& s);
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
 size_t generic_bwd_smem_bytes(int C, int DK, int DV);
 
 }  // namespace carve

@@ -1,0 +1,627 @@
+// carve_tc_fwd.cu -- tensor-core (tcgen05 / TMEM / TMA) forward of the CARVE
+// recurrent core for bf16 inputs, dk = dv = 128, chunks of 64 or 128 tokens.
+//
+// One CTA (8 warps) walks one (sequence, head) pair through its blocks of
+// C = 64 tokens.  The fp32 state S (dv x dk) lives in tensor memory for the
+// whole walk; a bf16 copy in shared memory is the MMA operand.  Per block,
+// with the notation of the chunk form (CARVE summaries, gist.science,
+// section 3, "Chunkability Boundary": erase on the key axis only, so one
+// triangular solve per block serves every value row):
+//
+//   transform   Gamma = exp(cumsum g), K~ = K Gamma, Q~ = Q Gamma_{t-1},
+//               K^ = K / Gamma, kap^ = sigmoid(bx + U_b m_c) K^, W = w V
+//               (section 2.3: key-axis decay; section 2.1: content gate)
+//   MMA 1       G = [K~; Q~] [kap^ | K^]^T   ->  [A | M ; P_kap | P_k]
+//               D1 = S [K~; Q~]^T             ->  [(K~ S^T)^T | (Q~ S^T)^T]
+//   MMA 2       D1 += W^T [M; P_k]^T          ->  [R^T | (Q~ S^T + P_k W)^T]
+//   solve       Y = [T - I; -P_kap T], T = (I + A)^{-1}, by back-substitution
+//               of Y (I + A) = -[A; P_kap] in registers (one row per thread)
+//   MMA 3       D1 += R^T Y^T                 ->  [E^T | O^T]   (E = T R)
+//   output      o_t = row t of O; m_{c+1} = mean of the chunk's o_t
+//   MMA 4       S += W^T K^ - E^T kap^ ;  S <- S Diag(gamma)
+//
+// The transposed products put one value row v of S, R, E and O in TMEM lane
+// v, so each thread owns a value row: the chunk mean is a per-thread sum.
+// Raw input tiles arrive by TMA (128-byte swizzle) into buffers whose layout
+// is exactly the UMMA canonical layout, so the element-wise transform writes
+// operands at the offsets it reads them from.  The next block's v, g, b_x
+// tiles are requested right after the transform, its k, q tiles as soon as
+// MMA 1 has released their buffer.
+#include <cudaTypedefs.h>
+
+#include "carve_internal.cuh"
+#include "sm100_ptx.cuh"
+
+namespace carve {
+namespace {
+
+using namespace ptx;
+
+constexpr int kThreads = 256;
+constexpr int kBlk = 64;   // tokens per block
+constexpr int kDK = 128;   // key width
+constexpr int kDV = 128;   // value rows per CTA
+constexpr int kRMax = 32;  // rank of U_b held in registers
+
+// shared memory map (bytes from a 1024-aligned base); 128-byte swizzled
+// tiles are 64-column blocks of `rows` x 128 B.
+constexpr uint32_t OFF_X = 0;          // [K~; Q~]   2 blk x 128 rows  32 KB
+constexpr uint32_t OFF_KH = 32768;     // K^         2 blk x  64 rows  16 KB
+constexpr uint32_t OFF_KP = 49152;     // kap^       2 blk x  64 rows  16 KB
+constexpr uint32_t OFF_W = 65536;      // w V        2 blk x  64 rows  16 KB
+constexpr uint32_t OFF_MY = 81920;     // [M;P_k] then Y, 128 rows     16 KB
+constexpr uint32_t OFF_RE = 98304;     // R^T then -E^T, 128 rows      16 KB
+constexpr uint32_t OFF_SB = 114688;    // S (bf16)   2 blk x 128 rows  32 KB
+constexpr uint32_t OFF_RV = 147456;    // raw v      2 blk x  64 rows  16 KB
+constexpr uint32_t OFF_RG = 163840;    // raw g                        16 KB
+constexpr uint32_t OFF_RB = 180224;    // raw b_x                      16 KB
+constexpr uint32_t OFF_AF = 196608;    // A fp32 64 x 64 row-major     16 KB
+constexpr uint32_t OFF_SMALL = 212992;
+constexpr uint32_t SM_GAM = 0;         // gamma_j            128 f32
+constexpr uint32_t SM_P = 512;         // (U_b m)_j          128 f32
+constexpr uint32_t SM_W = 1024;        // w_t                 64 f32
+constexpr uint32_t SM_M = 1280;        // m_v                128 f32
+constexpr uint32_t SM_H = 1792;        // U_down m            64 f32
+constexpr uint32_t SM_HALF = 2048;     // half-block g sums  128 f32
+constexpr uint32_t SM_BAR = 2560;      // 6 mbarriers
+constexpr uint32_t SM_TMEM = 2624;     // TMEM base address
+constexpr uint32_t SM_ABORT = 2628;    // abort flag
+constexpr uint32_t kSmallBytes = 2688;
+constexpr uint32_t OFF_UU = 215808;    // U_up^T bf16 [kRMax][128]      8 KB
+constexpr uint32_t kSmemBytes = OFF_UU + 8192 + 1024;
+static_assert(OFF_SMALL + kSmallBytes <= OFF_UU, "shared memory map overlap");
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
+
+// TMEM columns (fp32, lanes = rows)
+constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
+constexpr uint32_t TM_D1 = 128;  // [R|..] -> [E|O]  [v][n]     128 cols
+constexpr uint32_t TM_GK = 256;  // [A; P_kap]       [i][t]      64 cols
+constexpr uint32_t TM_GM = 320;  // [M; P_k]         [i][t]      64 cols
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, false);
+constexpr uint32_t ID_AMN = idesc_bf16(128, 128, true, false);
+constexpr uint32_t ID_AMN_BMN = idesc_bf16(128, 128, true, true);
+constexpr uint32_t ID_BMN = idesc_bf16(128, 128, false, true);
+
+constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
+
+__device__ __forceinline__ float ldbf(const uint8_t* p) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
+}
+__device__ __forceinline__ void stbf(uint8_t* p, float x) {
+  *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
+}
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float sigm(float x) {
+  return __fdividef(1.0f, 1.0f + __expf(-x));
+}
+__device__ __forceinline__ void bar_named(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+// 8 fp32 values -> one 16-byte chunk of bf16 at `p`.
+__device__ __forceinline__ void st_chunk(uint8_t* p, const float* x) {
+  uint4 u;
+  u.x = pack2(x[0], x[1]);
+  u.y = pack2(x[2], x[3]);
+  u.z = pack2(x[4], x[5]);
+  u.w = pack2(x[6], x[7]);
+  *reinterpret_cast<uint4*>(p) = u;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
+                  const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_g,
+                  const __grid_constant__ CUtensorMap tm_bx) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* s_gam = reinterpret_cast<float*>(sm + OFF_SMALL + SM_GAM);
+  float* s_p = reinterpret_cast<float*>(sm + OFF_SMALL + SM_P);
+  float* s_w = reinterpret_cast<float*>(sm + OFF_SMALL + SM_W);
+  float* s_m = reinterpret_cast<float*>(sm + OFF_SMALL + SM_M);
+  float* s_h = reinterpret_cast<float*>(sm + OFF_SMALL + SM_H);
+  float* s_half = reinterpret_cast<float*>(sm + OFF_SMALL + SM_HALF);
+  float* s_af = reinterpret_cast<float*>(sm + OFF_AF);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_SMALL + SM_BAR);
+  uint64_t* bar_vgb = bars + 0;  // TMA v, g, b_x
+  uint64_t* bar_kq = bars + 1;   // TMA k, q
+  uint64_t* bar_m1 = bars + 2;   // MMA 1 (Grams, S X^T)
+  uint64_t* bar_m2 = bars + 3;   // MMA 2 (W^T [M;P_k]^T)
+  uint64_t* bar_m3 = bars + 4;   // MMA 3 (R^T Y^T)
+  uint64_t* bar_m4 = bars + 5;   // MMA 4 (state update)
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SMALL + SM_TMEM);
+  volatile uint32_t* s_abort =
+      reinterpret_cast<volatile uint32_t*>(sm + OFF_SMALL + SM_ABORT);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int half = warp >> 2;                 // 0: warps 0-3, 1: warps 4-7
+  const int row = (warp & 3) * 32 + lane;     // TMEM lane owned by the thread
+  const int pair = blockIdx.x, b = pair / a.H, h = pair - b * a.H;
+  const int T = a.T, H = a.H, R = a.R, NB = a.NB;
+  const int bpc = a.L / kBlk;
+  const size_t SZ = (size_t)kDV * kDK;
+  const __nv_bfloat16* w_in = static_cast<const __nv_bfloat16*>(a.w);
+  const __nv_bfloat16* ud = static_cast<const __nv_bfloat16*>(a.u_down);
+  const __nv_bfloat16* uu = static_cast<const __nv_bfloat16*>(a.u_up);
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
+
+  if (tid == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+    *s_abort = 0;
+    mbar_init_fence();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+    prefetch_tmap(&tm_g);
+    prefetch_tmap(&tm_bx);
+  }
+  if (warp == 0) {
+    tmem_alloc(s_tmem, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // lane base
+
+  // Bounded wait on an mbarrier phase; on expiry record CARVE_ERR_TIMEOUT,
+  // raise the CTA-wide abort flag and return (callers keep the barrier
+  // sequence, the block loop exits at its next check).
+  auto wait = [&](uint64_t* bar, uint32_t parity, uint32_t where) {
+    const long long t0 = clock64();
+    while (!*s_abort) {
+      if (mbar_try_wait(bar, parity)) return;
+      if (clock64() - t0 > kSpinCycles) {
+        atomicExch(&a.hdr->status, (uint32_t)CARVE_ERR_TIMEOUT);
+        a.hdr->where = where;
+        *s_abort = 1;
+      }
+    }
+  };
+
+  // U_b factors: thread (r = tid/8, part = tid%8) holds U_down[h][r][16 part
+  // .. 16 part + 15] in registers; U_up[h] is kept transposed in shared
+  // memory (s_uu[r][j], zero for r >= R).
+  float ud_r[16];
+  __nv_bfloat16* s_uu = reinterpret_cast<__nv_bfloat16*>(sm + OFF_UU);
+  {
+    const int r = tid >> 3, part = tid & 7;
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      ud_r[i] = (r < R) ? __bfloat162float(
+                              ud[((size_t)h * R + r) * kDV + 16 * part + i])
+                        : 0.f;
+    for (int e = tid; e < kRMax * kDK; e += kThreads) {
+      const int r2 = e / kDK, jj = e - r2 * kDK;
+      s_uu[e] = (r2 < R) ? uu[((size_t)h * kDK + jj) * R + r2]
+                         : __float2bfloat16_rn(0.f);
+    }
+  }
+
+  // content gate: s_p = U_up (U_down s_m)
+  auto gate = [&]() {
+    {
+      const int r = tid >> 3, part = tid & 7;
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc = fmaf(ud_r[i], s_m[16 * part + i], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      if (part == 0) s_h[r] = acc;
+    }
+    __syncthreads();
+    if (tid < 128) {
+      float acc = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < kRMax; ++r)
+        acc = fmaf(__bfloat162float(s_uu[r * kDK + tid]), s_h[r], acc);
+      s_p[tid] = acc;
+    }
+    __syncthreads();
+  };
+
+  auto issue_vgb = [&](int ib) {
+    const int tok = b * T + ib * kBlk;
+    mbar_expect_tx(bar_vgb, 3 * 16384);
+    tma_load_3d(sm + OFF_RV, &tm_v, bar_vgb, 0, h, tok);
+    tma_load_3d(sm + OFF_RV + 8192, &tm_v, bar_vgb, 64, h, tok);
+    tma_load_3d(sm + OFF_RG, &tm_g, bar_vgb, 0, h, tok);
+    tma_load_3d(sm + OFF_RG + 8192, &tm_g, bar_vgb, 64, h, tok);
+    tma_load_3d(sm + OFF_RB, &tm_bx, bar_vgb, 0, h, tok);
+    tma_load_3d(sm + OFF_RB + 8192, &tm_bx, bar_vgb, 64, h, tok);
+  };
+  auto issue_kq = [&](int ib) {
+    const int tok = b * T + ib * kBlk;
+    mbar_expect_tx(bar_kq, 2 * 16384);
+    tma_load_3d(sm + OFF_X, &tm_k, bar_kq, 0, h, tok);
+    tma_load_3d(sm + OFF_X + 16384, &tm_k, bar_kq, 64, h, tok);
+    tma_load_3d(sm + OFF_X + 8192, &tm_q, bar_kq, 0, h, tok);
+    tma_load_3d(sm + OFF_X + 16384 + 8192, &tm_q, bar_kq, 64, h, tok);
+  };
+
+  // ---- initial state: S0 -> TMEM (fp32) and the bf16 operand copy
+  {
+    const int c0 = half * 64;
+    const float* s0 = a.S0 ? a.S0 + (size_t)pair * SZ + (size_t)row * kDK + c0
+                           : nullptr;
+    float* ck = a.ck_S ? a.ck_S + (size_t)pair * (NB + 1) * SZ +
+                             (size_t)row * kDK + c0
+                       : nullptr;
+    float vals[32];
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+#pragma unroll
+      for (int i = 0; i < 32; i += 4) {
+        float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + part * 32 + i)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+        vals[i] = x.x; vals[i + 1] = x.y; vals[i + 2] = x.z; vals[i + 3] = x.w;
+        if (ck) *reinterpret_cast<float4*>(ck + part * 32 + i) = x;
+      }
+      tmem_st32(tl + TM_S + c0 + part * 32, vals);
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_chunk(sm + OFF_SB + sw128_chunk(row, half, part * 4 + c8, 128),
+                 vals + c8 * 8);
+    }
+  }
+  if (tid < 128) s_m[tid] = a.m0 ? a.m0[(size_t)pair * kDV + tid] : 0.f;
+  tmem_st_wait();
+  __syncthreads();
+  gate();
+  if (a.ck_m && tid < 128) a.ck_m[(size_t)pair * a.NC * kDV + tid] = s_m[tid];
+  if (tid == 0 && NB > 0) {
+    issue_vgb(0);
+    issue_kq(0);
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  float msum = 0.f;  // warps 4-7: this chunk's sum of o for value row `row`
+  for (int ib = 0; ib < NB; ++ib) {
+    const uint32_t par = (uint32_t)(ib & 1);
+    const int t0 = ib * kBlk;
+    const bool chunk_end = ((ib + 1) % bpc) == 0;
+
+    // ---- 1. inputs of this block
+    wait(bar_vgb, par, 1);
+    wait(bar_kq, par, 2);
+    if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)b * T + t0 + tid) * H + h]);
+    const int j = tid & 127;  // key channel of this thread in the transform
+    if (half == 0) {
+      float G = 0.f;
+#pragma unroll 8
+      for (int t = 0; t < 32; ++t) G += ldbf(sm + OFF_RG + sw128_off(t, j, 64));
+      s_half[j] = G;
+    }
+    __syncthreads();
+
+    // ---- 2. transform: decay scan, gated and decayed operands, W = w V
+    {
+      float G = half ? s_half[j] : 0.f;
+      float gprev = half ? __expf(G) : 1.f;  // Gamma_{t-1}
+      const float pj = s_p[j];
+#pragma unroll 4
+      for (int tt = 0; tt < 32; ++tt) {
+        const int t = half * 32 + tt;
+        const uint32_t oj = sw128_off(t, j, 64);
+        const uint32_t ok = sw128_off(t, j, 128);
+        const uint32_t oq = sw128_off(64 + t, j, 128);
+        const float kk = ldbf(sm + OFF_X + ok);
+        const float qq = ldbf(sm + OFF_X + oq);
+        const float bb = sigm(ldbf(sm + OFF_RB + oj) + pj);
+        G += ldbf(sm + OFF_RG + oj);
+        const float gam = __expf(G), igam = __expf(-G);
+        stbf(sm + OFF_X + ok, kk * gam);
+        stbf(sm + OFF_X + oq, qq * gprev);
+        const float kh = kk * igam;
+        stbf(sm + OFF_KH + oj, kh);
+        stbf(sm + OFF_KP + oj, bb * kh);
+        gprev = gam;
+      }
+      if (half) s_gam[j] = gprev;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = tid + 256 * i;  // 16-byte chunk of the 64 x 128 v tile
+      const int rr = (c >> 3) & 63;
+      const uint32_t off = (uint32_t)((c >> 9) * 8192 + (rr >> 3) * 1024 +
+                                      (rr & 7) * 128 + (c & 7) * 16);
+      const uint4 x = *reinterpret_cast<const uint4*>(sm + OFF_RV + off);
+      const float wt = s_w[rr];
+      const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
+      uint4 y;
+      uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(xv[e]);
+        yv[e] = pack2(f.x * wt, f.y * wt);
+      }
+      *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (*s_abort) break;
+
+    // ---- 3. MMA 1; the raw v, g, b_x buffers are free for the next block
+    if (tid == 0) {
+      if (ib + 1 < NB) issue_vgb(ib + 1);
+      tc_fence_after();
+      const uint32_t x0 = smem_u32(sm + OFF_X), kp0 = smem_u32(sm + OFF_KP);
+      const uint32_t kh0 = smem_u32(sm + OFF_KH), sb0 = smem_u32(sm + OFF_SB);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+        const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
+        umma_bf16(tmem + TM_GK, desc_kmajor_sw128(x0 + kx),
+                  desc_kmajor_sw128(kp0 + k64), ID_N64, ks > 0);
+        umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
+                  desc_kmajor_sw128(kh0 + k64), ID_N64, ks > 0);
+        umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
+                  desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
+      }
+      umma_commit(bar_m1);
+    }
+    wait(bar_m1, par, 3);
+    tc_fence_after();
+    if (tid == 0 && ib + 1 < NB && !*s_abort) issue_kq(ib + 1);
+
+    const int gi = row;                        // Gram row of this thread
+    const int gr = gi < 64 ? gi : gi - 64;     // its token index in the block
+    float vals[32];
+    if (half == 1) {
+      // ---- 4a. [M; P_k] (strictly lower) -> bf16 operand; MMA 2; R^T
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + TM_GM + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (part * 32 + e >= gr) vals[e] = 0.f;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_MY + sw128_chunk(gi, 0, part * 4 + c8, 128),
+                   vals + c8 * 8);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      bar_named(1, 128);
+      if (tid == 128 && !*s_abort) {
+        tc_fence_after();
+        const uint32_t w0 = smem_u32(sm + OFF_W), my0 = smem_u32(sm + OFF_MY);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+          umma_bf16(tmem + TM_D1, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
+                    desc_kmajor_sw128(my0 + ks * 32), ID_AMN, 1);
+        umma_commit(bar_m2);
+      }
+      wait(bar_m2, par, 4);
+      tc_fence_after();
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + TM_D1 + part * 32, vals);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
+                   vals + c8 * 8);
+      }
+      fence_async_smem();
+    } else {
+      // ---- 4b. Y (I + A) = -[A; P_kap], back-substitution per row
+      float y[64];
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + TM_GK + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float gv = (part * 32 + e < gr) ? vals[e] : 0.f;
+          y[part * 32 + e] = -gv;
+          vals[e] = gv;
+        }
+        if (gi < 64) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(s_af + gi * 64 + part * 32 + e) =
+                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+        }
+      }
+      bar_named(2, 128);
+#pragma unroll
+      for (int jj = 63; jj >= 1; --jj) {
+        const float yj = y[jj];
+        const float4* arow = reinterpret_cast<const float4*>(s_af + jj * 64);
+#pragma unroll
+        for (int l4 = 0; l4 < (jj + 3) / 4; ++l4) {
+          const float4 av = arow[l4];
+          if (4 * l4 + 0 < jj) y[4 * l4 + 0] = fmaf(-yj, av.x, y[4 * l4 + 0]);
+          if (4 * l4 + 1 < jj) y[4 * l4 + 1] = fmaf(-yj, av.y, y[4 * l4 + 1]);
+          if (4 * l4 + 2 < jj) y[4 * l4 + 2] = fmaf(-yj, av.z, y[4 * l4 + 2]);
+          if (4 * l4 + 3 < jj) y[4 * l4 + 3] = fmaf(-yj, av.w, y[4 * l4 + 3]);
+        }
+      }
+      wait(bar_m2, par, 5);  // [M; P_k] consumed: Y may take its place
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8)
+        st_chunk(sm + OFF_MY + sw128_chunk(gi, 0, c8, 128), y + c8 * 8);
+      fence_async_smem();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*s_abort) break;
+
+    // ---- 5. MMA 3: D1 += R^T Y^T -> [E^T | O^T]
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t re0 = smem_u32(sm + OFF_RE), my0 = smem_u32(sm + OFF_MY);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tmem + TM_D1, desc_kmajor_sw128(re0 + ks * 32),
+                  desc_kmajor_sw128(my0 + ks * 32), ID_N128, 1);
+      umma_commit(bar_m3);
+    }
+    wait(bar_m3, par, 6);
+    tc_fence_after();
+    if (half == 0) {
+      // -E^T -> bf16 operand of the state update
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + TM_D1 + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) vals[e] = -vals[e];
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
+                   vals + c8 * 8);
+      }
+      fence_async_smem();
+    } else {
+      // O^T: outputs o_t (value row `row`) and the chunk sum for m
+      __nv_bfloat16* orow = o + ((size_t)b * T + t0) * H * kDV + (size_t)h * kDV + row;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + TM_D1 + 64 + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          msum += vals[e];
+          orow[(size_t)(part * 32 + e) * H * kDV] = __float2bfloat16_rn(vals[e]);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*s_abort) break;
+
+    // ---- 6. MMA 4: S += W^T K^ - E^T kap^
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KH);
+      const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = smem_u32(sm + OFF_KP);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
+                  desc_mnmajor_sw128(kh0 + ks * 2048, 8192), ID_AMN_BMN, 1);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tmem + TM_S, desc_kmajor_sw128(re0 + ks * 32),
+                  desc_mnmajor_sw128(kp0 + ks * 2048, 8192), ID_BMN, 1);
+      umma_commit(bar_m4);
+    }
+    wait(bar_m4, par, 7);
+    tc_fence_after();
+
+    // ---- 7. S <- S Diag(gamma); bf16 copy; checkpoint / final state
+    {
+      const int c0 = half * 64;
+      float* ck = a.ck_S ? a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
+                               (size_t)row * kDK + c0
+                         : nullptr;
+      float* st = (a.S_T && ib == NB - 1)
+                      ? a.S_T + (size_t)pair * SZ + (size_t)row * kDK + c0
+                      : nullptr;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + TM_S + c0 + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) vals[e] *= s_gam[c0 + part * 32 + e];
+        tmem_st32(tl + TM_S + c0 + part * 32, vals);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_SB + sw128_chunk(row, half, part * 4 + c8, 128),
+                   vals + c8 * 8);
+        if (ck) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(ck + part * 32 + e) =
+                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+        }
+        if (st) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(st + part * 32 + e) =
+                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+        }
+      }
+      tmem_st_wait();
+    }
+    fence_async_smem();
+    if (chunk_end && half == 1) {
+      s_m[row] = msum / (float)a.L;
+      msum = 0.f;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (chunk_end && ib + 1 < NB) {
+      gate();
+      if (a.ck_m && tid < 128)
+        a.ck_m[((size_t)pair * a.NC + (ib + 1) / bpc) * kDV + tid] = s_m[tid];
+    }
+  }
+
+  if (a.m_T && tid < 128) a.m_T[(size_t)pair * kDV + tid] = s_m[tid];
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault,
+                                &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [B*T, H, D] bf16 tensor viewed as 3-D (D innermost); boxes of 64 x 1 x 64
+// with the 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)kBlk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool tc_fwd_supported(const carve_shape& s) {
+  return s.dtype == CARVE_BF16 && s.DK == kDK && s.DV == kDV &&
+         s.L % kBlk == 0 && s.R <= kRMax && s.T > 0;
+}
+
+cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
+  CUtensorMap mq, mk, mv, mg, mb;
+  const long long rows = (long long)a.B * a.T;
+  if (!make_map(&mq, a.q, kDK, a.H, rows) || !make_map(&mk, a.k, kDK, a.H, rows) ||
+      !make_map(&mv, a.v, kDV, a.H, rows) || !make_map(&mg, a.g, kDK, a.H, rows) ||
+      !make_map(&mb, a.bx, kDK, a.H, rows))
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(
+      fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  if (e != cudaSuccess) return e;
+  fwd_tc_kernel<<<a.B * a.H, kThreads, kSmemBytes, st>>>(a, mq, mk, mv, mg, mb);
+  return cudaGetLastError();
+}
+
+}  // namespace carve

@@ -52,6 +52,8 @@ SHAPES = [
     (1, 2, 256, 64, 64, 8, 128),     # chunk solved as two blocks
     (2, 1, 64, 16, 16, 1, 1),        # L = 1
     (1, 1, 256, 64, 256, 8, 64),     # widest value dimension
+    (1, 2, 192, 128, 128, 32, 64),   # tensor-core forward (bf16)
+    (2, 1, 256, 128, 128, 8, 128),   # tensor-core forward, two blocks/chunk
 ]
 
 
@@ -179,3 +181,36 @@ def test_training_fwd_bwd():
     pairs = sample_pairs(cfg["B"], cfg["H"], 3, seed=4)
     errs = bwd_errors(inp, cfg["L"], gro, pairs=pairs, du_heads=[5])
     assert_within(errs, 1e-2, "training fwd+bwd")
+
+
+# ------------------------------------------ tensor-core vs generic path -----
+
+TC_CASES = [
+    # B, H, T, R, L
+    (1, 1, 64, 32, 64),
+    (2, 3, 320, 32, 64),
+    (1, 2, 384, 8, 128),
+    (1, 1, 128, 0, 64),
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_tensor_core_forward_matches_oracle_and_generic(case, monkeypatch):
+    B, H, T, R, L = case
+    cfg = dict(B=B, H=H, T=T, DK=128, DV=128, R=R, L=L)
+    inp = inputs(cfg, 21, torch.bfloat16)
+    if R > 0:
+        inp["u_down"] = (inp["u_down"].float() * 25).to(torch.bfloat16)
+        inp["u_up"] = (inp["u_up"].float() * 25).to(torch.bfloat16)
+    _rand_state(inp, 22)
+    shape = carve.make_shape(B, T, H, 128, 128, R, L, torch.bfloat16)
+    assert carve.fwd_path(shape) == "tc"
+    assert_within(fwd_errors(inp, L), 1e-2, "tensor-core fwd")
+    _, o_tc, S_tc, m_tc, _ = run_fwd(inp, L, training=True)
+    monkeypatch.setenv("CARVE_FWD_PATH", "generic")
+    assert carve.fwd_path(shape) == "generic"
+    _, o_g, S_g, m_g, _ = run_fwd(inp, L, training=True)
+    from _parity import rel as _rel
+    assert _rel(o_tc.float().cpu(), o_g.float().cpu()) < 1e-2
+    assert _rel(S_tc.cpu(), S_g.cpu()) < 1e-2
+    assert _rel(m_tc.cpu(), m_g.cpu()) < 1e-2
