@@ -44,6 +44,14 @@ bool use_tc_fwd(const carve_shape& s) {
 }
 bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
 
+// Backward kernel family: tensor-core where it applies (the same shapes as
+// the tensor-core forward); CARVE_BWD_PATH=generic forces the generic one.
+bool use_tc_bwd(const carve_shape& s) {
+  const char* env = getenv("CARVE_BWD_PATH");
+  if (env && strcmp(env, "generic") == 0) return false;
+  return tc_fwd_supported(s);
+}
+
 }  // namespace
 
 extern "C" {
@@ -155,7 +163,9 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbx = db_x; a.dw = dw;
   a.du_down = du_down; a.du_up = du_up; a.dS0 = dS0; a.dm0 = dm0;
   a.hdr = (WsHeader*)ws;
-  cudaError_t e = launch_bwd_generic(a, s.dtype, (cudaStream_t)stream);
+  cudaError_t e = use_tc_bwd(s)
+                      ? launch_bwd_tc(a, (cudaStream_t)stream)
+                      : launch_bwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 

@@ -65,6 +65,9 @@ inline WsLayout ws_layout(const carve_shape& s, bool training) {
   if (training) {
     size_t sb = generic_bwd_scratch_floats(w.C, s.DK, s.DV);
     sc = sc > sb ? sc : sb;
+    // the tensor-core backward keeps per-chunk gate records here instead
+    const size_t gr = (size_t)(w.NC > 0 ? w.NC : 1) * (s.DK + 2 * s.R);
+    sc = sc > gr ? sc : gr;
   }
   w.scratch_per_pair = sc;
   w.scratch = off;
@@ -124,6 +127,11 @@ size_t generic_fwd_smem_bytes(int C, int DK, int DV);
 // R <= 32, T > 0.
 bool tc_fwd_supported(const carve_shape& s);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
+
+// Tensor-core backward (carve_tc_bwd.cu), same shapes as the forward.  Its
+// per-chunk gate records (B*H*NC*(DK + 2R) floats) live in the scratch area.
+size_t tc_bwd_gate_record_floats(const carve_shape& s);
+cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st);
 size_t generic_bwd_smem_bytes(int C, int DK, int DV);
 
 }  // namespace carve

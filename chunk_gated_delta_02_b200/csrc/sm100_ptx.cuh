@@ -148,6 +148,23 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float* in) {
       "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// 16 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* out) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
+        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
+        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) out[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -176,6 +193,14 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn,
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) |
          ((b_mn ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// Same, with A (bit 13) and/or B (bit 14) negated by the tensor core.
+__host__ __device__ constexpr uint32_t idesc_bf16_neg(int M, int N, bool a_mn,
+                                                      bool b_mn, bool neg_a,
+                                                      bool neg_b) {
+  return idesc_bf16(M, N, a_mn, b_mn) | ((neg_a ? 1u : 0u) << 13) |
+         ((neg_b ? 1u : 0u) << 14);
 }
 
 // Byte offset of element (row, col) in a tile stored as 64-column blocks
