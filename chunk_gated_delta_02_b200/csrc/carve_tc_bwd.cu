@@ -273,6 +273,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sm + R_DSB + 8192, &tm_g, bar_in, 64, h, tok);
       tma_load_3d(sm + R_DSB + 16384, &tm_bx, bar_in, 0, h, tok);
       tma_load_3d(sm + R_DSB + 24576, &tm_bx, bar_in, 64, h, tok);
+      if (ib > 0) {  // the next block visited: its tiles and start state -> L2
+        const int tn = tok - kBlk;
+#pragma unroll
+        for (int x0 = 0; x0 < 128; x0 += 64) {
+          tma_prefetch_3d(&tm_k, x0, h, tn);
+          tma_prefetch_3d(&tm_q, x0, h, tn);
+          tma_prefetch_3d(&tm_v, x0, h, tn);
+          tma_prefetch_3d(&tm_do, x0, h, tn);
+          tma_prefetch_3d(&tm_g, x0, h, tn);
+          tma_prefetch_3d(&tm_bx, x0, h, tn);
+        }
+        const float* nxt = a.ck_S + ((size_t)pair * (NB + 1) + ib - 1) * SZ;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) bulk_prefetch_l2(nxt + q4 * 4096, 16384);
+      }
     }
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
     {
@@ -317,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float qq = ldbf(sm + R_X + oq);
         const float bb = sigm(ldbf(sm + R_DSB + 16384 + oj) + pj);
         G += ldbf(sm + R_DSB + oj);
-        const float gam = __expf(G), igam = __expf(-G);
+        const float gam = __expf(G), igam = __fdividef(1.0f, gam);
         stbf(sm + R_X + ok, kk * gam);
         stbf(sm + R_X + oq, qq * gprev);
         const float kh = kk * igam;
@@ -391,7 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(bar1, par, 12);
     tc_fence_after();
 
-    // ---- S4: masks; R^T += W^T M^T ; solve T
+    // ---- S4/S5: warps 4-7: [M; P_k] mask, R^T += W^T M^T, R -> EW rows
+    //      0..63, dS~ = dS gamma (in TMEM), dlog gamma; warps 0-3:
+    //      [A; P_kap] masks and the inversion T = (I + A)^{-1}, concurrently
     const int gi = row, gr = gi < 64 ? gi : gi - 64;
     if (half == 1) {
 #pragma unroll
@@ -407,6 +424,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_async_smem();
       tc_fence_before();
+      s_x[row] = 0.f;  // dlog gamma accumulator
       bar_named(1, 128);
       if (tid == 128 && !*s_abort) {
         tc_fence_after();
@@ -417,21 +435,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                     desc_kmajor_sw128(mp0 + ks * 32), ID_MK64, 1);
         umma_commit(bar2);
       }
+      wait(bar2, par, 13);
+      tc_fence_after();
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + T_RE + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          stbf(sm + R_EW + sw128_off(part * 32 + e, row, 128), vals[e]);
+      }
+#pragma unroll 1
+      for (int hc = 0; hc < 2; ++hc) {
+        const int c0 = hc * 64;
+        const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
+                          (size_t)row * kDK + c0;
+        float prod[64];
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+          tmem_ld32(tl + T_DS + c0 + part * 32, vals);
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(sn + part * 32 + e);
+            prod[part * 32 + e] = vals[e] * x.x;
+            prod[part * 32 + e + 1] = vals[e + 1] * x.y;
+            prod[part * 32 + e + 2] = vals[e + 2] * x.z;
+            prod[part * 32 + e + 3] = vals[e + 3] * x.w;
+          }
+#pragma unroll
+          for (int e = 0; e < 32; ++e) vals[e] *= s_gam[c0 + part * 32 + e];
+          tmem_st32(tl + T_DS + c0 + part * 32, vals);
+        }
+        float hi[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) hi[i] = prod[32 + i];
+        const float s_lo = warp_reduce_scatter32(prod, lane);
+        const float s_hi = warp_reduce_scatter32(hi, lane);
+        atomicAdd(&s_x[c0 + lane], s_lo);
+        atomicAdd(&s_x[c0 + 32 + lane], s_hi);
+      }
+      tmem_st_wait();
     } else {
-      float y[64];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         tmem_ld32(tl + T_G + part * 32, vals);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float gv = (part * 32 + e < gr) ? vals[e] : 0.f;
-          y[part * 32 + e] = -gv;
-          vals[e] = gv;
-        }
+        for (int e = 0; e < 32; ++e)
+          if (part * 32 + e >= gr) vals[e] = 0.f;
         if (gi < 64) {
 #pragma unroll
           for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(s_af + gi * 64 + part * 32 + e) =
+            *reinterpret_cast<float4*>(s_af + fsw(gi, part * 32 + e)) =
                 make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
         } else {
 #pragma unroll
@@ -441,83 +494,42 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       bar_named(2, 128);
+      // T = (I + A)^{-1}: raw b_x is dead, its half of the region holds T in
+      // fp32; the T buffer serves as scratch first
+      float* s_tf = reinterpret_cast<float*>(sm + R_DSB + 16384);
+      unit_lower_inverse64(s_af, s_tf, reinterpret_cast<float*>(sm + R_TT), 2);
       if (gi < 64) {
+        float trow[64];
 #pragma unroll
-        for (int jj = 63; jj >= 1; --jj) {
-          const float yj = y[jj];
-          const float4* arow = reinterpret_cast<const float4*>(s_af + jj * 64);
-#pragma unroll
-          for (int l4 = 0; l4 < (jj + 3) / 4; ++l4) {
-            const float4 av = arow[l4];
-            if (4 * l4 + 0 < jj) y[4 * l4 + 0] = fmaf(-yj, av.x, y[4 * l4 + 0]);
-            if (4 * l4 + 1 < jj) y[4 * l4 + 1] = fmaf(-yj, av.y, y[4 * l4 + 1]);
-            if (4 * l4 + 2 < jj) y[4 * l4 + 2] = fmaf(-yj, av.z, y[4 * l4 + 2]);
-            if (4 * l4 + 3 < jj) y[4 * l4 + 3] = fmaf(-yj, av.w, y[4 * l4 + 3]);
-          }
+        for (int e = 0; e < 64; e += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(s_tf + fsw(gi, e));
+          trow[e] = x.x; trow[e + 1] = x.y; trow[e + 2] = x.z; trow[e + 3] = x.w;
         }
 #pragma unroll
-        for (int e = 0; e < 64; ++e) y[e] += (e == gi) ? 1.f : 0.f;  // T = (T-I)+I
-#pragma unroll
         for (int c8 = 0; c8 < 8; ++c8)
-          st_chunk(sm + R_TT + sw128_chunk(gi, 0, c8, 64), y + c8 * 8);
+          st_chunk(sm + R_TT + sw128_chunk(gi, 0, c8, 64), trow + c8 * 8);
       }
       fence_async_smem();
     }
-    if (tid < 128) s_x[tid] = 0.f;  // dlog gamma accumulator
     tc_fence_before();
     __syncthreads();
     if (*s_abort) break;
-
-    // ---- S5: R -> EW rows 0..63 ; dS~ = dS gamma -> TMEM and bf16 ; dlog gamma
-    wait(bar2, par, 13);
+    // dS~ (TMEM) -> bf16 operand, into the region the inversion released
     tc_fence_after();
-    if (half == 0) {
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_RE + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          stbf(sm + R_EW + sw128_off(part * 32 + e, row, 128), vals[e]);
-      }
-    }
     {
       const int c0 = half * 64;
-      const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
-                        (size_t)row * kDK + c0;
-      float prod[64];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         tmem_ld32(tl + T_DS + c0 + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(sn + part * 32 + e);
-          prod[part * 32 + e] = vals[e] * x.x;
-          prod[part * 32 + e + 1] = vals[e + 1] * x.y;
-          prod[part * 32 + e + 2] = vals[e + 2] * x.z;
-          prod[part * 32 + e + 3] = vals[e + 3] * x.w;
-        }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) vals[e] *= s_gam[c0 + part * 32 + e];
-        tmem_st32(tl + T_DS + c0 + part * 32, vals);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
           st_chunk(sm + R_DSB + sw128_chunk(row, half, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
-      // reduce over the 32 value rows of this warp, two columns per lane
-      float hi[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) hi[i] = prod[32 + i];
-      const float s_lo = warp_reduce_scatter32(prod, lane);
-      const float s_hi = warp_reduce_scatter32(hi, lane);
-      atomicAdd(&s_x[c0 + lane], s_lo);
-      atomicAdd(&s_x[c0 + 32 + lane], s_hi);
-      tmem_st_wait();
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (*s_abort) break;
 
     // ---- S6: E^T = R^T T^T ; dE^T = -dS~ kap^T - dO^T P_kap
     if (tid == 0) {
@@ -698,70 +710,72 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(bar_gb, par, 18);
     tc_fence_after();
 
-    // ---- S12: per key channel j: dq, dk, db_x, dg, dp
+    // ---- S12: per key channel j: dq, dk, db_x, dg, dp.  Pass 1 (ascending
+    //      tokens) carries Gamma and forms every per-token gradient and the
+    //      log-Gamma gradients dG_t; pass 2 (descending) sums dg_t = sum_{s>=t} dG_s.
     {
       const int jj = row;                 // key channel (TMEM lane)
       const int tb = half == 0 ? 32 : 0;  // token range [tb, tb + 32)
       const float pj = s_p[jj];
-      const float dlg = s_x[jj];
-      float gl[32];
-      float G = 0.f;
+      const size_t tstride = (size_t)H * kDK;
+      const size_t x0 = ((size_t)tok * H + h) * kDK + jj;
+      float Gs = 0.f;                     // log Gamma before the range
       if (half == 0) {
 #pragma unroll 8
-        for (int t = 0; t < 32; ++t) G += ldbf(sm + R_SB + sw128_off(t, jj, 64));
+        for (int t = 0; t < 32; ++t) Gs += ldbf(sm + R_SB + sw128_off(t, jj, 64));
       }
-      const float Gstart = G;
-#pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        G += ldbf(sm + R_SB + sw128_off(tb + t, jj, 64));
-        gl[t] = G;
-      }
-      float acc = 0.f, next_q = 0.f;
-      float dgl[32];
+      float G = Gs, gprev = __expf(Gs);
+      float dGv[32];
+      float qfirst = 0.f;                 // dQ~ Q~ of the range's first token
       float d7k[16], d7q[16], d8p[16], d8h[16];
 #pragma unroll
-      for (int sub = 1; sub >= 0; --sub) {
+      for (int sub = 0; sub < 2; ++sub) {
         const int tsub = tb + 16 * sub;
         tmem_ld16(tl + T_G + tsub, d7k);
         tmem_ld16(tl + T_G + 64 + tsub, d7q);
         tmem_ld16(tl + T_RE + tsub, d8p);
         tmem_ld16(tl + T_RE + 64 + tsub, d8h);
 #pragma unroll
-        for (int e = 15; e >= 0; --e) {
-          const int tl_ = 16 * sub + e;   // index within the range
+        for (int e = 0; e < 16; ++e) {
+          const int tl_ = 16 * sub + e;
           const int t = tb + tl_;
-          const size_t x = (((size_t)tok + t) * H + h) * kDK + jj;
-          const float Gt = gl[tl_];
-          const float Gm = tl_ > 0 ? gl[tl_ - 1] : Gstart;
-          const float gam = __expf(Gt), igam = __expf(-Gt), gamm = __expf(Gm);
-          const float bb = sigm(ldbf(sm + R_SB + 16384 + sw128_off(t, jj, 64)) + pj);
+          const uint32_t o64 = sw128_off(t, jj, 64);
+          G += ldbf(sm + R_SB + o64);
+          const float gam = __expf(G), igam = __fdividef(1.0f, gam);
+          const float bb = sigm(ldbf(sm + R_SB + 16384 + o64) + pj);
           const float kt = ldbf(sm + R_X + sw128_off(t, jj, 128));
           const float qt = ldbf(sm + R_X + sw128_off(64 + t, jj, 128));
-          const float kh = ldbf(sm + R_KH + sw128_off(t, jj, 64));
-          const float kp = ldbf(sm + R_KP + sw128_off(t, jj, 64));
+          const float kh = ldbf(sm + R_KH + o64);
+          const float kp = ldbf(sm + R_KP + o64);
           const float dKt = d7k[e], dQt = d7q[e], dKp = -d8p[e], dKh = d8h[e];
-          dq[x] = __float2bfloat16_rn(dQt * gamm);
+          const size_t x = x0 + (size_t)t * tstride;
+          dq[x] = __float2bfloat16_rn(dQt * gprev);
           dk[x] = __float2bfloat16_rn(dKt * gam + dKh * igam + dKp * bb * igam);
           const float dz = dKp * kh * bb * (1.f - bb);
           dbx[x] = __float2bfloat16_rn(dz);
           dp_acc += dz;
-          float dG = dKt * kt - dKh * kh - dKp * kp + next_q;
-          if (t == kBlk - 1) dG += dlg;
-          acc += dG;
-          if (half == 0)
-            dg[x] = __float2bfloat16_rn(acc);
+          const float qp = dQt * qt;        // Q~_t reads Gamma_{t-1}
+          dGv[tl_] = dKt * kt - dKh * kh - dKp * kp;
+          if (tl_ > 0)
+            dGv[tl_ - 1] += qp;
           else
-            dgl[tl_] = acc;
-          next_q = dQt * qt;
+            qfirst = qp;
+          gprev = gam;
         }
       }
-      if (half == 0) s_gam[jj] = acc + next_q;  // suffix total + dQ~_32 Q~_32
-      __syncthreads();
-      if (half == 1) {
-        const float off = s_gam[jj];
+      if (half == 0) {
+        dGv[31] += s_x[jj];                 // t = 63: gradient of log gamma
+        float tot = qfirst;                 // dG_31 (lower half) reads Q~_32
 #pragma unroll
-        for (int t = 0; t < 32; ++t)
-          dg[(((size_t)tok + t) * H + h) * kDK + jj] = __float2bfloat16_rn(dgl[t] + off);
+        for (int i = 0; i < 32; ++i) tot += dGv[i];
+        s_gam[jj] = tot;                    // hand-off to the lower half
+      }
+      __syncthreads();
+      float acc = half == 1 ? s_gam[jj] : 0.f;
+#pragma unroll
+      for (int i = 31; i >= 0; --i) {
+        acc += dGv[i];
+        dg[x0 + (size_t)(tb + i) * tstride] = __float2bfloat16_rn(acc);
       }
     }
 

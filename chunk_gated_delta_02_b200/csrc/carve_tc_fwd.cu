@@ -14,11 +14,11 @@
 //   MMA 1       G = [K~; Q~] [kap^ | K^]^T   ->  [A | M ; P_kap | P_k]
 //               D1 = S [K~; Q~]^T             ->  [(K~ S^T)^T | (Q~ S^T)^T]
 //   MMA 2       D1 += W^T [M; P_k]^T          ->  [R^T | (Q~ S^T + P_k W)^T]
-//   solve       Y = [T - I; -P_kap T], T = (I + A)^{-1}, by back-substitution
-//               of Y (I + A) = -[A; P_kap] in registers (one row per thread)
-//   MMA 3       D1 += R^T Y^T                 ->  [E^T | O^T]   (E = T R)
-//   output      o_t = row t of O; m_{c+1} = mean of the chunk's o_t
+//   solve       T = (I + A)^{-1} by 16 x 16 blocks (all threads, fp32)
+//   MMA 3a      E^T = R^T T^T                 (E = T R, the WY pseudo-values)
+//   MMA 3b      D1[O] -= E^T P_kap^T          ->  O^T = (Q~ S^T + P_k W - P_kap E)^T
 //   MMA 4       S += W^T K^ - E^T kap^ ;  S <- S Diag(gamma)
+//   output      o_t = row t of O; m_{c+1} = mean of the chunk's o_t
 //
 // The transposed products put one value row v of S, R, E and O in TMEM lane
 // v, so each thread owns a value row: the chunk mean is a per-thread sum.
@@ -31,11 +31,15 @@
 
 #include "carve_internal.cuh"
 #include "sm100_ptx.cuh"
+#include "tc_common.cuh"
 
 namespace carve {
 namespace {
 
 using namespace ptx;
+using tc::fsw;
+using tc::sigm;
+using tc::unit_lower_inverse64;
 
 constexpr int kThreads = 256;
 constexpr int kBlk = 64;   // tokens per block
@@ -83,7 +87,8 @@ constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, false);
 constexpr uint32_t ID_N128 = idesc_bf16(128, 128, false, false);
 constexpr uint32_t ID_AMN = idesc_bf16(128, 128, true, false);
 constexpr uint32_t ID_AMN_BMN = idesc_bf16(128, 128, true, true);
-constexpr uint32_t ID_BMN = idesc_bf16(128, 128, false, true);
+constexpr uint32_t ID_N64_NA = idesc_bf16_neg(128, 64, false, false, true, false);
+constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false);
 
 constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
 
@@ -96,9 +101,6 @@ __device__ __forceinline__ void stbf(uint8_t* p, float x) {
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ float sigm(float x) {
-  return __fdividef(1.0f, 1.0f + __expf(-x));
 }
 __device__ __forceinline__ void bar_named(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -293,7 +295,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t0 = ib * kBlk;
     const bool chunk_end = ((ib + 1) % bpc) == 0;
 
-    // ---- 1. inputs of this block
+    // ---- 1. inputs of this block (block ib + 2's tiles -> L2 ahead of
+    //         their loads, which are issued during block ib + 1)
+    if (tid == 0 && ib + 2 < NB) {
+      const int tn = b * T + (ib + 2) * kBlk;
+#pragma unroll
+      for (int x0 = 0; x0 < 128; x0 += 64) {
+        tma_prefetch_3d(&tm_k, x0, h, tn);
+        tma_prefetch_3d(&tm_q, x0, h, tn);
+        tma_prefetch_3d(&tm_v, x0, h, tn);
+        tma_prefetch_3d(&tm_g, x0, h, tn);
+        tma_prefetch_3d(&tm_bx, x0, h, tn);
+      }
+    }
     wait(bar_vgb, par, 1);
     wait(bar_kq, par, 2);
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)b * T + t0 + tid) * H + h]);
@@ -321,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float qq = ldbf(sm + OFF_X + oq);
         const float bb = sigm(ldbf(sm + OFF_RB + oj) + pj);
         G += ldbf(sm + OFF_RG + oj);
-        const float gam = __expf(G), igam = __expf(-G);
+        const float gam = __expf(G), igam = __fdividef(1.0f, gam);
         stbf(sm + OFF_X + ok, kk * gam);
         stbf(sm + OFF_X + oq, qq * gprev);
         const float kh = kk * igam;
@@ -379,8 +393,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gi = row;                        // Gram row of this thread
     const int gr = gi < 64 ? gi : gi - 64;     // its token index in the block
     float vals[32];
+    // the bf16 S copy is dead until step 7: its buffer holds T (fp32),
+    // the inversion's scratch and the bf16 P_kap operand meanwhile
+    float* s_tf = reinterpret_cast<float*>(sm + OFF_SB);
+    uint8_t* pq = sm + OFF_SB + 24576;
     if (half == 1) {
-      // ---- 4a. [M; P_k] (strictly lower) -> bf16 operand; MMA 2; R^T
+      // ---- 4a. [M; P_k] (strictly lower) -> bf16 operand; MMA 2
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         tmem_ld32(tl + TM_GM + part * 32, vals);
@@ -404,7 +422,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                     desc_kmajor_sw128(my0 + ks * 32), ID_AMN, 1);
         umma_commit(bar_m2);
       }
-      wait(bar_m2, par, 4);
+    } else {
+      // ---- 4b. [A; P_kap] (strictly lower): A -> fp32 for the inversion,
+      //          P_kap -> bf16 operand
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(tl + TM_GK + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (part * 32 + e >= gr) vals[e] = 0.f;
+        if (gi < 64) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(s_af + fsw(gi, part * 32 + e)) =
+                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+        } else {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8)
+            st_chunk(pq + sw128_chunk(gr, 0, part * 4 + c8, 64), vals + c8 * 8);
+        }
+      }
+    }
+    if (half == 1) {
+      // R^T -> bf16 operand, concurrently with the inversion
+      wait(bar_m2, par, 4);  // [M; P_k] consumed, R^T complete
       tc_fence_after();
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
@@ -414,76 +455,81 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
-      fence_async_smem();
     } else {
-      // ---- 4b. Y (I + A) = -[A; P_kap], back-substitution per row
-      float y[64];
+      // ---- 4c. T = (I + A)^{-1}, blocked, warp-level tensor cores (warps 0-3)
+      bar_named(2, 128);
+      unit_lower_inverse64(s_af, s_tf, s_tf + 4096, 2);
+      wait(bar_m2, par, 5);  // [M; P_k] consumed: T may take its place
+    }
+    if (half == 0 && gi < 64) {
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + TM_GK + part * 32, vals);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const float gv = (part * 32 + e < gr) ? vals[e] : 0.f;
-          y[part * 32 + e] = -gv;
-          vals[e] = gv;
+        for (int e = 0; e < 32; e += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(s_tf + fsw(gi, part * 32 + e));
+          vals[e] = x.x; vals[e + 1] = x.y; vals[e + 2] = x.z; vals[e + 3] = x.w;
         }
-        if (gi < 64) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(s_af + gi * 64 + part * 32 + e) =
-                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
-        }
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_MY + sw128_chunk(gi, 0, part * 4 + c8, 64), vals + c8 * 8);
       }
-      bar_named(2, 128);
-#pragma unroll
-      for (int jj = 63; jj >= 1; --jj) {
-        const float yj = y[jj];
-        const float4* arow = reinterpret_cast<const float4*>(s_af + jj * 64);
-#pragma unroll
-        for (int l4 = 0; l4 < (jj + 3) / 4; ++l4) {
-          const float4 av = arow[l4];
-          if (4 * l4 + 0 < jj) y[4 * l4 + 0] = fmaf(-yj, av.x, y[4 * l4 + 0]);
-          if (4 * l4 + 1 < jj) y[4 * l4 + 1] = fmaf(-yj, av.y, y[4 * l4 + 1]);
-          if (4 * l4 + 2 < jj) y[4 * l4 + 2] = fmaf(-yj, av.z, y[4 * l4 + 2]);
-          if (4 * l4 + 3 < jj) y[4 * l4 + 3] = fmaf(-yj, av.w, y[4 * l4 + 3]);
-        }
-      }
-      wait(bar_m2, par, 5);  // [M; P_k] consumed: Y may take its place
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8)
-        st_chunk(sm + OFF_MY + sw128_chunk(gi, 0, c8, 128), y + c8 * 8);
-      fence_async_smem();
     }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- 5. MMA 3: D1 += R^T Y^T -> [E^T | O^T]
+    // ---- 5. MMA 3a: E^T = R^T T^T
     if (tid == 0) {
       tc_fence_after();
       const uint32_t re0 = smem_u32(sm + OFF_RE), my0 = smem_u32(sm + OFF_MY);
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + TM_D1, desc_kmajor_sw128(re0 + ks * 32),
-                  desc_kmajor_sw128(my0 + ks * 32), ID_N128, 1);
+                  desc_kmajor_sw128(my0 + ks * 32), ID_N64, ks > 0);
       umma_commit(bar_m3);
     }
     wait(bar_m3, par, 6);
     tc_fence_after();
     if (half == 0) {
-      // -E^T -> bf16 operand of the state update
+      // E^T -> bf16 operand (negated by the MMAs that use it)
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
         tmem_ld32(tl + TM_D1 + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) vals[e] = -vals[e];
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
           st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
       fence_async_smem();
-    } else {
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*s_abort) break;
+
+    // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S += W^T K^ - E^T kap^
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KH);
+      const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = smem_u32(sm + OFF_KP);
+      const uint32_t pq0 = smem_u32(pq);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tmem + TM_D1 + 64, desc_kmajor_sw128(re0 + ks * 32),
+                  desc_kmajor_sw128(pq0 + ks * 32), ID_N64_NA, 1);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
+                  desc_mnmajor_sw128(kh0 + ks * 2048, 8192), ID_AMN_BMN, 1);
+#pragma unroll
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tmem + TM_S, desc_kmajor_sw128(re0 + ks * 32),
+                  desc_mnmajor_sw128(kp0 + ks * 2048, 8192), ID_BMN_NA, 1);
+      umma_commit(bar_m4);
+    }
+    wait(bar_m4, par, 7);
+    tc_fence_after();
+    if (half == 1) {
       // O^T: outputs o_t (value row `row`) and the chunk sum for m
       __nv_bfloat16* orow = o + ((size_t)b * T + t0) * H * kDV + (size_t)h * kDV + row;
 #pragma unroll
@@ -496,27 +542,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
-
-    // ---- 6. MMA 4: S += W^T K^ - E^T kap^
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KH);
-      const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = smem_u32(sm + OFF_KP);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
-                  desc_mnmajor_sw128(kh0 + ks * 2048, 8192), ID_AMN_BMN, 1);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        umma_bf16(tmem + TM_S, desc_kmajor_sw128(re0 + ks * 32),
-                  desc_mnmajor_sw128(kp0 + ks * 2048, 8192), ID_BMN, 1);
-      umma_commit(bar_m4);
-    }
-    wait(bar_m4, par, 7);
-    tc_fence_after();
 
     // ---- 7. S <- S Diag(gamma); bf16 copy; checkpoint / final state
     {

@@ -20,8 +20,13 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// Logistic function with one MUFU op: sigma(x) = 0.5 tanh(x / 2) + 0.5
+// (tanh.approx.f32, max error about 2^-11 -- below the bf16 rounding of the
+// operands it scales; sigma(-inf) = 0, sigma(+inf) = 1 exactly).
 __device__ __forceinline__ float sigm(float x) {
-  return __fdividef(1.0f, 1.0f + __expf(-x));
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(0.5f * x));
+  return fmaf(0.5f, y, 0.5f);
 }
 __device__ __forceinline__ void bar_named(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -54,6 +59,209 @@ __device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t parity,
       hdr->where = where;
       *abort_flag = 1;
     }
+  }
+}
+
+}  // namespace tc
+}  // namespace carve
+
+namespace carve {
+namespace tc {
+
+// Index of element (r, c) of a 64 x 64 fp32 matrix stored row-major with the
+// float4 groups of each row XOR-permuted by (r % 8): rows 256 B apart then
+// fall in different banks, and float4 groups stay contiguous.
+__device__ __forceinline__ int fsw(int r, int c) {
+  return r * 64 + (c ^ ((r & 7) << 2));
+}
+
+// Index of element (R, c) of the four diagonal 16 x 16 blocks of a 64 x 64
+// matrix stored compactly (row R in [0, 64), column c in [0, 16) within the
+// block); float4 groups XOR-permuted so that the rows of a warp's fragment
+// loads hit distinct banks.
+__device__ __forceinline__ int csw(int R, int c) {
+  return R * 16 + (c ^ (((R >> 1) & 3) << 2));
+}
+template <bool CPT>
+__device__ __forceinline__ int mx(int R, int C) {
+  return CPT ? csw(R, C & 15) : fsw(R, C);
+}
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+// c (16 x 8 fp32 fragment) += a (16 x 8 tf32) * b (8 x 8 tf32), warp-wide.
+__device__ __forceinline__ void mma_tf32(float* c, const uint32_t* a,
+                                         const uint32_t* b) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Warp-level 16 x 16 tile product on shared-memory fp32 matrices:
+// acc (two 16 x 8 fragments) += X[xr .., xc .. xc + 16 NB) * Y[yr .., yc .. yc + 16).
+// XC / YC select the compact (csw) or full (fsw) layout.  All fragments are
+// loaded first and every 16-wide K block accumulates into its own registers,
+// so the dependent chain is one load, one convert and two MMAs deep.
+template <bool XC, bool YC, int NB>
+__device__ __forceinline__ void tile_mac(float* acc, const float* X, int xr,
+                                         int xc, const float* Y, int yr,
+                                         int yc) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  float xa[NB][2][4], yb[NB][2][2][2];
+#pragma unroll
+  for (int kb = 0; kb < NB; ++kb)
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      const int c = xc + 16 * kb + 8 * kk + t;
+      xa[kb][kk][0] = X[mx<XC>(xr + g, c)];
+      xa[kb][kk][1] = X[mx<XC>(xr + g + 8, c)];
+      xa[kb][kk][2] = X[mx<XC>(xr + g, c + 4)];
+      xa[kb][kk][3] = X[mx<XC>(xr + g + 8, c + 4)];
+#pragma unroll
+      for (int nn = 0; nn < 2; ++nn) {
+        const int r = yr + 16 * kb + 8 * kk + t;
+        yb[kb][kk][nn][0] = Y[mx<YC>(r, yc + 8 * nn + g)];
+        yb[kb][kk][nn][1] = Y[mx<YC>(r + 4, yc + 8 * nn + g)];
+      }
+    }
+  float part[NB][8];
+#pragma unroll
+  for (int kb = 0; kb < NB; ++kb) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[kb][i] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 2; ++kk) {
+      uint32_t a[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) a[i] = to_tf32(xa[kb][kk][i]);
+#pragma unroll
+      for (int nn = 0; nn < 2; ++nn) {
+        uint32_t b[2] = {to_tf32(yb[kb][kk][nn][0]), to_tf32(yb[kb][kk][nn][1])};
+        mma_tf32(part[kb] + 4 * nn, a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int kb = 0; kb < NB; ++kb)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += part[kb][i];
+}
+// acc (two 16 x 8 fragments) <- / -> a 16 x 16 tile of Z at (zr, zc), scaled.
+template <bool ZC>
+__device__ __forceinline__ void tile_ld(float* acc, const float* Z, int zr,
+                                        int zc) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nn = 0; nn < 2; ++nn) {
+    acc[4 * nn + 0] = Z[mx<ZC>(zr + g, zc + 8 * nn + 2 * t)];
+    acc[4 * nn + 1] = Z[mx<ZC>(zr + g, zc + 8 * nn + 2 * t + 1)];
+    acc[4 * nn + 2] = Z[mx<ZC>(zr + g + 8, zc + 8 * nn + 2 * t)];
+    acc[4 * nn + 3] = Z[mx<ZC>(zr + g + 8, zc + 8 * nn + 2 * t + 1)];
+  }
+}
+template <bool ZC>
+__device__ __forceinline__ void tile_st(float* Z, int zr, int zc,
+                                        const float* acc, float s) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nn = 0; nn < 2; ++nn) {
+    Z[mx<ZC>(zr + g, zc + 8 * nn + 2 * t)] = s * acc[4 * nn + 0];
+    Z[mx<ZC>(zr + g, zc + 8 * nn + 2 * t + 1)] = s * acc[4 * nn + 1];
+    Z[mx<ZC>(zr + g + 8, zc + 8 * nn + 2 * t)] = s * acc[4 * nn + 2];
+    Z[mx<ZC>(zr + g + 8, zc + 8 * nn + 2 * t + 1)] = s * acc[4 * nn + 3];
+  }
+}
+
+// T = (I + A)^{-1} for a strictly lower 64 x 64 fp32 matrix A (layout fsw),
+// by 16 x 16 blocks on the warp-level tensor cores (tf32 in, fp32 out; T is
+// rounded to bf16 by its users).  Diagonal blocks: with N = A_II nilpotent
+// (N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8), i.e.
+// P = I - N and P <- P + P N^(2^k), one warp per block; then the
+// off-diagonal blocks level by level, one warp per block,
+//   T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ   (I - J = 1, 2, 3).
+// Called by warps 0..3 only (128 threads, named barrier `bar_id`); the
+// other warps of the CTA are free meanwhile.  T (layout fsw) goes to `tf`;
+// `ws` is >= 2048 floats of scratch.  Ends with that named barrier.
+static __device__ __noinline__ void unit_lower_inverse64(const float* af, float* tf,
+                                                  float* ws, int bar_id) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  float* n2 = ws;          // N^2, later N^8   (compact diagonal blocks)
+  float* n4 = ws + 1024;   // N^4
+  // P = I - N on the diagonal blocks, zero above the block diagonal; one
+  // float4 group (4 columns of one 16-column block) per step
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int e = tid + 128 * i;        // float4 group index, 0..1023
+    const int r = e >> 4, c = (e & 15) << 2;
+    const int br = r >> 4, bc = c >> 4;
+    if (bc == br) {
+      float4 v = *reinterpret_cast<const float4*>(af + fsw(r, c));
+      v.x = (r == c) ? 1.f : -v.x;
+      v.y = (r == c + 1) ? 1.f : -v.y;
+      v.z = (r == c + 2) ? 1.f : -v.z;
+      v.w = (r == c + 3) ? 1.f : -v.w;
+      *reinterpret_cast<float4*>(tf + fsw(r, c)) = v;
+    } else if (bc > br) {
+      *reinterpret_cast<float4*>(tf + fsw(r, c)) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  bar_named(bar_id, 128);
+  float acc[8], acc2[8];
+  if (warp < 4) {
+    const int o = 16 * warp;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    tile_mac<false, false, 1>(acc, af, o, o, af, o, o);        // N^2
+    tile_st<true>(n2, o, o, acc, 1.f);
+    __syncwarp();
+    tile_ld<false>(acc, tf, o, o);                             // P (I + N^2)
+    tile_mac<false, true, 1>(acc, tf, o, o, n2, o, o);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc2[i] = 0.f;
+    tile_mac<true, true, 1>(acc2, n2, o, o, n2, o, o);         // N^4
+    __syncwarp();
+    tile_st<false>(tf, o, o, acc, 1.f);
+    tile_st<true>(n4, o, o, acc2, 1.f);
+    __syncwarp();
+    tile_ld<false>(acc, tf, o, o);                             // P (I + N^4)
+    tile_mac<false, true, 1>(acc, tf, o, o, n4, o, o);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc2[i] = 0.f;
+    tile_mac<true, true, 1>(acc2, n4, o, o, n4, o, o);         // N^8
+    __syncwarp();
+    tile_st<false>(tf, o, o, acc, 1.f);
+    tile_st<true>(n2, o, o, acc2, 1.f);
+    __syncwarp();
+    tile_ld<false>(acc, tf, o, o);                             // P (I + N^8)
+    tile_mac<false, true, 1>(acc, tf, o, o, n2, o, o);
+    __syncwarp();
+    tile_st<false>(tf, o, o, acc, 1.f);
+  }
+  bar_named(bar_id, 128);
+#pragma unroll
+  for (int d = 1; d <= 3; ++d) {
+    if (warp < 4 - d) {
+      const int J = warp, I = warp + d;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      // X = sum_{K=J}^{I-1} A_IK T_KJ  (contiguous K range 16 J .. 16 I)
+      if (d == 1) tile_mac<false, false, 1>(acc, af, 16 * I, 16 * J, tf, 16 * J, 16 * J);
+      if (d == 2) tile_mac<false, false, 2>(acc, af, 16 * I, 16 * J, tf, 16 * J, 16 * J);
+      if (d == 3) tile_mac<false, false, 3>(acc, af, 16 * I, 16 * J, tf, 16 * J, 16 * J);
+      tile_st<false>(tf, 16 * I, 16 * J, acc, 1.f);   // T_IJ slot is free
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+      tile_mac<false, false, 1>(acc, tf, 16 * I, 16 * I, tf, 16 * I, 16 * J);
+      __syncwarp();
+      tile_st<false>(tf, 16 * I, 16 * J, acc, -1.f);
+    }
+    bar_named(bar_id, 128);
   }
 }
 
