@@ -44,12 +44,13 @@ bool use_tc_fwd(const carve_shape& s) {
 }
 bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
 
-// Backward kernel family: tensor-core where it applies (the same shapes as
-// the tensor-core forward); CARVE_BWD_PATH=generic forces the generic one.
+// Backward kernel family: tensor-core where the tensor-core forward ran (it
+// reads that forward's records); CARVE_BWD_PATH=generic forces the generic
+// one, which needs only the checkpoints either forward writes.
 bool use_tc_bwd(const carve_shape& s) {
   const char* env = getenv("CARVE_BWD_PATH");
   if (env && strcmp(env, "generic") == 0) return false;
-  return tc_fwd_supported(s);
+  return use_tc_fwd(s);
 }
 
 }  // namespace
@@ -113,6 +114,8 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   a.ck_m = training ? (float*)(ws + L.ck_m) : nullptr;
   a.scratch = (float*)(ws + L.scratch);
   a.scratch_per_pair = L.scratch_per_pair;
+  a.tc_rec = training && L.tc_rec ? (uint8_t*)(ws + L.tc_rec) : nullptr;
+  a.gin = training && L.gin ? (float*)(ws + L.gin) : nullptr;
   a.hdr = (WsHeader*)ws;
   cudaError_t e = use_tc_fwd(s)
                       ? launch_fwd_tc(a, (cudaStream_t)stream)
@@ -160,6 +163,8 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   a.scratch = (float*)(ws + L.scratch);
   a.scratch_per_pair = L.scratch_per_pair;
   a.du = (float*)(ws + L.du);
+  a.tc_rec = L.tc_rec ? (const uint8_t*)(ws + L.tc_rec) : nullptr;
+  a.gin = L.gin ? (const float*)(ws + L.gin) : nullptr;
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbx = db_x; a.dw = dw;
   a.du_down = du_down; a.du_up = du_up; a.dS0 = dS0; a.dm0 = dm0;
   a.hdr = (WsHeader*)ws;

@@ -18,10 +18,25 @@ constexpr int kMaxBlock = 64;  // tokens per solver block (C = min(L, 64))
 // Device status word at the start of the workspace.
 struct WsHeader {
   uint32_t status;   // carve_status written by kernels (sticky)
-  uint32_t magic;    // kWsMagic once a training forward wrote checkpoints
+  uint32_t magic;    // which training forward wrote the checkpoints
   uint32_t where;    // diagnostic: which wait gave up
   uint32_t pad[61];
 };
+constexpr uint32_t kWsMagicTc = 0xCA7E7C01u;  // tensor-core forward: tc records valid
+
+// Per-block record the tensor-core training forward leaves for the backward:
+// shared-memory images (128-byte swizzled UMMA layout of a 1024-aligned
+// base) of the bf16 state operand S, of E^T and of T = (I + A)^{-1}.
+constexpr size_t kTcRecS = 0;          // S    [v 128][j 128] bf16  32 KB
+constexpr size_t kTcRecE = 32768;      // E^T  [v 128][t 64]  bf16  16 KB
+constexpr size_t kTcRecT = 49152;      // T    [t 64][s 64]   bf16   8 KB
+constexpr size_t kTcRecBytes = 57344;
+
+// Tensor-core kernels: bf16, DK = DV = 128, L % 64 == 0, R <= 32, T > 0.
+inline bool tc_shape(const carve_shape& s) {
+  return s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 128 &&
+         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0;
+}
 static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
 
 // Layout of the workspace (byte offsets, 256-aligned).
@@ -34,6 +49,8 @@ struct WsLayout {
   size_t scratch;      // per-pair fp32 scratch of the generic kernels
   size_t scratch_per_pair;  // floats
   size_t du;           // [B*H][R*DV + DK*R] fp32 per-pair U_b gradients
+  size_t tc_rec;       // [B*H][NB] tensor-core records (kTcRecBytes each)
+  size_t gin;          // [B*H][NC][DK + R] fp32 chunk gate inputs p_c | h_c
   size_t total;
 };
 
@@ -66,7 +83,7 @@ inline WsLayout ws_layout(const carve_shape& s, bool training) {
     size_t sb = generic_bwd_scratch_floats(w.C, s.DK, s.DV);
     sc = sc > sb ? sc : sb;
     // the tensor-core backward keeps per-chunk gate records here instead
-    const size_t gr = (size_t)(w.NC > 0 ? w.NC : 1) * (s.DK + 2 * s.R);
+    const size_t gr = (size_t)(w.NC > 0 ? w.NC : 1) * (s.DK + s.R);
     sc = sc > gr ? sc : gr;
   }
   w.scratch_per_pair = sc;
@@ -75,6 +92,12 @@ inline WsLayout ws_layout(const carve_shape& s, bool training) {
   if (training) {
     w.du = off;
     off = align256(off + P * ((size_t)s.R * s.DV + (size_t)s.DK * s.R) * 4);
+    if (tc_shape(s)) {
+      w.tc_rec = off;
+      off = align256(off + P * (size_t)w.NB * kTcRecBytes);
+      w.gin = off;
+      off = align256(off + P * (size_t)w.NC * (s.DK + s.R) * 4);
+    }
   }
   w.total = off;
   return w;
@@ -101,6 +124,8 @@ struct FwdArgs {
   float* ck_m;     // NULL unless training
   float* scratch;  // generic kernels only
   size_t scratch_per_pair;
+  uint8_t* tc_rec;  // tensor-core records; NULL unless training
+  float* gin;       // chunk gate inputs p_c | h_c; NULL unless training
   WsHeader* hdr;
 };
 
@@ -113,6 +138,8 @@ struct BwdArgs {
   float* scratch;
   size_t scratch_per_pair;
   float* du;  // per-pair partial U_b gradients
+  const uint8_t* tc_rec;  // records of the tensor-core forward
+  const float* gin;       // its chunk gate inputs p_c | h_c
   void *dq, *dk, *dv, *dg, *dbx, *dw;
   float *du_down, *du_up, *dS0, *dm0;
   WsHeader* hdr;
@@ -128,8 +155,9 @@ size_t generic_fwd_smem_bytes(int C, int DK, int DV);
 bool tc_fwd_supported(const carve_shape& s);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
 
-// Tensor-core backward (carve_tc_bwd.cu), same shapes as the forward.  Its
-// per-chunk gate records (B*H*NC*(DK + 2R) floats) live in the scratch area.
+// Tensor-core backward (carve_tc_bwd.cu), same shapes as the forward; it
+// reads the tensor-core forward's records.  Its per-chunk gate gradients
+// (B*H*NC*(DK + R) floats: dp | dh) live in the scratch area.
 size_t tc_bwd_gate_record_floats(const carve_shape& s);
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st);
 size_t generic_bwd_smem_bytes(int C, int DK, int DV);

@@ -4,28 +4,31 @@
 // Exact reverse mode of the chunk form (see carve_tc_fwd.cu).  One CTA
 // walks the blocks of one (sequence, head) pair from last to first.  The
 // gradient of the block-end state, dS (dv x dk, fp32), lives in tensor
-// memory for the whole walk; each block is recomputed from its
-// checkpointed start state S and the chunk's gate input m_c.
+// memory for the whole walk.  Per block the training forward left a record
+// (the bf16 state operand S, E^T and T = (I + A)^{-1}, as shared-memory
+// images) and the chunk's gate vector p_c; the element-wise transform and
+// the Gram matrices are recomputed from the inputs.
 //
 // Per block, with dO = d_o + dm_{c+1} / L (the gate feedback: the next
 // chunk's mean reads these outputs) and dS~ = dS Diag(gamma):
 //
-//   recompute  A, M, P_k, P_kap, T = (I + A)^{-1}, R = K~ S^T + M W, E = T R
+//   recompute  M, P_k, P_kap (strictly lower Grams)
 //   dE   = -kap^ dS~^T - P_kap^T dO          dR = T^T dE
 //   G2   = [dR; dO] [E; W]^T = [[-dA, dM], [-dP_kap, dP_k]]  (strictly lower)
 //   dW   = K^ dS~^T + P_k^T dO + M^T dR     -> dv = w dW, dw = rowsum(dW V)
 //   [dK~; dQ~]   = [dR; dO] S + G2 [-kap^; K^]
 //   [-dkap^; dK^] = G2^T [K~; Q~] + [E; W] dS~
 //   dS_prev = dS~ + dR^T K~ + dO^T Q~
+//   dlog gamma_j = sum_v dS S_new  (S_new: the fp32 checkpoint of the block end)
 //   per key channel: dq, dk, db_x, dg (reverse cumulative sum of the
 //   log-Gamma gradients), dp = sum_t db_x  (the gate's logit gradient)
 //
 // All products are M = 128 tcgen05 MMAs, most in transposed form so that the
 // 128 lanes are value rows or key channels.  Shared memory (227 KB) is
-// time-shared: raw g / b_x, the solve's A and the bf16 dS~ share one region;
-// the C x C gradient G2 reuses the Gram buffers once their MMAs retired.
-// At each chunk start the gate gradient (dp, h = U_down m, dh = U_up^T dp)
-// is recorded so that a second kernel forms dU_up, dU_down in fixed order.
+// time-shared: raw g / b_x and the bf16 dS~ share one region; the C x C
+// gradient G2 reuses the Gram and T buffers once their MMAs retired.  At each
+// chunk start the gate gradient (dp, dh = U_up^T dp) is recorded so that a
+// second kernel forms dU_up, dU_down in fixed order.
 #include <cudaTypedefs.h>
 
 #include "carve_internal.cuh"
@@ -45,24 +48,26 @@ constexpr int kDV = 128;
 constexpr int kRMax = 32;
 
 // shared memory map (bytes; the dynamic shared memory base is required to
-// be 1024-aligned, which the kernel checks).
-constexpr uint32_t R_X = 0;          // [K~; Q~]            32 KB
-constexpr uint32_t R_KH = 32768;     // K^                  16 KB
-constexpr uint32_t R_KP = 49152;     // kap^                16 KB
-constexpr uint32_t R_EW = 65536;     // [R -> E ; W]        32 KB
-constexpr uint32_t R_RO = 98304;     // [dE -> dR ; dO]     32 KB
-constexpr uint32_t R_DSB = 131072;   // raw g, b_x | A fp32 | dS~ bf16  32 KB
-constexpr uint32_t R_SB = 163840;    // S bf16 | raw g, b_x (reload)     32 KB
-constexpr uint32_t R_MP = 196608;    // [M; P_k] | G2 cols 0..63         16 KB
-constexpr uint32_t R_PQ = 212992;    // P_kap    | G2 cols 64..127 (1/2)  8 KB
-constexpr uint32_t R_TT = 221184;    // T        | G2 cols 64..127 (2/2)  8 KB
+// be 1024-aligned, which the kernel checks).  Tiles are 128-byte swizzled
+// 64-column blocks of `rows` x 128 B, the UMMA canonical layout.
+constexpr uint32_t R_X = 0;          // [K~; Q~]                        32 KB
+constexpr uint32_t R_KH = 32768;     // K^                              16 KB
+constexpr uint32_t R_KP = 49152;     // kap^                            16 KB
+constexpr uint32_t R_ET = 65536;     // E^T (forward record)            16 KB
+constexpr uint32_t R_W = 81920;      // raw v -> W = w V                16 KB
+constexpr uint32_t R_RO = 98304;     // [dE -> dR ; dO]                 32 KB
+constexpr uint32_t R_DSB = 131072;   // raw g, b_x | dS~ bf16           32 KB
+constexpr uint32_t R_SB = 163840;    // S bf16 (record) | raw g, b_x    32 KB
+constexpr uint32_t R_MP = 196608;    // [M; P_k] | G2 cols 0..63        16 KB
+constexpr uint32_t R_PQ = 212992;    // P_kap    | G2 cols 64..127 (1/2) 8 KB
+constexpr uint32_t R_TT = 221184;    // T (record) | G2 cols 64..127 (2/2) 8 KB
 constexpr uint32_t R_SM = 229376;    // small region
 constexpr uint32_t SM_P = 0;         // p_j                128 f32
 constexpr uint32_t SM_DMN = 512;     // dm fed into dO     128 f32
 constexpr uint32_t SM_X = 1024;      // g half sums | dlog gamma | dp   128 f32
 constexpr uint32_t SM_GAM = 1536;    // gamma | dg hand-off | dh parts  128 f32
 constexpr uint32_t SM_W = 2048;      // w_t                 64 f32
-constexpr uint32_t SM_DW = 2304;     // dw sums | h, dh     64 f32
+constexpr uint32_t SM_DW = 2304;     // dw sums | dh        64 f32
 constexpr uint32_t SM_BAR = 2560;    // 8 mbarriers
 constexpr uint32_t SM_TMEM = 2624;
 constexpr uint32_t SM_ABORT = 2628;
@@ -73,13 +78,13 @@ static_assert(R_PQ == R_MP + 16384 && R_TT == R_PQ + 8192, "G2 blocks");
 // TMEM columns
 constexpr uint32_t T_DS = 0;     // dS [v][j]
 constexpr uint32_t T_G = 128;    // [A|M ; P_kap|P_k] [i][t]  -> [dK~^T | dQ~^T]
-constexpr uint32_t T_RE = 256;   // R^T -> E^T -> dW^T        -> [-dkap^T | dK^T]
+constexpr uint32_t T_RE = 256;   // dW^T  -> [-dkap^T | dK^T] (128 cols)
 constexpr uint32_t T_DER = 320;  // dE^T -> dR^T
 constexpr uint32_t T_G2 = 384;   // raw G2 [r][c]
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t ID_KK64 = idesc_bf16(128, 64, false, false);
-constexpr uint32_t ID_KK128 = idesc_bf16(128, 128, false, false);
+constexpr uint32_t ID_KM64 = idesc_bf16(128, 64, false, true);
 constexpr uint32_t ID_MK64 = idesc_bf16(128, 64, true, false);
 constexpr uint32_t ID_MK128 = idesc_bf16(128, 128, true, false);
 constexpr uint32_t ID_MM64 = idesc_bf16(128, 64, true, true);
@@ -106,7 +111,7 @@ __device__ __forceinline__ float warp_reduce_scatter32(float* v, int lane) {
 
 struct BwdTcArgs {
   BwdArgs a;
-  float* gate_rec;  // [B*H][NC][DK + 2R]: dp | h | dh per chunk
+  float* gate_rec;  // [B*H][NC][DK + R]: dp | dh per chunk
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -129,7 +134,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_in = bars + 0;
   uint64_t* bar_gb = bars + 1;
   uint64_t* bar1 = bars + 2;
-  uint64_t* bar2 = bars + 3;
   uint64_t* bar3 = bars + 4;
   uint64_t* bar4 = bars + 5;
   uint64_t* bar5 = bars + 6;
@@ -137,7 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + R_SM + SM_TMEM);
   volatile uint32_t* s_abort =
       reinterpret_cast<volatile uint32_t*>(sm + R_SM + SM_ABORT);
-  float* s_af = reinterpret_cast<float*>(sm + R_DSB);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int half = warp >> 2;
@@ -155,12 +158,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   __nv_bfloat16* dg = static_cast<__nv_bfloat16*>(a.dg);
   __nv_bfloat16* dbx = static_cast<__nv_bfloat16*>(a.dbx);
   __nv_bfloat16* dw = static_cast<__nv_bfloat16*>(a.dw);
-  const int GR = kDK + 2 * R;  // floats per gate record
+  const int GR = kDK + R;  // floats per gate record and per gate input
 
-  if ((smem_u32(sm) & 1023u) != 0) {  // layout assumption broken: refuse
+  // layout assumption broken, or the workspace was not written by the
+  // tensor-core training forward: refuse
+  if ((smem_u32(sm) & 1023u) != 0 || a.hdr->magic != kWsMagicTc) {
     if (tid == 0) {
-      atomicExch(&a.hdr->status, (uint32_t)CARVE_ERR_UNSUPPORTED);
-      a.hdr->where = 99;
+      const bool align = (smem_u32(sm) & 1023u) != 0;
+      atomicExch(&a.hdr->status, (uint32_t)(align ? CARVE_ERR_UNSUPPORTED
+                                                  : CARVE_ERR_WORKSPACE));
+      a.hdr->where = align ? 99 : 98;
     }
     return;
   }
@@ -231,49 +238,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool chunk_first = ib % bpc == 0;       // last visited block of c
     const int tok = b * T + t0;
     float* rec = args.gate_rec + ((size_t)pair * NC + c) * GR;
+    const uint8_t* trec = a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes;
 
-    // ---- S0: gate of chunk c (p = U_up U_down m_c), once per chunk
+    // ---- S0: gate of chunk c, p = U_up U_down m_c (forward record)
     if (chunk_last) {
-      if (half == 1) {
-        const float mv = a.ck_m[((size_t)pair * NC + c) * kDV + row];
-        float pr[kRMax];
-#pragma unroll
-        for (int r = 0; r < kRMax; ++r) pr[r] = ureg[r] * mv;
-        const float hsum = warp_reduce_scatter32(pr, lane);
-        s_x[(warp - 4) * 32 + lane] = hsum;  // per-warp partials
-      }
-      __syncthreads();
-      if (tid < 32) {
-        const float hv = s_x[tid] + s_x[32 + tid] + s_x[64 + tid] + s_x[96 + tid];
-        s_dw[tid] = hv;  // h
-        if (tid < R) rec[kDK + tid] = hv;
-      }
-      __syncthreads();
-      if (half == 0) {
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < kRMax; ++r) acc = fmaf(ureg[r], s_dw[r], acc);
-        s_p[tid] = acc;
-      }
+      if (tid < 128) s_p[tid] = a.gin[((size_t)pair * NC + c) * GR + tid];
       dp_acc = 0.f;
     }
 
-    // ---- S1: inputs: TMA of k, q, v, d_o, g, b_x; S_c -> bf16
+    // ---- S1: inputs: TMA of k, q, v, d_o, g, b_x; records S, E^T, T
     if (tid == 0) {
-      mbar_expect_tx(bar_in, 6 * 16384);
+      mbar_expect_tx(bar_in, 6 * 16384 + (uint32_t)kTcRecBytes);
       tma_load_3d(sm + R_X, &tm_k, bar_in, 0, h, tok);
       tma_load_3d(sm + R_X + 16384, &tm_k, bar_in, 64, h, tok);
       tma_load_3d(sm + R_X + 8192, &tm_q, bar_in, 0, h, tok);
       tma_load_3d(sm + R_X + 24576, &tm_q, bar_in, 64, h, tok);
-      tma_load_3d(sm + R_EW + 8192, &tm_v, bar_in, 0, h, tok);
-      tma_load_3d(sm + R_EW + 24576, &tm_v, bar_in, 64, h, tok);
+      tma_load_3d(sm + R_W, &tm_v, bar_in, 0, h, tok);
+      tma_load_3d(sm + R_W + 8192, &tm_v, bar_in, 64, h, tok);
       tma_load_3d(sm + R_RO + 8192, &tm_do, bar_in, 0, h, tok);
       tma_load_3d(sm + R_RO + 24576, &tm_do, bar_in, 64, h, tok);
       tma_load_3d(sm + R_DSB, &tm_g, bar_in, 0, h, tok);
       tma_load_3d(sm + R_DSB + 8192, &tm_g, bar_in, 64, h, tok);
       tma_load_3d(sm + R_DSB + 16384, &tm_bx, bar_in, 0, h, tok);
       tma_load_3d(sm + R_DSB + 24576, &tm_bx, bar_in, 64, h, tok);
-      if (ib > 0) {  // the next block visited: its tiles and start state -> L2
+      bulk_load(sm + R_SB, trec + kTcRecS, 32768, bar_in);
+      bulk_load(sm + R_ET, trec + kTcRecE, 16384, bar_in);
+      bulk_load(sm + R_TT, trec + kTcRecT, 8192, bar_in);
+      if (ib > 0) {  // the next block visited: its tiles, record and end state -> L2
         const int tn = tok - kBlk;
 #pragma unroll
         for (int x0 = 0; x0 < 128; x0 += 64) {
@@ -284,29 +275,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_prefetch_3d(&tm_g, x0, h, tn);
           tma_prefetch_3d(&tm_bx, x0, h, tn);
         }
-        const float* nxt = a.ck_S + ((size_t)pair * (NB + 1) + ib - 1) * SZ;
+        bulk_prefetch_l2(trec - kTcRecBytes, (uint32_t)kTcRecBytes);
+        const float* nxt = a.ck_S + ((size_t)pair * (NB + 1) + ib) * SZ;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) bulk_prefetch_l2(nxt + q4 * 4096, 16384);
       }
     }
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
-    {
-      const int c0 = half * 64;
-      const float* src = a.ck_S + ((size_t)pair * (NB + 1) + ib) * SZ +
-                         (size_t)row * kDK + c0;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(src + part * 32 + i);
-          vals[i] = x.x; vals[i + 1] = x.y; vals[i + 2] = x.z; vals[i + 3] = x.w;
-        }
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + R_SB + sw128_chunk(row, half, part * 4 + c8, 128),
-                   vals + c8 * 8);
-      }
-    }
     wait(bar_in, par, 11);
     const int j = tid & 127;
     if (half == 0) {
@@ -317,9 +292,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
 
-    // ---- S2: transform
+    // ---- S2: transform (the half sums in s_x are consumed and zeroed: the
+    //      same words accumulate dlog gamma next)
     {
-      float G = half ? s_x[j] : 0.f;
+      float G = 0.f;
+      if (half) {
+        G = s_x[j];
+        s_x[j] = 0.f;
+      }
       float gprev = half ? __expf(G) : 1.f;
       const float pj = s_p[j];
 #pragma unroll 4
@@ -348,11 +328,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 4; ++i) {
         const int cidx = tid + 256 * i;  // 16-byte chunk of a 64 x 128 tile
         const int kb = cidx >> 9, rr = (cidx >> 3) & 63, ch = cidx & 7;
-        const uint32_t off = (uint32_t)(kb * 16384 + 8192 + (rr >> 3) * 1024 +
-                                        (rr & 7) * 128 + ch * 16);
-        // W = w V (rows 64.. of EW)
+        const uint32_t sub = (uint32_t)((rr >> 3) * 1024 + (rr & 7) * 128 + ch * 16);
+        // W = w V in place
         {
-          const uint4 x = *reinterpret_cast<const uint4*>(sm + R_EW + off);
+          const uint32_t off = (uint32_t)(kb * 8192) + sub;
+          const uint4 x = *reinterpret_cast<const uint4*>(sm + R_W + off);
           const float wt = s_w[rr];
           const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
           uint4 y;
@@ -362,10 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 f = __bfloat1622float2(xv[e]);
             yv[e] = pack2(f.x * wt, f.y * wt);
           }
-          *reinterpret_cast<uint4*>(sm + R_EW + off) = y;
+          *reinterpret_cast<uint4*>(sm + R_W + off) = y;
         }
         // dO = d_o + dm / L (rows 64.. of RO); logical column of the chunk
         {
+          const uint32_t off = (uint32_t)(kb * 16384 + 8192) + sub;
           const uint4 x = *reinterpret_cast<const uint4*>(sm + R_RO + off);
           const int v0 = kb * 64 + ((ch ^ (rr & 7)) << 3);
           const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
@@ -385,11 +366,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- S3: G = X [kap^ | K^]^T ;  R^T = S K~^T
+    // ---- S3: G = X [kap^ | K^]^T
     if (tid == 0) {
       tc_fence_after();
       const uint32_t x0 = smem_u32(sm + R_X), kp0 = smem_u32(sm + R_KP);
-      const uint32_t kh0 = smem_u32(sm + R_KH), sb0 = smem_u32(sm + R_SB);
+      const uint32_t kh0 = smem_u32(sm + R_KH);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -398,94 +379,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                   desc_kmajor_sw128(kp0 + k64), ID_KK64, ks > 0);
         umma_bf16(tmem + T_G + 64, desc_kmajor_sw128(x0 + kx),
                   desc_kmajor_sw128(kh0 + k64), ID_KK64, ks > 0);
-        umma_bf16(tmem + T_RE, desc_kmajor_sw128(sb0 + kx),
-                  desc_kmajor_sw128(x0 + kx), ID_KK64, ks > 0);
       }
       umma_commit(bar1);
     }
-    wait(bar1, par, 12);
-    tc_fence_after();
 
-    // ---- S4/S5: warps 4-7: [M; P_k] mask, R^T += W^T M^T, R -> EW rows
-    //      0..63, dS~ = dS gamma (in TMEM), dlog gamma; warps 0-3:
-    //      [A; P_kap] masks and the inversion T = (I + A)^{-1}, concurrently
-    const int gi = row, gr = gi < 64 ? gi : gi - 64;
-    if (half == 1) {
+    // ---- S4: dS~ = dS Diag(gamma) (TMEM, and its bf16 operand over the
+    //      consumed raw g, b_x) with dlog gamma_j = sum_v dS S_new; then the
+    //      strictly lower [M; P_k] (warps 4-7) and P_kap (warps 2-3) operands
+    {
+      const int c0 = half * 64;
+      const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
+                        (size_t)row * kDK + c0;
+      float prod[64];
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_G + 64 + part * 32, vals);
+        tmem_ld32(tl + T_DS + c0 + part * 32, vals);
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (part * 32 + e >= gr) vals[e] = 0.f;
+        for (int e = 0; e < 32; e += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(sn + part * 32 + e);
+          prod[part * 32 + e] = vals[e] * x.x;
+          prod[part * 32 + e + 1] = vals[e + 1] * x.y;
+          prod[part * 32 + e + 2] = vals[e + 2] * x.z;
+          prod[part * 32 + e + 3] = vals[e + 3] * x.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e) vals[e] *= s_gam[c0 + part * 32 + e];
+        tmem_st32(tl + T_DS + c0 + part * 32, vals);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + R_MP + sw128_chunk(gi, 0, part * 4 + c8, 128),
+          st_chunk(sm + R_DSB + sw128_chunk(row, half, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
-      fence_async_smem();
-      tc_fence_before();
-      s_x[row] = 0.f;  // dlog gamma accumulator
-      bar_named(1, 128);
-      if (tid == 128 && !*s_abort) {
-        tc_fence_after();
-        const uint32_t w0 = smem_u32(sm + R_EW + 8192), mp0 = smem_u32(sm + R_MP);
+      float hi[32];
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-          umma_bf16(tmem + T_RE, desc_mnmajor_sw128(w0 + ks * 2048, 16384),
-                    desc_kmajor_sw128(mp0 + ks * 32), ID_MK64, 1);
-        umma_commit(bar2);
-      }
-      wait(bar2, par, 13);
-      tc_fence_after();
+      for (int i = 0; i < 32; ++i) hi[i] = prod[32 + i];
+      const float s_lo = warp_reduce_scatter32(prod, lane);
+      const float s_hi = warp_reduce_scatter32(hi, lane);
+      atomicAdd(&s_x[c0 + lane], s_lo);
+      atomicAdd(&s_x[c0 + 32 + lane], s_hi);
+    }
+    wait(bar1, par, 12);
+    tc_fence_after();
+    const int gi = row, gr = gi < 64 ? gi : gi - 64;
+    if (half == 1 || gi >= 64) {
 #pragma unroll
       for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_RE + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          stbf(sm + R_EW + sw128_off(part * 32 + e, row, 128), vals[e]);
-      }
-#pragma unroll 1
-      for (int hc = 0; hc < 2; ++hc) {
-        const int c0 = hc * 64;
-        const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
-                          (size_t)row * kDK + c0;
-        float prod[64];
-#pragma unroll
-        for (int part = 0; part < 2; ++part) {
-          tmem_ld32(tl + T_DS + c0 + part * 32, vals);
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(sn + part * 32 + e);
-            prod[part * 32 + e] = vals[e] * x.x;
-            prod[part * 32 + e + 1] = vals[e + 1] * x.y;
-            prod[part * 32 + e + 2] = vals[e + 2] * x.z;
-            prod[part * 32 + e + 3] = vals[e + 3] * x.w;
-          }
-#pragma unroll
-          for (int e = 0; e < 32; ++e) vals[e] *= s_gam[c0 + part * 32 + e];
-          tmem_st32(tl + T_DS + c0 + part * 32, vals);
-        }
-        float hi[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) hi[i] = prod[32 + i];
-        const float s_lo = warp_reduce_scatter32(prod, lane);
-        const float s_hi = warp_reduce_scatter32(hi, lane);
-        atomicAdd(&s_x[c0 + lane], s_lo);
-        atomicAdd(&s_x[c0 + 32 + lane], s_hi);
-      }
-      tmem_st_wait();
-    } else {
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_G + part * 32, vals);
+        tmem_ld32(tl + T_G + (half ? 64 : 0) + part * 32, vals);
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           if (part * 32 + e >= gr) vals[e] = 0.f;
-        if (gi < 64) {
+        if (half) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(s_af + fsw(gi, part * 32 + e)) =
-                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+          for (int c8 = 0; c8 < 4; ++c8)
+            st_chunk(sm + R_MP + sw128_chunk(gi, 0, part * 4 + c8, 128),
+                     vals + c8 * 8);
         } else {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8)
@@ -493,54 +440,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                      vals + c8 * 8);
         }
       }
-      bar_named(2, 128);
-      // T = (I + A)^{-1}: raw b_x is dead, its half of the region holds T in
-      // fp32; the T buffer serves as scratch first
-      float* s_tf = reinterpret_cast<float*>(sm + R_DSB + 16384);
-      unit_lower_inverse64(s_af, s_tf, reinterpret_cast<float*>(sm + R_TT), 2);
-      if (gi < 64) {
-        float trow[64];
-#pragma unroll
-        for (int e = 0; e < 64; e += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(s_tf + fsw(gi, e));
-          trow[e] = x.x; trow[e + 1] = x.y; trow[e + 2] = x.z; trow[e + 3] = x.w;
-        }
-#pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8)
-          st_chunk(sm + R_TT + sw128_chunk(gi, 0, c8, 64), trow + c8 * 8);
-      }
-      fence_async_smem();
     }
-    tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
-    // dS~ (TMEM) -> bf16 operand, into the region the inversion released
-    tc_fence_after();
-    {
-      const int c0 = half * 64;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_DS + c0 + part * 32, vals);
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + R_DSB + sw128_chunk(row, half, part * 4 + c8, 128),
-                   vals + c8 * 8);
-      }
-    }
+    tmem_st_wait();
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (*s_abort) break;
 
-    // ---- S6: E^T = R^T T^T ; dE^T = -dS~ kap^T - dO^T P_kap
+    // ---- S6: dE^T = -dS~ kap^T - dO^T P_kap
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ew0 = smem_u32(sm + R_EW), tt0 = smem_u32(sm + R_TT);
       const uint32_t dsb0 = smem_u32(sm + R_DSB), kp0 = smem_u32(sm + R_KP);
       const uint32_t ro0 = smem_u32(sm + R_RO), pq0 = smem_u32(sm + R_PQ);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
-        umma_bf16(tmem + T_RE, desc_mnmajor_sw128(ew0 + ks * 2048, 16384),
-                  desc_kmajor_sw128(tt0 + ks * 32), ID_MK64, ks > 0);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks)
         umma_bf16(tmem + T_DER,
@@ -557,15 +468,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(bar3, par, 14);
     tc_fence_after();
 
-    // ---- S7: E -> EW rows 0..63 ; dE -> RO rows 0..63 ; dR^T = dE^T T
+    // ---- S7: dE -> RO rows 0..63 (tokens split between the halves);
+    //      dR^T = dE^T T
+    tmem_ld32(tl + T_DER + half * 32, vals);
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      tmem_ld32(tl + (half == 0 ? T_RE : T_DER) + part * 32, vals);
-      uint8_t* base = sm + (half == 0 ? R_EW : R_RO);
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        stbf(base + sw128_off(part * 32 + e, row, 128), vals[e]);
-    }
+    for (int e = 0; e < 32; ++e)
+      stbf(sm + R_RO + sw128_off(half * 32 + e, row, 128), vals[e]);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -579,40 +487,38 @@ __global__ void __launch_bounds__(kThreads, 1)
                   desc_mnmajor_sw128(tt0 + ks * 2048, 8192), ID_MM64, ks > 0);
       umma_commit(bar4);
     }
+    if (tid < 64) s_dw[tid] = 0.f;
     wait(bar4, par, 15);
     tc_fence_after();
 
     // ---- S8: dR -> RO rows 0..63
-    if (half == 1) {
+    tmem_ld32(tl + T_DER + half * 32, vals);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_DER + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          stbf(sm + R_RO + sw128_off(part * 32 + e, row, 128), vals[e]);
-      }
-      fence_async_smem();
-    }
-    if (tid < 64) s_dw[tid] = 0.f;
+    for (int e = 0; e < 32; ++e)
+      stbf(sm + R_RO + sw128_off(half * 32 + e, row, 128), vals[e]);
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- S9: G2raw, dW^T, dS += dR^T K~ + dO^T Q~, D7^T = S^T [dR; dO]^T
+    // ---- S9: G2raw = [dR; dO] [E; W]^T, dW^T, dS += [dR; dO]^T [K~; Q~],
+    //      D7^T = S^T [dR; dO]^T
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ro0 = smem_u32(sm + R_RO), ew0 = smem_u32(sm + R_EW);
-      const uint32_t dsb0 = smem_u32(sm + R_DSB), kh0 = smem_u32(sm + R_KH);
-      const uint32_t mp0 = smem_u32(sm + R_MP), x0 = smem_u32(sm + R_X);
-      const uint32_t sb0 = smem_u32(sm + R_SB);
+      const uint32_t ro0 = smem_u32(sm + R_RO), et0 = smem_u32(sm + R_ET);
+      const uint32_t w0 = smem_u32(sm + R_W), dsb0 = smem_u32(sm + R_DSB);
+      const uint32_t kh0 = smem_u32(sm + R_KH), mp0 = smem_u32(sm + R_MP);
+      const uint32_t x0 = smem_u32(sm + R_X), sb0 = smem_u32(sm + R_SB);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+        const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
         umma_bf16(tmem + T_G2, desc_kmajor_sw128(ro0 + kx),
-                  desc_kmajor_sw128(ew0 + kx), ID_KK128, ks > 0);
+                  desc_mnmajor_sw128(et0 + ks * 2048, 16384), ID_KM64, ks > 0);
+        umma_bf16(tmem + T_G2 + 64, desc_kmajor_sw128(ro0 + kx),
+                  desc_kmajor_sw128(w0 + k64), ID_KK64, ks > 0);
         umma_bf16(tmem + T_RE, desc_kmajor_sw128(dsb0 + kx),
-                  desc_kmajor_sw128(kh0 + (ks >> 2) * 8192 + (ks & 3) * 32),
-                  ID_KK64, ks > 0);
+                  desc_kmajor_sw128(kh0 + k64), ID_KK64, ks > 0);
         umma_bf16(tmem + T_G, desc_mnmajor_sw128(sb0 + ks * 2048, 16384),
                   desc_kmajor_sw128(ro0 + kx), ID_MK128, ks > 0);
       }
@@ -661,7 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; ++e) {
           const int t = part * 32 + e;
           dvrow[(size_t)t * H * kDV] = __float2bfloat16_rn(s_w[t] * vals[e]);
-          prod[t] = vals[e] * ldbf(sm + R_EW + sw128_off(64 + t, row, 128));
+          prod[t] = vals[e] * ldbf(sm + R_W + sw128_off(t, row, 64));
         }
       }
       float hi[32];
@@ -687,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t kp0 = smem_u32(sm + R_KP), kh0 = smem_u32(sm + R_KH);
       const uint32_t mp0 = smem_u32(sm + R_MP), pq0 = smem_u32(sm + R_PQ);
       const uint32_t x0 = smem_u32(sm + R_X), dsb0 = smem_u32(sm + R_DSB);
-      const uint32_t ew0 = smem_u32(sm + R_EW);
+      const uint32_t et0 = smem_u32(sm + R_ET), w0 = smem_u32(sm + R_W);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t a0 = (ks < 4 ? kp0 : kh0) + (ks & 3) * 2048;
@@ -700,10 +606,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_RE, desc_mnmajor_sw128(x0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(mp0 + ks * 2048, 16384), ID_MM128, ks > 0);
 #pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
+      for (int ks = 0; ks < 8; ++ks) {
         umma_bf16(tmem + T_RE, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
-                  desc_kmajor_sw128(ew0 + (ks >> 2) * 16384 + (ks & 3) * 32),
-                  ID_MK128, 1);
+                  desc_mnmajor_sw128(et0 + ks * 2048, 16384), ID_MM64, 1);
+        umma_bf16(tmem + T_RE + 64, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
+                  desc_kmajor_sw128(w0 + (ks >> 2) * 8192 + (ks & 3) * 32),
+                  ID_MK64, 1);
+      }
       umma_commit(bar7);
     }
     wait(bar7, par, 17);
@@ -800,14 +709,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncthreads();
       if (tid < 32) {
         const float dhv = s_gam[tid] + s_gam[32 + tid] + s_gam[64 + tid] + s_gam[96 + tid];
-        s_dw[32 + tid] = dhv;
-        if (tid < R) rec[kDK + R + tid] = dhv;
+        s_dw[tid] = dhv;
+        if (tid < R) rec[kDK + tid] = dhv;
       }
       __syncthreads();
       if (half == 1) {  // dm[v] = sum_r U_down[r][v] dh[r]
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < kRMax; ++r) acc = fmaf(ureg[r], s_dw[32 + r], acc);
+        for (int r = 0; r < kRMax; ++r) acc = fmaf(ureg[r], s_dw[r], acc);
         s_dmn[row] = acc;
       }
       dp_acc = 0.f;
@@ -843,11 +752,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // dU_up[h][j][r] = sum_{b,c} dp[b,h,c][j] h[b,h,c][r]
 // dU_down[h][r][v] = sum_{b,c} dh[b,h,c][r] m[b,h,c][v]   (fixed order)
+// dp, dh come from the backward's gate records, h = U_down m_c from the
+// forward's gate inputs, m_c from its checkpoints.
 __global__ void du_from_gate_records(const float* __restrict__ rec,
+                                     const float* __restrict__ gin,
                                      const float* __restrict__ ck_m, int B,
                                      int H, int NC, int R, int DK, int DV,
                                      float* du_down, float* du_up) {
-  const int GR = DK + 2 * R;
+  const int GR = DK + R;
   const size_t per = (size_t)DK * R + (size_t)R * DV;
   const size_t n = (size_t)H * per;
   for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n;
@@ -859,8 +771,8 @@ __global__ void du_from_gate_records(const float* __restrict__ rec,
       const int jj = (int)(e / R), r = (int)(e % R);
       for (int bb = 0; bb < B; ++bb)
         for (int c = 0; c < NC; ++c) {
-          const float* g = rec + ((size_t)(bb * H + h) * NC + c) * GR;
-          acc += g[jj] * g[DK + r];
+          const size_t o = ((size_t)(bb * H + h) * NC + c) * GR;
+          acc += rec[o + jj] * gin[o + DK + r];
         }
       du_up[(size_t)h * DK * R + e] = acc;
     } else {
@@ -868,8 +780,8 @@ __global__ void du_from_gate_records(const float* __restrict__ rec,
       const int r = (int)(e2 / DV), v = (int)(e2 % DV);
       for (int bb = 0; bb < B; ++bb)
         for (int c = 0; c < NC; ++c) {
-          const float* g = rec + ((size_t)(bb * H + h) * NC + c) * GR;
-          acc += g[DK + R + r] * ck_m[((size_t)(bb * H + h) * NC + c) * DV + v];
+          const size_t o = ((size_t)(bb * H + h) * NC + c);
+          acc += rec[o * GR + DK + r] * ck_m[o * DV + v];
         }
       du_down[(size_t)h * R * DV + e2] = acc;
     }
@@ -905,11 +817,12 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows) {
 }  // namespace
 
 size_t tc_bwd_gate_record_floats(const carve_shape& s) {
-  return (size_t)s.B * s.H * (size_t)(s.T / s.L) * (s.DK + 2 * s.R);
+  return (size_t)s.B * s.H * (size_t)(s.T / s.L) * (s.DK + s.R);
 }
 
 cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mg, mb, mdo;
+  if (!a.tc_rec || !a.gin) return cudaErrorInvalidValue;
   const long long rows = (long long)a.B * a.T;
   if (!make_map(&mq, a.q, kDK, a.H, rows) || !make_map(&mk, a.k, kDK, a.H, rows) ||
       !make_map(&mv, a.v, kDV, a.H, rows) || !make_map(&mg, a.g, kDK, a.H, rows) ||
@@ -927,8 +840,8 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
   if (n > 0) {
     int blocks = (int)((n + 255) / 256);
     if (blocks > 4 * 148) blocks = 4 * 148;
-    du_from_gate_records<<<blocks, 256, 0, st>>>(a.scratch, a.ck_m, a.B, a.H,
-                                                 a.NC, a.R, a.DK, a.DV,
+    du_from_gate_records<<<blocks, 256, 0, st>>>(a.scratch, a.gin, a.ck_m, a.B,
+                                                 a.H, a.NC, a.R, a.DK, a.DV,
                                                  a.du_down, a.du_up);
   }
   return cudaGetLastError();

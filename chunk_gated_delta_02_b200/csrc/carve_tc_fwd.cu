@@ -156,6 +156,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(a.o);
 
   if (tid == 0) {
+    if (a.tc_rec && blockIdx.x == 0) a.hdr->magic = kWsMagicTc;
     for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
     *s_abort = 0;
     mbar_init_fence();
@@ -209,8 +210,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // content gate: s_p = U_up (U_down s_m)
-  auto gate = [&]() {
+  // content gate of chunk c: s_p = U_up (U_down s_m); training records p_c
+  // and h_c = U_down m_c for the backward
+  auto gate = [&](int c) {
     {
       const int r = tid >> 3, part = tid & 7;
       float acc = 0.f;
@@ -230,6 +232,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_p[tid] = acc;
     }
     __syncthreads();
+    if (a.gin) {
+      float* gp = a.gin + ((size_t)pair * a.NC + c) * (kDK + R);
+      if (tid < 128)
+        gp[tid] = s_p[tid];
+      else if (tid - 128 < R)
+        gp[kDK + tid - 128] = s_h[tid - 128];
+    }
   };
 
   auto issue_vgb = [&](int ib) {
@@ -279,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid < 128) s_m[tid] = a.m0 ? a.m0[(size_t)pair * kDV + tid] : 0.f;
   tmem_st_wait();
   __syncthreads();
-  gate();
+  gate(0);
   if (a.ck_m && tid < 128) a.ck_m[(size_t)pair * a.NC * kDV + tid] = s_m[tid];
   if (tid == 0 && NB > 0) {
     issue_vgb(0);
@@ -294,9 +303,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t par = (uint32_t)(ib & 1);
     const int t0 = ib * kBlk;
     const bool chunk_end = ((ib + 1) % bpc) == 0;
+    uint8_t* rec = a.tc_rec ? a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes
+                            : nullptr;
 
     // ---- 1. inputs of this block (block ib + 2's tiles -> L2 ahead of
-    //         their loads, which are issued during block ib + 1)
+    //         their loads, which are issued during block ib + 1); training
+    //         records the block's bf16 state operand
+    if (tid == 0 && rec) {
+      bulk_store(rec + kTcRecS, sm + OFF_SB, 32768);
+      bulk_commit();
+    }
     if (tid == 0 && ib + 2 < NB) {
       const int tn = b * T + (ib + 2) * kBlk;
 #pragma unroll
@@ -364,6 +380,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
     }
     fence_async_smem();
+    if (tid == 0 && rec) bulk_wait_read_all();  // S record read: SB reusable
     __syncthreads();
     if (*s_abort) break;
 
@@ -488,6 +505,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + TM_D1, desc_kmajor_sw128(re0 + ks * 32),
                   desc_kmajor_sw128(my0 + ks * 32), ID_N64, ks > 0);
       umma_commit(bar_m3);
+      if (rec) {
+        bulk_store(rec + kTcRecT, sm + OFF_MY, 8192);
+        bulk_commit();
+      }
     }
     wait(bar_m3, par, 6);
     tc_fence_after();
@@ -509,6 +530,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S += W^T K^ - E^T kap^
     if (tid == 0) {
+      if (rec) {
+        bulk_store(rec + kTcRecE, sm + OFF_RE, 16384);
+        bulk_commit();
+      }
       tc_fence_after();
       const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KH);
       const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = smem_u32(sm + OFF_KP);
@@ -582,16 +607,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_m[row] = msum / (float)a.L;
       msum = 0.f;
     }
+    if (tid == 0 && rec) bulk_wait_read_all();  // T, E^T records read
     tc_fence_before();
     __syncthreads();
     if (chunk_end && ib + 1 < NB) {
-      gate();
+      gate((ib + 1) / bpc);
       if (a.ck_m && tid < 128)
         a.ck_m[((size_t)pair * a.NC + (ib + 1) / bpc) * kDV + tid] = s_m[tid];
     }
   }
 
   if (a.m_T && tid < 128) a.m_T[(size_t)pair * kDV + tid] = s_m[tid];
+  if (tid == 0 && a.tc_rec) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -630,10 +657,7 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows) {
 
 }  // namespace
 
-bool tc_fwd_supported(const carve_shape& s) {
-  return s.dtype == CARVE_BF16 && s.DK == kDK && s.DV == kDV &&
-         s.L % kBlk == 0 && s.R <= kRMax && s.T > 0;
-}
+bool tc_fwd_supported(const carve_shape& s) { return tc_shape(s); }
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mg, mb;
