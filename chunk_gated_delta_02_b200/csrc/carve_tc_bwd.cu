@@ -41,11 +41,10 @@ namespace {
 using namespace ptx;
 using namespace tc;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kBlk = 64;
 constexpr int kDK = 128;
 constexpr int kDV = 128;
-constexpr int kRMax = 32;
 
 // shared memory map (bytes; the dynamic shared memory base is required to
 // be 1024-aligned, which the kernel checks).  Tiles are 128-byte swizzled
@@ -109,11 +108,50 @@ __device__ __forceinline__ float warp_reduce_scatter32(float* v, int lane) {
   return v[0];
 }
 
+// Sum over the 32 lanes of a warp of v[i] (i < 16): lanes l and l ^ 16 end
+// with the sum of index l % 16 in v[0].  (15 + 1 shuffles.)
+__device__ __forceinline__ float warp_reduce_scatter16(float* v, int lane) {
+#pragma unroll
+  for (int k = 8; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const float send = up ? v[i] : v[i + k];
+      const float keep = up ? v[i + k] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+    }
+  }
+  return v[0] + __shfl_xor_sync(0xffffffffu, v[0], 16);
+}
+
+// Sum over the 32 lanes of a warp of v[i] (i < 8): lanes l, l ^ 8, l ^ 16,
+// l ^ 24 end with the sum of index l % 8 in v[0].
+__device__ __forceinline__ float warp_reduce_scatter8(float* v, int lane) {
+#pragma unroll
+  for (int k = 4; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const float send = up ? v[i] : v[i + k];
+      const float keep = up ? v[i + k] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+    }
+  }
+  float x = v[0] + __shfl_xor_sync(0xffffffffu, v[0], 8);
+  return x + __shfl_xor_sync(0xffffffffu, x, 16);
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
 struct BwdTcArgs {
   BwdArgs a;
   float* gate_rec;  // [B*H][NC][DK + R]: dp | dh per chunk
 };
 
+// 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or key
+// channels 32 qd .. 32 qd + 31) and column group gp = w / 4, so every
+// element-wise phase is split four ways along the TMEM columns.
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_tc_kernel(const BwdTcArgs args,
                   const __grid_constant__ CUtensorMap tm_q,
@@ -141,10 +179,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + R_SM + SM_TMEM);
   volatile uint32_t* s_abort =
       reinterpret_cast<volatile uint32_t*>(sm + R_SM + SM_ABORT);
+  // fp32 scratch of the epilogue and the gate backward (the dO / dR buffer
+  // is free once the last MMA that reads it retired)
+  float* s_scr = reinterpret_cast<float*>(sm + R_RO);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = warp >> 2;
-  const int row = (warp & 3) * 32 + lane;
+  const int qd = warp & 3, gp = warp >> 2;
+  const int row = qd * 32 + lane;
   const int pair = blockIdx.x, b = pair / a.H, h = pair - b * a.H;
   const int T = a.T, H = a.H, R = a.R, NB = a.NB, NC = a.NC;
   const int bpc = a.L / kBlk;
@@ -190,36 +231,40 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+  const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
 
-  // U_b factors: threads < 128 hold U_up[h][tid][:], threads >= 128 hold
-  // U_down[h][:][tid - 128].
-  float ureg[kRMax];
+  // U_b factors as bf16 pairs: U_up[h][row][8 gp .. 8 gp + 7] and
+  // U_down[h][8 gp .. 8 gp + 7][row] (zero beyond R)
+  uint32_t uup[4], udn[4];
 #pragma unroll
-  for (int r = 0; r < kRMax; ++r) {
-    float x = 0.f;
-    if (r < R)
-      x = half == 0 ? __bfloat162float(uu[((size_t)h * kDK + tid) * R + r])
-                    : __bfloat162float(ud[((size_t)h * R + r) * kDV + row]);
-    ureg[r] = x;
+  for (int i = 0; i < 4; ++i) {
+    const int r0 = 8 * gp + 2 * i;
+    float u0 = 0.f, u1 = 0.f, d0 = 0.f, d1 = 0.f;
+    if (r0 < R) {
+      u0 = __bfloat162float(uu[((size_t)h * kDK + row) * R + r0]);
+      d0 = __bfloat162float(ud[((size_t)h * R + r0) * kDV + row]);
+    }
+    if (r0 + 1 < R) {
+      u1 = __bfloat162float(uu[((size_t)h * kDK + row) * R + r0 + 1]);
+      d1 = __bfloat162float(ud[((size_t)h * R + r0 + 1) * kDV + row]);
+    }
+    uup[i] = pack2(u0, u1);
+    udn[i] = pack2(d0, d1);
   }
 
   // dS <- dS_T (or 0); dm <- dm_T (or 0)
   {
-    const int c0 = half * 64;
+    const int c0 = gp * 32;
     const float* src = a.dS_T ? a.dS_T + (size_t)pair * SZ + (size_t)row * kDK + c0
                               : nullptr;
     float vals[32];
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        const float4 x = src ? *reinterpret_cast<const float4*>(src + part * 32 + i)
-                             : make_float4(0.f, 0.f, 0.f, 0.f);
-        vals[i] = x.x; vals[i + 1] = x.y; vals[i + 2] = x.z; vals[i + 3] = x.w;
-      }
-      tmem_st32(tl + T_DS + c0 + part * 32, vals);
+    for (int i = 0; i < 32; i += 4) {
+      const float4 x = src ? *reinterpret_cast<const float4*>(src + i)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+      vals[i] = x.x; vals[i + 1] = x.y; vals[i + 2] = x.z; vals[i + 3] = x.w;
     }
+    tmem_st32(tl + T_DS + c0, vals);
     tmem_st_wait();
   }
   if (tid < 128) s_dmn[tid] = a.dm_T ? a.dm_T[(size_t)pair * kDV + tid] : 0.f;
@@ -228,8 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait_bar(bar, par, where, s_abort, a.hdr);
   };
 
-  float dp_acc = 0.f;   // this thread's share of dp_j for the current chunk
-  float vals[32];
+  float dp_acc = 0.f;   // dp_j share (channel row, this warp's token quarter)
   for (int ib = NB - 1, it = 0; ib >= 0; --ib, ++it) {
     const uint32_t par = (uint32_t)(it & 1);
     const int t0 = ib * kBlk;
@@ -282,65 +326,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
+    // w_t of the token row this thread scales in W = w V
+    const float wrow = __bfloat162float(w_in[((size_t)tok + (tid >> 3)) * H + h]);
     wait(bar_in, par, 11);
-    const int j = tid & 127;
-    if (half == 0) {
-      float G = 0.f;
-#pragma unroll 8
-      for (int t = 0; t < 32; ++t) G += ldbf(sm + R_DSB + sw128_off(t, j, 64));
-      s_x[j] = G;
-    }
-    __syncthreads();
+    __syncthreads();  // s_p of S0
 
-    // ---- S2: transform (the half sums in s_x are consumed and zeroed: the
-    //      same words accumulate dlog gamma next)
-    {
-      float G = 0.f;
-      if (half) {
-        G = s_x[j];
-        s_x[j] = 0.f;
-      }
-      float gprev = half ? __expf(G) : 1.f;
-      const float pj = s_p[j];
-#pragma unroll 4
-      for (int tt = 0; tt < 32; ++tt) {
-        const int t = half * 32 + tt;
-        const uint32_t oj = sw128_off(t, j, 64);
-        const uint32_t ok = sw128_off(t, j, 128);
-        const uint32_t oq = sw128_off(64 + t, j, 128);
-        const float kk = ldbf(sm + R_X + ok);
-        const float qq = ldbf(sm + R_X + oq);
-        const float bb = sigm(ldbf(sm + R_DSB + 16384 + oj) + pj);
-        G += ldbf(sm + R_DSB + oj);
-        const float gam = __expf(G), igam = __fdividef(1.0f, gam);
-        stbf(sm + R_X + ok, kk * gam);
-        stbf(sm + R_X + oq, qq * gprev);
-        const float kh = kk * igam;
-        stbf(sm + R_KH + oj, kh);
-        stbf(sm + R_KP + oj, bb * kh);
-        gprev = gam;
-      }
-      if (half) s_gam[j] = gprev;
-    }
+    // ---- S2: transform; s_x is cleared: it accumulates dlog gamma next
+    tc::transform_block<16>(sm + R_X, sm + R_KH, sm + R_KP, sm + R_DSB,
+                            sm + R_DSB + 16384, s_p, s_gam,
+                            reinterpret_cast<float*>(sm + R_MP), 3);
+    if (tid < 128) s_x[tid] = 0.f;
     {
       const float invL = 1.0f / (float)a.L;
+      const int rr = tid >> 3, ch = tid & 7;  // token row, 16-byte chunk
+      const uint32_t sub = (uint32_t)((rr >> 3) * 1024 + (rr & 7) * 128 + ch * 16);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int cidx = tid + 256 * i;  // 16-byte chunk of a 64 x 128 tile
-        const int kb = cidx >> 9, rr = (cidx >> 3) & 63, ch = cidx & 7;
-        const uint32_t sub = (uint32_t)((rr >> 3) * 1024 + (rr & 7) * 128 + ch * 16);
+      for (int kb = 0; kb < 2; ++kb) {
         // W = w V in place
         {
           const uint32_t off = (uint32_t)(kb * 8192) + sub;
           const uint4 x = *reinterpret_cast<const uint4*>(sm + R_W + off);
-          const float wt = s_w[rr];
           const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
           uint4 y;
           uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(xv[e]);
-            yv[e] = pack2(f.x * wt, f.y * wt);
+            yv[e] = pack2(f.x * wrow, f.y * wrow);
           }
           *reinterpret_cast<uint4*>(sm + R_W + off) = y;
         }
@@ -349,14 +361,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t off = (uint32_t)(kb * 16384 + 8192) + sub;
           const uint4 x = *reinterpret_cast<const uint4*>(sm + R_RO + off);
           const int v0 = kb * 64 + ((ch ^ (rr & 7)) << 3);
+          const float4 m0 = *reinterpret_cast<const float4*>(s_dmn + v0);
+          const float4 m1 = *reinterpret_cast<const float4*>(s_dmn + v0 + 4);
+          const float dm8[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
           const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
           uint4 y;
           uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(xv[e]);
-            yv[e] = pack2(f.x + s_dmn[v0 + 2 * e] * invL,
-                          f.y + s_dmn[v0 + 2 * e + 1] * invL);
+            yv[e] = pack2(fmaf(dm8[2 * e], invL, f.x), fmaf(dm8[2 * e + 1], invL, f.y));
           }
           *reinterpret_cast<uint4*>(sm + R_RO + off) = y;
         }
@@ -385,58 +399,54 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- S4: dS~ = dS Diag(gamma) (TMEM, and its bf16 operand over the
     //      consumed raw g, b_x) with dlog gamma_j = sum_v dS S_new; then the
-    //      strictly lower [M; P_k] (warps 4-7) and P_kap (warps 2-3) operands
+    //      strictly lower [M; P_k] and P_kap operands
     {
-      const int c0 = half * 64;
+      const int c0 = gp * 32;
       const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
                         (size_t)row * kDK + c0;
-      float prod[64];
+      float vals[32], prod[32];
+      tmem_ld32(tl + T_DS + c0, vals);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_DS + c0 + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(sn + part * 32 + e);
-          prod[part * 32 + e] = vals[e] * x.x;
-          prod[part * 32 + e + 1] = vals[e + 1] * x.y;
-          prod[part * 32 + e + 2] = vals[e + 2] * x.z;
-          prod[part * 32 + e + 3] = vals[e + 3] * x.w;
-        }
-#pragma unroll
-        for (int e = 0; e < 32; ++e) vals[e] *= s_gam[c0 + part * 32 + e];
-        tmem_st32(tl + T_DS + c0 + part * 32, vals);
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + R_DSB + sw128_chunk(row, half, part * 4 + c8, 128),
-                   vals + c8 * 8);
+      for (int e = 0; e < 32; e += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(sn + e);
+        prod[e] = vals[e] * x.x;
+        prod[e + 1] = vals[e + 1] * x.y;
+        prod[e + 2] = vals[e + 2] * x.z;
+        prod[e + 3] = vals[e + 3] * x.w;
       }
-      float hi[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) hi[i] = prod[32 + i];
-      const float s_lo = warp_reduce_scatter32(prod, lane);
-      const float s_hi = warp_reduce_scatter32(hi, lane);
-      atomicAdd(&s_x[c0 + lane], s_lo);
-      atomicAdd(&s_x[c0 + 32 + lane], s_hi);
+      for (int e = 0; e < 32; e += 4) {
+        const float4 gm = *reinterpret_cast<const float4*>(s_gam + c0 + e);
+        vals[e] *= gm.x; vals[e + 1] *= gm.y; vals[e + 2] *= gm.z; vals[e + 3] *= gm.w;
+      }
+      tmem_st32(tl + T_DS + c0, vals);
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_chunk(sm + R_DSB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
+                 vals + c8 * 8);
+      atomicAdd(&s_x[c0 + lane], warp_reduce_scatter32(prod, lane));
     }
     wait(bar1, par, 12);
     tc_fence_after();
-    const int gi = row, gr = gi < 64 ? gi : gi - 64;
-    if (half == 1 || gi >= 64) {
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_G + (half ? 64 : 0) + part * 32, vals);
+    {
+      const int gr = row < 64 ? row : row - 64;
+      const bool mp = gp < 2;
+      if (mp || row >= 64) {
+        const int piece = gp & 1;
+        float vals[32];
+        tmem_ld32(tl + T_G + (mp ? 64 : 0) + piece * 32, vals);
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          if (part * 32 + e >= gr) vals[e] = 0.f;
-        if (half) {
+          if (piece * 32 + e >= gr) vals[e] = 0.f;
+        if (mp) {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8)
-            st_chunk(sm + R_MP + sw128_chunk(gi, 0, part * 4 + c8, 128),
+            st_chunk(sm + R_MP + sw128_chunk(row, 0, piece * 4 + c8, 128),
                      vals + c8 * 8);
         } else {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8)
-            st_chunk(sm + R_PQ + sw128_chunk(gr, 0, part * 4 + c8, 64),
+            st_chunk(sm + R_PQ + sw128_chunk(gr, 0, piece * 4 + c8, 64),
                      vals + c8 * 8);
         }
       }
@@ -468,12 +478,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(bar3, par, 14);
     tc_fence_after();
 
-    // ---- S7: dE -> RO rows 0..63 (tokens split between the halves);
+    // ---- S7: dE -> RO rows 0..63 (16 tokens per column group);
     //      dR^T = dE^T T
-    tmem_ld32(tl + T_DER + half * 32, vals);
+    {
+      float vals[16];
+      tmem_ld16(tl + T_DER + gp * 16, vals);
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      stbf(sm + R_RO + sw128_off(half * 32 + e, row, 128), vals[e]);
+      for (int e = 0; e < 16; ++e)
+        stbf(sm + R_RO + sw128_off(gp * 16 + e, row, 128), vals[e]);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -492,10 +505,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
 
     // ---- S8: dR -> RO rows 0..63
-    tmem_ld32(tl + T_DER + half * 32, vals);
+    {
+      float vals[16];
+      tmem_ld16(tl + T_DER + gp * 16, vals);
 #pragma unroll
-    for (int e = 0; e < 32; ++e)
-      stbf(sm + R_RO + sw128_off(half * 32 + e, row, 128), vals[e]);
+      for (int e = 0; e < 16; ++e)
+        stbf(sm + R_RO + sw128_off(gp * 16 + e, row, 128), vals[e]);
+    }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -535,7 +551,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(bar5, par, 16);
     tc_fence_after();
 
-    // ---- S10: reload raw g, b_x into SB; G2 (masked, bf16); dv, dw
+    // ---- S10: reload raw g, b_x into SB; G2 (masked, bf16; 32 columns per
+    //      group); dv, dw (16 tokens per group)
     if (tid == 0 && !*s_abort) {
       mbar_expect_tx(bar_gb, 2 * 16384);
       tma_load_3d(sm + R_SB, &tm_g, bar_gb, 0, h, tok);
@@ -543,41 +560,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(sm + R_SB + 16384, &tm_bx, bar_gb, 0, h, tok);
       tma_load_3d(sm + R_SB + 24576, &tm_bx, bar_gb, 64, h, tok);
     }
-    if (half == 1) {
+    {
       const int rl = row & 63;
+      float vals[32];
+      tmem_ld32(tl + T_G2 + gp * 32, vals);
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        tmem_ld32(tl + T_G2 + q4 * 32, vals);
+      for (int e = 0; e < 32; ++e)
+        if (((gp & 1) * 32 + e) >= rl) vals[e] = 0.f;
+      uint8_t* blk = sm + ((gp >> 1) == 0 ? R_MP : R_PQ);
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (((q4 & 1) * 32 + e) >= rl) vals[e] = 0.f;
-        uint8_t* blk = sm + ((q4 >> 1) == 0 ? R_MP : R_PQ);
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(blk + sw128_chunk(row, 0, (q4 & 1) * 4 + c8, 128), vals + c8 * 8);
-      }
-      fence_async_smem();
-    } else {
-      float prod[64];
-      __nv_bfloat16* dvrow = dv + (size_t)tok * H * kDV + (size_t)h * kDV + row;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_RE + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int t = part * 32 + e;
-          dvrow[(size_t)t * H * kDV] = __float2bfloat16_rn(s_w[t] * vals[e]);
-          prod[t] = vals[e] * ldbf(sm + R_W + sw128_off(t, row, 64));
-        }
-      }
-      float hi[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) hi[i] = prod[32 + i];
-      const float s_lo = warp_reduce_scatter32(prod, lane);
-      const float s_hi = warp_reduce_scatter32(hi, lane);
-      atomicAdd(&s_dw[lane], s_lo);
-      atomicAdd(&s_dw[32 + lane], s_hi);
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_chunk(blk + sw128_chunk(row, 0, (gp & 1) * 4 + c8, 128), vals + c8 * 8);
     }
+    {
+      float vals[16], prod[16];
+      tmem_ld16(tl + T_RE + gp * 16, vals);
+      __nv_bfloat16* dvrow = dv + ((size_t)tok + gp * 16) * H * kDV +
+                             (size_t)h * kDV + row;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = gp * 16 + e;
+        dvrow[(size_t)e * H * kDV] = __float2bfloat16_rn(s_w[t] * vals[e]);
+        prod[e] = vals[e] * ldbf(sm + R_W + sw128_off(t, row, 64));
+      }
+      const float sdw = warp_reduce_scatter16(prod, lane);
+      if (lane < 16) atomicAdd(&s_dw[gp * 16 + lane], sdw);
+    }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     if (*s_abort) break;
@@ -619,34 +628,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(bar_gb, par, 18);
     tc_fence_after();
 
-    // ---- S12: per key channel j: dq, dk, db_x, dg, dp.  Pass 1 (ascending
-    //      tokens) carries Gamma and forms every per-token gradient and the
-    //      log-Gamma gradients dG_t; pass 2 (descending) sums dg_t = sum_{s>=t} dG_s.
+    // ---- S12: per key channel j = row and token quarter gp: dq, dk, db_x,
+    //      dg, dp.  Ascending pass: Gamma from the quarter's log-decay prefix,
+    //      every per-token gradient and the log-Gamma gradients dG_t;
+    //      descending pass: dg_t = sum_{s >= t} dG_s with the later quarters'
+    //      sums exchanged through shared memory.
     {
-      const int jj = row;                 // key channel (TMEM lane)
-      const int tb = half == 0 ? 32 : 0;  // token range [tb, tb + 32)
+      const int jj = row;
+      const int tb = gp * 16;             // token range [tb, tb + 16)
+      float* s_gq = s_scr;                // [4][128] quarter log-decay sums
+      float* s_lq = s_scr + 512;          // [4][128] quarter dG sums
+      float* s_qf = s_scr + 1024;         // [4][128] dQ~ Q~ of a quarter's first token
+      {
+        float gsum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) gsum += ldbf(sm + R_SB + sw128_off(tb + e, jj, 64));
+        s_gq[gp * 128 + jj] = gsum;
+      }
+      __syncthreads();
+      float G = 0.f;                      // log Gamma before the range
+      for (int g2 = 0; g2 < gp; ++g2) G += s_gq[g2 * 128 + jj];
       const float pj = s_p[jj];
       const size_t tstride = (size_t)H * kDK;
       const size_t x0 = ((size_t)tok * H + h) * kDK + jj;
-      float Gs = 0.f;                     // log Gamma before the range
-      if (half == 0) {
-#pragma unroll 8
-        for (int t = 0; t < 32; ++t) Gs += ldbf(sm + R_SB + sw128_off(t, jj, 64));
-      }
-      float G = Gs, gprev = __expf(Gs);
-      float dGv[32];
-      float qfirst = 0.f;                 // dQ~ Q~ of the range's first token
-      float d7k[16], d7q[16], d8p[16], d8h[16];
+      float gprev = __expf(G);
+      float dGv[16];
+      float qfirst = 0.f;
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
-        const int tsub = tb + 16 * sub;
-        tmem_ld16(tl + T_G + tsub, d7k);
-        tmem_ld16(tl + T_G + 64 + tsub, d7q);
-        tmem_ld16(tl + T_RE + tsub, d8p);
-        tmem_ld16(tl + T_RE + 64 + tsub, d8h);
+        float d7k[8], d7q[8], d8p[8], d8h[8];
+        const int tsub = tb + 8 * sub;
+        tmem_ld8(tl + T_G + tsub, d7k);
+        tmem_ld8(tl + T_G + 64 + tsub, d7q);
+        tmem_ld8(tl + T_RE + tsub, d8p);
+        tmem_ld8(tl + T_RE + 64 + tsub, d8h);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int tl_ = 16 * sub + e;
+        for (int e = 0; e < 8; ++e) {
+          const int tl_ = 8 * sub + e;
           const int t = tb + tl_;
           const uint32_t o64 = sw128_off(t, jj, 64);
           G += ldbf(sm + R_SB + o64);
@@ -672,53 +690,66 @@ __global__ void __launch_bounds__(kThreads, 1)
           gprev = gam;
         }
       }
-      if (half == 0) {
-        dGv[31] += s_x[jj];                 // t = 63: gradient of log gamma
-        float tot = qfirst;                 // dG_31 (lower half) reads Q~_32
+      float lsum = 0.f;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) tot += dGv[i];
-        s_gam[jj] = tot;                    // hand-off to the lower half
-      }
+      for (int i = 0; i < 16; ++i) lsum += dGv[i];
+      s_lq[gp * 128 + jj] = lsum;
+      s_qf[gp * 128 + jj] = qfirst;
       __syncthreads();
-      float acc = half == 1 ? s_gam[jj] : 0.f;
+      // dG_{tb+15} reads the next quarter's first Q~ term (t = 63: the
+      // gradient of log gamma); the later quarters' sums seed the suffix
+      const float dlg = s_x[jj];
+      dGv[15] += gp < 3 ? s_qf[(gp + 1) * 128 + jj] : dlg;
+      float acc = 0.f;
+      for (int g2 = gp + 1; g2 < 4; ++g2)
+        acc += s_lq[g2 * 128 + jj] + (g2 < 3 ? s_qf[(g2 + 1) * 128 + jj] : dlg);
 #pragma unroll
-      for (int i = 31; i >= 0; --i) {
+      for (int i = 15; i >= 0; --i) {
         acc += dGv[i];
         dg[x0 + (size_t)(tb + i) * tstride] = __float2bfloat16_rn(acc);
       }
     }
 
-    // ---- S13: gate of chunk c once all its blocks are done
+    // ---- S13: gate of chunk c once all its blocks are done:
+    //      dp_j -> dh = U_up^T dp -> dm = U_down^T dh
     if (chunk_first) {
-      if (half == 0) s_x[row] = dp_acc;
+      float* s_dpq = s_scr + 2048;        // [4][128] dp quarter sums
+      float* s_dhq = s_scr + 2560;        // [4][32] dh partials (per quadrant)
+      float* s_dmq = s_scr + 2688;        // [4][128] dm partials (per group)
+      s_dpq[gp * 128 + row] = dp_acc;
       __syncthreads();
-      if (half == 1) {
-        const float dpj = s_x[row] + dp_acc;
-        s_x[row] = dpj;
-        rec[row] = dpj;
-      }
-      __syncthreads();
-      if (half == 0) {  // dh[r] = sum_j U_up[j][r] dp[j]
-        float pr[kRMax];
-        const float dpj = s_x[tid];
+      const float dpj = s_dpq[row] + s_dpq[128 + row] + s_dpq[256 + row] +
+                        s_dpq[384 + row];
+      if (gp == 0) rec[row] = dpj;
+      {  // dh[r], r = 8 gp + i: this quadrant's channels
+        float pr[8];
 #pragma unroll
-        for (int r = 0; r < kRMax; ++r) pr[r] = ureg[r] * dpj;
-        const float part = warp_reduce_scatter32(pr, lane);
-        s_gam[warp * 32 + lane] = part;
+        for (int i = 0; i < 4; ++i) {
+          pr[2 * i] = bf_lo(uup[i]) * dpj;
+          pr[2 * i + 1] = bf_hi(uup[i]) * dpj;
+        }
+        const float part = warp_reduce_scatter8(pr, lane);
+        if (lane < 8) s_dhq[qd * 32 + gp * 8 + lane] = part;
       }
       __syncthreads();
       if (tid < 32) {
-        const float dhv = s_gam[tid] + s_gam[32 + tid] + s_gam[64 + tid] + s_gam[96 + tid];
+        const float dhv = s_dhq[tid] + s_dhq[32 + tid] + s_dhq[64 + tid] + s_dhq[96 + tid];
         s_dw[tid] = dhv;
         if (tid < R) rec[kDK + tid] = dhv;
       }
       __syncthreads();
-      if (half == 1) {  // dm[v] = sum_r U_down[r][v] dh[r]
+      {  // dm[v] partial over r = 8 gp .. 8 gp + 7, v = row
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < kRMax; ++r) acc = fmaf(ureg[r], s_dw[r], acc);
-        s_dmn[row] = acc;
+        for (int i = 0; i < 4; ++i) {
+          acc = fmaf(bf_lo(udn[i]), s_dw[8 * gp + 2 * i], acc);
+          acc = fmaf(bf_hi(udn[i]), s_dw[8 * gp + 2 * i + 1], acc);
+        }
+        s_dmq[gp * 128 + row] = acc;
       }
+      __syncthreads();
+      if (tid < 128)
+        s_dmn[tid] = s_dmq[tid] + s_dmq[128 + tid] + s_dmq[256 + tid] + s_dmq[384 + tid];
       dp_acc = 0.f;
     }
     fence_async_smem();
@@ -728,17 +759,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- dS0, dm0
   if (!*s_abort) {
-    const int c0 = half * 64;
+    const int c0 = gp * 32;
     if (a.dS0) {
       float* dst = a.dS0 + (size_t)pair * SZ + (size_t)row * kDK + c0;
+      float vals[32];
+      tmem_ld32(tl + T_DS + c0, vals);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + T_DS + c0 + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4*>(dst + part * 32 + e) =
-              make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
-      }
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dst + e) =
+            make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
     }
     if (a.dm0 && tid < 128) a.dm0[(size_t)pair * kDV + tid] = s_dmn[tid];
   }

@@ -37,8 +37,10 @@ namespace carve {
 namespace {
 
 using namespace ptx;
+using tc::bar_named;
 using tc::fsw;
-using tc::sigm;
+using tc::pack2;
+using tc::st_chunk;
 using tc::unit_lower_inverse64;
 
 constexpr int kThreads = 256;
@@ -63,10 +65,8 @@ constexpr uint32_t OFF_AF = 196608;    // A fp32 64 x 64 row-major     16 KB
 constexpr uint32_t OFF_SMALL = 212992;
 constexpr uint32_t SM_GAM = 0;         // gamma_j            128 f32
 constexpr uint32_t SM_P = 512;         // (U_b m)_j          128 f32
-constexpr uint32_t SM_W = 1024;        // w_t                 64 f32
 constexpr uint32_t SM_M = 1280;        // m_v                128 f32
 constexpr uint32_t SM_H = 1792;        // U_down m            64 f32
-constexpr uint32_t SM_HALF = 2048;     // half-block g sums  128 f32
 constexpr uint32_t SM_BAR = 2560;      // 6 mbarriers
 constexpr uint32_t SM_TMEM = 2624;     // TMEM base address
 constexpr uint32_t SM_ABORT = 2628;    // abort flag
@@ -92,30 +92,6 @@ constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false
 
 constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
 
-__device__ __forceinline__ float ldbf(const uint8_t* p) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p));
-}
-__device__ __forceinline__ void stbf(uint8_t* p, float x) {
-  *reinterpret_cast<__nv_bfloat16*>(p) = __float2bfloat16_rn(x);
-}
-__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-__device__ __forceinline__ void bar_named(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
-// 8 fp32 values -> one 16-byte chunk of bf16 at `p`.
-__device__ __forceinline__ void st_chunk(uint8_t* p, const float* x) {
-  uint4 u;
-  u.x = pack2(x[0], x[1]);
-  u.y = pack2(x[2], x[3]);
-  u.z = pack2(x[4], x[5]);
-  u.w = pack2(x[6], x[7]);
-  *reinterpret_cast<uint4*>(p) = u;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -127,10 +103,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* s_gam = reinterpret_cast<float*>(sm + OFF_SMALL + SM_GAM);
   float* s_p = reinterpret_cast<float*>(sm + OFF_SMALL + SM_P);
-  float* s_w = reinterpret_cast<float*>(sm + OFF_SMALL + SM_W);
   float* s_m = reinterpret_cast<float*>(sm + OFF_SMALL + SM_M);
   float* s_h = reinterpret_cast<float*>(sm + OFF_SMALL + SM_H);
-  float* s_half = reinterpret_cast<float*>(sm + OFF_SMALL + SM_HALF);
   float* s_af = reinterpret_cast<float*>(sm + OFF_AF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_SMALL + SM_BAR);
   uint64_t* bar_vgb = bars + 0;  // TMA v, g, b_x
@@ -324,43 +298,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_3d(&tm_bx, x0, h, tn);
       }
     }
+    // w_t of the two token rows this thread scales in W = w V
+    const float w_lo = __bfloat162float(w_in[((size_t)b * T + t0 + (tid >> 3)) * H + h]);
+    const float w_hi = __bfloat162float(w_in[((size_t)b * T + t0 + (tid >> 3) + 32) * H + h]);
     wait(bar_vgb, par, 1);
     wait(bar_kq, par, 2);
-    if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)b * T + t0 + tid) * H + h]);
-    const int j = tid & 127;  // key channel of this thread in the transform
-    if (half == 0) {
-      float G = 0.f;
-#pragma unroll 8
-      for (int t = 0; t < 32; ++t) G += ldbf(sm + OFF_RG + sw128_off(t, j, 64));
-      s_half[j] = G;
-    }
-    __syncthreads();
 
     // ---- 2. transform: decay scan, gated and decayed operands, W = w V
-    {
-      float G = half ? s_half[j] : 0.f;
-      float gprev = half ? __expf(G) : 1.f;  // Gamma_{t-1}
-      const float pj = s_p[j];
-#pragma unroll 4
-      for (int tt = 0; tt < 32; ++tt) {
-        const int t = half * 32 + tt;
-        const uint32_t oj = sw128_off(t, j, 64);
-        const uint32_t ok = sw128_off(t, j, 128);
-        const uint32_t oq = sw128_off(64 + t, j, 128);
-        const float kk = ldbf(sm + OFF_X + ok);
-        const float qq = ldbf(sm + OFF_X + oq);
-        const float bb = sigm(ldbf(sm + OFF_RB + oj) + pj);
-        G += ldbf(sm + OFF_RG + oj);
-        const float gam = __expf(G), igam = __fdividef(1.0f, gam);
-        stbf(sm + OFF_X + ok, kk * gam);
-        stbf(sm + OFF_X + oq, qq * gprev);
-        const float kh = kk * igam;
-        stbf(sm + OFF_KH + oj, kh);
-        stbf(sm + OFF_KP + oj, bb * kh);
-        gprev = gam;
-      }
-      if (half) s_gam[j] = gprev;
-    }
+    tc::transform_block<8>(sm + OFF_X, sm + OFF_KH, sm + OFF_KP, sm + OFF_RG,
+                        sm + OFF_RB, s_p, s_gam, s_af, 3);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int c = tid + 256 * i;  // 16-byte chunk of the 64 x 128 v tile
@@ -368,7 +314,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t off = (uint32_t)((c >> 9) * 8192 + (rr >> 3) * 1024 +
                                       (rr & 7) * 128 + (c & 7) * 16);
       const uint4 x = *reinterpret_cast<const uint4*>(sm + OFF_RV + off);
-      const float wt = s_w[rr];
+      const float wt = (i & 1) ? w_hi : w_lo;
       const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
       uint4 y;
       uint32_t* yv = reinterpret_cast<uint32_t*>(&y);

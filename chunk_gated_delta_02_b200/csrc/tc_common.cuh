@@ -41,6 +41,127 @@ __device__ __forceinline__ void st_chunk(uint8_t* p, const float* x) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
+// 16-byte chunk of bf16 -> 8 fp32 values.
+__device__ __forceinline__ void ld_chunk(const uint8_t* p, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
+
+// Element-wise transform of one block of 64 tokens x 128 key channels (CARVE
+// summaries, gist.science, section 2.3: decay on the key axis; section 2.1:
+// the content gate b = sigmoid(b_x + U_b m_c)):
+//   Gamma_t = exp(sum_{u <= t} g_u)   K~ = K Gamma    Q~_t = Q_t Gamma_{t-1}
+//   K^ = K / Gamma                    kap^ = b K^     gamma = Gamma_63
+// All tiles are 128-byte swizzled 64-column blocks.  `x` holds [K; Q]
+// (128 rows per column block; rewritten in place to [K~; Q~]), `graw` and
+// `braw` raw g and b_x (64 rows per column block), `kh`, `kp` receive K^ and
+// kap^, `s_gam` gamma.  `s_p` holds p_j = (U_b m_c)_j; `red` is NW * 64
+// floats of scratch.  Called by NW warps: half of them per column block;
+// thread (chunk of 8 channels, group of TPT = 128 / (4 NW) consecutive
+// tokens) touches one 16-byte chunk per row, the 8 threads of a
+// quarter-warp the 8 chunks of one row (conflict-free under the swizzle).
+// The log-decay prefix over the token groups is a shuffle scan inside each
+// warp plus the totals of the preceding warps (named barriers bar_id,
+// bar_id + 1 for the two column blocks).
+template <int NW>
+__device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
+                                                uint8_t* kp,
+                                                const uint8_t* graw,
+                                                const uint8_t* braw,
+                                                const float* s_p, float* s_gam,
+                                                float* red, int bar_id) {
+  constexpr int WPB = NW / 2;         // warps per column block
+  constexpr int TPT = 64 / (4 * WPB); // tokens per thread
+  constexpr int NG = 64 / TPT;        // token groups
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = warp / WPB, wq = warp % WPB, ch = lane & 7, t4 = lane >> 3;
+  const int tg = wq * 4 + t4;        // tokens TPT tg .. TPT tg + TPT - 1
+  const int j0 = blk * 64 + ch * 8;  // channels j0 .. j0 + 7
+  auto off64 = [&](int t) {
+    return (uint32_t)(blk * 8192 + t * 128 + ((ch ^ (t & 7)) << 4));
+  };
+  auto off128 = [&](int t) {
+    return (uint32_t)(blk * 16384 + t * 128 + ((ch ^ (t & 7)) << 4));
+  };
+  float gl[TPT][8];  // inclusive log-decay sums inside the token group
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) {
+    float gv[8];
+    ld_chunk(graw + off64(TPT * tg + i), gv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
+  }
+  float ex[8];  // exclusive prefix of the token group
+  float wt[8];  // running inclusive sum over the warp's groups
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float tot = gl[TPT - 1][e];
+    float incl = tot;
+    float v = __shfl_up_sync(0xffffffffu, incl, 8);
+    if (t4 >= 1) incl += v;
+    v = __shfl_up_sync(0xffffffffu, incl, 16);
+    if (t4 >= 2) incl += v;
+    ex[e] = incl - tot;
+    wt[e] = incl;  // t4 == 3: the warp's total
+  }
+  if (t4 == 3) {
+    *reinterpret_cast<float4*>(red + wq * 128 + j0) =
+        make_float4(wt[0], wt[1], wt[2], wt[3]);
+    *reinterpret_cast<float4*>(red + wq * 128 + j0 + 4) =
+        make_float4(wt[4], wt[5], wt[6], wt[7]);
+  }
+  bar_named(bar_id + blk, WPB * 32);
+  for (int w2 = 0; w2 < wq; ++w2) {
+    const float4 a = *reinterpret_cast<const float4*>(red + w2 * 128 + j0);
+    const float4 b = *reinterpret_cast<const float4*>(red + w2 * 128 + j0 + 4);
+    ex[0] += a.x; ex[1] += a.y; ex[2] += a.z; ex[3] += a.w;
+    ex[4] += b.x; ex[5] += b.y; ex[6] += b.z; ex[7] += b.w;
+  }
+  float pj[8], gprev[8];
+  {
+    const float4 a = *reinterpret_cast<const float4*>(s_p + j0);
+    const float4 b = *reinterpret_cast<const float4*>(s_p + j0 + 4);
+    pj[0] = a.x; pj[1] = a.y; pj[2] = a.z; pj[3] = a.w;
+    pj[4] = b.x; pj[5] = b.y; pj[6] = b.z; pj[7] = b.w;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) gprev[e] = __expf(ex[e]);  // Gamma_{TPT tg - 1}
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) {
+    const int t = TPT * tg + i;
+    float kv[8], qv[8], bv[8], o_kt[8], o_qt[8], o_kh[8], o_kp[8];
+    ld_chunk(x + off128(t), kv);
+    ld_chunk(x + off128(64 + t), qv);
+    ld_chunk(braw + off64(t), bv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float gam = __expf(ex[e] + gl[i][e]);
+      const float igam = __fdividef(1.0f, gam);
+      const float bb = sigm(bv[e] + pj[e]);
+      o_kt[e] = kv[e] * gam;
+      o_qt[e] = qv[e] * gprev[e];
+      o_kh[e] = kv[e] * igam;
+      o_kp[e] = bb * o_kh[e];
+      gprev[e] = gam;
+    }
+    st_chunk(x + off128(t), o_kt);
+    st_chunk(x + off128(64 + t), o_qt);
+    st_chunk(kh + off64(t), o_kh);
+    st_chunk(kp + off64(t), o_kp);
+  }
+  if (tg == NG - 1) {  // gamma = Gamma_63
+    *reinterpret_cast<float4*>(s_gam + j0) =
+        make_float4(gprev[0], gprev[1], gprev[2], gprev[3]);
+    *reinterpret_cast<float4*>(s_gam + j0 + 4) =
+        make_float4(gprev[4], gprev[5], gprev[6], gprev[7]);
+  }
+}
+
 constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
 
 // Bounded wait on an mbarrier phase.  On expiry: record CARVE_ERR_TIMEOUT
