@@ -67,12 +67,24 @@ constexpr uint32_t SM_X = 1024;      // g half sums | dlog gamma | dp   128 f32
 constexpr uint32_t SM_GAM = 1536;    // gamma | dg hand-off | dh parts  128 f32
 constexpr uint32_t SM_W = 2048;      // w_t                 64 f32
 constexpr uint32_t SM_DW = 2304;     // dw sums | dh        64 f32
-constexpr uint32_t SM_BAR = 2560;    // 8 mbarriers
-constexpr uint32_t SM_TMEM = 2624;
-constexpr uint32_t SM_ABORT = 2628;
+constexpr uint32_t SM_BAR = 2560;    // 9 mbarriers
+constexpr uint32_t SM_TMEM = 2640;
+constexpr uint32_t SM_ABORT = 2644;
 constexpr uint32_t kSmemBytes = 232448;
 static_assert(R_SM + 2688 <= kSmemBytes, "small region");
 static_assert(R_PQ == R_MP + 16384 && R_TT == R_PQ + 8192, "G2 blocks");
+
+// mbarriers (index into the small region's array)
+constexpr int B_IN = 0;    // k, q, d_o of this block
+constexpr int B_GB = 1;    // raw g, b_x again for the epilogue
+constexpr int B_1 = 2;     // MMA S3
+constexpr int B_SB = 3;    // bf16 state record
+constexpr int B_3 = 4;     // MMA S6
+constexpr int B_4 = 5;     // MMA S7
+constexpr int B_5 = 6;     // MMA S9
+constexpr int B_7 = 7;     // MMA S11
+constexpr int B_PRE = 8;   // v, g, b_x, E^T and T records
+constexpr int kNumBars = 9;
 
 // TMEM columns
 constexpr uint32_t T_DS = 0;     // dS [v][j]
@@ -169,19 +181,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_w = reinterpret_cast<float*>(sm + R_SM + SM_W);
   float* s_dw = reinterpret_cast<float*>(sm + R_SM + SM_DW);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + R_SM + SM_BAR);
-  uint64_t* bar_in = bars + 0;
-  uint64_t* bar_gb = bars + 1;
-  uint64_t* bar1 = bars + 2;
-  uint64_t* bar3 = bars + 4;
-  uint64_t* bar4 = bars + 5;
-  uint64_t* bar5 = bars + 6;
-  uint64_t* bar7 = bars + 7;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + R_SM + SM_TMEM);
   volatile uint32_t* s_abort =
       reinterpret_cast<volatile uint32_t*>(sm + R_SM + SM_ABORT);
-  // fp32 scratch of the epilogue and the gate backward (the dO / dR buffer
-  // is free once the last MMA that reads it retired)
-  float* s_scr = reinterpret_cast<float*>(sm + R_RO);
+  // fp32 scratch of the epilogue and the gate backward (the G2 buffer is
+  // free once the last MMA that reads it retired)
+  float* s_scr = reinterpret_cast<float*>(sm + R_MP);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, gp = warp >> 2;
@@ -213,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     return;
   }
   if (tid == 0) {
-    for (int i = 0; i < 8; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
     *s_abort = 0;
     mbar_init_fence();
     prefetch_tmap(&tm_q);
@@ -269,20 +274,77 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (tid < 128) s_dmn[tid] = a.dm_T ? a.dm_T[(size_t)pair * kDV + tid] : 0.f;
 
-  auto wait = [&](uint64_t* bar, uint32_t par, uint32_t where) {
-    wait_bar(bar, par, where, s_abort, a.hdr);
+  // Every barrier has at most one phase in flight.  `npar` holds the parity
+  // each thread waits for next; thread 0 also tracks in `pend` the phases it
+  // started (copies issued, MMAs committed) so that an aborting CTA drains
+  // them before it exits.
+  uint32_t npar = 0, pend = 0;
+  auto wait = [&](int i, uint32_t where) {
+    if (wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr)) {
+      npar ^= 1u << i;
+      pend &= ~(1u << i);
+    }
   };
+  auto mark = [&](int i) { pend |= 1u << i; };
+  auto tok_of = [&](int blk) { return b * T + blk * kBlk; };
+  const uint8_t* rec0 = a.tc_rec + (size_t)pair * NB * kTcRecBytes;
+  // k, q -> X; d_o -> RO rows 64..127
+  auto issue_top = [&](int blk) {
+    const int tk = tok_of(blk);
+    mbar_expect_tx(bars + B_IN, 3 * 16384);
+    tma_load_3d(sm + R_X, &tm_k, bars + B_IN, 0, h, tk);
+    tma_load_3d(sm + R_X + 16384, &tm_k, bars + B_IN, 64, h, tk);
+    tma_load_3d(sm + R_X + 8192, &tm_q, bars + B_IN, 0, h, tk);
+    tma_load_3d(sm + R_X + 24576, &tm_q, bars + B_IN, 64, h, tk);
+    tma_load_3d(sm + R_RO + 8192, &tm_do, bars + B_IN, 0, h, tk);
+    tma_load_3d(sm + R_RO + 24576, &tm_do, bars + B_IN, 64, h, tk);
+    mark(B_IN);
+  };
+  // the block's bf16 state operand (forward record) -> SB
+  auto issue_sb = [&](int blk) {
+    mbar_expect_tx(bars + B_SB, 32768);
+    bulk_load(sm + R_SB, rec0 + (size_t)blk * kTcRecBytes + kTcRecS, 32768,
+              bars + B_SB);
+    mark(B_SB);
+  };
+  // v -> W; g, b_x -> DSB; records E^T -> ET, T -> TT
+  auto issue_pre = [&](int blk) {
+    const int tk = tok_of(blk);
+    const uint8_t* r = rec0 + (size_t)blk * kTcRecBytes;
+    mbar_expect_tx(bars + B_PRE, 4 * 16384 + 8192);
+    tma_load_3d(sm + R_W, &tm_v, bars + B_PRE, 0, h, tk);
+    tma_load_3d(sm + R_W + 8192, &tm_v, bars + B_PRE, 64, h, tk);
+    tma_load_3d(sm + R_DSB, &tm_g, bars + B_PRE, 0, h, tk);
+    tma_load_3d(sm + R_DSB + 8192, &tm_g, bars + B_PRE, 64, h, tk);
+    tma_load_3d(sm + R_DSB + 16384, &tm_bx, bars + B_PRE, 0, h, tk);
+    tma_load_3d(sm + R_DSB + 24576, &tm_bx, bars + B_PRE, 64, h, tk);
+    bulk_load(sm + R_ET, r + kTcRecE, 16384, bars + B_PRE);
+    bulk_load(sm + R_TT, r + kTcRecT, 8192, bars + B_PRE);
+    mark(B_PRE);
+  };
+  // raw g, b_x again for the epilogue -> RO
+  auto issue_gb = [&](int blk) {
+    const int tk = tok_of(blk);
+    mbar_expect_tx(bars + B_GB, 2 * 16384);
+    tma_load_3d(sm + R_RO, &tm_g, bars + B_GB, 0, h, tk);
+    tma_load_3d(sm + R_RO + 8192, &tm_g, bars + B_GB, 64, h, tk);
+    tma_load_3d(sm + R_RO + 16384, &tm_bx, bars + B_GB, 0, h, tk);
+    tma_load_3d(sm + R_RO + 24576, &tm_bx, bars + B_GB, 64, h, tk);
+    mark(B_GB);
+  };
+  if (tid == 0) {
+    issue_sb(NB - 1);
+    issue_pre(NB - 1);
+  }
 
   float dp_acc = 0.f;   // dp_j share (channel row, this warp's token quarter)
-  for (int ib = NB - 1, it = 0; ib >= 0; --ib, ++it) {
-    const uint32_t par = (uint32_t)(it & 1);
+  for (int ib = NB - 1; ib >= 0; --ib) {
     const int t0 = ib * kBlk;
     const int c = ib / bpc;
     const bool chunk_last = (ib + 1) % bpc == 0;  // first visited block of c
     const bool chunk_first = ib % bpc == 0;       // last visited block of c
     const int tok = b * T + t0;
     float* rec = args.gate_rec + ((size_t)pair * NC + c) * GR;
-    const uint8_t* trec = a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes;
 
     // ---- S0: gate of chunk c, p = U_up U_down m_c (forward record)
     if (chunk_last) {
@@ -290,27 +352,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       dp_acc = 0.f;
     }
 
-    // ---- S1: inputs: TMA of k, q, v, d_o, g, b_x; records S, E^T, T
+    // ---- S1: inputs.  k, q, d_o now; the rest was requested during the
+    //      previous block.  Block ib - 1's tiles, record and end state -> L2.
     if (tid == 0) {
-      mbar_expect_tx(bar_in, 6 * 16384 + (uint32_t)kTcRecBytes);
-      tma_load_3d(sm + R_X, &tm_k, bar_in, 0, h, tok);
-      tma_load_3d(sm + R_X + 16384, &tm_k, bar_in, 64, h, tok);
-      tma_load_3d(sm + R_X + 8192, &tm_q, bar_in, 0, h, tok);
-      tma_load_3d(sm + R_X + 24576, &tm_q, bar_in, 64, h, tok);
-      tma_load_3d(sm + R_W, &tm_v, bar_in, 0, h, tok);
-      tma_load_3d(sm + R_W + 8192, &tm_v, bar_in, 64, h, tok);
-      tma_load_3d(sm + R_RO + 8192, &tm_do, bar_in, 0, h, tok);
-      tma_load_3d(sm + R_RO + 24576, &tm_do, bar_in, 64, h, tok);
-      tma_load_3d(sm + R_DSB, &tm_g, bar_in, 0, h, tok);
-      tma_load_3d(sm + R_DSB + 8192, &tm_g, bar_in, 64, h, tok);
-      tma_load_3d(sm + R_DSB + 16384, &tm_bx, bar_in, 0, h, tok);
-      tma_load_3d(sm + R_DSB + 24576, &tm_bx, bar_in, 64, h, tok);
-      bulk_load(sm + R_SB, trec + kTcRecS, 32768, bar_in);
-      bulk_load(sm + R_ET, trec + kTcRecE, 16384, bar_in);
-      bulk_load(sm + R_TT, trec + kTcRecT, 8192, bar_in);
-      if (ib > 0) {  // the next block visited: its tiles, record and end state -> L2
+      issue_top(ib);
+      if (ib > 0) {
         const int tn = tok - kBlk;
-#pragma unroll
+#pragma unroll 1
         for (int x0 = 0; x0 < 128; x0 += 64) {
           tma_prefetch_3d(&tm_k, x0, h, tn);
           tma_prefetch_3d(&tm_q, x0, h, tn);
@@ -319,16 +367,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_prefetch_3d(&tm_g, x0, h, tn);
           tma_prefetch_3d(&tm_bx, x0, h, tn);
         }
-        bulk_prefetch_l2(trec - kTcRecBytes, (uint32_t)kTcRecBytes);
+        bulk_prefetch_l2(rec0 + (size_t)(ib - 1) * kTcRecBytes, (uint32_t)kTcRecBytes);
         const float* nxt = a.ck_S + ((size_t)pair * (NB + 1) + ib) * SZ;
-#pragma unroll
+#pragma unroll 1
         for (int q4 = 0; q4 < 4; ++q4) bulk_prefetch_l2(nxt + q4 * 4096, 16384);
       }
     }
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
     // w_t of the token row this thread scales in W = w V
     const float wrow = __bfloat162float(w_in[((size_t)tok + (tid >> 3)) * H + h]);
-    wait(bar_in, par, 11);
+    wait(B_SB, 10);
+    wait(B_PRE, 11);
+    wait(B_IN, 12);
     __syncthreads();  // s_p of S0
 
     // ---- S2: transform; s_x is cleared: it accumulates dlog gamma next
@@ -376,6 +426,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // the block-end state S_new (dlog gamma), loaded ahead of S4
+    float4 snv[8];
+    {
+      const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
+                        (size_t)row * kDK + gp * 32;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) snv[e] = *reinterpret_cast<const float4*>(sn + 4 * e);
+    }
     fence_async_smem();
     __syncthreads();
     if (*s_abort) break;
@@ -385,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t x0 = smem_u32(sm + R_X), kp0 = smem_u32(sm + R_KP);
       const uint32_t kh0 = smem_u32(sm + R_KH);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
         const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
@@ -394,7 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_G + 64, desc_kmajor_sw128(x0 + kx),
                   desc_kmajor_sw128(kh0 + k64), ID_KK64, ks > 0);
       }
-      umma_commit(bar1);
+      umma_commit(bars + B_1);
+      mark(B_1);
     }
 
     // ---- S4: dS~ = dS Diag(gamma) (TMEM, and its bf16 operand over the
@@ -402,17 +461,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      strictly lower [M; P_k] and P_kap operands
     {
       const int c0 = gp * 32;
-      const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
-                        (size_t)row * kDK + c0;
       float vals[32], prod[32];
       tmem_ld32(tl + T_DS + c0, vals);
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 x = *reinterpret_cast<const float4*>(sn + e);
-        prod[e] = vals[e] * x.x;
-        prod[e + 1] = vals[e + 1] * x.y;
-        prod[e + 2] = vals[e + 2] * x.z;
-        prod[e + 3] = vals[e + 3] * x.w;
+      for (int e = 0; e < 8; ++e) {
+        prod[4 * e] = vals[4 * e] * snv[e].x;
+        prod[4 * e + 1] = vals[4 * e + 1] * snv[e].y;
+        prod[4 * e + 2] = vals[4 * e + 2] * snv[e].z;
+        prod[4 * e + 3] = vals[4 * e + 3] * snv[e].w;
       }
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
@@ -426,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                  vals + c8 * 8);
       atomicAdd(&s_x[c0 + lane], warp_reduce_scatter32(prod, lane));
     }
-    wait(bar1, par, 12);
+    wait(B_1, 13);
     tc_fence_after();
     {
       const int gr = row < 64 ? row : row - 64;
@@ -462,20 +518,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t dsb0 = smem_u32(sm + R_DSB), kp0 = smem_u32(sm + R_KP);
       const uint32_t ro0 = smem_u32(sm + R_RO), pq0 = smem_u32(sm + R_PQ);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 8; ++ks)
         umma_bf16(tmem + T_DER,
                   desc_kmajor_sw128(dsb0 + (ks >> 2) * 16384 + (ks & 3) * 32),
                   desc_kmajor_sw128(kp0 + (ks >> 2) * 8192 + (ks & 3) * 32),
                   ID_KK64_NA, ks > 0);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + T_DER,
                   desc_mnmajor_sw128(ro0 + 8192 + ks * 2048, 16384),
                   desc_mnmajor_sw128(pq0 + ks * 2048, 8192), ID_MM64_NA, 1);
-      umma_commit(bar3);
+      umma_commit(bars + B_3);
+      mark(B_3);
     }
-    wait(bar3, par, 14);
+    wait(B_3, 14);
     tc_fence_after();
 
     // ---- S7: dE -> RO rows 0..63 (16 tokens per column group);
@@ -494,14 +551,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ro0 = smem_u32(sm + R_RO), tt0 = smem_u32(sm + R_TT);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + T_DER, desc_mnmajor_sw128(ro0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(tt0 + ks * 2048, 8192), ID_MM64, ks > 0);
-      umma_commit(bar4);
+      umma_commit(bars + B_4);
+      mark(B_4);
     }
     if (tid < 64) s_dw[tid] = 0.f;
-    wait(bar4, par, 15);
+    wait(B_4, 15);
     tc_fence_after();
 
     // ---- S8: dR -> RO rows 0..63
@@ -525,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t w0 = smem_u32(sm + R_W), dsb0 = smem_u32(sm + R_DSB);
       const uint32_t kh0 = smem_u32(sm + R_KH), mp0 = smem_u32(sm + R_MP);
       const uint32_t x0 = smem_u32(sm + R_X), sb0 = smem_u32(sm + R_SB);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
         const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
@@ -538,32 +596,31 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_G, desc_mnmajor_sw128(sb0 + ks * 2048, 16384),
                   desc_kmajor_sw128(ro0 + kx), ID_MK128, ks > 0);
       }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
         umma_bf16(tmem + T_RE, desc_mnmajor_sw128(ro0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(mp0 + ks * 2048, 16384), ID_MM64, 1);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
         umma_bf16(tmem + T_DS, desc_mnmajor_sw128(ro0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(x0 + ks * 2048, 16384), ID_MM128, 1);
-      umma_commit(bar5);
+      }
+      umma_commit(bars + B_5);
+      mark(B_5);
     }
-    wait(bar5, par, 16);
+    wait(B_5, 16);
     tc_fence_after();
 
-    // ---- S10: reload raw g, b_x into SB; G2 (masked, bf16; 32 columns per
-    //      group); dv, dw (16 tokens per group)
+    // ---- S10: the epilogue's raw g, b_x -> RO, block ib - 1's state
+    //      operand -> SB; G2 (masked, bf16; 32 columns per group); dv, dw
+    //      (16 tokens per group)
     if (tid == 0 && !*s_abort) {
-      mbar_expect_tx(bar_gb, 2 * 16384);
-      tma_load_3d(sm + R_SB, &tm_g, bar_gb, 0, h, tok);
-      tma_load_3d(sm + R_SB + 8192, &tm_g, bar_gb, 64, h, tok);
-      tma_load_3d(sm + R_SB + 16384, &tm_bx, bar_gb, 0, h, tok);
-      tma_load_3d(sm + R_SB + 24576, &tm_bx, bar_gb, 64, h, tok);
+      issue_gb(ib);
+      if (ib > 0) issue_sb(ib - 1);
     }
     {
       const int rl = row & 63;
-      float vals[32];
+      float vals[32], dwv[16];
       tmem_ld32(tl + T_G2 + gp * 32, vals);
+      tmem_ld16(tl + T_RE + gp * 16, dwv);
 #pragma unroll
       for (int e = 0; e < 32; ++e)
         if (((gp & 1) * 32 + e) >= rl) vals[e] = 0.f;
@@ -571,19 +628,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8)
         st_chunk(blk + sw128_chunk(row, 0, (gp & 1) * 4 + c8, 128), vals + c8 * 8);
-    }
-    {
-      float vals[16], prod[16];
-      tmem_ld16(tl + T_RE + gp * 16, vals);
       __nv_bfloat16* dvrow = dv + ((size_t)tok + gp * 16) * H * kDV +
                              (size_t)h * kDV + row;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         const int t = gp * 16 + e;
-        dvrow[(size_t)e * H * kDV] = __float2bfloat16_rn(s_w[t] * vals[e]);
-        prod[e] = vals[e] * ldbf(sm + R_W + sw128_off(t, row, 64));
+        dvrow[(size_t)e * H * kDV] = __float2bfloat16_rn(s_w[t] * dwv[e]);
+        dwv[e] *= ldbf(sm + R_W + sw128_off(t, row, 64));
       }
-      const float sdw = warp_reduce_scatter16(prod, lane);
+      const float sdw = warp_reduce_scatter16(dwv, lane);
       if (lane < 16) atomicAdd(&s_dw[gp * 16 + lane], sdw);
     }
     fence_async_smem();
@@ -603,29 +656,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t mp0 = smem_u32(sm + R_MP), pq0 = smem_u32(sm + R_PQ);
       const uint32_t x0 = smem_u32(sm + R_X), dsb0 = smem_u32(sm + R_DSB);
       const uint32_t et0 = smem_u32(sm + R_ET), w0 = smem_u32(sm + R_W);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t a0 = (ks < 4 ? kp0 : kh0) + (ks & 3) * 2048;
         const uint32_t g2 = (ks < 4 ? mp0 : pq0) + (ks & 3) * 32;
         umma_bf16(tmem + T_G, desc_mnmajor_sw128(a0, 8192),
                   desc_kmajor_sw128(g2), ks < 4 ? ID_MK128_NA : ID_MK128, 1);
       }
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks)
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
         umma_bf16(tmem + T_RE, desc_mnmajor_sw128(x0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(mp0 + ks * 2048, 16384), ID_MM128, ks > 0);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
         umma_bf16(tmem + T_RE, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(et0 + ks * 2048, 16384), ID_MM64, 1);
         umma_bf16(tmem + T_RE + 64, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
                   desc_kmajor_sw128(w0 + (ks >> 2) * 8192 + (ks & 3) * 32),
                   ID_MK64, 1);
       }
-      umma_commit(bar7);
+      umma_commit(bars + B_7);
+      mark(B_7);
     }
-    wait(bar7, par, 17);
-    wait(bar_gb, par, 18);
+    wait(B_7, 17);
+    // block ib - 1's v, g, b_x, E^T, T into the buffers S11 released
+    if (tid == 0 && ib > 0 && !*s_abort) issue_pre(ib - 1);
+    wait(B_GB, 18);
     tc_fence_after();
 
     // ---- S12: per key channel j = row and token quarter gp: dq, dk, db_x,
@@ -642,7 +696,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         float gsum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) gsum += ldbf(sm + R_SB + sw128_off(tb + e, jj, 64));
+        for (int e = 0; e < 16; ++e) gsum += ldbf(sm + R_RO + sw128_off(tb + e, jj, 64));
         s_gq[gp * 128 + jj] = gsum;
       }
       __syncthreads();
@@ -656,25 +710,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       float qfirst = 0.f;
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
-        float d7k[8], d7q[8], d8p[8], d8h[8];
+        float dd[32];  // dK~ | dQ~ | -dkap^ | dK^ of 8 tokens
         const int tsub = tb + 8 * sub;
-        tmem_ld8(tl + T_G + tsub, d7k);
-        tmem_ld8(tl + T_G + 64 + tsub, d7q);
-        tmem_ld8(tl + T_RE + tsub, d8p);
-        tmem_ld8(tl + T_RE + 64 + tsub, d8h);
+        tmem_ld8x4(tl + T_G + tsub, tl + T_G + 64 + tsub, tl + T_RE + tsub,
+                   tl + T_RE + 64 + tsub, dd);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int tl_ = 8 * sub + e;
           const int t = tb + tl_;
           const uint32_t o64 = sw128_off(t, jj, 64);
-          G += ldbf(sm + R_SB + o64);
+          G += ldbf(sm + R_RO + o64);
           const float gam = __expf(G), igam = __fdividef(1.0f, gam);
-          const float bb = sigm(ldbf(sm + R_SB + 16384 + o64) + pj);
+          const float bb = sigm(ldbf(sm + R_RO + 16384 + o64) + pj);
           const float kt = ldbf(sm + R_X + sw128_off(t, jj, 128));
           const float qt = ldbf(sm + R_X + sw128_off(64 + t, jj, 128));
           const float kh = ldbf(sm + R_KH + o64);
           const float kp = ldbf(sm + R_KP + o64);
-          const float dKt = d7k[e], dQt = d7q[e], dKp = -d8p[e], dKh = d8h[e];
+          const float dKt = dd[e], dQt = dd[8 + e], dKp = -dd[16 + e], dKh = dd[24 + e];
           const size_t x = x0 + (size_t)t * tstride;
           dq[x] = __float2bfloat16_rn(dQt * gprev);
           dk[x] = __float2bfloat16_rn(dKt * gam + dKh * igam + dKp * bb * igam);
@@ -757,8 +809,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
 
-  // ---- dS0, dm0
-  if (!*s_abort) {
+  // ---- dS0, dm0; an aborted CTA first lets its copies and MMAs land
+  if (*s_abort) {
+    if (tid == 0)
+      for (int i = 0; i < kNumBars; ++i)
+        if ((pend >> i) & 1u) drain_bar(bars + i, (npar >> i) & 1u);
+  } else {
     const int c0 = gp * 32;
     if (a.dS0) {
       float* dst = a.dS0 + (size_t)pair * SZ + (size_t)row * kDK + c0;

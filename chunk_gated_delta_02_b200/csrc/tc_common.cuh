@@ -168,19 +168,30 @@ constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
 // and the wait site in the workspace header, raise the CTA abort flag and
 // return (the caller keeps its barrier sequence; the block loop exits at
 // its next check of the flag).
-__device__ __forceinline__ void wait_bar(uint64_t* bar, uint32_t parity,
+// Returns whether the phase completed.
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
                                          uint32_t where,
                                          volatile uint32_t* abort_flag,
                                          WsHeader* hdr) {
   const long long t0 = clock64();
   while (!*abort_flag) {
-    if (ptx::mbar_try_wait(bar, parity)) return;
+    if (ptx::mbar_try_wait(bar, parity)) return true;
     if (clock64() - t0 > kSpinCycles) {
       atomicExch(&hdr->status, (uint32_t)CARVE_ERR_TIMEOUT);
       hdr->where = where;
       *abort_flag = 1;
     }
   }
+  return false;
+}
+
+// Bounded wait that ignores the abort flag: before a CTA that aborted
+// exits, its copies and MMAs still in flight are given up to ~1 s each to
+// land (their shared and tensor memory must outlive them).
+__device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!ptx::mbar_try_wait(bar, parity))
+    if (clock64() - t0 > kSpinCycles) return;
 }
 
 }  // namespace tc
