@@ -257,19 +257,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     udn[i] = pack2(d0, d1);
   }
 
-  // dS <- dS_T (or 0); dm <- dm_T (or 0)
+  // dS <- dS_T (or 0); dm <- dm_T (or 0).  dlog gamma_j = sum_v dS S_new
+  // of the next block visited: this thread's share (column 32 gp + lane,
+  // rows of its quadrant) rides in `dlg_part` until that block's S4; for the
+  // last block S_new is the fp32 final state, later ones take the bf16 state
+  // record of the block after them.
+  float dlg_part = 0.f;
   {
     const int c0 = gp * 32;
     const float* src = a.dS_T ? a.dS_T + (size_t)pair * SZ + (size_t)row * kDK + c0
                               : nullptr;
-    float vals[32];
+    const float* sfin = a.ck_S + ((size_t)pair * (NB + 1) + NB) * SZ +
+                        (size_t)row * kDK + c0;
+    float vals[32], prod[32];
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {
       const float4 x = src ? *reinterpret_cast<const float4*>(src + i)
                            : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 y = *reinterpret_cast<const float4*>(sfin + i);
       vals[i] = x.x; vals[i + 1] = x.y; vals[i + 2] = x.z; vals[i + 3] = x.w;
+      prod[i] = x.x * y.x; prod[i + 1] = x.y * y.y;
+      prod[i + 2] = x.z * y.z; prod[i + 3] = x.w * y.w;
     }
     tmem_st32(tl + T_DS + c0, vals);
+    dlg_part = warp_reduce_scatter32(prod, lane);
     tmem_st_wait();
   }
   if (tid < 128) s_dmn[tid] = a.dm_T ? a.dm_T[(size_t)pair * kDV + tid] : 0.f;
@@ -338,6 +349,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   float dp_acc = 0.f;   // dp_j share (channel row, this warp's token quarter)
+  float p_next = tid < 128 ? a.gin[((size_t)pair * NC + NC - 1) * GR + tid] : 0.f;
   for (int ib = NB - 1; ib >= 0; --ib) {
     const int t0 = ib * kBlk;
     const int c = ib / bpc;
@@ -346,14 +358,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tok = b * T + t0;
     float* rec = args.gate_rec + ((size_t)pair * NC + c) * GR;
 
-    // ---- S0: gate of chunk c, p = U_up U_down m_c (forward record)
+    // ---- S0: gate of chunk c, p = U_up U_down m_c (forward record,
+    //      fetched during the previous block)
     if (chunk_last) {
-      if (tid < 128) s_p[tid] = a.gin[((size_t)pair * NC + c) * GR + tid];
+      if (tid < 128) s_p[tid] = p_next;
       dp_acc = 0.f;
     }
 
     // ---- S1: inputs.  k, q, d_o now; the rest was requested during the
-    //      previous block.  Block ib - 1's tiles, record and end state -> L2.
+    //      previous block.  Block ib - 1's tiles and record -> L2.
     if (tid == 0) {
       issue_top(ib);
       if (ib > 0) {
@@ -368,12 +381,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_prefetch_3d(&tm_bx, x0, h, tn);
         }
         bulk_prefetch_l2(rec0 + (size_t)(ib - 1) * kTcRecBytes, (uint32_t)kTcRecBytes);
-        const float* nxt = a.ck_S + ((size_t)pair * (NB + 1) + ib) * SZ;
-#pragma unroll 1
-        for (int q4 = 0; q4 < 4; ++q4) bulk_prefetch_l2(nxt + q4 * 4096, 16384);
       }
     }
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
+    if (chunk_first && ib > 0 && tid < 128)  // the next block starts chunk c - 1
+      p_next = a.gin[((size_t)pair * NC + c - 1) * GR + tid];
     // w_t of the token row this thread scales in W = w V
     const float wrow = __bfloat162float(w_in[((size_t)tok + (tid >> 3)) * H + h]);
     wait(B_SB, 10);
@@ -426,14 +438,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-    // the block-end state S_new (dlog gamma), loaded ahead of S4
-    float4 snv[8];
-    {
-      const float* sn = a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
-                        (size_t)row * kDK + gp * 32;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) snv[e] = *reinterpret_cast<const float4*>(sn + 4 * e);
-    }
     fence_async_smem();
     __syncthreads();
     if (*s_abort) break;
@@ -457,19 +461,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- S4: dS~ = dS Diag(gamma) (TMEM, and its bf16 operand over the
-    //      consumed raw g, b_x) with dlog gamma_j = sum_v dS S_new; then the
-    //      strictly lower [M; P_k] and P_kap operands
+    //      consumed raw g, b_x), dlog gamma; then the strictly lower
+    //      [M; P_k] and P_kap operands
     {
       const int c0 = gp * 32;
-      float vals[32], prod[32];
+      float vals[32];
       tmem_ld32(tl + T_DS + c0, vals);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        prod[4 * e] = vals[4 * e] * snv[e].x;
-        prod[4 * e + 1] = vals[4 * e + 1] * snv[e].y;
-        prod[4 * e + 2] = vals[4 * e + 2] * snv[e].z;
-        prod[4 * e + 3] = vals[4 * e + 3] * snv[e].w;
-      }
 #pragma unroll
       for (int e = 0; e < 32; e += 4) {
         const float4 gm = *reinterpret_cast<const float4*>(s_gam + c0 + e);
@@ -480,7 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c8 = 0; c8 < 4; ++c8)
         st_chunk(sm + R_DSB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
                  vals + c8 * 8);
-      atomicAdd(&s_x[c0 + lane], warp_reduce_scatter32(prod, lane));
+      atomicAdd(&s_x[c0 + lane], dlg_part);
     }
     wait(B_1, 13);
     tc_fence_after();
@@ -609,12 +606,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(B_5, 16);
     tc_fence_after();
 
-    // ---- S10: the epilogue's raw g, b_x -> RO, block ib - 1's state
-    //      operand -> SB; G2 (masked, bf16; 32 columns per group); dv, dw
-    //      (16 tokens per group)
-    if (tid == 0 && !*s_abort) {
-      issue_gb(ib);
-      if (ib > 0) issue_sb(ib - 1);
+    // ---- S10: the epilogue's raw g, b_x -> RO; dlog gamma share of block
+    //      ib - 1 (its S_new is this block's state record, still in SB);
+    //      G2 (masked, bf16; 32 columns per group); dv, dw (16 tokens per group)
+    if (tid == 0 && !*s_abort) issue_gb(ib);
+    if (ib > 0) {
+      float vals[32], sv[32];
+      tmem_ld32(tl + T_DS + gp * 32, vals);
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        ld_chunk(sm + R_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
+                 sv + c8 * 8);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) vals[e] *= sv[e];
+      dlg_part = warp_reduce_scatter32(vals, lane);
     }
     {
       const int rl = row & 63;
@@ -649,8 +654,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           __float2bfloat16_rn(wt != 0.f ? s_dw[tid] / wt : 0.f);
     }
 
-    // ---- S11: D7^T += [-kap^; K^]^T G2^T ; D8^T = X^T G2 + dS~^T [E; W]^T
+    // ---- S11: D7^T += [-kap^; K^]^T G2^T ; D8^T = X^T G2 + dS~^T [E; W]^T;
+    //      block ib - 1's state operand -> SB (read above)
     if (tid == 0) {
+      if (ib > 0 && !*s_abort) issue_sb(ib - 1);
       tc_fence_after();
       const uint32_t kp0 = smem_u32(sm + R_KP), kh0 = smem_u32(sm + R_KH);
       const uint32_t mp0 = smem_u32(sm + R_MP), pq0 = smem_u32(sm + R_PQ);
@@ -722,10 +729,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           G += ldbf(sm + R_RO + o64);
           const float gam = __expf(G), igam = __fdividef(1.0f, gam);
           const float bb = sigm(ldbf(sm + R_RO + 16384 + o64) + pj);
-          const float kt = ldbf(sm + R_X + sw128_off(t, jj, 128));
           const float qt = ldbf(sm + R_X + sw128_off(64 + t, jj, 128));
           const float kh = ldbf(sm + R_KH + o64);
-          const float kp = ldbf(sm + R_KP + o64);
+          const float kt = kh * gam * gam;  // K~ = K^ Gamma^2
+          const float kp = bb * kh;         // kap^ = b K^
           const float dKt = dd[e], dQt = dd[8 + e], dKp = -dd[16 + e], dKh = dd[24 + e];
           const size_t x = x0 + (size_t)t * tstride;
           dq[x] = __float2bfloat16_rn(dQt * gprev);
@@ -838,38 +845,63 @@ __global__ void __launch_bounds__(kThreads, 1)
 // dU_up[h][j][r] = sum_{b,c} dp[b,h,c][j] h[b,h,c][r]
 // dU_down[h][r][v] = sum_{b,c} dh[b,h,c][r] m[b,h,c][v]   (fixed order)
 // dp, dh come from the backward's gate records, h = U_down m_c from the
-// forward's gate inputs, m_c from its checkpoints.
-__global__ void du_from_gate_records(const float* __restrict__ rec,
-                                     const float* __restrict__ gin,
-                                     const float* __restrict__ ck_m, int B,
-                                     int H, int NC, int R, int DK, int DV,
-                                     float* du_down, float* du_up) {
-  const int GR = DK + R;
-  const size_t per = (size_t)DK * R + (size_t)R * DV;
-  const size_t n = (size_t)H * per;
-  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n;
-       idx += (size_t)gridDim.x * blockDim.x) {
-    const int h = (int)(idx / per);
-    const size_t e = idx - (size_t)h * per;
-    float acc = 0.f;
-    if (e < (size_t)DK * R) {
-      const int jj = (int)(e / R), r = (int)(e % R);
-      for (int bb = 0; bb < B; ++bb)
-        for (int c = 0; c < NC; ++c) {
-          const size_t o = ((size_t)(bb * H + h) * NC + c) * GR;
-          acc += rec[o + jj] * gin[o + DK + r];
+// forward's gate inputs, m_c from its checkpoints.  CTA (h, part) forms the
+// channel rows 32 part .. + 31 of dU_up and value columns 32 part .. + 31 of
+// dU_down, walking the (b, c) records in order through 64-record slabs in
+// shared memory; R <= 32.
+constexpr int kDuThreads = 256;
+constexpr int kDuSlab = 64;
+__global__ void __launch_bounds__(kDuThreads)
+    du_from_gate_records(const float* __restrict__ rec,
+                         const float* __restrict__ gin,
+                         const float* __restrict__ ck_m, int B, int H, int NC,
+                         int R, float* du_down, float* du_up) {
+  __shared__ __align__(16) float s_dp[kDuSlab][32];
+  __shared__ __align__(16) float s_hv[kDuSlab][32];
+  __shared__ __align__(16) float s_dh[kDuSlab][32];
+  __shared__ __align__(16) float s_m[kDuSlab][32];
+  const int h = blockIdx.x, part = blockIdx.y, t = threadIdx.x;
+  const int GR = kDK + R;
+  const int N = B * NC;
+  const int hi = t >> 3, lo4 = 4 * (t & 7);
+  float up[4] = {0.f, 0.f, 0.f, 0.f}, dn[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int n0 = 0; n0 < N; n0 += kDuSlab) {
+    for (int idx = t; idx < kDuSlab * 32; idx += kDuThreads) {
+      const int n = n0 + (idx >> 5), k = idx & 31;
+      float dp = 0.f, hv = 0.f, dh = 0.f, mv = 0.f;
+      if (n < N) {
+        const int bb = n / NC, c = n - bb * NC;
+        const size_t o = ((size_t)bb * H + h) * NC + c;
+        dp = rec[o * GR + 32 * part + k];
+        mv = ck_m[o * kDV + 32 * part + k];
+        if (k < R) {
+          hv = gin[o * GR + kDK + k];
+          dh = rec[o * GR + kDK + k];
         }
-      du_up[(size_t)h * DK * R + e] = acc;
-    } else {
-      const size_t e2 = e - (size_t)DK * R;
-      const int r = (int)(e2 / DV), v = (int)(e2 % DV);
-      for (int bb = 0; bb < B; ++bb)
-        for (int c = 0; c < NC; ++c) {
-          const size_t o = ((size_t)(bb * H + h) * NC + c);
-          acc += rec[o * GR + DK + r] * ck_m[o * DV + v];
-        }
-      du_down[(size_t)h * R * DV + e2] = acc;
+      }
+      s_dp[idx >> 5][k] = dp;
+      s_hv[idx >> 5][k] = hv;
+      s_dh[idx >> 5][k] = dh;
+      s_m[idx >> 5][k] = mv;
     }
+    __syncthreads();
+    const int ns = min(kDuSlab, N - n0);
+    for (int n = 0; n < ns; ++n) {
+      const float a = s_dp[n][hi], d = s_dh[n][hi];
+      const float4 hv = *reinterpret_cast<const float4*>(&s_hv[n][lo4]);
+      const float4 mv = *reinterpret_cast<const float4*>(&s_m[n][lo4]);
+      up[0] = fmaf(a, hv.x, up[0]); up[1] = fmaf(a, hv.y, up[1]);
+      up[2] = fmaf(a, hv.z, up[2]); up[3] = fmaf(a, hv.w, up[3]);
+      dn[0] = fmaf(d, mv.x, dn[0]); dn[1] = fmaf(d, mv.y, dn[1]);
+      dn[2] = fmaf(d, mv.z, dn[2]); dn[3] = fmaf(d, mv.w, dn[3]);
+    }
+    __syncthreads();
+  }
+  const int j = 32 * part + hi;  // dU_up row; dU_down row is r = hi
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    if (lo4 + k < R) du_up[((size_t)h * kDK + j) * R + lo4 + k] = up[k];
+    if (hi < R) du_down[((size_t)h * R + hi) * kDV + 32 * part + lo4 + k] = dn[k];
   }
 }
 
@@ -921,14 +953,9 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
                                                          mb, mdo);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const size_t n = (size_t)a.H * ((size_t)a.DK * a.R + (size_t)a.R * a.DV);
-  if (n > 0) {
-    int blocks = (int)((n + 255) / 256);
-    if (blocks > 4 * 148) blocks = 4 * 148;
-    du_from_gate_records<<<blocks, 256, 0, st>>>(a.scratch, a.gin, a.ck_m, a.B,
-                                                 a.H, a.NC, a.R, a.DK, a.DV,
-                                                 a.du_down, a.du_up);
-  }
+  if (a.R > 0)
+    du_from_gate_records<<<dim3(a.H, kDK / 32), kDuThreads, 0, st>>>(
+        a.scratch, a.gin, a.ck_m, a.B, a.H, a.NC, a.R, a.du_down, a.du_up);
   return cudaGetLastError();
 }
 
