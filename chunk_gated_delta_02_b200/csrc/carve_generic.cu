@@ -257,6 +257,14 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
   const int C = a.C, DK = a.DK, DV = a.DV, R = a.R, H = a.H, T = a.T;
   const int pair = blockIdx.x, b = pair / H, h = pair - b * H;
   const int tid = threadIdx.x, nt = blockDim.x;
+  // the fp32 block checkpoints exist only after this family's forward
+  if (a.hdr->magic != kWsMagic) {
+    if (tid == 0) {
+      atomicExch(&a.hdr->status, (uint32_t)CARVE_ERR_WORKSPACE);
+      a.hdr->where = 97;
+    }
+    return;
+  }
   const TIn* q = (const TIn*)a.q;
   const TIn* k = (const TIn*)a.k;
   const TIn* v = (const TIn*)a.v;

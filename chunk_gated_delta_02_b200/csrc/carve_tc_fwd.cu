@@ -1,7 +1,7 @@
 // carve_tc_fwd.cu -- tensor-core (tcgen05 / TMEM / TMA) forward of the CARVE
 // recurrent core for bf16 inputs, dk = dv = 128, chunks of 64 or 128 tokens.
 //
-// One CTA (8 warps) walks one (sequence, head) pair through its blocks of
+// One CTA (16 warps) walks one (sequence, head) pair through its blocks of
 // C = 64 tokens.  The fp32 state S (dv x dk) lives in tensor memory for the
 // whole walk; a bf16 copy in shared memory is the MMA operand.  Per block,
 // with the notation of the chunk form (CARVE summaries, gist.science,
@@ -14,7 +14,7 @@
 //   MMA 1       G = [K~; Q~] [kap^ | K^]^T   ->  [A | M ; P_kap | P_k]
 //               D1 = S [K~; Q~]^T             ->  [(K~ S^T)^T | (Q~ S^T)^T]
 //   MMA 2       D1 += W^T [M; P_k]^T          ->  [R^T | (Q~ S^T + P_k W)^T]
-//   solve       T = (I + A)^{-1} by 16 x 16 blocks (all threads, fp32)
+//   solve       T = (I + A)^{-1} by 16 x 16 blocks (warps 0-3, tf32)
 //   MMA 3a      E^T = R^T T^T                 (E = T R, the WY pseudo-values)
 //   MMA 3b      D1[O] -= E^T P_kap^T          ->  O^T = (Q~ S^T + P_k W - P_kap E)^T
 //   MMA 4       S += W^T K^ - E^T kap^ ;  S <- S Diag(gamma)
@@ -26,7 +26,9 @@
 // is exactly the UMMA canonical layout, so the element-wise transform writes
 // operands at the offsets it reads them from.  The next block's v, g, b_x
 // tiles are requested right after the transform, its k, q tiles as soon as
-// MMA 1 has released their buffer.
+// MMA 1 has released their buffer.  In training mode the block's bf16 S
+// operand, E^T and T go to the workspace by bulk copies (the backward's
+// records); of the fp32 states only the final one is kept.
 #include <cudaTypedefs.h>
 
 #include "carve_internal.cuh"
@@ -43,7 +45,7 @@ using tc::pack2;
 using tc::st_chunk;
 using tc::unit_lower_inverse64;
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kBlk = 64;   // tokens per block
 constexpr int kDK = 128;   // key width
 constexpr int kDV = 128;   // value rows per CTA
@@ -67,7 +69,7 @@ constexpr uint32_t SM_GAM = 0;         // gamma_j            128 f32
 constexpr uint32_t SM_P = 512;         // (U_b m)_j          128 f32
 constexpr uint32_t SM_M = 1280;        // m_v                128 f32
 constexpr uint32_t SM_H = 1792;        // U_down m            64 f32
-constexpr uint32_t SM_BAR = 2560;      // 6 mbarriers
+constexpr uint32_t SM_BAR = 2560;      // kNumBars mbarriers
 constexpr uint32_t SM_TMEM = 2624;     // TMEM base address
 constexpr uint32_t SM_ABORT = 2628;    // abort flag
 constexpr uint32_t kSmallBytes = 2688;
@@ -75,6 +77,16 @@ constexpr uint32_t OFF_UU = 215808;    // U_up^T bf16 [kRMax][128]      8 KB
 constexpr uint32_t kSmemBytes = OFF_UU + 8192 + 1024;
 static_assert(OFF_SMALL + kSmallBytes <= OFF_UU, "shared memory map overlap");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
+
+// mbarriers (index into the small region's array)
+constexpr int B_VGB = 0;   // TMA v, g, b_x
+constexpr int B_KQ = 1;    // TMA k, q
+constexpr int B_M1 = 2;    // MMA 1 (Grams, S X^T)
+constexpr int B_M2 = 3;    // MMA 2 (W^T [M;P_k]^T)
+constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
+constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
+constexpr int B_D1 = 6;    // MMA 1, second half (S X^T)
+constexpr int kNumBars = 7;
 
 // TMEM columns (fp32, lanes = rows)
 constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
@@ -90,8 +102,10 @@ constexpr uint32_t ID_AMN_BMN = idesc_bf16(128, 128, true, true);
 constexpr uint32_t ID_N64_NA = idesc_bf16_neg(128, 64, false, false, true, false);
 constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false);
 
-constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
 
+// 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
+// rows 32 qd .. 32 qd + 31) and column group gp = w / 4.  Warps 0-3 also
+// run the triangular solve while warps 4-11 prepare [M; P_k] and R^T.
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -107,19 +121,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_h = reinterpret_cast<float*>(sm + OFF_SMALL + SM_H);
   float* s_af = reinterpret_cast<float*>(sm + OFF_AF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_SMALL + SM_BAR);
-  uint64_t* bar_vgb = bars + 0;  // TMA v, g, b_x
-  uint64_t* bar_kq = bars + 1;   // TMA k, q
-  uint64_t* bar_m1 = bars + 2;   // MMA 1 (Grams, S X^T)
-  uint64_t* bar_m2 = bars + 3;   // MMA 2 (W^T [M;P_k]^T)
-  uint64_t* bar_m3 = bars + 4;   // MMA 3 (R^T Y^T)
-  uint64_t* bar_m4 = bars + 5;   // MMA 4 (state update)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SMALL + SM_TMEM);
   volatile uint32_t* s_abort =
       reinterpret_cast<volatile uint32_t*>(sm + OFF_SMALL + SM_ABORT);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int half = warp >> 2;                 // 0: warps 0-3, 1: warps 4-7
-  const int row = (warp & 3) * 32 + lane;     // TMEM lane owned by the thread
+  const int qd = warp & 3, gp = warp >> 2;
+  const int row = qd * 32 + lane;             // TMEM lane owned by the thread
   const int pair = blockIdx.x, b = pair / a.H, h = pair - b * a.H;
   const int T = a.T, H = a.H, R = a.R, NB = a.NB;
   const int bpc = a.L / kBlk;
@@ -131,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     if (a.tc_rec && blockIdx.x == 0) a.hdr->magic = kWsMagicTc;
-    for (int i = 0; i < 6; ++i) mbar_init(bars + i, 1);
+    for (int i = 0; i < kNumBars; ++i) mbar_init(bars + i, 1);
     *s_abort = 0;
     mbar_init_fence();
     prefetch_tmap(&tm_q);
@@ -148,34 +156,32 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
-  const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);  // lane base
+  const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);  // lane base
 
-  // Bounded wait on an mbarrier phase; on expiry record CARVE_ERR_TIMEOUT,
-  // raise the CTA-wide abort flag and return (callers keep the barrier
-  // sequence, the block loop exits at its next check).
-  auto wait = [&](uint64_t* bar, uint32_t parity, uint32_t where) {
-    const long long t0 = clock64();
-    while (!*s_abort) {
-      if (mbar_try_wait(bar, parity)) return;
-      if (clock64() - t0 > kSpinCycles) {
-        atomicExch(&a.hdr->status, (uint32_t)CARVE_ERR_TIMEOUT);
-        a.hdr->where = where;
-        *s_abort = 1;
-      }
+  // Every barrier has at most one phase in flight.  `npar` holds the parity
+  // each thread waits for next; thread 0 also tracks in `pend` the phases it
+  // started (copies issued, MMAs committed) so that an aborting CTA drains
+  // them before it exits.
+  uint32_t npar = 0, pend = 0;
+  auto wait = [&](int i, uint32_t where) {
+    if (tc::wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr)) {
+      npar ^= 1u << i;
+      pend &= ~(1u << i);
     }
   };
+  auto mark = [&](int i) { pend |= 1u << i; };
 
-  // U_b factors: thread (r = tid/8, part = tid%8) holds U_down[h][r][16 part
-  // .. 16 part + 15] in registers; U_up[h] is kept transposed in shared
-  // memory (s_uu[r][j], zero for r >= R).
-  float ud_r[16];
+  // U_b factors: thread (r = tid / 16, part = tid % 16) holds U_down[h][r]
+  // [8 part .. 8 part + 7] in registers; U_up[h] is kept transposed in
+  // shared memory (s_uu[r][j], zero for r >= R).
+  float ud_r[8];
   __nv_bfloat16* s_uu = reinterpret_cast<__nv_bfloat16*>(sm + OFF_UU);
   {
-    const int r = tid >> 3, part = tid & 7;
+    const int r = tid >> 4, part = tid & 15;
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < 8; ++i)
       ud_r[i] = (r < R) ? __bfloat162float(
-                              ud[((size_t)h * R + r) * kDV + 16 * part + i])
+                              ud[((size_t)h * R + r) * kDV + 8 * part + i])
                         : 0.f;
     for (int e = tid; e < kRMax * kDK; e += kThreads) {
       const int r2 = e / kDK, jj = e - r2 * kDK;
@@ -188,13 +194,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // and h_c = U_down m_c for the backward
   auto gate = [&](int c) {
     {
-      const int r = tid >> 3, part = tid & 7;
+      const int r = tid >> 4, part = tid & 15;
       float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) acc = fmaf(ud_r[i], s_m[16 * part + i], acc);
+      for (int i = 0; i < 8; ++i) acc = fmaf(ud_r[i], s_m[8 * part + i], acc);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
       if (part == 0) s_h[r] = acc;
     }
     __syncthreads();
@@ -204,67 +211,58 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int r = 0; r < kRMax; ++r)
         acc = fmaf(__bfloat162float(s_uu[r * kDK + tid]), s_h[r], acc);
       s_p[tid] = acc;
+      if (a.gin) a.gin[((size_t)pair * a.NC + c) * (kDK + R) + tid] = acc;
+    } else if (a.gin && tid - 128 < R) {
+      a.gin[((size_t)pair * a.NC + c) * (kDK + R) + kDK + tid - 128] = s_h[tid - 128];
     }
     __syncthreads();
-    if (a.gin) {
-      float* gp = a.gin + ((size_t)pair * a.NC + c) * (kDK + R);
-      if (tid < 128)
-        gp[tid] = s_p[tid];
-      else if (tid - 128 < R)
-        gp[kDK + tid - 128] = s_h[tid - 128];
-    }
   };
 
   auto issue_vgb = [&](int ib) {
     const int tok = b * T + ib * kBlk;
-    mbar_expect_tx(bar_vgb, 3 * 16384);
-    tma_load_3d(sm + OFF_RV, &tm_v, bar_vgb, 0, h, tok);
-    tma_load_3d(sm + OFF_RV + 8192, &tm_v, bar_vgb, 64, h, tok);
-    tma_load_3d(sm + OFF_RG, &tm_g, bar_vgb, 0, h, tok);
-    tma_load_3d(sm + OFF_RG + 8192, &tm_g, bar_vgb, 64, h, tok);
-    tma_load_3d(sm + OFF_RB, &tm_bx, bar_vgb, 0, h, tok);
-    tma_load_3d(sm + OFF_RB + 8192, &tm_bx, bar_vgb, 64, h, tok);
+    mbar_expect_tx(bars + B_VGB, 3 * 16384);
+    tma_load_3d(sm + OFF_RV, &tm_v, bars + B_VGB, 0, h, tok);
+    tma_load_3d(sm + OFF_RV + 8192, &tm_v, bars + B_VGB, 64, h, tok);
+    tma_load_3d(sm + OFF_RG, &tm_g, bars + B_VGB, 0, h, tok);
+    tma_load_3d(sm + OFF_RG + 8192, &tm_g, bars + B_VGB, 64, h, tok);
+    tma_load_3d(sm + OFF_RB, &tm_bx, bars + B_VGB, 0, h, tok);
+    tma_load_3d(sm + OFF_RB + 8192, &tm_bx, bars + B_VGB, 64, h, tok);
+    mark(B_VGB);
   };
   auto issue_kq = [&](int ib) {
     const int tok = b * T + ib * kBlk;
-    mbar_expect_tx(bar_kq, 2 * 16384);
-    tma_load_3d(sm + OFF_X, &tm_k, bar_kq, 0, h, tok);
-    tma_load_3d(sm + OFF_X + 16384, &tm_k, bar_kq, 64, h, tok);
-    tma_load_3d(sm + OFF_X + 8192, &tm_q, bar_kq, 0, h, tok);
-    tma_load_3d(sm + OFF_X + 16384 + 8192, &tm_q, bar_kq, 64, h, tok);
+    mbar_expect_tx(bars + B_KQ, 2 * 16384);
+    tma_load_3d(sm + OFF_X, &tm_k, bars + B_KQ, 0, h, tok);
+    tma_load_3d(sm + OFF_X + 16384, &tm_k, bars + B_KQ, 64, h, tok);
+    tma_load_3d(sm + OFF_X + 8192, &tm_q, bars + B_KQ, 0, h, tok);
+    tma_load_3d(sm + OFF_X + 16384 + 8192, &tm_q, bars + B_KQ, 64, h, tok);
+    mark(B_KQ);
   };
 
   // ---- initial state: S0 -> TMEM (fp32) and the bf16 operand copy
   {
-    const int c0 = half * 64;
+    const int c0 = gp * 32;
     const float* s0 = a.S0 ? a.S0 + (size_t)pair * SZ + (size_t)row * kDK + c0
                            : nullptr;
-    float* ck = a.ck_S ? a.ck_S + (size_t)pair * (NB + 1) * SZ +
-                             (size_t)row * kDK + c0
-                       : nullptr;
     float vals[32];
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-#pragma unroll
-      for (int i = 0; i < 32; i += 4) {
-        float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + part * 32 + i)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
-        vals[i] = x.x; vals[i + 1] = x.y; vals[i + 2] = x.z; vals[i + 3] = x.w;
-        if (ck) *reinterpret_cast<float4*>(ck + part * 32 + i) = x;
-      }
-      tmem_st32(tl + TM_S + c0 + part * 32, vals);
-#pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8)
-        st_chunk(sm + OFF_SB + sw128_chunk(row, half, part * 4 + c8, 128),
-                 vals + c8 * 8);
+    for (int i = 0; i < 32; i += 4) {
+      float4 x = s0 ? *reinterpret_cast<const float4*>(s0 + i)
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      vals[i] = x.x; vals[i + 1] = x.y; vals[i + 2] = x.z; vals[i + 3] = x.w;
     }
+    tmem_st32(tl + TM_S + c0, vals);
+#pragma unroll
+    for (int c8 = 0; c8 < 4; ++c8)
+      st_chunk(sm + OFF_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
+               vals + c8 * 8);
   }
   if (tid < 128) s_m[tid] = a.m0 ? a.m0[(size_t)pair * kDV + tid] : 0.f;
   tmem_st_wait();
   __syncthreads();
   gate(0);
   if (a.ck_m && tid < 128) a.ck_m[(size_t)pair * a.NC * kDV + tid] = s_m[tid];
-  if (tid == 0 && NB > 0) {
+  if (tid == 0) {
     issue_vgb(0);
     issue_kq(0);
   }
@@ -272,9 +270,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
 
-  float msum = 0.f;  // warps 4-7: this chunk's sum of o for value row `row`
+  float msum = 0.f;  // this thread's token quarter of the chunk's sum of o, row `row`
+  float* s_mq = s_af;  // [4][128] quarter sums of o at a chunk end (A buffer is free)
   for (int ib = 0; ib < NB; ++ib) {
-    const uint32_t par = (uint32_t)(ib & 1);
     const int t0 = ib * kBlk;
     const bool chunk_end = ((ib + 1) % bpc) == 0;
     uint8_t* rec = a.tc_rec ? a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes
@@ -287,43 +285,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_store(rec + kTcRecS, sm + OFF_SB, 32768);
       bulk_commit();
     }
-    if (tid == 0 && ib + 2 < NB) {
-      const int tn = b * T + (ib + 2) * kBlk;
-#pragma unroll
-      for (int x0 = 0; x0 < 128; x0 += 64) {
-        tma_prefetch_3d(&tm_k, x0, h, tn);
-        tma_prefetch_3d(&tm_q, x0, h, tn);
-        tma_prefetch_3d(&tm_v, x0, h, tn);
-        tma_prefetch_3d(&tm_g, x0, h, tn);
-        tma_prefetch_3d(&tm_bx, x0, h, tn);
-      }
-    }
-    // w_t of the two token rows this thread scales in W = w V
-    const float w_lo = __bfloat162float(w_in[((size_t)b * T + t0 + (tid >> 3)) * H + h]);
-    const float w_hi = __bfloat162float(w_in[((size_t)b * T + t0 + (tid >> 3) + 32) * H + h]);
-    wait(bar_vgb, par, 1);
-    wait(bar_kq, par, 2);
+    // w_t of the token row this thread scales in W = w V
+    const float wrow = __bfloat162float(w_in[((size_t)b * T + t0 + (tid >> 3)) * H + h]);
+    wait(B_VGB, 1);
+    wait(B_KQ, 2);
 
     // ---- 2. transform: decay scan, gated and decayed operands, W = w V
-    tc::transform_block<8>(sm + OFF_X, sm + OFF_KH, sm + OFF_KP, sm + OFF_RG,
-                        sm + OFF_RB, s_p, s_gam, s_af, 3);
+    tc::transform_block<16>(sm + OFF_X, sm + OFF_KH, sm + OFF_KP, sm + OFF_RG,
+                            sm + OFF_RB, s_p, s_gam, s_af, 3);
+    {
+      const int rr = tid >> 3, ch = tid & 7;  // token row, 16-byte chunk
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int c = tid + 256 * i;  // 16-byte chunk of the 64 x 128 v tile
-      const int rr = (c >> 3) & 63;
-      const uint32_t off = (uint32_t)((c >> 9) * 8192 + (rr >> 3) * 1024 +
-                                      (rr & 7) * 128 + (c & 7) * 16);
-      const uint4 x = *reinterpret_cast<const uint4*>(sm + OFF_RV + off);
-      const float wt = (i & 1) ? w_hi : w_lo;
-      const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
-      uint4 y;
-      uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
+      for (int kb = 0; kb < 2; ++kb) {
+        const uint32_t off = (uint32_t)(kb * 8192 + (rr >> 3) * 1024 +
+                                        (rr & 7) * 128 + ch * 16);
+        const uint4 x = *reinterpret_cast<const uint4*>(sm + OFF_RV + off);
+        const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
+        uint4 y;
+        uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(xv[e]);
-        yv[e] = pack2(f.x * wt, f.y * wt);
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(xv[e]);
+          yv[e] = pack2(f.x * wrow, f.y * wrow);
+        }
+        *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
       }
-      *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
     }
     fence_async_smem();
     if (tid == 0 && rec) bulk_wait_read_all();  // S record read: SB reusable
@@ -336,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t x0 = smem_u32(sm + OFF_X), kp0 = smem_u32(sm + OFF_KP);
       const uint32_t kh0 = smem_u32(sm + OFF_KH), sb0 = smem_u32(sm + OFF_SB);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
         const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
@@ -344,74 +330,102 @@ __global__ void __launch_bounds__(kThreads, 1)
                   desc_kmajor_sw128(kp0 + k64), ID_N64, ks > 0);
         umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
                   desc_kmajor_sw128(kh0 + k64), ID_N64, ks > 0);
+      }
+      umma_commit(bars + B_M1);
+      mark(B_M1);
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
         umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
                   desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
       }
-      umma_commit(bar_m1);
+      umma_commit(bars + B_D1);
+      mark(B_D1);
     }
-    wait(bar_m1, par, 3);
+    wait(B_M1, 3);
     tc_fence_after();
-    if (tid == 0 && ib + 1 < NB && !*s_abort) issue_kq(ib + 1);
 
-    const int gi = row;                        // Gram row of this thread
-    const int gr = gi < 64 ? gi : gi - 64;     // its token index in the block
-    float vals[32];
+    const int gr = row < 64 ? row : row - 64;  // token index of Gram row `row`
     // the bf16 S copy is dead until step 7: its buffer holds T (fp32),
     // the inversion's scratch and the bf16 P_kap operand meanwhile
     float* s_tf = reinterpret_cast<float*>(sm + OFF_SB);
     uint8_t* pq = sm + OFF_SB + 24576;
-    if (half == 1) {
-      // ---- 4a. [M; P_k] (strictly lower) -> bf16 operand; MMA 2
-#pragma unroll
+    if (gp == 0) {
+      // ---- 4a. [A; P_kap] (strictly lower): A -> fp32 for the inversion,
+      //          P_kap -> bf16 operand; T = (I + A)^{-1} (warps 0-3).  The
+      //          second half of MMA 1 still reads SB: P_kap and the solve's
+      //          scratch go there only once it retired.
+#pragma unroll 1
       for (int part = 0; part < 2; ++part) {
+        float vals[32];
+        tmem_ld32(tl + TM_GK + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (part * 32 + e >= gr) vals[e] = 0.f;
+        if (row < 64) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(s_af + fsw(row, part * 32 + e)) =
+                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+        } else {
+          if (part == 0) wait(B_D1, 10);
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8)
+            st_chunk(pq + sw128_chunk(gr, 0, part * 4 + c8, 64), vals + c8 * 8);
+        }
+      }
+      if (row < 64) wait(B_D1, 10);
+      bar_named(2, 128);
+      unit_lower_inverse64(s_af, s_tf, s_tf + 4096, 2);
+      wait(B_M2, 5);  // [M; P_k] consumed: T may take its place
+      if (row < 64) {
+#pragma unroll 1
+        for (int part = 0; part < 2; ++part) {
+          float vals[32];
+#pragma unroll
+          for (int e = 0; e < 32; e += 4) {
+            const float4 x = *reinterpret_cast<const float4*>(s_tf + fsw(row, part * 32 + e));
+            vals[e] = x.x; vals[e + 1] = x.y; vals[e + 2] = x.z; vals[e + 3] = x.w;
+          }
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8)
+            st_chunk(sm + OFF_MY + sw128_chunk(row, 0, part * 4 + c8, 64), vals + c8 * 8);
+        }
+      }
+    } else if (gp <= 2) {
+      // ---- 4b. [M; P_k] (strictly lower, 32 columns per group) -> bf16
+      //          operand; MMA 2; R^T -> bf16 operand (warps 4-11)
+      const int part = gp - 1;
+      {
+        float vals[32];
         tmem_ld32(tl + TM_GM + part * 32, vals);
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           if (part * 32 + e >= gr) vals[e] = 0.f;
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + OFF_MY + sw128_chunk(gi, 0, part * 4 + c8, 128),
+          st_chunk(sm + OFF_MY + sw128_chunk(row, 0, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
       fence_async_smem();
       tc_fence_before();
-      bar_named(1, 128);
+      bar_named(1, 256);
       if (tid == 128 && !*s_abort) {
+        wait(B_D1, 9);  // S X^T retired: X is free for the next block's k, q
+        if (ib + 1 < NB) issue_kq(ib + 1);
         tc_fence_after();
         const uint32_t w0 = smem_u32(sm + OFF_W), my0 = smem_u32(sm + OFF_MY);
-#pragma unroll
+#pragma unroll 1
         for (int ks = 0; ks < 4; ++ks)
           umma_bf16(tmem + TM_D1, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
                     desc_kmajor_sw128(my0 + ks * 32), ID_AMN, 1);
-        umma_commit(bar_m2);
+        umma_commit(bars + B_M2);
+        mark(B_M2);
       }
-    } else {
-      // ---- 4b. [A; P_kap] (strictly lower): A -> fp32 for the inversion,
-      //          P_kap -> bf16 operand
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + TM_GK + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (part * 32 + e >= gr) vals[e] = 0.f;
-        if (gi < 64) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(s_af + fsw(gi, part * 32 + e)) =
-                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
-        } else {
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8)
-            st_chunk(pq + sw128_chunk(gr, 0, part * 4 + c8, 64), vals + c8 * 8);
-        }
-      }
-    }
-    if (half == 1) {
-      // R^T -> bf16 operand, concurrently with the inversion
-      wait(bar_m2, par, 4);  // [M; P_k] consumed, R^T complete
+      wait(B_M2, 4);  // [M; P_k] consumed, R^T complete
       tc_fence_after();
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
+      {
+        float vals[32];
         tmem_ld32(tl + TM_D1 + part * 32, vals);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
@@ -419,23 +433,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                    vals + c8 * 8);
       }
     } else {
-      // ---- 4c. T = (I + A)^{-1}, blocked, warp-level tensor cores (warps 0-3)
-      bar_named(2, 128);
-      unit_lower_inverse64(s_af, s_tf, s_tf + 4096, 2);
-      wait(bar_m2, par, 5);  // [M; P_k] consumed: T may take its place
-    }
-    if (half == 0 && gi < 64) {
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-#pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(s_tf + fsw(gi, part * 32 + e));
-          vals[e] = x.x; vals[e + 1] = x.y; vals[e + 2] = x.z; vals[e + 3] = x.w;
+      // warps 12-15: block ib + 2's tiles -> L2 (their loads are issued
+      // during block ib + 1)
+      if (tid == 384 && ib + 2 < NB) {
+        const int tn = b * T + (ib + 2) * kBlk;
+#pragma unroll 1
+        for (int x0 = 0; x0 < 128; x0 += 64) {
+          tma_prefetch_3d(&tm_k, x0, h, tn);
+          tma_prefetch_3d(&tm_q, x0, h, tn);
+          tma_prefetch_3d(&tm_v, x0, h, tn);
+          tma_prefetch_3d(&tm_g, x0, h, tn);
+          tma_prefetch_3d(&tm_bx, x0, h, tn);
         }
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + OFF_MY + sw128_chunk(gi, 0, part * 4 + c8, 64), vals + c8 * 8);
       }
+      wait(B_M2, 6);  // keeps every thread's view of the barrier phases in step
     }
     fence_async_smem();
     tc_fence_before();
@@ -446,28 +457,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t re0 = smem_u32(sm + OFF_RE), my0 = smem_u32(sm + OFF_MY);
-#pragma unroll
+#pragma unroll 1
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + TM_D1, desc_kmajor_sw128(re0 + ks * 32),
                   desc_kmajor_sw128(my0 + ks * 32), ID_N64, ks > 0);
-      umma_commit(bar_m3);
+      umma_commit(bars + B_M3);
+      mark(B_M3);
       if (rec) {
         bulk_store(rec + kTcRecT, sm + OFF_MY, 8192);
         bulk_commit();
       }
     }
-    wait(bar_m3, par, 6);
+    wait(B_M3, 7);
     tc_fence_after();
-    if (half == 0) {
-      // E^T -> bf16 operand (negated by the MMAs that use it)
+    if (gp < 2) {
+      // E^T -> bf16 operand (negated by the MMAs that use it), 32 columns
+      // per group
+      float vals[32];
+      tmem_ld32(tl + TM_D1 + gp * 32, vals);
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + TM_D1 + part * 32, vals);
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
-                   vals + c8 * 8);
-      }
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_chunk(sm + OFF_RE + sw128_chunk(row, 0, gp * 4 + c8, 128),
+                 vals + c8 * 8);
       fence_async_smem();
     }
     tc_fence_before();
@@ -484,86 +495,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KH);
       const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = smem_u32(sm + OFF_KP);
       const uint32_t pq0 = smem_u32(pq);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
+#pragma unroll 1
+      for (int ks = 0; ks < 4; ++ks) {
         umma_bf16(tmem + TM_D1 + 64, desc_kmajor_sw128(re0 + ks * 32),
                   desc_kmajor_sw128(pq0 + ks * 32), ID_N64_NA, 1);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
                   desc_mnmajor_sw128(kh0 + ks * 2048, 8192), ID_AMN_BMN, 1);
-#pragma unroll
-      for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + TM_S, desc_kmajor_sw128(re0 + ks * 32),
                   desc_mnmajor_sw128(kp0 + ks * 2048, 8192), ID_BMN_NA, 1);
-      umma_commit(bar_m4);
-    }
-    wait(bar_m4, par, 7);
-    tc_fence_after();
-    if (half == 1) {
-      // O^T: outputs o_t (value row `row`) and the chunk sum for m
-      __nv_bfloat16* orow = o + ((size_t)b * T + t0) * H * kDV + (size_t)h * kDV + row;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + TM_D1 + 64 + part * 32, vals);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          msum += vals[e];
-          orow[(size_t)(part * 32 + e) * H * kDV] = __float2bfloat16_rn(vals[e]);
-        }
       }
+      umma_commit(bars + B_M4);
+      mark(B_M4);
     }
+    wait(B_M4, 8);
+    tc_fence_after();
 
-    // ---- 7. S <- S Diag(gamma); bf16 copy; checkpoint / final state
+    // ---- 7. outputs o_t (16 tokens per group) and their chunk sum;
+    //         S <- S Diag(gamma) (32 columns per group), bf16 copy,
+    //         checkpoint / final state
     {
-      const int c0 = half * 64;
-      float* ck = a.ck_S ? a.ck_S + ((size_t)pair * (NB + 1) + ib + 1) * SZ +
-                               (size_t)row * kDK + c0
-                         : nullptr;
+      float vals[32];
+      tmem_ld16x2(tl + TM_D1 + 64 + gp * 16, tl + TM_S + gp * 32 + 16, vals);
+      __nv_bfloat16* orow = o + ((size_t)b * T + t0 + gp * 16) * H * kDV +
+                            (size_t)h * kDV + row;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        msum += vals[e];
+        orow[(size_t)e * H * kDV] = __float2bfloat16_rn(vals[e]);
+      }
+      float sv[32];
+      tmem_ld16(tl + TM_S + gp * 32, sv);
+#pragma unroll
+      for (int e = 0; e < 16; ++e) sv[16 + e] = vals[16 + e];
+      const int c0 = gp * 32;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4) {
+        const float4 gm = *reinterpret_cast<const float4*>(s_gam + c0 + e);
+        sv[e] *= gm.x; sv[e + 1] *= gm.y; sv[e + 2] *= gm.z; sv[e + 3] *= gm.w;
+      }
+      tmem_st32(tl + TM_S + c0, sv);
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8)
+        st_chunk(sm + OFF_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
+                 sv + c8 * 8);
+      // fp32 checkpoints: the final state only (the backward of this family
+      // reads the bf16 records; the fp32 state ends dlog gamma of the last block)
+      float* ck = (a.ck_S && ib == NB - 1)
+                      ? a.ck_S + ((size_t)pair * (NB + 1) + NB) * SZ +
+                            (size_t)row * kDK + c0
+                      : nullptr;
       float* st = (a.S_T && ib == NB - 1)
                       ? a.S_T + (size_t)pair * SZ + (size_t)row * kDK + c0
                       : nullptr;
+      if (ck) {
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(tl + TM_S + c0 + part * 32, vals);
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(ck + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
+      }
+      if (st) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) vals[e] *= s_gam[c0 + part * 32 + e];
-        tmem_st32(tl + TM_S + c0 + part * 32, vals);
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8)
-          st_chunk(sm + OFF_SB + sw128_chunk(row, half, part * 4 + c8, 128),
-                   vals + c8 * 8);
-        if (ck) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(ck + part * 32 + e) =
-                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
-        }
-        if (st) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(st + part * 32 + e) =
-                make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
-        }
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4*>(st + e) = make_float4(sv[e], sv[e + 1], sv[e + 2], sv[e + 3]);
       }
       tmem_st_wait();
     }
     fence_async_smem();
-    if (chunk_end && half == 1) {
-      s_m[row] = msum / (float)a.L;
-      msum = 0.f;
-    }
+    if (chunk_end) s_mq[gp * 128 + row] = msum;
     if (tid == 0 && rec) bulk_wait_read_all();  // T, E^T records read
     tc_fence_before();
     __syncthreads();
-    if (chunk_end && ib + 1 < NB) {
-      gate((ib + 1) / bpc);
-      if (a.ck_m && tid < 128)
-        a.ck_m[((size_t)pair * a.NC + (ib + 1) / bpc) * kDV + tid] = s_m[tid];
+    if (chunk_end) {
+      if (tid < 128)
+        s_m[tid] = (s_mq[tid] + s_mq[128 + tid] + s_mq[256 + tid] + s_mq[384 + tid]) /
+                   (float)a.L;
+      msum = 0.f;
+      __syncthreads();
+      if (ib + 1 < NB) {
+        gate((ib + 1) / bpc);
+        if (a.ck_m && tid < 128)
+          a.ck_m[((size_t)pair * a.NC + (ib + 1) / bpc) * kDV + tid] = s_m[tid];
+      }
     }
   }
 
-  if (a.m_T && tid < 128) a.m_T[(size_t)pair * kDV + tid] = s_m[tid];
+  if (*s_abort) {
+    if (tid == 0 || tid == 128)  // the threads that start copies and MMAs
+      for (int i = 0; i < kNumBars; ++i)
+        if ((pend >> i) & 1u) tc::drain_bar(bars + i, (npar >> i) & 1u);
+  } else if (a.m_T && tid < 128) {
+    a.m_T[(size_t)pair * kDV + tid] = s_m[tid];
+  }
   if (tid == 0 && a.tc_rec) bulk_wait_all();
   tc_fence_before();
   __syncthreads();

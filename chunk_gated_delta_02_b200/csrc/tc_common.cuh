@@ -310,91 +310,93 @@ __device__ __forceinline__ void tile_st(float* Z, int zr, int zc,
 }
 
 // T = (I + A)^{-1} for a strictly lower 64 x 64 fp32 matrix A (layout fsw),
-// by 16 x 16 blocks on the warp-level tensor cores (tf32 in, fp32 out; T is
-// rounded to bf16 by its users).  Diagonal blocks: with N = A_II nilpotent
-// (N^16 = 0), (I + N)^{-1} = (I - N)(I + N^2)(I + N^4)(I + N^8), i.e.
-// P = I - N and P <- P + P N^(2^k), one warp per block; then the
-// off-diagonal blocks level by level, one warp per block,
-//   T_IJ = -D_I sum_{K=J}^{I-1} A_IK T_KJ   (I - J = 1, 2, 3).
-// Called by warps 0..3 only (128 threads, named barrier `bar_id`); the
-// other warps of the CTA are free meanwhile.  T (layout fsw) goes to `tf`;
-// `ws` is >= 2048 floats of scratch.  Ends with that named barrier.
+// by 16 x 16 blocks.  (1) Diagonal blocks by forward substitution in fp32,
+// one thread per column (threads 0..63): t_i = -sum_{k<i} a_ik t_k with the
+// row loaded as float4 groups and the terms before k = i - 1 summed ahead of
+// t_{i-1}.  (2) Pairs of blocks merge into 32 x 32 blocks,
+// T_10 = -T_11 (A_10 T_00), one warp per pair.  (3) The two 32 x 32 blocks
+// merge, T_BA = -T_B (A_BA T_A), one warp per 16 x 16 output tile.  (2) and
+// (3) run on the warp-level tensor cores (tf32 in, fp32 out; T is rounded to
+// bf16 by its users).  Called by warps 0..3 only (128 threads, named barrier
+// `bar_id`); the other warps of the CTA are free meanwhile.  T (layout fsw)
+// goes to `tf`; `ws` is >= 2048 floats of scratch.  Ends with that named
+// barrier.
 static __device__ __noinline__ void unit_lower_inverse64(const float* af, float* tf,
                                                   float* ws, int bar_id) {
   const int tid = threadIdx.x, warp = tid >> 5;
-  float* n2 = ws;          // N^2, later N^8   (compact diagonal blocks)
-  float* n4 = ws + 1024;   // N^4
-  // P = I - N on the diagonal blocks, zero above the block diagonal; one
-  // float4 group (4 columns of one 16-column block) per step
+  // zero blocks above the diagonal (6 blocks, 3 float4 per thread)
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int e = tid + 128 * i;        // float4 group index, 0..1023
-    const int r = e >> 4, c = (e & 15) << 2;
-    const int br = r >> 4, bc = c >> 4;
-    if (bc == br) {
-      float4 v = *reinterpret_cast<const float4*>(af + fsw(r, c));
-      v.x = (r == c) ? 1.f : -v.x;
-      v.y = (r == c + 1) ? 1.f : -v.y;
-      v.z = (r == c + 2) ? 1.f : -v.z;
-      v.w = (r == c + 3) ? 1.f : -v.w;
-      *reinterpret_cast<float4*>(tf + fsw(r, c)) = v;
-    } else if (bc > br) {
-      *reinterpret_cast<float4*>(tf + fsw(r, c)) = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int q = 0; q < 3; ++q) {
+    const int e = tid + 128 * q;          // 0..383
+    const int blk = e >> 6, r = (e & 63) >> 2, c4 = (e & 3) << 2;
+    const int bi = blk < 3 ? 0 : (blk < 5 ? 1 : 2);
+    const int bj = blk < 3 ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+    *reinterpret_cast<float4*>(tf + fsw(16 * bi + r, 16 * bj + c4)) =
+        make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  // (1) diagonal blocks
+  if (tid < 64) {
+    const int o = 16 * (tid >> 4), j = tid & 15;
+    float t[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float acc = 0.f;
+      if (i > 0) {
+        float a[16];
+#pragma unroll
+        for (int g = 0; g < (i + 3) / 4; ++g) {
+          const float4 v = *reinterpret_cast<const float4*>(af + fsw(o + i, o + 4 * g));
+          a[4 * g] = v.x; a[4 * g + 1] = v.y; a[4 * g + 2] = v.z; a[4 * g + 3] = v.w;
+        }
+        float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int k = 0; k < i - 1; ++k) p[k & 3] = fmaf(a[k], t[k], p[k & 3]);
+        acc = fmaf(a[i - 1], t[i - 1], (p[0] + p[1]) + (p[2] + p[3]));
+      }
+      t[i] = i < j ? 0.f : (i == j ? 1.f : -acc);
     }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) tf[fsw(o + i, o + j)] = t[i];
   }
   bar_named(bar_id, 128);
-  float acc[8], acc2[8];
-  if (warp < 4) {
-    const int o = 16 * warp;
+  // (2) T_10 = -T_11 (A_10 T_00) for the block pairs (0, 1) and (2, 3)
+  if (warp < 2) {
+    const int o0 = 32 * warp, o1 = o0 + 16;
+    float acc[8], acc2[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = acc2[i] = 0.f;
+    tile_mac<false, false, 1>(acc, af, o1, o0, tf, o0, o0);
+    tile_st<false>(tf, o1, o0, acc, 1.f);
+    __syncwarp();
+    tile_mac<false, false, 1>(acc2, tf, o1, o1, tf, o1, o0);
+    __syncwarp();
+    tile_st<false>(tf, o1, o0, acc2, -1.f);
+  }
+  bar_named(bar_id, 128);
+  // (3) T_BA = -T_B (A_BA T_A): output tile (I, J), I = 2, 3, J = 0, 1
+  const int I = 2 + (warp >> 1), J = warp & 1;
+  {
+    float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    tile_mac<false, false, 1>(acc, af, o, o, af, o, o);        // N^2
-    tile_st<true>(n2, o, o, acc, 1.f);
-    __syncwarp();
-    tile_ld<false>(acc, tf, o, o);                             // P (I + N^2)
-    tile_mac<false, true, 1>(acc, tf, o, o, n2, o, o);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc2[i] = 0.f;
-    tile_mac<true, true, 1>(acc2, n2, o, o, n2, o, o);         // N^4
-    __syncwarp();
-    tile_st<false>(tf, o, o, acc, 1.f);
-    tile_st<true>(n4, o, o, acc2, 1.f);
-    __syncwarp();
-    tile_ld<false>(acc, tf, o, o);                             // P (I + N^4)
-    tile_mac<false, true, 1>(acc, tf, o, o, n4, o, o);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc2[i] = 0.f;
-    tile_mac<true, true, 1>(acc2, n4, o, o, n4, o, o);         // N^8
-    __syncwarp();
-    tile_st<false>(tf, o, o, acc, 1.f);
-    tile_st<true>(n2, o, o, acc2, 1.f);
-    __syncwarp();
-    tile_ld<false>(acc, tf, o, o);                             // P (I + N^8)
-    tile_mac<false, true, 1>(acc, tf, o, o, n2, o, o);
-    __syncwarp();
-    tile_st<false>(tf, o, o, acc, 1.f);
+    if (J == 0)
+      tile_mac<false, false, 2>(acc, af, 16 * I, 0, tf, 0, 0);
+    else
+      tile_mac<false, false, 1>(acc, af, 16 * I, 16, tf, 16, 16);
+    tile_st<false>(ws, 16 * (I - 2), 16 * J, acc, 1.f);
   }
   bar_named(bar_id, 128);
+  {
+    float acc[8];
 #pragma unroll
-  for (int d = 1; d <= 3; ++d) {
-    if (warp < 4 - d) {
-      const int J = warp, I = warp + d;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      // X = sum_{K=J}^{I-1} A_IK T_KJ  (contiguous K range 16 J .. 16 I)
-      if (d == 1) tile_mac<false, false, 1>(acc, af, 16 * I, 16 * J, tf, 16 * J, 16 * J);
-      if (d == 2) tile_mac<false, false, 2>(acc, af, 16 * I, 16 * J, tf, 16 * J, 16 * J);
-      if (d == 3) tile_mac<false, false, 3>(acc, af, 16 * I, 16 * J, tf, 16 * J, 16 * J);
-      tile_st<false>(tf, 16 * I, 16 * J, acc, 1.f);   // T_IJ slot is free
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-      tile_mac<false, false, 1>(acc, tf, 16 * I, 16 * I, tf, 16 * I, 16 * J);
-      __syncwarp();
-      tile_st<false>(tf, 16 * I, 16 * J, acc, -1.f);
-    }
-    bar_named(bar_id, 128);
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    if (I == 2)
+      tile_mac<false, false, 1>(acc, tf, 32, 32, ws, 0, 16 * J);
+    else
+      tile_mac<false, false, 2>(acc, tf, 48, 32, ws, 0, 16 * J);
+    tile_st<false>(tf, 16 * I, 16 * J, acc, -1.f);
   }
+  bar_named(bar_id, 128);
 }
 
 }  // namespace tc

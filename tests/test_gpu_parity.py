@@ -244,10 +244,20 @@ def test_tensor_core_backward_matches_oracle_and_generic(case, monkeypatch):
     g_tc = carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
                            d["u_down"], d["u_up"], L, dd["d_o"], ws,
                            dd["dS_T"], dd["dm_T"])
+    # the generic backward needs the generic forward's fp32 checkpoints: it
+    # refuses the tensor-core forward's workspace
+    assert carve.get_status(ws) == 0
     monkeypatch.setenv("CARVE_BWD_PATH", "generic")
+    carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
+                    d["u_down"], d["u_up"], L, dd["d_o"], ws,
+                    dd["dS_T"], dd["dm_T"])
+    assert carve.STATUS[carve.get_status(ws)] == "CARVE_ERR_WORKSPACE"
+    monkeypatch.setenv("CARVE_FWD_PATH", "generic")
+    _, _, _, _, ws_g = run_fwd(inp, L, training=True)
     g_ge = carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
-                           d["u_down"], d["u_up"], L, dd["d_o"], ws,
+                           d["u_down"], d["u_up"], L, dd["d_o"], ws_g,
                            dd["dS_T"], dd["dm_T"])
+    assert carve.get_status(ws_g) == 0
     torch.cuda.synchronize()
     from _parity import rel as _rel
     for name in g_tc:
