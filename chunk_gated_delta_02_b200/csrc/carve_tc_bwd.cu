@@ -89,9 +89,10 @@ constexpr int kNumBars = 9;
 // TMEM columns
 constexpr uint32_t T_DS = 0;     // dS [v][j]
 constexpr uint32_t T_G = 128;    // [A|M ; P_kap|P_k] [i][t]  -> [dK~^T | dQ~^T]
-constexpr uint32_t T_RE = 256;   // dW^T  -> [-dkap^T | dK^T] (128 cols)
+constexpr uint32_t T_RE = 256;   // dW^T
 constexpr uint32_t T_DER = 320;  // dE^T -> dR^T
-constexpr uint32_t T_G2 = 384;   // raw G2 [r][c]
+constexpr uint32_t T_G2 = 384;   // raw G2 [r][c] -> D8 = [-dkap^T | dK^T]
+constexpr uint32_t T_D8 = T_G2;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t ID_KK64 = idesc_bf16(128, 64, false, false);
@@ -367,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // ---- S1: inputs.  k, q, d_o now; the rest was requested during the
     //      previous block.  Block ib - 1's tiles and record -> L2.
-    if (tid == 0) {
-      issue_top(ib);
+    if (tid == 0) issue_top(ib);
+    if (tid == 32) {
       if (ib > 0) {
         const int tn = tok - kBlk;
 #pragma unroll 1
@@ -606,26 +607,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(B_5, 16);
     tc_fence_after();
 
-    // ---- S10: the epilogue's raw g, b_x -> RO; dlog gamma share of block
-    //      ib - 1 (its S_new is this block's state record, still in SB);
-    //      G2 (masked, bf16; 32 columns per group); dv, dw (16 tokens per group)
+    // ---- S10: the epilogue's raw g, b_x -> RO; G2 (masked, bf16; 32
+    //      columns per group)
     if (tid == 0 && !*s_abort) issue_gb(ib);
-    if (ib > 0) {
-      float vals[32], sv[32];
-      tmem_ld32(tl + T_DS + gp * 32, vals);
-#pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8)
-        ld_chunk(sm + R_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
-                 sv + c8 * 8);
-#pragma unroll
-      for (int e = 0; e < 32; ++e) vals[e] *= sv[e];
-      dlg_part = warp_reduce_scatter32(vals, lane);
-    }
     {
       const int rl = row & 63;
-      float vals[32], dwv[16];
+      float vals[32];
       tmem_ld32(tl + T_G2 + gp * 32, vals);
-      tmem_ld16(tl + T_RE + gp * 16, dwv);
 #pragma unroll
       for (int e = 0; e < 32; ++e)
         if (((gp & 1) * 32 + e) >= rl) vals[e] = 0.f;
@@ -633,31 +621,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8)
         st_chunk(blk + sw128_chunk(row, 0, (gp & 1) * 4 + c8, 128), vals + c8 * 8);
-      __nv_bfloat16* dvrow = dv + ((size_t)tok + gp * 16) * H * kDV +
-                             (size_t)h * kDV + row;
-#pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const int t = gp * 16 + e;
-        dvrow[(size_t)e * H * kDV] = __float2bfloat16_rn(s_w[t] * dwv[e]);
-        dwv[e] *= ldbf(sm + R_W + sw128_off(t, row, 64));
-      }
-      const float sdw = warp_reduce_scatter16(dwv, lane);
-      if (lane < 16) atomicAdd(&s_dw[gp * 16 + lane], sdw);
     }
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
     if (*s_abort) break;
-    if (tid < 64) {  // dw_t = sum_v dW V = (sum_v dW W) / w_t
-      const float wt = s_w[tid];
-      dw[((size_t)tok + tid) * H + h] =
-          __float2bfloat16_rn(wt != 0.f ? s_dw[tid] / wt : 0.f);
-    }
 
-    // ---- S11: D7^T += [-kap^; K^]^T G2^T ; D8^T = X^T G2 + dS~^T [E; W]^T;
-    //      block ib - 1's state operand -> SB (read above)
+    // ---- S11: D7^T += [-kap^; K^]^T G2^T ; D8^T = X^T G2 + dS~^T [E; W]^T
+    //      (into the columns G2 left); meanwhile dv, dw (16 tokens per group)
+    //      and the dlog gamma share of block ib - 1 (its S_new is this
+    //      block's state record, still in SB)
     if (tid == 0) {
-      if (ib > 0 && !*s_abort) issue_sb(ib - 1);
       tc_fence_after();
       const uint32_t kp0 = smem_u32(sm + R_KP), kh0 = smem_u32(sm + R_KH);
       const uint32_t mp0 = smem_u32(sm + R_MP), pq0 = smem_u32(sm + R_PQ);
@@ -672,17 +646,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
-        umma_bf16(tmem + T_RE, desc_mnmajor_sw128(x0 + ks * 2048, 16384),
+        umma_bf16(tmem + T_D8, desc_mnmajor_sw128(x0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(mp0 + ks * 2048, 16384), ID_MM128, ks > 0);
-        umma_bf16(tmem + T_RE, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
+        umma_bf16(tmem + T_D8, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(et0 + ks * 2048, 16384), ID_MM64, 1);
-        umma_bf16(tmem + T_RE + 64, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
+        umma_bf16(tmem + T_D8 + 64, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
                   desc_kmajor_sw128(w0 + (ks >> 2) * 8192 + (ks & 3) * 32),
                   ID_MK64, 1);
       }
       umma_commit(bars + B_7);
       mark(B_7);
     }
+    if (ib > 0) {
+      float vals[32];
+      tmem_ld32(tl + T_DS + gp * 32, vals);
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        float sv[8];
+        ld_chunk(sm + R_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128), sv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) vals[8 * c8 + e] *= sv[e];
+      }
+      dlg_part = warp_reduce_scatter32(vals, lane);
+    }
+    {
+      float dwv[16];
+      tmem_ld16(tl + T_RE + gp * 16, dwv);
+      __nv_bfloat16* dvrow = dv + ((size_t)tok + gp * 16) * H * kDV +
+                             (size_t)h * kDV + row;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int t = gp * 16 + e;
+        dvrow[(size_t)e * H * kDV] = __float2bfloat16_rn(s_w[t] * dwv[e]);
+        dwv[e] *= ldbf(sm + R_W + sw128_off(t, row, 64));
+      }
+      const float sdw = warp_reduce_scatter16(dwv, lane);
+      if (lane < 16) atomicAdd(&s_dw[gp * 16 + lane], sdw);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (tid < 64) {  // dw_t = sum_v dW V = (sum_v dW W) / w_t
+      const float wt = s_w[tid];
+      dw[((size_t)tok + tid) * H + h] =
+          __float2bfloat16_rn(wt != 0.f ? s_dw[tid] / wt : 0.f);
+    }
+    // block ib - 1's state operand -> SB (read above)
+    if (tid == 0 && ib > 0 && !*s_abort) issue_sb(ib - 1);
     wait(B_7, 17);
     // block ib - 1's v, g, b_x, E^T, T into the buffers S11 released
     if (tid == 0 && ib > 0 && !*s_abort) issue_pre(ib - 1);
@@ -719,8 +728,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int sub = 0; sub < 2; ++sub) {
         float dd[32];  // dK~ | dQ~ | -dkap^ | dK^ of 8 tokens
         const int tsub = tb + 8 * sub;
-        tmem_ld8x4(tl + T_G + tsub, tl + T_G + 64 + tsub, tl + T_RE + tsub,
-                   tl + T_RE + 64 + tsub, dd);
+        tmem_ld8x4(tl + T_G + tsub, tl + T_G + 64 + tsub, tl + T_D8 + tsub,
+                   tl + T_D8 + 64 + tsub, dd);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           const int tl_ = 8 * sub + e;
