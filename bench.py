@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--mode train|fwd]
                     [--workload layer_1p3b|long_context|tiny] [--impl carve|reference]
+                    [--seq-len T]   (a shorter sequence, for profiler captures)
 
 One step = one pass of the whole hot path over one batch: the training-mode
 forward (chunk walk, gate, WY solve, state update, checkpoints) plus the
@@ -17,6 +18,7 @@ scaling; the time is the max over ranks.
 Prints ONE JSON line on rank 0.
 """
 import argparse
+import hashlib
 import json
 import os
 import statistics
@@ -62,6 +64,37 @@ def fwd_bytes(K, V, e):
 
 def bwd_bytes(K, V, e):
     return e * (8 * K + 3 * V + 2)      # q k g bx v w d_o in, 6 grads out
+
+
+def kernel_sources_sha1():
+    """Hash of the CUDA sources: DRAM counters taken on other sources are stale."""
+    d = os.path.join(HERE, "chunk_gated_delta_02_b200", "csrc")
+    h = hashlib.sha1()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic(kernel, cfg, token_heads):
+    """DRAM bytes (read + write) per launch of `kernel` at this shape, from
+    the ncu capture summarised in profiles/tc_traffic.json (a smaller case of
+    the same kernel, scaled by token-heads), or None when that capture was
+    taken on other kernel sources or another shape family."""
+    p = os.path.join(HERE, "profiles", "tc_traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    if d.get("sources_sha1") != kernel_sources_sha1():
+        return None
+    k = d.get("kernels", {}).get(kernel)
+    if not k:
+        return None
+    for n in ("DK", "DV", "L", "R"):
+        if k["shape"][n] != cfg[n]:
+            return None
+    return k["dram_bytes_per_token_head"] * token_heads
 
 
 class ClockSampler:
@@ -193,7 +226,9 @@ def run_reference(args, cfg, ws, rank):
 
 
 def config_dict(args, cfg):
-    return {"workload": "%s %s" % (args.workload,
+    name = args.workload if not args.seq_len else "%s(T=%d)" % (args.workload,
+                                                               args.seq_len)
+    return {"workload": "%s %s" % (name,
                                    "fwd+bwd" if args.mode == "train" else "fwd"),
             "B": cfg["B"], "T": cfg["T"], "H": cfg["H"], "DK": cfg["DK"],
             "DV": cfg["DV"], "L": cfg["L"], "R": cfg["R"],
@@ -211,10 +246,14 @@ def main():
     ap.add_argument("--impl", choices=["carve", "reference"], default="carve")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override T (profiler captures of a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "carve":
         ap.error("--warmup must be >= 3")
     cfg = dict(WORKLOADS[args.workload])
+    if args.seq_len:
+        cfg["T"] = args.seq_len
     ws, rank, local = dist_init() if args.impl == "carve" else (
         int(os.environ.get("WORLD_SIZE", "1")),
         int(os.environ.get("RANK", "0")), 0)
@@ -309,8 +348,9 @@ def main():
         dom, dom_ms, dom_b, dom_f = "bwd", bwd_ms, bwd_b, bwd_f
     else:
         dom, dom_ms, dom_b, dom_f = "fwd", fwd_ms, fwd_b, fwd_f
-    peak = pk["hbm"] if dom == "fwd" else pk["hbm"]
+    peak = pk["hbm"]
     achieved = dom_b / (dom_ms * 1e-3) / 1e9
+    traffic = measured_traffic(dom + "_tc", cfg, B * T * H)
     roof_t_fwd = max(fwd_f / (pk["bf16"] * 1e12), fwd_b / (pk["hbm"] * 1e9))
     roof_t_all = max((fwd_f + (bwd_f if training else 0)) / (pk["bf16"] * 1e12),
                      (fwd_b + (bwd_b if training else 0)) / (pk["hbm"] * 1e9))
@@ -324,7 +364,7 @@ def main():
                                                        dtype)),
         "roofline": {"bound": "hbm", "kernel": "carve_chunk_" + dom,
                      "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak, "traffic": traffic,
                      "peak_src": pk["src"] + " hbm_gbs",
                      "algorithmic_bytes": dom_b, "algorithmic_flops": dom_f,
                      "ms_per_launch": dom_ms},
