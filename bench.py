@@ -374,7 +374,10 @@ def main():
                 "roofline_ms": roof_t_fwd * 1e3,
                 "frac": roof_t_fwd * 1e3 / fwd_ms},
         "bwd": {"ms": bwd_ms} if training else None,
-        "gpu_launches": args.steps * (3 if training else 1),
+        # per step: the forward; the backward kernel and, with R > 0, the two
+        # dU reduction kernels
+        "gpu_launches": args.steps * ((2 + (2 if R > 0 else 0)) if training
+                                      else 1),
         "clocks": clk,
     }
 

@@ -387,35 +387,46 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
     if (chunk_first && ib > 0 && tid < 128)  // the next block starts chunk c - 1
       p_next = a.gin[((size_t)pair * NC + c - 1) * GR + tid];
-    // w_t of the token row this thread scales in W = w V
-    const float wrow = __bfloat162float(w_in[((size_t)tok + (tid >> 3)) * H + h]);
+    // w_t of the two token rows a thread of warps 8-15 scales in W = w V
+    float w_lo = 0.f, w_hi = 0.f;
+    if (warp >= 8) {
+      const size_t r0 = (size_t)tok + ((tid - 256) >> 3);
+      w_lo = __bfloat162float(w_in[r0 * H + h]);
+      w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+    }
     wait(B_SB, 10);
     wait(B_PRE, 11);
     wait(B_IN, 12);
     __syncthreads();  // s_p of S0
 
-    // ---- S2: transform; s_x is cleared: it accumulates dlog gamma next
-    tc::transform_block<16>(sm + R_X, sm + R_KH, sm + R_KP, sm + R_DSB,
-                            sm + R_DSB + 16384, s_p, s_gam,
-                            reinterpret_cast<float*>(sm + R_MP), 3);
-    if (tid < 128) s_x[tid] = 0.f;
-    {
+    // ---- S2: transform (warps 0-7 the key side; warps 8-15 W = w V and
+    //      dO = d_o + dm / L meanwhile); s_x is cleared: it accumulates
+    //      dlog gamma next
+    if (warp < 8) {
+      tc::transform_block<8>(sm + R_X, sm + R_KH, sm + R_KP, sm + R_DSB,
+                             sm + R_DSB + 16384, s_p, s_gam,
+                             reinterpret_cast<float*>(sm + R_MP), 3);
+      if (tid < 128) s_x[tid] = 0.f;
+    } else {
       const float invL = 1.0f / (float)a.L;
-      const int rr = tid >> 3, ch = tid & 7;  // token row, 16-byte chunk
-      const uint32_t sub = (uint32_t)((rr >> 3) * 1024 + (rr & 7) * 128 + ch * 16);
+      const int u = tid - 256;
+      const int rr = u >> 3, ch = u & 7;  // token rows rr, rr + 32; 16-byte chunk
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
+      for (int i = 0; i < 4; ++i) {
+        const int r = rr + 32 * (i & 1), kb = i >> 1;
+        const uint32_t sub = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ch * 16);
         // W = w V in place
         {
           const uint32_t off = (uint32_t)(kb * 8192) + sub;
           const uint4 x = *reinterpret_cast<const uint4*>(sm + R_W + off);
+          const float wt = (i & 1) ? w_hi : w_lo;
           const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
           uint4 y;
           uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = __bfloat1622float2(xv[e]);
-            yv[e] = pack2(f.x * wrow, f.y * wrow);
+            yv[e] = pack2(f.x * wt, f.y * wt);
           }
           *reinterpret_cast<uint4*>(sm + R_W + off) = y;
         }
@@ -423,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           const uint32_t off = (uint32_t)(kb * 16384 + 8192) + sub;
           const uint4 x = *reinterpret_cast<const uint4*>(sm + R_RO + off);
-          const int v0 = kb * 64 + ((ch ^ (rr & 7)) << 3);
+          const int v0 = kb * 64 + ((ch ^ (r & 7)) << 3);
           const float4 m0 = *reinterpret_cast<const float4*>(s_dmn + v0);
           const float4 m1 = *reinterpret_cast<const float4*>(s_dmn + v0 + 4);
           const float dm8[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
@@ -851,38 +862,38 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// dU_up[h][j][r] = sum_{b,c} dp[b,h,c][j] h[b,h,c][r]
-// dU_down[h][r][v] = sum_{b,c} dh[b,h,c][r] m[b,h,c][v]   (fixed order)
+// dU_up[h][j][r] = sum_b sum_c dp[b,h,c][j] h[b,h,c][r]
+// dU_down[h][r][v] = sum_b sum_c dh[b,h,c][r] m[b,h,c][v]   (fixed order)
 // dp, dh come from the backward's gate records, h = U_down m_c from the
-// forward's gate inputs, m_c from its checkpoints.  CTA (h, part) forms the
-// channel rows 32 part .. + 31 of dU_up and value columns 32 part .. + 31 of
-// dU_down, walking the (b, c) records in order through 64-record slabs in
-// shared memory; R <= 32.
+// forward's gate inputs, m_c from its checkpoints.  Stage 1: CTA (pair,
+// part) sums the pair's chunks in order for the channel rows 32 part .. + 31
+// of dU_up and the value columns 32 part .. + 31 of dU_down, through
+// 64-record slabs in shared memory, into the pair's slot of the workspace
+// (layout: dU_down [R][DV] then dU_up [DK][R]); stage 2 sums the pairs of a
+// head over b in order.  R <= 32.
 constexpr int kDuThreads = 256;
 constexpr int kDuSlab = 64;
 __global__ void __launch_bounds__(kDuThreads)
-    du_from_gate_records(const float* __restrict__ rec,
-                         const float* __restrict__ gin,
-                         const float* __restrict__ ck_m, int B, int H, int NC,
-                         int R, float* du_down, float* du_up) {
+    du_pair_partials(const float* __restrict__ rec,
+                     const float* __restrict__ gin,
+                     const float* __restrict__ ck_m, int NC, int R,
+                     float* __restrict__ part) {
   __shared__ __align__(16) float s_dp[kDuSlab][32];
   __shared__ __align__(16) float s_hv[kDuSlab][32];
   __shared__ __align__(16) float s_dh[kDuSlab][32];
   __shared__ __align__(16) float s_m[kDuSlab][32];
-  const int h = blockIdx.x, part = blockIdx.y, t = threadIdx.x;
+  const int pair = blockIdx.x, pt = blockIdx.y, t = threadIdx.x;
   const int GR = kDK + R;
-  const int N = B * NC;
   const int hi = t >> 3, lo4 = 4 * (t & 7);
   float up[4] = {0.f, 0.f, 0.f, 0.f}, dn[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int n0 = 0; n0 < N; n0 += kDuSlab) {
+  for (int c0 = 0; c0 < NC; c0 += kDuSlab) {
     for (int idx = t; idx < kDuSlab * 32; idx += kDuThreads) {
-      const int n = n0 + (idx >> 5), k = idx & 31;
+      const int c = c0 + (idx >> 5), k = idx & 31;
       float dp = 0.f, hv = 0.f, dh = 0.f, mv = 0.f;
-      if (n < N) {
-        const int bb = n / NC, c = n - bb * NC;
-        const size_t o = ((size_t)bb * H + h) * NC + c;
-        dp = rec[o * GR + 32 * part + k];
-        mv = ck_m[o * kDV + 32 * part + k];
+      if (c < NC) {
+        const size_t o = (size_t)pair * NC + c;
+        dp = rec[o * GR + 32 * pt + k];
+        mv = ck_m[o * kDV + 32 * pt + k];
         if (k < R) {
           hv = gin[o * GR + kDK + k];
           dh = rec[o * GR + kDK + k];
@@ -894,7 +905,7 @@ __global__ void __launch_bounds__(kDuThreads)
       s_m[idx >> 5][k] = mv;
     }
     __syncthreads();
-    const int ns = min(kDuSlab, N - n0);
+    const int ns = min(kDuSlab, NC - c0);
     for (int n = 0; n < ns; ++n) {
       const float a = s_dp[n][hi], d = s_dh[n][hi];
       const float4 hv = *reinterpret_cast<const float4*>(&s_hv[n][lo4]);
@@ -906,11 +917,29 @@ __global__ void __launch_bounds__(kDuThreads)
     }
     __syncthreads();
   }
-  const int j = 32 * part + hi;  // dU_up row; dU_down row is r = hi
+  float* base = part + (size_t)pair * ((size_t)R * kDV + (size_t)kDK * R);
+  const int j = 32 * pt + hi;  // dU_up row; dU_down row is r = hi
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    if (lo4 + k < R) du_up[((size_t)h * kDK + j) * R + lo4 + k] = up[k];
-    if (hi < R) du_down[((size_t)h * R + hi) * kDV + 32 * part + lo4 + k] = dn[k];
+    if (hi < R) base[(size_t)hi * kDV + 32 * pt + lo4 + k] = dn[k];
+    if (lo4 + k < R) base[(size_t)R * kDV + (size_t)j * R + lo4 + k] = up[k];
+  }
+}
+
+__global__ void du_sum_pairs(const float* __restrict__ part, int B, int H,
+                             int R, float* du_down, float* du_up) {
+  const size_t per = (size_t)R * kDV + (size_t)kDK * R;
+  const size_t n = (size_t)H * per;
+  for (size_t idx = blockIdx.x * (size_t)blockDim.x + threadIdx.x; idx < n;
+       idx += (size_t)gridDim.x * blockDim.x) {
+    const int h = (int)(idx / per);
+    const size_t e = idx - (size_t)h * per;
+    float acc = 0.f;
+    for (int bb = 0; bb < B; ++bb) acc += part[((size_t)bb * H + h) * per + e];
+    if (e < (size_t)R * kDV)
+      du_down[(size_t)h * R * kDV + e] = acc;
+    else
+      du_up[(size_t)h * kDK * R + (e - (size_t)R * kDV)] = acc;
   }
 }
 
@@ -962,9 +991,16 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
                                                          mb, mdo);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (a.R > 0)
-    du_from_gate_records<<<dim3(a.H, kDK / 32), kDuThreads, 0, st>>>(
-        a.scratch, a.gin, a.ck_m, a.B, a.H, a.NC, a.R, a.du_down, a.du_up);
+  if (a.R > 0) {
+    du_pair_partials<<<dim3(a.B * a.H, kDK / 32), kDuThreads, 0, st>>>(
+        a.scratch, a.gin, a.ck_m, a.NC, a.R, a.du);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const size_t n = (size_t)a.H * ((size_t)a.R * kDV + (size_t)kDK * a.R);
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 4 * 148) blocks = 4 * 148;
+    du_sum_pairs<<<blocks, 256, 0, st>>>(a.du, a.B, a.H, a.R, a.du_down, a.du_up);
+  }
   return cudaGetLastError();
 }
 

@@ -190,14 +190,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // content gate of chunk c: s_p = U_up (U_down s_m); training records p_c
-  // and h_c = U_down m_c for the backward
-  auto gate = [&](int c) {
+  // content gate of chunk c: s_p = U_up (U_down m); training records p_c
+  // and h_c = U_down m_c for the backward.  m_v = scale * (sum of the four
+  // partial sums mq[q * 128 + v]), so the chunk mean needs no pass of its own.
+  auto gate = [&](int c, const float* mq, float scale) {
     {
       const int r = tid >> 4, part = tid & 15;
       float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc = fmaf(ud_r[i], s_m[8 * part + i], acc);
+      for (int i = 0; i < 8; ++i) {
+        const int v = 8 * part + i;
+        acc = fmaf(ud_r[i], (mq[v] + mq[128 + v]) + (mq[256 + v] + mq[384 + v]), acc);
+      }
+      acc *= scale;
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       acc += __shfl_xor_sync(0xffffffffu, acc, 4);
@@ -257,10 +262,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       st_chunk(sm + OFF_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
                vals + c8 * 8);
   }
-  if (tid < 128) s_m[tid] = a.m0 ? a.m0[(size_t)pair * kDV + tid] : 0.f;
+  float* s_mq = s_af;  // [4][128] partial sums of m (A buffer is free then)
+  if (tid < 128) {
+    const float m0 = a.m0 ? a.m0[(size_t)pair * kDV + tid] : 0.f;
+    s_m[tid] = m0;
+    s_mq[tid] = m0;
+    s_mq[128 + tid] = s_mq[256 + tid] = s_mq[384 + tid] = 0.f;
+  }
   tmem_st_wait();
   __syncthreads();
-  gate(0);
+  gate(0, s_mq, 1.f);
   if (a.ck_m && tid < 128) a.ck_m[(size_t)pair * a.NC * kDV + tid] = s_m[tid];
   if (tid == 0) {
     issue_vgb(0);
@@ -271,7 +282,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   float msum = 0.f;  // this thread's token quarter of the chunk's sum of o, row `row`
-  float* s_mq = s_af;  // [4][128] quarter sums of o at a chunk end (A buffer is free)
   for (int ib = 0; ib < NB; ++ib) {
     const int t0 = ib * kBlk;
     const bool chunk_end = ((ib + 1) % bpc) == 0;
@@ -285,28 +295,38 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_store(rec + kTcRecS, sm + OFF_SB, 32768);
       bulk_commit();
     }
-    // w_t of the token row this thread scales in W = w V
-    const float wrow = __bfloat162float(w_in[((size_t)b * T + t0 + (tid >> 3)) * H + h]);
+    // w_t of the two token rows a thread of warps 8-15 scales in W = w V
+    float w_lo = 0.f, w_hi = 0.f;
+    if (warp >= 8) {
+      const size_t r0 = (size_t)b * T + t0 + ((tid - 256) >> 3);
+      w_lo = __bfloat162float(w_in[r0 * H + h]);
+      w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+    }
     wait(B_VGB, 1);
     wait(B_KQ, 2);
 
     // ---- 2. transform: decay scan, gated and decayed operands, W = w V
-    tc::transform_block<16>(sm + OFF_X, sm + OFF_KH, sm + OFF_KP, sm + OFF_RG,
-                            sm + OFF_RB, s_p, s_gam, s_af, 3);
-    {
-      const int rr = tid >> 3, ch = tid & 7;  // token row, 16-byte chunk
+    //      (warps 0-7 the key side, warps 8-15 W = w V meanwhile)
+    if (warp < 8) {
+      tc::transform_block<8>(sm + OFF_X, sm + OFF_KH, sm + OFF_KP, sm + OFF_RG,
+                             sm + OFF_RB, s_p, s_gam, s_af, 3);
+    } else {
+      const int u = tid - 256;
+      const int rr = u >> 3, ch = u & 7;  // token rows rr, rr + 32; 16-byte chunk
 #pragma unroll
-      for (int kb = 0; kb < 2; ++kb) {
-        const uint32_t off = (uint32_t)(kb * 8192 + (rr >> 3) * 1024 +
-                                        (rr & 7) * 128 + ch * 16);
+      for (int i = 0; i < 4; ++i) {
+        const int r = rr + 32 * (i & 1), kb = i >> 1;
+        const uint32_t off = (uint32_t)(kb * 8192 + (r >> 3) * 1024 +
+                                        (r & 7) * 128 + ch * 16);
         const uint4 x = *reinterpret_cast<const uint4*>(sm + OFF_RV + off);
+        const float wt = (i & 1) ? w_hi : w_lo;
         const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
         uint4 y;
         uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 f = __bfloat1622float2(xv[e]);
-          yv[e] = pack2(f.x * wrow, f.y * wrow);
+          yv[e] = pack2(f.x * wt, f.y * wt);
         }
         *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
       }
@@ -565,16 +585,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_before();
     __syncthreads();
     if (chunk_end) {
-      if (tid < 128)
-        s_m[tid] = (s_mq[tid] + s_mq[128 + tid] + s_mq[256 + tid] + s_mq[384 + tid]) /
-                   (float)a.L;
-      msum = 0.f;
-      __syncthreads();
-      if (ib + 1 < NB) {
-        gate((ib + 1) / bpc);
-        if (a.ck_m && tid < 128)
-          a.ck_m[((size_t)pair * a.NC + (ib + 1) / bpc) * kDV + tid] = s_m[tid];
+      // m = chunk mean of o: the quarter sums are folded into the gate's
+      // first GEMV; s_m keeps m for m_T and the checkpoint
+      const float invL = 1.0f / (float)a.L;
+      if (tid < 128) {
+        const float m = (s_mq[tid] + s_mq[128 + tid] + s_mq[256 + tid] + s_mq[384 + tid]) * invL;
+        s_m[tid] = m;
+        if (a.ck_m && ib + 1 < NB)
+          a.ck_m[((size_t)pair * a.NC + (ib + 1) / bpc) * kDV + tid] = m;
       }
+      msum = 0.f;
+      if (ib + 1 < NB) gate((ib + 1) / bpc, s_mq, invL);
     }
   }
 
