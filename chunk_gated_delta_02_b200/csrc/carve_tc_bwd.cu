@@ -367,21 +367,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // ---- S1: inputs.  k, q, d_o now; the rest was requested during the
-    //      previous block.  Block ib - 1's tiles and record -> L2.
+    //      previous block.  Block ib - 1's k, q, d_o tiles -> L2.
     if (tid == 0) issue_top(ib);
-    if (tid == 32) {
-      if (ib > 0) {
-        const int tn = tok - kBlk;
+    if (tid == 32 && ib > 0) {  // (the rest of block ib - 1 loads a block ahead)
+      const int tn = tok - kBlk;
 #pragma unroll 1
-        for (int x0 = 0; x0 < 128; x0 += 64) {
-          tma_prefetch_3d(&tm_k, x0, h, tn);
-          tma_prefetch_3d(&tm_q, x0, h, tn);
-          tma_prefetch_3d(&tm_v, x0, h, tn);
-          tma_prefetch_3d(&tm_do, x0, h, tn);
-          tma_prefetch_3d(&tm_g, x0, h, tn);
-          tma_prefetch_3d(&tm_bx, x0, h, tn);
-        }
-        bulk_prefetch_l2(rec0 + (size_t)(ib - 1) * kTcRecBytes, (uint32_t)kTcRecBytes);
+      for (int x0 = 0; x0 < 128; x0 += 64) {
+        tma_prefetch_3d(&tm_k, x0, h, tn);
+        tma_prefetch_3d(&tm_q, x0, h, tn);
+        tma_prefetch_3d(&tm_do, x0, h, tn);
       }
     }
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);

@@ -172,8 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto mark = [&](int i) { pend |= 1u << i; };
 
   // U_b factors: thread (r = tid / 16, part = tid % 16) holds U_down[h][r]
-  // [8 part .. 8 part + 7] in registers; U_up[h] is kept transposed in
-  // shared memory (s_uu[r][j], zero for r >= R).
+  // [part + 16 i], i < 8, in registers (lanes read consecutive m values);
+  // U_up[h] is kept transposed in shared memory (s_uu[r][j], zero for r >= R).
   float ud_r[8];
   __nv_bfloat16* s_uu = reinterpret_cast<__nv_bfloat16*>(sm + OFF_UU);
   {
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       ud_r[i] = (r < R) ? __bfloat162float(
-                              ud[((size_t)h * R + r) * kDV + 8 * part + i])
+                              ud[((size_t)h * R + r) * kDV + part + 16 * i])
                         : 0.f;
     for (int e = tid; e < kRMax * kDK; e += kThreads) {
       const int r2 = e / kDK, jj = e - r2 * kDK;
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc = 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int v = 8 * part + i;
+        const int v = part + 16 * i;
         acc = fmaf(ud_r[i], (mq[v] + mq[128 + v]) + (mq[256 + v] + mq[384 + v]), acc);
       }
       acc *= scale;
@@ -210,15 +210,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (part == 0) s_h[r] = acc;
     }
     __syncthreads();
-    if (tid < 128) {
+    {  // p_j: four threads per channel j = tid / 4, 8 ranks each
+      const int jj = tid >> 2, rq = tid & 3;
       float acc = 0.f;
-#pragma unroll 8
-      for (int r = 0; r < kRMax; ++r)
-        acc = fmaf(__bfloat162float(s_uu[r * kDK + tid]), s_h[r], acc);
-      s_p[tid] = acc;
-      if (a.gin) a.gin[((size_t)pair * a.NC + c) * (kDK + R) + tid] = acc;
-    } else if (a.gin && tid - 128 < R) {
-      a.gin[((size_t)pair * a.NC + c) * (kDK + R) + kDK + tid - 128] = s_h[tid - 128];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        acc = fmaf(__bfloat162float(s_uu[(8 * rq + i) * kDK + jj]), s_h[8 * rq + i], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (rq == 0) {
+        s_p[jj] = acc;
+        if (a.gin) a.gin[((size_t)pair * a.NC + c) * (kDK + R) + jj] = acc;
+      }
+      if (a.gin && rq == 1 && jj < R)
+        a.gin[((size_t)pair * a.NC + c) * (kDK + R) + kDK + jj] = s_h[jj];
     }
     __syncthreads();
   };
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- 1. inputs of this block (block ib + 2's tiles -> L2 ahead of
     //         their loads, which are issued during block ib + 1); training
     //         records the block's bf16 state operand
-    if (tid == 0 && rec) {
+    if (tid == 256 && rec) {  // (a warp of the light half of the transform)
       bulk_store(rec + kTcRecS, sm + OFF_SB, 32768);
       bulk_commit();
     }
@@ -332,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     fence_async_smem();
-    if (tid == 0 && rec) bulk_wait_read_all();  // S record read: SB reusable
+    if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
     __syncthreads();
     if (*s_abort) break;
 
@@ -452,22 +457,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
-    } else {
-      // warps 12-15: block ib + 2's tiles -> L2 (their loads are issued
-      // during block ib + 1)
-      if (tid == 384 && ib + 2 < NB) {
-        const int tn = b * T + (ib + 2) * kBlk;
-#pragma unroll 1
-        for (int x0 = 0; x0 < 128; x0 += 64) {
-          tma_prefetch_3d(&tm_k, x0, h, tn);
-          tma_prefetch_3d(&tm_q, x0, h, tn);
-          tma_prefetch_3d(&tm_v, x0, h, tn);
-          tma_prefetch_3d(&tm_g, x0, h, tn);
-          tma_prefetch_3d(&tm_bx, x0, h, tn);
-        }
-      }
-      wait(B_M2, 6);  // keeps every thread's view of the barrier phases in step
     }
+    // (warps 12-15 do not wait on MMA 2: they park at the barrier below
+    // instead of polling while warps 0-3 solve)
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -606,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (a.m_T && tid < 128) {
     a.m_T[(size_t)pair * kDV + tid] = s_m[tid];
   }
-  if (tid == 0 && a.tc_rec) bulk_wait_all();
+  if ((tid == 0 || tid == 256) && a.tc_rec) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
