@@ -37,10 +37,10 @@ bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
 // Forward kernel family for a valid shape: the tensor-core kernel where it
 // applies, else the generic one.  CARVE_FWD_PATH=generic forces the generic
 // kernel (both are GPU kernels; used to cross-check the two paths).
-bool use_tc_fwd(const carve_shape& s) {
+bool use_tc_fwd(const carve_shape& s, bool training) {
   const char* env = getenv("CARVE_FWD_PATH");
   if (env && strcmp(env, "generic") == 0) return false;
-  return tc_fwd_supported(s);
+  return tc_fwd_supported(s, training);
 }
 bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
 
@@ -50,7 +50,7 @@ bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
 bool use_tc_bwd(const carve_shape& s) {
   const char* env = getenv("CARVE_BWD_PATH");
   if (env && strcmp(env, "generic") == 0) return false;
-  return use_tc_fwd(s);
+  return use_tc_fwd(s, true);
 }
 
 }  // namespace
@@ -76,7 +76,7 @@ const char* carve_status_str(carve_status s) {
 
 const char* carve_fwd_path(const carve_shape* shape) {
   if (check_shape(shape) != CARVE_OK) return nullptr;
-  return use_tc_fwd(*shape) ? "tc" : "generic";
+  return use_tc_fwd(*shape, false) ? "tc" : "generic";
 }
 
 carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
@@ -117,7 +117,7 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   a.tc_rec = training && L.tc_rec ? (uint8_t*)(ws + L.tc_rec) : nullptr;
   a.gin = training && L.gin ? (float*)(ws + L.gin) : nullptr;
   a.hdr = (WsHeader*)ws;
-  cudaError_t e = use_tc_fwd(s)
+  cudaError_t e = use_tc_fwd(s, training != 0)
                       ? launch_fwd_tc(a, (cudaStream_t)stream)
                       : launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;

@@ -32,9 +32,17 @@ constexpr size_t kTcRecE = 32768;      // E^T  [v 128][t 64]  bf16  16 KB
 constexpr size_t kTcRecT = 49152;      // T    [t 64][s 64]   bf16   8 KB
 constexpr size_t kTcRecBytes = 57344;
 
-// Tensor-core kernels: bf16, DK = DV = 128, L % 64 == 0, R <= 32, T > 0.
+// Tensor-core kernels: bf16, DK = DV = 128, L % 64 == 0, R <= 32, T > 0
+// (the training forward, whose records this describes, and the backward).
 inline bool tc_shape(const carve_shape& s) {
   return s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 128 &&
+         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0;
+}
+// The tensor-core forward also runs DV = 256 (two CTAs per pair) without
+// training.
+inline bool tc_fwd_shape(const carve_shape& s, bool training) {
+  if (tc_shape(s)) return true;
+  return !training && s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 256 &&
          s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0;
 }
 static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
@@ -150,9 +158,8 @@ cudaError_t launch_fwd_generic(const FwdArgs& a, int dtype, cudaStream_t st);
 cudaError_t launch_bwd_generic(const BwdArgs& a, int dtype, cudaStream_t st);
 size_t generic_fwd_smem_bytes(int C, int DK, int DV);
 
-// Tensor-core forward (carve_tc_fwd.cu): bf16, DK = DV = 128, L % 64 == 0,
-// R <= 32, T > 0.
-bool tc_fwd_supported(const carve_shape& s);
+// Tensor-core forward (carve_tc_fwd.cu): see tc_fwd_shape.
+bool tc_fwd_supported(const carve_shape& s, bool training);
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st);
 
 // Tensor-core backward (carve_tc_bwd.cu), same shapes as the forward; it

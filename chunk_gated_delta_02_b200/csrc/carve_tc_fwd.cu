@@ -67,6 +67,7 @@ constexpr uint32_t OFF_AF = 196608;    // A fp32 64 x 64 row-major     16 KB
 constexpr uint32_t OFF_SMALL = 212992;
 constexpr uint32_t SM_GAM = 0;         // gamma_j            128 f32
 constexpr uint32_t SM_P = 512;         // (U_b m)_j          128 f32
+constexpr uint32_t SM_HX = 1024;       // the other CTA's half of U_down m, 2 x 32 f32
 constexpr uint32_t SM_M = 1280;        // m_v                128 f32
 constexpr uint32_t SM_H = 1792;        // U_down m            64 f32
 constexpr uint32_t SM_BAR = 2560;      // kNumBars mbarriers
@@ -86,7 +87,8 @@ constexpr int B_M2 = 3;    // MMA 2 (W^T [M;P_k]^T)
 constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
 constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
 constexpr int B_D1 = 6;    // MMA 1, second half (S X^T)
-constexpr int kNumBars = 7;
+constexpr int B_X = 7;     // dv = 256: the other CTA's half of U_down m arrived
+constexpr int kNumBars = 8;
 
 // TMEM columns (fp32, lanes = rows)
 constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
@@ -119,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_p = reinterpret_cast<float*>(sm + OFF_SMALL + SM_P);
   float* s_m = reinterpret_cast<float*>(sm + OFF_SMALL + SM_M);
   float* s_h = reinterpret_cast<float*>(sm + OFF_SMALL + SM_H);
+  float* s_hx = reinterpret_cast<float*>(sm + OFF_SMALL + SM_HX);
   float* s_af = reinterpret_cast<float*>(sm + OFF_AF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + OFF_SMALL + SM_BAR);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(sm + OFF_SMALL + SM_TMEM);
@@ -128,7 +131,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qd = warp & 3, gp = warp >> 2;
   const int row = qd * 32 + lane;             // TMEM lane owned by the thread
-  const int pair = blockIdx.x, b = pair / a.H, h = pair - b * a.H;
+  // dv = 256: a cluster of two CTAs per pair, each with 128 value rows (the
+  // rows of S evolve independently given the chunk's key-side quantities,
+  // which both CTAs form); they exchange their halves of U_down m per chunk
+  const bool dv2 = a.DV == 2 * kDV;
+  const int vh = dv2 ? (int)(blockIdx.x & 1) : 0;
+  const int DVt = a.DV, v0 = kDV * vh;        // tensors' value width; first row here
+  const int pair = dv2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int b = pair / a.H, h = pair - b * a.H;
   const int T = a.T, H = a.H, R = a.R, NB = a.NB;
   const int bpc = a.L / kBlk;
   const size_t SZ = (size_t)kDV * kDK;
@@ -154,6 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (dv2) cluster_sync();  // both CTAs' barriers exist before any remote arrive
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);  // lane base
@@ -181,7 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int i = 0; i < 8; ++i)
       ud_r[i] = (r < R) ? __bfloat162float(
-                              ud[((size_t)h * R + r) * kDV + part + 16 * i])
+                              ud[((size_t)h * R + r) * DVt + v0 + part + 16 * i])
                         : 0.f;
     for (int e = tid; e < kRMax * kDK; e += kThreads) {
       const int r2 = e / kDK, jj = e - r2 * kDK;
@@ -210,12 +221,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (part == 0) s_h[r] = acc;
     }
     __syncthreads();
+    const float* hv = s_h;
+    if (dv2) {
+      // send this CTA's half of h to the other CTA's slot, arrive on its
+      // barrier; wait for the other half in our slot and add (double
+      // buffered by chunk parity: a slot is rewritten only after its reader
+      // arrived on the writer's barrier for the next chunk)
+      float* slot = s_hx + 32 * (c & 1);
+      if (tid == 0) {
+        const uint32_t peer = (uint32_t)(vh ^ 1);
+        const uint32_t dst = cluster_map(slot, peer);
+#pragma unroll 1
+        for (int r = 0; r < 32; ++r) st_cluster_f32(dst + 4 * r, s_h[r]);
+        mbar_arrive_remote(cluster_map(bars + B_X, peer));
+      }
+      wait(B_X, 20);
+      fence_acquire_cluster();
+      if (tid < 32) slot[tid] += s_h[tid];
+      __syncthreads();
+      hv = slot;
+    }
     {  // p_j: four threads per channel j = tid / 4, 8 ranks each
       const int jj = tid >> 2, rq = tid & 3;
       float acc = 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        acc = fmaf(__bfloat162float(s_uu[(8 * rq + i) * kDK + jj]), s_h[8 * rq + i], acc);
+        acc = fmaf(__bfloat162float(s_uu[(8 * rq + i) * kDK + jj]), hv[8 * rq + i], acc);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       if (rq == 0) {
@@ -231,8 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto issue_vgb = [&](int ib) {
     const int tok = b * T + ib * kBlk;
     mbar_expect_tx(bars + B_VGB, 3 * 16384);
-    tma_load_3d(sm + OFF_RV, &tm_v, bars + B_VGB, 0, h, tok);
-    tma_load_3d(sm + OFF_RV + 8192, &tm_v, bars + B_VGB, 64, h, tok);
+    tma_load_3d(sm + OFF_RV, &tm_v, bars + B_VGB, v0, h, tok);
+    tma_load_3d(sm + OFF_RV + 8192, &tm_v, bars + B_VGB, v0 + 64, h, tok);
     tma_load_3d(sm + OFF_RG, &tm_g, bars + B_VGB, 0, h, tok);
     tma_load_3d(sm + OFF_RG + 8192, &tm_g, bars + B_VGB, 64, h, tok);
     tma_load_3d(sm + OFF_RB, &tm_bx, bars + B_VGB, 0, h, tok);
@@ -252,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- initial state: S0 -> TMEM (fp32) and the bf16 operand copy
   {
     const int c0 = gp * 32;
-    const float* s0 = a.S0 ? a.S0 + (size_t)pair * SZ + (size_t)row * kDK + c0
+    const float* s0 = a.S0 ? a.S0 + ((size_t)pair * DVt + v0 + row) * kDK + c0
                            : nullptr;
     float vals[32];
 #pragma unroll
@@ -269,7 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   float* s_mq = s_af;  // [4][128] partial sums of m (A buffer is free then)
   if (tid < 128) {
-    const float m0 = a.m0 ? a.m0[(size_t)pair * kDV + tid] : 0.f;
+    const float m0 = a.m0 ? a.m0[(size_t)pair * DVt + v0 + tid] : 0.f;
     s_m[tid] = m0;
     s_mq[tid] = m0;
     s_mq[128 + tid] = s_mq[256 + tid] = s_mq[384 + tid] = 0.f;
@@ -528,12 +559,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       float vals[32];
       tmem_ld16x2(tl + TM_D1 + 64 + gp * 16, tl + TM_S + gp * 32 + 16, vals);
-      __nv_bfloat16* orow = o + ((size_t)b * T + t0 + gp * 16) * H * kDV +
-                            (size_t)h * kDV + row;
+      __nv_bfloat16* orow = o + ((size_t)b * T + t0 + gp * 16) * H * DVt +
+                            (size_t)h * DVt + v0 + row;
 #pragma unroll
       for (int e = 0; e < 16; ++e) {
         msum += vals[e];
-        orow[(size_t)e * H * kDV] = __float2bfloat16_rn(vals[e]);
+        orow[(size_t)e * H * DVt] = __float2bfloat16_rn(vals[e]);
       }
       float sv[32];
       tmem_ld16(tl + TM_S + gp * 32, sv);
@@ -557,7 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             (size_t)row * kDK + c0
                       : nullptr;
       float* st = (a.S_T && ib == NB - 1)
-                      ? a.S_T + (size_t)pair * SZ + (size_t)row * kDK + c0
+                      ? a.S_T + ((size_t)pair * DVt + v0 + row) * kDK + c0
                       : nullptr;
       if (ck) {
 #pragma unroll
@@ -596,11 +627,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) tc::drain_bar(bars + i, (npar >> i) & 1u);
   } else if (a.m_T && tid < 128) {
-    a.m_T[(size_t)pair * kDV + tid] = s_m[tid];
+    a.m_T[(size_t)pair * DVt + v0 + tid] = s_m[tid];
   }
   if ((tid == 0 || tid == 256) && a.tc_rec) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
+  // neither CTA of a pair leaves while the other may still write to it
+  if (dv2) cluster_sync();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
@@ -637,19 +670,41 @@ bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows) {
 
 }  // namespace
 
-bool tc_fwd_supported(const carve_shape& s) { return tc_shape(s); }
+bool tc_fwd_supported(const carve_shape& s, bool training) {
+  return tc_fwd_shape(s, training);
+}
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mg, mb;
   const long long rows = (long long)a.B * a.T;
+  const bool dv2 = a.DV == 2 * kDV;
+  if (dv2 && (a.ck_S || a.tc_rec)) return cudaErrorInvalidValue;  // inference only
   if (!make_map(&mq, a.q, kDK, a.H, rows) || !make_map(&mk, a.k, kDK, a.H, rows) ||
-      !make_map(&mv, a.v, kDV, a.H, rows) || !make_map(&mg, a.g, kDK, a.H, rows) ||
+      !make_map(&mv, a.v, a.DV, a.H, rows) || !make_map(&mg, a.g, kDK, a.H, rows) ||
       !make_map(&mb, a.bx, kDK, a.H, rows))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(
       fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  fwd_tc_kernel<<<a.B * a.H, kThreads, kSmemBytes, st>>>(a, mq, mk, mv, mg, mb);
+  if (!dv2) {
+    fwd_tc_kernel<<<a.B * a.H, kThreads, kSmemBytes, st>>>(a, mq, mk, mv, mg, mb);
+    return cudaGetLastError();
+  }
+  // dv = 256: clusters of two CTAs, one per value half
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * a.B * a.H);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, fwd_tc_kernel, a, mq, mk, mv, mg, mb);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

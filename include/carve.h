@@ -59,6 +59,10 @@ typedef enum { CARVE_BF16 = 0, CARVE_FP32 = 1 } carve_dtype;
  * Supported: B, H >= 1; T >= 0 with T % L == 0; DK, DV multiples of 16 in
  * [16, 256]; 0 <= R <= 64; L in [1, 64] or a multiple of 64 up to 256.
  * Anything else returns CARVE_ERR_UNSUPPORTED.
+ * Kernel families: bf16 with DK = 128, L a multiple of 64, R <= 32, T > 0
+ * runs on the tensor cores for DV = 128 (forward, training forward and
+ * backward) and DV = 256 (forward without training); every other shape,
+ * and fp32 inputs, on the generic CUDA-core kernels.
  */
 typedef struct {
   int32_t B, T, H, DK, DV, R, L;
@@ -187,9 +191,9 @@ carve_status carve_reset_status(void* workspace, void* stream);
 /* Static, human-readable name of a status code. */
 const char* carve_status_str(carve_status status);
 
-/* Name of the kernel family carve_chunk_fwd would use for this shape
- * ("tc" for the tcgen05 path, "generic" otherwise), or NULL if
- * unsupported. */
+/* Name of the kernel family carve_chunk_fwd with training = 0 would use
+ * for this shape ("tc" for the tcgen05 path, "generic" otherwise), or NULL
+ * if unsupported. */
 const char* carve_fwd_path(const carve_shape* shape);
 
 #ifdef __cplusplus

@@ -216,6 +216,35 @@ def test_tensor_core_forward_matches_oracle_and_generic(case, monkeypatch):
     assert _rel(m_tc.cpu(), m_g.cpu()) < 1e-2
 
 
+TC_DV256_CASES = [
+    # B, H, T, R, L  (dv = 256: a cluster of two CTAs per (b, h))
+    (1, 1, 64, 32, 64),
+    (1, 2, 320, 32, 64),
+    (2, 1, 256, 16, 128),
+]
+
+
+@pytest.mark.parametrize("case", TC_DV256_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_tensor_core_forward_dv256_matches_oracle_and_generic(case, monkeypatch):
+    B, H, T, R, L = case
+    cfg = dict(B=B, H=H, T=T, DK=128, DV=256, R=R, L=L)
+    inp = inputs(cfg, 41, torch.bfloat16)
+    if R > 0:  # a gate the value halves really have to share
+        inp["u_down"] = (inp["u_down"].float() * 25).to(torch.bfloat16)
+        inp["u_up"] = (inp["u_up"].float() * 25).to(torch.bfloat16)
+    _rand_state(inp, 42)
+    shape = carve.make_shape(B, T, H, 128, 256, R, L, torch.bfloat16)
+    assert carve.fwd_path(shape) == "tc"
+    assert_within(fwd_errors(inp, L), 1e-2, "tensor-core fwd, dv = 256")
+    _, o_tc, S_tc, m_tc, _ = run_fwd(inp, L)
+    monkeypatch.setenv("CARVE_FWD_PATH", "generic")
+    _, o_g, S_g, m_g, _ = run_fwd(inp, L)
+    from _parity import rel as _rel
+    assert _rel(o_tc.float().cpu(), o_g.float().cpu()) < 1e-2
+    assert _rel(S_tc.cpu(), S_g.cpu()) < 1e-2
+    assert _rel(m_tc.cpu(), m_g.cpu()) < 1e-2
+
+
 BWD_CASES = [
     # B, H, T, R, L
     (1, 1, 128, 32, 64),
