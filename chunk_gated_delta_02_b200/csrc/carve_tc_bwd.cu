@@ -50,8 +50,7 @@ constexpr int kDV = 128;
 // be 1024-aligned, which the kernel checks).  Tiles are 128-byte swizzled
 // 64-column blocks of `rows` x 128 B, the UMMA canonical layout.
 constexpr uint32_t R_X = 0;          // [K~; Q~]                        32 KB
-constexpr uint32_t R_KH = 32768;     // K^                              16 KB
-constexpr uint32_t R_KP = 49152;     // kap^                            16 KB
+constexpr uint32_t R_KHP = 32768;    // [K^; kap^] 2 blk x 128 rows     32 KB
 constexpr uint32_t R_ET = 65536;     // E^T (forward record)            16 KB
 constexpr uint32_t R_W = 81920;      // raw v -> W = w V                16 KB
 constexpr uint32_t R_RO = 98304;     // [dE -> dR ; dO]                 32 KB
@@ -96,6 +95,7 @@ constexpr uint32_t T_D8 = T_G2;
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t ID_KK64 = idesc_bf16(128, 64, false, false);
+constexpr uint32_t ID_KK128 = idesc_bf16(128, 128, false, false);
 constexpr uint32_t ID_KM64 = idesc_bf16(128, 64, false, true);
 constexpr uint32_t ID_MK64 = idesc_bf16(128, 64, true, false);
 constexpr uint32_t ID_MK128 = idesc_bf16(128, 128, true, false);
@@ -349,6 +349,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     issue_pre(NB - 1);
   }
 
+  // w_t of the two token rows a thread of warps 8-15 scales in W = w V,
+  // fetched one block ahead into registers
+  float w_lo = 0.f, w_hi = 0.f;
+  if (warp >= 8) {
+    const size_t r0 = (size_t)b * T + (NB - 1) * kBlk + ((tid - 256) >> 3);
+    w_lo = __bfloat162float(w_in[r0 * H + h]);
+    w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+  }
   float dp_acc = 0.f;   // dp_j share (channel row, this warp's token quarter)
   float p_next = tid < 128 ? a.gin[((size_t)pair * NC + NC - 1) * GR + tid] : 0.f;
   for (int ib = NB - 1; ib >= 0; --ib) {
@@ -381,13 +389,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
     if (chunk_first && ib > 0 && tid < 128)  // the next block starts chunk c - 1
       p_next = a.gin[((size_t)pair * NC + c - 1) * GR + tid];
-    // w_t of the two token rows a thread of warps 8-15 scales in W = w V
-    float w_lo = 0.f, w_hi = 0.f;
-    if (warp >= 8) {
-      const size_t r0 = (size_t)tok + ((tid - 256) >> 3);
-      w_lo = __bfloat162float(w_in[r0 * H + h]);
-      w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
-    }
     wait(B_SB, 10);
     wait(B_PRE, 11);
     wait(B_IN, 12);
@@ -397,9 +398,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      dO = d_o + dm / L meanwhile); s_x is cleared: it accumulates
     //      dlog gamma next
     if (warp < 8) {
-      tc::transform_block<8>(sm + R_X, sm + R_KH, sm + R_KP, sm + R_DSB,
+      tc::transform_block<8>(sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB,
                              sm + R_DSB + 16384, s_p, s_gam,
-                             reinterpret_cast<float*>(sm + R_MP), 3);
+                             reinterpret_cast<float*>(sm + R_MP), 3, 16384);
       if (tid < 128) s_x[tid] = 0.f;
     } else {
       const float invL = 1.0f / (float)a.L;
@@ -443,24 +444,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(sm + R_RO + off) = y;
         }
       }
+      if (ib > 0) {  // the next block's w_t
+        const size_t r0 = (size_t)b * T + (ib - 1) * kBlk + ((tid - 256) >> 3);
+        w_lo = __bfloat162float(w_in[r0 * H + h]);
+        w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+      }
     }
     fence_async_smem();
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- S3: G = X [kap^ | K^]^T
+    // ---- S3: G = X [K^; kap^]^T (one N = 128 product per k-step):
+    //      columns 0-63 [M; P_k], 64-127 [A; P_kap]
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t x0 = smem_u32(sm + R_X), kp0 = smem_u32(sm + R_KP);
-      const uint32_t kh0 = smem_u32(sm + R_KH);
+      const uint32_t x0 = smem_u32(sm + R_X), khp0 = smem_u32(sm + R_KHP);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-        const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
         umma_bf16(tmem + T_G, desc_kmajor_sw128(x0 + kx),
-                  desc_kmajor_sw128(kp0 + k64), ID_KK64, ks > 0);
-        umma_bf16(tmem + T_G + 64, desc_kmajor_sw128(x0 + kx),
-                  desc_kmajor_sw128(kh0 + k64), ID_KK64, ks > 0);
+                  desc_kmajor_sw128(khp0 + kx), ID_KK128, ks > 0);
       }
       umma_commit(bars + B_1);
       mark(B_1);
@@ -493,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (mp || row >= 64) {
         const int piece = gp & 1;
         float vals[32];
-        tmem_ld32(tl + T_G + (mp ? 64 : 0) + piece * 32, vals);
+        tmem_ld32(tl + T_G + (mp ? 0 : 64) + piece * 32, vals);
 #pragma unroll
         for (int e = 0; e < 32; ++e)
           if (piece * 32 + e >= gr) vals[e] = 0.f;
@@ -519,13 +522,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- S6: dE^T = -dS~ kap^T - dO^T P_kap
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t dsb0 = smem_u32(sm + R_DSB), kp0 = smem_u32(sm + R_KP);
+      const uint32_t dsb0 = smem_u32(sm + R_DSB), kp0 = smem_u32(sm + R_KHP) + 8192;
       const uint32_t ro0 = smem_u32(sm + R_RO), pq0 = smem_u32(sm + R_PQ);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks)
         umma_bf16(tmem + T_DER,
                   desc_kmajor_sw128(dsb0 + (ks >> 2) * 16384 + (ks & 3) * 32),
-                  desc_kmajor_sw128(kp0 + (ks >> 2) * 8192 + (ks & 3) * 32),
+                  desc_kmajor_sw128(kp0 + (ks >> 2) * 16384 + (ks & 3) * 32),
                   ID_KK64_NA, ks > 0);
 #pragma unroll 1
       for (int ks = 0; ks < 4; ++ks)
@@ -584,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t ro0 = smem_u32(sm + R_RO), et0 = smem_u32(sm + R_ET);
       const uint32_t w0 = smem_u32(sm + R_W), dsb0 = smem_u32(sm + R_DSB);
-      const uint32_t kh0 = smem_u32(sm + R_KH), mp0 = smem_u32(sm + R_MP);
+      const uint32_t kh0 = smem_u32(sm + R_KHP), mp0 = smem_u32(sm + R_MP);
       const uint32_t x0 = smem_u32(sm + R_X), sb0 = smem_u32(sm + R_SB);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
@@ -595,7 +598,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_G2 + 64, desc_kmajor_sw128(ro0 + kx),
                   desc_kmajor_sw128(w0 + k64), ID_KK64, ks > 0);
         umma_bf16(tmem + T_RE, desc_kmajor_sw128(dsb0 + kx),
-                  desc_kmajor_sw128(kh0 + k64), ID_KK64, ks > 0);
+                  desc_kmajor_sw128(kh0 + kx), ID_KK64, ks > 0);
         umma_bf16(tmem + T_G, desc_mnmajor_sw128(sb0 + ks * 2048, 16384),
                   desc_kmajor_sw128(ro0 + kx), ID_MK128, ks > 0);
       }
@@ -638,7 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      block's state record, still in SB)
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t kp0 = smem_u32(sm + R_KP), kh0 = smem_u32(sm + R_KH);
+      const uint32_t kh0 = smem_u32(sm + R_KHP), kp0 = kh0 + 8192;
       const uint32_t mp0 = smem_u32(sm + R_MP), pq0 = smem_u32(sm + R_PQ);
       const uint32_t x0 = smem_u32(sm + R_X), dsb0 = smem_u32(sm + R_DSB);
       const uint32_t et0 = smem_u32(sm + R_ET), w0 = smem_u32(sm + R_W);
@@ -646,7 +649,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t a0 = (ks < 4 ? kp0 : kh0) + (ks & 3) * 2048;
         const uint32_t g2 = (ks < 4 ? mp0 : pq0) + (ks & 3) * 32;
-        umma_bf16(tmem + T_G, desc_mnmajor_sw128(a0, 8192),
+        umma_bf16(tmem + T_G, desc_mnmajor_sw128(a0, 16384),
                   desc_kmajor_sw128(g2), ks < 4 ? ID_MK128_NA : ID_MK128, 1);
       }
 #pragma unroll 1
@@ -744,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float gam = __expf(G), igam = __fdividef(1.0f, gam);
           const float bb = sigm(ldbf(sm + R_RO + 16384 + o64) + pj);
           const float qt = ldbf(sm + R_X + sw128_off(64 + t, jj, 128));
-          const float kh = ldbf(sm + R_KH + o64);
+          const float kh = ldbf(sm + R_KHP + sw128_off(t, jj, 128));
           const float kt = kh * gam * gam;  // K~ = K^ Gamma^2
           const float kp = bb * kh;         // kap^ = b K^
           const float dKt = dd[e], dQt = dd[8 + e], dKp = -dd[16 + e], dKh = dd[24 + e];

@@ -54,8 +54,7 @@ constexpr int kRMax = 32;  // rank of U_b held in registers
 // shared memory map (bytes from a 1024-aligned base); 128-byte swizzled
 // tiles are 64-column blocks of `rows` x 128 B.
 constexpr uint32_t OFF_X = 0;          // [K~; Q~]   2 blk x 128 rows  32 KB
-constexpr uint32_t OFF_KH = 32768;     // K^         2 blk x  64 rows  16 KB
-constexpr uint32_t OFF_KP = 49152;     // kap^       2 blk x  64 rows  16 KB
+constexpr uint32_t OFF_KHP = 32768;    // [K^; kap^] 2 blk x 128 rows  32 KB
 constexpr uint32_t OFF_W = 65536;      // w V        2 blk x  64 rows  16 KB
 constexpr uint32_t OFF_MY = 81920;     // [M;P_k] then Y, 128 rows     16 KB
 constexpr uint32_t OFF_RE = 98304;     // R^T then -E^T, 128 rows      16 KB
@@ -93,8 +92,8 @@ constexpr int kNumBars = 8;
 // TMEM columns (fp32, lanes = rows)
 constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
 constexpr uint32_t TM_D1 = 128;  // [R|..] -> [E|O]  [v][n]     128 cols
-constexpr uint32_t TM_GK = 256;  // [A; P_kap]       [i][t]      64 cols
-constexpr uint32_t TM_GM = 320;  // [M; P_k]         [i][t]      64 cols
+constexpr uint32_t TM_GM = 256;  // [M; P_k]         [i][t]      64 cols
+constexpr uint32_t TM_GK = 320;  // [A; P_kap]       [i][t]      64 cols
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, false);
@@ -317,6 +316,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
 
+  // w_t of the two token rows a thread of warps 8-15 scales in W = w V,
+  // fetched one block ahead into registers
+  float w_lo = 0.f, w_hi = 0.f;
+  if (warp >= 8) {
+    const size_t r0 = (size_t)b * T + ((tid - 256) >> 3);
+    w_lo = __bfloat162float(w_in[r0 * H + h]);
+    w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+  }
   float msum = 0.f;  // this thread's token quarter of the chunk's sum of o, row `row`
   for (int ib = 0; ib < NB; ++ib) {
     const int t0 = ib * kBlk;
@@ -331,21 +338,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_store(rec + kTcRecS, sm + OFF_SB, 32768);
       bulk_commit();
     }
-    // w_t of the two token rows a thread of warps 8-15 scales in W = w V
-    float w_lo = 0.f, w_hi = 0.f;
-    if (warp >= 8) {
-      const size_t r0 = (size_t)b * T + t0 + ((tid - 256) >> 3);
-      w_lo = __bfloat162float(w_in[r0 * H + h]);
-      w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
-    }
     wait(B_VGB, 1);
     wait(B_KQ, 2);
 
     // ---- 2. transform: decay scan, gated and decayed operands, W = w V
     //      (warps 0-7 the key side, warps 8-15 W = w V meanwhile)
     if (warp < 8) {
-      tc::transform_block<8>(sm + OFF_X, sm + OFF_KH, sm + OFF_KP, sm + OFF_RG,
-                             sm + OFF_RB, s_p, s_gam, s_af, 3);
+      tc::transform_block<8>(sm + OFF_X, sm + OFF_KHP, sm + OFF_KHP + 8192,
+                             sm + OFF_RG, sm + OFF_RB, s_p, s_gam, s_af, 3,
+                             16384);
     } else {
       const int u = tid - 256;
       const int rr = u >> 3, ch = u & 7;  // token rows rr, rr + 32; 16-byte chunk
@@ -366,6 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
       }
+      if (ib + 1 < NB) {  // the next block's w_t
+        const size_t r0 = (size_t)b * T + (ib + 1) * kBlk + ((tid - 256) >> 3);
+        w_lo = __bfloat162float(w_in[r0 * H + h]);
+        w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+      }
     }
     fence_async_smem();
     if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
@@ -376,16 +382,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0) {
       if (ib + 1 < NB) issue_vgb(ib + 1);
       tc_fence_after();
-      const uint32_t x0 = smem_u32(sm + OFF_X), kp0 = smem_u32(sm + OFF_KP);
-      const uint32_t kh0 = smem_u32(sm + OFF_KH), sb0 = smem_u32(sm + OFF_SB);
+      const uint32_t x0 = smem_u32(sm + OFF_X), khp0 = smem_u32(sm + OFF_KHP);
+      const uint32_t sb0 = smem_u32(sm + OFF_SB);
+      // G = [K~; Q~] [K^; kap^]^T in one N = 128 product per k-step:
+      // columns 0-63 [M; P_k], 64-127 [A; P_kap]
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-        const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
-        umma_bf16(tmem + TM_GK, desc_kmajor_sw128(x0 + kx),
-                  desc_kmajor_sw128(kp0 + k64), ID_N64, ks > 0);
         umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
-                  desc_kmajor_sw128(kh0 + k64), ID_N64, ks > 0);
+                  desc_kmajor_sw128(khp0 + kx), ID_N128, ks > 0);
       }
       umma_commit(bars + B_M1);
       mark(B_M1);
@@ -535,17 +540,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         bulk_commit();
       }
       tc_fence_after();
-      const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KH);
-      const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = smem_u32(sm + OFF_KP);
+      const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KHP);
+      const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = kh0 + 8192;
       const uint32_t pq0 = smem_u32(pq);
 #pragma unroll 1
       for (int ks = 0; ks < 4; ++ks) {
         umma_bf16(tmem + TM_D1 + 64, desc_kmajor_sw128(re0 + ks * 32),
                   desc_kmajor_sw128(pq0 + ks * 32), ID_N64_NA, 1);
         umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
-                  desc_mnmajor_sw128(kh0 + ks * 2048, 8192), ID_AMN_BMN, 1);
+                  desc_mnmajor_sw128(kh0 + ks * 2048, 16384), ID_AMN_BMN, 1);
         umma_bf16(tmem + TM_S, desc_kmajor_sw128(re0 + ks * 32),
-                  desc_mnmajor_sw128(kp0 + ks * 2048, 8192), ID_BMN_NA, 1);
+                  desc_mnmajor_sw128(kp0 + ks * 2048, 16384), ID_BMN_NA, 1);
       }
       umma_commit(bars + B_M4);
       mark(B_M4);

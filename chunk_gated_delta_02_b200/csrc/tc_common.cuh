@@ -60,7 +60,7 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* p, float* x) {
 // All tiles are 128-byte swizzled 64-column blocks.  `x` holds [K; Q]
 // (128 rows per column block; rewritten in place to [K~; Q~]), `graw` and
 // `braw` raw g and b_x (64 rows per column block), `kh`, `kp` receive K^ and
-// kap^, `s_gam` gamma.  `s_p` holds p_j = (U_b m_c)_j; `red` is NW * 64
+// kap^ (64 rows per column block, blocks `khs` bytes apart), `s_gam` gamma.  `s_p` holds p_j = (U_b m_c)_j; `red` is NW * 64
 // floats of scratch.  Called by NW warps: half of them per column block;
 // thread (chunk of 8 channels, group of TPT = 128 / (4 NW) consecutive
 // tokens) touches one 16-byte chunk per row, the 8 threads of a
@@ -74,7 +74,8 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
                                                 const uint8_t* graw,
                                                 const uint8_t* braw,
                                                 const float* s_p, float* s_gam,
-                                                float* red, int bar_id) {
+                                                float* red, int bar_id,
+                                                uint32_t khs = 8192) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
@@ -87,6 +88,9 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
   };
   auto off128 = [&](int t) {
     return (uint32_t)(blk * 16384 + t * 128 + ((ch ^ (t & 7)) << 4));
+  };
+  auto offk = [&](int t) {
+    return (uint32_t)(blk * khs + t * 128 + ((ch ^ (t & 7)) << 4));
   };
   float gl[TPT][8];  // inclusive log-decay sums inside the token group
 #pragma unroll
@@ -151,8 +155,8 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
     }
     st_chunk(x + off128(t), o_kt);
     st_chunk(x + off128(64 + t), o_qt);
-    st_chunk(kh + off64(t), o_kh);
-    st_chunk(kp + off64(t), o_kp);
+    st_chunk(kh + offk(t), o_kh);
+    st_chunk(kp + offk(t), o_kp);
   }
   if (tg == NG - 1) {  // gamma = Gamma_63
     *reinterpret_cast<float4*>(s_gam + j0) =
