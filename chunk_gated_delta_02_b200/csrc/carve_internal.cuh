@@ -26,9 +26,9 @@ constexpr uint32_t kWsMagicTc = 0xCA7E7C01u;  // tensor-core forward: tc records
 
 // Per-block record the tensor-core training forward leaves for the backward:
 // shared-memory images (128-byte swizzled UMMA layout of a 1024-aligned
-// base) of the bf16 state operand S, of E^T and of T = (I + A)^{-1}.
+// base) of the bf16 state operand S, of E and of T = (I + A)^{-1}.
 constexpr size_t kTcRecS = 0;          // S    [v 128][j 128] bf16  32 KB
-constexpr size_t kTcRecE = 32768;      // E^T  [v 128][t 64]  bf16  16 KB
+constexpr size_t kTcRecE = 32768;      // E    [t 64][v 128]  bf16  16 KB (2 x 8 KB column blocks)
 constexpr size_t kTcRecT = 49152;      // T    [t 64][s 64]   bf16   8 KB
 constexpr size_t kTcRecBytes = 57344;
 

@@ -5,7 +5,7 @@
 // walks the blocks of one (sequence, head) pair from last to first.  The
 // gradient of the block-end state, dS (dv x dk, fp32), lives in tensor
 // memory for the whole walk.  Per block the training forward left a record
-// (the bf16 state operand S, E^T and T = (I + A)^{-1}, as shared-memory
+// (the bf16 state operand S, E and T = (I + A)^{-1}, as shared-memory
 // images) and the chunk's gate vector p_c; the element-wise transform and
 // the Gram matrices are recomputed from the inputs.
 //
@@ -51,8 +51,7 @@ constexpr int kDV = 128;
 // 64-column blocks of `rows` x 128 B, the UMMA canonical layout.
 constexpr uint32_t R_X = 0;          // [K~; Q~]                        32 KB
 constexpr uint32_t R_KHP = 32768;    // [K^; kap^] 2 blk x 128 rows     32 KB
-constexpr uint32_t R_ET = 65536;     // E^T (forward record)            16 KB
-constexpr uint32_t R_W = 81920;      // raw v -> W = w V                16 KB
+constexpr uint32_t R_EW = 65536;     // [E (record); raw v -> W = w V]  32 KB
 constexpr uint32_t R_RO = 98304;     // [dE -> dR ; dO]                 32 KB
 constexpr uint32_t R_DSB = 131072;   // raw g, b_x | dS~ bf16           32 KB
 constexpr uint32_t R_SB = 163840;    // S bf16 (record) | raw g, b_x    32 KB
@@ -82,7 +81,7 @@ constexpr int B_3 = 4;     // MMA S6
 constexpr int B_4 = 5;     // MMA S7
 constexpr int B_5 = 6;     // MMA S9
 constexpr int B_7 = 7;     // MMA S11
-constexpr int B_PRE = 8;   // v, g, b_x, E^T and T records
+constexpr int B_PRE = 8;   // v, g, b_x, E and T records
 constexpr int kNumBars = 9;
 
 // TMEM columns
@@ -96,8 +95,6 @@ constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t ID_KK64 = idesc_bf16(128, 64, false, false);
 constexpr uint32_t ID_KK128 = idesc_bf16(128, 128, false, false);
-constexpr uint32_t ID_KM64 = idesc_bf16(128, 64, false, true);
-constexpr uint32_t ID_MK64 = idesc_bf16(128, 64, true, false);
 constexpr uint32_t ID_MK128 = idesc_bf16(128, 128, true, false);
 constexpr uint32_t ID_MM64 = idesc_bf16(128, 64, true, true);
 constexpr uint32_t ID_MM128 = idesc_bf16(128, 128, true, true);
@@ -319,18 +316,20 @@ __global__ void __launch_bounds__(kThreads, 1)
               bars + B_SB);
     mark(B_SB);
   };
-  // v -> W; g, b_x -> DSB; records E^T -> ET, T -> TT
+  // v -> W (rows 64.. of EW); g, b_x -> DSB; records E -> rows 0..63 of EW,
+  // T -> TT
   auto issue_pre = [&](int blk) {
     const int tk = tok_of(blk);
     const uint8_t* r = rec0 + (size_t)blk * kTcRecBytes;
     mbar_expect_tx(bars + B_PRE, 4 * 16384 + 8192);
-    tma_load_3d(sm + R_W, &tm_v, bars + B_PRE, 0, h, tk);
-    tma_load_3d(sm + R_W + 8192, &tm_v, bars + B_PRE, 64, h, tk);
+    tma_load_3d(sm + R_EW + 8192, &tm_v, bars + B_PRE, 0, h, tk);
+    tma_load_3d(sm + R_EW + 24576, &tm_v, bars + B_PRE, 64, h, tk);
     tma_load_3d(sm + R_DSB, &tm_g, bars + B_PRE, 0, h, tk);
     tma_load_3d(sm + R_DSB + 8192, &tm_g, bars + B_PRE, 64, h, tk);
     tma_load_3d(sm + R_DSB + 16384, &tm_bx, bars + B_PRE, 0, h, tk);
     tma_load_3d(sm + R_DSB + 24576, &tm_bx, bars + B_PRE, 64, h, tk);
-    bulk_load(sm + R_ET, r + kTcRecE, 16384, bars + B_PRE);
+    bulk_load(sm + R_EW, r + kTcRecE, 8192, bars + B_PRE);
+    bulk_load(sm + R_EW + 16384, r + kTcRecE + 8192, 8192, bars + B_PRE);
     bulk_load(sm + R_TT, r + kTcRecT, 8192, bars + B_PRE);
     mark(B_PRE);
   };
@@ -410,10 +409,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < 4; ++i) {
         const int r = rr + 32 * (i & 1), kb = i >> 1;
         const uint32_t sub = (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ch * 16);
-        // W = w V in place
+        // W = w V in place (rows 64.. of EW)
         {
-          const uint32_t off = (uint32_t)(kb * 8192) + sub;
-          const uint4 x = *reinterpret_cast<const uint4*>(sm + R_W + off);
+          const uint32_t off = (uint32_t)(kb * 16384 + 8192) + sub;
+          const uint4 x = *reinterpret_cast<const uint4*>(sm + R_EW + off);
           const float wt = (i & 1) ? w_hi : w_lo;
           const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
           uint4 y;
@@ -423,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2 f = __bfloat1622float2(xv[e]);
             yv[e] = pack2(f.x * wt, f.y * wt);
           }
-          *reinterpret_cast<uint4*>(sm + R_W + off) = y;
+          *reinterpret_cast<uint4*>(sm + R_EW + off) = y;
         }
         // dO = d_o + dm / L (rows 64.. of RO); logical column of the chunk
         {
@@ -585,18 +584,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      D7^T = S^T [dR; dO]^T
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t ro0 = smem_u32(sm + R_RO), et0 = smem_u32(sm + R_ET);
-      const uint32_t w0 = smem_u32(sm + R_W), dsb0 = smem_u32(sm + R_DSB);
+      const uint32_t ro0 = smem_u32(sm + R_RO), ew0 = smem_u32(sm + R_EW);
+      const uint32_t dsb0 = smem_u32(sm + R_DSB);
       const uint32_t kh0 = smem_u32(sm + R_KHP), mp0 = smem_u32(sm + R_MP);
       const uint32_t x0 = smem_u32(sm + R_X), sb0 = smem_u32(sm + R_SB);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-        const uint32_t k64 = (ks >> 2) * 8192 + (ks & 3) * 32;
         umma_bf16(tmem + T_G2, desc_kmajor_sw128(ro0 + kx),
-                  desc_mnmajor_sw128(et0 + ks * 2048, 16384), ID_KM64, ks > 0);
-        umma_bf16(tmem + T_G2 + 64, desc_kmajor_sw128(ro0 + kx),
-                  desc_kmajor_sw128(w0 + k64), ID_KK64, ks > 0);
+                  desc_kmajor_sw128(ew0 + kx), ID_KK128, ks > 0);
         umma_bf16(tmem + T_RE, desc_kmajor_sw128(dsb0 + kx),
                   desc_kmajor_sw128(kh0 + kx), ID_KK64, ks > 0);
         umma_bf16(tmem + T_G, desc_mnmajor_sw128(sb0 + ks * 2048, 16384),
@@ -644,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t kh0 = smem_u32(sm + R_KHP), kp0 = kh0 + 8192;
       const uint32_t mp0 = smem_u32(sm + R_MP), pq0 = smem_u32(sm + R_PQ);
       const uint32_t x0 = smem_u32(sm + R_X), dsb0 = smem_u32(sm + R_DSB);
-      const uint32_t et0 = smem_u32(sm + R_ET), w0 = smem_u32(sm + R_W);
+      const uint32_t ew0 = smem_u32(sm + R_EW);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t a0 = (ks < 4 ? kp0 : kh0) + (ks & 3) * 2048;
@@ -657,10 +653,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_D8, desc_mnmajor_sw128(x0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(mp0 + ks * 2048, 16384), ID_MM128, ks > 0);
         umma_bf16(tmem + T_D8, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
-                  desc_mnmajor_sw128(et0 + ks * 2048, 16384), ID_MM64, 1);
-        umma_bf16(tmem + T_D8 + 64, desc_mnmajor_sw128(dsb0 + ks * 2048, 16384),
-                  desc_kmajor_sw128(w0 + (ks >> 2) * 8192 + (ks & 3) * 32),
-                  ID_MK64, 1);
+                  desc_kmajor_sw128(ew0 + (ks >> 2) * 16384 + (ks & 3) * 32),
+                  ID_MK128, 1);
       }
       umma_commit(bars + B_7);
       mark(B_7);
@@ -686,7 +680,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < 16; ++e) {
         const int t = gp * 16 + e;
         dvrow[(size_t)e * H * kDV] = __float2bfloat16_rn(s_w[t] * dwv[e]);
-        dwv[e] *= ldbf(sm + R_W + sw128_off(t, row, 64));
+        dwv[e] *= ldbf(sm + R_EW + sw128_off(64 + t, row, 128));
       }
       const float sdw = warp_reduce_scatter16(dwv, lane);
       if (lane < 16) atomicAdd(&s_dw[gp * 16 + lane], sdw);
@@ -701,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // block ib - 1's state operand -> SB (read above)
     if (tid == 0 && ib > 0 && !*s_abort) issue_sb(ib - 1);
     wait(B_7, 17);
-    // block ib - 1's v, g, b_x, E^T, T into the buffers S11 released
+    // block ib - 1's v, g, b_x, E, T into the buffers S11 released
     if (tid == 0 && ib > 0 && !*s_abort) issue_pre(ib - 1);
     wait(B_GB, 18);
     tc_fence_after();

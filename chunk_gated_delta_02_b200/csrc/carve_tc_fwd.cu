@@ -73,8 +73,9 @@ constexpr uint32_t SM_BAR = 2560;      // kNumBars mbarriers
 constexpr uint32_t SM_TMEM = 2624;     // TMEM base address
 constexpr uint32_t SM_ABORT = 2628;    // abort flag
 constexpr uint32_t kSmallBytes = 2688;
-constexpr uint32_t OFF_UU = 215808;    // U_up^T bf16 [kRMax][128]      8 KB
-constexpr uint32_t kSmemBytes = OFF_UU + 8192 + 1024;
+constexpr uint32_t OFF_UU = 215808;    // U_up^T bf16 [kRMax][kUuLd]   8.5 KB
+constexpr int kUuLd = 128 + 8;         // row pitch: 16 B of padding per row
+constexpr uint32_t kSmemBytes = OFF_UU + kRMax * kUuLd * 2 + 1024;
 static_assert(OFF_SMALL + kSmallBytes <= OFF_UU, "shared memory map overlap");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
 
@@ -94,6 +95,7 @@ constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
 constexpr uint32_t TM_D1 = 128;  // [R|..] -> [E|O]  [v][n]     128 cols
 constexpr uint32_t TM_GM = 256;  // [M; P_k]         [i][t]      64 cols
 constexpr uint32_t TM_GK = 320;  // [A; P_kap]       [i][t]      64 cols
+constexpr uint32_t TM_E = 384;   // E = T R (training) [t][v], lanes 0-63  128 cols
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t ID_N64 = idesc_bf16(128, 64, false, false);
@@ -183,7 +185,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // U_b factors: thread (r = tid / 16, part = tid % 16) holds U_down[h][r]
   // [part + 16 i], i < 8, in registers (lanes read consecutive m values);
-  // U_up[h] is kept transposed in shared memory (s_uu[r][j], zero for r >= R).
+  // U_up[h] is kept transposed in shared memory (s_uu[r][j], zero for r >= R;
+  // rows kUuLd apart so that the four rows a warp reads hit different banks).
   float ud_r[8];
   __nv_bfloat16* s_uu = reinterpret_cast<__nv_bfloat16*>(sm + OFF_UU);
   {
@@ -195,8 +198,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         : 0.f;
     for (int e = tid; e < kRMax * kDK; e += kThreads) {
       const int r2 = e / kDK, jj = e - r2 * kDK;
-      s_uu[e] = (r2 < R) ? uu[((size_t)h * kDK + jj) * R + r2]
-                         : __float2bfloat16_rn(0.f);
+      s_uu[r2 * kUuLd + jj] = (r2 < R) ? uu[((size_t)h * kDK + jj) * R + r2]
+                                       : __float2bfloat16_rn(0.f);
     }
   }
 
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc = 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        acc = fmaf(__bfloat162float(s_uu[(8 * rq + i) * kDK + jj]), hv[8 * rq + i], acc);
+        acc = fmaf(__bfloat162float(s_uu[(8 * rq + i) * kUuLd + jj]), hv[8 * rq + i], acc);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       if (rq == 0) {
@@ -297,7 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       st_chunk(sm + OFF_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
                vals + c8 * 8);
   }
-  float* s_mq = s_af;  // [4][128] partial sums of m (A buffer is free then)
+  // [4][128] partial sums of m: in the R^T / E^T buffer, free once MMA 4
+  // retired (the A buffer holds the E record meanwhile)
+  float* s_mq = reinterpret_cast<float*>(sm + OFF_RE);
   if (tid < 128) {
     const float m0 = a.m0 ? a.m0[(size_t)pair * DVt + v0 + tid] : 0.f;
     s_m[tid] = m0;
@@ -501,14 +506,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- 5. MMA 3a: E^T = R^T T^T
+    // ---- 5. MMA 3a: E^T = R^T T^T; training also E = T R (lanes 0-63; the
+    //         rows of MY past T only feed the unused lanes) for the record
     if (tid == 0) {
       tc_fence_after();
       const uint32_t re0 = smem_u32(sm + OFF_RE), my0 = smem_u32(sm + OFF_MY);
 #pragma unroll 1
-      for (int ks = 0; ks < 4; ++ks)
+      for (int ks = 0; ks < 4; ++ks) {
         umma_bf16(tmem + TM_D1, desc_kmajor_sw128(re0 + ks * 32),
                   desc_kmajor_sw128(my0 + ks * 32), ID_N64, ks > 0);
+        if (rec)
+          umma_bf16(tmem + TM_E, desc_kmajor_sw128(my0 + ks * 32),
+                    desc_kmajor_sw128(re0 + ks * 32), ID_N128, ks > 0);
+      }
       umma_commit(bars + B_M3);
       mark(B_M3);
       if (rec) {
@@ -528,6 +538,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         st_chunk(sm + OFF_RE + sw128_chunk(row, 0, gp * 4 + c8, 128),
                  vals + c8 * 8);
       fence_async_smem();
+    } else if (rec && qd < 2) {
+      // E [t][v] (K-major, the backward's operand layout) -> the A buffer,
+      // 64 value columns per warp
+#pragma unroll 1
+      for (int pc = 2 * (gp - 2); pc < 2 * (gp - 2) + 2; ++pc) {
+        float vals[32];
+        tmem_ld32(tl + TM_E + pc * 32, vals);
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_AF + sw128_chunk(row, pc >> 1, (pc & 1) * 4 + c8, 64),
+                   vals + c8 * 8);
+      }
+      fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
@@ -536,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S += W^T K^ - E^T kap^
     if (tid == 0) {
       if (rec) {
-        bulk_store(rec + kTcRecE, sm + OFF_RE, 16384);
+        bulk_store(rec + kTcRecE, sm + OFF_AF, 16384);
         bulk_commit();
       }
       tc_fence_after();
