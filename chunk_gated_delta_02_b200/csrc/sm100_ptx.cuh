@@ -53,6 +53,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
       "r"(smem_u32(bar))
       : "memory");
 }
+// 3-D tiled store from shared memory, tracked by the issuing thread's bulk
+// groups (bulk_commit / bulk_wait_*).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map,
+                                             const void* src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], "
+      "[%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 // Prefetch a 3-D tile (same box as the loads) into L2 only.
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0,
                                                 int c1, int c2) {
