@@ -73,7 +73,7 @@ static_assert(R_SM + 2688 <= kSmemBytes, "small region");
 static_assert(R_PQ == R_MP + 16384 && R_TT == R_PQ + 8192, "G2 blocks");
 
 // mbarriers (index into the small region's array)
-constexpr int B_IN = 0;    // k, q, d_o of this block
+constexpr int B_IN = 0;    // q, d_o of this block
 constexpr int B_GB = 1;    // raw g, b_x again for the epilogue
 constexpr int B_1 = 2;     // MMA S3
 constexpr int B_SB = 3;    // bf16 state record
@@ -300,9 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // k, q -> X; d_o -> RO rows 64..127
   auto issue_top = [&](int blk) {
     const int tk = tok_of(blk);
-    mbar_expect_tx(bars + B_IN, 3 * 16384);
-    tma_load_3d(sm + R_X, &tm_k, bars + B_IN, 0, h, tk);
-    tma_load_3d(sm + R_X + 16384, &tm_k, bars + B_IN, 64, h, tk);
+    mbar_expect_tx(bars + B_IN, 2 * 16384);
     tma_load_3d(sm + R_X + 8192, &tm_q, bars + B_IN, 0, h, tk);
     tma_load_3d(sm + R_X + 24576, &tm_q, bars + B_IN, 64, h, tk);
     tma_load_3d(sm + R_RO + 8192, &tm_do, bars + B_IN, 0, h, tk);
@@ -316,12 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               bars + B_SB);
     mark(B_SB);
   };
-  // v -> W (rows 64.. of EW); g, b_x -> DSB; records E -> rows 0..63 of EW,
-  // T -> TT
+  // k -> X rows 0..63; v -> W (rows 64.. of EW); g, b_x -> DSB; records
+  // E -> rows 0..63 of EW, T -> TT
   auto issue_pre = [&](int blk) {
     const int tk = tok_of(blk);
     const uint8_t* r = rec0 + (size_t)blk * kTcRecBytes;
-    mbar_expect_tx(bars + B_PRE, 4 * 16384 + 8192);
+    mbar_expect_tx(bars + B_PRE, 5 * 16384 + 8192);
+    // k -> rows 0..63 of X: K~ is no longer read once the D7 / D8 MMAs
+    // retired (the epilogue takes K~ from K^)
+    tma_load_3d(sm + R_X, &tm_k, bars + B_PRE, 0, h, tk);
+    tma_load_3d(sm + R_X + 16384, &tm_k, bars + B_PRE, 64, h, tk);
     tma_load_3d(sm + R_EW + 8192, &tm_v, bars + B_PRE, 0, h, tk);
     tma_load_3d(sm + R_EW + 24576, &tm_v, bars + B_PRE, 64, h, tk);
     tma_load_3d(sm + R_DSB, &tm_g, bars + B_PRE, 0, h, tk);
@@ -373,8 +375,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       dp_acc = 0.f;
     }
 
-    // ---- S1: inputs.  k, q, d_o now; the rest was requested during the
-    //      previous block.  Block ib - 1's k, q, d_o tiles -> L2.
+    // ---- S1: inputs.  q, d_o now; the rest was requested during the
+    //      previous block.  Block ib - 1's q, d_o tiles -> L2 (and k, which
+    //      loads during this block).
     if (tid == 0) issue_top(ib);
     if (tid == 32 && ib > 0) {  // (the rest of block ib - 1 loads a block ahead)
       const int tn = tok - kBlk;

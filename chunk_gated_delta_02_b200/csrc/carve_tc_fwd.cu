@@ -203,8 +203,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // content gate of chunk c: s_p = U_up (U_down m); training records p_c
-  // and h_c = U_down m_c for the backward.  m_v = scale * (sum of the four
+  // content gate of chunk c: s_p = U_up (U_down m) (training records p_c,
+  // h_c = U_down m_c and m_c for the backward during the chunk's first block).  m_v = scale * (sum of the four
   // partial sums mq[q * 128 + v]), so the chunk mean needs no pass of its own.
   auto gate = [&](int c, const float* mq, float scale) {
     {
@@ -251,12 +251,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc = fmaf(__bfloat162float(s_uu[(8 * rq + i) * kUuLd + jj]), hv[8 * rq + i], acc);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if (rq == 0) {
-        s_p[jj] = acc;
-        if (a.gin) a.gin[((size_t)pair * a.NC + c) * (kDK + R) + jj] = acc;
-      }
-      if (a.gin && rq == 1 && jj < R)
-        a.gin[((size_t)pair * a.NC + c) * (kDK + R) + kDK + jj] = s_h[jj];
+      if (rq == 0) s_p[jj] = acc;
     }
     __syncthreads();
   };
@@ -312,7 +307,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tmem_st_wait();
   __syncthreads();
   gate(0, s_mq, 1.f);
-  if (a.ck_m && tid < 128) a.ck_m[(size_t)pair * a.NC * kDV + tid] = s_m[tid];
   if (tid == 0) {
     issue_vgb(0);
     issue_kq(0);
@@ -498,6 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
+    } else if (a.gin && ib % bpc == 0) {
+      // warps 12-15, idle here: the chunk's gate records for the backward
+      // (p_c, h_c, m_c: s_p, s_h, s_m hold them until the chunk's end)
+      const int u = tid - 384, c = ib / bpc;
+      a.gin[((size_t)pair * a.NC + c) * (kDK + R) + u] = s_p[u];
+      if (u < R) a.gin[((size_t)pair * a.NC + c) * (kDK + R) + kDK + u] = s_h[u];
+      if (a.ck_m) a.ck_m[((size_t)pair * a.NC + c) * kDV + u] = s_m[u];
     }
     // (warps 12-15 do not wait on MMA 2: they park at the barrier below
     // instead of polling while warps 0-3 solve)
@@ -640,10 +641,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // first GEMV; s_m keeps m for m_T and the checkpoint
       const float invL = 1.0f / (float)a.L;
       if (tid < 128) {
-        const float m = (s_mq[tid] + s_mq[128 + tid] + s_mq[256 + tid] + s_mq[384 + tid]) * invL;
-        s_m[tid] = m;
-        if (a.ck_m && ib + 1 < NB)
-          a.ck_m[((size_t)pair * a.NC + (ib + 1) / bpc) * kDV + tid] = m;
+        s_m[tid] = (s_mq[tid] + s_mq[128 + tid] + s_mq[256 + tid] + s_mq[384 + tid]) * invL;
       }
       msum = 0.f;
       if (ib + 1 < NB) gate((ib + 1) / bpc, s_mq, invL);

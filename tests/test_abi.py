@@ -66,6 +66,21 @@ def test_status_strings_and_path(lib):
         assert lib.carve_status_str(code).decode() == name
     assert lib.carve_fwd_path(ctypes.byref(shape())) is not None
     assert lib.carve_fwd_path(ctypes.byref(shape(DK=24))) is None
+    # kernel family selection (host logic only): tensor cores for bf16,
+    # DK = 128, L % 64 == 0, R <= 32 and DV = 128 or 256; generic otherwise
+    path = lambda **kw: lib.carve_fwd_path(ctypes.byref(shape(**kw))).decode()
+    tc = dict(DK=128, DV=128, R=32, L=64, T=128, dtype=carve.CARVE_BF16)
+    assert path(**tc) == "tc"
+    assert path(**dict(tc, DV=256)) == "tc"
+    assert path(**dict(tc, L=128)) == "tc"
+    for other in (dict(DV=64), dict(DK=64), dict(L=32), dict(R=48),
+                  dict(dtype=carve.CARVE_FP32), dict(DV=192)):
+        assert path(**dict(tc, **other)) == "generic", other
+    # training on the tensor-core family adds the per-block records
+    # (56 KiB per block and pair) on top of the fp32 checkpoints
+    B, H, NB = 2, 3, 128 // 64
+    extra = ws_bytes(lib, shape(**tc), 1) - ws_bytes(lib, shape(**tc), 0)
+    assert extra >= B * H * NB * 57344 + B * H * (NB + 1) * 128 * 128 * 4
 
 
 FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
