@@ -8,13 +8,15 @@
 // section 3, "Chunkability Boundary": erase on the key axis only, so one
 // triangular solve per block serves every value row):
 //
-//   transform   Gamma = exp(cumsum g), K~ = K Gamma, Q~ = Q Gamma_{t-1},
-//               K^ = K / Gamma, kap^ = sigmoid(bx + U_b m_c) K^, W = w V
-//               (section 2.3: key-axis decay; section 2.1: content gate)
-//   MMA 1       G = [K~; Q~] [kap^ | K^]^T   ->  [A | M ; P_kap | P_k]
-//               D1 = S [K~; Q~]^T             ->  [(K~ S^T)^T | (Q~ S^T)^T]
+//   keys        Gamma = exp(cumsum g), K~ = K Gamma, Q~ = Q Gamma_{t-1},
+//               K^ = K / Gamma (warps 0-7; section 2.3: key-axis decay)
+//   gate, W     first block of a chunk: p = U_up U_down m_c (section 2.1);
+//               W = w V (warps 8-15, meanwhile)
+//   MMA 1       D1 = S [K~; Q~]^T             ->  [(K~ S^T)^T | (Q~ S^T)^T]
+//               (issued while the other threads form kap^ = sigmoid(bx + p) K^)
+//               G = [K~; Q~] [K^; kap^]^T     ->  [M ; P_k | A ; P_kap]
 //   MMA 2       D1 += W^T [M; P_k]^T          ->  [R^T | (Q~ S^T + P_k W)^T]
-//   solve       T = (I + A)^{-1} by 16 x 16 blocks (warps 0-3, tf32)
+//   solve       T = (I + A)^{-1} by 16 x 16 blocks (warps 0-3)
 //   MMA 3a      E^T = R^T T^T                 (E = T R, the WY pseudo-values)
 //   MMA 3b      D1[O] -= E^T P_kap^T          ->  O^T = (Q~ S^T + P_k W - P_kap E)^T
 //   MMA 4       S += W^T K^ - E^T kap^ ;  S <- S Diag(gamma)
@@ -25,10 +27,10 @@
 // Raw input tiles arrive by TMA (128-byte swizzle) into buffers whose layout
 // is exactly the UMMA canonical layout, so the element-wise transform writes
 // operands at the offsets it reads them from.  The next block's v, g, b_x
-// tiles are requested right after the transform, its k, q tiles as soon as
-// MMA 1 has released their buffer.  In training mode the block's bf16 S
-// operand, E^T and T go to the workspace by bulk copies (the backward's
-// records); of the fp32 states only the final one is kept.
+// tiles are requested once kap^ is formed, its k, q tiles as soon as MMA 1
+// has released their buffer.  In training mode the block's bf16 S operand,
+// E and T go to the workspace by bulk copies (the backward's records); of
+// the fp32 states only the final one is kept.
 #include <cudaTypedefs.h>
 
 #include "carve_internal.cuh"
@@ -86,9 +88,8 @@ constexpr int B_M1 = 2;    // MMA 1 (Grams, S X^T)
 constexpr int B_M2 = 3;    // MMA 2 (W^T [M;P_k]^T)
 constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
 constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
-constexpr int B_D1 = 6;    // MMA 1, second half (S X^T)
-constexpr int B_X = 7;     // dv = 256: the other CTA's half of U_down m arrived
-constexpr int kNumBars = 8;
+constexpr int B_X = 6;     // dv = 256: the other CTA's half of U_down m arrived
+constexpr int kNumBars = 7;
 
 // TMEM columns (fp32, lanes = rows)
 constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
@@ -108,7 +109,8 @@ constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false
 
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
 // rows 32 qd .. 32 qd + 31) and column group gp = w / 4.  Warps 0-3 also
-// run the triangular solve while warps 4-11 prepare [M; P_k] and R^T.
+// run the triangular solve while warps 4-11 prepare [M; P_k] and R^T; warps
+// 8-15 form the gate and W while warps 0-7 run the key-side transform.
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -183,19 +185,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   auto mark = [&](int i) { pend |= 1u << i; };
 
-  // U_b factors: thread (r = tid / 16, part = tid % 16) holds U_down[h][r]
-  // [part + 16 i], i < 8, in registers (lanes read consecutive m values);
-  // U_up[h] is kept transposed in shared memory (s_uu[r][j], zero for r >= R;
-  // rows kUuLd apart so that the four rows a warp reads hit different banks).
-  float ud_r[8];
+  // U_b factors: thread u = tid - 256 of warps 8-15 (r = u / 8, part = u % 8)
+  // holds U_down[h][r][part + 8 i], i < 16, in registers as bf16 pairs
+  // (i = 2 n, 2 n + 1 in ud_p[n]; lanes read consecutive m values); U_up[h]
+  // is kept transposed in shared memory (s_uu[r][j], zero for r >= R; rows
+  // kUuLd apart so that rows 4 apart fall in different banks).
+  uint32_t ud_p[8];
   __nv_bfloat16* s_uu = reinterpret_cast<__nv_bfloat16*>(sm + OFF_UU);
   {
-    const int r = tid >> 4, part = tid & 15;
+    const int r = (tid & 255) >> 3, part = tid & 7;
+    const unsigned short* udr = reinterpret_cast<const unsigned short*>(ud) +
+                                ((size_t)h * R + r) * DVt + v0 + part;
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
-      ud_r[i] = (r < R) ? __bfloat162float(
-                              ud[((size_t)h * R + r) * DVt + v0 + part + 16 * i])
-                        : 0.f;
+    for (int n = 0; n < 8; ++n)
+      ud_p[n] = (warp >= 8 && r < R)
+                    ? (uint32_t)udr[16 * n] | ((uint32_t)udr[16 * n + 8] << 16)
+                    : 0u;
     for (int e = tid; e < kRMax * kDK; e += kThreads) {
       const int r2 = e / kDK, jj = e - r2 * kDK;
       s_uu[r2 * kUuLd + jj] = (r2 < R) ? uu[((size_t)h * kDK + jj) * R + r2]
@@ -203,26 +208,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // content gate of chunk c: s_p = U_up (U_down m) (training records p_c,
-  // h_c = U_down m_c and m_c for the backward during the chunk's first block).  m_v = scale * (sum of the four
-  // partial sums mq[q * 128 + v]), so the chunk mean needs no pass of its own.
-  auto gate = [&](int c, const float* mq, float scale) {
+  // content gate of chunk c, on warps 8-15 (u = tid - 256): m_c = the mean
+  // of the previous chunk's o from its four token-quarter partial sums
+  // (m_0 is set up front), h = U_down m_c, s_p = U_up h.  Training records
+  // p_c, h_c and m_c for the backward during the chunk's first block.
+  const float invL = 1.0f / (float)a.L;
+  float* s_mq = reinterpret_cast<float*>(sm + OFF_RE);  // [4][128] partial sums of m
+  auto gate = [&](int c) {
+    const int u = tid - 256;
+    if (c > 0 && u < 128)
+      s_m[u] = ((s_mq[u] + s_mq[128 + u]) + (s_mq[256 + u] + s_mq[384 + u])) * invL;
+    bar_named(6, 256);
     {
-      const int r = tid >> 4, part = tid & 15;
+      const int r = u >> 3, part = u & 7;
       float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int v = part + 16 * i;
-        acc = fmaf(ud_r[i], (mq[v] + mq[128 + v]) + (mq[256 + v] + mq[384 + v]), acc);
+      for (int n = 0; n < 8; ++n) {
+        acc = fmaf(__uint_as_float(ud_p[n] << 16), s_m[part + 16 * n], acc);
+        acc = fmaf(__uint_as_float(ud_p[n] & 0xffff0000u), s_m[part + 16 * n + 8], acc);
       }
-      acc *= scale;
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 8);
       if (part == 0) s_h[r] = acc;
     }
-    __syncthreads();
+    bar_named(6, 256);
     const float* hv = s_h;
     if (dv2) {
       // send this CTA's half of h to the other CTA's slot, arrive on its
@@ -230,7 +240,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // buffered by chunk parity: a slot is rewritten only after its reader
       // arrived on the writer's barrier for the next chunk)
       float* slot = s_hx + 32 * (c & 1);
-      if (tid == 0) {
+      if (u == 0) {
         const uint32_t peer = (uint32_t)(vh ^ 1);
         const uint32_t dst = cluster_map(slot, peer);
 #pragma unroll 1
@@ -239,21 +249,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait(B_X, 20);
       fence_acquire_cluster();
-      if (tid < 32) slot[tid] += s_h[tid];
-      __syncthreads();
+      if (u < 32) slot[u] += s_h[u];
+      bar_named(6, 256);
       hv = slot;
     }
-    {  // p_j: four threads per channel j = tid / 4, 8 ranks each
-      const int jj = tid >> 2, rq = tid & 3;
+    {  // p_j: two threads per channel j = u / 2, 16 ranks each (rank sets
+       // 4 apart, so the pair reads U_up rows in different banks)
+      const int jj = u >> 1, rq = u & 1;
       float acc = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        acc = fmaf(__bfloat162float(s_uu[(8 * rq + i) * kUuLd + jj]), hv[8 * rq + i], acc);
+      for (int i = 0; i < 16; ++i) {
+        const int r = (i & 3) + 8 * (i >> 2) + 4 * rq;
+        acc = fmaf(__bfloat162float(s_uu[r * kUuLd + jj]), hv[r], acc);
+      }
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       if (rq == 0) s_p[jj] = acc;
     }
-    __syncthreads();
   };
 
   auto issue_vgb = [&](int ib) {
@@ -295,33 +306,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       st_chunk(sm + OFF_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
                vals + c8 * 8);
   }
-  // [4][128] partial sums of m: in the R^T / E^T buffer, free once MMA 4
-  // retired (the A buffer holds the E record meanwhile)
-  float* s_mq = reinterpret_cast<float*>(sm + OFF_RE);
-  if (tid < 128) {
-    const float m0 = a.m0 ? a.m0[(size_t)pair * DVt + v0 + tid] : 0.f;
-    s_m[tid] = m0;
-    s_mq[tid] = m0;
-    s_mq[128 + tid] = s_mq[256 + tid] = s_mq[384 + tid] = 0.f;
-  }
-  tmem_st_wait();
-  __syncthreads();
-  gate(0, s_mq, 1.f);
+  if (tid < 128) s_m[tid] = a.m0 ? a.m0[(size_t)pair * DVt + v0 + tid] : 0.f;
   if (tid == 0) {
     issue_vgb(0);
     issue_kq(0);
   }
-  fence_async_smem();
+  tmem_st_wait();
   tc_fence_before();
   __syncthreads();
 
   // w_t of the two token rows a thread of warps 8-15 scales in W = w V,
-  // fetched one block ahead into registers
-  float w_lo = 0.f, w_hi = 0.f;
+  // fetched one block ahead into registers (raw bf16 bits: converted only
+  // when used, so the loads' latency is not waited for at issue)
+  const unsigned short* w_bits = reinterpret_cast<const unsigned short*>(w_in);
+  uint32_t w_lo = 0, w_hi = 0;
   if (warp >= 8) {
     const size_t r0 = (size_t)b * T + ((tid - 256) >> 3);
-    w_lo = __bfloat162float(w_in[r0 * H + h]);
-    w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+    w_lo = w_bits[r0 * H + h];
+    w_hi = w_bits[(r0 + 32) * H + h];
   }
   float msum = 0.f;  // this thread's token quarter of the chunk's sum of o, row `row`
   for (int ib = 0; ib < NB; ++ib) {
@@ -330,23 +332,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* rec = a.tc_rec ? a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes
                             : nullptr;
 
-    // ---- 1. inputs of this block (block ib + 2's tiles -> L2 ahead of
-    //         their loads, which are issued during block ib + 1); training
-    //         records the block's bf16 state operand
-    if (tid == 256 && rec) {  // (a warp of the light half of the transform)
+    // ---- 1. training records the block's bf16 state operand
+    if (tid == 256 && rec) {  // (warps 8-15 have the lighter share below)
       bulk_store(rec + kTcRecS, sm + OFF_SB, 32768);
       bulk_commit();
     }
-    wait(B_VGB, 1);
-    wait(B_KQ, 2);
 
-    // ---- 2. transform: decay scan, gated and decayed operands, W = w V
-    //      (warps 0-7 the key side, warps 8-15 W = w V meanwhile)
+    // ---- 2. key side of the transform (warps 0-7): decay scan, K~, Q~, K^;
+    //      meanwhile warps 8-15 form the chunk's gate p (first block of a
+    //      chunk) and W = w V
     if (warp < 8) {
-      tc::transform_block<8>(sm + OFF_X, sm + OFF_KHP, sm + OFF_KHP + 8192,
-                             sm + OFF_RG, sm + OFF_RB, s_p, s_gam, s_af, 3,
-                             16384);
+      wait(B_VGB, 1);
+      wait(B_KQ, 2);
+      tc::transform_keys<8>(sm + OFF_X, sm + OFF_KHP, sm + OFF_RG, s_gam, s_af,
+                            3, 16384);
     } else {
+      if (ib % bpc == 0) gate(ib / bpc);
+      wait(B_VGB, 1);
       const int u = tid - 256;
       const int rr = u >> 3, ch = u & 7;  // token rows rr, rr + 32; 16-byte chunk
 #pragma unroll
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t off = (uint32_t)(kb * 8192 + (r >> 3) * 1024 +
                                         (r & 7) * 128 + ch * 16);
         const uint4 x = *reinterpret_cast<const uint4*>(sm + OFF_RV + off);
-        const float wt = (i & 1) ? w_hi : w_lo;
+        const float wt = __uint_as_float(((i & 1) ? w_hi : w_lo) << 16);
         const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
         uint4 y;
         uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
@@ -368,23 +370,39 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ib + 1 < NB) {  // the next block's w_t
         const size_t r0 = (size_t)b * T + (ib + 1) * kBlk + ((tid - 256) >> 3);
-        w_lo = __bfloat162float(w_in[r0 * H + h]);
-        w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+        w_lo = w_bits[r0 * H + h];
+        w_hi = w_bits[(r0 + 32) * H + h];
       }
+    }
+    fence_async_smem();
+    __syncthreads();
+    if (*s_abort) break;
+
+    // ---- 3. D1 = S [K~; Q~]^T is issued while the other warps form
+    //      kap^ = sigmoid(b_x + p) K^; then G = [K~; Q~] [K^; kap^]^T in one
+    //      N = 128 product per k-step (columns 0-63 [M; P_k], 64-127
+    //      [A; P_kap]).  The commit after G covers D1 as well.
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t x0 = smem_u32(sm + OFF_X), sb0 = smem_u32(sm + OFF_SB);
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+        umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
+                  desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
+      }
+    } else if (tid >= 32) {
+      tc::kappa_block(sm + OFF_KHP, sm + OFF_KHP + 8192, sm + OFF_RB, s_p,
+                      16384, tid - 32, kThreads - 32);
     }
     fence_async_smem();
     if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
     __syncthreads();
     if (*s_abort) break;
-
-    // ---- 3. MMA 1; the raw v, g, b_x buffers are free for the next block
-    if (tid == 0) {
+    if (tid == 0) {  // the raw v, g, b_x buffers are free for the next block
       if (ib + 1 < NB) issue_vgb(ib + 1);
       tc_fence_after();
       const uint32_t x0 = smem_u32(sm + OFF_X), khp0 = smem_u32(sm + OFF_KHP);
-      const uint32_t sb0 = smem_u32(sm + OFF_SB);
-      // G = [K~; Q~] [K^; kap^]^T in one N = 128 product per k-step:
-      // columns 0-63 [M; P_k], 64-127 [A; P_kap]
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
@@ -393,14 +411,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(bars + B_M1);
       mark(B_M1);
-#pragma unroll 1
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-        umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
-                  desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
-      }
-      umma_commit(bars + B_D1);
-      mark(B_D1);
     }
     wait(B_M1, 3);
     tc_fence_after();
@@ -412,9 +422,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* pq = sm + OFF_SB + 24576;
     if (gp == 0) {
       // ---- 4a. [A; P_kap] (strictly lower): A -> fp32 for the inversion,
-      //          P_kap -> bf16 operand; T = (I + A)^{-1} (warps 0-3).  The
-      //          second half of MMA 1 still reads SB: P_kap and the solve's
-      //          scratch go there only once it retired.
+      //          P_kap -> bf16 operand; T = (I + A)^{-1} (warps 0-3)
 #pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         float vals[32];
@@ -428,13 +436,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             *reinterpret_cast<float4*>(s_af + fsw(row, part * 32 + e)) =
                 make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
         } else {
-          if (part == 0) wait(B_D1, 10);
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8)
             st_chunk(pq + sw128_chunk(gr, 0, part * 4 + c8, 64), vals + c8 * 8);
         }
       }
-      if (row < 64) wait(B_D1, 10);
       bar_named(2, 128);
       unit_lower_inverse64(s_af, s_tf, s_tf + 4096, 2);
       wait(B_M2, 5);  // [M; P_k] consumed: T may take its place
@@ -471,8 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       bar_named(1, 256);
       if (tid == 128 && !*s_abort) {
-        wait(B_D1, 9);  // S X^T retired: X is free for the next block's k, q
-        if (ib + 1 < NB) issue_kq(ib + 1);
+        if (ib + 1 < NB) issue_kq(ib + 1);  // MMA 1 retired: X is free
         tc_fence_after();
         const uint32_t w0 = smem_u32(sm + OFF_W), my0 = smem_u32(sm + OFF_MY);
 #pragma unroll 1
@@ -636,24 +641,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 0 && rec) bulk_wait_read_all();  // T, E^T records read
     tc_fence_before();
     __syncthreads();
-    if (chunk_end) {
-      // m = chunk mean of o: the quarter sums are folded into the gate's
-      // first GEMV; s_m keeps m for m_T and the checkpoint
-      const float invL = 1.0f / (float)a.L;
-      if (tid < 128) {
-        s_m[tid] = (s_mq[tid] + s_mq[128 + tid] + s_mq[256 + tid] + s_mq[384 + tid]) * invL;
-      }
-      msum = 0.f;
-      if (ib + 1 < NB) gate((ib + 1) / bpc, s_mq, invL);
-    }
+    if (chunk_end) msum = 0.f;
   }
 
   if (*s_abort) {
     if (tid == 0 || tid == 128)  // the threads that start copies and MMAs
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) tc::drain_bar(bars + i, (npar >> i) & 1u);
-  } else if (a.m_T && tid < 128) {
-    a.m_T[(size_t)pair * DVt + v0 + tid] = s_m[tid];
+  } else if (a.m_T && tid < 128) {  // the last chunk's mean
+    a.m_T[(size_t)pair * DVt + v0 + tid] =
+        ((s_mq[tid] + s_mq[128 + tid]) + (s_mq[256 + tid] + s_mq[384 + tid])) * invL;
   }
   if ((tid == 0 || tid == 256) && a.tc_rec) bulk_wait_all();
   tc_fence_before();

@@ -166,6 +166,116 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
   }
 }
 
+// The key side of transform_block (Gamma, K~, Q~, K^, gamma), without the
+// gate: kap^ = b K^ follows from kappa_block once p is known.
+template <int NW>
+__device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
+                                               const uint8_t* graw,
+                                               float* s_gam, float* red,
+                                               int bar_id, uint32_t khs) {
+  constexpr int WPB = NW / 2;         // warps per column block
+  constexpr int TPT = 64 / (4 * WPB); // tokens per thread
+  constexpr int NG = 64 / TPT;        // token groups
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int blk = warp / WPB, wq = warp % WPB, ch = lane & 7, t4 = lane >> 3;
+  const int tg = wq * 4 + t4;        // tokens TPT tg .. TPT tg + TPT - 1
+  const int j0 = blk * 64 + ch * 8;  // channels j0 .. j0 + 7
+  auto off64 = [&](int t) {
+    return (uint32_t)(blk * 8192 + t * 128 + ((ch ^ (t & 7)) << 4));
+  };
+  auto off128 = [&](int t) {
+    return (uint32_t)(blk * 16384 + t * 128 + ((ch ^ (t & 7)) << 4));
+  };
+  auto offk = [&](int t) {
+    return (uint32_t)(blk * khs + t * 128 + ((ch ^ (t & 7)) << 4));
+  };
+  float gl[TPT][8];  // inclusive log-decay sums inside the token group
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) {
+    float gv[8];
+    ld_chunk(graw + off64(TPT * tg + i), gv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
+  }
+  float ex[8];  // exclusive prefix of the token group
+  float wt[8];  // running inclusive sum over the warp's groups
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float tot = gl[TPT - 1][e];
+    float incl = tot;
+    float v = __shfl_up_sync(0xffffffffu, incl, 8);
+    if (t4 >= 1) incl += v;
+    v = __shfl_up_sync(0xffffffffu, incl, 16);
+    if (t4 >= 2) incl += v;
+    ex[e] = incl - tot;
+    wt[e] = incl;  // t4 == 3: the warp's total
+  }
+  if (t4 == 3) {
+    *reinterpret_cast<float4*>(red + wq * 128 + j0) =
+        make_float4(wt[0], wt[1], wt[2], wt[3]);
+    *reinterpret_cast<float4*>(red + wq * 128 + j0 + 4) =
+        make_float4(wt[4], wt[5], wt[6], wt[7]);
+  }
+  bar_named(bar_id + blk, WPB * 32);
+  for (int w2 = 0; w2 < wq; ++w2) {
+    const float4 a = *reinterpret_cast<const float4*>(red + w2 * 128 + j0);
+    const float4 b = *reinterpret_cast<const float4*>(red + w2 * 128 + j0 + 4);
+    ex[0] += a.x; ex[1] += a.y; ex[2] += a.z; ex[3] += a.w;
+    ex[4] += b.x; ex[5] += b.y; ex[6] += b.z; ex[7] += b.w;
+  }
+  float gprev[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) gprev[e] = __expf(ex[e]);  // Gamma_{TPT tg - 1}
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) {
+    const int t = TPT * tg + i;
+    float kv[8], qv[8], o_kt[8], o_qt[8], o_kh[8];
+    ld_chunk(x + off128(t), kv);
+    ld_chunk(x + off128(64 + t), qv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const float gam = __expf(ex[e] + gl[i][e]);
+      const float igam = __fdividef(1.0f, gam);
+      o_kt[e] = kv[e] * gam;
+      o_qt[e] = qv[e] * gprev[e];
+      o_kh[e] = kv[e] * igam;
+      gprev[e] = gam;
+    }
+    st_chunk(x + off128(t), o_kt);
+    st_chunk(x + off128(64 + t), o_qt);
+    st_chunk(kh + offk(t), o_kh);
+  }
+  if (tg == NG - 1) {  // gamma = Gamma_63
+    *reinterpret_cast<float4*>(s_gam + j0) =
+        make_float4(gprev[0], gprev[1], gprev[2], gprev[3]);
+    *reinterpret_cast<float4*>(s_gam + j0 + 4) =
+        make_float4(gprev[4], gprev[5], gprev[6], gprev[7]);
+  }
+}
+
+// kap^ = sigmoid(b_x + p) K^ for one block (the gate half of
+// transform_block), from the bf16 K^ already in shared memory: thread t_id of
+// n_thr takes 16-byte chunks t_id, t_id + n_thr, ... of the 64 x 128 tile;
+// the 8 threads of a quarter-warp take the 8 chunks of one row.
+__device__ __forceinline__ void kappa_block(const uint8_t* kh, uint8_t* kp,
+                                            const uint8_t* braw,
+                                            const float* s_p, uint32_t khs,
+                                            int t_id, int n_thr) {
+  for (int c = t_id; c < 1024; c += n_thr) {
+    const int t = c >> 4, blk = (c >> 3) & 1, ch = c & 7;
+    const uint32_t sw = (uint32_t)(t * 128 + ((ch ^ (t & 7)) << 4));
+    float kv[8], bv[8], o[8];
+    ld_chunk(kh + blk * khs + sw, kv);
+    ld_chunk(braw + blk * 8192 + sw, bv);
+    const float4 p0 = *reinterpret_cast<const float4*>(s_p + blk * 64 + ch * 8);
+    const float4 p1 = *reinterpret_cast<const float4*>(s_p + blk * 64 + ch * 8 + 4);
+    const float pj[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = sigm(bv[e] + pj[e]) * kv[e];
+    st_chunk(kp + blk * khs + sw, o);
+  }
+}
+
 constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
 
 // Bounded wait on an mbarrier phase.  On expiry: record CARVE_ERR_TIMEOUT
