@@ -351,12 +351,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // w_t of the two token rows a thread of warps 8-15 scales in W = w V,
-  // fetched one block ahead into registers
-  float w_lo = 0.f, w_hi = 0.f;
+  // fetched one block ahead into registers (raw bf16 bits: converted only
+  // when used, so the loads' latency is not waited for at issue)
+  const unsigned short* w_bits = reinterpret_cast<const unsigned short*>(w_in);
+  uint32_t w_lo = 0, w_hi = 0;
   if (warp >= 8) {
     const size_t r0 = (size_t)b * T + (NB - 1) * kBlk + ((tid - 256) >> 3);
-    w_lo = __bfloat162float(w_in[r0 * H + h]);
-    w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+    w_lo = w_bits[r0 * H + h];
+    w_hi = w_bits[(r0 + 32) * H + h];
   }
   float dp_acc = 0.f;   // dp_j share (channel row, this warp's token quarter)
   float p_next = tid < 128 ? a.gin[((size_t)pair * NC + NC - 1) * GR + tid] : 0.f;
@@ -416,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
           const uint32_t off = (uint32_t)(kb * 16384 + 8192) + sub;
           const uint4 x = *reinterpret_cast<const uint4*>(sm + R_EW + off);
-          const float wt = (i & 1) ? w_hi : w_lo;
+          const float wt = __uint_as_float(((i & 1) ? w_hi : w_lo) << 16);
           const __nv_bfloat162* xv = reinterpret_cast<const __nv_bfloat162*>(&x);
           uint4 y;
           uint32_t* yv = reinterpret_cast<uint32_t*>(&y);
@@ -448,8 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (ib > 0) {  // the next block's w_t
         const size_t r0 = (size_t)b * T + (ib - 1) * kBlk + ((tid - 256) >> 3);
-        w_lo = __bfloat162float(w_in[r0 * H + h]);
-        w_hi = __bfloat162float(w_in[(r0 + 32) * H + h]);
+        w_lo = w_bits[r0 * H + h];
+        w_hi = w_bits[(r0 + 32) * H + h];
       }
     }
     fence_async_smem();

@@ -66,18 +66,20 @@ constexpr uint32_t OFF_RG = 163840;    // raw g                        16 KB
 constexpr uint32_t OFF_RB = 180224;    // raw b_x                      16 KB
 constexpr uint32_t OFF_AF = 196608;    // A fp32 64 x 64 row-major     16 KB
 constexpr uint32_t OFF_SMALL = 212992;
-constexpr uint32_t SM_GAM = 0;         // gamma_j            128 f32
+constexpr uint32_t SM_GAM = 0;         // gamma_j (even blocks) 128 f32
 constexpr uint32_t SM_P = 512;         // (U_b m)_j          128 f32
 constexpr uint32_t SM_HX = 1024;       // the other CTA's half of U_down m, 2 x 32 f32
 constexpr uint32_t SM_M = 1280;        // m_v                128 f32
 constexpr uint32_t SM_H = 1792;        // U_down m            64 f32
+constexpr uint32_t SM_GAM1 = 2048;     // gamma_j (odd blocks)  128 f32
 constexpr uint32_t SM_BAR = 2560;      // kNumBars mbarriers
 constexpr uint32_t SM_TMEM = 2624;     // TMEM base address
 constexpr uint32_t SM_ABORT = 2628;    // abort flag
 constexpr uint32_t kSmallBytes = 2688;
 constexpr uint32_t OFF_UU = 215808;    // U_up^T bf16 [kRMax][kUuLd]   8.5 KB
 constexpr int kUuLd = 128 + 8;         // row pitch: 16 B of padding per row
-constexpr uint32_t kSmemBytes = OFF_UU + kRMax * kUuLd * 2 + 1024;
+constexpr uint32_t OFF_RED = OFF_UU + kRMax * kUuLd * 2;  // decay-scan scratch 2 KB
+constexpr uint32_t kSmemBytes = OFF_RED + 2048 + 1024;
 static_assert(OFF_SMALL + kSmallBytes <= OFF_UU, "shared memory map overlap");
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
 
@@ -107,6 +109,13 @@ constexpr uint32_t ID_N64_NA = idesc_bf16_neg(128, 64, false, false, true, false
 constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false);
 
 
+// Key side of one block's transform by warps 8-15 (one out-of-line copy of
+// the unrolled code serves the prologue and the block loop).
+static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* rg, float* gam,
+                                            float* red) {
+  tc::transform_keys<8>(x, rg, rg, gam, red, 3, 8192, 8);
+}
+
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
 // rows 32 qd .. 32 qd + 31) and column group gp = w / 4.  Warps 0-3 also
 // run the triangular solve while warps 4-11 prepare [M; P_k] and R^T; warps
@@ -120,7 +129,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float* s_gam = reinterpret_cast<float*>(sm + OFF_SMALL + SM_GAM);
+  float* s_gam0 = reinterpret_cast<float*>(sm + OFF_SMALL + SM_GAM);
+  float* s_gam1 = reinterpret_cast<float*>(sm + OFF_SMALL + SM_GAM1);
+  float* s_red = reinterpret_cast<float*>(sm + OFF_RED);
   float* s_p = reinterpret_cast<float*>(sm + OFF_SMALL + SM_P);
   float* s_m = reinterpret_cast<float*>(sm + OFF_SMALL + SM_M);
   float* s_h = reinterpret_cast<float*>(sm + OFF_SMALL + SM_H);
@@ -278,6 +289,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_load_3d(sm + OFF_RB + 8192, &tm_bx, bars + B_VGB, 64, h, tok);
     mark(B_VGB);
   };
+  // k, q, g of block ib -> L2 ahead of their loads
+  auto prefetch_kqg = [&](int ib) {
+    const int tok = b * T + ib * kBlk;
+#pragma unroll 1
+    for (int x = 0; x < kDK; x += 64) {
+      tma_prefetch_3d(&tm_k, x, h, tok);
+      tma_prefetch_3d(&tm_q, x, h, tok);
+      tma_prefetch_3d(&tm_g, x, h, tok);
+    }
+  };
   auto issue_kq = [&](int ib) {
     const int tok = b * T + ib * kBlk;
     mbar_expect_tx(bars + B_KQ, 2 * 16384);
@@ -286,6 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_load_3d(sm + OFF_X + 8192, &tm_q, bars + B_KQ, 0, h, tok);
     tma_load_3d(sm + OFF_X + 16384 + 8192, &tm_q, bars + B_KQ, 64, h, tok);
     mark(B_KQ);
+  };
+
+  // key side of block nb's transform (warps 8-15): K~, Q~ in place in X,
+  // K^ over the raw g tile (RG), gamma into its parity's buffer
+  auto keys = [&](int nb) {
+    wait(B_VGB, 1);
+    wait(B_KQ, 2);
+    keys_w8(sm + OFF_X, sm + OFF_RG, (nb & 1) ? s_gam1 : s_gam0, s_red);
   };
 
   // ---- initial state: S0 -> TMEM (fp32) and the bf16 operand copy
@@ -307,21 +336,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                vals + c8 * 8);
   }
   if (tid < 128) s_m[tid] = a.m0 ? a.m0[(size_t)pair * DVt + v0 + tid] : 0.f;
-  if (tid == 0) {
-    issue_vgb(0);
-    issue_kq(0);
-  }
+  if (tid == 0) issue_vgb(0);
+  if (tid == 256) issue_kq(0);
+  if (tid == 32 && NB > 1) prefetch_kqg(1);
   tmem_st_wait();
   tc_fence_before();
   __syncthreads();
+  if (warp >= 8) keys(0);
+  fence_async_smem();
+  __syncthreads();
 
-  // w_t of the two token rows a thread of warps 8-15 scales in W = w V,
+  // w_t of the two token rows a thread of warps 0-7 scales in W = w V,
   // fetched one block ahead into registers (raw bf16 bits: converted only
   // when used, so the loads' latency is not waited for at issue)
   const unsigned short* w_bits = reinterpret_cast<const unsigned short*>(w_in);
   uint32_t w_lo = 0, w_hi = 0;
-  if (warp >= 8) {
-    const size_t r0 = (size_t)b * T + ((tid - 256) >> 3);
+  if (warp < 8) {
+    const size_t r0 = (size_t)b * T + (tid >> 3);
     w_lo = w_bits[r0 * H + h];
     w_hi = w_bits[(r0 + 32) * H + h];
   }
@@ -332,25 +363,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* rec = a.tc_rec ? a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes
                             : nullptr;
 
-    // ---- 1. training records the block's bf16 state operand
-    if (tid == 256 && rec) {  // (warps 8-15 have the lighter share below)
+    float* s_gam = (ib & 1) ? s_gam1 : s_gam0;  // this block's gamma
+
+    // ---- 1. training records the block's bf16 state operand; block
+    //      ib + 2's k, q, g tiles -> L2
+    if (tid == 256 && rec) {
       bulk_store(rec + kTcRecS, sm + OFF_SB, 32768);
       bulk_commit();
     }
+    if (tid == 32 && ib + 2 < NB) prefetch_kqg(ib + 2);
 
-    // ---- 2. key side of the transform (warps 0-7): decay scan, K~, Q~, K^;
-    //      meanwhile warps 8-15 form the chunk's gate p (first block of a
-    //      chunk) and W = w V
+    // ---- 2. the key side (K~, Q~ in X; K^ in RG) was formed during the
+    //      previous block's solve.  D1 = S [K~; Q~]^T (issued by thread 0),
+    //      W = w V (warps 0-7); the chunk's gate p (warps 8-15, first block
+    //      of a chunk)
     if (warp < 8) {
+      if (tid == 0) {
+        tc_fence_after();
+        const uint32_t x0 = smem_u32(sm + OFF_X), sb0 = smem_u32(sm + OFF_SB);
+#pragma unroll 1
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+          umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
+                    desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
+        }
+      }
       wait(B_VGB, 1);
-      wait(B_KQ, 2);
-      tc::transform_keys<8>(sm + OFF_X, sm + OFF_KHP, sm + OFF_RG, s_gam, s_af,
-                            3, 16384);
-    } else {
-      if (ib % bpc == 0) gate(ib / bpc);
-      wait(B_VGB, 1);
-      const int u = tid - 256;
-      const int rr = u >> 3, ch = u & 7;  // token rows rr, rr + 32; 16-byte chunk
+      const int rr = tid >> 3, ch = tid & 7;  // token rows rr, rr + 32; 16-byte chunk
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = rr + 32 * (i & 1), kb = i >> 1;
@@ -369,32 +408,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
       }
       if (ib + 1 < NB) {  // the next block's w_t
-        const size_t r0 = (size_t)b * T + (ib + 1) * kBlk + ((tid - 256) >> 3);
+        const size_t r0 = (size_t)b * T + (ib + 1) * kBlk + (tid >> 3);
         w_lo = w_bits[r0 * H + h];
         w_hi = w_bits[(r0 + 32) * H + h];
       }
+    } else if (ib % bpc == 0) {
+      gate(ib / bpc);
     }
     fence_async_smem();
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- 3. D1 = S [K~; Q~]^T is issued while the other warps form
-    //      kap^ = sigmoid(b_x + p) K^; then G = [K~; Q~] [K^; kap^]^T in one
-    //      N = 128 product per k-step (columns 0-63 [M; P_k], 64-127
-    //      [A; P_kap]).  The commit after G covers D1 as well.
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t x0 = smem_u32(sm + OFF_X), sb0 = smem_u32(sm + OFF_SB);
-#pragma unroll 1
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-        umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
-                  desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
-      }
-    } else if (tid >= 32) {
-      tc::kappa_block(sm + OFF_KHP, sm + OFF_KHP + 8192, sm + OFF_RB, s_p,
-                      16384, tid - 32, kThreads - 32);
-    }
+    // ---- 3. K^ -> its operand slot and kap^ = sigmoid(b_x + p) K^; then
+    //      G = [K~; Q~] [K^; kap^]^T in one N = 128 product per k-step
+    //      (columns 0-63 [M; P_k], 64-127 [A; P_kap]).  The commit after G
+    //      covers D1 as well.
+    tc::kappa_block(sm + OFF_RG, sm + OFF_KHP, sm + OFF_KHP + 8192, sm + OFF_RB,
+                    s_p, 16384, tid, kThreads);
     fence_async_smem();
     if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
     __syncthreads();
@@ -414,6 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     wait(B_M1, 3);
     tc_fence_after();
+    // MMA 1 retired: X takes the next block's k, q
+    if (tid == 256 && ib + 1 < NB && !*s_abort) issue_kq(ib + 1);
 
     const int gr = row < 64 ? row : row - 64;  // token index of Gram row `row`
     // the bf16 S copy is dead until step 7: its buffer holds T (fp32),
@@ -477,7 +509,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       bar_named(1, 256);
       if (tid == 128 && !*s_abort) {
-        if (ib + 1 < NB) issue_kq(ib + 1);  // MMA 1 retired: X is free
         tc_fence_after();
         const uint32_t w0 = smem_u32(sm + OFF_W), my0 = smem_u32(sm + OFF_MY);
 #pragma unroll 1
@@ -498,15 +529,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                    vals + c8 * 8);
       }
     } else if (a.gin && ib % bpc == 0) {
-      // warps 12-15, idle here: the chunk's gate records for the backward
-      // (p_c, h_c, m_c: s_p, s_h, s_m hold them until the chunk's end)
+      // warps 12-15: the chunk's gate records for the backward (p_c, h_c,
+      // m_c: s_p, s_h, s_m hold them until the chunk's end)
       const int u = tid - 384, c = ib / bpc;
       a.gin[((size_t)pair * a.NC + c) * (kDK + R) + u] = s_p[u];
       if (u < R) a.gin[((size_t)pair * a.NC + c) * (kDK + R) + kDK + u] = s_h[u];
       if (a.ck_m) a.ck_m[((size_t)pair * a.NC + c) * kDV + u] = s_m[u];
     }
-    // (warps 12-15 do not wait on MMA 2: they park at the barrier below
-    // instead of polling while warps 0-3 solve)
+    // ---- 4c. warps 8-15, free while warps 0-3 solve: the key side of the
+    //          next block's transform (X and the raw g tile are free)
+    if (warp >= 8 && ib + 1 < NB) keys(ib + 1);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -645,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   if (*s_abort) {
-    if (tid == 0 || tid == 128)  // the threads that start copies and MMAs
+    if (tid == 0 || tid == 128 || tid == 256)  // the threads that start copies and MMAs
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) tc::drain_bar(bars + i, (npar >> i) & 1u);
   } else if (a.m_T && tid < 128) {  // the last chunk's mean

@@ -167,16 +167,20 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
 }
 
 // The key side of transform_block (Gamma, K~, Q~, K^, gamma), without the
-// gate: kap^ = b K^ follows from kappa_block once p is known.
+// gate: kap^ = b K^ follows from kappa_block once p is known.  Run by warps
+// wbase .. wbase + NW - 1.  With khs = 8192, K^ may overwrite the raw g
+// tile in place (kh == graw): each thread reads all its g chunks before it
+// writes K^ to the same offsets, and no other thread touches them.
 template <int NW>
 __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
                                                const uint8_t* graw,
                                                float* s_gam, float* red,
-                                               int bar_id, uint32_t khs) {
+                                               int bar_id, uint32_t khs,
+                                               int wbase) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int warp = (threadIdx.x >> 5) - wbase, lane = threadIdx.x & 31;
   const int blk = warp / WPB, wq = warp % WPB, ch = lane & 7, t4 = lane >> 3;
   const int tg = wq * 4 + t4;        // tokens TPT tg .. TPT tg + TPT - 1
   const int j0 = blk * 64 + ch * 8;  // channels j0 .. j0 + 7
@@ -254,24 +258,28 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
 }
 
 // kap^ = sigmoid(b_x + p) K^ for one block (the gate half of
-// transform_block), from the bf16 K^ already in shared memory: thread t_id of
-// n_thr takes 16-byte chunks t_id, t_id + n_thr, ... of the 64 x 128 tile;
-// the 8 threads of a quarter-warp take the 8 chunks of one row.
-__device__ __forceinline__ void kappa_block(const uint8_t* kh, uint8_t* kp,
-                                            const uint8_t* braw,
+// transform_block), from the bf16 K^ at `kh_src` (64-row column blocks
+// 8192 B apart); K^ is copied to `kh` and kap^ written to `kp` (column blocks
+// `khs` apart).  Thread t_id of n_thr takes 16-byte chunks t_id,
+// t_id + n_thr, ... of the 64 x 128 tile; the 8 threads of a quarter-warp
+// take the 8 chunks of one row (conflict-free under the swizzle).
+__device__ __forceinline__ void kappa_block(const uint8_t* kh_src, uint8_t* kh,
+                                            uint8_t* kp, const uint8_t* braw,
                                             const float* s_p, uint32_t khs,
                                             int t_id, int n_thr) {
   for (int c = t_id; c < 1024; c += n_thr) {
     const int t = c >> 4, blk = (c >> 3) & 1, ch = c & 7;
     const uint32_t sw = (uint32_t)(t * 128 + ((ch ^ (t & 7)) << 4));
+    const uint4 kraw = *reinterpret_cast<const uint4*>(kh_src + blk * 8192 + sw);
     float kv[8], bv[8], o[8];
-    ld_chunk(kh + blk * khs + sw, kv);
+    ld_chunk(kh_src + blk * 8192 + sw, kv);
     ld_chunk(braw + blk * 8192 + sw, bv);
     const float4 p0 = *reinterpret_cast<const float4*>(s_p + blk * 64 + ch * 8);
     const float4 p1 = *reinterpret_cast<const float4*>(s_p + blk * 64 + ch * 8 + 4);
     const float pj[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
 #pragma unroll
     for (int e = 0; e < 8; ++e) o[e] = sigm(bv[e] + pj[e]) * kv[e];
+    *reinterpret_cast<uint4*>(kh + blk * khs + sw) = kraw;
     st_chunk(kp + blk * khs + sw, o);
   }
 }
