@@ -398,17 +398,37 @@ __global__ void __launch_bounds__(kThreads, 1)
     wait(B_IN, 12);
     __syncthreads();  // s_p of S0
 
-    // ---- S2: transform (warps 0-7 the key side; warps 8-15 W = w V and
-    //      dO = d_o + dm / L meanwhile); s_x is cleared: it accumulates
-    //      dlog gamma next
+    // ---- S2: transform (warps 0-7 the key side; warps 8-15 first the gate
+    //      b = sigmoid(b_x + p) in fp16 over the raw b_x tile, handed to
+    //      warps 0-7 by named barrier 7, then W = w V and dO = d_o + dm / L);
+    //      s_x is cleared: it accumulates dlog gamma next
     if (warp < 8) {
       tc::transform_block<8>(sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB,
-                             sm + R_DSB + 16384, s_p, s_gam,
-                             reinterpret_cast<float*>(sm + R_MP), 3, 16384);
+                             sm + R_DSB + 16384, s_gam,
+                             reinterpret_cast<float*>(sm + R_MP), 3, 16384, 7,
+                             kThreads);
       if (tid < 128) s_x[tid] = 0.f;
     } else {
-      const float invL = 1.0f / (float)a.L;
       const int u = tid - 256;
+      // b: chunk c = u + 256 i of the 64 x 128 tile (row c / 16, column
+      // block (c / 8) % 2, 16-byte chunk c % 8; a quarter-warp per row)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c = u + 256 * i;
+        const int t = c >> 4, kb = (c >> 3) & 1, ch = c & 7;
+        const uint32_t off = (uint32_t)(16384 + kb * 8192 + t * 128 + ((ch ^ (t & 7)) << 4));
+        float bv[8];
+        ld_chunk(sm + R_DSB + off, bv);
+        const int j0 = kb * 64 + ch * 8;
+        const float4 p0 = *reinterpret_cast<const float4*>(s_p + j0);
+        const float4 p1 = *reinterpret_cast<const float4*>(s_p + j0 + 4);
+        const float pj[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) bv[e] = sigm(bv[e] + pj[e]);
+        tc::st_chunk_h(sm + R_DSB + off, bv);
+      }
+      bar_arrive_named(7, kThreads);
+      const float invL = 1.0f / (float)a.L;
       const int rr = u >> 3, ch = u & 7;  // token rows rr, rr + 32; 16-byte chunk
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -716,10 +736,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* s_gq = s_scr;                // [4][128] quarter log-decay sums
       float* s_lq = s_scr + 512;          // [4][128] quarter dG sums
       float* s_qf = s_scr + 1024;         // [4][128] dQ~ Q~ of a quarter's first token
+      float gv[16];  // the range's log-decays, kept for the ascending pass
       {
         float gsum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) gsum += ldbf(sm + R_RO + sw128_off(tb + e, jj, 64));
+        for (int e = 0; e < 16; ++e) {
+          gv[e] = ldbf(sm + R_RO + sw128_off(tb + e, jj, 64));
+          gsum += gv[e];
+        }
         s_gq[gp * 128 + jj] = gsum;
       }
       __syncthreads();
@@ -742,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int tl_ = 8 * sub + e;
           const int t = tb + tl_;
           const uint32_t o64 = sw128_off(t, jj, 64);
-          G += ldbf(sm + R_RO + o64);
+          G += gv[tl_];
           const float gam = __expf(G), igam = __fdividef(1.0f, gam);
           const float bb = sigm(ldbf(sm + R_RO + 16384 + o64) + pj);
           const float qt = ldbf(sm + R_X + sw128_off(64 + t, jj, 128));
@@ -752,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float dKt = dd[e], dQt = dd[8 + e], dKp = -dd[16 + e], dKh = dd[24 + e];
           const size_t x = x0 + (size_t)t * tstride;
           dq[x] = __float2bfloat16_rn(dQt * gprev);
-          dk[x] = __float2bfloat16_rn(dKt * gam + dKh * igam + dKp * bb * igam);
+          dk[x] = __float2bfloat16_rn(fmaf(dKt, gam, fmaf(dKp, bb, dKh) * igam));
           const float dz = dKp * kh * bb * (1.f - bb);
           dbx[x] = __float2bfloat16_rn(dz);
           dp_acc += dz;

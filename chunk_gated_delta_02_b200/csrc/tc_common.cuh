@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 #include "carve_internal.cuh"
@@ -31,6 +32,11 @@ __device__ __forceinline__ float sigm(float x) {
 __device__ __forceinline__ void bar_named(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Arrive on named barrier `id` (n threads in all) without waiting: the
+// producer side of a hand-off whose consumers bar_named(id, n).
+__device__ __forceinline__ void bar_arrive_named(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 // 8 fp32 values -> one 16-byte chunk of bf16 at `p`.
 __device__ __forceinline__ void st_chunk(uint8_t* p, const float* x) {
   uint4 u;
@@ -39,6 +45,29 @@ __device__ __forceinline__ void st_chunk(uint8_t* p, const float* x) {
   u.z = pack2(x[4], x[5]);
   u.w = pack2(x[6], x[7]);
   *reinterpret_cast<uint4*>(p) = u;
+}
+
+// 8 fp32 values -> one 16-byte chunk of fp16 at `p`.
+__device__ __forceinline__ void st_chunk_h(uint8_t* p, const float* x) {
+  uint4 u;
+  uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const __half2 hv = __floats2half2_rn(x[2 * i], x[2 * i + 1]);
+    w[i] = *reinterpret_cast<const uint32_t*>(&hv);
+  }
+  *reinterpret_cast<uint4*>(p) = u;
+}
+// 16-byte chunk of fp16 -> 8 fp32 values.
+__device__ __forceinline__ void ld_chunk_h(const uint8_t* p, float* x) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const __half2* hv = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(hv[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
 }
 
 // 16-byte chunk of bf16 -> 8 fp32 values.
@@ -58,10 +87,13 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* p, float* x) {
 //   Gamma_t = exp(sum_{u <= t} g_u)   K~ = K Gamma    Q~_t = Q_t Gamma_{t-1}
 //   K^ = K / Gamma                    kap^ = b K^     gamma = Gamma_63
 // All tiles are 128-byte swizzled 64-column blocks.  `x` holds [K; Q]
-// (128 rows per column block; rewritten in place to [K~; Q~]), `graw` and
-// `braw` raw g and b_x (64 rows per column block), `kh`, `kp` receive K^ and
-// kap^ (64 rows per column block, blocks `khs` bytes apart), `s_gam` gamma.  `s_p` holds p_j = (U_b m_c)_j; `red` is NW * 64
-// floats of scratch.  Called by NW warps: half of them per column block;
+// (128 rows per column block; rewritten in place to [K~; Q~]), `graw` raw g
+// and `bsm` the gate b itself in fp16 (b lies in (0, 1), where fp16 keeps
+// 11 significant bits; 64 rows per column block; formed by other
+// warps, which arrive on named barrier `bar_b` of `n_b` threads once it is
+// written: the token loop waits there), `kh`, `kp` receive K^ and kap^ (64
+// rows per column block, blocks `khs` bytes apart), `s_gam` gamma.  `red`
+// is NW * 64 floats of scratch.  Called by NW warps: half of them per column block;
 // thread (chunk of 8 channels, group of TPT = 128 / (4 NW) consecutive
 // tokens) touches one 16-byte chunk per row, the 8 threads of a
 // quarter-warp the 8 chunks of one row (conflict-free under the swizzle).
@@ -72,10 +104,10 @@ template <int NW>
 __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
                                                 uint8_t* kp,
                                                 const uint8_t* graw,
-                                                const uint8_t* braw,
-                                                const float* s_p, float* s_gam,
-                                                float* red, int bar_id,
-                                                uint32_t khs = 8192) {
+                                                const uint8_t* bsm,
+                                                float* s_gam, float* red,
+                                                int bar_id, uint32_t khs,
+                                                int bar_b, int n_b) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
@@ -126,31 +158,25 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
     ex[0] += a.x; ex[1] += a.y; ex[2] += a.z; ex[3] += a.w;
     ex[4] += b.x; ex[5] += b.y; ex[6] += b.z; ex[7] += b.w;
   }
-  float pj[8], gprev[8];
-  {
-    const float4 a = *reinterpret_cast<const float4*>(s_p + j0);
-    const float4 b = *reinterpret_cast<const float4*>(s_p + j0 + 4);
-    pj[0] = a.x; pj[1] = a.y; pj[2] = a.z; pj[3] = a.w;
-    pj[4] = b.x; pj[5] = b.y; pj[6] = b.z; pj[7] = b.w;
-  }
+  float gprev[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) gprev[e] = __expf(ex[e]);  // Gamma_{TPT tg - 1}
+  bar_named(bar_b, n_b);  // b written
 #pragma unroll
   for (int i = 0; i < TPT; ++i) {
     const int t = TPT * tg + i;
     float kv[8], qv[8], bv[8], o_kt[8], o_qt[8], o_kh[8], o_kp[8];
     ld_chunk(x + off128(t), kv);
     ld_chunk(x + off128(64 + t), qv);
-    ld_chunk(braw + off64(t), bv);
+    ld_chunk_h(bsm + off64(t), bv);
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float gam = __expf(ex[e] + gl[i][e]);
       const float igam = __fdividef(1.0f, gam);
-      const float bb = sigm(bv[e] + pj[e]);
       o_kt[e] = kv[e] * gam;
       o_qt[e] = qv[e] * gprev[e];
       o_kh[e] = kv[e] * igam;
-      o_kp[e] = bb * o_kh[e];
+      o_kp[e] = bv[e] * o_kh[e];
       gprev[e] = gam;
     }
     st_chunk(x + off128(t), o_kt);
