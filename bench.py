@@ -147,16 +147,21 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def dist_init():
+def dist_init(backend="nccl"):
+    """One process per GPU (torchrun's RANK / LOCAL_RANK / WORLD_SIZE); the
+    process group only carries the barrier and the max-over-ranks timing.
+    backend="gloo" runs the same host logic on CPU ranks."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if ws > 1:
         import datetime
-        torch.cuda.set_device(local)
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            kw["device_id"] = torch.device("cuda", local)
         torch.distributed.init_process_group(
-            "nccl", timeout=datetime.timedelta(seconds=120),
-            device_id=torch.device("cuda", local))
+            backend, timeout=datetime.timedelta(seconds=120), **kw)
     return ws, rank, local
 
 
@@ -166,11 +171,28 @@ def barrier(ws):
 
 
 def max_over_ranks(x, ws):
+    """The slowest rank's time: every rank passes its own, all get the max."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_batch(cfg, rank, dtype):
+    """This rank's own batch of the full shape (weak scaling: independent
+    sequences, seeded by rank): inputs and the output gradient d_o."""
+    inp = make_inputs(seed=1000 + rank, dtype=dtype, **cfg)
+    gro = make_grad_outputs(seed=1000 + rank, dtype=dtype, **cfg)
+    host = {k: v for k, v in inp.items() if v is not None}
+    host["d_o"] = gro["d_o"]
+    return host
+
+
+def job_tokens_per_s(tokens_per_rank, ws, ms_per_step):
+    """Whole-job throughput: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * ws / (ms_per_step * 1e-3)
 
 
 def oracle_sample(cfg, mode, seed, threads=None):
@@ -267,10 +289,7 @@ def main():
     dtype = torch.bfloat16
     B, T, H, DK, DV, R, L = (cfg[n] for n in ("B", "T", "H", "DK", "DV", "R",
                                               "L"))
-    inp = make_inputs(seed=1000 + rank, dtype=dtype, **cfg)
-    gro = make_grad_outputs(seed=1000 + rank, dtype=dtype, **cfg)
-    host = {k: v for k, v in inp.items() if v is not None}
-    host["d_o"] = gro["d_o"]
+    host = rank_batch(cfg, rank, dtype)
     d = {k: v.to(dev) for k, v in host.items()}
     d.setdefault("S0", None)
     training = args.mode == "train"
@@ -335,7 +354,7 @@ def main():
 
     ms_step = total_ms / args.steps
     tokens = B * T
-    value = tokens * ws / (ms_step * 1e-3)
+    value = job_tokens_per_s(tokens, ws, ms_step)
 
     # roofline of the dominant kernel (fwd or bwd), HBM-bound
     pk = peaks()
@@ -382,9 +401,18 @@ def main():
     }
 
     # end to end through the public API: pinned host inputs -> device, step,
-    # results -> pinned host, all inside the timed region
+    # results -> pinned host, all inside the timed region.  Two device sets
+    # of inputs and outputs: step i uses set i % 2, so step i's results copy
+    # out while step i + 1's inputs copy in (PCIe is full duplex) and the
+    # kernels run between them, each copy direction on its own stream.
     if not args.no_e2e:
         pin = {k: v.pin_memory() for k, v in host.items()}
+        d_sets = [d, {k: (torch.empty_like(v) if v is not None else None)
+                      for k, v in d.items()}]
+        o_sets = [o, torch.empty_like(o)]
+        g_sets = ([grads, {k: (torch.empty_like(v) if v is not None else None)
+                           for k, v in grads.items()}]
+                  if training else [None, None])
         outs_host = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory()}
         if training:
             for k, v in grads.items():
@@ -392,32 +420,63 @@ def main():
                     outs_host[k] = torch.empty(v.shape, dtype=v.dtype).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in pin.values())
         d2h = sum(v.numel() * v.element_size() for v in outs_host.values())
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in, ev_comp, ev_out = ([torch.cuda.Event() for _ in range(2)]
+                                  for _ in range(3))
+        count = [0]
 
         def e2e_step():
-            for k, v in pin.items():
-                d[k].copy_(v, non_blocking=True)
-            step()
-            outs_host["o"].copy_(o, non_blocking=True)
+            i = count[0]
+            count[0] += 1
+            sset = i % 2
+            ds, os_, gs = d_sets[sset], o_sets[sset], g_sets[sset]
+            with torch.cuda.stream(s_in):
+                if i >= 2:  # the kernels of step i - 2 have read this set
+                    s_in.wait_event(ev_comp[sset])
+                for k, v in pin.items():
+                    ds[k].copy_(v, non_blocking=True)
+                ev_in[sset].record(s_in)
+            stream.wait_event(ev_in[sset])
+            if i >= 2:  # step i - 2's results have left this set
+                stream.wait_event(ev_out[sset])
+            carve.chunk_fwd(ds["q"], ds["k"], ds["v"], ds["g"], ds["bx"],
+                            ds["w"], ds["u_down"], ds["u_up"], L, ds.get("S0"),
+                            None, training=training, workspace=wsb, o=os_,
+                            want_state=False)
             if training:
-                for k, v in grads.items():
-                    if v is not None:
-                        outs_host[k].copy_(v, non_blocking=True)
+                carve.chunk_bwd(ds["q"], ds["k"], ds["v"], ds["g"], ds["bx"],
+                                ds["w"], ds["u_down"], ds["u_up"], L,
+                                ds["d_o"], wsb, out=gs)
+            ev_comp[sset].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_comp[sset])
+                outs_host["o"].copy_(os_, non_blocking=True)
+                if training:
+                    for k, v in gs.items():
+                        if v is not None:
+                            outs_host[k].copy_(v, non_blocking=True)
+                ev_out[sset].record(s_out)
+            return sset
 
         for _ in range(2):
             e2e_step()
         torch.cuda.synchronize()
         barrier(ws)
         a, b = (torch.cuda.Event(enable_timing=True) for _ in range(2))
-        n_e2e = max(3, args.steps // 2)
-        a.record(stream)
+        n_e2e = max(6, args.steps // 2)
+        a.record(s_in)
         for _ in range(n_e2e):
-            e2e_step()
+            last = e2e_step()
+        stream.wait_event(ev_out[last])
         b.record(stream)
         torch.cuda.synchronize()
+        assert carve.get_status(wsb) == 0, "device status word set"
         e2e_ms = max_over_ranks(a.elapsed_time(b) / n_e2e, ws)
-        line["e2e"] = {"value": tokens * ws / (e2e_ms * 1e-3),
+        line["e2e"] = {"value": job_tokens_per_s(tokens, ws, e2e_ms),
                        "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+                       "pipelining": "double-buffered: step i's D2H overlaps "
+                                     "step i+1's H2D (separate streams)"}
 
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         secs, ptoks, npairs, thr = oracle_sample(cfg, args.mode, 7)
