@@ -41,6 +41,7 @@ namespace carve {
 namespace {
 
 using namespace ptx;
+using tc::bar_arrive_named;
 using tc::bar_named;
 using tc::fsw;
 using tc::pack2;
@@ -276,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       if (rq == 0) s_p[jj] = acc;
     }
+    bar_named(6, 256);  // p visible to all of warps 8-15
   };
 
   auto issue_vgb = [&](int ib) {
@@ -412,14 +414,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         w_lo = w_bits[r0 * H + h];
         w_hi = w_bits[(r0 + 32) * H + h];
       }
-    } else if (ib % bpc == 0) {
-      gate(ib / bpc);
+      bar_named(5, kThreads);  // p formed (warps 8-15 arrive after the gate)
+    } else {
+      if (ib % bpc == 0) gate(ib / bpc);
+      bar_arrive_named(5, kThreads);
     }
-    fence_async_smem();
-    __syncthreads();
-    if (*s_abort) break;
 
-    // ---- 3. K^ -> its operand slot and kap^ = sigmoid(b_x + p) K^; then
+    // ---- 3. K^ -> its operand slot and kap^ = sigmoid(b_x + p) K^ (all
+    //      warps, each as soon as its part above is done); then
     //      G = [K~; Q~] [K^; kap^]^T in one N = 128 product per k-step
     //      (columns 0-63 [M; P_k], 64-127 [A; P_kap]).  The commit after G
     //      covers D1 as well.
@@ -455,22 +457,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (gp == 0) {
       // ---- 4a. [A; P_kap] (strictly lower): A -> fp32 for the inversion,
       //          P_kap -> bf16 operand; T = (I + A)^{-1} (warps 0-3)
-#pragma unroll 1
-      for (int part = 0; part < 2; ++part) {
-        float vals[32];
-        tmem_ld32(tl + TM_GK + part * 32, vals);
+      {
+        float vals[64];  // the whole Gram row in one TMEM load
+        tmem_ld64(tl + TM_GK, vals);
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (part * 32 + e >= gr) vals[e] = 0.f;
+        for (int e = 0; e < 64; ++e)
+          if (e >= gr) vals[e] = 0.f;
         if (row < 64) {
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(s_af + fsw(row, part * 32 + e)) =
+          for (int e = 0; e < 64; e += 4)
+            *reinterpret_cast<float4*>(s_af + fsw(row, e)) =
                 make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
         } else {
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8)
-            st_chunk(pq + sw128_chunk(gr, 0, part * 4 + c8, 64), vals + c8 * 8);
+          for (int c8 = 0; c8 < 8; ++c8)
+            st_chunk(pq + sw128_chunk(gr, 0, c8, 64), vals + c8 * 8);
         }
       }
       bar_named(2, 128);
