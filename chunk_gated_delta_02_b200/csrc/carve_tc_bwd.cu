@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mark(B_GB);
   };
   if (tid == 0) {
+    issue_top(NB - 1);
     issue_sb(NB - 1);
     issue_pre(NB - 1);
   }
@@ -377,10 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       dp_acc = 0.f;
     }
 
-    // ---- S1: inputs.  q, d_o now; the rest was requested during the
-    //      previous block.  Block ib - 1's q, d_o tiles -> L2 (and k, which
-    //      loads during this block).
-    if (tid == 0) issue_top(ib);
+    // ---- S1: inputs, all requested during the previous block (q, d_o
+    //      in its epilogue).  Block ib - 1's q, d_o tiles -> L2 (and k,
+    //      which loads during this block).
     if (tid == 32 && ib > 0) {  // (the rest of block ib - 1 loads a block ahead)
       const int tn = tok - kBlk;
 #pragma unroll 1
@@ -795,6 +795,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       s_lq[gp * 128 + jj] = lsum;
       s_qf[gp * 128 + jj] = qfirst;
       __syncthreads();
+      // the ascending pass was the last reader of Q~ (X rows 64..127) and of
+      // the raw g, b_x (RO): block ib - 1's q, d_o load from here on
+      if (tid == 0 && ib > 0 && !*s_abort) issue_top(ib - 1);
       // dG_{tb+15} reads the next quarter's first Q~ term (t = 63: the
       // gradient of log gamma); the later quarters' sums seed the suffix
       const float dlg = s_x[jj];

@@ -9,11 +9,12 @@
 // triangular solve per block serves every value row):
 //
 //   keys        Gamma = exp(cumsum g), K~ = K Gamma, Q~ = Q Gamma_{t-1},
-//               K^ = K / Gamma (warps 0-7; section 2.3: key-axis decay)
-//   gate, W     first block of a chunk: p = U_up U_down m_c (section 2.1);
-//               W = w V (warps 8-15, meanwhile)
+//               K^ = K / Gamma (section 2.3: key-axis decay; warps 8-15,
+//               during the previous block's solve)
+//   gate, W     first block of a chunk: p = U_up U_down m_c (section 2.1;
+//               warps 8-15); W = w V (warps 0-7, meanwhile)
 //   MMA 1       D1 = S [K~; Q~]^T             ->  [(K~ S^T)^T | (Q~ S^T)^T]
-//               (issued while the other threads form kap^ = sigmoid(bx + p) K^)
+//               (issued first; warps 1-15 then form kap^ = sigmoid(bx + p) K^)
 //               G = [K~; Q~] [K^; kap^]^T     ->  [M ; P_k | A ; P_kap]
 //   MMA 2       D1 += W^T [M; P_k]^T          ->  [R^T | (Q~ S^T + P_k W)^T]
 //   solve       T = (I + A)^{-1} by 16 x 16 blocks (warps 0-3)
@@ -87,7 +88,7 @@ static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
 // mbarriers (index into the small region's array)
 constexpr int B_VGB = 0;   // TMA v, g, b_x
 constexpr int B_KQ = 1;    // TMA k, q
-constexpr int B_M1 = 2;    // MMA 1 (Grams, S X^T)
+constexpr int B_M1 = 2;    // MMA 1 (S X^T and the Grams)
 constexpr int B_M2 = 3;    // MMA 2 (W^T [M;P_k]^T)
 constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
 constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
@@ -414,19 +415,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         w_lo = w_bits[r0 * H + h];
         w_hi = w_bits[(r0 + 32) * H + h];
       }
-      bar_named(5, kThreads);  // p formed (warps 8-15 arrive after the gate)
+      // p formed (warps 8-15 arrive after the gate); warp 0, late from
+      // issuing D1, goes straight to the block barrier
+      if (warp > 0) bar_named(5, kThreads - 32);
     } else {
       if (ib % bpc == 0) gate(ib / bpc);
-      bar_arrive_named(5, kThreads);
+      bar_arrive_named(5, kThreads - 32);
     }
 
-    // ---- 3. K^ -> its operand slot and kap^ = sigmoid(b_x + p) K^ (all
-    //      warps, each as soon as its part above is done); then
+    // ---- 3. K^ -> its operand slot and kap^ = sigmoid(b_x + p) K^ (warps
+    //      1-15, each as soon as its part above is done); then
     //      G = [K~; Q~] [K^; kap^]^T in one N = 128 product per k-step
     //      (columns 0-63 [M; P_k], 64-127 [A; P_kap]).  The commit after G
     //      covers D1 as well.
-    tc::kappa_block(sm + OFF_RG, sm + OFF_KHP, sm + OFF_KHP + 8192, sm + OFF_RB,
-                    s_p, 16384, tid, kThreads);
+    if (warp > 0)
+      tc::kappa_block(sm + OFF_RG, sm + OFF_KHP, sm + OFF_KHP + 8192,
+                      sm + OFF_RB, s_p, 16384, tid - 32, kThreads - 32);
     fence_async_smem();
     if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
     __syncthreads();
