@@ -512,6 +512,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                  vals + c8 * 8);
       atomicAdd(&s_x[c0 + lane], dlg_part);
     }
+    // dE^T = -dS~ kap^T needs only dS~ and kap^: issued now, it runs while
+    // the Grams are masked
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && !*s_abort) {
+      tc_fence_after();
+      const uint32_t dsb0 = smem_u32(sm + R_DSB), kp0 = smem_u32(sm + R_KHP) + 8192;
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks)
+        umma_bf16(tmem + T_DER,
+                  desc_kmajor_sw128(dsb0 + (ks >> 2) * 16384 + (ks & 3) * 32),
+                  desc_kmajor_sw128(kp0 + (ks >> 2) * 16384 + (ks & 3) * 32),
+                  ID_KK64_NA, ks > 0);
+    }
     wait(B_1, 13);
     tc_fence_after();
     {
@@ -543,17 +558,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- S6: dE^T = -dS~ kap^T - dO^T P_kap
+    // ---- S6: dE^T = -dS~ kap^T (issued in S4) - dO^T P_kap
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t dsb0 = smem_u32(sm + R_DSB), kp0 = smem_u32(sm + R_KHP) + 8192;
       const uint32_t ro0 = smem_u32(sm + R_RO), pq0 = smem_u32(sm + R_PQ);
-#pragma unroll 1
-      for (int ks = 0; ks < 8; ++ks)
-        umma_bf16(tmem + T_DER,
-                  desc_kmajor_sw128(dsb0 + (ks >> 2) * 16384 + (ks & 3) * 32),
-                  desc_kmajor_sw128(kp0 + (ks >> 2) * 16384 + (ks & 3) * 32),
-                  ID_KK64_NA, ks > 0);
 #pragma unroll 1
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + T_DER,

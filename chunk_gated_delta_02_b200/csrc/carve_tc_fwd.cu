@@ -20,7 +20,7 @@
 //   solve       T = (I + A)^{-1} by 16 x 16 blocks (warps 0-3)
 //   MMA 3a      E^T = R^T T^T                 (E = T R, the WY pseudo-values)
 //   MMA 3b      D1[O] -= E^T P_kap^T          ->  O^T = (Q~ S^T + P_k W - P_kap E)^T
-//   MMA 4       S += W^T K^ - E^T kap^ ;  S <- S Diag(gamma)
+//   MMA 4       S += W^T K^ (issued with MMA 2) - E^T kap^ ;  S <- S Diag(gamma)
 //   output      o_t = row t of O; m_{c+1} = mean of the chunk's o_t
 //
 // The transposed products put one value row v of S, R, E and O in TMEM lane
@@ -93,7 +93,8 @@ constexpr int B_M2 = 3;    // MMA 2 (W^T [M;P_k]^T)
 constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
 constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
 constexpr int B_X = 6;     // dv = 256: the other CTA's half of U_down m arrived
-constexpr int kNumBars = 7;
+constexpr int B_WK = 7;    // S += W^T K^ (issued with MMA 2)
+constexpr int kNumBars = 8;
 
 // TMEM columns (fp32, lanes = rows)
 constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
@@ -522,6 +523,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     desc_kmajor_sw128(my0 + ks * 32), ID_AMN, 1);
         umma_commit(bars + B_M2);
         mark(B_M2);
+        // the E-independent half of MMA 4, S += W^T K^, off the critical
+        // path (TM_S is next read after MMA 4)
+        const uint32_t kh0 = smem_u32(sm + OFF_KHP);
+#pragma unroll 1
+        for (int ks = 0; ks < 4; ++ks)
+          umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
+                    desc_mnmajor_sw128(kh0 + ks * 2048, 16384), ID_AMN_BMN, 1);
+        umma_commit(bars + B_WK);
+        mark(B_WK);
       }
       wait(B_M2, 4);  // [M; P_k] consumed, R^T complete
       tc_fence_after();
@@ -599,22 +609,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (*s_abort) break;
 
-    // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S += W^T K^ - E^T kap^
+    // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S -= E^T kap^ (W^T K^
+    //      was added with MMA 2)
+    wait(B_WK, 11);
     if (tid == 0) {
       if (rec) {
         bulk_store(rec + kTcRecE, sm + OFF_AF, 16384);
         bulk_commit();
       }
       tc_fence_after();
-      const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KHP);
-      const uint32_t re0 = smem_u32(sm + OFF_RE), kp0 = kh0 + 8192;
-      const uint32_t pq0 = smem_u32(pq);
+      const uint32_t kp0 = smem_u32(sm + OFF_KHP) + 8192;
+      const uint32_t re0 = smem_u32(sm + OFF_RE), pq0 = smem_u32(pq);
 #pragma unroll 1
       for (int ks = 0; ks < 4; ++ks) {
         umma_bf16(tmem + TM_D1 + 64, desc_kmajor_sw128(re0 + ks * 32),
                   desc_kmajor_sw128(pq0 + ks * 32), ID_N64_NA, 1);
-        umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
-                  desc_mnmajor_sw128(kh0 + ks * 2048, 16384), ID_AMN_BMN, 1);
         umma_bf16(tmem + TM_S, desc_kmajor_sw128(re0 + ks * 32),
                   desc_mnmajor_sw128(kp0 + ks * 2048, 16384), ID_BMN_NA, 1);
       }
