@@ -361,6 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     w_lo = w_bits[r0 * H + h];
     w_hi = w_bits[(r0 + 32) * H + h];
   }
+  bool dm_pending = false;  // s_dmn still to be summed from the last chunk's partials
   float dp_acc = 0.f;   // dp_j share (channel row, this warp's token quarter)
   float p_next = tid < 128 ? a.gin[((size_t)pair * NC + NC - 1) * GR + tid] : 0.f;
   for (int ib = NB - 1; ib >= 0; --ib) {
@@ -377,6 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid < 128) s_p[tid] = p_next;
       dp_acc = 0.f;
     }
+    if (dm_pending && tid < 128) {  // dm of the chunk after this one (S13)
+      const float* s_dmq = reinterpret_cast<const float*>(sm + R_MP) + 2688;
+      s_dmn[tid] = (s_dmq[tid] + s_dmq[128 + tid]) + (s_dmq[256 + tid] + s_dmq[384 + tid]);
+    }
+    dm_pending = false;
 
     // ---- S1: inputs, all requested during the previous block (q, d_o
     //      in its epilogue).  Block ib - 1's q, d_o tiles -> L2 (and k,
@@ -390,7 +396,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_3d(&tm_do, x0, h, tn);
       }
     }
-    if (tid < 64) s_w[tid] = __bfloat162float(w_in[((size_t)tok + tid) * H + h]);
     if (chunk_first && ib > 0 && tid < 128)  // the next block starts chunk c - 1
       p_next = a.gin[((size_t)pair * NC + c - 1) * GR + tid];
     wait(B_SB, 10);
@@ -467,6 +472,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           *reinterpret_cast<uint4*>(sm + R_RO + off) = y;
         }
+      }
+      if ((u & 7) == 0) {  // this block's w_t for dv, dw (S11)
+        s_w[u >> 3] = __uint_as_float(w_lo << 16);
+        s_w[(u >> 3) + 32] = __uint_as_float(w_hi << 16);
       }
       if (ib > 0) {  // the next block's w_t
         const size_t r0 = (size_t)b * T + (ib - 1) * kBlk + ((tid - 256) >> 3);
@@ -842,24 +851,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane < 8) s_dhq[qd * 32 + gp * 8 + lane] = part;
       }
       __syncthreads();
-      if (tid < 32) {
-        const float dhv = s_dhq[tid] + s_dhq[32 + tid] + s_dhq[64 + tid] + s_dhq[96 + tid];
-        s_dw[tid] = dhv;
-        if (tid < R) rec[kDK + tid] = dhv;
-      }
-      __syncthreads();
-      {  // dm[v] partial over r = 8 gp .. 8 gp + 7, v = row
+      // dh[r] = sum of the four quadrants' partials, formed where it is
+      // used; dm[v] partial over r = 8 gp .. 8 gp + 7, v = row (summed
+      // into s_dmn at the next block's start, after the block barrier)
+      auto dh = [&](int r) {
+        return (s_dhq[r] + s_dhq[32 + r]) + (s_dhq[64 + r] + s_dhq[96 + r]);
+      };
+      if (tid < R) rec[kDK + tid] = dh(tid);
+      {
         float acc = 0.f;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          acc = fmaf(bf_lo(udn[i]), s_dw[8 * gp + 2 * i], acc);
-          acc = fmaf(bf_hi(udn[i]), s_dw[8 * gp + 2 * i + 1], acc);
+          acc = fmaf(bf_lo(udn[i]), dh(8 * gp + 2 * i), acc);
+          acc = fmaf(bf_hi(udn[i]), dh(8 * gp + 2 * i + 1), acc);
         }
         s_dmq[gp * 128 + row] = acc;
       }
-      __syncthreads();
-      if (tid < 128)
-        s_dmn[tid] = s_dmq[tid] + s_dmq[128 + tid] + s_dmq[256 + tid] + s_dmq[384 + tid];
+      dm_pending = true;
       dp_acc = 0.f;
     }
     fence_async_smem();
@@ -883,7 +891,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         *reinterpret_cast<float4*>(dst + e) =
             make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
     }
-    if (a.dm0 && tid < 128) a.dm0[(size_t)pair * kDV + tid] = s_dmn[tid];
+    if (a.dm0 && tid < 128) {  // chunk 0's dm, from S13's partials
+      const float* s_dmq = reinterpret_cast<const float*>(sm + R_MP) + 2688;
+      a.dm0[(size_t)pair * kDV + tid] =
+          (s_dmq[tid] + s_dmq[128 + tid]) + (s_dmq[256 + tid] + s_dmq[384 + tid]);
+    }
   }
   tc_fence_before();
   __syncthreads();
