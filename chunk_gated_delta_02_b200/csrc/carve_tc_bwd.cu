@@ -363,7 +363,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   bool dm_pending = false;  // s_dmn still to be summed from the last chunk's partials
   float dp_acc = 0.f;   // dp_j share (channel row, this warp's token quarter)
-  float p_next = tid < 128 ? a.gin[((size_t)pair * NC + NC - 1) * GR + tid] : 0.f;
+  // p of the last chunk (the first visited); later chunks' p arrive by
+  // async copies issued in the previous block's epilogue
+  if (tid < 128) s_p[tid] = a.gin[((size_t)pair * NC + NC - 1) * GR + tid];
   for (int ib = NB - 1; ib >= 0; --ib) {
     const int t0 = ib * kBlk;
     const int c = ib / bpc;
@@ -373,9 +375,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* rec = args.gate_rec + ((size_t)pair * NC + c) * GR;
 
     // ---- S0: gate of chunk c, p = U_up U_down m_c (forward record,
-    //      fetched during the previous block)
+    //      copied into s_p during the previous block; published by the
+    //      barrier at the end of S1)
     if (chunk_last) {
-      if (tid < 128) s_p[tid] = p_next;
+      if (ib < NB - 1 && tid < 32) cp_async_wait_all();
       dp_acc = 0.f;
     }
     if (dm_pending && tid < 128) {  // dm of the chunk after this one (S13)
@@ -396,8 +399,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_3d(&tm_do, x0, h, tn);
       }
     }
-    if (chunk_first && ib > 0 && tid < 128)  // the next block starts chunk c - 1
-      p_next = a.gin[((size_t)pair * NC + c - 1) * GR + tid];
     wait(B_SB, 10);
     wait(B_PRE, 11);
     wait(B_IN, 12);
@@ -815,6 +816,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // the ascending pass was the last reader of Q~ (X rows 64..127) and of
       // the raw g, b_x (RO): block ib - 1's q, d_o load from here on
       if (tid == 0 && ib > 0 && !*s_abort) issue_top(ib - 1);
+      // s_p was last read above: the next block starts chunk c - 1
+      if (chunk_first && ib > 0 && tid < 32) {
+        cp_async16(s_p + 4 * tid, a.gin + ((size_t)pair * NC + c - 1) * GR + 4 * tid);
+        cp_async_commit();
+      }
       // dG_{tb+15} reads the next quarter's first Q~ term (t = 63: the
       // gradient of log gamma); the later quarters' sums seed the suffix
       const float dlg = s_x[jj];
@@ -875,6 +881,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
   }
 
+  if (tid < 32) cp_async_wait_all();  // (an aborted walk may leave one in flight)
   // ---- dS0, dm0; an aborted CTA first lets its copies and MMAs land
   if (*s_abort) {
     if (tid == 0)

@@ -80,6 +80,20 @@ __device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) 
                "r"(bytes)
                : "memory");
 }
+// 16 bytes global -> shared per thread without a register round trip
+// (completion by the issuing thread's async-copy groups).
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // Untiled bulk copies (addresses 16-byte aligned, size a multiple of 16).
 // Global -> shared, completion counted on `bar` like the tiled loads.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src,
