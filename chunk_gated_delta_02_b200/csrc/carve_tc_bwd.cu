@@ -773,6 +773,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       float gprev = __expf(G);
       float dGv[16];
       float qfirst = 0.f;
+      // Outputs leave as bf16 pairs of neighbouring channels: for each pair
+      // of tokens (2u, 2u + 1) the even lane of a lane pair stores token 2u
+      // and the odd lane token 2u + 1, each after one shuffle (half the
+      // store instructions of one 2-byte store per value).
+      const bool odd = (lane & 1) != 0;
+      const size_t xp = x0 - (jj & 1);    // element offset of the pair's even channel
+      auto st_pair = [&](__nv_bfloat16* base, int t_even, float v_even, float v_odd) {
+        const float recv = __shfl_xor_sync(0xffffffffu, odd ? v_even : v_odd, 1);
+        const __nv_bfloat162 pr = odd ? __floats2bfloat162_rn(recv, v_odd)
+                                      : __floats2bfloat162_rn(v_even, recv);
+        *reinterpret_cast<__nv_bfloat162*>(
+            base + xp + (size_t)(t_even + (odd ? 1 : 0)) * tstride) = pr;
+      };
+      float hq = 0.f, hk = 0.f, hz = 0.f;  // the even token's values
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
         float dd[32];  // dK~ | dQ~ | -dkap^ | dK^ of 8 tokens
@@ -792,11 +806,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float kt = kh * gam * gam;  // K~ = K^ Gamma^2
           const float kp = bb * kh;         // kap^ = b K^
           const float dKt = dd[e], dQt = dd[8 + e], dKp = -dd[16 + e], dKh = dd[24 + e];
-          const size_t x = x0 + (size_t)t * tstride;
-          dq[x] = __float2bfloat16_rn(dQt * gprev);
-          dk[x] = __float2bfloat16_rn(fmaf(dKt, gam, fmaf(dKp, bb, dKh) * igam));
+          const float vq = dQt * gprev;
+          const float vk = fmaf(dKt, gam, fmaf(dKp, bb, dKh) * igam);
           const float dz = dKp * kh * bb * (1.f - bb);
-          dbx[x] = __float2bfloat16_rn(dz);
+          if ((e & 1) == 0) {
+            hq = vq; hk = vk; hz = dz;
+          } else {
+            st_pair(dq, t - 1, hq, vq);
+            st_pair(dk, t - 1, hk, vk);
+            st_pair(dbx, t - 1, hz, dz);
+          }
           dp_acc += dz;
           const float qp = dQt * qt;        // Q~_t reads Gamma_{t-1}
           dGv[tl_] = dKt * kt - dKh * kh - dKp * kp;
@@ -828,10 +847,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc = 0.f;
       for (int g2 = gp + 1; g2 < 4; ++g2)
         acc += s_lq[g2 * 128 + jj] + (g2 < 3 ? s_qf[(g2 + 1) * 128 + jj] : dlg);
+      float hg = 0.f;  // the odd token's suffix sum
 #pragma unroll
       for (int i = 15; i >= 0; --i) {
         acc += dGv[i];
-        dg[x0 + (size_t)(tb + i) * tstride] = __float2bfloat16_rn(acc);
+        if (i & 1)
+          hg = acc;
+        else
+          st_pair(dg, tb + i, acc, hg);
       }
     }
 

@@ -639,12 +639,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     {
       float vals[32];
       tmem_ld16x2(tl + TM_D1 + 64 + gp * 16, tl + TM_S + gp * 32 + 16, vals);
-      __nv_bfloat16* orow = o + ((size_t)b * T + t0 + gp * 16) * H * DVt +
-                            (size_t)h * DVt + v0 + row;
+      // o leaves as bf16 pairs of neighbouring value rows: for tokens
+      // (2u, 2u + 1) the even lane of a lane pair stores token 2u and the
+      // odd lane token 2u + 1, after one shuffle (half the store count)
+      const bool odd = (lane & 1) != 0;
+      __nv_bfloat16* orow = o + ((size_t)b * T + t0 + gp * 16 + (odd ? 1 : 0)) * H * DVt +
+                            (size_t)h * DVt + v0 + (row & ~1);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        msum += vals[e];
-        orow[(size_t)e * H * DVt] = __float2bfloat16_rn(vals[e]);
+      for (int e = 0; e < 16; e += 2) {
+        msum += vals[e] + vals[e + 1];
+        const float recv = __shfl_xor_sync(0xffffffffu, odd ? vals[e] : vals[e + 1], 1);
+        *reinterpret_cast<__nv_bfloat162*>(orow + (size_t)e * H * DVt) =
+            odd ? __floats2bfloat162_rn(recv, vals[e + 1])
+                : __floats2bfloat162_rn(vals[e], recv);
       }
       float sv[32];
       tmem_ld16(tl + TM_S + gp * 32, sv);
