@@ -65,7 +65,7 @@ constexpr uint32_t SM_X = 1024;      // g half sums | dlog gamma | dp   128 f32
 constexpr uint32_t SM_GAM = 1536;    // gamma | dg hand-off | dh parts  128 f32
 constexpr uint32_t SM_W = 2048;      // w_t                 64 f32
 constexpr uint32_t SM_DW = 2304;     // dw sums | dh        64 f32
-constexpr uint32_t SM_BAR = 2560;    // 9 mbarriers
+constexpr uint32_t SM_BAR = 2560;    // 10 mbarriers
 constexpr uint32_t SM_TMEM = 2640;
 constexpr uint32_t SM_ABORT = 2644;
 constexpr uint32_t kSmemBytes = 232448;
@@ -82,7 +82,9 @@ constexpr int B_4 = 5;     // MMA S7
 constexpr int B_5 = 6;     // MMA S9
 constexpr int B_7 = 7;     // MMA S11
 constexpr int B_PRE = 8;   // v, g, b_x, E and T records
-constexpr int kNumBars = 9;
+constexpr int B_7B = 9;    // MMA S11, the D8 half (issued by thread 256)
+constexpr int kNumBars = 10;
+static_assert(SM_BAR + 8 * kNumBars <= SM_TMEM, "mbarriers");
 
 // TMEM columns
 constexpr uint32_t T_DS = 0;     // dS [v][j]
@@ -678,12 +680,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      (into the columns G2 left); meanwhile dv, dw (16 tokens per group)
     //      and the dlog gamma share of block ib - 1 (its S_new is this
     //      block's state record, still in SB)
+    //      Two issuers, so that neither warp is late for the barrier below
+    //      by the whole batch: thread 0 the D7 half, thread 256 the D8 half
+    //      (separate accumulators, separate commits).
     if (tid == 0) {
       tc_fence_after();
       const uint32_t kh0 = smem_u32(sm + R_KHP), kp0 = kh0 + 8192;
       const uint32_t mp0 = smem_u32(sm + R_MP), pq0 = smem_u32(sm + R_PQ);
-      const uint32_t x0 = smem_u32(sm + R_X), dsb0 = smem_u32(sm + R_DSB);
-      const uint32_t ew0 = smem_u32(sm + R_EW);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t a0 = (ks < 4 ? kp0 : kh0) + (ks & 3) * 2048;
@@ -691,6 +694,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_G, desc_mnmajor_sw128(a0, 16384),
                   desc_kmajor_sw128(g2), ks < 4 ? ID_MK128_NA : ID_MK128, 1);
       }
+      umma_commit(bars + B_7);
+      mark(B_7);
+    } else if (tid == 256) {
+      tc_fence_after();
+      const uint32_t mp0 = smem_u32(sm + R_MP);
+      const uint32_t x0 = smem_u32(sm + R_X), dsb0 = smem_u32(sm + R_DSB);
+      const uint32_t ew0 = smem_u32(sm + R_EW);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         umma_bf16(tmem + T_D8, desc_mnmajor_sw128(x0 + ks * 2048, 16384),
@@ -699,8 +709,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                   desc_kmajor_sw128(ew0 + (ks >> 2) * 16384 + (ks & 3) * 32),
                   ID_MK128, 1);
       }
-      umma_commit(bars + B_7);
-      mark(B_7);
+      umma_commit(bars + B_7B);
+      mark(B_7B);
     }
     if (ib > 0) {
       float vals[32];
@@ -738,6 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // block ib - 1's state operand -> SB (read above)
     if (tid == 0 && ib > 0 && !*s_abort) issue_sb(ib - 1);
     wait(B_7, 17);
+    wait(B_7B, 20);
     // block ib - 1's v, g, b_x, E, T into the buffers S11 released
     if (tid == 0 && ib > 0 && !*s_abort) issue_pre(ib - 1);
     wait(B_GB, 18);
@@ -907,7 +918,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid < 32) cp_async_wait_all();  // (an aborted walk may leave one in flight)
   // ---- dS0, dm0; an aborted CTA first lets its copies and MMAs land
   if (*s_abort) {
-    if (tid == 0)
+    if (tid == 0 || tid == 256)  // the threads that start copies and MMAs
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) drain_bar(bars + i, (npar >> i) & 1u);
   } else {
