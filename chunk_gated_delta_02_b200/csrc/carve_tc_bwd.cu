@@ -525,11 +525,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       atomicAdd(&s_x[c0 + lane], dlg_part);
     }
     // dE^T = -dS~ kap^T needs only dS~ and kap^: issued now, it runs while
-    // the Grams are masked
+    // the Grams are masked; thread 288 issues it (and S6), its warp has no
+    // masking to do
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (tid == 0 && !*s_abort) {
+    if (tid == 288 && !*s_abort) {
       tc_fence_after();
       const uint32_t dsb0 = smem_u32(sm + R_DSB), kp0 = smem_u32(sm + R_KHP) + 8192;
 #pragma unroll 1
@@ -571,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*s_abort) break;
 
     // ---- S6: dE^T = -dS~ kap^T (issued in S4) - dO^T P_kap
-    if (tid == 0) {
+    if (tid == 288) {
       tc_fence_after();
       const uint32_t ro0 = smem_u32(sm + R_RO), pq0 = smem_u32(sm + R_PQ);
 #pragma unroll 1
@@ -918,7 +919,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid < 32) cp_async_wait_all();  // (an aborted walk may leave one in flight)
   // ---- dS0, dm0; an aborted CTA first lets its copies and MMAs land
   if (*s_abort) {
-    if (tid == 0 || tid == 256)  // the threads that start copies and MMAs
+    if (tid == 0 || tid == 256 || tid == 288)  // the threads that start copies and MMAs
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) drain_bar(bars + i, (npar >> i) & 1u);
   } else {
