@@ -65,9 +65,9 @@ constexpr uint32_t SM_X = 1024;      // g half sums | dlog gamma | dp   128 f32
 constexpr uint32_t SM_GAM = 1536;    // gamma | dg hand-off | dh parts  128 f32
 constexpr uint32_t SM_W = 2048;      // w_t                 64 f32
 constexpr uint32_t SM_DW = 2304;     // dw sums | dh        64 f32
-constexpr uint32_t SM_BAR = 2560;    // 10 mbarriers
-constexpr uint32_t SM_TMEM = 2640;
-constexpr uint32_t SM_ABORT = 2644;
+constexpr uint32_t SM_BAR = 2560;    // 11 mbarriers
+constexpr uint32_t SM_TMEM = 2648;
+constexpr uint32_t SM_ABORT = 2652;
 constexpr uint32_t kSmemBytes = 232448;
 static_assert(R_SM + 2688 <= kSmemBytes, "small region");
 static_assert(R_PQ == R_MP + 16384 && R_TT == R_PQ + 8192, "G2 blocks");
@@ -83,7 +83,8 @@ constexpr int B_5 = 6;     // MMA S9
 constexpr int B_7 = 7;     // MMA S11
 constexpr int B_PRE = 8;   // v, g, b_x, E and T records
 constexpr int B_7B = 9;    // MMA S11, the D8 half (issued by thread 256)
-constexpr int kNumBars = 10;
+constexpr int B_5B = 10;   // MMA S9, the dW^T and dS half (issued by thread 256)
+constexpr int kNumBars = 11;
 static_assert(SM_BAR + 8 * kNumBars <= SM_TMEM, "mbarriers");
 
 // TMEM columns
@@ -627,22 +628,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (*s_abort) break;
 
     // ---- S9: G2raw = [dR; dO] [E; W]^T, dW^T, dS += [dR; dO]^T [K~; Q~],
-    //      D7^T = S^T [dR; dO]^T
+    //      D7^T = S^T [dR; dO]^T.  Two issuers with their own commits:
+    //      thread 0 G2 and D7 (TMEM columns T_G2, T_G), thread 256 dW^T and
+    //      dS (T_RE, T_DS)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ro0 = smem_u32(sm + R_RO), ew0 = smem_u32(sm + R_EW);
-      const uint32_t dsb0 = smem_u32(sm + R_DSB);
-      const uint32_t kh0 = smem_u32(sm + R_KHP), mp0 = smem_u32(sm + R_MP);
-      const uint32_t x0 = smem_u32(sm + R_X), sb0 = smem_u32(sm + R_SB);
+      const uint32_t sb0 = smem_u32(sm + R_SB);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
         umma_bf16(tmem + T_G2, desc_kmajor_sw128(ro0 + kx),
                   desc_kmajor_sw128(ew0 + kx), ID_KK128, ks > 0);
-        umma_bf16(tmem + T_RE, desc_kmajor_sw128(dsb0 + kx),
-                  desc_kmajor_sw128(kh0 + kx), ID_KK64, ks > 0);
         umma_bf16(tmem + T_G, desc_mnmajor_sw128(sb0 + ks * 2048, 16384),
                   desc_kmajor_sw128(ro0 + kx), ID_MK128, ks > 0);
+      }
+      umma_commit(bars + B_5);
+      mark(B_5);
+    } else if (tid == 256) {
+      tc_fence_after();
+      const uint32_t ro0 = smem_u32(sm + R_RO), dsb0 = smem_u32(sm + R_DSB);
+      const uint32_t kh0 = smem_u32(sm + R_KHP), mp0 = smem_u32(sm + R_MP);
+      const uint32_t x0 = smem_u32(sm + R_X);
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+        umma_bf16(tmem + T_RE, desc_kmajor_sw128(dsb0 + kx),
+                  desc_kmajor_sw128(kh0 + kx), ID_KK64, ks > 0);
       }
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
@@ -651,10 +663,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_DS, desc_mnmajor_sw128(ro0 + ks * 2048, 16384),
                   desc_mnmajor_sw128(x0 + ks * 2048, 16384), ID_MM128, 1);
       }
-      umma_commit(bars + B_5);
-      mark(B_5);
+      umma_commit(bars + B_5B);
+      mark(B_5B);
     }
     wait(B_5, 16);
+    wait(B_5B, 21);
     tc_fence_after();
 
     // ---- S10: the epilogue's raw g, b_x -> RO; G2 (masked, bf16; 32
