@@ -121,8 +121,9 @@ static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* rg, float* gam,
 
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
 // rows 32 qd .. 32 qd + 31) and column group gp = w / 4.  Warps 0-3 also
-// run the triangular solve while warps 4-11 prepare [M; P_k] and R^T; warps
-// 8-15 form the gate and W while warps 0-7 run the key-side transform.
+// run the triangular solve while warps 4-11 prepare [M; P_k] and R^T and
+// warps 8-15 then run the next block's key-side transform; at the top of a
+// block warps 8-15 form the gate while warps 0-7 form W.
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -187,9 +188,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);  // lane base
 
   // Every barrier has at most one phase in flight.  `npar` holds the parity
-  // each thread waits for next; thread 0 also tracks in `pend` the phases it
-  // started (copies issued, MMAs committed) so that an aborting CTA drains
-  // them before it exits.
+  // each thread waits for next; the issuing threads also track in `pend`
+  // the phases they started (copies issued, MMAs committed) so that an
+  // aborting CTA drains them before it exits.
   uint32_t npar = 0, pend = 0;
   auto wait = [&](int i, uint32_t where) {
     if (tc::wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr)) {
@@ -691,7 +692,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_async_smem();
     if (chunk_end) s_mq[gp * 128 + row] = msum;
-    if (tid == 0 && rec) bulk_wait_read_all();  // T, E^T records read
+    if (tid == 0 && rec) bulk_wait_read_all();  // T, E records read
     tc_fence_before();
     __syncthreads();
     if (chunk_end) msum = 0.f;
