@@ -287,9 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid < 128) s_dmn[tid] = a.dm_T ? a.dm_T[(size_t)pair * kDV + tid] : 0.f;
 
   // Every barrier has at most one phase in flight.  `npar` holds the parity
-  // each thread waits for next; thread 0 also tracks in `pend` the phases it
-  // started (copies issued, MMAs committed) so that an aborting CTA drains
-  // them before it exits.
+  // each thread waits for next; the issuing threads also track in `pend`
+  // the phases they started (copies issued, MMAs committed) so that an
+  // aborting CTA drains them before it exits.
   uint32_t npar = 0, pend = 0;
   auto wait = [&](int i, uint32_t where) {
     if (wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr)) {
