@@ -53,17 +53,6 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
       "r"(smem_u32(bar))
       : "memory");
 }
-// 3-D tiled store from shared memory, tracked by the issuing thread's bulk
-// groups (bulk_commit / bulk_wait_*).
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map,
-                                             const void* src, int c0, int c1,
-                                             int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], "
-      "[%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
-      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
-      : "memory");
-}
 // Prefetch a 3-D tile (same box as the loads) into L2 only.
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0,
                                                 int c1, int c2) {
@@ -72,13 +61,6 @@ __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0,
           reinterpret_cast<uint64_t>(map)),
       "r"(c0), "r"(c1), "r"(c2)
       : "memory");
-}
-// Prefetch `bytes` (multiple of 16) of contiguous global memory into L2.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(
-                   reinterpret_cast<uint64_t>(p)),
-               "r"(bytes)
-               : "memory");
 }
 // 16 bytes global -> shared per thread without a register round trip
 // (completion by the issuing thread's async-copy groups).
@@ -267,19 +249,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* out) {
       : "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) out[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* out) {
-  uint32_t r[8];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
-        "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-#pragma unroll
-  for (int i = 0; i < 8; ++i) out[i] = __uint_as_float(r[i]);
 }
 
 // 64 consecutive columns (this warp's 32 lanes) in one load.
