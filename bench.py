@@ -2,7 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--mode train|fwd]
                     [--workload layer_1p3b|long_context|tiny] [--impl carve|reference]
-                    [--seq-len T]   (a shorter sequence, for profiler captures)
+                    [--chunk L] [--seq-len T] [--no-extras]
 
 One step = one pass of the whole hot path over one batch: the training-mode
 forward (chunk walk, gate, WY solve, state update, checkpoints) plus the
@@ -10,6 +10,17 @@ backward (reverse chunk walk and the U_b gradient reduction) -- or the
 forward alone with --mode fwd.  Inputs are synthetic (seeded, the
 distributions of chunk_gated_delta_02_b200/inputs.py) and resident in HBM
 when the timed region starts; they are larger than the 126 MB L2.
+
+On one GPU the line also carries, timed the same way (CUDA events on the
+launch stream, the same warm-up, clocks sampled throughout):
+  fwd_infer     the 1.3B-layer inference forward, with its own roofline and
+                oracle baseline
+  sweep         that forward at chunk lengths 16, 32, 64, 128: tokens/s,
+                roofline fraction, kernel family and the oracle error on one
+                (sequence, head) pair per length
+  long_context  the B=1, H=16, T=65536, dv=256 forward, with the bound its
+                sequential chunk chain sets (--no-extras skips all three;
+                --seq-len / --chunk change the main workload for profiling)
 
 Multi-GPU (torchrun, one process per GPU): every rank runs its own batch of
 the same shape (independent sequences, no data-path collective) -> weak
@@ -64,6 +75,31 @@ def fwd_bytes(K, V, e):
 
 def bwd_bytes(K, V, e):
     return e * (8 * K + 3 * V + 2)      # q k g bx v w d_o in, 6 grads out
+
+
+def roofline(flops, nbytes, pk, sustained=False):
+    """Roofline time of one launch: the larger of its FLOPs over the dense
+    bf16 tensor peak and its bytes over the HBM bandwidth (both measured).
+    Returns (seconds, bound, peak, unit)."""
+    peak_f = (pk["bf16_sus"] if sustained else pk["bf16"]) * 1e12
+    t_f, t_b = flops / peak_f, nbytes / (pk["hbm"] * 1e9)
+    if t_f > t_b:
+        return t_f, "tensor", peak_f / 1e12, "TFLOP/s"
+    return t_b, "hbm", pk["hbm"], "GB/s"
+
+
+def roof_obj(name, flops, nbytes, ms, pk, traffic=None):
+    """The `roofline` object of one kernel launch of `ms` milliseconds."""
+    t, bound, peak, unit = roofline(flops, nbytes, pk)
+    work = flops / 1e12 if bound == "tensor" else nbytes / 1e9
+    achieved = work / (ms * 1e-3)
+    return {"bound": bound, "kernel": name, "achieved": achieved,
+            "peak": peak, "unit": unit, "frac": achieved / peak,
+            "traffic": traffic,
+            "peak_src": pk["src"] + (" bf16_tflops" if bound == "tensor"
+                                     else " hbm_gbs"),
+            "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+            "roofline_ms": t * 1e3, "ms_per_launch": ms}
 
 
 def kernel_sources_sha1():
@@ -195,13 +231,19 @@ def job_tokens_per_s(tokens_per_rank, ws, ms_per_step):
     return tokens_per_rank * ws / (ms_per_step * 1e-3)
 
 
+def host_cores():
+    """(logical CPUs of the host, CPUs this process may run on)."""
+    return os.cpu_count() or 1, len(os.sched_getaffinity(0))
+
+
 def oracle_sample(cfg, mode, seed, threads=None):
     """Time the fp64 oracle on a bounded sample of the workload: `n` whole
-    (sequence, head) pairs at the full sequence length.  Returns
+    (sequence, head) pairs at the full sequence length, one thread per pair,
+    n = every CPU this process may run on (at most B * H pairs).  Returns
     (seconds, pair_tokens, n_pairs, threads)."""
     from oracle import ref
-    n = threads or max(1, len(os.sched_getaffinity(0)))
-    n = min(n, 16, cfg["B"] * cfg["H"])
+    n = threads or host_cores()[1]
+    n = max(1, min(n, cfg["B"] * cfg["H"]))
     inp = make_inputs(seed=seed, dtype=torch.bfloat16,
                       **dict(cfg, B=1, H=n))
     gro = make_grad_outputs(seed=seed, dtype=torch.bfloat16,
@@ -215,6 +257,19 @@ def oracle_sample(cfg, mode, seed, threads=None):
         ref.bwd_batch(inp, cfg["L"], gro["d_o"], pairs=pairs, threads=n)
     dt = time.perf_counter() - t0
     return dt, n * cfg["T"], n, n
+
+
+def cpu_baseline_obj(cfg, mode, seed):
+    secs, ptoks, npairs, thr = oracle_sample(cfg, mode, seed)
+    ncpu, naff = host_cores()
+    return {"value": ptoks / cfg["H"] / secs, "unit": "tokens/s",
+            "cores": thr, "host_cpus": ncpu, "affinity_cpus": naff,
+            "kind": "oracle",
+            "sample": "%d (sequence, head) pairs x %d tokens, %s, fp64, one "
+                      "thread per pair on %d of %d usable CPUs; tokens = "
+                      "pair-tokens / H" % (
+                          npairs, cfg["T"],
+                          "fwd+bwd" if mode == "train" else "fwd", thr, naff)}
 
 
 def run_reference(args, cfg, ws, rank):
@@ -241,6 +296,8 @@ def run_reference(args, cfg, ws, rank):
             "dtype": "f64", "data": "synthetic",
             "config": config_dict(args, cfg),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr,
+                             "host_cpus": host_cores()[0],
+                             "affinity_cpus": host_cores()[1],
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s",
                     "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -250,12 +307,142 @@ def run_reference(args, cfg, ws, rank):
 def config_dict(args, cfg):
     name = args.workload if not args.seq_len else "%s(T=%d)" % (args.workload,
                                                                args.seq_len)
+    if args.chunk:
+        name += "(L=%d)" % args.chunk
     return {"workload": "%s %s" % (name,
                                    "fwd+bwd" if args.mode == "train" else "fwd"),
             "B": cfg["B"], "T": cfg["T"], "H": cfg["H"], "DK": cfg["DK"],
             "DV": cfg["DV"], "L": cfg["L"], "R": cfg["R"],
             "state": "fp32", "l2": "inputs larger than L2 (no flush needed)",
             "parallelism": "independent sequences per rank (dp%d)" % args.gpus}
+
+
+def time_launches(fn, stream, warmup, iters):
+    """Average milliseconds of fn() over `iters` back-to-back calls on
+    `stream` (CUDA events around the batch, after `warmup` calls)."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    a, b = (torch.cuda.Event(enable_timing=True) for _ in range(2))
+    a.record(stream)
+    for _ in range(iters):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / iters
+
+
+def fwd_call(carve, d, L, training=False, ws=None, o=None):
+    return carve.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
+                           d["u_down"], d["u_up"], L, d.get("S0"), None,
+                           training=training, workspace=ws, o=o,
+                           want_state=False)
+
+
+def pair_error(carve, host, d, L, bh):
+    """max|delta| / max|ref| of o and S_T on one (sequence, head) pair: the
+    forward at chunk length L on the GPU against the fp64 oracle."""
+    from oracle import ref
+    import numpy as np
+    o, S_T, _, _ = carve.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["bx"],
+                                   d["w"], d["u_down"], d["u_up"], L,
+                                   d.get("S0"), None)
+    torch.cuda.synchronize()
+    b, h = bh
+    oo, SS, _ = ref.fwd_batch(host, L, pairs=[bh], threads=1)[bh]
+
+    def rel(x, y):
+        x = x.detach().double().cpu().numpy()
+        return float(np.abs(x - y).max() / np.abs(y).max())
+    return {"o": rel(o[b, :, h, :], oo), "S_T": rel(S_T[b, h], SS)}
+
+
+def extras(carve, args, pk, host, d, stream, fwd_ms_train):
+    """Inference forward, chunk-length sweep and long-context forward at
+    their full sizes (one GPU), each timed like the main step."""
+    cfg = WORKLOADS["layer_1p3b"]
+    B, T, H, DK, DV, R = (cfg[n] for n in ("B", "T", "H", "DK", "DV", "R"))
+    th = B * T * H
+    it = max(5, args.steps)
+    out = {}
+    ws = None
+    o = torch.empty_like(d["v"])
+
+    # fwd_infer: config 1, training = 0
+    L = cfg["L"]
+    _, _, _, ws = fwd_call(carve, d, L, o=o)
+    ms = time_launches(lambda: fwd_call(carve, d, L, ws=ws, o=o), stream,
+                       args.warmup, it)
+    assert carve.get_status(ws) == 0, "device status word set"
+    ro = roof_obj("carve_chunk_fwd", fwd_flops(L, DK, DV) * th,
+                  fwd_bytes(DK, DV, 2) * th, ms, pk,
+                  measured_traffic("fwd_tc", dict(cfg, L=L), th))
+    out["fwd_infer"] = {
+        "workload": "layer_1p3b fwd (training = 0)", "ms": ms,
+        "tokens_per_s": B * T / (ms * 1e-3), "roofline": ro,
+        "kernel_path": carve.fwd_path(carve.make_shape(B, T, H, DK, DV, R, L,
+                                                       torch.bfloat16)),
+        "training_fwd_ms": fwd_ms_train,
+        "cpu_baseline": (cpu_baseline_obj(cfg, "fwd", 7)
+                         if not args.no_cpu_baseline else None)}
+
+    # sweep: config 2, L in {16, 32, 64, 128}, forward only
+    sweep = []
+    for Ls in (16, 32, 64, 128):
+        shape = carve.make_shape(B, T, H, DK, DV, R, Ls, torch.bfloat16)
+        _, _, _, wsl = fwd_call(carve, d, Ls, o=o)
+        n_it = it if carve.fwd_path(shape) == "tc" else 2
+        msl = time_launches(lambda: fwd_call(carve, d, Ls, ws=wsl, o=o),
+                            stream, 1 if n_it == 2 else args.warmup, n_it)
+        assert carve.get_status(wsl) == 0, "device status word set"
+        rl = roof_obj("carve_chunk_fwd", fwd_flops(Ls, DK, DV) * th,
+                      fwd_bytes(DK, DV, 2) * th, msl, pk)
+        err = (pair_error(carve, host, d, Ls, (B - 1, H - 1))
+               if not args.no_cpu_baseline else None)
+        sweep.append({"L": Ls, "ms": msl, "tokens_per_s": B * T / (msl * 1e-3),
+                      "frac": rl["frac"], "bound": rl["bound"],
+                      "roofline_ms": rl["roofline_ms"],
+                      "kernel_path": carve.fwd_path(shape),
+                      "timed_launches": n_it,
+                      "oracle_error_pair": [B - 1, H - 1],
+                      "oracle_error": err})
+        del wsl
+    out["sweep"] = sweep
+
+    # long_context: config 3 (dv = 256, S0 != 0), forward
+    lc = WORKLOADS["long_context"]
+    hl = make_inputs(seed=3, dtype=torch.bfloat16, **lc)
+    dl = {k: (v.to(d["q"].device) if v is not None else None)
+          for k, v in hl.items()}
+    Bl, Tl, Hl, DKl, DVl, Rl, Ll = (lc[n] for n in ("B", "T", "H", "DK", "DV",
+                                                    "R", "L"))
+    ol = torch.empty_like(dl["v"])
+    _, _, _, wsc = fwd_call(carve, dl, Ll, o=ol)
+    msc = time_launches(lambda: fwd_call(carve, dl, Ll, ws=wsc, o=ol), stream,
+                        args.warmup, max(3, args.steps // 2))
+    assert carve.get_status(wsc) == 0, "device status word set"
+    thl = Bl * Tl * Hl
+    rc = roof_obj("carve_chunk_fwd", fwd_flops(Ll, DKl, DVl) * thl,
+                  fwd_bytes(DKl, DVl, 2) * thl + 2 * Bl * Hl * DVl * DKl * 4,
+                  msc, pk)
+    # the chunk chain: each (sequence, head) walks Tl / 64 blocks one after
+    # another (the content gate of a chunk needs the previous chunk's
+    # outputs), on 2 CTAs per pair (B * H * 2 = 32 of 148 SMs busy).  At the
+    # per-block latency of the 1.3B-layer inference forward that chain takes:
+    per_block_us = 1e3 * ms / (T // 64)
+    chain_ms = per_block_us * (Tl // 64) * 1e-3
+    out["long_context"] = {
+        "workload": "long_context fwd (B=1, H=16, T=65536, dk=128, dv=256, "
+                    "S0 ~ N(0, 0.01))",
+        "ms": msc, "tokens_per_s": Bl * Tl / (msc * 1e-3), "roofline": rc,
+        "kernel_path": carve.fwd_path(carve.make_shape(
+            Bl, Tl, Hl, DKl, DVl, Rl, Ll, torch.bfloat16)),
+        "chain_bound": {"blocks_per_pair": Tl // 64,
+                        "per_block_us_at_layer_1p3b": per_block_us,
+                        "chain_ms": chain_ms, "frac": chain_ms / msc,
+                        "busy_sms": 2 * Bl * Hl, "sms": 148}}
+    del dl, hl, ol, wsc
+    return out
 
 
 def main():
@@ -268,14 +455,20 @@ def main():
     ap.add_argument("--impl", choices=["carve", "reference"], default="carve")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip fwd_infer, sweep and long_context")
     ap.add_argument("--seq-len", type=int, default=None,
                     help="override T (profiler captures of a smaller case)")
+    ap.add_argument("--chunk", type=int, default=None,
+                    help="override the chunk length L of the main workload")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "carve":
         ap.error("--warmup must be >= 3")
     cfg = dict(WORKLOADS[args.workload])
     if args.seq_len:
         cfg["T"] = args.seq_len
+    if args.chunk:
+        cfg["L"] = args.chunk
     ws, rank, local = dist_init() if args.impl == "carve" else (
         int(os.environ.get("WORLD_SIZE", "1")),
         int(os.environ.get("RANK", "0")), 0)
@@ -356,23 +549,24 @@ def main():
     tokens = B * T
     value = job_tokens_per_s(tokens, ws, ms_step)
 
-    # roofline of the dominant kernel (fwd or bwd), HBM-bound
+    # roofline of the dominant kernel (fwd or bwd): max(FLOPs / bf16 peak,
+    # bytes / HBM bandwidth), both measured
     pk = peaks()
     e = 2
-    fwd_b = fwd_bytes(DK, DV, e) * B * T * H
-    bwd_b = bwd_bytes(DK, DV, e) * B * T * H
-    fwd_f = fwd_flops(L, DK, DV) * B * T * H
-    bwd_f = bwd_flops(L, DK, DV) * B * T * H
+    th = B * T * H
+    fwd_b = fwd_bytes(DK, DV, e) * th
+    bwd_b = bwd_bytes(DK, DV, e) * th
+    fwd_f = fwd_flops(L, DK, DV) * th
+    bwd_f = bwd_flops(L, DK, DV) * th
     if training and bwd_ms >= fwd_ms:
         dom, dom_ms, dom_b, dom_f = "bwd", bwd_ms, bwd_b, bwd_f
     else:
         dom, dom_ms, dom_b, dom_f = "fwd", fwd_ms, fwd_b, fwd_f
-    peak = pk["hbm"]
-    achieved = dom_b / (dom_ms * 1e-3) / 1e9
-    traffic = measured_traffic(dom + "_tc", cfg, B * T * H)
-    roof_t_fwd = max(fwd_f / (pk["bf16"] * 1e12), fwd_b / (pk["hbm"] * 1e9))
-    roof_t_all = max((fwd_f + (bwd_f if training else 0)) / (pk["bf16"] * 1e12),
-                     (fwd_b + (bwd_b if training else 0)) / (pk["hbm"] * 1e9))
+    traffic = measured_traffic(dom + "_tc" + ("_train" if dom == "fwd" and
+                                              training else ""), cfg, th)
+    roof_t_fwd = roofline(fwd_f, fwd_b, pk)[0]
+    roof_t_all = roofline(fwd_f + (bwd_f if training else 0),
+                          fwd_b + (bwd_b if training else 0), pk)[0]
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
@@ -381,23 +575,22 @@ def main():
         "config": config_dict(args, cfg),
         "kernel_path": carve.fwd_path(carve.make_shape(B, T, H, DK, DV, R, L,
                                                        dtype)),
-        "roofline": {"bound": "hbm", "kernel": "carve_chunk_" + dom,
-                     "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "peak_src": pk["src"] + " hbm_gbs",
-                     "algorithmic_bytes": dom_b, "algorithmic_flops": dom_f,
-                     "ms_per_launch": dom_ms},
+        "roofline": roof_obj("carve_chunk_" + dom, dom_f, dom_b, dom_ms, pk,
+                             traffic),
         "step_roofline": {"roofline_ms": roof_t_all * 1e3,
                           "frac": roof_t_all * 1e3 / ms_step},
         "fwd": {"ms": fwd_ms, "tokens_per_s": tokens / (fwd_ms * 1e-3),
                 "roofline_ms": roof_t_fwd * 1e3,
-                "frac": roof_t_fwd * 1e3 / fwd_ms},
+                "frac": roof_t_fwd * 1e3 / fwd_ms,
+                "training": training},
         "bwd": {"ms": bwd_ms} if training else None,
+        "workspace": {"bytes": int(wsb.numel()),
+                      "bytes_per_token_head": wsb.numel() / th,
+                      "training": training},
         # per step: the forward; the backward kernel and, with R > 0, the two
         # dU reduction kernels
         "gpu_launches": args.steps * ((2 + (2 if R > 0 else 0)) if training
                                       else 1),
-        "clocks": clk,
     }
 
     # end to end through the public API: pinned host inputs -> device, step,
@@ -478,14 +671,17 @@ def main():
                        "pipelining": "double-buffered: step i's D2H overlaps "
                                      "step i+1's H2D (separate streams)"}
 
+    line["clocks"] = clk
+    if (ws == 1 and not args.no_extras and args.workload == "layer_1p3b"
+            and not args.seq_len and not args.chunk):
+        xclk = ClockSampler(dev)
+        xclk.start()
+        time.sleep(0.3)
+        line.update(extras(carve, args, pk, host, d, stream,
+                           fwd_ms if training else None))
+        line["extras_clocks"] = xclk.stop()
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        secs, ptoks, npairs, thr = oracle_sample(cfg, args.mode, 7)
-        line["cpu_baseline"] = {
-            "value": ptoks / H / secs, "unit": "tokens/s", "cores": thr,
-            "kind": "oracle",
-            "sample": "%d (sequence, head) pairs x %d tokens, %s, fp64; "
-                      "tokens = pair-tokens / H" % (
-                          npairs, T, "fwd+bwd" if training else "fwd")}
+        line["cpu_baseline"] = cpu_baseline_obj(cfg, args.mode, 7)
     if rank == 0:
         print(json.dumps(line), flush=True)
     if ws > 1:

@@ -7,10 +7,10 @@
 
 using namespace carve;
 
-namespace {
+namespace carve {
 
-bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
-
+// The supported-shape check every entry point applies first (declared in
+// carve_internal.cuh so that the allocation-free entry point shares it).
 carve_status check_shape(const carve_shape* s) {
   if (!s) return CARVE_ERR_INVALID_ARG;
   if (s->B < 1 || s->H < 1 || s->T < 0 || s->R < 0 || s->L < 1 ||
@@ -32,6 +32,27 @@ carve_status check_shape(const carve_shape* s) {
   return CARVE_OK;
 }
 
+// Test-only knobs, read from the environment on every call (unset in
+// normal use): CARVE_TEST_WAIT_CYCLES lowers the cycles a device-side wait
+// spins before it gives up; CARVE_TEST_STALL_BLOCK makes CTA 0 of the
+// tensor-core kernels redirect the MMA commit of that block to a barrier
+// nobody waits on, so that a wait runs out and the timeout path runs.
+void test_knobs(long long* spin, int* stall_block) {
+  *spin = kSpinCycles;
+  *stall_block = -1;
+  if (const char* e = getenv("CARVE_TEST_WAIT_CYCLES")) {
+    const long long v = atoll(e);
+    if (v > 0 && v < kSpinCycles) *spin = v;
+  }
+  if (const char* e = getenv("CARVE_TEST_STALL_BLOCK")) *stall_block = atoi(e);
+}
+
+}  // namespace carve
+
+namespace {
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
 bool ptr_ok(const void* p) { return p != nullptr && aligned16(p); }
 
 // Forward kernel family for a valid shape: the tensor-core kernel where it
@@ -46,7 +67,8 @@ bool opt_ptr_ok(const void* p) { return p == nullptr || aligned16(p); }
 
 // Backward kernel family: tensor-core where the tensor-core forward ran (it
 // reads that forward's records); CARVE_BWD_PATH=generic forces the generic
-// one, which needs only the checkpoints either forward writes.
+// one, which reads the generic forward's per-block fp32 checkpoints (a
+// tensor-core workspace has none and is refused).
 bool use_tc_bwd(const carve_shape& s) {
   const char* env = getenv("CARVE_BWD_PATH");
   if (env && strcmp(env, "generic") == 0) return false;
@@ -59,7 +81,8 @@ extern "C" {
 
 size_t carve_workspace_bytes(const carve_shape* shape, int training) {
   if (check_shape(shape) != CARVE_OK) return 0;
-  return ws_layout(*shape, training != 0).total;
+  return ws_layout(*shape, training != 0, use_tc_fwd(*shape, training != 0))
+      .total;
 }
 
 const char* carve_status_str(carve_status s) {
@@ -99,7 +122,8 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   if (!opt_ptr_ok(S0) || !opt_ptr_ok(m0) || !opt_ptr_ok(S_T) ||
       !opt_ptr_ok(m_T))
     return CARVE_ERR_INVALID_ARG;
-  const WsLayout L = ws_layout(s, training != 0);
+  const bool tc = use_tc_fwd(s, training != 0);
+  const WsLayout L = ws_layout(s, training != 0, tc);
   if (!workspace || !aligned16(workspace)) return CARVE_ERR_WORKSPACE;
   if (workspace_bytes < L.total) return CARVE_ERR_WORKSPACE;
 
@@ -117,8 +141,8 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   a.tc_rec = training && L.tc_rec ? (uint8_t*)(ws + L.tc_rec) : nullptr;
   a.gin = training && L.gin ? (float*)(ws + L.gin) : nullptr;
   a.hdr = (WsHeader*)ws;
-  cudaError_t e = use_tc_fwd(s, training != 0)
-                      ? launch_fwd_tc(a, (cudaStream_t)stream)
+  test_knobs(&a.spin, &a.stall_block);
+  cudaError_t e = tc ? launch_fwd_tc(a, (cudaStream_t)stream)
                       : launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
@@ -148,7 +172,11 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   if (!opt_ptr_ok(dS_T) || !opt_ptr_ok(dm_T) || !opt_ptr_ok(dS0) ||
       !opt_ptr_ok(dm0))
     return CARVE_ERR_INVALID_ARG;
-  const WsLayout L = ws_layout(s, true);
+  // the workspace layout of the forward family this backward reads (a
+  // tensor-core workspace is too small for the generic backward's layout:
+  // that mismatch is refused here)
+  const bool tc = use_tc_bwd(s);
+  const WsLayout L = ws_layout(s, true, tc);
   if (!workspace || !aligned16(workspace)) return CARVE_ERR_WORKSPACE;
   if (workspace_bytes < L.total) return CARVE_ERR_WORKSPACE;
 
@@ -168,8 +196,8 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbx = db_x; a.dw = dw;
   a.du_down = du_down; a.du_up = du_up; a.dS0 = dS0; a.dm0 = dm0;
   a.hdr = (WsHeader*)ws;
-  cudaError_t e = use_tc_bwd(s)
-                      ? launch_bwd_tc(a, (cudaStream_t)stream)
+  test_knobs(&a.spin, &a.stall_block);
+  cudaError_t e = tc ? launch_bwd_tc(a, (cudaStream_t)stream)
                       : launch_bwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }

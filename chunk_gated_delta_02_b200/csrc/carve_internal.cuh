@@ -14,6 +14,9 @@ constexpr uint32_t kWsMagic = 0xCA7E0001u;
 constexpr size_t kHeaderBytes = 256;
 constexpr int kMaxR = 64;
 constexpr int kMaxBlock = 64;  // tokens per solver block (C = min(L, 64))
+// Cycles a device-side wait spins before it records CARVE_ERR_TIMEOUT
+// (about 1 s at the B200's clocks).
+constexpr long long kSpinCycles = 1LL << 31;
 
 // Device status word at the start of the workspace.
 struct WsHeader {
@@ -47,14 +50,17 @@ inline bool tc_fwd_shape(const carve_shape& s, bool training) {
 }
 static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
 
-// Layout of the workspace (byte offsets, 256-aligned).
+// Layout of the workspace (byte offsets, 256-aligned).  `tc` says which
+// forward family writes it (the tensor-core one keeps only what its own
+// backward reads).
 struct WsLayout {
   int C;    // tokens per solver block
   int NB;   // blocks per sequence
   int NC;   // chunks per sequence
-  size_t ck_S;         // [B*H][NB+1][DV][DK] fp32 block-start states
+  int ck_slots;        // fp32 states kept per pair: NB + 1 (generic), 1 (tc)
+  size_t ck_S;         // [B*H][ck_slots][DV][DK] fp32 block-start states
   size_t ck_m;         // [B*H][NC][DV] fp32 chunk gate inputs m_c
-  size_t scratch;      // per-pair fp32 scratch of the generic kernels
+  size_t scratch;      // per-pair fp32 scratch (generic kernels; tc: dp | dh)
   size_t scratch_per_pair;  // floats
   size_t du;           // [B*H][R*DV + DK*R] fp32 per-pair U_b gradients
   size_t tc_rec;       // [B*H][NB] tensor-core records (kTcRecBytes each)
@@ -73,26 +79,34 @@ inline size_t generic_bwd_scratch_floats(int C, int DK, int DV) {
   return 9 * (size_t)C * DK + 7 * (size_t)C * DV + 2 * (size_t)DV * DK;
 }
 
-inline WsLayout ws_layout(const carve_shape& s, bool training) {
+// tc: the tensor-core forward writes this workspace.  It needs no generic
+// scratch; in training it keeps the final fp32 state only (its backward
+// walks the bf16 state records), the chunk gate inputs, the records, and
+// scratch for the backward's per-chunk gate gradients.
+inline WsLayout ws_layout(const carve_shape& s, bool training, bool tc) {
   WsLayout w{};
   w.C = block_len(s.L);
   w.NB = s.T / w.C;
   w.NC = s.T / s.L;
+  w.ck_slots = tc ? 1 : w.NB + 1;
   const size_t P = (size_t)s.B * s.H;
+  const size_t NCc = (size_t)(w.NC > 0 ? w.NC : 1);
   size_t off = kHeaderBytes;
   if (training) {
     w.ck_S = off;
-    off = align256(off + P * (size_t)(w.NB + 1) * s.DV * s.DK * 4);
+    off = align256(off + P * (size_t)w.ck_slots * s.DV * s.DK * 4);
     w.ck_m = off;
-    off = align256(off + P * (size_t)(w.NC > 0 ? w.NC : 1) * s.DV * 4);
+    off = align256(off + P * NCc * s.DV * 4);
   }
-  size_t sc = generic_fwd_scratch_floats(w.C, s.DK, s.DV);
-  if (training) {
-    size_t sb = generic_bwd_scratch_floats(w.C, s.DK, s.DV);
-    sc = sc > sb ? sc : sb;
-    // the tensor-core backward keeps per-chunk gate records here instead
-    const size_t gr = (size_t)(w.NC > 0 ? w.NC : 1) * (s.DK + s.R);
-    sc = sc > gr ? sc : gr;
+  size_t sc = 0;
+  if (!tc) {
+    sc = generic_fwd_scratch_floats(w.C, s.DK, s.DV);
+    if (training) {
+      const size_t sb = generic_bwd_scratch_floats(w.C, s.DK, s.DV);
+      sc = sc > sb ? sc : sb;
+    }
+  } else if (training) {
+    sc = NCc * (s.DK + s.R);  // the backward's per-chunk gate gradients
   }
   w.scratch_per_pair = sc;
   w.scratch = off;
@@ -100,11 +114,11 @@ inline WsLayout ws_layout(const carve_shape& s, bool training) {
   if (training) {
     w.du = off;
     off = align256(off + P * ((size_t)s.R * s.DV + (size_t)s.DK * s.R) * 4);
-    if (tc_shape(s)) {
+    if (tc) {
       w.tc_rec = off;
       off = align256(off + P * (size_t)w.NB * kTcRecBytes);
       w.gin = off;
-      off = align256(off + P * (size_t)w.NC * (s.DK + s.R) * 4);
+      off = align256(off + P * NCc * (s.DK + s.R) * 4);
     }
   }
   w.total = off;
@@ -135,6 +149,8 @@ struct FwdArgs {
   uint8_t* tc_rec;  // tensor-core records; NULL unless training
   float* gin;       // chunk gate inputs p_c | h_c; NULL unless training
   WsHeader* hdr;
+  long long spin;   // cycles a device-side wait spins before it gives up
+  int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
 };
 
 struct BwdArgs {
@@ -151,7 +167,14 @@ struct BwdArgs {
   void *dq, *dk, *dv, *dg, *dbx, *dw;
   float *du_down, *du_up, *dS0, *dm0;
   WsHeader* hdr;
+  long long spin;   // cycles a device-side wait spins before it gives up
+  int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
 };
+
+// Host-side checks (carve_api.cu): the supported-shape check of every entry
+// point, and the test-only wait limit / stall knobs.
+carve_status check_shape(const carve_shape* s);
+void test_knobs(long long* spin, int* stall_block);
 
 // Host launchers (carve_generic.cu).
 cudaError_t launch_fwd_generic(const FwdArgs& a, int dtype, cudaStream_t st);

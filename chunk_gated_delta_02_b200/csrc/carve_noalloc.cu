@@ -13,10 +13,9 @@
 // scratch placed in the file-scope device array below instead of a
 // workspace.  The array is part of the library's device image, so every
 // GPU that loads libcarve holds CARVE_NOALLOC_SCRATCH_BYTES of it until the
-// process exits.  Its device address is looked up once per device, on the
-// first call made with that device current.
-#include <mutex>
-
+// process exits.  Its device address is looked up on every call, with the
+// caller's device current (a host-side query that allocates nothing; a
+// pointer cached across calls could outlive a device reset).
 #include "carve_internal.cuh"
 
 namespace {
@@ -29,26 +28,14 @@ using namespace carve;
 static __device__ __align__(256) unsigned char
     g_noalloc_scratch[CARVE_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_mu;
-void* g_addr[kMaxDevices];     // device address of g_noalloc_scratch
-bool g_ready[kMaxDevices];
-
-// Once per device, with that device current: resolve the array's device
-// address (host code cannot use the symbol itself as a pointer).
+// The array's device address on the current device (host code cannot use
+// the symbol itself as a pointer: in host code it names a host-side
+// stand-in).  Looked up on every call.
 carve_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return CARVE_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return CARVE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_ready[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
-      return CARVE_ERR_CUDA;
-    g_addr[dev] = p;
-    g_ready[dev] = true;
-  }
-  *out = g_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p)
+    return CARVE_ERR_CUDA;
+  *out = p;
   return CARVE_OK;
 }
 
@@ -63,11 +50,9 @@ extern "C" carve_status carve_chunk_fwd_noalloc(
     const void* g, const void* b_x, const void* w, const void* u_down,
     const void* u_up, const float* S0, const float* m0, void* o, float* S_T,
     float* m_T, void* stream) {
-  if (!shape || shape->B < 1 || shape->H < 1 || shape->T < 0 ||
-      shape->R < 0 || shape->L < 1 || shape->DK < 1 || shape->DV < 1)
-    return CARVE_ERR_INVALID_ARG;
-  // same supported set as carve_chunk_fwd (0 = invalid or unsupported)
-  if (carve_workspace_bytes(shape, 0) == 0) return CARVE_ERR_UNSUPPORTED;
+  // the supported set and status codes of carve_chunk_fwd
+  carve_status st = check_shape(shape);
+  if (st != CARVE_OK) return st;
   const carve_shape& s = *shape;
   if (s.T > 0 && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) ||
                   !ptr_ok(b_x) || !ptr_ok(w) || !ptr_ok(o)))
@@ -85,7 +70,7 @@ extern "C" carve_status carve_chunk_fwd_noalloc(
   if (need > CARVE_NOALLOC_SCRATCH_BYTES) return CARVE_ERR_WORKSPACE;
 
   void* base = nullptr;
-  carve_status st = scratch_address(&base);
+  st = scratch_address(&base);
   if (st != CARVE_OK) return st;
 
   FwdArgs a{};
@@ -99,6 +84,8 @@ extern "C" carve_status carve_chunk_fwd_noalloc(
   a.scratch = (float*)((char*)base + kHeaderBytes);
   a.scratch_per_pair = per_pair;
   a.hdr = (WsHeader*)base;
+  a.spin = kSpinCycles;
+  a.stall_block = -1;
   cudaError_t e = launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }

@@ -65,9 +65,9 @@ constexpr uint32_t SM_X = 1024;      // g half sums | dlog gamma | dp   128 f32
 constexpr uint32_t SM_GAM = 1536;    // gamma | dg hand-off | dh parts  128 f32
 constexpr uint32_t SM_W = 2048;      // w_t                 64 f32
 constexpr uint32_t SM_DW = 2304;     // dw sums | dh        64 f32
-constexpr uint32_t SM_BAR = 2560;    // 11 mbarriers
-constexpr uint32_t SM_TMEM = 2648;
-constexpr uint32_t SM_ABORT = 2652;
+constexpr uint32_t SM_BAR = 2560;    // kNumBars mbarriers
+constexpr uint32_t SM_TMEM = 2664;
+constexpr uint32_t SM_ABORT = 2668;
 constexpr uint32_t kSmemBytes = 232448;
 static_assert(R_SM + 2688 <= kSmemBytes, "small region");
 static_assert(R_PQ == R_MP + 16384 && R_TT == R_PQ + 8192, "G2 blocks");
@@ -84,7 +84,9 @@ constexpr int B_7 = 7;     // MMA S11
 constexpr int B_PRE = 8;   // v, g, b_x, E and T records
 constexpr int B_7B = 9;    // MMA S11, the D8 half (issued by thread 256)
 constexpr int B_5B = 10;   // MMA S9, the dW^T and dS half (issued by thread 256)
-constexpr int kNumBars = 11;
+constexpr int B_TEST = 11; // test only: the redirected commit of a stalled block
+constexpr int B_FIN = 12;  // an aborting CTA: thread 288's MMAs not yet committed
+constexpr int kNumBars = 13;
 static_assert(SM_BAR + 8 * kNumBars <= SM_TMEM, "mbarriers");
 
 // TMEM columns
@@ -268,8 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int c0 = gp * 32;
     const float* src = a.dS_T ? a.dS_T + (size_t)pair * SZ + (size_t)row * kDK + c0
                               : nullptr;
-    const float* sfin = a.ck_S + ((size_t)pair * (NB + 1) + NB) * SZ +
-                        (size_t)row * kDK + c0;
+    const float* sfin = a.ck_S + (size_t)pair * SZ + (size_t)row * kDK + c0;
     float vals[32], prod[32];
 #pragma unroll
     for (int i = 0; i < 32; i += 4) {
@@ -291,8 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the phases they started (copies issued, MMAs committed) so that an
   // aborting CTA drains them before it exits.
   uint32_t npar = 0, pend = 0;
+  bool der_open = false;  // thread 288 issued S4's MMAs, S6 has not committed them
   auto wait = [&](int i, uint32_t where) {
-    if (wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr)) {
+    if (wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr, a.spin)) {
       npar ^= 1u << i;
       pend &= ~(1u << i);
     }
@@ -488,8 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     fence_async_smem();
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
 
     // ---- S3: G = X [K^; kap^]^T (one N = 128 product per k-step):
     //      columns 0-63 [M; P_k], 64-127 [A; P_kap]
@@ -502,8 +503,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + T_G, desc_kmajor_sw128(x0 + kx),
                   desc_kmajor_sw128(khp0 + kx), ID_KK128, ks > 0);
       }
-      umma_commit(bars + B_1);
-      mark(B_1);
+      // test only: CTA 0 of a chosen block commits to a barrier nobody
+      // waits on, so the wait for S3 below runs out (the products still
+      // complete and are drained before the CTA exits)
+      const int bm = (ib == a.stall_block && blockIdx.x == 0) ? B_TEST : B_1;
+      umma_commit(bars + bm);
+      mark(bm);
     }
 
     // ---- S4: dS~ = dS Diag(gamma) (TMEM, and its bf16 operand over the
@@ -540,6 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   desc_kmajor_sw128(dsb0 + (ks >> 2) * 16384 + (ks & 3) * 32),
                   desc_kmajor_sw128(kp0 + (ks >> 2) * 16384 + (ks & 3) * 32),
                   ID_KK64_NA, ks > 0);
+      der_open = true;
     }
     wait(B_1, 13);
     tc_fence_after();
@@ -569,8 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_st_wait();
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
 
     // ---- S6: dE^T = -dS~ kap^T (issued in S4) - dO^T P_kap
     if (tid == 288) {
@@ -583,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   desc_mnmajor_sw128(pq0 + ks * 2048, 8192), ID_MM64_NA, 1);
       umma_commit(bars + B_3);
       mark(B_3);
+      der_open = false;
     }
     wait(B_3, 14);
     tc_fence_after();
@@ -598,8 +604,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
     if (tid == 0) {
       tc_fence_after();
       const uint32_t ro0 = smem_u32(sm + R_RO), tt0 = smem_u32(sm + R_TT);
@@ -624,8 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
 
     // ---- S9: G2raw = [dR; dO] [E; W]^T, dW^T, dS += [dR; dO]^T [K~; Q~],
     //      D7^T = S^T [dR; dO]^T.  Two issuers with their own commits:
@@ -687,8 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
 
     // ---- S11: D7^T += [-kap^; K^]^T G2^T ; D8^T = X^T G2 + dS~^T [E; W]^T
     //      (into the columns G2 left); meanwhile dv, dw (16 tokens per group)
@@ -932,6 +935,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid < 32) cp_async_wait_all();  // (an aborted walk may leave one in flight)
   // ---- dS0, dm0; an aborted CTA first lets its copies and MMAs land
   if (*s_abort) {
+    if (tid == 288 && der_open) {  // S4's MMAs were issued, S6 never committed them
+      umma_commit(bars + B_FIN);
+      mark(B_FIN);
+    }
     if (tid == 0 || tid == 256 || tid == 288)  // the threads that start copies and MMAs
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) drain_bar(bars + i, (npar >> i) & 1u);

@@ -75,8 +75,8 @@ constexpr uint32_t SM_M = 1280;        // m_v                128 f32
 constexpr uint32_t SM_H = 1792;        // U_down m            64 f32
 constexpr uint32_t SM_GAM1 = 2048;     // gamma_j (odd blocks)  128 f32
 constexpr uint32_t SM_BAR = 2560;      // kNumBars mbarriers
-constexpr uint32_t SM_TMEM = 2624;     // TMEM base address
-constexpr uint32_t SM_ABORT = 2628;    // abort flag
+constexpr uint32_t SM_TMEM = 2640;     // TMEM base address
+constexpr uint32_t SM_ABORT = 2644;    // abort flag
 constexpr uint32_t kSmallBytes = 2688;
 constexpr uint32_t OFF_UU = 215808;    // U_up^T bf16 [kRMax][kUuLd]   8.5 KB
 constexpr int kUuLd = 128 + 8;         // row pitch: 16 B of padding per row
@@ -94,7 +94,10 @@ constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
 constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
 constexpr int B_X = 6;     // dv = 256: the other CTA's half of U_down m arrived
 constexpr int B_WK = 7;    // S += W^T K^ (issued with MMA 2)
-constexpr int kNumBars = 8;
+constexpr int B_TEST = 8;  // test only: the redirected commit of a stalled block
+constexpr int B_FIN = 9;   // an aborting CTA: thread 0's D1 MMAs not yet committed
+constexpr int kNumBars = 10;
+static_assert(SM_BAR + 8 * kNumBars <= SM_TMEM, "mbarriers");
 
 // TMEM columns (fp32, lanes = rows)
 constexpr uint32_t TM_S = 0;     // state S          [v][j]     128 cols
@@ -192,8 +195,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the phases they started (copies issued, MMAs committed) so that an
   // aborting CTA drains them before it exits.
   uint32_t npar = 0, pend = 0;
+  bool d1_open = false;  // thread 0 issued D1, the commit after G is still to come
   auto wait = [&](int i, uint32_t where) {
-    if (tc::wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr)) {
+    if (tc::wait_bar(bars + i, (npar >> i) & 1u, where, s_abort, a.hdr, a.spin)) {
       npar ^= 1u << i;
       pend &= ~(1u << i);
     }
@@ -392,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
                     desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
         }
+        d1_open = true;
       }
       wait(B_VGB, 1);
       const int rr = tid >> 3, ch = tid & 7;  // token rows rr, rr + 32; 16-byte chunk
@@ -435,8 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                       sm + OFF_RB, s_p, 16384, tid - 32, kThreads - 32);
     fence_async_smem();
     if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
     if (tid == 0) {  // the raw v, g, b_x buffers are free for the next block
       if (ib + 1 < NB) issue_vgb(ib + 1);
       tc_fence_after();
@@ -447,8 +451,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
                   desc_kmajor_sw128(khp0 + kx), ID_N128, ks > 0);
       }
-      umma_commit(bars + B_M1);
-      mark(B_M1);
+      // test only: CTA 0 of a chosen block commits to a barrier nobody
+      // waits on, so the wait for MMA 1 below runs out (the products still
+      // complete and are drained before the CTA exits)
+      const int bm = (ib == a.stall_block && blockIdx.x == 0) ? B_TEST : B_M1;
+      umma_commit(bars + bm);
+      mark(bm);
+      d1_open = false;
     }
     wait(B_M1, 3);
     tc_fence_after();
@@ -557,8 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp >= 8 && ib + 1 < NB) keys(ib + 1);
     fence_async_smem();
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;
 
     // ---- 5. MMA 3a: E^T = R^T T^T; training also E = T R (lanes 0-63; the
     //         rows of MY past T only feed the unused lanes) for the record
@@ -607,8 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
     }
     tc_fence_before();
-    __syncthreads();
-    if (*s_abort) break;
+    if (__syncthreads_or(*s_abort)) break;
 
     // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S -= E^T kap^ (W^T K^
     //      was added with MMA 2)
@@ -669,11 +676,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c8 = 0; c8 < 4; ++c8)
         st_chunk(sm + OFF_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
                  sv + c8 * 8);
-      // fp32 checkpoints: the final state only (the backward of this family
-      // reads the bf16 records; the fp32 state ends dlog gamma of the last block)
+      // fp32 checkpoint: the final state only, one slot per pair (the
+      // backward of this family reads the bf16 records; the fp32 state ends
+      // dlog gamma of the last block)
       float* ck = (a.ck_S && ib == NB - 1)
-                      ? a.ck_S + ((size_t)pair * (NB + 1) + NB) * SZ +
-                            (size_t)row * kDK + c0
+                      ? a.ck_S + (size_t)pair * SZ + (size_t)row * kDK + c0
                       : nullptr;
       float* st = (a.S_T && ib == NB - 1)
                       ? a.S_T + ((size_t)pair * DVt + v0 + row) * kDK + c0
@@ -699,6 +706,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   if (*s_abort) {
+    if (tid == 0 && d1_open) {  // D1 was issued, the commit after G never came
+      umma_commit(bars + B_FIN);
+      mark(B_FIN);
+    }
     if (tid == 0 || tid == 128 || tid == 256)  // the threads that start copies and MMAs
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) tc::drain_bar(bars + i, (npar >> i) & 1u);

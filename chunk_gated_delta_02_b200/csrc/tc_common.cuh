@@ -310,21 +310,21 @@ __device__ __forceinline__ void kappa_block(const uint8_t* kh_src, uint8_t* kh,
   }
 }
 
-constexpr long long kSpinCycles = 1LL << 31;  // ~1 s before a wait gives up
-
-// Bounded wait on an mbarrier phase.  On expiry: record CARVE_ERR_TIMEOUT
-// and the wait site in the workspace header, raise the CTA abort flag and
-// return (the caller keeps its barrier sequence; the block loop exits at
-// its next check of the flag).
+// Bounded wait on an mbarrier phase: gives up after `spin` cycles
+// (kSpinCycles unless a test lowers it).  On expiry: record
+// CARVE_ERR_TIMEOUT and the wait site in the workspace header, raise the CTA
+// abort flag and return (the caller keeps its barrier sequence; every later
+// wait returns at once, and the block loop exits at its next block-wide
+// check of the flag, which every thread takes together).
 // Returns whether the phase completed.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
                                          uint32_t where,
                                          volatile uint32_t* abort_flag,
-                                         WsHeader* hdr) {
+                                         WsHeader* hdr, long long spin) {
   const long long t0 = clock64();
   while (!*abort_flag) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > kSpinCycles) {
+    if (clock64() - t0 > spin) {
       atomicExch(&hdr->status, (uint32_t)CARVE_ERR_TIMEOUT);
       hdr->where = where;
       *abort_flag = 1;
@@ -334,8 +334,9 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity,
 }
 
 // Bounded wait that ignores the abort flag: before a CTA that aborted
-// exits, its copies and MMAs still in flight are given up to ~1 s each to
-// land (their shared and tensor memory must outlive them).
+// exits, its copies and MMAs still in flight are given up to kSpinCycles
+// (~1 s) each to land (their shared and tensor memory must outlive them);
+// the limit is never lowered.
 __device__ __forceinline__ void drain_bar(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
   while (!ptx::mbar_try_wait(bar, parity))

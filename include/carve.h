@@ -71,10 +71,15 @@ typedef struct {
 
 /*
  * Bytes of device workspace carve_chunk_fwd / carve_chunk_bwd need for this
- * shape.  training != 0 adds the per-block state checkpoints and per-chunk
- * gate inputs that carve_chunk_bwd reads.  Returns 0 for an invalid or
- * unsupported shape.  The workspace starts with a 256-byte header holding
- * the device status word (see carve_get_status).
+ * shape.  training != 0 adds what carve_chunk_bwd reads: on the tensor-core
+ * path the final fp32 state, the per-chunk gate inputs and the per-block
+ * records (bf16 state operand, E and T; 56 KiB per 64-token block); on the
+ * generic path the fp32 state at every block start.  Returns 0 for an
+ * invalid or unsupported shape.  The workspace starts with a 256-byte
+ * header holding the device status word (see carve_get_status).  The size
+ * depends on which kernel family runs (carve_fwd_path; the environment
+ * override CARVE_FWD_PATH=generic selects the generic one), so query it
+ * under the same setting as the calls that use it.
  */
 size_t carve_workspace_bytes(const carve_shape* shape, int training);
 
@@ -157,8 +162,10 @@ carve_status carve_chunk_bwd(const carve_shape* shape,
  *   - Needs 256 + B*H*(4*C*DK + 4*C*DV + DV*DK)*4 bytes of that array,
  *     C = min(L, 64); a larger shape returns CARVE_ERR_WORKSPACE and
  *     enqueues nothing.
- *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, which allocates nothing).  The first call on a
+ *     device may also load the library's device code there: make that first
+ *     call before any stream capture.
  *   - Every call on a device shares the one array and leaves its contents
  *     behind; the kernel writes every scratch element before reading it, so
  *     nothing has to be cleared between calls.  Calls whose kernels overlap
@@ -180,8 +187,16 @@ carve_status carve_chunk_fwd_noalloc(const carve_shape* shape,
  * Synchronises `stream`, then reads the device status word that kernels
  * write into the workspace header (CARVE_OK, or CARVE_ERR_TIMEOUT when a
  * bounded device-side wait gave up; the kernel then skipped the rest of its
- * work and left its outputs unspecified).  The word is sticky until
- * carve_reset_status.
+ * work and left its outputs unspecified; CARVE_ERR_WORKSPACE when a
+ * backward was given a workspace the other kernel family wrote).  The word
+ * is sticky until carve_reset_status.
+ *
+ * Every wait of the tensor-core kernels on a copy, an MMA or the partner
+ * CTA gives up after about 1 s (2^31 cycles).  Two environment variables
+ * exist for tests of that path only: CARVE_TEST_WAIT_CYCLES lowers the
+ * limit, and CARVE_TEST_STALL_BLOCK=n makes CTA 0 send the commit of block
+ * n's first MMA batch to a barrier nobody waits on, so that its wait runs
+ * out (the MMAs still complete and are waited for before the CTA exits).
  */
 carve_status carve_get_status(const void* workspace, void* stream);
 

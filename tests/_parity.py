@@ -105,7 +105,18 @@ def bwd_errors(inp, L, grads, pairs=None, du_heads=()):
     return acc.errors()
 
 
+# (what, tol, {tensor: max|delta| / max|ref|}) of every comparison made in
+# this process; tests/conftest.py prints them at the end of the run so that
+# the log shows the headroom under each tolerance.
+MARGINS = []
+
+
+def record(what, tol, errs):
+    MARGINS.append((what, tol, dict(errs)))
+
+
 def assert_within(errs, tol, what=""):
+    record(what, tol, errs)
     bad = {k: v for k, v in errs.items() if not (v <= tol)}
     assert not bad, "%s exceeds %.1e: %s (all: %s)" % (what, tol, bad, errs)
 

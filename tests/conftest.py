@@ -26,3 +26,20 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Headroom of every parity comparison of the run: the worst tensor of
+    each (max|delta| / max|ref| and its share of the tolerance)."""
+    mod = sys.modules.get("_parity")
+    margins = getattr(mod, "MARGINS", None) if mod else None
+    if not margins:
+        return
+    tr = terminalreporter
+    tr.write_sep("-", "parity margins (max|delta| / max|ref|, worst tensor)")
+    for what, tol, errs in margins:
+        if not errs:
+            continue
+        name, worst = max(errs.items(), key=lambda kv: kv[1])
+        tr.write_line("%-48s %-8s %.2e  (%3.0f%% of %.0e)" % (
+            what[:48], name, worst, 100.0 * worst / tol, tol))

@@ -77,10 +77,39 @@ def test_status_strings_and_path(lib):
                   dict(dtype=carve.CARVE_FP32), dict(DV=192)):
         assert path(**dict(tc, **other)) == "generic", other
     # training on the tensor-core family adds the per-block records
-    # (56 KiB per block and pair) on top of the fp32 checkpoints
-    B, H, NB = 2, 3, 128 // 64
-    extra = ws_bytes(lib, shape(**tc), 1) - ws_bytes(lib, shape(**tc), 0)
-    assert extra >= B * H * NB * 57344 + B * H * (NB + 1) * 128 * 128 * 4
+    # (56 KiB per block and pair), one fp32 state per pair (the final one),
+    # the chunk gate inputs and gradients, and the per-pair dU partials
+    B, H, NB, NC, R = 2, 3, 128 // 64, 128 // 64, 32
+    a256 = lambda x: (x + 255) // 256 * 256
+    expect = (256 + a256(B * H * 128 * 128 * 4) + a256(B * H * NC * 128 * 4)
+              + a256(B * H * NC * (128 + R) * 4)
+              + a256(B * H * (R * 128 + 128 * R) * 4)
+              + a256(B * H * NB * 57344) + a256(B * H * NC * (128 + R) * 4))
+    assert ws_bytes(lib, shape(**tc), 1) == expect
+    # the tensor-core inference forward needs the header only
+    assert ws_bytes(lib, shape(**tc), 0) == 256
+
+
+def test_workspace_follows_the_kernel_family(lib, monkeypatch):
+    # the generic kernels keep the fp32 state at every block start and a
+    # per-pair scratch, so the same shape needs more when they are selected
+    tc = shape(DK=128, DV=128, R=32, L=64, T=128, dtype=carve.CARVE_BF16)
+    n_tc = (ws_bytes(lib, tc, 0), ws_bytes(lib, tc, 1))
+    monkeypatch.setenv("CARVE_FWD_PATH", "generic")
+    assert lib.carve_fwd_path(ctypes.byref(tc)).decode() == "generic"
+    n_ge = (ws_bytes(lib, tc, 0), ws_bytes(lib, tc, 1))
+    B, H, NB = 2, 3, 2
+    assert n_ge[1] - n_ge[0] >= B * H * (NB + 1) * 128 * 128 * 4
+    assert n_ge[0] > n_tc[0]
+    # a backward given a workspace sized for the tensor-core forward while
+    # the generic backward is selected is refused on the host
+    monkeypatch.delenv("CARVE_FWD_PATH")
+    monkeypatch.setenv("CARVE_BWD_PATH", "generic")
+    ins = [FAKE] * 8 + [FAKE, None, None]
+    outs = [FAKE] * 8 + [None, None]
+    rc = lib.carve_chunk_bwd(ctypes.byref(tc), *ins, FAKE,
+                             ctypes.c_size_t(n_tc[1]), *outs, None)
+    assert carve.STATUS[rc] == "CARVE_ERR_WORKSPACE"
 
 
 FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
@@ -133,6 +162,35 @@ def test_bwd_validation_returns_before_launch(lib):
     # first, so that this call can never reach a launch)
     assert ws_bytes(lib, s, 0) < need
     assert call(s, FAKE, ws_bytes(lib, s, 0)) == 3
+
+
+def call_noalloc(lib, s, **over):
+    f = lib.carve_chunk_fwd_noalloc
+    f.argtypes = [ctypes.POINTER(carve.Shape)] + [ctypes.c_void_p] * 14
+    f.restype = ctypes.c_int
+    args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, bx=FAKE, w=FAKE, ud=FAKE,
+                uu=FAKE, S0=None, m0=None, o=FAKE, S_T=None, m_T=None)
+    args.update(over)
+    return f(ctypes.byref(s) if s is not None else None, args["q"], args["k"],
+             args["v"], args["g"], args["bx"], args["w"], args["ud"],
+             args["uu"], args["S0"], args["m0"], args["o"], args["S_T"],
+             args["m_T"], None)
+
+
+def test_noalloc_validation_matches_the_workspace_entry_point(lib):
+    # the allocation-free forward applies the same shape check and returns
+    # the same codes as carve_chunk_fwd, all before any launch
+    s = shape()
+    need = ws_bytes(lib, s, 0)
+    for bad in (dict(dtype=7), dict(B=0), dict(L=0), dict(DK=24),
+                dict(T=100), dict(R=65), dict(L=96)):
+        want = call_fwd(lib, shape(**bad), FAKE, need)
+        assert want in (1, 2), bad
+        assert call_noalloc(lib, shape(**bad)) == want, bad
+    assert call_noalloc(lib, None) == 1
+    assert call_noalloc(lib, s, q=None) == 1
+    assert call_noalloc(lib, s, v=MIS) == 1
+    assert call_noalloc(lib, s, m_T=MIS) == 1
 
 
 def test_binding_refuses_cpu_tensors():

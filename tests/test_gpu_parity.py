@@ -77,13 +77,14 @@ def test_shapes_fwd_bwd(shape, dt):
         inp["u_down"] = (inp["u_down"].float() * 25).to(DT[dt])
         inp["u_up"] = (inp["u_up"].float() * 25).to(DT[dt])
     _rand_state(inp, 12)
-    assert_within(fwd_errors(inp, L), TOL[DT[dt]], "fwd")
+    tag = "x".join(map(str, shape)) + " " + dt
+    assert_within(fwd_errors(inp, L), TOL[DT[dt]], "fwd " + tag)
     gro = grad_outputs(cfg, 13, DT[dt])
     gen = torch.Generator().manual_seed(14)
     gro["dS_T"] = torch.randn((B, H, DV, DK), generator=gen)
     gro["dm_T"] = torch.randn((B, H, DV), generator=gen)
     assert_within(bwd_errors(inp, L, gro, du_heads=range(H)), TOL[DT[dt]],
-                  "bwd")
+                  "bwd " + tag)
 
 
 def test_empty_sequence_returns_initial_state():
@@ -205,7 +206,7 @@ def test_tensor_core_forward_matches_oracle_and_generic(case, monkeypatch):
     _rand_state(inp, 22)
     shape = carve.make_shape(B, T, H, 128, 128, R, L, torch.bfloat16)
     assert carve.fwd_path(shape) == "tc"
-    assert_within(fwd_errors(inp, L), 1e-2, "tensor-core fwd")
+    assert_within(fwd_errors(inp, L), 1e-2, "tensor-core fwd %s" % (case,))
     _, o_tc, S_tc, m_tc, _ = run_fwd(inp, L, training=True)
     monkeypatch.setenv("CARVE_FWD_PATH", "generic")
     assert carve.fwd_path(shape) == "generic"
@@ -235,7 +236,7 @@ def test_tensor_core_forward_dv256_matches_oracle_and_generic(case, monkeypatch)
     _rand_state(inp, 42)
     shape = carve.make_shape(B, T, H, 128, 256, R, L, torch.bfloat16)
     assert carve.fwd_path(shape) == "tc"
-    assert_within(fwd_errors(inp, L), 1e-2, "tensor-core fwd, dv = 256")
+    assert_within(fwd_errors(inp, L), 1e-2, "tc fwd dv=256 %s" % (case,))
     _, o_tc, S_tc, m_tc, _ = run_fwd(inp, L)
     monkeypatch.setenv("CARVE_FWD_PATH", "generic")
     _, o_g, S_g, m_g, _ = run_fwd(inp, L)
@@ -267,20 +268,22 @@ def test_tensor_core_backward_matches_oracle_and_generic(case, monkeypatch):
     gro["dS_T"] = torch.randn((B, H, 128, 128), generator=gen)
     gro["dm_T"] = torch.randn((B, H, 128), generator=gen)
     assert_within(bwd_errors(inp, L, gro, du_heads=range(H)), 1e-2,
-                  "tensor-core bwd")
+                  "tensor-core bwd %s" % (case,))
     d, _, _, _, ws = run_fwd(inp, L, training=True)
     dd = to_dev(gro)
     g_tc = carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
                            d["u_down"], d["u_up"], L, dd["d_o"], ws,
                            dd["dS_T"], dd["dm_T"])
-    # the generic backward needs the generic forward's fp32 checkpoints: it
-    # refuses the tensor-core forward's workspace
+    # the generic backward needs the generic forward's fp32 checkpoints,
+    # which a tensor-core workspace does not hold: refused on the host
     assert carve.get_status(ws) == 0
     monkeypatch.setenv("CARVE_BWD_PATH", "generic")
-    carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
-                    d["u_down"], d["u_up"], L, dd["d_o"], ws,
-                    dd["dS_T"], dd["dm_T"])
-    assert carve.STATUS[carve.get_status(ws)] == "CARVE_ERR_WORKSPACE"
+    with pytest.raises(carve.CarveError) as exc:
+        carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
+                        d["u_down"], d["u_up"], L, dd["d_o"], ws,
+                        dd["dS_T"], dd["dm_T"])
+    assert carve.STATUS[exc.value.code] == "CARVE_ERR_WORKSPACE"
+    assert carve.get_status(ws) == 0
     monkeypatch.setenv("CARVE_FWD_PATH", "generic")
     _, _, _, _, ws_g = run_fwd(inp, L, training=True)
     g_ge = carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
@@ -292,3 +295,38 @@ def test_tensor_core_backward_matches_oracle_and_generic(case, monkeypatch):
     for name in g_tc:
         if g_tc[name] is not None and g_tc[name].numel():
             assert _rel(g_tc[name].float().cpu(), g_ge[name].float().cpu()) < 1e-2, name
+
+
+# ------------------------------- full size, every pair: tc vs generic ----
+
+def _all_pairs(a, b):
+    from _parity import rel as _rel
+    return _rel(a.float().cpu(), b.float().cpu())
+
+
+def test_layer_1p3b_every_pair_tensor_core_vs_generic(monkeypatch):
+    """Every (sequence, head) pair of the full 1.3B-layer forward and
+    training backward: the tensor-core kernels against the generic CUDA-core
+    kernels (both GPU paths; the oracle comparison of sampled pairs is in
+    the tests above).  Catches pair-indexing faults in unsampled pairs."""
+    cfg = WORKLOADS["layer_1p3b"]
+    inp = inputs(cfg, 9, torch.bfloat16)
+    gro = grad_outputs(cfg, 9, torch.bfloat16)
+    d, dd = to_dev(inp), to_dev(gro)
+    L = cfg["L"]
+    res = {}
+    for path in ("tc", "generic"):
+        if path == "generic":
+            monkeypatch.setenv("CARVE_FWD_PATH", "generic")
+        o, S_T, m_T, ws = carve.chunk_fwd(d["q"], d["k"], d["v"], d["g"],
+                                          d["bx"], d["w"], d["u_down"],
+                                          d["u_up"], L, training=True)
+        gr = carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
+                             d["u_down"], d["u_up"], L, dd["d_o"], ws)
+        torch.cuda.synchronize()
+        assert carve.get_status(ws) == 0
+        res[path] = dict(gr, o=o, S_T=S_T, m_T=m_T)
+        del ws
+    errs = {k: _all_pairs(res["tc"][k], res["generic"][k])
+            for k in res["tc"] if res["tc"][k] is not None}
+    assert_within(errs, 1e-2, "1.3B layer, all 128 pairs, tc vs generic")

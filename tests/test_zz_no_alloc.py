@@ -11,7 +11,9 @@ The test calls it through the C ABI twice in a row, on different inputs,
 and checks each result against carve_chunk_fwd on the same inputs within
 the parity tolerance (max|delta| / max|ref| <= 1e-2 for bf16 inputs, 1e-4
 for fp32).  The test itself allocates its tensors with torch; the entry
-point under test does not allocate.  This file is collected last.
+point under test does not allocate.  It runs after the parity tests (only
+the sentinel-margin guards come later), so a run that stops at its first
+failure has exercised the rest of the library first.
 """
 import ctypes
 
