@@ -409,6 +409,46 @@ def extras(carve, args, pk, host, d, stream, fwd_ms_train):
         del wsl
     out["sweep"] = sweep
 
+    # decode: one new token per (sequence, head) at the 1.3B-layer shape,
+    # fp32 state S read and written once per step
+    dev = d["q"].device
+    L = cfg["L"]
+    tok = {n: d[n][:, 0].contiguous() for n in ("q", "k", "v", "g", "bx", "w")}
+    Sd = torch.randn((B, H, DV, DK), device=dev) * 0.1
+    md = torch.zeros((B, H, DV), device=dev)
+    od = torch.zeros((B, H, DV), device=dev)
+    pos = torch.full((B,), 5, dtype=torch.int32, device=dev)
+    outd = torch.empty((B, H, DV), dtype=d["q"].dtype, device=dev)
+    step = lambda: carve.decode_step(tok["q"], tok["k"], tok["v"], tok["g"],
+                                     tok["bx"], tok["w"], d["u_down"],
+                                     d["u_up"], L, pos, Sd, md, od, o=outd)
+    # the state (B H DV DK fp32 = 8 MiB here) fits in L2: write a buffer
+    # larger than L2 between timed steps so that each reads S from HBM
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(it)]
+    for _ in range(args.warmup):
+        step()
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    msd = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+    pairs = B * H
+    dec_bytes = pairs * (2 * DV * DK * 4 + 2 * (4 * DK + 2 * DV + 1)
+                         + 4 * DV * 4)
+    dec_flops = pairs * (6 * DV * DK + 2 * DV * DK)
+    rdec = roof_obj("carve_decode_step", dec_flops, dec_bytes, msd, pk)
+    out["decode"] = {
+        "workload": "layer_1p3b decode step (B=8, H=16, dk=dv=128, r=32, "
+                    "L=64; one token per sequence)",
+        "ms": msd, "tokens_per_s": B / (msd * 1e-3), "roofline": rdec,
+        "timing": "median of %d single steps, L2 flushed before each" % it,
+        "bytes_per_pair_step": dec_bytes / pairs}
+    del flush
+
     # long_context: config 3 (dv = 256, S0 != 0), forward
     lc = WORKLOADS["long_context"]
     hl = make_inputs(seed=3, dtype=torch.bfloat16, **lc)

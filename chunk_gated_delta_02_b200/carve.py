@@ -22,12 +22,13 @@ STATUS = {0: "CARVE_OK", 1: "CARVE_ERR_INVALID_ARG", 2: "CARVE_ERR_UNSUPPORTED",
 # Entry points declared in include/carve.h (the ABI test checks the list).
 EXPORTS = ("carve_workspace_bytes", "carve_chunk_fwd", "carve_chunk_bwd",
            "carve_get_status", "carve_reset_status", "carve_status_str",
-           "carve_fwd_path", "carve_chunk_fwd_noalloc")
+           "carve_fwd_path", "carve_chunk_fwd_noalloc", "carve_decode_step")
 
 
 class Shape(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_int32)
-                for n in ("B", "T", "H", "DK", "DV", "R", "L", "dtype")]
+    _fields_ = ([(n, ctypes.c_int32)
+                 for n in ("B", "T", "H", "DK", "DV", "R", "L", "dtype")]
+                + [("decay_scale", ctypes.c_float)])
 
 
 class CarveError(RuntimeError):
@@ -65,6 +66,8 @@ def lib():
         L.carve_status_str.restype = ctypes.c_char_p
         L.carve_fwd_path.argtypes = [sp]
         L.carve_fwd_path.restype = ctypes.c_char_p
+        L.carve_decode_step.argtypes = [sp] + [vp] * 13 + [vp]
+        L.carve_decode_step.restype = i32
         _lib = L
     return _lib
 
@@ -77,9 +80,11 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def make_shape(B, T, H, DK, DV, R, L, dtype):
+def make_shape(B, T, H, DK, DV, R, L, dtype, decay_scale=0.0):
+    """decay_scale > 0: `g` holds raw decay logits a and the kernels use
+    g = -decay_scale * softplus(a); the backward then returns dL/da."""
     return Shape(B, T, H, DK, DV, R, L, _DTYPES[dtype] if isinstance(
-        dtype, torch.dtype) else int(dtype))
+        dtype, torch.dtype) else int(dtype), float(decay_scale))
 
 
 def workspace_bytes(shape, training):
@@ -118,13 +123,15 @@ def _dims(q, v, u_down):
 
 
 def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
-              training=False, workspace=None, o=None, want_state=True):
+              training=False, workspace=None, o=None, want_state=True,
+              decay_scale=0.0):
     """Forward pass.  Returns (o, S_T, m_T, workspace).
 
     q, k, g, bx [B, T, H, DK]; v [B, T, H, DV]; w [B, T, H]; u_down
     [H, R, DV]; u_up [H, DK, R] -- all bf16 or all fp32.  S0 [B, H, DV, DK]
     and m0 [B, H, DV] fp32 or None.  With training=True the returned
-    workspace holds what chunk_bwd needs."""
+    workspace holds what chunk_bwd needs.  decay_scale > 0: g holds raw
+    decay logits a, the log-decay is -decay_scale * softplus(a)."""
     dev = q.device
     dt = q.dtype
     if dt not in _DTYPES:
@@ -139,7 +146,7 @@ def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
         _check(S0, "S0", torch.float32, (B, H, DV, DK), dev)
     if m0 is not None:
         _check(m0, "m0", torch.float32, (B, H, DV), dev)
-    shape = make_shape(B, T, H, DK, DV, R, L, dt)
+    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale)
     nbytes = workspace_bytes(shape, training)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
@@ -161,11 +168,12 @@ def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
 
 
 def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
-              dm_T=None, want_dS0=True, out=None):
-    """Backward pass after a training-mode chunk_fwd with the same inputs.
-    Returns a dict: dq dk dg dbx [B, T, H, DK], dv [B, T, H, DV], dw
-    [B, T, H] (input dtype); du_down [H, R, DV], du_up [H, DK, R], dS0
-    [B, H, DV, DK], dm0 [B, H, DV] (fp32)."""
+              dm_T=None, want_dS0=True, out=None, decay_scale=0.0):
+    """Backward pass after a training-mode chunk_fwd with the same inputs
+    (and the same decay_scale; with decay_scale > 0, "dg" is dL/da of the
+    raw decay logits).  Returns a dict: dq dk dg dbx [B, T, H, DK], dv
+    [B, T, H, DV], dw [B, T, H] (input dtype); du_down [H, R, DV], du_up
+    [H, DK, R], dS0 [B, H, DV, DK], dm0 [B, H, DV] (fp32)."""
     dev = q.device
     dt = q.dtype
     B, T, H, DK, DV, R = _dims(q, v, u_down)
@@ -174,7 +182,7 @@ def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
         _check(dS_T, "dS_T", torch.float32, (B, H, DV, DK), dev)
     if dm_T is not None:
         _check(dm_T, "dm_T", torch.float32, (B, H, DV), dev)
-    shape = make_shape(B, T, H, DK, DV, R, L, dt)
+    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale)
     if out is None:
         e = lambda s, d=dt: torch.empty(s, dtype=d, device=dev)
         out = dict(dq=e((B, T, H, DK)), dk=e((B, T, H, DK)),
@@ -197,6 +205,42 @@ def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
     return out
 
 
+def decode_step(q, k, v, g, bx, w, u_down, u_up, L, pos, S, m, osum, o=None,
+                decay_scale=0.0):
+    """One recurrent decode step (one new token per (sequence, head)).
+
+    q, k, g, bx [B, H, DK]; v [B, H, DV]; w [B, H] (bf16 or fp32); u_down
+    [H, R, DV], u_up [H, DK, R]; pos [B] int32 (tokens already processed,
+    read only); S [B, H, DV, DK], m, osum [B, H, DV] fp32, updated in place.
+    Returns o [B, H, DV]."""
+    dev = q.device
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError("dtype must be bfloat16 or float32")
+    B, H, DK = q.shape
+    DV = v.shape[-1]
+    R = u_down.shape[1] if u_down is not None else 0
+    for t, n, s in ((q, "q", (B, H, DK)), (k, "k", (B, H, DK)),
+                    (v, "v", (B, H, DV)), (g, "g", (B, H, DK)),
+                    (bx, "bx", (B, H, DK)), (w, "w", (B, H)),
+                    (u_down, "u_down", (H, R, DV)), (u_up, "u_up", (H, DK, R))):
+        _check(t, n, dt, s, dev)
+    _check(pos, "pos", torch.int32, (B,), dev)
+    _check(S, "S", torch.float32, (B, H, DV, DK), dev)
+    _check(m, "m", torch.float32, (B, H, DV), dev)
+    _check(osum, "osum", torch.float32, (B, H, DV), dev)
+    if o is None:
+        o = torch.empty((B, H, DV), dtype=dt, device=dev)
+    shape = make_shape(B, 1, H, DK, DV, R, L, dt, decay_scale)
+    rc = lib().carve_decode_step(
+        ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(bx),
+        _ptr(w), _ptr(u_down), _ptr(u_up), _ptr(pos), _ptr(S), _ptr(m),
+        _ptr(osum), _ptr(o), _stream(dev))
+    if rc != 0:
+        raise CarveError("carve_decode_step", rc)
+    return o
+
+
 def get_status(workspace):
     """Synchronise the current stream and read the device status word."""
     return lib().carve_get_status(_ptr(workspace), _stream(workspace.device))
@@ -207,11 +251,13 @@ class CarveFunction(torch.autograd.Function):
     u_down, u_up, S0, m0, L)."""
 
     @staticmethod
-    def forward(ctx, q, k, v, g, bx, w, u_down, u_up, S0, m0, L):
+    def forward(ctx, q, k, v, g, bx, w, u_down, u_up, S0, m0, L,
+                decay_scale=0.0):
         o, S_T, m_T, ws = chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0,
-                                    m0, training=True)
+                                    m0, training=True, decay_scale=decay_scale)
         ctx.save_for_backward(q, k, v, g, bx, w, u_down, u_up, ws)
         ctx.L = L
+        ctx.decay_scale = decay_scale
         ctx.has_S0, ctx.has_m0 = S0 is not None, m0 is not None
         return o, S_T, m_T
 
@@ -222,13 +268,17 @@ class CarveFunction(torch.autograd.Function):
             if d_o is None else d_o.contiguous()
         gr = chunk_bwd(q, k, v, g, bx, w, u_down, u_up, ctx.L, d_o, ws,
                        None if dS_T is None else dS_T.contiguous(),
-                       None if dm_T is None else dm_T.contiguous())
+                       None if dm_T is None else dm_T.contiguous(),
+                       decay_scale=ctx.decay_scale)
         return (gr["dq"], gr["dk"], gr["dv"], gr["dg"], gr["dbx"], gr["dw"],
                 gr["du_down"].to(u_down.dtype), gr["du_up"].to(u_up.dtype),
                 gr["dS0"] if ctx.has_S0 else None,
-                gr["dm0"] if ctx.has_m0 else None, None)
+                gr["dm0"] if ctx.has_m0 else None, None, None)
 
 
-def carve(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None):
-    """Differentiable CARVE recurrent core; returns (o, S_T, m_T)."""
-    return CarveFunction.apply(q, k, v, g, bx, w, u_down, u_up, S0, m0, L)
+def carve(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
+          decay_scale=0.0):
+    """Differentiable CARVE recurrent core; returns (o, S_T, m_T).
+    decay_scale > 0: g holds raw decay logits (see chunk_fwd)."""
+    return CarveFunction.apply(q, k, v, g, bx, w, u_down, u_up, S0, m0, L,
+                               decay_scale)

@@ -18,6 +18,8 @@ carve_status check_shape(const carve_shape* s) {
     return CARVE_ERR_INVALID_ARG;
   if (s->dtype != CARVE_BF16 && s->dtype != CARVE_FP32)
     return CARVE_ERR_INVALID_ARG;
+  if (!(s->decay_scale >= 0.f) || s->decay_scale > 3.0e38f)  // NaN, < 0, inf
+    return CARVE_ERR_INVALID_ARG;
   if (s->DK % 16 || s->DV % 16 || s->DK > 256 || s->DV > 256)
     return CARVE_ERR_UNSUPPORTED;
   if (s->R > kMaxR) return CARVE_ERR_UNSUPPORTED;
@@ -141,6 +143,7 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   a.tc_rec = training && L.tc_rec ? (uint8_t*)(ws + L.tc_rec) : nullptr;
   a.gin = training && L.gin ? (float*)(ws + L.gin) : nullptr;
   a.hdr = (WsHeader*)ws;
+  a.dscale = s.decay_scale;
   test_knobs(&a.spin, &a.stall_block);
   cudaError_t e = tc ? launch_fwd_tc(a, (cudaStream_t)stream)
                       : launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
@@ -196,10 +199,39 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   a.dq = dq; a.dk = dk; a.dv = dv; a.dg = dg; a.dbx = db_x; a.dw = dw;
   a.du_down = du_down; a.du_up = du_up; a.dS0 = dS0; a.dm0 = dm0;
   a.hdr = (WsHeader*)ws;
+  a.dscale = s.decay_scale;
   test_knobs(&a.spin, &a.stall_block);
   cudaError_t e = tc ? launch_bwd_tc(a, (cudaStream_t)stream)
                       : launch_bwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_decode_step(const carve_shape* shape, const void* q,
+                               const void* k, const void* v, const void* g,
+                               const void* b_x, const void* w,
+                               const void* u_down, const void* u_up,
+                               const int32_t* pos, float* S, float* m,
+                               float* osum, void* o, void* stream) {
+  if (!shape) return CARVE_ERR_INVALID_ARG;
+  carve_shape s = *shape;
+  s.T = 0;  // one token per call: the sequence length plays no part
+  carve_status st = check_shape(&s);
+  if (st != CARVE_OK) return st;
+  if (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) || !ptr_ok(b_x) ||
+      !ptr_ok(w) || !ptr_ok(pos) || !ptr_ok(S) || !ptr_ok(m) ||
+      !ptr_ok(osum) || !ptr_ok(o))
+    return CARVE_ERR_INVALID_ARG;
+  if (s.R > 0 && (!ptr_ok(u_down) || !ptr_ok(u_up)))
+    return CARVE_ERR_INVALID_ARG;
+  DecArgs a{};
+  a.B = s.B; a.H = s.H; a.DK = s.DK; a.DV = s.DV; a.R = s.R; a.L = s.L;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.bx = b_x; a.w = w;
+  a.u_down = u_down; a.u_up = u_up; a.pos = pos;
+  a.S = S; a.m = m; a.osum = osum; a.o = o;
+  a.dscale = s.decay_scale;
+  return launch_decode(a, s.dtype, (cudaStream_t)stream) == cudaSuccess
+             ? CARVE_OK
+             : CARVE_ERR_CUDA;
 }
 
 carve_status carve_get_status(const void* workspace, void* stream) {

@@ -107,7 +107,8 @@ __device__ void block_operands(const TIn* q, const TIn* k, const TIn* v,
                                const float* s_p, int b, int h, int t0, int T,
                                int H, int C, int DK, int DV, float* Kt,
                                float* Kh, float* Qt, float* Kp, float* Gl,
-                               float* s_gam, float* s_w, float* W) {
+                               float* s_gam, float* s_w, float* W,
+                               float dscale) {
   for (int j = threadIdx.x; j < DK; j += blockDim.x) {
     float G = 0.f;
     for (int i = 0; i < C; ++i) {
@@ -115,7 +116,7 @@ __device__ void block_operands(const TIn* q, const TIn* k, const TIn* v,
       const float kk = ldf(k, x), qq = ldf(q, x);
       const float bb = sigm(ldf(bx, x) + s_p[j]);
       const float Gm = G;
-      G += ldf(g, x);
+      G += decay_act(ldf(g, x), dscale);
       const float gam = expf(G), igam = expf(-G);
       Kt[i * DK + j] = kk * gam;
       Kh[i * DK + j] = kk * igam;
@@ -208,7 +209,7 @@ __global__ void __launch_bounds__(kThreads) fwd_generic_kernel(FwdArgs a) {
         for (size_t i = tid; i < SZ; i += nt) dst[i] = S[i];
       }
       block_operands(q, k, v, g, bx, w, s_p, b, h, t0, T, H, C, DK, DV, Kt,
-                     Kh, Qt, Kp, (float*)nullptr, s_gam, s_w, W);
+                     Kh, Qt, Kp, (float*)nullptr, s_gam, s_w, W, a.dscale);
       block_grams(Kt, Kh, Qt, Kp, C, DK, sA, sT, sM, sPk, sPq);
       // R = K~ S^T + M W ;  E = T R
       mm(Rr, DV, Kt, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
@@ -344,7 +345,7 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
       const float* S = a.ck_S + ((size_t)pair * (a.NB + 1) + ib) * SZ;
       const float* Sn = S + SZ;  // state at the end of this block
       block_operands(q, k, v, g, bx, w, s_p, b, h, t0, T, H, C, DK, DV, Kt,
-                     Kh, Qt, Kp, Gl, s_gam, s_w, W);
+                     Kh, Qt, Kp, Gl, s_gam, s_w, W, a.dscale);
       block_grams(Kt, Kh, Qt, Kp, C, DK, sA, sT, sM, sPk, sPq);
       mm(Rr, DV, Kt, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
       mm(Rr, DV, sM, C, 1, W, DV, 1, C, DV, C, 1.f, true, false);
@@ -435,7 +436,10 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
           if (i == C - 1) dG += s_dlg[j];
           if (i + 1 < C) dG += dQt[e + DK] * Qt[e + DK];
           acc += dG;
-          stf(dg, x, acc);
+          // with raw decay logits, dL/da = dL/dg * (-s sigmoid(a))
+          stf(dg, x, a.dscale > 0.f
+                         ? acc * -a.dscale * sigm(ldf(g, x))
+                         : acc);
         }
       }
       __syncthreads();

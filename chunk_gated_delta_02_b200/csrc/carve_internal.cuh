@@ -41,12 +41,14 @@ inline bool tc_shape(const carve_shape& s) {
   return s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 128 &&
          s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0;
 }
-// The tensor-core forward also runs DV = 256 (two CTAs per pair) without
-// training.
+// The tensor-core forward also runs, without training, DV = 256 (two CTAs
+// per pair) and chunks of 16, 32 or 48 tokens (one chunk per block, the
+// 64-row tiles zero past the chunk).
 inline bool tc_fwd_shape(const carve_shape& s, bool training) {
   if (tc_shape(s)) return true;
-  return !training && s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 256 &&
-         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0;
+  const bool chunk_ok = s.L % kMaxBlock == 0 || (s.L < kMaxBlock && s.L % 16 == 0);
+  return !training && s.dtype == CARVE_BF16 && s.DK == 128 &&
+         (s.DV == 128 || s.DV == 256) && chunk_ok && s.R <= 32 && s.T > 0;
 }
 static_assert(sizeof(WsHeader) == kHeaderBytes, "header size");
 
@@ -125,6 +127,18 @@ inline WsLayout ws_layout(const carve_shape& s, bool training, bool tc) {
   return w;
 }
 
+// The decay activation applied to raw logits when decay_scale s > 0:
+// g = -s softplus(a), softplus(a) = max(a, 0) + log1p(exp(-|a|)); s == 0
+// passes g through.  Its derivative dg/da = -s sigmoid(a) is formed by the
+// backward kernels from g itself: sigmoid(a) = 1 - exp(-softplus(a)) =
+// -expm1(g / s).
+__device__ __forceinline__ float decay_act(float a, float s) {
+  return s > 0.f ? -s * (fmaxf(a, 0.f) + log1pf(expf(-fabsf(a)))) : a;
+}
+__device__ __forceinline__ float decay_act_grad(float g, float s) {
+  return s > 0.f ? s * expm1f(g / s) : 1.f;
+}
+
 // Element load/store in the I/O dtype, arithmetic in fp32.
 __device__ __forceinline__ float ldf(const float* p, size_t i) { return p[i]; }
 __device__ __forceinline__ float ldf(const __nv_bfloat16* p, size_t i) {
@@ -151,6 +165,7 @@ struct FwdArgs {
   WsHeader* hdr;
   long long spin;   // cycles a device-side wait spins before it gives up
   int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
+  float dscale;     // decay activation scale (0: g is the log-decay)
 };
 
 struct BwdArgs {
@@ -169,7 +184,19 @@ struct BwdArgs {
   WsHeader* hdr;
   long long spin;   // cycles a device-side wait spins before it gives up
   int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
+  float dscale;     // decay activation scale (0: g is the log-decay)
 };
+
+// Arguments of the decode step (one token per (sequence, head)).
+struct DecArgs {
+  int B, H, DK, DV, R, L;
+  const void *q, *k, *v, *g, *bx, *w, *u_down, *u_up;  // [B, H, D] one token
+  const int32_t* pos;  // [B] tokens already processed per sequence
+  float *S, *m, *osum;  // [B, H, DV, DK], [B, H, DV], [B, H, DV] in/out
+  void* o;              // [B, H, DV]
+  float dscale;         // decay activation scale (0: g is the log-decay)
+};
+cudaError_t launch_decode(const DecArgs& a, int dtype, cudaStream_t st);
 
 // Host-side checks (carve_api.cu): the supported-shape check of every entry
 // point, and the test-only wait limit / stall knobs.

@@ -86,6 +86,7 @@ extern "C" carve_status carve_chunk_fwd_noalloc(
   a.hdr = (WsHeader*)base;
   a.spin = kSpinCycles;
   a.stall_block = -1;
+  a.dscale = s.decay_scale;
   cudaError_t e = launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }

@@ -107,21 +107,7 @@ constexpr uint32_t ID_KK64_NA = idesc_bf16_neg(128, 64, false, false, true, fals
 constexpr uint32_t ID_MM64_NA = idesc_bf16_neg(128, 64, true, true, true, false);
 constexpr uint32_t ID_MK128_NA = idesc_bf16_neg(128, 128, true, false, true, false);
 
-// Sum over the 32 lanes of a warp of v[i] (i < 32): lane l ends with the
-// sum of index l in v[0].  (Reduce-scatter: 31 shuffles.)
-__device__ __forceinline__ float warp_reduce_scatter32(float* v, int lane) {
-#pragma unroll
-  for (int k = 16; k >= 1; k >>= 1) {
-    const bool up = (lane & k) != 0;
-#pragma unroll
-    for (int i = 0; i < k; ++i) {
-      const float send = up ? v[i] : v[i + k];
-      const float keep = up ? v[i + k] : v[i];
-      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
-    }
-  }
-  return v[0];
-}
+using tc::warp_reduce_scatter32;
 
 // Sum over the 32 lanes of a warp of v[i] (i < 16): lanes l and l ^ 16 end
 // with the sum of index l % 16 in v[0].  (15 + 1 shuffles.)
@@ -417,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::transform_block<8>(sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB,
                              sm + R_DSB + 16384, s_gam,
                              reinterpret_cast<float*>(sm + R_MP), 3, 16384, 7,
-                             kThreads);
+                             kThreads, a.dscale);
       if (tid < 128) s_x[tid] = 0.f;
     } else {
       const int u = tid - 256;
@@ -787,7 +773,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float gsum = 0.f;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          gv[e] = ldbf(sm + R_RO + sw128_off(tb + e, jj, 64));
+          gv[e] = decay_act(ldbf(sm + R_RO + sw128_off(tb + e, jj, 64)), a.dscale);
           gsum += gv[e];
         }
         s_gq[gp * 128 + jj] = gsum;
@@ -875,14 +861,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       float acc = 0.f;
       for (int g2 = gp + 1; g2 < 4; ++g2)
         acc += s_lq[g2 * 128 + jj] + (g2 < 3 ? s_qf[(g2 + 1) * 128 + jj] : dlg);
+      // with raw decay logits a (decay_scale s > 0) the output is dL/da =
+      // dL/dg * s expm1(g / s), formed from the log-decay itself
+      const float dsc = a.dscale;
       float hg = 0.f;  // the odd token's suffix sum
 #pragma unroll
       for (int i = 15; i >= 0; --i) {
         acc += dGv[i];
+        const float out = dsc > 0.f ? acc * decay_act_grad(gv[i], dsc) : acc;
         if (i & 1)
-          hg = acc;
+          hg = out;
         else
-          st_pair(dg, tb + i, acc, hg);
+          st_pair(dg, tb + i, out, hg);
       }
     }
 

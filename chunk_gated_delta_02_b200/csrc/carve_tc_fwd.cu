@@ -50,7 +50,7 @@ using tc::st_chunk;
 using tc::unit_lower_inverse64;
 
 constexpr int kThreads = 512;
-constexpr int kBlk = 64;   // tokens per block
+constexpr int kBlk = 64;   // rows of a token tile (tokens per block C <= 64)
 constexpr int kDK = 128;   // key width
 constexpr int kDV = 128;   // value rows per CTA
 constexpr int kRMax = 32;  // rank of U_b held in registers
@@ -75,8 +75,8 @@ constexpr uint32_t SM_M = 1280;        // m_v                128 f32
 constexpr uint32_t SM_H = 1792;        // U_down m            64 f32
 constexpr uint32_t SM_GAM1 = 2048;     // gamma_j (odd blocks)  128 f32
 constexpr uint32_t SM_BAR = 2560;      // kNumBars mbarriers
-constexpr uint32_t SM_TMEM = 2640;     // TMEM base address
-constexpr uint32_t SM_ABORT = 2644;    // abort flag
+constexpr uint32_t SM_TMEM = 2648;     // TMEM base address
+constexpr uint32_t SM_ABORT = 2652;    // abort flag
 constexpr uint32_t kSmallBytes = 2688;
 constexpr uint32_t OFF_UU = 215808;    // U_up^T bf16 [kRMax][kUuLd]   8.5 KB
 constexpr int kUuLd = 128 + 8;         // row pitch: 16 B of padding per row
@@ -96,7 +96,8 @@ constexpr int B_X = 6;     // dv = 256: the other CTA's half of U_down m arrived
 constexpr int B_WK = 7;    // S += W^T K^ (issued with MMA 2)
 constexpr int B_TEST = 8;  // test only: the redirected commit of a stalled block
 constexpr int B_FIN = 9;   // an aborting CTA: thread 0's D1 MMAs not yet committed
-constexpr int kNumBars = 10;
+constexpr int B_GM = 10;   // the next block's [M; P_k], issued in step 6
+constexpr int kNumBars = 11;
 static_assert(SM_BAR + 8 * kNumBars <= SM_TMEM, "mbarriers");
 
 // TMEM columns (fp32, lanes = rows)
@@ -116,10 +117,12 @@ constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false
 
 
 // Key side of one block's transform by warps 8-15 (one out-of-line copy of
-// the unrolled code serves the prologue and the block loop).
-static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* rg, float* gam,
-                                            float* red) {
-  tc::transform_keys<8>(x, rg, rg, gam, red, 3, 8192, 8);
+// the unrolled code serves the prologue and the block loop): K~, Q~ in place
+// in X, K^ straight into rows 0..63 of its operand slot in KHP.
+static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* kh,
+                                            const uint8_t* rg, float* gam,
+                                            float* red, float dscale) {
+  tc::transform_keys<8>(x, kh, rg, gam, red, 3, 16384, 8, dscale);
 }
 
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
@@ -161,7 +164,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int pair = dv2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int b = pair / a.H, h = pair - b * a.H;
   const int T = a.T, H = a.H, R = a.R, NB = a.NB;
-  const int bpc = a.L / kBlk;
+  // blocks of C = min(L, 64) tokens; with C < 64 (chunks of 16, 32 or 48
+  // tokens) the block is a chunk and rows C..63 of every token tile stay
+  // zero, which contributes nothing to any product (see below)
+  const int C = a.C;
+  const int bpc = a.L / C;
   const size_t SZ = (size_t)kDV * kDK;
   const __nv_bfloat16* w_in = static_cast<const __nv_bfloat16*>(a.w);
   const __nv_bfloat16* ud = static_cast<const __nv_bfloat16*>(a.u_down);
@@ -178,6 +185,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_g);
     prefetch_tmap(&tm_bx);
+  }
+  if (C < kBlk) {
+    // blocks shorter than the 64-row tiles: every token tile starts zero.
+    // The copies only ever write rows 0..C-1; rows C..63 then stay zero
+    // through the in-place transform (K~ = K Gamma, Q~, K^ = K / Gamma of a
+    // zero row are zero; a zero log-decay leaves gamma = Gamma_{C-1}), so
+    // those rows add nothing to the Grams, R, E, O or the state update.
+    const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid; i < 32768 / 16; i += kThreads)
+      *reinterpret_cast<uint4*>(sm + OFF_X + 16 * i) = z;
+    for (int i = tid; i < 49152 / 16; i += kThreads)
+      *reinterpret_cast<uint4*>(sm + OFF_RV + 16 * i) = z;  // RV, RG, RB
+    fence_async_smem();
   }
   if (warp == 0) {
     tmem_alloc(s_tmem, kTmemCols);
@@ -227,17 +247,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  // content gate of chunk c, on warps 8-15 (u = tid - 256): m_c = the mean
-  // of the previous chunk's o from its four token-quarter partial sums
-  // (m_0 is set up front), h = U_down m_c, s_p = U_up h.  Training records
-  // p_c, h_c and m_c for the backward during the chunk's first block.
+  // content gate of chunk c, on warps 8-15 (u = tid - 256): from m_c in
+  // s_m (m_0 set up front, later ones formed at the previous chunk's end),
+  // h = U_down m_c, s_p = U_up h.  Training records p_c, h_c and m_c for
+  // the backward during the chunk's first block.
   const float invL = 1.0f / (float)a.L;
-  float* s_mq = reinterpret_cast<float*>(sm + OFF_RE);  // [4][128] partial sums of m
+  // pieces of the chunk mean, in the rows of MY that [M; P_k] leaves once
+  // MMA 2 has read it: c_O[2][128] (row sums of Q~ S^T + P_k W over each
+  // half of the tokens), eu[2][128] (E^T u over each half of the columns)
+  // and u2[2][64] (column sums of P_kap over each half of the tokens)
+  float* s_co = reinterpret_cast<float*>(sm + OFF_MY + 8192);
+  float* s_eu = s_co + 256;
+  float* s_u2 = s_co + 512;
   auto gate = [&](int c) {
     const int u = tid - 256;
-    if (c > 0 && u < 128)
-      s_m[u] = ((s_mq[u] + s_mq[128 + u]) + (s_mq[256 + u] + s_mq[384 + u])) * invL;
-    bar_named(6, 256);
+    bar_named(6, 256);  // s_m visible to all of warps 8-15
     {
       const int r = u >> 3, part = u & 7;
       float acc = 0.f;
@@ -288,8 +312,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   auto issue_vgb = [&](int ib) {
-    const int tok = b * T + ib * kBlk;
-    mbar_expect_tx(bars + B_VGB, 3 * 16384);
+    const int tok = b * T + ib * C;
+    mbar_expect_tx(bars + B_VGB, 3 * 2 * 128 * C);
     tma_load_3d(sm + OFF_RV, &tm_v, bars + B_VGB, v0, h, tok);
     tma_load_3d(sm + OFF_RV + 8192, &tm_v, bars + B_VGB, v0 + 64, h, tok);
     tma_load_3d(sm + OFF_RG, &tm_g, bars + B_VGB, 0, h, tok);
@@ -300,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   // k, q, g of block ib -> L2 ahead of their loads
   auto prefetch_kqg = [&](int ib) {
-    const int tok = b * T + ib * kBlk;
+    const int tok = b * T + ib * C;
 #pragma unroll 1
     for (int x = 0; x < kDK; x += 64) {
       tma_prefetch_3d(&tm_k, x, h, tok);
@@ -309,8 +333,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
   auto issue_kq = [&](int ib) {
-    const int tok = b * T + ib * kBlk;
-    mbar_expect_tx(bars + B_KQ, 2 * 16384);
+    const int tok = b * T + ib * C;
+    mbar_expect_tx(bars + B_KQ, 2 * 2 * 128 * C);
     tma_load_3d(sm + OFF_X, &tm_k, bars + B_KQ, 0, h, tok);
     tma_load_3d(sm + OFF_X + 16384, &tm_k, bars + B_KQ, 64, h, tok);
     tma_load_3d(sm + OFF_X + 8192, &tm_q, bars + B_KQ, 0, h, tok);
@@ -319,11 +343,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   // key side of block nb's transform (warps 8-15): K~, Q~ in place in X,
-  // K^ over the raw g tile (RG), gamma into its parity's buffer
+  // K^ into its operand slot (rows 0..63 of KHP), gamma into its parity's
+  // buffer
   auto keys = [&](int nb) {
     wait(B_VGB, 1);
     wait(B_KQ, 2);
-    keys_w8(sm + OFF_X, sm + OFF_RG, (nb & 1) ? s_gam1 : s_gam0, s_red);
+    keys_w8(sm + OFF_X, sm + OFF_KHP, sm + OFF_RG, (nb & 1) ? s_gam1 : s_gam0,
+            s_red, a.dscale);
   };
 
   // ---- initial state: S0 -> TMEM (fp32) and the bf16 operand copy
@@ -351,23 +377,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   tmem_st_wait();
   tc_fence_before();
   __syncthreads();
-  if (warp >= 8) keys(0);
+  if (warp >= 8) {  // block 0's key side and chunk 0's gate
+    keys(0);
+    gate(0);
+  }
   fence_async_smem();
   __syncthreads();
 
-  // w_t of the two token rows a thread of warps 0-7 scales in W = w V,
+  // w_t of the two token rows a thread of warps 8-15 scales in W = w V,
   // fetched one block ahead into registers (raw bf16 bits: converted only
   // when used, so the loads' latency is not waited for at issue)
   const unsigned short* w_bits = reinterpret_cast<const unsigned short*>(w_in);
   uint32_t w_lo = 0, w_hi = 0;
-  if (warp < 8) {
-    const size_t r0 = (size_t)b * T + (tid >> 3);
-    w_lo = w_bits[r0 * H + h];
-    w_hi = w_bits[(r0 + 32) * H + h];
+  if (warp >= 8) {
+    const int wr = (tid - 256) >> 3;
+    const size_t r0 = (size_t)b * T + wr;
+    w_lo = wr < C ? w_bits[r0 * H + h] : 0u;
+    w_hi = wr + 32 < C ? w_bits[(r0 + 32) * H + h] : 0u;
   }
-  float msum = 0.f;  // this thread's token quarter of the chunk's sum of o, row `row`
   for (int ib = 0; ib < NB; ++ib) {
-    const int t0 = ib * kBlk;
+    const int t0 = ib * C;
     const bool chunk_end = ((ib + 1) % bpc) == 0;
     uint8_t* rec = a.tc_rec ? a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes
                             : nullptr;
@@ -382,24 +411,39 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 32 && ib + 2 < NB) prefetch_kqg(ib + 2);
 
-    // ---- 2. the key side (K~, Q~ in X; K^ in RG) was formed during the
-    //      previous block's solve.  D1 = S [K~; Q~]^T (issued by thread 0),
-    //      W = w V (warps 0-7); the chunk's gate p (warps 8-15, first block
-    //      of a chunk)
-    if (warp < 8) {
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t x0 = smem_u32(sm + OFF_X), sb0 = smem_u32(sm + OFF_SB);
+    // ---- 2. the key side (K~, Q~ in X; K^ in KHP) was formed during the
+    //      previous block's solve, the chunk's gate p at the previous
+    //      chunk's end, and the b-independent half of the Grams, [M; P_k] =
+    //      [K~; Q~] K^T, issued with the previous block's MMA 3b / 4 (here
+    //      for block 0).  Thread 0 issues D1 = S [K~; Q~]^T; warps 8-15 form
+    //      W = w V; then warps 1-15 form kap^ = sigmoid(b_x + p) K^ next to
+    //      K^ (warps 8-15 waited for this block's v, g, b_x tiles in its key
+    //      transform)
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t x0 = smem_u32(sm + OFF_X), sb0 = smem_u32(sm + OFF_SB);
+      const uint32_t kh0 = smem_u32(sm + OFF_KHP);
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+        umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
+                  desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
+      }
+      if (ib == 0) {  // later blocks' [M; P_k] was issued in step 6 before
 #pragma unroll 1
         for (int ks = 0; ks < 8; ++ks) {
           const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
-                    desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
+          umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
+                    desc_kmajor_sw128(kh0 + kx), ID_N64, ks > 0);
         }
-        d1_open = true;
       }
+      d1_open = true;
+    }
+    if (warp < 8) {
       wait(B_VGB, 1);
-      const int rr = tid >> 3, ch = tid & 7;  // token rows rr, rr + 32; 16-byte chunk
+    } else {
+      const int u = tid - 256;
+      const int rr = u >> 3, ch = u & 7;  // token rows rr, rr + 32; 16-byte chunk
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int r = rr + 32 * (i & 1), kb = i >> 1;
@@ -417,39 +461,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
       }
-      if (ib + 1 < NB) {  // the next block's w_t
-        const size_t r0 = (size_t)b * T + (ib + 1) * kBlk + (tid >> 3);
-        w_lo = w_bits[r0 * H + h];
-        w_hi = w_bits[(r0 + 32) * H + h];
+      if (ib + 1 < NB) {  // the next block's w_t (0 past the block's C tokens)
+        const size_t r0 = (size_t)b * T + (ib + 1) * C + rr;
+        w_lo = rr < C ? w_bits[r0 * H + h] : 0u;
+        w_hi = rr + 32 < C ? w_bits[(r0 + 32) * H + h] : 0u;
       }
-      // p formed (warps 8-15 arrive after the gate); warp 0, late from
-      // issuing D1, goes straight to the block barrier
-      if (warp > 0) bar_named(5, kThreads - 32);
-    } else {
-      if (ib % bpc == 0) gate(ib / bpc);
-      bar_arrive_named(5, kThreads - 32);
     }
 
-    // ---- 3. K^ -> its operand slot and kap^ = sigmoid(b_x + p) K^ (warps
-    //      1-15, each as soon as its part above is done); then
-    //      G = [K~; Q~] [K^; kap^]^T in one N = 128 product per k-step
-    //      (columns 0-63 [M; P_k], 64-127 [A; P_kap]).  The commit after G
-    //      covers D1 as well.
+    // ---- 3. kap^ (warps 1-15); then the gate half of the Grams,
+    //      [A; P_kap] = [K~; Q~] kap^T.  The commit after it covers D1 and
+    //      [M; P_k] as well.
     if (warp > 0)
-      tc::kappa_block(sm + OFF_RG, sm + OFF_KHP, sm + OFF_KHP + 8192,
-                      sm + OFF_RB, s_p, 16384, tid - 32, kThreads - 32);
+      tc::kappa_in_place(sm + OFF_KHP, sm + OFF_RB, s_p, 16384, tid - 32,
+                         kThreads - 32);
     fence_async_smem();
     if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
     if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
     if (tid == 0) {  // the raw v, g, b_x buffers are free for the next block
       if (ib + 1 < NB) issue_vgb(ib + 1);
       tc_fence_after();
-      const uint32_t x0 = smem_u32(sm + OFF_X), khp0 = smem_u32(sm + OFF_KHP);
+      const uint32_t x0 = smem_u32(sm + OFF_X);
+      const uint32_t kp0 = smem_u32(sm + OFF_KHP) + 8192;
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-        umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
-                  desc_kmajor_sw128(khp0 + kx), ID_N128, ks > 0);
+        umma_bf16(tmem + TM_GK, desc_kmajor_sw128(x0 + kx),
+                  desc_kmajor_sw128(kp0 + kx), ID_N64, ks > 0);
       }
       // test only: CTA 0 of a chosen block commits to a barrier nobody
       // waits on, so the wait for MMA 1 below runs out (the products still
@@ -510,6 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- 4b. [M; P_k] (strictly lower, 32 columns per group) -> bf16
       //          operand; MMA 2; R^T -> bf16 operand (warps 4-11)
       const int part = gp - 1;
+      if (ib > 0) {  // [M; P_k] of this block, issued in the previous block's step 6
+        wait(B_GM, 13);
+        tc_fence_after();
+      }
       {
         float vals[32];
         tmem_ld32(tl + TM_GM + part * 32, vals);
@@ -553,6 +594,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
                    vals + c8 * 8);
       }
+      // the chunk mean without waiting for O: with u_i = sum_t P_kap[t][i],
+      // sum_t o_t = sum_t (Q~ S^T + P_k W)[t] - E^T u.  This group's half of
+      // the tokens of the first term, and (warps of lanes 64..127, the
+      // P_kap rows) its half of the columns of u
+      {
+        float vals[32];
+        tmem_ld32(tl + TM_D1 + 64 + part * 32, vals);
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sum += vals[e];
+        s_co[part * 128 + row] = sum;
+      }
+      if (qd >= 2) {
+        float vals[32];
+        tmem_ld32(tl + TM_GK + part * 32, vals);
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (part * 32 + e >= gr) vals[e] = 0.f;  // strictly lower
+        s_u2[(qd - 2) * 64 + part * 32 + lane] = tc::warp_reduce_scatter32(vals, lane);
+      }
     } else if (a.gin && ib % bpc == 0) {
       // warps 12-15: the chunk's gate records for the backward (p_c, h_c,
       // m_c: s_p, s_h, s_m hold them until the chunk's end)
@@ -562,8 +623,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (a.ck_m) a.ck_m[((size_t)pair * a.NC + c) * kDV + u] = s_m[u];
     }
     // ---- 4c. warps 8-15, free while warps 0-3 solve: the key side of the
-    //          next block's transform (X and the raw g tile are free)
-    if (warp >= 8 && ib + 1 < NB) keys(ib + 1);
+    //          next block's transform (X is free; K^'s slot once S += W^T K^
+    //          has read it)
+    if (warp >= 8) {
+      wait(B_WK, 12);
+      if (ib + 1 < NB) keys(ib + 1);
+    }
     fence_async_smem();
     tc_fence_before();
     if (__syncthreads_or(*s_abort)) break;
@@ -592,9 +657,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     if (gp < 2) {
       // E^T -> bf16 operand (negated by the MMAs that use it), 32 columns
-      // per group
+      // per group; this group's half of E^T u for the chunk mean
       float vals[32];
       tmem_ld32(tl + TM_D1 + gp * 32, vals);
+      float eu = 0.f;
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        eu = fmaf(vals[e], s_u2[gp * 32 + e] + s_u2[64 + gp * 32 + e], eu);
+      s_eu[gp * 128 + row] = eu;
 #pragma unroll
       for (int c8 = 0; c8 < 4; ++c8)
         st_chunk(sm + OFF_RE + sw128_chunk(row, 0, gp * 4 + c8, 128),
@@ -618,8 +688,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__syncthreads_or(*s_abort)) break;
 
     // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S -= E^T kap^ (W^T K^
-    //      was added with MMA 2)
-    wait(B_WK, 11);
+    //      was added with MMA 2).  Meanwhile warps 8-15: the block's sum of
+    //      o and, at a chunk's end, its mean m_{c+1} and the next chunk's
+    //      gate p = U_up U_down m_{c+1}
+    if (warp < 8) wait(B_WK, 11);
+    if (warp >= 8) {
+      const int u = tid - 256;
+      if (u < 128) {
+        const float bs = (s_co[u] + s_co[128 + u]) - (s_eu[u] + s_eu[128 + u]);
+        const float acc = (ib % bpc == 0) ? bs : s_m[u] + bs;
+        s_m[u] = chunk_end ? acc * invL : acc;
+      }
+      if (chunk_end && ib + 1 < NB) gate(ib / bpc + 1);
+    }
     if (tid == 0) {
       if (rec) {
         bulk_store(rec + kTcRecE, sm + OFF_AF, 16384);
@@ -637,6 +718,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(bars + B_M4);
       mark(B_M4);
+      if (ib + 1 < NB) {
+        // the next block's b-independent Grams [M; P_k] = [K~; Q~] K^T: its
+        // key side is in X and KHP (step 4c) and TM_GM was read in step 4b.
+        // Its own commit: only step 4b of the next block waits for it.
+        const uint32_t x0 = smem_u32(sm + OFF_X), kh0 = smem_u32(sm + OFF_KHP);
+#pragma unroll 1
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+          umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
+                    desc_kmajor_sw128(kh0 + kx), ID_N64, ks > 0);
+        }
+        umma_commit(bars + B_GM);
+        mark(B_GM);
+      }
     }
     wait(B_M4, 8);
     tc_fence_after();
@@ -653,13 +748,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool odd = (lane & 1) != 0;
       __nv_bfloat16* orow = o + ((size_t)b * T + t0 + gp * 16 + (odd ? 1 : 0)) * H * DVt +
                             (size_t)h * DVt + v0 + (row & ~1);
+      const bool live = gp * 16 < C;  // token group inside the block (C % 16 == 0)
 #pragma unroll
       for (int e = 0; e < 16; e += 2) {
-        msum += vals[e] + vals[e + 1];
         const float recv = __shfl_xor_sync(0xffffffffu, odd ? vals[e] : vals[e + 1], 1);
-        *reinterpret_cast<__nv_bfloat162*>(orow + (size_t)e * H * DVt) =
-            odd ? __floats2bfloat162_rn(recv, vals[e + 1])
-                : __floats2bfloat162_rn(vals[e], recv);
+        if (live)
+          *reinterpret_cast<__nv_bfloat162*>(orow + (size_t)e * H * DVt) =
+              odd ? __floats2bfloat162_rn(recv, vals[e + 1])
+                  : __floats2bfloat162_rn(vals[e], recv);
       }
       float sv[32];
       tmem_ld16(tl + TM_S + gp * 32, sv);
@@ -698,11 +794,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
     }
     fence_async_smem();
-    if (chunk_end) s_mq[gp * 128 + row] = msum;
     if (tid == 0 && rec) bulk_wait_read_all();  // T, E records read
     tc_fence_before();
     __syncthreads();
-    if (chunk_end) msum = 0.f;
   }
 
   if (*s_abort) {
@@ -714,8 +808,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) tc::drain_bar(bars + i, (npar >> i) & 1u);
   } else if (a.m_T && tid < 128) {  // the last chunk's mean
-    a.m_T[(size_t)pair * DVt + v0 + tid] =
-        ((s_mq[tid] + s_mq[128 + tid]) + (s_mq[256 + tid] + s_mq[384 + tid])) * invL;
+    a.m_T[(size_t)pair * DVt + v0 + tid] = s_m[tid];
   }
   if ((tid == 0 || tid == 256) && a.tc_rec) bulk_wait_all();
   tc_fence_before();
@@ -741,14 +834,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [B*T, H, D] bf16 tensor viewed as 3-D (D innermost); boxes of 64 x 1 x 64
-// with the 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows) {
+// [B*T, H, D] bf16 tensor viewed as 3-D (D innermost); boxes of
+// 64 x 1 x box_rows (the block's C tokens) with the 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int D, int H, long long rows,
+              int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
   cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kBlk};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base),
             dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -767,9 +861,12 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
   const long long rows = (long long)a.B * a.T;
   const bool dv2 = a.DV == 2 * kDV;
   if (dv2 && (a.ck_S || a.tc_rec)) return cudaErrorInvalidValue;  // inference only
-  if (!make_map(&mq, a.q, kDK, a.H, rows) || !make_map(&mk, a.k, kDK, a.H, rows) ||
-      !make_map(&mv, a.v, a.DV, a.H, rows) || !make_map(&mg, a.g, kDK, a.H, rows) ||
-      !make_map(&mb, a.bx, kDK, a.H, rows))
+  const int C = a.C;
+  if (C < 16 || C > kBlk || C % 16 || (C < kBlk && (a.ck_S || a.tc_rec)))
+    return cudaErrorInvalidValue;  // training: blocks of 64 only
+  if (!make_map(&mq, a.q, kDK, a.H, rows, C) || !make_map(&mk, a.k, kDK, a.H, rows, C) ||
+      !make_map(&mv, a.v, a.DV, a.H, rows, C) || !make_map(&mg, a.g, kDK, a.H, rows, C) ||
+      !make_map(&mb, a.bx, kDK, a.H, rows, C))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(
       fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);

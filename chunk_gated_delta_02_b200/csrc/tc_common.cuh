@@ -83,7 +83,8 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* p, float* x) {
 
 // Element-wise transform of one block of 64 tokens x 128 key channels (CARVE
 // summaries, gist.science, section 2.3: decay on the key axis; section 2.1:
-// the content gate b = sigmoid(b_x + U_b m_c)):
+// the content gate b = sigmoid(b_x + U_b m_c)); with dscale > 0 the g tile
+// holds raw decay logits a and the log-decay is -dscale softplus(a):
 //   Gamma_t = exp(sum_{u <= t} g_u)   K~ = K Gamma    Q~_t = Q_t Gamma_{t-1}
 //   K^ = K / Gamma                    kap^ = b K^     gamma = Gamma_63
 // All tiles are 128-byte swizzled 64-column blocks.  `x` holds [K; Q]
@@ -107,7 +108,8 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
                                                 const uint8_t* bsm,
                                                 float* s_gam, float* red,
                                                 int bar_id, uint32_t khs,
-                                                int bar_b, int n_b) {
+                                                int bar_b, int n_b,
+                                                float dscale) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
@@ -130,7 +132,8 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
+    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0)
+      gl[i][e] = (i ? gl[i - 1][e] : 0.f) + decay_act(gv[e], dscale);
   }
   float ex[8];  // exclusive prefix of the token group
   float wt[8];  // running inclusive sum over the warp's groups
@@ -202,7 +205,7 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
                                                const uint8_t* graw,
                                                float* s_gam, float* red,
                                                int bar_id, uint32_t khs,
-                                               int wbase) {
+                                               int wbase, float dscale) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
@@ -225,7 +228,8 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
+    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0)
+      gl[i][e] = (i ? gl[i - 1][e] : 0.f) + decay_act(gv[e], dscale);
   }
   float ex[8];  // exclusive prefix of the token group
   float wt[8];  // running inclusive sum over the warp's groups
@@ -281,6 +285,46 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
     *reinterpret_cast<float4*>(s_gam + j0 + 4) =
         make_float4(gprev[4], gprev[5], gprev[6], gprev[7]);
   }
+}
+
+// kap^ = sigmoid(b_x + p) K^ for one block, with K^ already in its operand
+// slot: `kh` holds K^ in rows 0..63 of each 128-row column block (blocks
+// `khs` bytes apart) and kap^ goes to rows 64..127 of the same blocks.
+// Thread t_id of n_thr takes 16-byte chunks t_id, t_id + n_thr, ... of the
+// 64 x 128 tile; the 8 threads of a quarter-warp take the 8 chunks of one
+// row (conflict-free under the swizzle).
+__device__ __forceinline__ void kappa_in_place(uint8_t* kh, const uint8_t* braw,
+                                               const float* s_p, uint32_t khs,
+                                               int t_id, int n_thr) {
+  for (int c = t_id; c < 1024; c += n_thr) {
+    const int t = c >> 4, blk = (c >> 3) & 1, ch = c & 7;
+    const uint32_t sw = (uint32_t)(t * 128 + ((ch ^ (t & 7)) << 4));
+    float kv[8], bv[8], o[8];
+    ld_chunk(kh + blk * khs + sw, kv);
+    ld_chunk(braw + blk * 8192 + sw, bv);
+    const float4 p0 = *reinterpret_cast<const float4*>(s_p + blk * 64 + ch * 8);
+    const float4 p1 = *reinterpret_cast<const float4*>(s_p + blk * 64 + ch * 8 + 4);
+    const float pj[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = sigm(bv[e] + pj[e]) * kv[e];
+    st_chunk(kh + blk * khs + 8192 + sw, o);
+  }
+}
+
+// Sum over the 32 lanes of a warp of v[i] (i < 32): lane l ends with the
+// sum of index l in v[0] (31 shuffles).
+__device__ __forceinline__ float warp_reduce_scatter32(float* v, int lane) {
+#pragma unroll
+  for (int k = 16; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const float send = up ? v[i] : v[i + k];
+      const float keep = up ? v[i + k] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+    }
+  }
+  return v[0];
 }
 
 // kap^ = sigmoid(b_x + p) K^ for one block (the gate half of

@@ -60,19 +60,28 @@ def _map_fp64(x, fn):
     return out.reshape(x.shape)
 
 
+# scale of the log-decay draw g = -softplus(z) * DECAY_SCALE; with
+# raw_decay=True the raw z itself is returned as g and the kernels apply
+# the activation with this scale
+DECAY_SCALE = 0.1
+
+
 def make_inputs(B, T, H, DK, DV, R, seed, dtype=torch.bfloat16, s0_std=0.0,
-                ub_zero=False, **_unused):
+                ub_zero=False, raw_decay=False, **_unused):
     """Draw one batch.  Returns a dict of CPU tensors:
     q k g bx [B, T, H, DK], v [B, T, H, DV], w [B, T, H], u_down [H, R, DV],
-    u_up [H, DK, R] in ``dtype``; S0 [B, H, DV, DK] fp32 or None."""
+    u_up [H, DK, R] in ``dtype``; S0 [B, H, DV, DK] fp32 or None.
+    raw_decay=True: g holds the N(0, 1) draw z instead of -softplus(z) * 0.1
+    (the same random numbers; for the kernels' fused decay activation)."""
     gen = torch.Generator().manual_seed(int(seed))
     out = {}
     out["q"] = _rows_l2_normalise(_normal(gen, (B, T, H, DK))).to(dtype)
     out["k"] = _rows_l2_normalise(_normal(gen, (B, T, H, DK))).to(dtype)
     out["v"] = _normal(gen, (B, T, H, DV)).to(dtype)
-    out["g"] = _map_fp64(_normal(gen, (B, T, H, DK)),
-                         lambda z: -torch.nn.functional.softplus(z) * 0.1
-                         ).to(dtype)
+    z = _normal(gen, (B, T, H, DK))
+    out["g"] = (z.to(dtype) if raw_decay else
+                _map_fp64(z, lambda x: -torch.nn.functional.softplus(x)
+                          * DECAY_SCALE).to(dtype))
     out["bx"] = _normal(gen, (B, T, H, DK)).to(dtype)
     out["w"] = _map_fp64(_normal(gen, (B, T, H)), torch.sigmoid).to(dtype)
     ud = _normal(gen, (H, R, DV), 0.02)

@@ -59,14 +59,22 @@ typedef enum { CARVE_BF16 = 0, CARVE_FP32 = 1 } carve_dtype;
  * Supported: B, H >= 1; T >= 0 with T % L == 0; DK, DV multiples of 16 in
  * [16, 256]; 0 <= R <= 64; L in [1, 64] or a multiple of 64 up to 256.
  * Anything else returns CARVE_ERR_UNSUPPORTED.
- * Kernel families: bf16 with DK = 128, L a multiple of 64, R <= 32, T > 0
- * runs on the tensor cores for DV = 128 (forward, training forward and
- * backward) and DV = 256 (forward without training); every other shape,
- * and fp32 inputs, on the generic CUDA-core kernels.
+ * Kernel families: bf16 with DK = 128, R <= 32, T > 0 runs on the tensor
+ * cores for DV = 128 with L a multiple of 64 (forward, training forward and
+ * backward), and for the forward without training also with DV = 256 and
+ * with L = 16, 32 or 48 (one chunk per 64-row tile); every other shape, and
+ * fp32 inputs, on the generic CUDA-core kernels.
  */
 typedef struct {
   int32_t B, T, H, DK, DV, R, L;
-  int32_t dtype; /* carve_dtype */
+  int32_t dtype;      /* carve_dtype */
+  float decay_scale;  /* 0: g is the log-decay itself (g <= 0);
+                       * s > 0: g holds raw decay logits a and the kernels
+                       * use g = -s * softplus(a) (the activation fused into
+                       * the chunk kernels, CARVE summaries, gist.science,
+                       * section 2.3 "Key-Axis Decay und Fusion"); the
+                       * backward then returns dL/da in dg.  Negative or
+                       * non-finite: CARVE_ERR_INVALID_ARG. */
 } carve_shape;
 
 /*
@@ -182,6 +190,44 @@ carve_status carve_chunk_fwd_noalloc(const carve_shape* shape,
                                      const float* S0, const float* m0,
                                      void* o, float* S_T, float* m_T,
                                      void* stream);
+
+/*
+ * One recurrent decode step for inference: the token form of the same
+ * recurrence, advancing every (sequence, head) by one new token (CARVE
+ * technical summary, gist.science, sections 1 and 2.1-2.3; the content
+ * signal m_c is the mean of the previous chunk's outputs, section 2.1).
+ *
+ *   shape        : B, H, DK, DV, R, L and dtype as for carve_chunk_fwd; T is
+ *                  ignored (one token)
+ *   q, k, g, b_x : [B, H, DK] dtype   the new token (g: log-decay, <= 0)
+ *   v            : [B, H, DV] dtype
+ *   w            : [B, H]     dtype
+ *   u_down, u_up : [H, R, DV], [H, DK, R] dtype (NULL allowed when R == 0)
+ *   pos          : [B] int32  tokens of each sequence already processed (the
+ *                  new token's index; read only: the caller advances it)
+ *   S            : [B, H, DV, DK] fp32 in/out   S_{t-1} -> S_t
+ *   m            : [B, H, DV] fp32 in/out       the current chunk's content
+ *                  signal m_c (zero for a new sequence, or m_T of a forward);
+ *                  replaced by the chunk's mean after its last token
+ *   osum         : [B, H, DV] fp32 in/out       sum of the current chunk's
+ *                  outputs so far (zero at a chunk boundary); reset to zero
+ *                  after the chunk's last token
+ *   o            : [B, H, DV] dtype   o_t = S_{t-1} q_t (overwritten)
+ *
+ * Per pair: p = U_up U_down m, b = sigmoid(b_x + p), o = S q,
+ * S' = S Diag(exp g), S = S' - (S' k)(b k)^T + w v k^T, osum += o, and when
+ * (pos + 1) % L == 0: m = osum / L, osum = 0.  A sequence processed by
+ * carve_chunk_fwd (T a multiple of L, final S_T and m_T) continues here with
+ * S = S_T, m = m_T, osum = 0, pos = T.  One CTA per (sequence, head); no
+ * workspace; asynchronous on `stream`.  Errors: INVALID_ARG, UNSUPPORTED,
+ * CUDA (launch failure).
+ */
+carve_status carve_decode_step(const carve_shape* shape,
+                               const void* q, const void* k, const void* v,
+                               const void* g, const void* b_x, const void* w,
+                               const void* u_down, const void* u_up,
+                               const int32_t* pos, float* S, float* m,
+                               float* osum, void* o, void* stream);
 
 /*
  * Synchronises `stream`, then reads the device status word that kernels

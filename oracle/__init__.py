@@ -13,6 +13,9 @@ Modules
 ``chunked``         the WY-form chunk solve written with dense fp64 linear
                     algebra; used only to pin the recurrence (the pages'
                     chunkability theorem says the two must agree).
+``decode``          the single-token decode step with its chunk bookkeeping.
+``activation``      the decay activation g = -s softplus(a) that the kernels
+                    can apply to raw decay logits, and its derivative.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` to closed
 forms, special-case reductions, a hand-computed example and finite

@@ -138,14 +138,29 @@ def _threads(threads):
         return max(1, os.cpu_count() or 1)
 
 
-def fwd_batch(inp, L, pairs=None, threads=None):
-    """Oracle forward over (b, h) pairs.  Returns {(b, h): (o, S_T, m_T)}."""
+def _activate(a, decay_scale):
+    """decay_scale > 0: the pair's `g` holds raw decay logits; replace them
+    by the log-decay the recurrence receives (oracle/activation.py).
+    Returns the raw logits (or None)."""
+    if not decay_scale:
+        return None
+    from .activation import decay_from_logits
+    raw = a["g"]
+    a["g"] = decay_from_logits(raw, decay_scale)
+    return raw
+
+
+def fwd_batch(inp, L, pairs=None, threads=None, decay_scale=0.0):
+    """Oracle forward over (b, h) pairs.  Returns {(b, h): (o, S_T, m_T)}.
+    decay_scale > 0: inp["g"] holds raw decay logits a, and the recurrence
+    runs on g = -decay_scale * softplus(a)."""
     B, _, H, _ = tuple(inp["q"].shape)
     if pairs is None:
         pairs = [(b, h) for b in range(B) for h in range(H)]
 
     def one(bh):
         a = pair_inputs(inp, *bh)
+        _activate(a, decay_scale)
         return bh, fwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
                             a["u_down"], a["u_up"], L, a["S0"], a["m0"])
 
@@ -153,10 +168,13 @@ def fwd_batch(inp, L, pairs=None, threads=None):
         return dict(ex.map(one, pairs))
 
 
-def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None):
+def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None,
+              decay_scale=0.0):
     """Oracle reverse pass over (b, h) pairs.  d_o [B, T, H, DV],
     dS_T [B, H, DV, DK] or None, dm_T [B, H, DV] or None.
-    Returns {(b, h): grads dict} (per-pair du_down / du_up, not summed)."""
+    Returns {(b, h): grads dict} (per-pair du_down / du_up, not summed).
+    decay_scale > 0: inp["g"] holds raw decay logits a, and "dg" is the
+    gradient with respect to a (chain rule through the activation)."""
     B, _, H, _ = tuple(inp["q"].shape)
     if pairs is None:
         pairs = [(b, h) for b in range(B) for h in range(H)]
@@ -164,12 +182,16 @@ def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None):
     def one(bh):
         b, h = bh
         a = pair_inputs(inp, b, h)
+        raw = _activate(a, decay_scale)
         do = np.ascontiguousarray(_np64(d_o[b, :, h, :]))
         dst = None if dS_T is None else np.ascontiguousarray(_np64(dS_T[b, h]))
         dmt = None if dm_T is None else np.ascontiguousarray(_np64(dm_T[b, h]))
-        return bh, bwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
-                            a["u_down"], a["u_up"], L, do, a["S0"], a["m0"],
-                            dst, dmt)
+        gr = bwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
+                      a["u_down"], a["u_up"], L, do, a["S0"], a["m0"], dst, dmt)
+        if raw is not None:
+            from .activation import decay_grad
+            gr["dg"] = gr["dg"] * decay_grad(raw, decay_scale)
+        return bh, gr
 
     with ThreadPoolExecutor(_threads(threads)) as ex:
         return dict(ex.map(one, pairs))

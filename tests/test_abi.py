@@ -38,10 +38,11 @@ def test_header_declarations_are_exported(lib):
 
 
 def shape(**kw):
-    d = dict(B=2, T=128, H=3, DK=64, DV=64, R=8, L=64, dtype=0)
+    d = dict(B=2, T=128, H=3, DK=64, DV=64, R=8, L=64, dtype=0,
+             decay_scale=0.0)
     d.update(kw)
     return carve.Shape(*(d[n] for n in ("B", "T", "H", "DK", "DV", "R", "L",
-                                        "dtype")))
+                                        "dtype", "decay_scale")))
 
 
 def ws_bytes(lib, s, training):
@@ -61,21 +62,41 @@ def test_workspace_bytes(lib):
     assert ws_bytes(lib, shape(T=0), 0) > 0
 
 
+def test_decay_scale_validation(lib):
+    # 0 (g is the log-decay) and any positive finite scale are accepted; a
+    # negative, NaN or infinite scale is an invalid argument
+    for ok in (0.0, 0.1, 5.0):
+        assert ws_bytes(lib, shape(decay_scale=ok), 0) > 0, ok
+    for bad in (-0.1, float("nan"), float("inf")):
+        assert ws_bytes(lib, shape(decay_scale=bad), 0) == 0, bad
+        assert call_fwd(lib, shape(decay_scale=bad), FAKE, 1 << 20) == 1, bad
+
+
 def test_status_strings_and_path(lib):
     for code, name in carve.STATUS.items():
         assert lib.carve_status_str(code).decode() == name
     assert lib.carve_fwd_path(ctypes.byref(shape())) is not None
     assert lib.carve_fwd_path(ctypes.byref(shape(DK=24))) is None
     # kernel family selection (host logic only): tensor cores for bf16,
-    # DK = 128, L % 64 == 0, R <= 32 and DV = 128 or 256; generic otherwise
+    # DK = 128, R <= 32, DV = 128 or 256 and L a multiple of 64, or (forward
+    # without training) L of 16, 32 or 48; generic otherwise
     path = lambda **kw: lib.carve_fwd_path(ctypes.byref(shape(**kw))).decode()
     tc = dict(DK=128, DV=128, R=32, L=64, T=128, dtype=carve.CARVE_BF16)
     assert path(**tc) == "tc"
     assert path(**dict(tc, DV=256)) == "tc"
     assert path(**dict(tc, L=128)) == "tc"
-    for other in (dict(DV=64), dict(DK=64), dict(L=32), dict(R=48),
+    for L in (16, 32):
+        assert path(**dict(tc, L=L)) == "tc", L
+        assert path(**dict(tc, L=L, DV=256)) == "tc", L
+    assert path(**dict(tc, L=48, T=96)) == "tc"
+    for other in (dict(DV=64), dict(DK=64), dict(L=8), dict(L=4), dict(R=48),
                   dict(dtype=carve.CARVE_FP32), dict(DV=192)):
         assert path(**dict(tc, **other)) == "generic", other
+    # training with chunks shorter than 64 tokens stays on the generic
+    # kernels: its workspace has the generic per-block checkpoints
+    s32 = shape(**dict(tc, L=32))
+    assert ws_bytes(lib, s32, 1) - ws_bytes(lib, s32, 0) >= \
+        2 * 3 * (128 // 32 + 1) * 128 * 128 * 4
     # training on the tensor-core family adds the per-block records
     # (56 KiB per block and pair), one fp32 state per pair (the final one),
     # the chunk gate inputs and gradients, and the per-pair dU partials

@@ -163,6 +163,9 @@ def test_layer_1p3b_fwd_zero_Ub():
 @pytest.mark.parametrize("L", [16, 32, 64, 128])
 def test_chunk_sweep_fwd(L):
     cfg = dict(WORKLOADS["layer_1p3b"], L=L)
+    shape = carve.make_shape(cfg["B"], cfg["T"], cfg["H"], cfg["DK"],
+                             cfg["DV"], cfg["R"], L, torch.bfloat16)
+    assert carve.fwd_path(shape) == "tc"  # every L of the sweep
     pairs = sample_pairs(cfg["B"], cfg["H"], 2, seed=L)
     errs = fwd_errors(inputs(cfg, 2, torch.bfloat16), L, pairs)
     assert_within(errs, 1e-2, "chunk sweep L=%d" % L)
@@ -211,6 +214,40 @@ def test_tensor_core_forward_matches_oracle_and_generic(case, monkeypatch):
     monkeypatch.setenv("CARVE_FWD_PATH", "generic")
     assert carve.fwd_path(shape) == "generic"
     _, o_g, S_g, m_g, _ = run_fwd(inp, L, training=True)
+    from _parity import rel as _rel
+    assert _rel(o_tc.float().cpu(), o_g.float().cpu()) < 1e-2
+    assert _rel(S_tc.cpu(), S_g.cpu()) < 1e-2
+    assert _rel(m_tc.cpu(), m_g.cpu()) < 1e-2
+
+
+SHORT_CHUNK_CASES = [
+    # B, H, T, DV, R, L  (chunks shorter than the 64-row tiles: the chunk is
+    # the block, rows past it stay zero)
+    (1, 2, 256, 128, 32, 16),
+    (2, 1, 320, 128, 8, 32),
+    (1, 1, 192, 128, 16, 48),
+    (1, 1, 64, 128, 0, 32),
+    (1, 2, 128, 256, 32, 16),
+    (1, 1, 160, 256, 16, 32),
+]
+
+
+@pytest.mark.parametrize("case", SHORT_CHUNK_CASES,
+                         ids=lambda c: "x".join(map(str, c)))
+def test_tensor_core_forward_short_chunks(case, monkeypatch):
+    B, H, T, DV, R, L = case
+    cfg = dict(B=B, H=H, T=T, DK=128, DV=DV, R=R, L=L)
+    inp = inputs(cfg, 61, torch.bfloat16)
+    if R > 0:  # a gate that really moves between chunks
+        inp["u_down"] = (inp["u_down"].float() * 25).to(torch.bfloat16)
+        inp["u_up"] = (inp["u_up"].float() * 25).to(torch.bfloat16)
+    _rand_state(inp, 62)
+    shape = carve.make_shape(B, T, H, 128, DV, R, L, torch.bfloat16)
+    assert carve.fwd_path(shape) == "tc"
+    assert_within(fwd_errors(inp, L), 1e-2, "tc fwd short chunks %s" % (case,))
+    _, o_tc, S_tc, m_tc, _ = run_fwd(inp, L)
+    monkeypatch.setenv("CARVE_FWD_PATH", "generic")
+    _, o_g, S_g, m_g, _ = run_fwd(inp, L)
     from _parity import rel as _rel
     assert _rel(o_tc.float().cpu(), o_g.float().cpu()) < 1e-2
     assert _rel(S_tc.cpu(), S_g.cpu()) < 1e-2
