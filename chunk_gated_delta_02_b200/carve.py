@@ -22,13 +22,14 @@ STATUS = {0: "CARVE_OK", 1: "CARVE_ERR_INVALID_ARG", 2: "CARVE_ERR_UNSUPPORTED",
 # Entry points declared in include/carve.h (the ABI test checks the list).
 EXPORTS = ("carve_workspace_bytes", "carve_chunk_fwd", "carve_chunk_bwd",
            "carve_get_status", "carve_reset_status", "carve_status_str",
-           "carve_fwd_path", "carve_chunk_fwd_noalloc", "carve_decode_step")
+           "carve_fwd_path", "carve_chunk_fwd_noalloc", "carve_decode_step",
+           "carve_chunk_fwd_varlen")
 
 
 class Shape(ctypes.Structure):
     _fields_ = ([(n, ctypes.c_int32)
                  for n in ("B", "T", "H", "DK", "DV", "R", "L", "dtype")]
-                + [("decay_scale", ctypes.c_float)])
+                + [("decay_scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int32)])
 
 
 class CarveError(RuntimeError):
@@ -68,6 +69,8 @@ def lib():
         L.carve_fwd_path.restype = ctypes.c_char_p
         L.carve_decode_step.argtypes = [sp] + [vp] * 13 + [vp]
         L.carve_decode_step.restype = i32
+        L.carve_chunk_fwd_varlen.argtypes = [sp] + [vp] * 15 + [sz, vp]
+        L.carve_chunk_fwd_varlen.restype = i32
         _lib = L
     return _lib
 
@@ -80,11 +83,14 @@ def _stream(device):
     return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
 
 
-def make_shape(B, T, H, DK, DV, R, L, dtype, decay_scale=0.0):
+def make_shape(B, T, H, DK, DV, R, L, dtype, decay_scale=0.0,
+               qk_l2norm=False):
     """decay_scale > 0: `g` holds raw decay logits a and the kernels use
-    g = -decay_scale * softplus(a); the backward then returns dL/da."""
+    g = -decay_scale * softplus(a); the backward then returns dL/da.
+    qk_l2norm: q and k are raw and the kernels normalise them per token."""
     return Shape(B, T, H, DK, DV, R, L, _DTYPES[dtype] if isinstance(
-        dtype, torch.dtype) else int(dtype), float(decay_scale))
+        dtype, torch.dtype) else int(dtype), float(decay_scale),
+        int(bool(qk_l2norm)))
 
 
 def workspace_bytes(shape, training):
@@ -124,7 +130,7 @@ def _dims(q, v, u_down):
 
 def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
               training=False, workspace=None, o=None, want_state=True,
-              decay_scale=0.0):
+              decay_scale=0.0, qk_l2norm=False):
     """Forward pass.  Returns (o, S_T, m_T, workspace).
 
     q, k, g, bx [B, T, H, DK]; v [B, T, H, DV]; w [B, T, H]; u_down
@@ -146,7 +152,7 @@ def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
         _check(S0, "S0", torch.float32, (B, H, DV, DK), dev)
     if m0 is not None:
         _check(m0, "m0", torch.float32, (B, H, DV), dev)
-    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale)
+    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
     nbytes = workspace_bytes(shape, training)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
@@ -167,8 +173,60 @@ def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
     return o, S_T, m_T, workspace
 
 
+def chunk_fwd_varlen(q, k, v, g, bx, w, u_down, u_up, L, cu_seqlens, S0=None,
+                     m0=None, workspace=None, o=None, want_state=True,
+                     decay_scale=0.0, qk_l2norm=False):
+    """Forward (no training) over packed sequences of different lengths.
+    Returns (o, S_T, m_T, workspace).
+
+    q, k, g, bx [T, H, DK]; v [T, H, DV]; w [T, H] (bf16 or fp32); u_down
+    [H, R, DV]; u_up [H, DK, R]; cu_seqlens [N + 1] int32 on the device
+    (sequence n is tokens cu_seqlens[n] .. cu_seqlens[n + 1] - 1); S0
+    [N, H, DV, DK], m0 [N, H, DV] fp32 or None.  S_T, m_T are per sequence."""
+    dev = q.device
+    dt = q.dtype
+    if dt not in _DTYPES:
+        raise ValueError("dtype must be bfloat16 or float32")
+    T, H, DK = q.shape
+    DV = v.shape[-1]
+    R = u_down.shape[1] if u_down is not None else 0
+    N = cu_seqlens.numel() - 1
+    if N < 1:
+        raise ValueError("cu_seqlens needs at least two entries")
+    for t, n, s in ((q, "q", (T, H, DK)), (k, "k", (T, H, DK)),
+                    (v, "v", (T, H, DV)), (g, "g", (T, H, DK)),
+                    (bx, "bx", (T, H, DK)), (w, "w", (T, H)),
+                    (u_down, "u_down", (H, R, DV)), (u_up, "u_up", (H, DK, R))):
+        _check(t, n, dt, s, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, (N + 1,), dev)
+    if S0 is not None:
+        _check(S0, "S0", torch.float32, (N, H, DV, DK), dev)
+    if m0 is not None:
+        _check(m0, "m0", torch.float32, (N, H, DV), dev)
+    shape = make_shape(N, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
+    nbytes = workspace_bytes(shape, False)
+    if workspace is None or workspace.numel() < nbytes:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        workspace[:256].zero_()
+    if o is None:
+        o = torch.zeros((T, H, DV), dtype=dt, device=dev)
+    S_T = m_T = None
+    if want_state:
+        S_T = torch.empty((N, H, DV, DK), dtype=torch.float32, device=dev)
+        m_T = torch.empty((N, H, DV), dtype=torch.float32, device=dev)
+    rc = lib().carve_chunk_fwd_varlen(
+        ctypes.byref(shape), _ptr(cu_seqlens), _ptr(q), _ptr(k), _ptr(v),
+        _ptr(g), _ptr(bx), _ptr(w), _ptr(u_down), _ptr(u_up), _ptr(S0),
+        _ptr(m0), _ptr(o), _ptr(S_T), _ptr(m_T), _ptr(workspace),
+        ctypes.c_size_t(workspace.numel()), _stream(dev))
+    if rc != 0:
+        raise CarveError("carve_chunk_fwd_varlen", rc)
+    return o, S_T, m_T, workspace
+
+
 def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
-              dm_T=None, want_dS0=True, out=None, decay_scale=0.0):
+              dm_T=None, want_dS0=True, out=None, decay_scale=0.0,
+              qk_l2norm=False):
     """Backward pass after a training-mode chunk_fwd with the same inputs
     (and the same decay_scale; with decay_scale > 0, "dg" is dL/da of the
     raw decay logits).  Returns a dict: dq dk dg dbx [B, T, H, DK], dv
@@ -182,7 +240,7 @@ def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
         _check(dS_T, "dS_T", torch.float32, (B, H, DV, DK), dev)
     if dm_T is not None:
         _check(dm_T, "dm_T", torch.float32, (B, H, DV), dev)
-    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale)
+    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
     if out is None:
         e = lambda s, d=dt: torch.empty(s, dtype=d, device=dev)
         out = dict(dq=e((B, T, H, DK)), dk=e((B, T, H, DK)),
@@ -206,7 +264,7 @@ def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
 
 
 def decode_step(q, k, v, g, bx, w, u_down, u_up, L, pos, S, m, osum, o=None,
-                decay_scale=0.0):
+                decay_scale=0.0, qk_l2norm=False):
     """One recurrent decode step (one new token per (sequence, head)).
 
     q, k, g, bx [B, H, DK]; v [B, H, DV]; w [B, H] (bf16 or fp32); u_down
@@ -231,7 +289,7 @@ def decode_step(q, k, v, g, bx, w, u_down, u_up, L, pos, S, m, osum, o=None,
     _check(osum, "osum", torch.float32, (B, H, DV), dev)
     if o is None:
         o = torch.empty((B, H, DV), dtype=dt, device=dev)
-    shape = make_shape(B, 1, H, DK, DV, R, L, dt, decay_scale)
+    shape = make_shape(B, 1, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
     rc = lib().carve_decode_step(
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(bx),
         _ptr(w), _ptr(u_down), _ptr(u_up), _ptr(pos), _ptr(S), _ptr(m),

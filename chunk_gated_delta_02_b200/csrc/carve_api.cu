@@ -20,12 +20,12 @@ carve_status check_shape(const carve_shape* s) {
     return CARVE_ERR_INVALID_ARG;
   if (!(s->decay_scale >= 0.f) || s->decay_scale > 3.0e38f)  // NaN, < 0, inf
     return CARVE_ERR_INVALID_ARG;
+  if (s->qk_l2norm != 0 && s->qk_l2norm != 1) return CARVE_ERR_INVALID_ARG;
   if (s->DK % 16 || s->DV % 16 || s->DK > 256 || s->DV > 256)
     return CARVE_ERR_UNSUPPORTED;
   if (s->R > kMaxR) return CARVE_ERR_UNSUPPORTED;
   if (!(s->L <= kMaxBlock || (s->L % kMaxBlock == 0 && s->L <= 256)))
     return CARVE_ERR_UNSUPPORTED;
-  if (s->T % s->L) return CARVE_ERR_UNSUPPORTED;
   // all element indices are computed in 64-bit; grid is B*H CTAs
   if ((long long)s->B * s->H > (1LL << 30)) return CARVE_ERR_UNSUPPORTED;
   const int C = block_len(s->L);
@@ -83,6 +83,7 @@ extern "C" {
 
 size_t carve_workspace_bytes(const carve_shape* shape, int training) {
   if (check_shape(shape) != CARVE_OK) return 0;
+  if (training && shape->T % shape->L) return 0;  // training: whole chunks
   return ws_layout(*shape, training != 0, use_tc_fwd(*shape, training != 0))
       .total;
 }
@@ -115,6 +116,7 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   carve_status st = check_shape(shape);
   if (st != CARVE_OK) return st;
   const carve_shape& s = *shape;
+  if (training && s.T % s.L) return CARVE_ERR_UNSUPPORTED;
   const bool tok = s.T > 0;
   if (tok && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) ||
               !ptr_ok(b_x) || !ptr_ok(w) || !ptr_ok(o)))
@@ -144,9 +146,52 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   a.gin = training && L.gin ? (float*)(ws + L.gin) : nullptr;
   a.hdr = (WsHeader*)ws;
   a.dscale = s.decay_scale;
+  a.qknorm = s.qk_l2norm;
   test_knobs(&a.spin, &a.stall_block);
   cudaError_t e = tc ? launch_fwd_tc(a, (cudaStream_t)stream)
                       : launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
+  return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
+}
+
+carve_status carve_chunk_fwd_varlen(
+    const carve_shape* shape, const int32_t* cu_seqlens, const void* q,
+    const void* k, const void* v, const void* g, const void* b_x,
+    const void* w, const void* u_down, const void* u_up, const float* S0,
+    const float* m0, void* o, float* S_T, float* m_T, void* workspace,
+    size_t workspace_bytes, void* stream) {
+  carve_status st = check_shape(shape);
+  if (st != CARVE_OK) return st;
+  const carve_shape& s = *shape;
+  if (!ptr_ok(cu_seqlens)) return CARVE_ERR_INVALID_ARG;
+  const bool tok = s.T > 0;
+  if (tok && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) ||
+              !ptr_ok(b_x) || !ptr_ok(w) || !ptr_ok(o)))
+    return CARVE_ERR_INVALID_ARG;
+  if (s.R > 0 && (!ptr_ok(u_down) || !ptr_ok(u_up)))
+    return CARVE_ERR_INVALID_ARG;
+  if (!opt_ptr_ok(S0) || !opt_ptr_ok(m0) || !opt_ptr_ok(S_T) ||
+      !opt_ptr_ok(m_T))
+    return CARVE_ERR_INVALID_ARG;
+  const bool tc = use_tc_fwd(s, false);
+  const WsLayout L = ws_layout(s, false, tc);
+  if (!workspace || !aligned16(workspace)) return CARVE_ERR_WORKSPACE;
+  if (workspace_bytes < L.total) return CARVE_ERR_WORKSPACE;
+  char* ws = (char*)workspace;
+  FwdArgs a{};
+  a.B = s.B; a.T = s.T; a.H = s.H; a.DK = s.DK; a.DV = s.DV; a.R = s.R;
+  a.L = s.L; a.C = L.C; a.NB = L.NB; a.NC = L.NC;
+  a.q = q; a.k = k; a.v = v; a.g = g; a.bx = b_x; a.w = w;
+  a.u_down = u_down; a.u_up = u_up; a.S0 = S0; a.m0 = m0;
+  a.o = o; a.S_T = S_T; a.m_T = m_T;
+  a.scratch = (float*)(ws + L.scratch);
+  a.scratch_per_pair = L.scratch_per_pair;
+  a.hdr = (WsHeader*)ws;
+  a.dscale = s.decay_scale;
+  a.qknorm = s.qk_l2norm;
+  a.cu = cu_seqlens;
+  test_knobs(&a.spin, &a.stall_block);
+  cudaError_t e = tc ? launch_fwd_tc(a, (cudaStream_t)stream)
+                     : launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }
 
@@ -163,6 +208,7 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   carve_status st = check_shape(shape);
   if (st != CARVE_OK) return st;
   const carve_shape& s = *shape;
+  if (s.T % s.L) return CARVE_ERR_UNSUPPORTED;  // training: whole chunks
   const bool tok = s.T > 0;
   if (tok && (!ptr_ok(q) || !ptr_ok(k) || !ptr_ok(v) || !ptr_ok(g) ||
               !ptr_ok(b_x) || !ptr_ok(w) || !ptr_ok(d_o) || !ptr_ok(dq) ||
@@ -200,6 +246,7 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   a.du_down = du_down; a.du_up = du_up; a.dS0 = dS0; a.dm0 = dm0;
   a.hdr = (WsHeader*)ws;
   a.dscale = s.decay_scale;
+  a.qknorm = s.qk_l2norm;
   test_knobs(&a.spin, &a.stall_block);
   cudaError_t e = tc ? launch_bwd_tc(a, (cudaStream_t)stream)
                       : launch_bwd_generic(a, s.dtype, (cudaStream_t)stream);
@@ -229,6 +276,7 @@ carve_status carve_decode_step(const carve_shape* shape, const void* q,
   a.u_down = u_down; a.u_up = u_up; a.pos = pos;
   a.S = S; a.m = m; a.osum = osum; a.o = o;
   a.dscale = s.decay_scale;
+  a.qknorm = s.qk_l2norm;
   return launch_decode(a, s.dtype, (cudaStream_t)stream) == cudaSuccess
              ? CARVE_OK
              : CARVE_ERR_CUDA;

@@ -140,6 +140,28 @@ __global__ void __launch_bounds__(kDecThreads)
     for (int i = tid; i < nu; i += kDecThreads) reinterpret_cast<uint4*>(s_uu)[i] = uu4[i];
   }
   __syncthreads();
+  if (a.qknorm) {  // fused normalisation: q / |q|, k / |k| (warp 0 reduces)
+    if (warp == 0) {
+      float sq = 0.f, sk = 0.f;
+      for (int j = lane; j < DK; j += 32) {
+        sq = fmaf(s_q[j], s_q[j], sq);
+        sk = fmaf(s_k[j], s_k[j], sk);
+      }
+      sq = allsum(sq);
+      sk = allsum(sk);
+      if (lane == 0) {  // s_kp is free until the gate below
+        s_kp[0] = sq > 0.f ? 1.0f / sqrtf(sq) : 0.f;
+        s_kp[1] = sk > 0.f ? 1.0f / sqrtf(sk) : 0.f;
+      }
+    }
+    __syncthreads();
+    const float iq = s_kp[0], ik = s_kp[1];
+    __syncthreads();  // every thread has read them before the gate rewrites s_kp
+    for (int j = tid; j < DK; j += kDecThreads) {
+      s_q[j] *= iq;
+      s_k[j] *= ik;
+    }
+  }
   for (int j = tid; j < DK; j += kDecThreads)
     s_al[j] = expf(decay_act(s_al[j], a.dscale));
   // h = U_down m_c: one warp per rank

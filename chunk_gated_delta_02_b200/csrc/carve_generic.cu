@@ -99,6 +99,34 @@ __device__ void content_gate(const TIn* ud, const TIn* uu, const float* s_m,
   __syncthreads();
 }
 
+// Per-token inverse Euclidean norms of q and k over DK for the block's Cb
+// tokens (one warp per token), or 1 when the inputs are used as given.
+template <typename TIn>
+__device__ void token_inv_norms(const TIn* q, const TIn* k, int b, int t0,
+                                int T, int h, int H, int Cb, int DK,
+                                float* s_qn, float* s_kn, int on) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = warp; i < Cb; i += blockDim.x >> 5) {
+    float sq = 0.f, sk = 0.f;
+    if (on)
+      for (int j = lane; j < DK; j += 32) {
+        const size_t x = bthd(b, t0 + i, h, j, T, H, DK);
+        const float qq = ldf(q, x), kk = ldf(k, x);
+        sq = fmaf(qq, qq, sq);
+        sk = fmaf(kk, kk, sk);
+      }
+    for (int o = 16; o >= 1; o >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      sk += __shfl_xor_sync(0xffffffffu, sk, o);
+    }
+    if (lane == 0) {
+      s_qn[i] = on ? 1.0f / sqrtf(sq) : 1.f;
+      s_kn[i] = on ? 1.0f / sqrtf(sk) : 1.f;
+    }
+  }
+  __syncthreads();
+}
+
 // Decay scan and gated operands of one block.  Writes K~, K^, Q~, kap^
 // ([C][DK] fp32), optionally log Gamma, and gamma (s_gam), plus W = w V.
 template <typename TIn>
@@ -108,12 +136,13 @@ __device__ void block_operands(const TIn* q, const TIn* k, const TIn* v,
                                int H, int C, int DK, int DV, float* Kt,
                                float* Kh, float* Qt, float* Kp, float* Gl,
                                float* s_gam, float* s_w, float* W,
-                               float dscale) {
+                               float dscale, const float* s_qn,
+                               const float* s_kn) {
   for (int j = threadIdx.x; j < DK; j += blockDim.x) {
     float G = 0.f;
     for (int i = 0; i < C; ++i) {
       const size_t x = bthd(b, t0 + i, h, j, T, H, DK);
-      const float kk = ldf(k, x), qq = ldf(q, x);
+      const float kk = ldf(k, x) * s_kn[i], qq = ldf(q, x) * s_qn[i];
       const float bb = sigm(ldf(bx, x) + s_p[j]);
       const float Gm = G;
       G += decay_act(ldf(g, x), dscale);
@@ -177,6 +206,8 @@ __global__ void __launch_bounds__(kThreads) fwd_generic_kernel(FwdArgs a) {
   float* s_p = s_h + kMaxR;   // DK
   float* s_gam = s_p + DK;    // DK
   float* s_w = s_gam + DK;    // C
+  float* s_qn = s_w + C;      // C: per-token inverse norms of q, k
+  float* s_kn = s_qn + C;     // C
 
   float* Kt = a.scratch + (size_t)pair * a.scratch_per_pair;
   float* Kh = Kt + C * DK;
@@ -193,54 +224,79 @@ __global__ void __launch_bounds__(kThreads) fwd_generic_kernel(FwdArgs a) {
     S[i] = a.S0 ? a.S0[(size_t)pair * SZ + i] : 0.f;
   for (int i = tid; i < DV; i += nt)
     s_m[i] = a.m0 ? a.m0[(size_t)pair * DV + i] : 0.f;
+  // this sequence's tokens: B sequences of T tokens, or packed sequences
+  // [cu[b], cu[b + 1]) of a T-token tensor; the last block may be partial
+  int tok0 = b * T, Tn = T;
+  if (a.cu) {
+    tok0 = a.cu[b];
+    Tn = a.cu[b + 1] - tok0;
+    if (tok0 < 0 || Tn < 0 || tok0 > T - Tn) {  // malformed offsets: skip
+      if (tid == 0) {
+        atomicExch(&a.hdr->status, (uint32_t)CARVE_ERR_INVALID_ARG);
+        a.hdr->where = 90;
+      }
+      tok0 = 0;
+      Tn = 0;
+    }
+  }
   __syncthreads();
 
-  const int bpc = a.L / C;
-  for (int c = 0; c < a.NC; ++c) {
-    if (a.ck_m)
-      for (int i = tid; i < DV; i += nt)
-        a.ck_m[((size_t)pair * a.NC + c) * DV + i] = s_m[i];
-    content_gate(ud, uu, s_m, s_h, s_p, h, R, DK, DV);
-    for (int i = tid; i < DV; i += nt) s_msum[i] = 0.f;
-    for (int blk = 0; blk < bpc; ++blk) {
-      const int ib = c * bpc + blk, t0 = ib * C;
+  // chunks of L tokens from the sequence's start, solved in blocks of up to
+  // C tokens (token addresses below use the packed index tok0 + t)
+  for (int t0 = 0; t0 < Tn; t0 += C) {
+    const int Cb = min(C, Tn - t0);
+    const int c = t0 / a.L, ib = t0 / C;
+    if (t0 % a.L == 0) {  // first block of chunk c: its gate
+      if (a.ck_m)
+        for (int i = tid; i < DV; i += nt)
+          a.ck_m[((size_t)pair * a.NC + c) * DV + i] = s_m[i];
+      content_gate(ud, uu, s_m, s_h, s_p, h, R, DK, DV);
+      for (int i = tid; i < DV; i += nt) s_msum[i] = 0.f;
+    }
+    {
+      const int tt = tok0 + t0;  // packed index of the block's first token
       if (a.ck_S) {
         float* dst = a.ck_S + ((size_t)pair * (a.NB + 1) + ib) * SZ;
         for (size_t i = tid; i < SZ; i += nt) dst[i] = S[i];
       }
-      block_operands(q, k, v, g, bx, w, s_p, b, h, t0, T, H, C, DK, DV, Kt,
-                     Kh, Qt, Kp, (float*)nullptr, s_gam, s_w, W, a.dscale);
-      block_grams(Kt, Kh, Qt, Kp, C, DK, sA, sT, sM, sPk, sPq);
+      token_inv_norms(q, k, 0, tt, T, h, H, Cb, DK, s_qn, s_kn, a.qknorm);
+      block_operands(q, k, v, g, bx, w, s_p, 0, h, tt, T, H, Cb, DK, DV, Kt,
+                     Kh, Qt, Kp, (float*)nullptr, s_gam, s_w, W, a.dscale,
+                     s_qn, s_kn);
+      block_grams(Kt, Kh, Qt, Kp, Cb, DK, sA, sT, sM, sPk, sPq);
       // R = K~ S^T + M W ;  E = T R
-      mm(Rr, DV, Kt, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
-      mm(Rr, DV, sM, C, 1, W, DV, 1, C, DV, C, 1.f, true, false);
-      mm(E, DV, sT, C, 1, Rr, DV, 1, C, DV, C, 1.f, false, false);
+      mm(Rr, DV, Kt, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
+      mm(Rr, DV, sM, Cb, 1, W, DV, 1, Cb, DV, Cb, 1.f, true, false);
+      mm(E, DV, sT, Cb, 1, Rr, DV, 1, Cb, DV, Cb, 1.f, false, false);
       // O = Q~ S^T + P_k W - P_kap E
-      mm(O, DV, Qt, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
-      mm(O, DV, sPk, C, 1, W, DV, 1, C, DV, C, 1.f, true, false);
-      mm(O, DV, sPq, C, 1, E, DV, 1, C, DV, C, -1.f, true, false);
-      for (int idx = tid; idx < C * DV; idx += nt) {
+      mm(O, DV, Qt, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
+      mm(O, DV, sPk, Cb, 1, W, DV, 1, Cb, DV, Cb, 1.f, true, false);
+      mm(O, DV, sPq, Cb, 1, E, DV, 1, Cb, DV, Cb, -1.f, true, false);
+      for (int idx = tid; idx < Cb * DV; idx += nt) {
         const int i = idx / DV, vv = idx - i * DV;
-        stf(o, bthd(b, t0 + i, h, vv, T, H, DV), O[idx]);
+        stf(o, bthd(0, tt + i, h, vv, T, H, DV), O[idx]);
       }
       for (int vv = tid; vv < DV; vv += nt) {
         float acc = 0.f;
-        for (int i = 0; i < C; ++i) acc += O[i * DV + vv];
+        for (int i = 0; i < Cb; ++i) acc += O[i * DV + vv];
         s_msum[vv] += acc;
       }
       // S <- (S + W^T K^ - E^T kap^) Diag(gamma)
       for (size_t idx = tid; idx < SZ; idx += nt) {
         const int vv = (int)(idx / DK), j = (int)(idx - (size_t)vv * DK);
         float acc = S[idx];
-        for (int i = 0; i < C; ++i)
+        for (int i = 0; i < Cb; ++i)
           acc = fmaf(W[i * DV + vv], Kh[i * DK + j],
                      fmaf(-E[i * DV + vv], Kp[i * DK + j], acc));
         S[idx] = acc * s_gam[j];
       }
       __syncthreads();
     }
-    for (int i = tid; i < DV; i += nt) s_m[i] = s_msum[i] / (float)a.L;
-    __syncthreads();
+    if ((t0 + Cb) % a.L == 0 || t0 + Cb == Tn) {  // chunk end (or the
+      // sequence's end inside a chunk: that partial mean still divides by L)
+      for (int i = tid; i < DV; i += nt) s_m[i] = s_msum[i] / (float)a.L;
+      __syncthreads();
+    }
   }
   if (a.ck_S) {
     float* dst = a.ck_S + ((size_t)pair * (a.NB + 1) + a.NB) * SZ;
@@ -301,6 +357,8 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
   float* s_dlg = s_gam + DK; // DK
   float* s_dp = s_dlg + DK;  // DK
   float* s_w = s_dp + DK;    // C
+  float* s_qn = s_w + C;     // C: per-token inverse norms of q, k
+  float* s_kn = s_qn + C;    // C
 
   float* Kt = a.scratch + (size_t)pair * a.scratch_per_pair;
   float* Kh = Kt + C * DK;
@@ -320,6 +378,8 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
   float* dW = dR + C * DV;
   float* dS = dW + C * DV;
   float* dSb = dS + (size_t)DV * DK;
+  float* Dq = dSb + (size_t)DV * DK;  // gradients of the unit q, k rows
+  float* Dk = Dq + C * DK;            // (fused normalisation only)
 
   float* dUd = a.du + (size_t)pair * ((size_t)R * DV + (size_t)DK * R);
   float* dUu = dUd + (size_t)R * DV;
@@ -344,8 +404,9 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
       const int ib = c * bpc + blk, t0 = ib * C;
       const float* S = a.ck_S + ((size_t)pair * (a.NB + 1) + ib) * SZ;
       const float* Sn = S + SZ;  // state at the end of this block
+      token_inv_norms(q, k, b, t0, T, h, H, C, DK, s_qn, s_kn, a.qknorm);
       block_operands(q, k, v, g, bx, w, s_p, b, h, t0, T, H, C, DK, DV, Kt,
-                     Kh, Qt, Kp, Gl, s_gam, s_w, W, a.dscale);
+                     Kh, Qt, Kp, Gl, s_gam, s_w, W, a.dscale, s_qn, s_kn);
       block_grams(Kt, Kh, Qt, Kp, C, DK, sA, sT, sM, sPk, sPq);
       mm(Rr, DV, Kt, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
       mm(Rr, DV, sM, C, 1, W, DV, 1, C, DV, C, 1.f, true, false);
@@ -425,10 +486,17 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
           const float G = Gl[e];
           const float Gm = i > 0 ? Gl[e - DK] : 0.f;
           const float gam = expf(G), igam = expf(-G);
-          const float kk = ldf(k, x);
+          const float kk = ldf(k, x) * s_kn[i];
           const float bb = sigm(ldf(bx, x) + s_p[j]);
-          stf(dq, x, dQt[e] * expf(Gm));
-          stf(dk, x, dKt[e] * gam + dKh[e] * igam + dKp[e] * bb * igam);
+          const float gq = dQt[e] * expf(Gm);
+          const float gk = dKt[e] * gam + dKh[e] * igam + dKp[e] * bb * igam;
+          if (a.qknorm) {  // gradients of the unit rows: projected below
+            Dq[e] = gq;
+            Dk[e] = gk;
+          } else {
+            stf(dq, x, gq);
+            stf(dk, x, gk);
+          }
           const float dz = dKp[e] * kk * igam * bb * (1.f - bb);
           stf(dbx, x, dz);
           s_dp[j] += dz;
@@ -443,6 +511,30 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
         }
       }
       __syncthreads();
+      if (a.qknorm) {
+        // fused normalisation: x^ = x / |x| per token, so the raw
+        // gradient is (dx^ - x^ (x^ . dx^)) / |x| (one warp per token)
+        const int warp = tid >> 5, lane = tid & 31;
+        for (int i = warp; i < C; i += nt >> 5) {
+          float dotq = 0.f, dotk = 0.f;
+          for (int j = lane; j < DK; j += 32) {
+            const size_t x = bthd(b, t0 + i, h, j, T, H, DK);
+            dotq = fmaf(ldf(q, x) * s_qn[i], Dq[i * DK + j], dotq);
+            dotk = fmaf(ldf(k, x) * s_kn[i], Dk[i * DK + j], dotk);
+          }
+          for (int o = 16; o >= 1; o >>= 1) {
+            dotq += __shfl_xor_sync(0xffffffffu, dotq, o);
+            dotk += __shfl_xor_sync(0xffffffffu, dotk, o);
+          }
+          for (int j = lane; j < DK; j += 32) {
+            const size_t x = bthd(b, t0 + i, h, j, T, H, DK);
+            const float qh = ldf(q, x) * s_qn[i], kh = ldf(k, x) * s_kn[i];
+            stf(dq, x, (Dq[i * DK + j] - qh * dotq) * s_qn[i]);
+            stf(dk, x, (Dk[i * DK + j] - kh * dotk) * s_kn[i]);
+          }
+        }
+        __syncthreads();
+      }
     }
     // gate of chunk c: p = U_up h, h = U_down m_c
     for (int idx = tid; idx < DK * R; idx += nt) {
@@ -496,10 +588,10 @@ __global__ void du_reduce_kernel(const float* __restrict__ part, int B, int H,
 }  // namespace
 
 size_t generic_fwd_smem_bytes(int C, int DK, int DV) {
-  return (size_t)(5 * C * C + 2 * DV + kMaxR + 2 * DK + C) * sizeof(float);
+  return (size_t)(5 * C * C + 2 * DV + kMaxR + 2 * DK + 3 * C) * sizeof(float);
 }
 size_t generic_bwd_smem_bytes(int C, int DK, int DV) {
-  return (size_t)(9 * C * C + 2 * DV + 2 * kMaxR + 4 * DK + C) * sizeof(float);
+  return (size_t)(9 * C * C + 2 * DV + 2 * kMaxR + 4 * DK + 3 * C) * sizeof(float);
 }
 
 cudaError_t launch_fwd_generic(const FwdArgs& a, int dtype, cudaStream_t st) {

@@ -39,13 +39,14 @@ constexpr size_t kTcRecBytes = 57344;
 // (the training forward, whose records this describes, and the backward).
 inline bool tc_shape(const carve_shape& s) {
   return s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 128 &&
-         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0;
+         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0 && !s.qk_l2norm;
 }
 // The tensor-core forward also runs, without training, DV = 256 (two CTAs
 // per pair) and chunks of 16, 32 or 48 tokens (one chunk per block, the
 // 64-row tiles zero past the chunk).
 inline bool tc_fwd_shape(const carve_shape& s, bool training) {
   if (tc_shape(s)) return true;
+  if (training) return false;
   const bool chunk_ok = s.L % kMaxBlock == 0 || (s.L < kMaxBlock && s.L % 16 == 0);
   return !training && s.dtype == CARVE_BF16 && s.DK == 128 &&
          (s.DV == 128 || s.DV == 256) && chunk_ok && s.R <= 32 && s.T > 0;
@@ -78,7 +79,7 @@ inline size_t generic_fwd_scratch_floats(int C, int DK, int DV) {
   return 4 * (size_t)C * DK + 4 * (size_t)C * DV + (size_t)DV * DK;
 }
 inline size_t generic_bwd_scratch_floats(int C, int DK, int DV) {
-  return 9 * (size_t)C * DK + 7 * (size_t)C * DV + 2 * (size_t)DV * DK;
+  return 11 * (size_t)C * DK + 7 * (size_t)C * DV + 2 * (size_t)DV * DK;
 }
 
 // tc: the tensor-core forward writes this workspace.  It needs no generic
@@ -166,6 +167,10 @@ struct FwdArgs {
   long long spin;   // cycles a device-side wait spins before it gives up
   int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
   float dscale;     // decay activation scale (0: g is the log-decay)
+  int qknorm;       // 1: q, k are normalised per token inside the kernels
+  // packed sequences: B sequences at token offsets cu[b] .. cu[b + 1] of a
+  // T-token tensor ([T, H, D] layouts), or NULL: B sequences of T tokens
+  const int32_t* cu;
 };
 
 struct BwdArgs {
@@ -185,6 +190,7 @@ struct BwdArgs {
   long long spin;   // cycles a device-side wait spins before it gives up
   int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
   float dscale;     // decay activation scale (0: g is the log-decay)
+  int qknorm;       // 1: q, k are normalised per token inside the kernels
 };
 
 // Arguments of the decode step (one token per (sequence, head)).
@@ -195,6 +201,7 @@ struct DecArgs {
   float *S, *m, *osum;  // [B, H, DV, DK], [B, H, DV], [B, H, DV] in/out
   void* o;              // [B, H, DV]
   float dscale;         // decay activation scale (0: g is the log-decay)
+  int qknorm;           // 1: q, k are normalised inside the kernel
 };
 cudaError_t launch_decode(const DecArgs& a, int dtype, cudaStream_t st);
 

@@ -403,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::transform_block<8>(sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB,
                              sm + R_DSB + 16384, s_gam,
                              reinterpret_cast<float*>(sm + R_MP), 3, 16384, 7,
-                             kThreads, a.dscale);
+                             kThreads, a.dscale, kBlk);
       if (tid < 128) s_x[tid] = 0.f;
     } else {
       const int u = tid - 256;

@@ -121,8 +121,9 @@ constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false
 // in X, K^ straight into rows 0..63 of its operand slot in KHP.
 static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* kh,
                                             const uint8_t* rg, float* gam,
-                                            float* red, float dscale) {
-  tc::transform_keys<8>(x, kh, rg, gam, red, 3, 16384, 8, dscale);
+                                            float* red, float dscale,
+                                            int nvalid, float* nrm) {
+  tc::transform_keys<8>(x, kh, rg, gam, red, 3, 16384, 8, dscale, nvalid, nrm);
 }
 
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
@@ -163,12 +164,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int DVt = a.DV, v0 = kDV * vh;        // tensors' value width; first row here
   const int pair = dv2 ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   const int b = pair / a.H, h = pair - b * a.H;
-  const int T = a.T, H = a.H, R = a.R, NB = a.NB;
+  const int T = a.T, H = a.H, R = a.R;
   // blocks of C = min(L, 64) tokens; with C < 64 (chunks of 16, 32 or 48
   // tokens) the block is a chunk and rows C..63 of every token tile stay
   // zero, which contributes nothing to any product (see below)
   const int C = a.C;
   const int bpc = a.L / C;
+  // this sequence's tokens: B sequences of T tokens, or packed sequences
+  // [cu[b], cu[b + 1]) of a T-token tensor; a last block may be partial
+  int tok0 = b * T, Tn = T;
+  if (a.cu) {
+    tok0 = a.cu[b];
+    Tn = a.cu[b + 1] - tok0;
+    if (tok0 < 0 || Tn < 0 || tok0 > T - Tn) {  // malformed offsets: skip
+      if (tid == 0) {
+        atomicExch(&a.hdr->status, (uint32_t)CARVE_ERR_INVALID_ARG);
+        a.hdr->where = 90;
+      }
+      tok0 = 0;
+      Tn = 0;
+    }
+  }
+  const int NB = (Tn + C - 1) / C;
   const size_t SZ = (size_t)kDV * kDK;
   const __nv_bfloat16* w_in = static_cast<const __nv_bfloat16*>(a.w);
   const __nv_bfloat16* ud = static_cast<const __nv_bfloat16*>(a.u_down);
@@ -312,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
 
   auto issue_vgb = [&](int ib) {
-    const int tok = b * T + ib * C;
+    const int tok = tok0 + ib * C;
     mbar_expect_tx(bars + B_VGB, 3 * 2 * 128 * C);
     tma_load_3d(sm + OFF_RV, &tm_v, bars + B_VGB, v0, h, tok);
     tma_load_3d(sm + OFF_RV + 8192, &tm_v, bars + B_VGB, v0 + 64, h, tok);
@@ -324,7 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   };
   // k, q, g of block ib -> L2 ahead of their loads
   auto prefetch_kqg = [&](int ib) {
-    const int tok = b * T + ib * C;
+    const int tok = tok0 + ib * C;
 #pragma unroll 1
     for (int x = 0; x < kDK; x += 64) {
       tma_prefetch_3d(&tm_k, x, h, tok);
@@ -333,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   };
   auto issue_kq = [&](int ib) {
-    const int tok = b * T + ib * C;
+    const int tok = tok0 + ib * C;
     mbar_expect_tx(bars + B_KQ, 2 * 2 * 128 * C);
     tma_load_3d(sm + OFF_X, &tm_k, bars + B_KQ, 0, h, tok);
     tma_load_3d(sm + OFF_X + 16384, &tm_k, bars + B_KQ, 64, h, tok);
@@ -344,12 +361,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // key side of block nb's transform (warps 8-15): K~, Q~ in place in X,
   // K^ into its operand slot (rows 0..63 of KHP), gamma into its parity's
-  // buffer
+  // buffer; with the fused normalisation, q and k divided by their norms
+  // first (the exchange buffer is in rows of MY that hold nothing while
+  // the key transform runs: [M; P_k] was read by MMA 2, T takes rows 0..63)
   auto keys = [&](int nb) {
     wait(B_VGB, 1);
     wait(B_KQ, 2);
+    const int cb = min(C, Tn - nb * C);  // tokens in block nb
+    if (cb < C) {
+      // a sequence ending inside the block: rows cb..C-1 of the raw k, q,
+      // g, v tiles hold the next sequence's tokens (or the copies' zero
+      // fill past the tensor) -- zeroed, so they add nothing, as in the
+      // 64-row tiles of short chunks
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      const int nrow = C - cb, u = tid - 256;
+      for (int i = u; i < nrow * 8 * 8; i += 256) {
+        const int r = cb + i / 64, set = (i / 8) & 7, c16 = i & 7;
+        // sets: K, Q rows of both column blocks in X; g, v of both blocks
+        uint8_t* base = set < 4 ? sm + OFF_X + (set & 1) * 16384 + (set >> 1) * 8192
+                                : (set < 6 ? sm + OFF_RG : sm + OFF_RV) + (set & 1) * 8192;
+        *reinterpret_cast<uint4*>(base + (r >> 3) * 1024 + (r & 7) * 128 + c16 * 16) = z;
+      }
+      bar_named(5, 256);
+    }
     keys_w8(sm + OFF_X, sm + OFF_KHP, sm + OFF_RG, (nb & 1) ? s_gam1 : s_gam0,
-            s_red, a.dscale);
+            s_red, a.dscale, cb,
+            a.qknorm ? reinterpret_cast<float*>(sm + OFF_MY + 12288) : nullptr);
   };
 
   // ---- initial state: S0 -> TMEM (fp32) and the bf16 operand copy
@@ -369,15 +406,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int c8 = 0; c8 < 4; ++c8)
       st_chunk(sm + OFF_SB + sw128_chunk(row, gp >> 1, (gp & 1) * 4 + c8, 128),
                vals + c8 * 8);
+    if (NB == 0 && a.S_T) {  // an empty sequence keeps its initial state
+      float* st = a.S_T + ((size_t)pair * DVt + v0 + row) * kDK + c0;
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(st + e) = make_float4(vals[e], vals[e + 1], vals[e + 2], vals[e + 3]);
+    }
   }
   if (tid < 128) s_m[tid] = a.m0 ? a.m0[(size_t)pair * DVt + v0 + tid] : 0.f;
-  if (tid == 0) issue_vgb(0);
-  if (tid == 256) issue_kq(0);
+  if (tid == 0 && NB > 0) issue_vgb(0);
+  if (tid == 256 && NB > 0) issue_kq(0);
   if (tid == 32 && NB > 1) prefetch_kqg(1);
   tmem_st_wait();
   tc_fence_before();
   __syncthreads();
-  if (warp >= 8) {  // block 0's key side and chunk 0's gate
+  if (warp >= 8 && NB > 0) {  // block 0's key side and chunk 0's gate
     keys(0);
     gate(0);
   }
@@ -390,14 +433,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const unsigned short* w_bits = reinterpret_cast<const unsigned short*>(w_in);
   uint32_t w_lo = 0, w_hi = 0;
   if (warp >= 8) {
-    const int wr = (tid - 256) >> 3;
-    const size_t r0 = (size_t)b * T + wr;
-    w_lo = wr < C ? w_bits[r0 * H + h] : 0u;
-    w_hi = wr + 32 < C ? w_bits[(r0 + 32) * H + h] : 0u;
+    const int wr = (tid - 256) >> 3, cb = min(C, Tn);
+    const size_t r0 = (size_t)tok0 + wr;
+    w_lo = wr < cb ? w_bits[r0 * H + h] : 0u;
+    w_hi = wr + 32 < cb ? w_bits[(r0 + 32) * H + h] : 0u;
   }
   for (int ib = 0; ib < NB; ++ib) {
     const int t0 = ib * C;
-    const bool chunk_end = ((ib + 1) % bpc) == 0;
+    const bool chunk_end = ((ib + 1) % bpc) == 0 || ib == NB - 1;
     uint8_t* rec = a.tc_rec ? a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes
                             : nullptr;
 
@@ -461,10 +504,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         *reinterpret_cast<uint4*>(sm + OFF_W + off) = y;
       }
-      if (ib + 1 < NB) {  // the next block's w_t (0 past the block's C tokens)
-        const size_t r0 = (size_t)b * T + (ib + 1) * C + rr;
-        w_lo = rr < C ? w_bits[r0 * H + h] : 0u;
-        w_hi = rr + 32 < C ? w_bits[(r0 + 32) * H + h] : 0u;
+      if (ib + 1 < NB) {  // the next block's w_t (0 past the block's tokens)
+        const int cb = min(C, Tn - (ib + 1) * C);
+        const size_t r0 = (size_t)tok0 + (ib + 1) * C + rr;
+        w_lo = rr < cb ? w_bits[r0 * H + h] : 0u;
+        w_hi = rr + 32 < cb ? w_bits[(r0 + 32) * H + h] : 0u;
       }
     }
 
@@ -746,13 +790,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (2u, 2u + 1) the even lane of a lane pair stores token 2u and the
       // odd lane token 2u + 1, after one shuffle (half the store count)
       const bool odd = (lane & 1) != 0;
-      __nv_bfloat16* orow = o + ((size_t)b * T + t0 + gp * 16 + (odd ? 1 : 0)) * H * DVt +
+      __nv_bfloat16* orow = o + ((size_t)tok0 + t0 + gp * 16 + (odd ? 1 : 0)) * H * DVt +
                             (size_t)h * DVt + v0 + (row & ~1);
-      const bool live = gp * 16 < C;  // token group inside the block (C % 16 == 0)
+      const int nlive = min(C, Tn - t0) - gp * 16 - (odd ? 1 : 0);  // this lane's tokens in the block
 #pragma unroll
       for (int e = 0; e < 16; e += 2) {
         const float recv = __shfl_xor_sync(0xffffffffu, odd ? vals[e] : vals[e + 1], 1);
-        if (live)
+        if (e < nlive)
           *reinterpret_cast<__nv_bfloat162*>(orow + (size_t)e * H * DVt) =
               odd ? __floats2bfloat162_rn(recv, vals[e + 1])
                   : __floats2bfloat162_rn(vals[e], recv);
@@ -858,7 +902,7 @@ bool tc_fwd_supported(const carve_shape& s, bool training) {
 
 cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
   CUtensorMap mq, mk, mv, mg, mb;
-  const long long rows = (long long)a.B * a.T;
+  const long long rows = a.cu ? (long long)a.T : (long long)a.B * a.T;
   const bool dv2 = a.DV == 2 * kDV;
   if (dv2 && (a.ck_S || a.tc_rec)) return cudaErrorInvalidValue;  // inference only
   const int C = a.C;

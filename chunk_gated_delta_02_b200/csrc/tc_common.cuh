@@ -84,7 +84,8 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* p, float* x) {
 // Element-wise transform of one block of 64 tokens x 128 key channels (CARVE
 // summaries, gist.science, section 2.3: decay on the key axis; section 2.1:
 // the content gate b = sigmoid(b_x + U_b m_c)); with dscale > 0 the g tile
-// holds raw decay logits a and the log-decay is -dscale softplus(a):
+// holds raw decay logits a and the log-decay is -dscale softplus(a); token
+// rows at or past `nvalid` (the block's length) get log-decay 0:
 //   Gamma_t = exp(sum_{u <= t} g_u)   K~ = K Gamma    Q~_t = Q_t Gamma_{t-1}
 //   K^ = K / Gamma                    kap^ = b K^     gamma = Gamma_63
 // All tiles are 128-byte swizzled 64-column blocks.  `x` holds [K; Q]
@@ -109,7 +110,7 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
                                                 float* s_gam, float* red,
                                                 int bar_id, uint32_t khs,
                                                 int bar_b, int n_b,
-                                                float dscale) {
+                                                float dscale, int nvalid) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
@@ -132,8 +133,10 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
 #pragma unroll
-    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0)
-      gl[i][e] = (i ? gl[i - 1][e] : 0.f) + decay_act(gv[e], dscale);
+    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0);
+                                 // rows past the block's nvalid tokens: 0
+      gl[i][e] = (i ? gl[i - 1][e] : 0.f) +
+                 (TPT * tg + i < nvalid ? decay_act(gv[e], dscale) : 0.f);
   }
   float ex[8];  // exclusive prefix of the token group
   float wt[8];  // running inclusive sum over the warp's groups
@@ -205,7 +208,8 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
                                                const uint8_t* graw,
                                                float* s_gam, float* red,
                                                int bar_id, uint32_t khs,
-                                               int wbase, float dscale) {
+                                               int wbase, float dscale,
+                                               int nvalid, float* nrm) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
@@ -222,14 +226,59 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
   auto offk = [&](int t) {
     return (uint32_t)(blk * khs + t * 128 + ((ch ^ (t & 7)) << 4));
   };
+  // fused q / k normalisation (nrm != nullptr): per-token inverse norms
+  // over the 128 channels.  Each thread sums the squares of its 8 channels
+  // of its TPT tokens, the 8 lanes of a token reduce by shuffles, and the
+  // two column blocks' warps exchange their halves through nrm
+  // ([2 blocks][64 tokens][k, q] floats) across named barrier bar_id + 4
+  // of the NW warps.  Zero rows (padding) get 0, not inf.
+  float ink[TPT], inq[TPT];
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) ink[i] = inq[i] = 1.f;
+  if (nrm) {
+    float sk[TPT], sq[TPT];
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+      const int t = TPT * tg + i;
+      float kv[8], qv[8];
+      ld_chunk(x + off128(t), kv);
+      ld_chunk(x + off128(64 + t), qv);
+      sk[i] = sq[i] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sk[i] = fmaf(kv[e], kv[e], sk[i]);
+        sq[i] = fmaf(qv[e], qv[e], sq[i]);
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
+        sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], o);
+      }
+      if (ch == 0) {
+        nrm[(blk * 64 + t) * 2] = sk[i];
+        nrm[(blk * 64 + t) * 2 + 1] = sq[i];
+      }
+    }
+    bar_named(bar_id + 4, NW * 32);
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+      const int t = TPT * tg + i;
+      const float tk = nrm[t * 2] + nrm[(64 + t) * 2];
+      const float tq = nrm[t * 2 + 1] + nrm[(64 + t) * 2 + 1];
+      ink[i] = tk > 0.f ? 1.0f / sqrtf(tk) : 0.f;
+      inq[i] = tq > 0.f ? 1.0f / sqrtf(tq) : 0.f;
+    }
+  }
   float gl[TPT][8];  // inclusive log-decay sums inside the token group
 #pragma unroll
   for (int i = 0; i < TPT; ++i) {
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
 #pragma unroll
-    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0)
-      gl[i][e] = (i ? gl[i - 1][e] : 0.f) + decay_act(gv[e], dscale);
+    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0);
+                                 // rows past the block's nvalid tokens: 0
+      gl[i][e] = (i ? gl[i - 1][e] : 0.f) +
+                 (TPT * tg + i < nvalid ? decay_act(gv[e], dscale) : 0.f);
   }
   float ex[8];  // exclusive prefix of the token group
   float wt[8];  // running inclusive sum over the warp's groups
@@ -266,6 +315,11 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
     float kv[8], qv[8], o_kt[8], o_qt[8], o_kh[8];
     ld_chunk(x + off128(t), kv);
     ld_chunk(x + off128(64 + t), qv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      kv[e] *= ink[i];
+      qv[e] *= inq[i];
+    }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float gam = __expf(ex[e] + gl[i][e]);

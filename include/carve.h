@@ -56,8 +56,11 @@ typedef enum { CARVE_BF16 = 0, CARVE_FP32 = 1 } carve_dtype;
 /*
  * Problem shape.  B sequences of T tokens, H heads, key width DK, value
  * width DV, rank R of U_b, chunk length L.
- * Supported: B, H >= 1; T >= 0 with T % L == 0; DK, DV multiples of 16 in
- * [16, 256]; 0 <= R <= 64; L in [1, 64] or a multiple of 64 up to 256.
+ * Supported: B, H >= 1; T >= 0; DK, DV multiples of 16 in [16, 256];
+ * 0 <= R <= 64; L in [1, 64] or a multiple of 64 up to 256.  Training
+ * (carve_chunk_fwd with training != 0, carve_chunk_bwd) needs T % L == 0;
+ * the forward without training takes any T (the last chunk of a sequence
+ * may be short; its mean, returned in m_T, still divides by L).
  * Anything else returns CARVE_ERR_UNSUPPORTED.
  * Kernel families: bf16 with DK = 128, R <= 32, T > 0 runs on the tensor
  * cores for DV = 128 with L a multiple of 64 (forward, training forward and
@@ -75,6 +78,13 @@ typedef struct {
                        * section 2.3 "Key-Axis Decay und Fusion"); the
                        * backward then returns dL/da in dg.  Negative or
                        * non-finite: CARVE_ERR_INVALID_ARG. */
+  int32_t qk_l2norm;  /* 0: q and k are used as given (the workloads pass
+                       * unit rows); 1: the kernels divide every token's q
+                       * and k by their Euclidean norms over DK themselves
+                       * (a fused prologue) and the backward returns the
+                       * gradients of the raw q and k.  Other values:
+                       * CARVE_ERR_INVALID_ARG.  Training with 1 runs on
+                       * the generic kernels. */
 } carve_shape;
 
 /*
@@ -121,6 +131,42 @@ carve_status carve_chunk_fwd(const carve_shape* shape,
                              void* o, float* S_T, float* m_T,
                              void* workspace, size_t workspace_bytes,
                              int training, void* stream);
+
+/*
+ * Forward without training over packed sequences of different lengths
+ * (variable-length batches; survey item NEXT-4, the chunk-0 rule of the
+ * pages applying to each sequence from its own start).
+ *
+ *   shape        : B = number of sequences, T = total packed tokens (any
+ *                  T >= 0), the other fields as for carve_chunk_fwd
+ *   cu_seqlens   : [B + 1] int32 DEVICE array: sequence b is tokens
+ *                  cu_seqlens[b] .. cu_seqlens[b + 1] - 1, with
+ *                  0 <= cu_seqlens[b] <= cu_seqlens[b + 1] <= T (checked on
+ *                  the device: a violation sets CARVE_ERR_INVALID_ARG in the
+ *                  status word and that sequence is skipped)
+ *   q, k, g, b_x : [T, H, DK] dtype   packed tokens
+ *   v            : [T, H, DV] dtype
+ *   w            : [T, H]     dtype
+ *   u_down, u_up : as for carve_chunk_fwd
+ *   S0, m0       : [B, H, DV, DK], [B, H, DV] fp32 per sequence, or NULL
+ *   o            : [T, H, DV] dtype   (tokens of no sequence are left as is)
+ *   S_T, m_T     : [B, H, DV, DK], [B, H, DV] fp32 per sequence, or NULL
+ *   workspace    : carve_workspace_bytes(shape, 0) bytes
+ *
+ * Chunks of L tokens start at each sequence's first token; a sequence's last
+ * chunk may be short (its mean, m_T, divides by L).  An empty sequence
+ * returns S_T = S0 and m_T = m0.  Errors as for carve_chunk_fwd.
+ */
+carve_status carve_chunk_fwd_varlen(const carve_shape* shape,
+                                    const int32_t* cu_seqlens,
+                                    const void* q, const void* k,
+                                    const void* v, const void* g,
+                                    const void* b_x, const void* w,
+                                    const void* u_down, const void* u_up,
+                                    const float* S0, const float* m0,
+                                    void* o, float* S_T, float* m_T,
+                                    void* workspace, size_t workspace_bytes,
+                                    void* stream);
 
 /*
  * Backward pass: exact reverse mode of carve_chunk_fwd (the gradient also

@@ -150,10 +150,23 @@ def _activate(a, decay_scale):
     return raw
 
 
-def fwd_batch(inp, L, pairs=None, threads=None, decay_scale=0.0):
+def _normalise(a, qk_norm):
+    """qk_norm: the pair's q and k are raw; replace them by their per-token
+    L2 normalisations (oracle/normalize.py).  Returns the raw (q, k)."""
+    if not qk_norm:
+        return None
+    from .normalize import l2_normalise
+    raw = (a["q"], a["k"])
+    a["q"], a["k"] = l2_normalise(a["q"]), l2_normalise(a["k"])
+    return raw
+
+
+def fwd_batch(inp, L, pairs=None, threads=None, decay_scale=0.0,
+              qk_norm=False):
     """Oracle forward over (b, h) pairs.  Returns {(b, h): (o, S_T, m_T)}.
     decay_scale > 0: inp["g"] holds raw decay logits a, and the recurrence
-    runs on g = -decay_scale * softplus(a)."""
+    runs on g = -decay_scale * softplus(a).  qk_norm: q and k are raw and
+    the recurrence runs on their per-token L2 normalisations."""
     B, _, H, _ = tuple(inp["q"].shape)
     if pairs is None:
         pairs = [(b, h) for b in range(B) for h in range(H)]
@@ -161,6 +174,7 @@ def fwd_batch(inp, L, pairs=None, threads=None, decay_scale=0.0):
     def one(bh):
         a = pair_inputs(inp, *bh)
         _activate(a, decay_scale)
+        _normalise(a, qk_norm)
         return bh, fwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
                             a["u_down"], a["u_up"], L, a["S0"], a["m0"])
 
@@ -169,12 +183,13 @@ def fwd_batch(inp, L, pairs=None, threads=None, decay_scale=0.0):
 
 
 def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None,
-              decay_scale=0.0):
+              decay_scale=0.0, qk_norm=False):
     """Oracle reverse pass over (b, h) pairs.  d_o [B, T, H, DV],
     dS_T [B, H, DV, DK] or None, dm_T [B, H, DV] or None.
     Returns {(b, h): grads dict} (per-pair du_down / du_up, not summed).
     decay_scale > 0: inp["g"] holds raw decay logits a, and "dg" is the
-    gradient with respect to a (chain rule through the activation)."""
+    gradient with respect to a (chain rule through the activation).
+    qk_norm: q and k are raw; "dq", "dk" are with respect to the raw ones."""
     B, _, H, _ = tuple(inp["q"].shape)
     if pairs is None:
         pairs = [(b, h) for b in range(B) for h in range(H)]
@@ -183,6 +198,7 @@ def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None,
         b, h = bh
         a = pair_inputs(inp, b, h)
         raw = _activate(a, decay_scale)
+        raw_qk = _normalise(a, qk_norm)
         do = np.ascontiguousarray(_np64(d_o[b, :, h, :]))
         dst = None if dS_T is None else np.ascontiguousarray(_np64(dS_T[b, h]))
         dmt = None if dm_T is None else np.ascontiguousarray(_np64(dm_T[b, h]))
@@ -191,6 +207,10 @@ def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None,
         if raw is not None:
             from .activation import decay_grad
             gr["dg"] = gr["dg"] * decay_grad(raw, decay_scale)
+        if raw_qk is not None:
+            from .normalize import l2_normalise_grad
+            gr["dq"] = l2_normalise_grad(raw_qk[0], gr["dq"])
+            gr["dk"] = l2_normalise_grad(raw_qk[1], gr["dk"])
         return bh, gr
 
     with ThreadPoolExecutor(_threads(threads)) as ex:

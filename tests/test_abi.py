@@ -39,10 +39,10 @@ def test_header_declarations_are_exported(lib):
 
 def shape(**kw):
     d = dict(B=2, T=128, H=3, DK=64, DV=64, R=8, L=64, dtype=0,
-             decay_scale=0.0)
+             decay_scale=0.0, qk_l2norm=0)
     d.update(kw)
     return carve.Shape(*(d[n] for n in ("B", "T", "H", "DK", "DV", "R", "L",
-                                        "dtype", "decay_scale")))
+                                        "dtype", "decay_scale", "qk_l2norm")))
 
 
 def ws_bytes(lib, s, training):
@@ -56,10 +56,13 @@ def test_workspace_bytes(lib):
     # training adds the block-start states: (NB + 1) states per pair
     P, NB, DV, DK = 2 * 3, 128 // 64, 64, 64
     assert trn - inf >= P * (NB + 1) * DV * DK * 4
-    for bad in (dict(DK=24), dict(DV=272), dict(L=96), dict(T=100),
+    for bad in (dict(DK=24), dict(DV=272), dict(L=96),
                 dict(R=65), dict(B=0), dict(dtype=7), dict(L=0)):
         assert ws_bytes(lib, shape(**bad), 0) == 0, bad
     assert ws_bytes(lib, shape(T=0), 0) > 0
+    # a short last chunk: the forward takes it, training does not
+    assert ws_bytes(lib, shape(T=100), 0) > 0
+    assert ws_bytes(lib, shape(T=100), 1) == 0
 
 
 def test_decay_scale_validation(lib):
@@ -70,6 +73,18 @@ def test_decay_scale_validation(lib):
     for bad in (-0.1, float("nan"), float("inf")):
         assert ws_bytes(lib, shape(decay_scale=bad), 0) == 0, bad
         assert call_fwd(lib, shape(decay_scale=bad), FAKE, 1 << 20) == 1, bad
+    # the fused q / k normalisation is on or off
+    assert ws_bytes(lib, shape(qk_l2norm=1), 1) > 0
+    for bad in (2, -1):
+        assert call_fwd(lib, shape(qk_l2norm=bad), FAKE, 1 << 20) == 1, bad
+    # it runs the tensor-core forward, and trains on the generic kernels
+    path = lambda **kw: lib.carve_fwd_path(ctypes.byref(shape(**kw))).decode()
+    tc = dict(DK=128, DV=128, R=32, L=64, T=128, dtype=carve.CARVE_BF16)
+    assert path(**dict(tc, qk_l2norm=1)) == "tc"
+    n_tc = ws_bytes(lib, shape(**tc), 1)
+    n_norm = ws_bytes(lib, shape(**dict(tc, qk_l2norm=1)), 1)
+    assert n_norm - ws_bytes(lib, shape(**dict(tc, qk_l2norm=1)), 0) >= \
+        2 * 3 * (128 // 64 + 1) * 128 * 128 * 4 and n_norm != n_tc
 
 
 def test_status_strings_and_path(lib):
@@ -137,7 +152,7 @@ FAKE = ctypes.c_void_p(1 << 20)          # aligned, never dereferenced
 MIS = ctypes.c_void_p((1 << 20) + 4)     # misaligned
 
 
-def call_fwd(lib, s, ws=None, nbytes=0, **over):
+def call_fwd(lib, s, ws=None, nbytes=0, training=0, **over):
     args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, bx=FAKE, w=FAKE, ud=FAKE,
                 uu=FAKE, S0=None, m0=None, o=FAKE, S_T=None, m_T=None)
     args.update(over)
@@ -145,7 +160,7 @@ def call_fwd(lib, s, ws=None, nbytes=0, **over):
         ctypes.byref(s) if s is not None else None, args["q"], args["k"],
         args["v"], args["g"], args["bx"], args["w"], args["ud"], args["uu"],
         args["S0"], args["m0"], args["o"], args["S_T"], args["m_T"], ws,
-        ctypes.c_size_t(nbytes), 0, None)
+        ctypes.c_size_t(nbytes), training, None)
 
 
 def test_fwd_validation_returns_before_launch(lib):
@@ -153,13 +168,38 @@ def test_fwd_validation_returns_before_launch(lib):
     need = ws_bytes(lib, s, 0)
     assert call_fwd(lib, None) == 1                       # no shape
     assert call_fwd(lib, shape(DK=24), FAKE, need) == 2   # unsupported
-    assert call_fwd(lib, shape(T=100), FAKE, need) == 2   # T % L != 0
+    assert call_fwd(lib, shape(T=100), FAKE, 1 << 30,
+                    training=1) == 2                      # training, T % L != 0
     assert call_fwd(lib, s, FAKE, need, q=None) == 1      # null input
     assert call_fwd(lib, s, FAKE, need, v=MIS) == 1       # misaligned
     assert call_fwd(lib, s, FAKE, need, S_T=MIS) == 1     # misaligned output
     assert call_fwd(lib, s, None, need) == 3              # no workspace
     assert call_fwd(lib, s, FAKE, need - 1) == 3          # too small
     assert call_fwd(lib, s, MIS, need) == 3               # misaligned ws
+
+
+def test_varlen_validation_returns_before_launch(lib):
+    f = lib.carve_chunk_fwd_varlen
+    f.argtypes = ([ctypes.POINTER(carve.Shape)] + [ctypes.c_void_p] * 15
+                  + [ctypes.c_size_t, ctypes.c_void_p])
+    f.restype = ctypes.c_int
+    s = shape(T=100)  # any total length
+    need = ws_bytes(lib, s, 0)
+
+    def call(sh, cu=FAKE, ws=FAKE, nbytes=need, **over):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, bx=FAKE, w=FAKE, ud=FAKE,
+                 uu=FAKE, S0=None, m0=None, o=FAKE, S_T=None, m_T=None)
+        a.update(over)
+        return f(ctypes.byref(sh), cu, a["q"], a["k"], a["v"], a["g"],
+                 a["bx"], a["w"], a["ud"], a["uu"], a["S0"], a["m0"], a["o"],
+                 a["S_T"], a["m_T"], ws, nbytes, None)
+
+    assert call(s, cu=None) == 1                          # no offsets
+    assert call(s, cu=MIS) == 1                           # misaligned offsets
+    assert call(shape(DK=24)) == 2
+    assert call(s, q=None) == 1
+    assert call(s, ws=None) == 3
+    assert call(s, nbytes=need - 1) == 3
 
 
 def test_bwd_validation_returns_before_launch(lib):
@@ -204,7 +244,7 @@ def test_noalloc_validation_matches_the_workspace_entry_point(lib):
     s = shape()
     need = ws_bytes(lib, s, 0)
     for bad in (dict(dtype=7), dict(B=0), dict(L=0), dict(DK=24),
-                dict(T=100), dict(R=65), dict(L=96)):
+                dict(R=65), dict(L=96)):
         want = call_fwd(lib, shape(**bad), FAKE, need)
         assert want in (1, 2), bad
         assert call_noalloc(lib, shape(**bad)) == want, bad
