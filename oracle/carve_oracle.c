@@ -40,6 +40,15 @@
  * carve_oracle_bwd is the exact reverse mode of carve_oracle_fwd, written as
  * a sequential reverse walk over tokens (chunk-start states are kept and each
  * chunk is re-run forward to recover the per-token states).
+ *
+ * The *_erase entry points take the erase form as an argument: 0 is the
+ * form above; 1 is the other erase that acts on the key axis only,
+ *   S_t = S' (I - (b_t (.) k_t) k_t^T) + w_t v_t k_t^T,  i.e.  e = S' kappa,
+ *   S_t = S' - e k_t^T + w_t v_t k_t^T,
+ * where the gated key reads the state and the plain key is written (the
+ * abstract and section 3 "Chunkability Boundary" require only that the
+ * erase act on the key axis; both forms are chunkable).  For a gate b that
+ * is the same on every key channel the two forms coincide.
  */
 #include <math.h>
 #include <stdlib.h>
@@ -70,35 +79,36 @@ static void content_projection(int DK, int DV, int R, const double* u_down,
 static void token_step(int DK, int DV, double* S, const double* q,
                        const double* k, const double* vv, const double* g,
                        const double* b, double w, double* o, double* e,
-                       double* alpha) {
+                       double* alpha, int erase) {
   /* o_t = S_{t-1} q_t */
   for (int v = 0; v < DV; ++v) {
     double acc = 0.0;
     for (int j = 0; j < DK; ++j) acc += S[(size_t)v * DK + j] * q[j];
     o[v] = acc;
   }
-  /* S' = S_{t-1} Diag(exp g_t) ; e = S' k_t */
+  /* S' = S_{t-1} Diag(exp g_t) ; e = S' k_t  (erase 1: e = S' (b (.) k_t)) */
   for (int j = 0; j < DK; ++j) alpha[j] = exp(g[j]);
   for (int v = 0; v < DV; ++v) {
     double acc = 0.0;
     for (int j = 0; j < DK; ++j) {
       S[(size_t)v * DK + j] *= alpha[j];
-      acc += S[(size_t)v * DK + j] * k[j];
+      acc += S[(size_t)v * DK + j] * (erase ? b[j] * k[j] : k[j]);
     }
     e[v] = acc;
   }
-  /* S_t = S' - e (b (.) k)^T + w v k^T */
+  /* S_t = S' - e (b (.) k)^T + w v k^T   (erase 1: S' - e k^T + w v k^T) */
   for (int v = 0; v < DV; ++v)
     for (int j = 0; j < DK; ++j)
-      S[(size_t)v * DK + j] += -e[v] * (b[j] * k[j]) + w * vv[v] * k[j];
+      S[(size_t)v * DK + j] +=
+          -e[v] * (erase ? k[j] : b[j] * k[j]) + w * vv[v] * k[j];
 }
 
-int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
-                     const double* q, const double* k, const double* v,
-                     const double* g, const double* bx, const double* w,
-                     const double* u_down, const double* u_up,
-                     const double* S0, const double* m0,
-                     double* o, double* S_T, double* m_T) {
+int carve_oracle_fwd_erase(int T, int DK, int DV, int R, int L, int erase,
+                           const double* q, const double* k, const double* v,
+                           const double* g, const double* bx, const double* w,
+                           const double* u_down, const double* u_up,
+                           const double* S0, const double* m0,
+                           double* o, double* S_T, double* m_T) {
   if (T < 0 || DK <= 0 || DV <= 0 || R < 0 || L <= 0) return 1;
   double* S = (double*)calloc((size_t)DV * DK, sizeof(double));
   double* m = (double*)calloc((size_t)DV, sizeof(double));
@@ -121,7 +131,7 @@ int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
       for (int j = 0; j < DK; ++j) b[j] = sigmoid(bx[(size_t)t * DK + j] + p[j]);
       token_step(DK, DV, S, q + (size_t)t * DK, k + (size_t)t * DK,
                  v + (size_t)t * DV, g + (size_t)t * DK, b, w[t],
-                 o + (size_t)t * DV, e, alpha);
+                 o + (size_t)t * DV, e, alpha, erase);
       for (int vv = 0; vv < DV; ++vv) msum[vv] += o[(size_t)t * DV + vv];
     }
     /* m_{c+1} = (1/L) sum over chunk c of o_t */
@@ -134,6 +144,16 @@ int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
   return 0;
 }
 
+int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
+                     const double* q, const double* k, const double* v,
+                     const double* g, const double* bx, const double* w,
+                     const double* u_down, const double* u_up,
+                     const double* S0, const double* m0,
+                     double* o, double* S_T, double* m_T) {
+  return carve_oracle_fwd_erase(T, DK, DV, R, L, 0, q, k, v, g, bx, w, u_down,
+                                u_up, S0, m0, o, S_T, m_T);
+}
+
 /*
  * Reverse mode of carve_oracle_fwd.
  *   d_o  : [T][DV]  upstream gradient of o
@@ -142,15 +162,16 @@ int carve_oracle_fwd(int T, int DK, int DV, int R, int L,
  * Outputs (all overwritten): dq, dk, dg, dbx [T][DK]; dv [T][DV]; dw [T];
  * du_down [R][DV]; du_up [DK][R]; dS0 [DV][DK]; dm0 [DV].
  */
-int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
-                     const double* q, const double* k, const double* v,
-                     const double* g, const double* bx, const double* w,
-                     const double* u_down, const double* u_up,
-                     const double* S0, const double* m0,
-                     const double* d_o, const double* dS_T, const double* dm_T,
-                     double* dq, double* dk, double* dv, double* dg,
-                     double* dbx, double* dw, double* du_down, double* du_up,
-                     double* dS0, double* dm0) {
+int carve_oracle_bwd_erase(int T, int DK, int DV, int R, int L, int erase,
+                           const double* q, const double* k, const double* v,
+                           const double* g, const double* bx, const double* w,
+                           const double* u_down, const double* u_up,
+                           const double* S0, const double* m0,
+                           const double* d_o, const double* dS_T,
+                           const double* dm_T, double* dq, double* dk,
+                           double* dv, double* dg, double* dbx, double* dw,
+                           double* du_down, double* du_up, double* dS0,
+                           double* dm0) {
   if (T < 0 || DK <= 0 || DV <= 0 || R < 0 || L <= 0) return 1;
   const size_t SZ = (size_t)DV * DK;
   const int NC = (T + L - 1) / L;
@@ -194,7 +215,7 @@ int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
       for (int j = 0; j < DK; ++j) b[j] = sigmoid(bx[(size_t)t * DK + j] + p[j]);
       token_step(DK, DV, S, q + (size_t)t * DK, k + (size_t)t * DK,
                  v + (size_t)t * DV, g + (size_t)t * DK, b, w[t], otmp, e,
-                 alpha);
+                 alpha, erase);
       for (int vv = 0; vv < DV; ++vv) msum[vv] += otmp[vv];
     }
     for (int vv = 0; vv < DV; ++vv) m[vv] = msum[vv] / (double)L;
@@ -216,7 +237,7 @@ int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
       for (int j = 0; j < DK; ++j) b[j] = sigmoid(bx[(size_t)t * DK + j] + p[j]);
       token_step(DK, DV, S, q + (size_t)t * DK, k + (size_t)t * DK,
                  v + (size_t)t * DV, g + (size_t)t * DK, b, w[t], otmp, e,
-                 alpha);
+                 alpha, erase);
     }
     memset(dp, 0, sizeof(double) * (size_t)DK);
     for (int t = t1 - 1; t >= t0; --t) {
@@ -235,12 +256,12 @@ int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
         kap[j] = b[j] * kt[j];
         alpha[j] = exp(gt[j]);
       }
-      /* recompute S' and e */
+      /* recompute S' and e (e = S' k, or S' kappa for erase 1) */
       for (int vv = 0; vv < DV; ++vv) {
         double acc = 0.0;
         for (int j = 0; j < DK; ++j) {
           Sp[(size_t)vv * DK + j] = St[(size_t)vv * DK + j] * alpha[j];
-          acc += Sp[(size_t)vv * DK + j] * kt[j];
+          acc += Sp[(size_t)vv * DK + j] * (erase ? kap[j] : kt[j]);
         }
         e[vv] = acc;
       }
@@ -258,24 +279,33 @@ int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
         for (int vv = 0; vv < DV; ++vv) acc += dS[(size_t)vv * DK + j] * vt[vv];
         dk[(size_t)t * DK + j] = wt * acc;
       }
-      /* erase term  -e kappa^T */
+      /* erase term  -e x^T with x = kappa (erase 0) or k (erase 1) */
       for (int vv = 0; vv < DV; ++vv) {
         double acc = 0.0;
-        for (int j = 0; j < DK; ++j) acc += dS[(size_t)vv * DK + j] * kap[j];
+        for (int j = 0; j < DK; ++j)
+          acc += dS[(size_t)vv * DK + j] * (erase ? kt[j] : kap[j]);
         de[vv] = -acc;
       }
       for (int j = 0; j < DK; ++j) {
         double acc = 0.0;
         for (int vv = 0; vv < DV; ++vv) acc += dS[(size_t)vv * DK + j] * e[vv];
-        dkap[j] = -acc;
+        if (erase)
+          dk[(size_t)t * DK + j] -= acc;  /* d/dx of -e x^T, x = k */
+        else
+          dkap[j] = -acc;                 /* x = kappa */
       }
-      /* e = S' k  ->  dS' = dS + de k^T ;  dk += S'^T de  (dS now holds dS') */
+      /* e = S' y, y = k (erase 0) or kappa (erase 1):  dS' = dS + de y^T,
+         dy = S'^T de  (dS now holds dS') */
       for (int vv = 0; vv < DV; ++vv)
-        for (int j = 0; j < DK; ++j) dS[(size_t)vv * DK + j] += de[vv] * kt[j];
+        for (int j = 0; j < DK; ++j)
+          dS[(size_t)vv * DK + j] += de[vv] * (erase ? kap[j] : kt[j]);
       for (int j = 0; j < DK; ++j) {
         double acc = 0.0;
         for (int vv = 0; vv < DV; ++vv) acc += Sp[(size_t)vv * DK + j] * de[vv];
-        dk[(size_t)t * DK + j] += acc;
+        if (erase)
+          dkap[j] = acc;
+        else
+          dk[(size_t)t * DK + j] += acc;
       }
       /* kappa = b (.) k ; b = sigmoid(bx + p) */
       for (int j = 0; j < DK; ++j) {
@@ -328,4 +358,18 @@ int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
   free(msum); free(dm_next); free(h); free(dh); free(p); free(dp); free(b);
   free(kap); free(dkap); free(alpha); free(e); free(de); free(otmp); free(dot);
   return 0;
+}
+
+int carve_oracle_bwd(int T, int DK, int DV, int R, int L,
+                     const double* q, const double* k, const double* v,
+                     const double* g, const double* bx, const double* w,
+                     const double* u_down, const double* u_up,
+                     const double* S0, const double* m0,
+                     const double* d_o, const double* dS_T, const double* dm_T,
+                     double* dq, double* dk, double* dv, double* dg,
+                     double* dbx, double* dw, double* du_down, double* du_up,
+                     double* dS0, double* dm0) {
+  return carve_oracle_bwd_erase(T, DK, DV, R, L, 0, q, k, v, g, bx, w, u_down,
+                                u_up, S0, m0, d_o, dS_T, dm_T, dq, dk, dv, dg,
+                                dbx, dw, du_down, du_up, dS0, dm0);
 }

@@ -23,6 +23,17 @@ derived by unrolling the recurrence over the tokens t = 1..n of a block:
 The gate b is fixed across a chunk of L tokens (it depends on m_c only), so a
 chunk may be solved as several consecutive blocks of ``block`` tokens; the
 chunk mean m_{c+1} still averages the L outputs of the whole chunk.
+
+For the other key-axis erase (erase = 1: S_t = S'(I - (b (.) k) k^T) +
+w v k^T, the gated key reads the state, the plain key is written) unrolling
+gives e_t = S'_t kap_t - w_t v_t and S_t = S'_t - e_t k_t^T, hence one
+triangular solve per chunk with the roles of the keys exchanged:
+
+  kap~ = b (.) K (.) Gamma
+  A    = strict_lower(kap~ K^T)
+  E    = (I + A)^{-1} (kap~ S^T - W)
+  O    = Q~ S^T - P_k E
+  S   <- (S - E^T K^) Diag(gamma)
 """
 import numpy as np
 
@@ -32,7 +43,7 @@ def _sigmoid(x):
 
 
 def chunked_fwd_pair(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
-                     block=None):
+                     block=None, erase=0):
     """Same contract as ``ref.fwd_pair``; returns (o, S_T, m_T)."""
     q, k, v, g, bx, w = (np.asarray(a, dtype=np.float64)
                          for a in (q, k, v, g, bx, w))
@@ -55,12 +66,20 @@ def chunked_fwd_pair(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
             K, Q = k[s0:s1], q[s0:s1]
             b = _sigmoid(bx[s0:s1] + p[None, :])
             Kt, Kh, Qt = K * Gam, K / Gam, Q * Gam_ex
+            W = w[s0:s1, None] * v[s0:s1]
+            if erase:
+                kap_t = b * K * Gam
+                A = np.tril(kap_t @ Kh.T, -1)
+                Pk = np.tril(Qt @ Kh.T, -1)
+                E = np.linalg.solve(np.eye(n) + A, kap_t @ S.T - W)
+                o[s0:s1] = Qt @ S.T - Pk @ E
+                S = (S - E.T @ Kh) * gam[None, :]
+                continue
             kap_h = b * K / Gam
             A = np.tril(Kt @ kap_h.T, -1)
             M = np.tril(Kt @ Kh.T, -1)
             Pk = np.tril(Qt @ Kh.T, -1)
             Pkap = np.tril(Qt @ kap_h.T, -1)
-            W = w[s0:s1, None] * v[s0:s1]
             E = np.linalg.solve(np.eye(n) + A, Kt @ S.T + M @ W)
             o[s0:s1] = Qt @ S.T + Pk @ W - Pkap @ E
             K_end, kap_end = Kh * gam[None, :], kap_h * gam[None, :]

@@ -35,6 +35,10 @@ def _load():
         lib.carve_oracle_fwd.restype = i
         lib.carve_oracle_bwd.argtypes = [i, i, i, i, i] + [d] * 23
         lib.carve_oracle_bwd.restype = i
+        lib.carve_oracle_fwd_erase.argtypes = [i, i, i, i, i, i] + [d] * 13
+        lib.carve_oracle_fwd_erase.restype = i
+        lib.carve_oracle_bwd_erase.argtypes = [i, i, i, i, i, i] + [d] * 23
+        lib.carve_oracle_bwd_erase.restype = i
         _lib = lib
     return _lib
 
@@ -50,8 +54,9 @@ def _c64(a):
     return None if a is None else np.ascontiguousarray(a, dtype=np.float64)
 
 
-def fwd_pair(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None):
-    """Returns (o [T, DV], S_T [DV, DK], m_T [DV]) in fp64."""
+def fwd_pair(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None, erase=0):
+    """Returns (o [T, DV], S_T [DV, DK], m_T [DV]) in fp64.  erase = 1: the
+    other key-axis erase form (see carve_oracle.c)."""
     q, k, v, g, bx, w, u_down, u_up, S0, m0 = map(
         _c64, (q, k, v, g, bx, w, u_down, u_up, S0, m0))
     T, DK = q.shape
@@ -60,8 +65,9 @@ def fwd_pair(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None):
     o = np.zeros((T, DV))
     S_T = np.zeros((DV, DK))
     m_T = np.zeros(DV)
-    rc = _load().carve_oracle_fwd(
-        T, DK, DV, R, int(L), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(bx),
+    rc = _load().carve_oracle_fwd_erase(
+        T, DK, DV, R, int(L), int(erase), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+        _ptr(bx),
         _ptr(w), _ptr(u_down), _ptr(u_up), _ptr(S0), _ptr(m0), _ptr(o),
         _ptr(S_T), _ptr(m_T))
     if rc != 0:
@@ -70,7 +76,7 @@ def fwd_pair(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None):
 
 
 def bwd_pair(q, k, v, g, bx, w, u_down, u_up, L, d_o, S0=None, m0=None,
-             dS_T=None, dm_T=None):
+             dS_T=None, dm_T=None, erase=0):
     """Reverse mode.  Returns a dict of fp64 gradients for one pair:
     dq, dk, dg, dbx [T, DK]; dv [T, DV]; dw [T]; du_down [R, DV];
     du_up [DK, R]; dS0 [DV, DK]; dm0 [DV]."""
@@ -84,8 +90,9 @@ def bwd_pair(q, k, v, g, bx, w, u_down, u_up, L, d_o, S0=None, m0=None,
                dbx=np.zeros((T, DK)), dw=np.zeros(T),
                du_down=np.zeros((R, DV)), du_up=np.zeros((DK, R)),
                dS0=np.zeros((DV, DK)), dm0=np.zeros(DV))
-    rc = _load().carve_oracle_bwd(
-        T, DK, DV, R, int(L), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(bx),
+    rc = _load().carve_oracle_bwd_erase(
+        T, DK, DV, R, int(L), int(erase), _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+        _ptr(bx),
         _ptr(w), _ptr(u_down), _ptr(u_up), _ptr(S0), _ptr(m0), _ptr(d_o),
         _ptr(dS_T), _ptr(dm_T), _ptr(out["dq"]), _ptr(out["dk"]),
         _ptr(out["dv"]), _ptr(out["dg"]), _ptr(out["dbx"]), _ptr(out["dw"]),
@@ -162,7 +169,7 @@ def _normalise(a, qk_norm):
 
 
 def fwd_batch(inp, L, pairs=None, threads=None, decay_scale=0.0,
-              qk_norm=False):
+              qk_norm=False, erase=0):
     """Oracle forward over (b, h) pairs.  Returns {(b, h): (o, S_T, m_T)}.
     decay_scale > 0: inp["g"] holds raw decay logits a, and the recurrence
     runs on g = -decay_scale * softplus(a).  qk_norm: q and k are raw and
@@ -176,14 +183,15 @@ def fwd_batch(inp, L, pairs=None, threads=None, decay_scale=0.0,
         _activate(a, decay_scale)
         _normalise(a, qk_norm)
         return bh, fwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
-                            a["u_down"], a["u_up"], L, a["S0"], a["m0"])
+                            a["u_down"], a["u_up"], L, a["S0"], a["m0"],
+                            erase)
 
     with ThreadPoolExecutor(_threads(threads)) as ex:
         return dict(ex.map(one, pairs))
 
 
 def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None,
-              decay_scale=0.0, qk_norm=False):
+              decay_scale=0.0, qk_norm=False, erase=0):
     """Oracle reverse pass over (b, h) pairs.  d_o [B, T, H, DV],
     dS_T [B, H, DV, DK] or None, dm_T [B, H, DV] or None.
     Returns {(b, h): grads dict} (per-pair du_down / du_up, not summed).
@@ -203,7 +211,8 @@ def bwd_batch(inp, L, d_o, dS_T=None, dm_T=None, pairs=None, threads=None,
         dst = None if dS_T is None else np.ascontiguousarray(_np64(dS_T[b, h]))
         dmt = None if dm_T is None else np.ascontiguousarray(_np64(dm_T[b, h]))
         gr = bwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
-                      a["u_down"], a["u_up"], L, do, a["S0"], a["m0"], dst, dmt)
+                      a["u_down"], a["u_up"], L, do, a["S0"], a["m0"], dst, dmt,
+                      erase)
         if raw is not None:
             from .activation import decay_grad
             gr["dg"] = gr["dg"] * decay_grad(raw, decay_scale)

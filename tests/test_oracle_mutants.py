@@ -16,9 +16,11 @@ SRC = os.path.join(ROOT, "oracle", "carve_oracle.c")
 
 MUTANTS = {
     # erase ignores the gate b (value-blind erase of the plain delta rule)
-    "erase_without_gate": ("-e[v] * (b[j] * k[j])", "-e[v] * k[j]"),
+    "erase_without_gate": ("-e[v] * (erase ? k[j] : b[j] * k[j])",
+                           "-e[v] * (erase ? k[j] : k[j])"),
     # erase with the wrong sign
-    "erase_sign": ("+= -e[v] * (b[j] * k[j])", "+= e[v] * (b[j] * k[j])"),
+    "erase_sign": ("-e[v] * (erase ? k[j] : b[j] * k[j]) + w",
+                   "e[v] * (erase ? k[j] : b[j] * k[j]) + w"),
     # decay applied on the value axis instead of the key axis
     "decay_on_value_axis": ("S[(size_t)v * DK + j] *= alpha[j];",
                             "S[(size_t)v * DK + j] *= alpha[v % DK];"),
@@ -34,6 +36,12 @@ MUTANTS = {
     "bwd_sigmoid_derivative": ("db * b[j] * (1.0 - b[j])", "db * b[j]"),
     # chunk-mean share of the upstream gradient not divided by L
     "bwd_mean_share": ("dm_next[vv] / (double)L;", "dm_next[vv];"),
+    # other erase form: the state read with the ungated key
+    "erase1_ungated_read": ("(erase ? b[j] * k[j] : k[j])",
+                            "(erase ? k[j] : k[j])"),
+    # other erase form: reverse pass with the wrong sign on the written key
+    "erase1_bwd_sign": ("dk[(size_t)t * DK + j] -= acc;",
+                        "dk[(size_t)t * DK + j] += acc;"),
     # reverse pass forgets the decay on the carried state gradient
     "bwd_decay": ("dS[(size_t)vv * DK + j] * alpha[j] + dot[vv] * qt[j]",
                   "dS[(size_t)vv * DK + j] + dot[vv] * qt[j]"),

@@ -41,9 +41,9 @@ def rand_pair(rng, T, DK, DV, R, ub_std=0.5, s0=True, m0=True, gscale=0.3):
         m0=rng.standard_normal(DV) * 0.5 if m0 else None)
 
 
-def run(a, L):
+def run(a, L, erase=0):
     return ref.fwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
-                        a["u_down"], a["u_up"], L, a["S0"], a["m0"])
+                        a["u_down"], a["u_up"], L, a["S0"], a["m0"], erase)
 
 
 # ---------------------------------------------------------------- golden ----
@@ -103,6 +103,30 @@ def test_chunked_solve_equals_token_recurrence(L):
     assert rel(oc, o) < 1e-12
     assert rel(Sc, S) < 1e-12
     assert rel(mc, m) < 1e-12
+
+
+@pytest.mark.parametrize("L", [1, 2, 3, 16])
+def test_other_erase_form_chunked_solve_equals_token_recurrence(L):
+    # the other key-axis erase, S' (I - (b (.) k) k^T): its single-key WY
+    # chunk form against the token loop
+    rng = np.random.default_rng(200 + L)
+    a = rand_pair(rng, T=37, DK=5, DV=4, R=2)
+    o, S, m = run(a, L, erase=1)
+    oc, Sc, mc = chunked_fwd_pair(**a, L=L, erase=1)
+    assert rel(oc, o) < 1e-12 and rel(Sc, S) < 1e-12 and rel(mc, m) < 1e-12
+
+
+def test_erase_forms_coincide_for_a_channel_constant_gate():
+    # k (b k)^T = (b k) k^T when b is the same on every key channel (U_b = 0
+    # and a channel-constant erase logit); with per-channel b they differ
+    rng = np.random.default_rng(9)
+    a = rand_pair(rng, T=30, DK=6, DV=4, R=2)
+    diff = max(rel(x, y) for x, y in zip(run(a, 4, 1), run(a, 4, 0)))
+    assert diff > 1e-3
+    a["bx"] = np.repeat(rng.standard_normal((30, 1)), 6, axis=1)
+    a["u_down"] = np.zeros_like(a["u_down"])
+    a["u_up"] = np.zeros_like(a["u_up"])
+    assert max(rel(x, y) for x, y in zip(run(a, 4, 1), run(a, 4, 0))) < 1e-13
 
 
 @pytest.mark.parametrize("block", [1, 2, 4, 8])
@@ -272,12 +296,13 @@ def test_per_channel_gate_state_stays_bounded():
 
 # ---------------------------------------------------------- backward --------
 
-def _loss_parts(a, L, Ro, RS, Rm):
-    o, S, m = run(a, L)
+def _loss_parts(a, L, Ro, RS, Rm, erase=0):
+    o, S, m = run(a, L, erase)
     return float((o * Ro).sum() + (S * RS).sum() + (m * Rm).sum())
 
 
-def test_backward_matches_central_finite_differences():
+@pytest.mark.parametrize("erase", [0, 1])
+def test_backward_matches_central_finite_differences(erase):
     rng = np.random.default_rng(13)
     T, DK, DV, R, L = 12, 4, 4, 2, 4
     a = rand_pair(rng, T, DK, DV, R, ub_std=0.8)
@@ -285,7 +310,8 @@ def test_backward_matches_central_finite_differences():
     RS = rng.standard_normal((DV, DK))
     Rm = rng.standard_normal(DV)
     gr = ref.bwd_pair(a["q"], a["k"], a["v"], a["g"], a["bx"], a["w"],
-                      a["u_down"], a["u_up"], L, Ro, a["S0"], a["m0"], RS, Rm)
+                      a["u_down"], a["u_up"], L, Ro, a["S0"], a["m0"], RS, Rm,
+                      erase)
     names = dict(q="dq", k="dk", v="dv", g="dg", bx="dbx", w="dw",
                  u_down="du_down", u_up="du_up", S0="dS0", m0="dm0")
     for name, gname in names.items():
@@ -299,8 +325,8 @@ def test_backward_matches_central_finite_differences():
             xp, xm = x.copy(), x.copy()
             xp[idx] += h
             xm[idx] -= h
-            fp = _loss_parts(dict(a, **{name: xp}), L, Ro, RS, Rm)
-            fm = _loss_parts(dict(a, **{name: xm}), L, Ro, RS, Rm)
+            fp = _loss_parts(dict(a, **{name: xp}), L, Ro, RS, Rm, erase)
+            fm = _loss_parts(dict(a, **{name: xm}), L, Ro, RS, Rm, erase)
             fd[idx] = (fp - fm) / (2 * h)
         err = rel(gr[gname], fd)
         assert err < 1e-6, (name, err)
