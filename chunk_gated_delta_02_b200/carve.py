@@ -29,7 +29,8 @@ EXPORTS = ("carve_workspace_bytes", "carve_chunk_fwd", "carve_chunk_bwd",
 class Shape(ctypes.Structure):
     _fields_ = ([(n, ctypes.c_int32)
                  for n in ("B", "T", "H", "DK", "DV", "R", "L", "dtype")]
-                + [("decay_scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int32)])
+                + [("decay_scale", ctypes.c_float), ("qk_l2norm", ctypes.c_int32),
+                   ("erase_form", ctypes.c_int32)])
 
 
 class CarveError(RuntimeError):
@@ -84,13 +85,14 @@ def _stream(device):
 
 
 def make_shape(B, T, H, DK, DV, R, L, dtype, decay_scale=0.0,
-               qk_l2norm=False):
+               qk_l2norm=False, erase_form=0):
     """decay_scale > 0: `g` holds raw decay logits a and the kernels use
     g = -decay_scale * softplus(a); the backward then returns dL/da.
-    qk_l2norm: q and k are raw and the kernels normalise them per token."""
+    qk_l2norm: q and k are raw and the kernels normalise them per token.
+    erase_form 1: the other key-axis erase S' (I - (b k) k^T)."""
     return Shape(B, T, H, DK, DV, R, L, _DTYPES[dtype] if isinstance(
         dtype, torch.dtype) else int(dtype), float(decay_scale),
-        int(bool(qk_l2norm)))
+        int(bool(qk_l2norm)), int(erase_form))
 
 
 def workspace_bytes(shape, training):
@@ -130,7 +132,7 @@ def _dims(q, v, u_down):
 
 def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
               training=False, workspace=None, o=None, want_state=True,
-              decay_scale=0.0, qk_l2norm=False):
+              decay_scale=0.0, qk_l2norm=False, erase_form=0):
     """Forward pass.  Returns (o, S_T, m_T, workspace).
 
     q, k, g, bx [B, T, H, DK]; v [B, T, H, DV]; w [B, T, H]; u_down
@@ -152,7 +154,8 @@ def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
         _check(S0, "S0", torch.float32, (B, H, DV, DK), dev)
     if m0 is not None:
         _check(m0, "m0", torch.float32, (B, H, DV), dev)
-    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
+    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm,
+                       erase_form)
     nbytes = workspace_bytes(shape, training)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
@@ -175,7 +178,7 @@ def chunk_fwd(q, k, v, g, bx, w, u_down, u_up, L, S0=None, m0=None,
 
 def chunk_fwd_varlen(q, k, v, g, bx, w, u_down, u_up, L, cu_seqlens, S0=None,
                      m0=None, workspace=None, o=None, want_state=True,
-                     decay_scale=0.0, qk_l2norm=False):
+                     decay_scale=0.0, qk_l2norm=False, erase_form=0):
     """Forward (no training) over packed sequences of different lengths.
     Returns (o, S_T, m_T, workspace).
 
@@ -203,7 +206,8 @@ def chunk_fwd_varlen(q, k, v, g, bx, w, u_down, u_up, L, cu_seqlens, S0=None,
         _check(S0, "S0", torch.float32, (N, H, DV, DK), dev)
     if m0 is not None:
         _check(m0, "m0", torch.float32, (N, H, DV), dev)
-    shape = make_shape(N, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
+    shape = make_shape(N, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm,
+                       erase_form)
     nbytes = workspace_bytes(shape, False)
     if workspace is None or workspace.numel() < nbytes:
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
@@ -226,7 +230,7 @@ def chunk_fwd_varlen(q, k, v, g, bx, w, u_down, u_up, L, cu_seqlens, S0=None,
 
 def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
               dm_T=None, want_dS0=True, out=None, decay_scale=0.0,
-              qk_l2norm=False):
+              qk_l2norm=False, erase_form=0):
     """Backward pass after a training-mode chunk_fwd with the same inputs
     (and the same decay_scale; with decay_scale > 0, "dg" is dL/da of the
     raw decay logits).  Returns a dict: dq dk dg dbx [B, T, H, DK], dv
@@ -240,7 +244,8 @@ def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
         _check(dS_T, "dS_T", torch.float32, (B, H, DV, DK), dev)
     if dm_T is not None:
         _check(dm_T, "dm_T", torch.float32, (B, H, DV), dev)
-    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
+    shape = make_shape(B, T, H, DK, DV, R, L, dt, decay_scale, qk_l2norm,
+                       erase_form)
     if out is None:
         e = lambda s, d=dt: torch.empty(s, dtype=d, device=dev)
         out = dict(dq=e((B, T, H, DK)), dk=e((B, T, H, DK)),
@@ -264,7 +269,7 @@ def chunk_bwd(q, k, v, g, bx, w, u_down, u_up, L, d_o, workspace, dS_T=None,
 
 
 def decode_step(q, k, v, g, bx, w, u_down, u_up, L, pos, S, m, osum, o=None,
-                decay_scale=0.0, qk_l2norm=False):
+                decay_scale=0.0, qk_l2norm=False, erase_form=0):
     """One recurrent decode step (one new token per (sequence, head)).
 
     q, k, g, bx [B, H, DK]; v [B, H, DV]; w [B, H] (bf16 or fp32); u_down
@@ -289,7 +294,8 @@ def decode_step(q, k, v, g, bx, w, u_down, u_up, L, pos, S, m, osum, o=None,
     _check(osum, "osum", torch.float32, (B, H, DV), dev)
     if o is None:
         o = torch.empty((B, H, DV), dtype=dt, device=dev)
-    shape = make_shape(B, 1, H, DK, DV, R, L, dt, decay_scale, qk_l2norm)
+    shape = make_shape(B, 1, H, DK, DV, R, L, dt, decay_scale, qk_l2norm,
+                       erase_form)
     rc = lib().carve_decode_step(
         ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(bx),
         _ptr(w), _ptr(u_down), _ptr(u_up), _ptr(pos), _ptr(S), _ptr(m),

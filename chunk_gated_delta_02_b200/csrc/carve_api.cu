@@ -21,6 +21,7 @@ carve_status check_shape(const carve_shape* s) {
   if (!(s->decay_scale >= 0.f) || s->decay_scale > 3.0e38f)  // NaN, < 0, inf
     return CARVE_ERR_INVALID_ARG;
   if (s->qk_l2norm != 0 && s->qk_l2norm != 1) return CARVE_ERR_INVALID_ARG;
+  if (s->erase_form != 0 && s->erase_form != 1) return CARVE_ERR_INVALID_ARG;
   if (s->DK % 16 || s->DV % 16 || s->DK > 256 || s->DV > 256)
     return CARVE_ERR_UNSUPPORTED;
   if (s->R > kMaxR) return CARVE_ERR_UNSUPPORTED;
@@ -147,6 +148,7 @@ carve_status carve_chunk_fwd(const carve_shape* shape, const void* q,
   a.hdr = (WsHeader*)ws;
   a.dscale = s.decay_scale;
   a.qknorm = s.qk_l2norm;
+  a.erase = s.erase_form;
   test_knobs(&a.spin, &a.stall_block);
   cudaError_t e = tc ? launch_fwd_tc(a, (cudaStream_t)stream)
                       : launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
@@ -188,6 +190,7 @@ carve_status carve_chunk_fwd_varlen(
   a.hdr = (WsHeader*)ws;
   a.dscale = s.decay_scale;
   a.qknorm = s.qk_l2norm;
+  a.erase = s.erase_form;
   a.cu = cu_seqlens;
   test_knobs(&a.spin, &a.stall_block);
   cudaError_t e = tc ? launch_fwd_tc(a, (cudaStream_t)stream)
@@ -247,6 +250,7 @@ carve_status carve_chunk_bwd(const carve_shape* shape, const void* q,
   a.hdr = (WsHeader*)ws;
   a.dscale = s.decay_scale;
   a.qknorm = s.qk_l2norm;
+  a.erase = s.erase_form;
   test_knobs(&a.spin, &a.stall_block);
   cudaError_t e = tc ? launch_bwd_tc(a, (cudaStream_t)stream)
                       : launch_bwd_generic(a, s.dtype, (cudaStream_t)stream);
@@ -277,6 +281,7 @@ carve_status carve_decode_step(const carve_shape* shape, const void* q,
   a.S = S; a.m = m; a.osum = osum; a.o = o;
   a.dscale = s.decay_scale;
   a.qknorm = s.qk_l2norm;
+  a.erase = s.erase_form;
   return launch_decode(a, s.dtype, (cudaStream_t)stream) == cudaSuccess
              ? CARVE_OK
              : CARVE_ERR_CUDA;

@@ -192,6 +192,14 @@ __global__ void __launch_bounds__(kDecThreads)
     alj[c] = in ? s_al[j] : 0.f;
     kpj[c] = in ? s_kp[j] : 0.f;
   }
+  // the key that reads the state and the one the erase writes along:
+  // e = S' k, S -= e (b k)^T; the other erase form: e = S' (b k), S -= e k^T
+  float erj[NJ], ewj[NJ];
+#pragma unroll
+  for (int c = 0; c < NJ; ++c) {
+    erj[c] = a.erase ? kpj[c] : kj[c];
+    ewj[c] = a.erase ? kj[c] : kpj[c];
+  }
   const float invL = 1.0f / (float)a.L;
   for (int r0 = warp * RW; r0 < DV; r0 += kDecWarps * RW) {
     if (r0 != warp * RW) load_rows(r0);
@@ -203,7 +211,7 @@ __global__ void __launch_bounds__(kDecThreads)
       for (int c = 0; c < NJ; ++c) {
         ov = fmaf(sv[r][c], qj[c], ov);
         sv[r][c] *= alj[c];  // S' = S Diag(exp g)
-        ev = fmaf(sv[r][c], kj[c], ev);
+        ev = fmaf(sv[r][c], erj[c], ev);
       }
       ov = allsum(ov);
       ev = allsum(ev);
@@ -213,7 +221,7 @@ __global__ void __launch_bounds__(kDecThreads)
         for (int c = 0; c < NJ; ++c) {
           const int j = lane + 32 * c;
           if (j < DK)
-            S[(size_t)row * DK + j] = fmaf(-ev, kpj[c], fmaf(wv, kj[c], sv[r][c]));
+            S[(size_t)row * DK + j] = fmaf(-ev, ewj[c], fmaf(wv, kj[c], sv[r][c]));
         }
         if (lane == r) {  // spread the per-row scalars over the warp's lanes
           stf(o, row, ov);

@@ -137,7 +137,7 @@ __device__ void block_operands(const TIn* q, const TIn* k, const TIn* v,
                                float* Kh, float* Qt, float* Kp, float* Gl,
                                float* s_gam, float* s_w, float* W,
                                float dscale, const float* s_qn,
-                               const float* s_kn) {
+                               const float* s_kn, int erase) {
   for (int j = threadIdx.x; j < DK; j += blockDim.x) {
     float G = 0.f;
     for (int i = 0; i < C; ++i) {
@@ -150,7 +150,8 @@ __device__ void block_operands(const TIn* q, const TIn* k, const TIn* v,
       Kt[i * DK + j] = kk * gam;
       Kh[i * DK + j] = kk * igam;
       Qt[i * DK + j] = qq * expf(Gm);
-      Kp[i * DK + j] = bb * kk * igam;
+      // kap^ = b K / Gamma; the other erase form reads with kap~ = b K Gamma
+      Kp[i * DK + j] = bb * kk * (erase ? gam : igam);
       if (Gl) Gl[i * DK + j] = G;
     }
     s_gam[j] = expf(G);
@@ -165,10 +166,18 @@ __device__ void block_operands(const TIn* q, const TIn* k, const TIn* v,
   __syncthreads();
 }
 
-// The four strictly-lower Gram matrices and T of one block.
+// The four strictly-lower Gram matrices and T of one block (the other
+// erase form: A = tril(kap~ K^T) and P_k only).
 __device__ void block_grams(const float* Kt, const float* Kh, const float* Qt,
                             const float* Kp, int C, int DK, float* sA,
-                            float* sT, float* sM, float* sPk, float* sPq) {
+                            float* sT, float* sM, float* sPk, float* sPq,
+                            int erase) {
+  if (erase) {
+    mm(sA, C, Kp, DK, 1, Kh, 1, DK, C, C, DK, 1.f, false, true);
+    mm(sPk, C, Qt, DK, 1, Kh, 1, DK, C, C, DK, 1.f, false, true);
+    unit_lower_inverse(sT, sA, C);
+    return;
+  }
   // X Y^T: A(i, k) = X[i*DK + k], B(k, j) = Y[j*DK + k]
   mm(sA, C, Kt, DK, 1, Kp, 1, DK, C, C, DK, 1.f, false, true);
   mm(sM, C, Kt, DK, 1, Kh, 1, DK, C, C, DK, 1.f, false, true);
@@ -262,16 +271,26 @@ __global__ void __launch_bounds__(kThreads) fwd_generic_kernel(FwdArgs a) {
       token_inv_norms(q, k, 0, tt, T, h, H, Cb, DK, s_qn, s_kn, a.qknorm);
       block_operands(q, k, v, g, bx, w, s_p, 0, h, tt, T, H, Cb, DK, DV, Kt,
                      Kh, Qt, Kp, (float*)nullptr, s_gam, s_w, W, a.dscale,
-                     s_qn, s_kn);
-      block_grams(Kt, Kh, Qt, Kp, Cb, DK, sA, sT, sM, sPk, sPq);
-      // R = K~ S^T + M W ;  E = T R
-      mm(Rr, DV, Kt, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
-      mm(Rr, DV, sM, Cb, 1, W, DV, 1, Cb, DV, Cb, 1.f, true, false);
-      mm(E, DV, sT, Cb, 1, Rr, DV, 1, Cb, DV, Cb, 1.f, false, false);
-      // O = Q~ S^T + P_k W - P_kap E
-      mm(O, DV, Qt, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
-      mm(O, DV, sPk, Cb, 1, W, DV, 1, Cb, DV, Cb, 1.f, true, false);
-      mm(O, DV, sPq, Cb, 1, E, DV, 1, Cb, DV, Cb, -1.f, true, false);
+                     s_qn, s_kn, a.erase);
+      block_grams(Kt, Kh, Qt, Kp, Cb, DK, sA, sT, sM, sPk, sPq, a.erase);
+      if (a.erase) {
+        // other erase form: R = kap~ S^T - W ; E = T R ; O = Q~ S^T - P_k E
+        mm(Rr, DV, Kp, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
+        for (int idx = tid; idx < Cb * DV; idx += nt) Rr[idx] -= W[idx];
+        __syncthreads();
+        mm(E, DV, sT, Cb, 1, Rr, DV, 1, Cb, DV, Cb, 1.f, false, false);
+        mm(O, DV, Qt, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
+        mm(O, DV, sPk, Cb, 1, E, DV, 1, Cb, DV, Cb, -1.f, true, false);
+      } else {
+        // R = K~ S^T + M W ;  E = T R
+        mm(Rr, DV, Kt, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
+        mm(Rr, DV, sM, Cb, 1, W, DV, 1, Cb, DV, Cb, 1.f, true, false);
+        mm(E, DV, sT, Cb, 1, Rr, DV, 1, Cb, DV, Cb, 1.f, false, false);
+        // O = Q~ S^T + P_k W - P_kap E
+        mm(O, DV, Qt, DK, 1, S, 1, DK, Cb, DV, DK, 1.f, false, false);
+        mm(O, DV, sPk, Cb, 1, W, DV, 1, Cb, DV, Cb, 1.f, true, false);
+        mm(O, DV, sPq, Cb, 1, E, DV, 1, Cb, DV, Cb, -1.f, true, false);
+      }
       for (int idx = tid; idx < Cb * DV; idx += nt) {
         const int i = idx / DV, vv = idx - i * DV;
         stf(o, bthd(0, tt + i, h, vv, T, H, DV), O[idx]);
@@ -282,12 +301,17 @@ __global__ void __launch_bounds__(kThreads) fwd_generic_kernel(FwdArgs a) {
         s_msum[vv] += acc;
       }
       // S <- (S + W^T K^ - E^T kap^) Diag(gamma)
+      //      (other erase form: S <- (S - E^T K^) Diag(gamma))
       for (size_t idx = tid; idx < SZ; idx += nt) {
         const int vv = (int)(idx / DK), j = (int)(idx - (size_t)vv * DK);
         float acc = S[idx];
-        for (int i = 0; i < Cb; ++i)
-          acc = fmaf(W[i * DV + vv], Kh[i * DK + j],
-                     fmaf(-E[i * DV + vv], Kp[i * DK + j], acc));
+        if (a.erase)
+          for (int i = 0; i < Cb; ++i)
+            acc = fmaf(-E[i * DV + vv], Kh[i * DK + j], acc);
+        else
+          for (int i = 0; i < Cb; ++i)
+            acc = fmaf(W[i * DV + vv], Kh[i * DK + j],
+                       fmaf(-E[i * DV + vv], Kp[i * DK + j], acc));
         S[idx] = acc * s_gam[j];
       }
       __syncthreads();
@@ -406,10 +430,17 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
       const float* Sn = S + SZ;  // state at the end of this block
       token_inv_norms(q, k, b, t0, T, h, H, C, DK, s_qn, s_kn, a.qknorm);
       block_operands(q, k, v, g, bx, w, s_p, b, h, t0, T, H, C, DK, DV, Kt,
-                     Kh, Qt, Kp, Gl, s_gam, s_w, W, a.dscale, s_qn, s_kn);
-      block_grams(Kt, Kh, Qt, Kp, C, DK, sA, sT, sM, sPk, sPq);
-      mm(Rr, DV, Kt, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
-      mm(Rr, DV, sM, C, 1, W, DV, 1, C, DV, C, 1.f, true, false);
+                     Kh, Qt, Kp, Gl, s_gam, s_w, W, a.dscale, s_qn, s_kn,
+                     a.erase);
+      block_grams(Kt, Kh, Qt, Kp, C, DK, sA, sT, sM, sPk, sPq, a.erase);
+      if (a.erase) {
+        mm(Rr, DV, Kp, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
+        for (int idx = tid; idx < C * DV; idx += nt) Rr[idx] -= W[idx];
+        __syncthreads();
+      } else {
+        mm(Rr, DV, Kt, DK, 1, S, 1, DK, C, DV, DK, 1.f, false, false);
+        mm(Rr, DV, sM, C, 1, W, DV, 1, C, DV, C, 1.f, true, false);
+      }
       mm(E, DV, sT, C, 1, Rr, DV, 1, C, DV, C, 1.f, false, false);
       // upstream gradient of O, including this chunk's share of dm_{c+1}
       for (int idx = tid; idx < C * DV; idx += nt) {
@@ -428,52 +459,87 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
         s_dlg[j] = acc;  // gradient of log gamma_j
       }
       __syncthreads();
-      // dE = -kap^ dS~^T - P_kap^T dO ;  dR = T^T dE
-      mm(dE, DV, Kp, DK, 1, dSb, 1, DK, C, DV, DK, -1.f, false, false);
-      mm(dE, DV, sPq, 1, C, dO, DV, 1, C, DV, C, -1.f, true, false);
-      mm(dR, DV, sT, 1, C, dE, DV, 1, C, DV, C, 1.f, false, false);
-      // gradients of the four Gram matrices (strictly lower)
-      mm(dA, C, dR, DV, 1, E, 1, DV, C, C, DV, -1.f, false, true);
-      mm(dM, C, dR, DV, 1, W, 1, DV, C, C, DV, 1.f, false, true);
-      mm(dPk, C, dO, DV, 1, W, 1, DV, C, C, DV, 1.f, false, true);
-      mm(dPq, C, dO, DV, 1, E, 1, DV, C, C, DV, -1.f, false, true);
-      // dW = K^ dS~^T + P_k^T dO + M^T dR
-      mm(dW, DV, Kh, DK, 1, dSb, 1, DK, C, DV, DK, 1.f, false, false);
-      mm(dW, DV, sPk, 1, C, dO, DV, 1, C, DV, C, 1.f, true, false);
-      mm(dW, DV, sM, 1, C, dR, DV, 1, C, DV, C, 1.f, true, false);
-      for (int idx = tid; idx < C * DV; idx += nt) {
-        const int i = idx / DV, vv = idx - i * DV;
-        stf(dv, bthd(b, t0 + i, h, vv, T, H, DV), s_w[i] * dW[idx]);
+      if (a.erase) {
+        // other erase form (R = kap~ S^T - W, A = tril(kap~ K^T),
+        // O = Q~ S^T - P_k E, S_new = (S - E^T K^) Diag(gamma)):
+        // dE = -K^ dS~^T - P_k^T dO ;  dR = T^T dE
+        mm(dE, DV, Kh, DK, 1, dSb, 1, DK, C, DV, DK, -1.f, false, false);
+        mm(dE, DV, sPk, 1, C, dO, DV, 1, C, DV, C, -1.f, true, false);
+        mm(dR, DV, sT, 1, C, dE, DV, 1, C, DV, C, 1.f, false, false);
+        mm(dA, C, dR, DV, 1, E, 1, DV, C, C, DV, -1.f, false, true);
+        mm(dPk, C, dO, DV, 1, E, 1, DV, C, C, DV, -1.f, false, true);
+        for (int idx = tid; idx < C * DV; idx += nt) dW[idx] = -dR[idx];
+        __syncthreads();
+        for (int idx = tid; idx < C * DV; idx += nt) {
+          const int i = idx / DV, vv = idx - i * DV;
+          stf(dv, bthd(b, t0 + i, h, vv, T, H, DV), s_w[i] * dW[idx]);
+        }
+        for (int i = tid; i < C; i += nt) {
+          float acc = 0.f;
+          for (int vv = 0; vv < DV; ++vv)
+            acc = fmaf(dW[i * DV + vv], ldf(v, bthd(b, t0 + i, h, vv, T, H, DV)), acc);
+          stf(dw, ((size_t)b * T + t0 + i) * H + h, acc);
+        }
+        for (int idx = tid; idx < C * DK; idx += nt) dKt[idx] = 0.f;
+        // dkap~ = dR S + dA K^ ;  dK^ = dA^T kap~ + dP_k^T Q~ - E dS~
+        mm(dKp, DK, dR, DV, 1, S, DK, 1, C, DK, DV, 1.f, false, false);
+        mm(dKp, DK, dA, C, 1, Kh, DK, 1, C, DK, C, 1.f, true, false);
+        mm(dKh, DK, dA, 1, C, Kp, DK, 1, C, DK, C, 1.f, false, false);
+        mm(dKh, DK, dPk, 1, C, Qt, DK, 1, C, DK, C, 1.f, true, false);
+        mm(dKh, DK, E, DV, 1, dSb, DK, 1, C, DK, DV, -1.f, true, false);
+        // dQ~ = dO S + dP_k K^
+        mm(dQt, DK, dO, DV, 1, S, DK, 1, C, DK, DV, 1.f, false, false);
+        mm(dQt, DK, dPk, C, 1, Kh, DK, 1, C, DK, C, 1.f, true, false);
+      } else {
+        // dE = -kap^ dS~^T - P_kap^T dO ;  dR = T^T dE
+        mm(dE, DV, Kp, DK, 1, dSb, 1, DK, C, DV, DK, -1.f, false, false);
+        mm(dE, DV, sPq, 1, C, dO, DV, 1, C, DV, C, -1.f, true, false);
+        mm(dR, DV, sT, 1, C, dE, DV, 1, C, DV, C, 1.f, false, false);
+        // gradients of the four Gram matrices (strictly lower)
+        mm(dA, C, dR, DV, 1, E, 1, DV, C, C, DV, -1.f, false, true);
+        mm(dM, C, dR, DV, 1, W, 1, DV, C, C, DV, 1.f, false, true);
+        mm(dPk, C, dO, DV, 1, W, 1, DV, C, C, DV, 1.f, false, true);
+        mm(dPq, C, dO, DV, 1, E, 1, DV, C, C, DV, -1.f, false, true);
+        // dW = K^ dS~^T + P_k^T dO + M^T dR
+        mm(dW, DV, Kh, DK, 1, dSb, 1, DK, C, DV, DK, 1.f, false, false);
+        mm(dW, DV, sPk, 1, C, dO, DV, 1, C, DV, C, 1.f, true, false);
+        mm(dW, DV, sM, 1, C, dR, DV, 1, C, DV, C, 1.f, true, false);
+        for (int idx = tid; idx < C * DV; idx += nt) {
+          const int i = idx / DV, vv = idx - i * DV;
+          stf(dv, bthd(b, t0 + i, h, vv, T, H, DV), s_w[i] * dW[idx]);
+        }
+        for (int i = tid; i < C; i += nt) {
+          float acc = 0.f;
+          for (int vv = 0; vv < DV; ++vv)
+            acc = fmaf(dW[i * DV + vv], ldf(v, bthd(b, t0 + i, h, vv, T, H, DV)), acc);
+          stf(dw, ((size_t)b * T + t0 + i) * H + h, acc);
+        }
+        // dK~ = dR S + dA kap^ + dM K^
+        mm(dKt, DK, dR, DV, 1, S, DK, 1, C, DK, DV, 1.f, false, false);
+        mm(dKt, DK, dA, C, 1, Kp, DK, 1, C, DK, C, 1.f, true, false);
+        mm(dKt, DK, dM, C, 1, Kh, DK, 1, C, DK, C, 1.f, true, false);
+        // dK^ = dM^T K~ + dP_k^T Q~ + W dS~
+        mm(dKh, DK, dM, 1, C, Kt, DK, 1, C, DK, C, 1.f, false, false);
+        mm(dKh, DK, dPk, 1, C, Qt, DK, 1, C, DK, C, 1.f, true, false);
+        mm(dKh, DK, W, DV, 1, dSb, DK, 1, C, DK, DV, 1.f, true, false);
+        // dkap^ = dA^T K~ + dP_kap^T Q~ - E dS~
+        mm(dKp, DK, dA, 1, C, Kt, DK, 1, C, DK, C, 1.f, false, false);
+        mm(dKp, DK, dPq, 1, C, Qt, DK, 1, C, DK, C, 1.f, true, false);
+        mm(dKp, DK, E, DV, 1, dSb, DK, 1, C, DK, DV, -1.f, true, false);
+        // dQ~ = dO S + dP_k K^ + dP_kap kap^
+        mm(dQt, DK, dO, DV, 1, S, DK, 1, C, DK, DV, 1.f, false, false);
+        mm(dQt, DK, dPk, C, 1, Kh, DK, 1, C, DK, C, 1.f, true, false);
+        mm(dQt, DK, dPq, C, 1, Kp, DK, 1, C, DK, C, 1.f, true, false);
       }
-      for (int i = tid; i < C; i += nt) {
-        float acc = 0.f;
-        for (int vv = 0; vv < DV; ++vv)
-          acc = fmaf(dW[i * DV + vv], ldf(v, bthd(b, t0 + i, h, vv, T, H, DV)), acc);
-        stf(dw, ((size_t)b * T + t0 + i) * H + h, acc);
-      }
-      // dK~ = dR S + dA kap^ + dM K^
-      mm(dKt, DK, dR, DV, 1, S, DK, 1, C, DK, DV, 1.f, false, false);
-      mm(dKt, DK, dA, C, 1, Kp, DK, 1, C, DK, C, 1.f, true, false);
-      mm(dKt, DK, dM, C, 1, Kh, DK, 1, C, DK, C, 1.f, true, false);
-      // dK^ = dM^T K~ + dP_k^T Q~ + W dS~
-      mm(dKh, DK, dM, 1, C, Kt, DK, 1, C, DK, C, 1.f, false, false);
-      mm(dKh, DK, dPk, 1, C, Qt, DK, 1, C, DK, C, 1.f, true, false);
-      mm(dKh, DK, W, DV, 1, dSb, DK, 1, C, DK, DV, 1.f, true, false);
-      // dkap^ = dA^T K~ + dP_kap^T Q~ - E dS~
-      mm(dKp, DK, dA, 1, C, Kt, DK, 1, C, DK, C, 1.f, false, false);
-      mm(dKp, DK, dPq, 1, C, Qt, DK, 1, C, DK, C, 1.f, true, false);
-      mm(dKp, DK, E, DV, 1, dSb, DK, 1, C, DK, DV, -1.f, true, false);
-      // dQ~ = dO S + dP_k K^ + dP_kap kap^
-      mm(dQt, DK, dO, DV, 1, S, DK, 1, C, DK, DV, 1.f, false, false);
-      mm(dQt, DK, dPk, C, 1, Kh, DK, 1, C, DK, C, 1.f, true, false);
-      mm(dQt, DK, dPq, C, 1, Kp, DK, 1, C, DK, C, 1.f, true, false);
       // gradient of the block-start state: dS~ + dO^T Q~ + dR^T K~
+      // (other erase form: dR^T kap~)
+      const float* Rk = a.erase ? Kp : Kt;
       for (size_t idx = tid; idx < SZ; idx += nt) {
         const int vv = (int)(idx / DK), j = (int)(idx - (size_t)vv * DK);
         float acc = dSb[idx];
         for (int i = 0; i < C; ++i)
           acc = fmaf(dO[i * DV + vv], Qt[i * DK + j],
-                     fmaf(dR[i * DV + vv], Kt[i * DK + j], acc));
+                     fmaf(dR[i * DV + vv], Rk[i * DK + j], acc));
         dS[idx] = acc;
       }
       // per key channel: chain rule through Gamma, the gate and the inputs;
@@ -489,7 +555,9 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
           const float kk = ldf(k, x) * s_kn[i];
           const float bb = sigm(ldf(bx, x) + s_p[j]);
           const float gq = dQt[e] * expf(Gm);
-          const float gk = dKt[e] * gam + dKh[e] * igam + dKp[e] * bb * igam;
+          // kap^ = b K / Gamma (kap~ = b K Gamma in the other erase form)
+          const float kps = a.erase ? gam : igam;
+          const float gk = dKt[e] * gam + dKh[e] * igam + dKp[e] * bb * kps;
           if (a.qknorm) {  // gradients of the unit rows: projected below
             Dq[e] = gq;
             Dk[e] = gk;
@@ -497,10 +565,11 @@ __global__ void __launch_bounds__(kThreads) bwd_generic_kernel(BwdArgs a) {
             stf(dq, x, gq);
             stf(dk, x, gk);
           }
-          const float dz = dKp[e] * kk * igam * bb * (1.f - bb);
+          const float dz = dKp[e] * kk * kps * bb * (1.f - bb);
           stf(dbx, x, dz);
           s_dp[j] += dz;
-          float dG = dKt[e] * Kt[e] - dKh[e] * Kh[e] - dKp[e] * Kp[e];
+          float dG = dKt[e] * Kt[e] - dKh[e] * Kh[e] +
+                     (a.erase ? dKp[e] : -dKp[e]) * Kp[e];
           if (i == C - 1) dG += s_dlg[j];
           if (i + 1 < C) dG += dQt[e + DK] * Qt[e + DK];
           acc += dG;

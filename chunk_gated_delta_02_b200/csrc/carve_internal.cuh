@@ -39,14 +39,15 @@ constexpr size_t kTcRecBytes = 57344;
 // (the training forward, whose records this describes, and the backward).
 inline bool tc_shape(const carve_shape& s) {
   return s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 128 &&
-         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0 && !s.qk_l2norm;
+         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0 && !s.qk_l2norm &&
+         !s.erase_form;
 }
 // The tensor-core forward also runs, without training, DV = 256 (two CTAs
 // per pair) and chunks of 16, 32 or 48 tokens (one chunk per block, the
 // 64-row tiles zero past the chunk).
 inline bool tc_fwd_shape(const carve_shape& s, bool training) {
   if (tc_shape(s)) return true;
-  if (training) return false;
+  if (training || s.erase_form) return false;
   const bool chunk_ok = s.L % kMaxBlock == 0 || (s.L < kMaxBlock && s.L % 16 == 0);
   return !training && s.dtype == CARVE_BF16 && s.DK == 128 &&
          (s.DV == 128 || s.DV == 256) && chunk_ok && s.R <= 32 && s.T > 0;
@@ -168,6 +169,7 @@ struct FwdArgs {
   int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
   float dscale;     // decay activation scale (0: g is the log-decay)
   int qknorm;       // 1: q, k are normalised per token inside the kernels
+  int erase;        // 1: the other erase form S' (I - (b k) k^T)
   // packed sequences: B sequences at token offsets cu[b] .. cu[b + 1] of a
   // T-token tensor ([T, H, D] layouts), or NULL: B sequences of T tokens
   const int32_t* cu;
@@ -191,6 +193,7 @@ struct BwdArgs {
   int stall_block;  // test only: block whose MMA commit CTA 0 redirects (-1: none)
   float dscale;     // decay activation scale (0: g is the log-decay)
   int qknorm;       // 1: q, k are normalised per token inside the kernels
+  int erase;        // 1: the other erase form S' (I - (b k) k^T)
 };
 
 // Arguments of the decode step (one token per (sequence, head)).
@@ -202,6 +205,7 @@ struct DecArgs {
   void* o;              // [B, H, DV]
   float dscale;         // decay activation scale (0: g is the log-decay)
   int qknorm;           // 1: q, k are normalised inside the kernel
+  int erase;            // 1: the other erase form S' (I - (b k) k^T)
 };
 cudaError_t launch_decode(const DecArgs& a, int dtype, cudaStream_t st);
 

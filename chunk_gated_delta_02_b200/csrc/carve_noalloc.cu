@@ -88,6 +88,7 @@ extern "C" carve_status carve_chunk_fwd_noalloc(
   a.stall_block = -1;
   a.dscale = s.decay_scale;
   a.qknorm = s.qk_l2norm;
+  a.erase = s.erase_form;
   cudaError_t e = launch_fwd_generic(a, s.dtype, (cudaStream_t)stream);
   return e == cudaSuccess ? CARVE_OK : CARVE_ERR_CUDA;
 }

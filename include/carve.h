@@ -85,6 +85,13 @@ typedef struct {
                        * gradients of the raw q and k.  Other values:
                        * CARVE_ERR_INVALID_ARG.  Training with 1 runs on
                        * the generic kernels. */
+  int32_t erase_form; /* 0: S' (I - k (b (.) k)^T) as above; 1: the other
+                       * erase that acts on the key axis only,
+                       * S' (I - (b (.) k) k^T) (the gated key reads the
+                       * state, the plain key is written; both forms are
+                       * chunkable, gist.science section 3).  Form 1 runs on
+                       * the generic kernels and the decode step.  Other
+                       * values: CARVE_ERR_INVALID_ARG. */
 } carve_shape;
 
 /*

@@ -36,8 +36,10 @@ def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-x))
 
 
-def decode_step(S, m, osum, pos, q, k, v, g, bx, w, u_down, u_up, L):
-    """One token for one (sequence, head) pair, in fp64.
+def decode_step(S, m, osum, pos, q, k, v, g, bx, w, u_down, u_up, L,
+                erase=0):
+    """One token for one (sequence, head) pair, in fp64.  erase = 1: the
+    other key-axis erase, e = S' (b * k) and S = S' - e k^T + w v k^T.
 
     S [DV, DK], m [DV], osum [DV]; q, k, g, bx [DK]; v [DV]; w scalar;
     u_down [R, DV]; u_up [DK, R].  Returns (o [DV], S, m, osum) after the
@@ -47,8 +49,12 @@ def decode_step(S, m, osum, pos, q, k, v, g, bx, w, u_down, u_up, L):
     b = sigmoid(bx + p)
     o = S @ q
     S1 = S * np.exp(g)[None, :]
-    e = S1 @ k
-    S_new = S1 - np.outer(e, b * k) + w * np.outer(v, k)
+    if erase:
+        e = S1 @ (b * k)
+        S_new = S1 - np.outer(e, k) + w * np.outer(v, k)
+    else:
+        e = S1 @ k
+        S_new = S1 - np.outer(e, b * k) + w * np.outer(v, k)
     osum_new = osum + o
     m_new = np.array(m, np.float64)
     if (pos + 1) % L == 0:
@@ -57,7 +63,8 @@ def decode_step(S, m, osum, pos, q, k, v, g, bx, w, u_down, u_up, L):
     return o, S_new, m_new, osum_new
 
 
-def decode_steps(S, m, osum, pos0, q, k, v, g, bx, w, u_down, u_up, L):
+def decode_steps(S, m, osum, pos0, q, k, v, g, bx, w, u_down, u_up, L,
+                 erase=0):
     """T consecutive steps for one pair: q, k, g, bx [T, DK], v [T, DV],
     w [T].  Returns (o [T, DV], S, m, osum)."""
     T = q.shape[0]
@@ -65,5 +72,5 @@ def decode_steps(S, m, osum, pos0, q, k, v, g, bx, w, u_down, u_up, L):
     for t in range(T):
         out[t], S, m, osum = decode_step(S, m, osum, pos0 + t, q[t], k[t],
                                          v[t], g[t], bx[t], w[t], u_down,
-                                         u_up, L)
+                                         u_up, L, erase)
     return out, S, m, osum

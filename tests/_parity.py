@@ -48,25 +48,28 @@ class Gathered:
                 for n in self.g}
 
 
-def run_fwd(inp, L, training=False, decay_scale=0.0, qk_l2norm=False):
+def run_fwd(inp, L, training=False, decay_scale=0.0, qk_l2norm=False,
+            erase_form=0):
     d = to_dev(inp)
     o, S_T, m_T, ws = carve.chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["bx"],
                                       d["w"], d["u_down"], d["u_up"], L,
                                       d["S0"], d["m0"], training=training,
                                       decay_scale=decay_scale,
-                                      qk_l2norm=qk_l2norm)
+                                      qk_l2norm=qk_l2norm,
+                                      erase_form=erase_form)
     torch.cuda.synchronize()
     return d, o, S_T, m_T, ws
 
 
-def fwd_errors(inp, L, pairs=None, decay_scale=0.0, qk_l2norm=False):
+def fwd_errors(inp, L, pairs=None, decay_scale=0.0, qk_l2norm=False,
+               erase_form=0):
     """GPU forward over the whole batch; oracle on `pairs` (default all).
     decay_scale > 0: inp["g"] holds raw decay logits (both sides activate)."""
     _, o, S_T, m_T, ws = run_fwd(inp, L, decay_scale=decay_scale,
-                                 qk_l2norm=qk_l2norm)
+                                 qk_l2norm=qk_l2norm, erase_form=erase_form)
     assert carve.get_status(ws) == 0
     res = ref.fwd_batch(inp, L, pairs=pairs, decay_scale=decay_scale,
-                        qk_norm=qk_l2norm)
+                        qk_norm=qk_l2norm, erase=erase_form)
     acc = Gathered()
     o_c, S_c, m_c = o.cpu(), S_T.cpu(), m_T.cpu()
     for (b, h), (oo, SS, mm) in res.items():
@@ -77,17 +80,19 @@ def fwd_errors(inp, L, pairs=None, decay_scale=0.0, qk_l2norm=False):
 
 
 def bwd_errors(inp, L, grads, pairs=None, du_heads=(), decay_scale=0.0,
-               qk_l2norm=False):
+               qk_l2norm=False, erase_form=0):
     """GPU training forward + backward; oracle reverse pass on `pairs`.
     du_down / du_up (summed over the batch) are compared for each head in
     `du_heads`, for which the oracle runs every sequence of that head."""
     d, o, S_T, m_T, ws = run_fwd(inp, L, training=True,
-                                 decay_scale=decay_scale, qk_l2norm=qk_l2norm)
+                                 decay_scale=decay_scale, qk_l2norm=qk_l2norm,
+                                 erase_form=erase_form)
     dd = to_dev(grads)
     gr = carve.chunk_bwd(d["q"], d["k"], d["v"], d["g"], d["bx"], d["w"],
                          d["u_down"], d["u_up"], L, dd["d_o"], ws,
                          dd.get("dS_T"), dd.get("dm_T"),
-                         decay_scale=decay_scale, qk_l2norm=qk_l2norm)
+                         decay_scale=decay_scale, qk_l2norm=qk_l2norm,
+                         erase_form=erase_form)
     torch.cuda.synchronize()
     assert carve.get_status(ws) == 0
     B, _, H, _ = inp["q"].shape
@@ -96,7 +101,7 @@ def bwd_errors(inp, L, grads, pairs=None, du_heads=(), decay_scale=0.0,
     need = sorted(set(pairs) | {(b, h) for h in du_heads for b in range(B)})
     res = ref.bwd_batch(inp, L, grads["d_o"], grads.get("dS_T"),
                         grads.get("dm_T"), pairs=need, decay_scale=decay_scale,
-                        qk_norm=qk_l2norm)
+                        qk_norm=qk_l2norm, erase=erase_form)
     g = {k: (None if v is None else v.cpu()) for k, v in gr.items()}
     acc = Gathered()
     for (b, h) in pairs:

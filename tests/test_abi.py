@@ -39,10 +39,11 @@ def test_header_declarations_are_exported(lib):
 
 def shape(**kw):
     d = dict(B=2, T=128, H=3, DK=64, DV=64, R=8, L=64, dtype=0,
-             decay_scale=0.0, qk_l2norm=0)
+             decay_scale=0.0, qk_l2norm=0, erase_form=0)
     d.update(kw)
     return carve.Shape(*(d[n] for n in ("B", "T", "H", "DK", "DV", "R", "L",
-                                        "dtype", "decay_scale", "qk_l2norm")))
+                                        "dtype", "decay_scale", "qk_l2norm",
+                                        "erase_form")))
 
 
 def ws_bytes(lib, s, training):
@@ -81,6 +82,10 @@ def test_decay_scale_validation(lib):
     path = lambda **kw: lib.carve_fwd_path(ctypes.byref(shape(**kw))).decode()
     tc = dict(DK=128, DV=128, R=32, L=64, T=128, dtype=carve.CARVE_BF16)
     assert path(**dict(tc, qk_l2norm=1)) == "tc"
+    # the other erase form runs on the generic kernels
+    assert path(**dict(tc, erase_form=1)) == "generic"
+    for bad in (2, -1):
+        assert call_fwd(lib, shape(erase_form=bad), FAKE, 1 << 20) == 1, bad
     n_tc = ws_bytes(lib, shape(**tc), 1)
     n_norm = ws_bytes(lib, shape(**dict(tc, qk_l2norm=1)), 1)
     assert n_norm - ws_bytes(lib, shape(**dict(tc, qk_l2norm=1)), 0) >= \

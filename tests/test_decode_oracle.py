@@ -49,6 +49,20 @@ def test_decode_steps_equal_token_recurrence(T, L):
         assert rel(m, m_c) < 1e-12
 
 
+def test_decode_steps_other_erase_form_equal_token_recurrence():
+    rng = np.random.default_rng(61)
+    a = rand_pair(rng, 13, 6, 5, 3, ub_std=0.8)
+    DV = 5
+    o, S, m, osum = decode.decode_steps(
+        a["S0"].copy(), a["m0"].copy(), np.zeros(DV), 0, a["q"], a["k"],
+        a["v"], a["g"], a["bx"], a["w"], a["u_down"], a["u_up"], 4, erase=1)
+    o_ref, S_ref, m_ref = ref.fwd_pair(a["q"], a["k"], a["v"], a["g"],
+                                       a["bx"], a["w"], a["u_down"],
+                                       a["u_up"], 4, a["S0"], a["m0"], erase=1)
+    assert rel(o, o_ref) < 1e-12 and rel(S, S_ref) < 1e-12
+    assert rel(osum / 4, m_ref) < 1e-12  # 13 tokens: a partial last chunk
+
+
 def test_decode_resumes_mid_chunk():
     # stopping after 6 tokens (mid-chunk, L = 4) and continuing from the
     # carried (S, m, osum, pos) equals one run over all 14 tokens
@@ -64,7 +78,7 @@ def test_decode_resumes_mid_chunk():
 
 
 def _broken(kind):
-    def step(S, m, osum, pos, q, k, v, g, bx, w, u_down, u_up, L):
+    def step(S, m, osum, pos, q, k, v, g, bx, w, u_down, u_up, L, erase=0):
         p = u_up @ (u_down @ m)
         b = decode.sigmoid(bx + p)
         o = S @ q
