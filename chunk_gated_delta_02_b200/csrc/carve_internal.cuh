@@ -140,6 +140,27 @@ __device__ __forceinline__ float decay_act(float a, float s) {
 __device__ __forceinline__ float decay_act_grad(float g, float s) {
   return s > 0.f ? s * expm1f(g / s) : 1.f;
 }
+// The same over 8 values passed by value (a row at or past `valid` gets
+// log-decay 0), kept out of line: the hot loops call it only under a
+// uniform s > 0 branch, so neither its code nor its transcendental
+// functions cost anything when the log-decay is given.
+struct F8 {
+  float x[8];
+};
+static __device__ __noinline__ F8 decay_act8(F8 v, float s, bool valid) {
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    v.x[e] = valid ? -s * (fmaxf(v.x[e], 0.f) + log1pf(expf(-fabsf(v.x[e])))) : 0.f;
+  return v;
+}
+static __device__ __forceinline__ void decay_act8(float* x, float s, bool valid) {
+  F8 v;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v.x[e] = x[e];
+  v = decay_act8(v, s, valid);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) x[e] = v.x[e];
+}
 
 // Element load/store in the I/O dtype, arithmetic in fp32.
 __device__ __forceinline__ float ldf(const float* p, size_t i) { return p[i]; }

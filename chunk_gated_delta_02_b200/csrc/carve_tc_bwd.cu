@@ -772,10 +772,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       {
         float gsum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          gv[e] = decay_act(ldbf(sm + R_RO + sw128_off(tb + e, jj, 64)), a.dscale);
-          gsum += gv[e];
+        for (int e = 0; e < 16; ++e) gv[e] = ldbf(sm + R_RO + sw128_off(tb + e, jj, 64));
+        if (a.dscale > 0.f) {  // raw decay logits (uniform branch)
+          decay_act8(gv, a.dscale, true);
+          decay_act8(gv + 8, a.dscale, true);
         }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) gsum += gv[e];
         s_gq[gp * 128 + jj] = gsum;
       }
       __syncthreads();
@@ -864,11 +867,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // with raw decay logits a (decay_scale s > 0) the output is dL/da =
       // dL/dg * s expm1(g / s), formed from the log-decay itself
       const float dsc = a.dscale;
+      if (dsc > 0.f) {  // uniform branch: dL/dg -> dL/da needs s expm1(g / s)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) gv[i] = decay_act_grad(gv[i], dsc);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) gv[i] = 1.f;
+      }
       float hg = 0.f;  // the odd token's suffix sum
 #pragma unroll
       for (int i = 15; i >= 0; --i) {
         acc += dGv[i];
-        const float out = dsc > 0.f ? acc * decay_act_grad(gv[i], dsc) : acc;
+        const float out = acc * gv[i];
         if (i & 1)
           hg = out;
         else

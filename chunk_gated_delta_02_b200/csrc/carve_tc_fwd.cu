@@ -96,7 +96,7 @@ constexpr int B_X = 6;     // dv = 256: the other CTA's half of U_down m arrived
 constexpr int B_WK = 7;    // S += W^T K^ (issued with MMA 2)
 constexpr int B_TEST = 8;  // test only: the redirected commit of a stalled block
 constexpr int B_FIN = 9;   // an aborting CTA: thread 0's D1 MMAs not yet committed
-constexpr int B_GM = 10;   // the next block's [M; P_k], issued in step 6
+constexpr int B_GM = 10;   // [M; P_k] (thread 32, step 2)
 constexpr int kNumBars = 11;
 static_assert(SM_BAR + 8 * kNumBars <= SM_TMEM, "mbarriers");
 
@@ -455,32 +455,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (tid == 32 && ib + 2 < NB) prefetch_kqg(ib + 2);
 
     // ---- 2. the key side (K~, Q~ in X; K^ in KHP) was formed during the
-    //      previous block's solve, the chunk's gate p at the previous
-    //      chunk's end, and the b-independent half of the Grams, [M; P_k] =
-    //      [K~; Q~] K^T, issued with the previous block's MMA 3b / 4 (here
-    //      for block 0).  Thread 0 issues D1 = S [K~; Q~]^T; warps 8-15 form
-    //      W = w V; then warps 1-15 form kap^ = sigmoid(b_x + p) K^ next to
-    //      K^ (warps 8-15 waited for this block's v, g, b_x tiles in its key
-    //      transform)
+    //      previous block's solve and the chunk's gate p at the previous
+    //      chunk's end.  Thread 0 issues D1 = S [K~; Q~]^T, thread 32 the
+    //      b-independent half of the Grams, [M; P_k] = [K~; Q~] K^T; warps
+    //      8-15 form W = w V; then warps 2-15 form kap^ = sigmoid(b_x + p) K^
+    //      next to K^ (warps 8-15 waited for this block's v, g, b_x tiles in
+    //      its key transform)
     if (tid == 0) {
       tc_fence_after();
       const uint32_t x0 = smem_u32(sm + OFF_X), sb0 = smem_u32(sm + OFF_SB);
-      const uint32_t kh0 = smem_u32(sm + OFF_KHP);
 #pragma unroll 1
       for (int ks = 0; ks < 8; ++ks) {
         const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
         umma_bf16(tmem + TM_D1, desc_kmajor_sw128(sb0 + kx),
                   desc_kmajor_sw128(x0 + kx), ID_N128, ks > 0);
       }
-      if (ib == 0) {  // later blocks' [M; P_k] was issued in step 6 before
-#pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
-                    desc_kmajor_sw128(kh0 + kx), ID_N64, ks > 0);
-        }
-      }
       d1_open = true;
+    } else if (tid == 32) {
+      // the b-independent half of the Grams, [M; P_k] = [K~; Q~] K^T, from a
+      // second issuer so that it runs beside D1; only step 4b waits for it
+      tc_fence_after();
+      const uint32_t x0 = smem_u32(sm + OFF_X), kh0 = smem_u32(sm + OFF_KHP);
+#pragma unroll 1
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
+        umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
+                  desc_kmajor_sw128(kh0 + kx), ID_N64, ks > 0);
+      }
+      umma_commit(bars + B_GM);
+      // this thread never waits on B_GM: it tracks the parity of the phase
+      // it just started (block ib's) so that an aborting CTA drains it
+      npar = (npar & ~(1u << B_GM)) | ((uint32_t)(ib & 1) << B_GM);
+      mark(B_GM);
     }
     if (warp < 8) {
       wait(B_VGB, 1);
@@ -512,12 +518,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
 
-    // ---- 3. kap^ (warps 1-15); then the gate half of the Grams,
-    //      [A; P_kap] = [K~; Q~] kap^T.  The commit after it covers D1 and
-    //      [M; P_k] as well.
-    if (warp > 0)
-      tc::kappa_in_place(sm + OFF_KHP, sm + OFF_RB, s_p, 16384, tid - 32,
-                         kThreads - 32);
+    // ---- 3. kap^ (warps 2-15; warps 0 and 1 issued the MMAs); then the
+    //      gate half of the Grams, [A; P_kap] = [K~; Q~] kap^T.  The commit
+    //      after it covers D1 as well.
+    if (warp > 1)
+      tc::kappa_in_place(sm + OFF_KHP, sm + OFF_RB, s_p, 16384, tid - 64,
+                         kThreads - 64);
     fence_async_smem();
     if (tid == 256 && rec) bulk_wait_read_all();  // S record read: SB reusable
     if (__syncthreads_or(*s_abort)) break;  // one decision for all threads
@@ -591,10 +597,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---- 4b. [M; P_k] (strictly lower, 32 columns per group) -> bf16
       //          operand; MMA 2; R^T -> bf16 operand (warps 4-11)
       const int part = gp - 1;
-      if (ib > 0) {  // [M; P_k] of this block, issued in the previous block's step 6
-        wait(B_GM, 13);
-        tc_fence_after();
-      }
+      wait(B_GM, 13);  // [M; P_k], issued by thread 32 in step 2
+      tc_fence_after();
       {
         float vals[32];
         tmem_ld32(tl + TM_GM + part * 32, vals);
@@ -762,20 +766,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       umma_commit(bars + B_M4);
       mark(B_M4);
-      if (ib + 1 < NB) {
-        // the next block's b-independent Grams [M; P_k] = [K~; Q~] K^T: its
-        // key side is in X and KHP (step 4c) and TM_GM was read in step 4b.
-        // Its own commit: only step 4b of the next block waits for it.
-        const uint32_t x0 = smem_u32(sm + OFF_X), kh0 = smem_u32(sm + OFF_KHP);
-#pragma unroll 1
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t kx = (ks >> 2) * 16384 + (ks & 3) * 32;
-          umma_bf16(tmem + TM_GM, desc_kmajor_sw128(x0 + kx),
-                    desc_kmajor_sw128(kh0 + kx), ID_N64, ks > 0);
-        }
-        umma_commit(bars + B_GM);
-        mark(B_GM);
-      }
     }
     wait(B_M4, 8);
     tc_fence_after();
@@ -848,7 +838,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(bars + B_FIN);
       mark(B_FIN);
     }
-    if (tid == 0 || tid == 128 || tid == 256)  // the threads that start copies and MMAs
+    if (tid == 0 || tid == 32 || tid == 128 || tid == 256)  // the threads that start copies and MMAs
       for (int i = 0; i < kNumBars; ++i)
         if ((pend >> i) & 1u) tc::drain_bar(bars + i, (npar >> i) & 1u);
   } else if (a.m_T && tid < 128) {  // the last chunk's mean

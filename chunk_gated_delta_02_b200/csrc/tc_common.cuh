@@ -132,11 +132,11 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
   for (int i = 0; i < TPT; ++i) {
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
+    // raw decay logits -> log-decay (dscale > 0; rows past the block's
+    // nvalid tokens: 0).  A uniform branch around an out-of-line helper.
+    if (dscale > 0.f) decay_act8(gv, dscale, TPT * tg + i < nvalid);
 #pragma unroll
-    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0);
-                                 // rows past the block's nvalid tokens: 0
-      gl[i][e] = (i ? gl[i - 1][e] : 0.f) +
-                 (TPT * tg + i < nvalid ? decay_act(gv[e], dscale) : 0.f);
+    for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
   }
   float ex[8];  // exclusive prefix of the token group
   float wt[8];  // running inclusive sum over the warp's groups
@@ -274,11 +274,11 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
   for (int i = 0; i < TPT; ++i) {
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
+    // raw decay logits -> log-decay (dscale > 0; rows past the block's
+    // nvalid tokens: 0).  A uniform branch around an out-of-line helper.
+    if (dscale > 0.f) decay_act8(gv, dscale, TPT * tg + i < nvalid);
 #pragma unroll
-    for (int e = 0; e < 8; ++e)  // raw decay logits -> log-decay (dscale > 0);
-                                 // rows past the block's nvalid tokens: 0
-      gl[i][e] = (i ? gl[i - 1][e] : 0.f) +
-                 (TPT * tg + i < nvalid ? decay_act(gv[e], dscale) : 0.f);
+    for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
   }
   float ex[8];  // exclusive prefix of the token group
   float wt[8];  // running inclusive sum over the warp's groups
