@@ -99,6 +99,8 @@ __global__ void __launch_bounds__(kDecThreads)
   // the first batch of this warp's state rows: requested before anything
   // else, so that the gate below runs while they are in flight
   float sv[RW][NJ];
+  float osv = 0.f;  // lane r < RW: the running output sum of row r0 + r
+  float* osum = a.osum + (size_t)pair * DV;
   auto load_rows = [&](int r0) {
 #pragma unroll
     for (int r = 0; r < RW; ++r)
@@ -107,6 +109,7 @@ __global__ void __launch_bounds__(kDecThreads)
         const int j = lane + 32 * c;
         sv[r][c] = (r0 + r < DV && j < DK) ? S[(size_t)(r0 + r) * DK + j] : 0.f;
       }
+    osv = (lane < RW && r0 + lane < DV) ? osum[r0 + lane] : 0.f;
   };
   load_rows(warp * RW);
 
@@ -116,7 +119,6 @@ __global__ void __launch_bounds__(kDecThreads)
   const TIn* bx = static_cast<const TIn*>(a.bx) + (size_t)pair * DK;
   const TIn* v = static_cast<const TIn*>(a.v) + (size_t)pair * DV;
   float* m = a.m + (size_t)pair * DV;
-  float* osum = a.osum + (size_t)pair * DV;
   TIn* o = static_cast<TIn*>(a.o) + (size_t)pair * DV;
   const float w = ldf(static_cast<const TIn*>(a.w), pair);
   const bool chunk_end = (a.pos[bseq] + 1) % a.L == 0;
@@ -172,12 +174,16 @@ __global__ void __launch_bounds__(kDecThreads)
     if (lane == 0) s_h[r] = acc;
   }
   __syncthreads();
-  // p = U_up h, b = sigmoid(b_x + p), b k
-  for (int j = tid; j < DK; j += kDecThreads) {
+  // p = U_up h (one warp per key channel j, lanes over the rank: rows of
+  // U_up read contiguously), b = sigmoid(b_x + p), b k
+  for (int j = warp; j < DK; j += kDecWarps) {
     float p = 0.f;
-    for (int r = 0; r < R; ++r) p = fmaf(ldf(s_uu, j * R + r), s_h[r], p);
-    const float bj = 1.0f / (1.0f + expf(-(s_bx[j] + p)));
-    s_kp[j] = bj * s_k[j];
+    for (int r = lane; r < R; r += 32) p = fmaf(ldf(s_uu, j * R + r), s_h[r], p);
+    p = allsum(p);
+    if (lane == 0) {
+      const float bj = 1.0f / (1.0f + expf(-(s_bx[j] + p)));
+      s_kp[j] = bj * s_k[j];
+    }
   }
   __syncthreads();
 
@@ -225,7 +231,7 @@ __global__ void __launch_bounds__(kDecThreads)
         }
         if (lane == r) {  // spread the per-row scalars over the warp's lanes
           stf(o, row, ov);
-          const float os = osum[row] + ov;
+          const float os = osv + ov;
           if (chunk_end) {
             m[row] = os * invL;
             osum[row] = 0.f;

@@ -93,7 +93,7 @@ constexpr int B_M2 = 3;    // MMA 2 (W^T [M;P_k]^T)
 constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
 constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
 constexpr int B_X = 6;     // dv = 256: the other CTA's half of U_down m arrived
-constexpr int B_WK = 7;    // S += W^T K^ (issued with MMA 2)
+constexpr int B_WK = 7;    // S += W^T K^ (thread 0, step 3)
 constexpr int B_TEST = 8;  // test only: the redirected commit of a stalled block
 constexpr int B_FIN = 9;   // an aborting CTA: thread 0's D1 MMAs not yet committed
 constexpr int B_GM = 10;   // [M; P_k] (thread 32, step 2)
@@ -545,6 +545,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(bars + bm);
       mark(bm);
       d1_open = false;
+      // the E-independent half of MMA 4, S += W^T K^ (W and K^ are final);
+      // its completion frees K^'s slot for the next block's key transform,
+      // which waits on B_WK; MMA 4 and the S update come later from this
+      // same thread, whose commit of MMA 3b / 4 covers it
+      const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KHP);
+#pragma unroll 1
+      for (int ks = 0; ks < 4; ++ks)
+        umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
+                  desc_mnmajor_sw128(kh0 + ks * 2048, 16384), ID_AMN_BMN, 1);
+      umma_commit(bars + B_WK);
+      // this thread never waits on B_WK: it tracks the parity of the phase
+      // it just started so that an aborting CTA drains it
+      npar = (npar & ~(1u << B_WK)) | ((uint32_t)(ib & 1) << B_WK);
+      mark(B_WK);
     }
     wait(B_M1, 3);
     tc_fence_after();
@@ -579,19 +593,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       bar_named(2, 128);
       unit_lower_inverse64(s_af, s_tf, s_tf + 4096, 2);
       wait(B_M2, 5);  // [M; P_k] consumed: T may take its place
-      if (row < 64) {
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
-          float vals[32];
+      {  // T -> bf16 operand: a half row (32 columns) per thread of warps 0-3
+        const int tr = tid & 63, part = tid >> 6;
+        float vals[32];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 x = *reinterpret_cast<const float4*>(s_tf + fsw(row, part * 32 + e));
-            vals[e] = x.x; vals[e + 1] = x.y; vals[e + 2] = x.z; vals[e + 3] = x.w;
-          }
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8)
-            st_chunk(sm + OFF_MY + sw128_chunk(row, 0, part * 4 + c8, 64), vals + c8 * 8);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 x = *reinterpret_cast<const float4*>(s_tf + fsw(tr, part * 32 + e));
+          vals[e] = x.x; vals[e + 1] = x.y; vals[e + 2] = x.z; vals[e + 3] = x.w;
         }
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_MY + sw128_chunk(tr, 0, part * 4 + c8, 64), vals + c8 * 8);
       }
     } else if (gp <= 2) {
       // ---- 4b. [M; P_k] (strictly lower, 32 columns per group) -> bf16
@@ -622,15 +634,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                     desc_kmajor_sw128(my0 + ks * 32), ID_AMN, 1);
         umma_commit(bars + B_M2);
         mark(B_M2);
-        // the E-independent half of MMA 4, S += W^T K^, off the critical
-        // path (TM_S is next read after MMA 4)
-        const uint32_t kh0 = smem_u32(sm + OFF_KHP);
-#pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks)
-          umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
-                    desc_mnmajor_sw128(kh0 + ks * 2048, 16384), ID_AMN_BMN, 1);
-        umma_commit(bars + B_WK);
-        mark(B_WK);
       }
       wait(B_M2, 4);  // [M; P_k] consumed, R^T complete
       tc_fence_after();
@@ -739,7 +742,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      was added with MMA 2).  Meanwhile warps 8-15: the block's sum of
     //      o and, at a chunk's end, its mean m_{c+1} and the next chunk's
     //      gate p = U_up U_down m_{c+1}
-    if (warp < 8) wait(B_WK, 11);
     if (warp >= 8) {
       const int u = tid - 256;
       if (u < 128) {
