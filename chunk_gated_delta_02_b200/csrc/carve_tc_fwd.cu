@@ -127,10 +127,12 @@ static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* kh,
 }
 
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
-// rows 32 qd .. 32 qd + 31) and column group gp = w / 4.  Warps 0-3 also
-// run the triangular solve while warps 4-11 prepare [M; P_k] and R^T and
-// warps 8-15 then run the next block's key-side transform; at the top of a
-// block warps 8-15 form the gate while warps 0-7 form W.
+// rows 32 qd .. 32 qd + 31) and column group gp = w / 4.  Thread 0 issues
+// D1, the gate Grams, S += W^T K^ and MMAs 3a, 3b, 4; thread 32 the
+// b-independent Grams; thread 128 MMA 2.  Warps 0-3 run the triangular
+// solve while warps 4-7 prepare [M; P_k], R^T and the chunk-mean pieces and
+// warps 8-15 run the next block's key-side transform; after MMA 3a warps
+// 8-15 form the chunk mean and the next chunk's gate.
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -362,8 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // key side of block nb's transform (warps 8-15): K~, Q~ in place in X,
   // K^ into its operand slot (rows 0..63 of KHP), gamma into its parity's
   // buffer; with the fused normalisation, q and k divided by their norms
-  // first (the exchange buffer is in rows of MY that hold nothing while
-  // the key transform runs: [M; P_k] was read by MMA 2, T takes rows 0..63)
+  // first (exchanged through the scan buffer)
   auto keys = [&](int nb) {
     wait(B_VGB, 1);
     wait(B_KQ, 2);
@@ -385,8 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bar_named(5, 256);
     }
     keys_w8(sm + OFF_X, sm + OFF_KHP, sm + OFF_RG, (nb & 1) ? s_gam1 : s_gam0,
-            s_red, a.dscale, cb,
-            a.qknorm ? reinterpret_cast<float*>(sm + OFF_MY + 12288) : nullptr);
+            s_red, a.dscale, cb, a.qknorm ? s_red : nullptr);
   };
 
   // ---- initial state: S0 -> TMEM (fp32) and the bf16 operand copy
@@ -605,13 +605,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c8 = 0; c8 < 4; ++c8)
           st_chunk(sm + OFF_MY + sw128_chunk(tr, 0, part * 4 + c8, 64), vals + c8 * 8);
       }
-    } else if (gp <= 2) {
-      // ---- 4b. [M; P_k] (strictly lower, 32 columns per group) -> bf16
-      //          operand; MMA 2; R^T -> bf16 operand (warps 4-11)
-      const int part = gp - 1;
+    } else if (gp == 1) {
+      // ---- 4b. warps 4-7 (their results are needed only after the solve):
+      //          [M; P_k] (strictly lower) -> bf16 operand; MMA 2; R^T ->
+      //          bf16 operand; the pieces of the chunk mean
       wait(B_GM, 13);  // [M; P_k], issued by thread 32 in step 2
       tc_fence_after();
-      {
+#pragma unroll 1
+      for (int part = 0; part < 2; ++part) {
         float vals[32];
         tmem_ld32(tl + TM_GM + part * 32, vals);
 #pragma unroll
@@ -624,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_async_smem();
       tc_fence_before();
-      bar_named(1, 256);
+      bar_named(1, 128);
       if (tid == 128 && !*s_abort) {
         tc_fence_after();
         const uint32_t w0 = smem_u32(sm + OFF_W), my0 = smem_u32(sm + OFF_MY);
@@ -637,35 +638,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait(B_M2, 4);  // [M; P_k] consumed, R^T complete
       tc_fence_after();
-      {
+#pragma unroll 1
+      for (int part = 0; part < 2; ++part) {
         float vals[32];
         tmem_ld32(tl + TM_D1 + part * 32, vals);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8)
           st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
                    vals + c8 * 8);
-      }
-      // the chunk mean without waiting for O: with u_i = sum_t P_kap[t][i],
-      // sum_t o_t = sum_t (Q~ S^T + P_k W)[t] - E^T u.  This group's half of
-      // the tokens of the first term, and (warps of lanes 64..127, the
-      // P_kap rows) its half of the columns of u
-      {
-        float vals[32];
+        // the chunk mean without waiting for O: with u_i = sum_t P_kap[t][i],
+        // sum_t o_t = sum_t (Q~ S^T + P_k W)[t] - E^T u.  Half of the tokens
+        // of the first term, and (warps of lanes 64..127, the P_kap rows)
+        // half of the columns of u
         tmem_ld32(tl + TM_D1 + 64 + part * 32, vals);
         float sum = 0.f;
 #pragma unroll
         for (int e = 0; e < 32; ++e) sum += vals[e];
         s_co[part * 128 + row] = sum;
-      }
-      if (qd >= 2) {
-        float vals[32];
-        tmem_ld32(tl + TM_GK + part * 32, vals);
+        if (qd >= 2) {
+          tmem_ld32(tl + TM_GK + part * 32, vals);
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (part * 32 + e >= gr) vals[e] = 0.f;  // strictly lower
-        s_u2[(qd - 2) * 64 + part * 32 + lane] = tc::warp_reduce_scatter32(vals, lane);
+          for (int e = 0; e < 32; ++e)
+            if (part * 32 + e >= gr) vals[e] = 0.f;  // strictly lower
+          s_u2[(qd - 2) * 64 + part * 32 + lane] = tc::warp_reduce_scatter32(vals, lane);
+        }
       }
-    } else if (a.gin && ib % bpc == 0) {
+    } else if (gp == 3 && a.gin && ib % bpc == 0) {
       // warps 12-15: the chunk's gate records for the backward (p_c, h_c,
       // m_c: s_p, s_h, s_m hold them until the chunk's end)
       const int u = tid - 384, c = ib / bpc;
@@ -677,7 +675,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     //          next block's transform (X is free; K^'s slot once S += W^T K^
     //          has read it)
     if (warp >= 8) {
+      // X and K^'s slot are free once S += W^T K^ (thread 0; its commit
+      // follows the gate Grams and D1) and [M; P_k] (thread 32's own
+      // commit) have read them
       wait(B_WK, 12);
+      wait(B_GM, 14);
       if (ib + 1 < NB) keys(ib + 1);
     }
     fence_async_smem();

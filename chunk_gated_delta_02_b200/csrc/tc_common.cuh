@@ -230,8 +230,9 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
   // over the 128 channels.  Each thread sums the squares of its 8 channels
   // of its TPT tokens, the 8 lanes of a token reduce by shuffles, and the
   // two column blocks' warps exchange their halves through nrm
-  // ([2 blocks][64 tokens][k, q] floats) across named barrier bar_id + 4
-  // of the NW warps.  Zero rows (padding) get 0, not inf.
+  // ([2 blocks][64 tokens][k, q] floats, 1 KB; it may alias `red`, which
+  // the scan below reuses after a second barrier) across named barrier
+  // bar_id + 4 of the NW warps.  Zero rows (padding) get 0, not inf.
   float ink[TPT], inq[TPT];
 #pragma unroll
   for (int i = 0; i < TPT; ++i) ink[i] = inq[i] = 1.f;
@@ -268,6 +269,7 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
       ink[i] = tk > 0.f ? 1.0f / sqrtf(tk) : 0.f;
       inq[i] = tq > 0.f ? 1.0f / sqrtf(tq) : 0.f;
     }
+    bar_named(bar_id + 4, NW * 32);  // nrm may be the scan buffer `red`
   }
   float gl[TPT][8];  // inclusive log-decay sums inside the token group
 #pragma unroll
