@@ -93,7 +93,7 @@ constexpr int B_M2 = 3;    // MMA 2 (W^T [M;P_k]^T)
 constexpr int B_M3 = 4;    // MMA 3a (R^T T^T)
 constexpr int B_M4 = 5;    // MMA 3b + 4 (outputs, state update)
 constexpr int B_X = 6;     // dv = 256: the other CTA's half of U_down m arrived
-constexpr int B_WK = 7;    // S += W^T K^ (thread 0, step 3)
+constexpr int B_WK = 7;    // S += W^T K^ (thread 256, step 3)
 constexpr int B_TEST = 8;  // test only: the redirected commit of a stalled block
 constexpr int B_FIN = 9;   // an aborting CTA: thread 0's D1 MMAs not yet committed
 constexpr int B_GM = 10;   // [M; P_k] (thread 32, step 2)
@@ -128,8 +128,8 @@ static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* kh,
 
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or Gram
 // rows 32 qd .. 32 qd + 31) and column group gp = w / 4.  Thread 0 issues
-// D1, the gate Grams, S += W^T K^ and MMAs 3a, 3b, 4; thread 32 the
-// b-independent Grams; thread 128 MMA 2.  Warps 0-3 run the triangular
+// D1, the gate Grams and MMAs 3a, 3b, 4; thread 32 the b-independent
+// Grams; thread 128 MMA 2; thread 256 S += W^T K^.  Warps 0-3 run the triangular
 // solve while warps 4-7 prepare [M; P_k], R^T and the chunk-mean pieces and
 // warps 8-15 run the next block's key-side transform; after MMA 3a warps
 // 8-15 form the chunk mean and the next chunk's gate.
@@ -545,25 +545,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       umma_commit(bars + bm);
       mark(bm);
       d1_open = false;
-      // the E-independent half of MMA 4, S += W^T K^ (W and K^ are final);
-      // its completion frees K^'s slot for the next block's key transform,
-      // which waits on B_WK; MMA 4 and the S update come later from this
-      // same thread, whose commit of MMA 3b / 4 covers it
+    }
+    wait(B_M1, 3);
+    tc_fence_after();
+    // MMA 1 retired: X takes the next block's k, q; and thread 256 (a
+    // warp that waits for it next) issues the E-independent half of MMA 4,
+    // S += W^T K^, whose completion frees K^'s slot for the next block's
+    // key transform (issued after the gate Grams so as not to delay A)
+    if (tid == 256 && !*s_abort) {
+      if (ib + 1 < NB) issue_kq(ib + 1);
+      tc_fence_after();
       const uint32_t w0 = smem_u32(sm + OFF_W), kh0 = smem_u32(sm + OFF_KHP);
 #pragma unroll 1
       for (int ks = 0; ks < 4; ++ks)
         umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
                   desc_mnmajor_sw128(kh0 + ks * 2048, 16384), ID_AMN_BMN, 1);
       umma_commit(bars + B_WK);
-      // this thread never waits on B_WK: it tracks the parity of the phase
-      // it just started so that an aborting CTA drains it
-      npar = (npar & ~(1u << B_WK)) | ((uint32_t)(ib & 1) << B_WK);
       mark(B_WK);
     }
-    wait(B_M1, 3);
-    tc_fence_after();
-    // MMA 1 retired: X takes the next block's k, q
-    if (tid == 256 && ib + 1 < NB && !*s_abort) issue_kq(ib + 1);
 
     const int gr = row < 64 ? row : row - 64;  // token index of Gram row `row`
     // the bf16 S copy is dead until step 7: its buffer holds T (fp32),
@@ -741,9 +740,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (__syncthreads_or(*s_abort)) break;
 
     // ---- 6. MMA 3b: O^T -= E^T P_kap^T ; MMA 4: S -= E^T kap^ (W^T K^
-    //      was added with MMA 2).  Meanwhile warps 8-15: the block's sum of
+    //      was added in step 3).  Meanwhile warps 8-15: the block's sum of
     //      o and, at a chunk's end, its mean m_{c+1} and the next chunk's
     //      gate p = U_up U_down m_{c+1}
+    if (warp < 8) wait(B_WK, 11);  // S += W^T K^ (thread 256) before MMA 4
     if (warp >= 8) {
       const int u = tid - 256;
       if (u < 128) {
