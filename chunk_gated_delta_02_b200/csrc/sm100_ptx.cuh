@@ -53,6 +53,17 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map,
       "r"(smem_u32(bar))
       : "memory");
 }
+// Shared -> global copy of a 3-D tile (bulk group; the tensor map's box and
+// swizzle give the shared-memory layout); rows past the tensor are clipped.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map,
+                                             const void* src, int c0, int c1,
+                                             int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, "
+      "%4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
 // Prefetch a 3-D tile (same box as the loads) into L2 only.
 __device__ __forceinline__ void tma_prefetch_3d(const CUtensorMap* map, int c0,
                                                 int c1, int c2) {

@@ -568,8 +568,9 @@ __device__ __forceinline__ void tile_st(float* Z, int zr, int zc,
 // (3) run on the warp-level tensor cores (tf32 in, fp32 out; T is rounded to
 // bf16 by its users).  Called by warps 0..3 only (128 threads, named barrier
 // `bar_id`); the other warps of the CTA are free meanwhile.  T (layout fsw)
-// goes to `tf`; `ws` is >= 2048 floats of scratch.  Ends with that named
-// barrier.
+// goes to `tf`, which may be `af` (in place: each block of A is read before
+// the block of T in its place is written); `ws` is >= 2048 floats of
+// scratch.  Ends with that named barrier.
 static __device__ __noinline__ void unit_lower_inverse64(const float* af, float* tf,
                                                   float* ws, int bar_id) {
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -583,10 +584,11 @@ static __device__ __noinline__ void unit_lower_inverse64(const float* af, float*
     *reinterpret_cast<float4*>(tf + fsw(16 * bi + r, 16 * bj + c4)) =
         make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  // (1) diagonal blocks
+  // (1) diagonal blocks (every read of A's diagonal blocks precedes the
+  // barrier before the stores, so `tf` may be `af`)
+  const int o = 16 * (tid >> 4), j = tid & 15;
+  float t[16];
   if (tid < 64) {
-    const int o = 16 * (tid >> 4), j = tid & 15;
-    float t[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       float acc = 0.f;
@@ -604,6 +606,9 @@ static __device__ __noinline__ void unit_lower_inverse64(const float* af, float*
       }
       t[i] = i < j ? 0.f : (i == j ? 1.f : -acc);
     }
+  }
+  bar_named(bar_id, 128);
+  if (tid < 64) {
 #pragma unroll
     for (int i = 0; i < 16; ++i) tf[fsw(o + i, o + j)] = t[i];
   }
@@ -615,6 +620,7 @@ static __device__ __noinline__ void unit_lower_inverse64(const float* af, float*
 #pragma unroll
     for (int i = 0; i < 8; ++i) acc[i] = acc2[i] = 0.f;
     tile_mac<false, false, 1>(acc, af, o1, o0, tf, o0, o0);
+    __syncwarp();  // A_10 read by every lane before its place takes A_10 T_00
     tile_st<false>(tf, o1, o0, acc, 1.f);
     __syncwarp();
     tile_mac<false, false, 1>(acc2, tf, o1, o1, tf, o1, o0);
