@@ -524,6 +524,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool more = ib + 1 < NB;
     float* s_gam = (ib & 1) ? s_gam1 : s_gam0;  // this block's gamma
     const int gr = row < 64 ? row : row - 64;  // token index of Gram row `row`
+    // token-axis products: K-steps of 16 over the block's C rows only (the
+    // rows past C of every token operand are zero)
+    const int nks = C >> 4;
 
     if (warp < 4) {
       // ================= S: warps 0-3 =================
@@ -554,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       bar_named(2, 128);
       // ---- S2. T = (I + A)^{-1} in place
-      unit_lower_inverse64(s_af, s_af, reinterpret_cast<float*>(sm + OFF_WS), 2);
+      unit_lower_inverse64(s_af, s_af, reinterpret_cast<float*>(sm + OFF_WS), 2, nks);
       wait(B_M2, 5);  // MMA 2 read [M; P_k]: T takes its rows of MY
       {  // T -> bf16 operand (and the record): a half row per thread
         const int tr = tid & 63, part = tid >> 6;
@@ -581,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t re0 = smem_u32(sm + OFF_RE), my0 = smem_u32(sm + OFF_MY);
 #pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks) {
+        for (int ks = 0; ks < nks; ++ks) {
           umma_bf16(tmem + TM_D1, desc_kmajor_sw128(re0 + ks * 32),
                     desc_kmajor_sw128(my0 + ks * 32), ID_N64, ks > 0);
           if (rec)
@@ -621,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kp0 = smem_u32(sm + OFF_KHP) + 8192;
         const uint32_t re0 = smem_u32(sm + OFF_RE), pq0 = smem_u32(sm + OFF_PQ);
 #pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks) {
+        for (int ks = 0; ks < nks; ++ks) {
           umma_bf16(tmem + TM_D1 + 64, desc_kmajor_sw128(re0 + ks * 32),
                     desc_kmajor_sw128(pq0 + ks * 32), ID_N64_NA, 1);
           umma_bf16(tmem + TM_S, desc_kmajor_sw128(re0 + ks * 32),
@@ -739,7 +742,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t w0 = smem_u32(sm + OFF_RV), my0 = smem_u32(sm + OFF_MY);
 #pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks)
+        for (int ks = 0; ks < nks; ++ks)
           umma_bf16(tmem + TM_D1, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
                     desc_kmajor_sw128(my0 + ks * 32), ID_AMN, 1);
         umma_commit(bars + B_M2);
@@ -876,7 +879,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t w0 = smem_u32(sm + OFF_RV), kh0 = smem_u32(sm + OFF_KHP);
 #pragma unroll 1
-        for (int ks = 0; ks < 4; ++ks)
+        for (int ks = 0; ks < nks; ++ks)
           umma_bf16(tmem + TM_S, desc_mnmajor_sw128(w0 + ks * 2048, 8192),
                     desc_mnmajor_sw128(kh0 + ks * 2048, 16384), ID_AMN_BMN, 1);
         umma_commit(bars + B_WK);

@@ -570,9 +570,12 @@ __device__ __forceinline__ void tile_st(float* Z, int zr, int zc,
 // `bar_id`); the other warps of the CTA are free meanwhile.  T (layout fsw)
 // goes to `tf`, which may be `af` (in place: each block of A is read before
 // the block of T in its place is written); `ws` is >= 2048 floats of
-// scratch.  Ends with that named barrier.
+// scratch.  With nblk < 4 the rows (and columns) past 16 nblk of A are zero,
+// so T is I there and block merges reaching only those rows are skipped.
+// Ends with that named barrier.
 static __device__ __noinline__ void unit_lower_inverse64(const float* af, float* tf,
-                                                  float* ws, int bar_id) {
+                                                  float* ws, int bar_id,
+                                                  int nblk = 4) {
   const int tid = threadIdx.x, warp = tid >> 5;
   // zero blocks above the diagonal (6 blocks, 3 float4 per thread)
 #pragma unroll
@@ -613,6 +616,9 @@ static __device__ __noinline__ void unit_lower_inverse64(const float* af, float*
     for (int i = 0; i < 16; ++i) tf[fsw(o + i, o + j)] = t[i];
   }
   bar_named(bar_id, 128);
+  // rows past 16 nblk are zero (padding tokens): T is I there and the
+  // merges that only reach those rows are skipped (nblk is uniform)
+  if (nblk <= 1) return;
   // (2) T_10 = -T_11 (A_10 T_00) for the block pairs (0, 1) and (2, 3)
   if (warp < 2) {
     const int o0 = 32 * warp, o1 = o0 + 16;
@@ -628,6 +634,7 @@ static __device__ __noinline__ void unit_lower_inverse64(const float* af, float*
     tile_st<false>(tf, o1, o0, acc2, -1.f);
   }
   bar_named(bar_id, 128);
+  if (nblk <= 2) return;
   // (3) T_BA = -T_B (A_BA T_A): output tile (I, J), I = 2, 3, J = 0, 1
   const int I = 2 + (warp >> 1), J = warp & 1;
   {
