@@ -13,18 +13,24 @@
 //
 // Memory-bound: every step reads and writes the fp32 state once.  Each value
 // row of S is independent once the key-side vectors (q, exp g, k, b k) are
-// known, so one CTA per (sequence, head) forms those vectors and the gate,
-// and its warps stream the rows: a warp holds a batch of rows in registers
-// (each row read as coalesced 128-byte segments), reduces S q and S' k with
-// butterfly shuffles, and writes the new row back.
+// known, so a (sequence, head) pair runs as a cluster of kSplit CTAs, each
+// owning a quarter of the value rows: every CTA forms the key-side vectors
+// and the gate itself (they are small), and its warps stream their rows: a
+// warp holds a batch of rows in registers (each row read as coalesced
+// 128-byte segments), reduces S q and S' k with butterfly shuffles, and
+// writes the new row back.  The gate of every CTA reads all of m_c, which a
+// chunk's last token rewrites row by row, so the CTAs of a cluster meet
+// once after staging m_c and before any of them can write it.
 #include <cuda_bf16.h>
 
 #include "carve_internal.cuh"
+#include "sm100_ptx.cuh"
 
 namespace carve {
 namespace {
 
-constexpr int kDecThreads = 512;   // 16 warps
+constexpr int kDecThreads = 128;   // 4 warps per CTA
+constexpr int kSplit = 4;          // CTAs (a cluster) per (sequence, head)
 constexpr int kDecWarps = kDecThreads / 32;
 constexpr int kRows = 8;           // value rows a warp holds at once (DK <= 128)
 
@@ -59,19 +65,6 @@ struct Vec<float> {
   }
 };
 
-// Copies n elements (a multiple of the vector width, 16-byte aligned) of
-// the I/O dtype into fp32 shared memory with 16-byte loads.
-template <typename TIn>
-__device__ __forceinline__ void stage(float* dst, const TIn* src, int n) {
-  constexpr int N = Vec<TIn>::N;
-  for (int i = threadIdx.x * N; i < n; i += kDecThreads * N) {
-    float x[N];
-    Vec<TIn>::load(src + i, x);
-#pragma unroll
-    for (int e = 0; e < N; ++e) dst[i + e] = x[e];
-  }
-}
-
 // NJ = columns per lane (DK <= 32 NJ)
 template <typename TIn, int NJ>
 __global__ void __launch_bounds__(kDecThreads)
@@ -86,15 +79,23 @@ __global__ void __launch_bounds__(kDecThreads)
   float* s_m = s_bx + DK;       // m_c          [DV]
   float* s_v = s_m + DV;        // v            [DV]
   float* s_h = s_v + DV;        // U_down m_c   [R]
-  // the head's U_b factors in the I/O dtype: U_down [R][DV], U_up [DK][R]
+  // the head's U_b factors in the I/O dtype, as stored: U_down [R][DV],
+  // U_up [DK][R]
   TIn* s_ud = reinterpret_cast<TIn*>(
       (reinterpret_cast<uintptr_t>(s_h + (R > 0 ? R : 1)) + 15) & ~uintptr_t(15));
   TIn* s_uu = s_ud + R * DV;
-  const int pair = blockIdx.x;
+  // raw copies of the token's vectors and m_c (16-byte aligned): q, k, g,
+  // b_x [DK], v [DV] in the I/O dtype, then m_c [DV] fp32
+  TIn* s_raw = s_uu + DK * R;
+  float* s_mraw = reinterpret_cast<float*>(s_raw + 4 * DK + DV);
+  const int pair = blockIdx.x / kSplit, part = blockIdx.x % kSplit;
   const int bseq = pair / a.H, h = pair - bseq * a.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* S = a.S + (size_t)pair * DV * DK;
   constexpr int RW = NJ > 4 ? kRows / 2 : kRows;  // rows per batch in registers
+  // this CTA's value rows [rlo, rhi)
+  const int rq = (DV + kSplit - 1) / kSplit;
+  const int rlo = part * rq, rhi = min(DV, rlo + rq);
 
   // the first batch of this warp's state rows: requested before anything
   // else, so that the gate below runs while they are in flight
@@ -107,11 +108,11 @@ __global__ void __launch_bounds__(kDecThreads)
 #pragma unroll
       for (int c = 0; c < NJ; ++c) {
         const int j = lane + 32 * c;
-        sv[r][c] = (r0 + r < DV && j < DK) ? S[(size_t)(r0 + r) * DK + j] : 0.f;
+        sv[r][c] = (r0 + r < rhi && j < DK) ? S[(size_t)(r0 + r) * DK + j] : 0.f;
       }
-    osv = (lane < RW && r0 + lane < DV) ? osum[r0 + lane] : 0.f;
+    osv = (lane < RW && r0 + lane < rhi) ? osum[r0 + lane] : 0.f;
   };
-  load_rows(warp * RW);
+  load_rows(rlo + warp * RW);
 
   const TIn* q = static_cast<const TIn*>(a.q) + (size_t)pair * DK;
   const TIn* k = static_cast<const TIn*>(a.k) + (size_t)pair * DK;
@@ -123,25 +124,51 @@ __global__ void __launch_bounds__(kDecThreads)
   const float w = ldf(static_cast<const TIn*>(a.w), pair);
   const bool chunk_end = (a.pos[bseq] + 1) % a.L == 0;
 
-  // the token's vectors, m_c and the head's U_b factors -> shared memory
-  // (16-byte loads; DK, DV and R * DV, DK * R are multiples of 8)
-  stage(s_q, q, DK);
-  stage(s_k, k, DK);
-  stage(s_al, g, DK);
-  stage(s_bx, bx, DK);
-  stage(s_v, v, DV);
-  for (int i = tid * 4; i < DV; i += kDecThreads * 4)
-    *reinterpret_cast<float4*>(s_m + i) = *reinterpret_cast<const float4*>(m + i);
-  if (R > 0) {  // raw 16-byte copies (R * DV and DK * R bytes are multiples of 16)
-    const uint4* ud4 = reinterpret_cast<const uint4*>(
+  // the head's U_b factors -> shared memory by asynchronous 16-byte copies
+  // (R * DV and DK * R elements fill whole 16-byte chunks: DK, DV are
+  // multiples of 16), in flight with the state rows; then the token's
+  // vectors and m_c
+  if (R > 0) {
+    const uint8_t* udg = reinterpret_cast<const uint8_t*>(
         static_cast<const TIn*>(a.u_down) + (size_t)h * R * DV);
-    const uint4* uu4 = reinterpret_cast<const uint4*>(
+    const uint8_t* uug = reinterpret_cast<const uint8_t*>(
         static_cast<const TIn*>(a.u_up) + (size_t)h * DK * R);
     const int nd = R * DV * (int)sizeof(TIn) / 16, nu = DK * R * (int)sizeof(TIn) / 16;
-    for (int i = tid; i < nd; i += kDecThreads) reinterpret_cast<uint4*>(s_ud)[i] = ud4[i];
-    for (int i = tid; i < nu; i += kDecThreads) reinterpret_cast<uint4*>(s_uu)[i] = uu4[i];
+    for (int i = tid; i < nd; i += kDecThreads)
+      ptx::cp_async16(reinterpret_cast<uint8_t*>(s_ud) + 16 * i, udg + 16 * i);
+    for (int i = tid; i < nu; i += kDecThreads)
+      ptx::cp_async16(reinterpret_cast<uint8_t*>(s_uu) + 16 * i, uug + 16 * i);
+  }
+  {  // every 16-byte chunk of the vectors and of m_c in one batch of copies
+    const int cv = DK * (int)sizeof(TIn) / 16, cw = DV * (int)sizeof(TIn) / 16;
+    const int nc = 4 * cv + cw + DV / 4;
+    for (int i = tid; i < nc; i += kDecThreads) {
+      const int which = i < 4 * cv ? i / cv : (i < 4 * cv + cw ? 4 : 5);
+      const int ci = which < 4 ? i - which * cv : (which == 4 ? i - 4 * cv : i - 4 * cv - cw);
+      const void* src = which == 0 ? (const void*)q : which == 1 ? (const void*)k
+                      : which == 2 ? (const void*)g : which == 3 ? (const void*)bx
+                      : which == 4 ? (const void*)v : (const void*)m;
+      uint8_t* dst = which < 5 ? reinterpret_cast<uint8_t*>(s_raw + which * DK)
+                               : reinterpret_cast<uint8_t*>(s_mraw);
+      ptx::cp_async16(dst + 16 * ci, static_cast<const uint8_t*>(src) + 16 * ci);
+    }
+    ptx::cp_async_commit();
+  }
+  ptx::cp_async_wait_all();
+  __syncthreads();
+  for (int j = tid; j < DK; j += kDecThreads) {
+    s_q[j] = ldf(s_raw, j);
+    s_k[j] = ldf(s_raw + DK, j);
+    s_al[j] = ldf(s_raw + 2 * DK, j);
+    s_bx[j] = ldf(s_raw + 3 * DK, j);
+  }
+  for (int i = tid; i < DV; i += kDecThreads) {
+    s_v[i] = ldf(s_raw + 4 * DK, i);
+    s_m[i] = s_mraw[i];
   }
   __syncthreads();
+  // every CTA of the pair has m_c: a chunk's last token may now rewrite it
+  ptx::cluster_sync();
   if (a.qknorm) {  // fused normalisation: q / |q|, k / |k| (warp 0 reduces)
     if (warp == 0) {
       float sq = 0.f, sk = 0.f;
@@ -166,24 +193,51 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   for (int j = tid; j < DK; j += kDecThreads)
     s_al[j] = expf(decay_act(s_al[j], a.dscale));
-  // h = U_down m_c: one warp per rank
-  for (int r = warp; r < R; r += kDecWarps) {
+  // h = U_down m_c: four threads per rank, each over a quarter of the
+  // values (every thread takes every pass, so that the whole warp meets the
+  // shuffles; ranks past R add nothing)
+  for (int base = 0; base < R; base += kDecThreads / 4) {
+    const int r = base + (tid >> 2), q4 = tid & 3;
     float acc = 0.f;
-    for (int i = lane; i < DV; i += 32) acc = fmaf(ldf(s_ud, r * DV + i), s_m[i], acc);
-    acc = allsum(acc);
-    if (lane == 0) s_h[r] = acc;
+    if (r < R) {  // a contiguous quarter of the row, 16-byte vectors
+      constexpr int VN = Vec<TIn>::N;
+      const int i0 = q4 * (DV / 4), i1 = i0 + DV / 4;
+      float a4[4] = {0.f, 0.f, 0.f, 0.f};
+      if ((DV / 4) % VN == 0) {
+        for (int i = i0; i < i1; i += VN) {
+          float u[VN];
+          Vec<TIn>::load(s_ud + (size_t)r * DV + i, u);
+#pragma unroll
+          for (int e = 0; e < VN; ++e) a4[e & 3] = fmaf(u[e], s_m[i + e], a4[e & 3]);
+        }
+      } else {
+        for (int i = i0; i < i1; ++i) a4[0] = fmaf(ldf(s_ud, r * DV + i), s_m[i], a4[0]);
+      }
+      acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    }
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (q4 == 0 && r < R) s_h[r] = acc;
   }
   __syncthreads();
-  // p = U_up h (one warp per key channel j, lanes over the rank: rows of
-  // U_up read contiguously), b = sigmoid(b_x + p), b k
-  for (int j = warp; j < DK; j += kDecWarps) {
-    float p = 0.f;
-    for (int r = lane; r < R; r += 32) p = fmaf(ldf(s_uu, j * R + r), s_h[r], p);
-    p = allsum(p);
-    if (lane == 0) {
-      const float bj = 1.0f / (1.0f + expf(-(s_bx[j] + p)));
-      s_kp[j] = bj * s_k[j];
+  // p = U_up h (a thread per key channel, its row of U_up read as 16-byte
+  // vectors when the row fills whole ones), b = sigmoid(b_x + p), b k
+  constexpr int VN = Vec<TIn>::N;
+  for (int j = tid; j < DK; j += kDecThreads) {
+    float p4[4] = {0.f, 0.f, 0.f, 0.f};
+    if (R % VN == 0) {
+      for (int r = 0; r < R; r += VN) {
+        float u[VN];
+        Vec<TIn>::load(s_uu + (size_t)j * R + r, u);
+#pragma unroll
+        for (int e = 0; e < VN; ++e) p4[e & 3] = fmaf(u[e], s_h[r + e], p4[e & 3]);
+      }
+    } else {
+      for (int r = 0; r < R; ++r) p4[0] = fmaf(ldf(s_uu, j * R + r), s_h[r], p4[0]);
     }
+    const float p = (p4[0] + p4[1]) + (p4[2] + p4[3]);
+    const float bj = 1.0f / (1.0f + expf(-(s_bx[j] + p)));
+    s_kp[j] = bj * s_k[j];
   }
   __syncthreads();
 
@@ -207,8 +261,8 @@ __global__ void __launch_bounds__(kDecThreads)
     ewj[c] = a.erase ? kj[c] : kpj[c];
   }
   const float invL = 1.0f / (float)a.L;
-  for (int r0 = warp * RW; r0 < DV; r0 += kDecWarps * RW) {
-    if (r0 != warp * RW) load_rows(r0);
+  for (int r0 = rlo + warp * RW; r0 < rhi; r0 += kDecWarps * RW) {
+    if (r0 != rlo + warp * RW) load_rows(r0);
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
       const int row = r0 + r;
@@ -221,7 +275,7 @@ __global__ void __launch_bounds__(kDecThreads)
       }
       ov = allsum(ov);
       ev = allsum(ev);
-      if (row < DV) {
+      if (row < rhi) {
         const float wv = w * s_v[row];
 #pragma unroll
         for (int c = 0; c < NJ; ++c) {
@@ -244,28 +298,39 @@ __global__ void __launch_bounds__(kDecThreads)
   }
 }
 
+template <typename TIn, int NJ>
+cudaError_t launch_nj(const DecArgs& a, size_t smem, cudaStream_t st) {
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(
+        decode_kernel<TIn, NJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.B * a.H) * kSplit);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kSplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<TIn, NJ>, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <typename TIn>
 cudaError_t launch_typed(const DecArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)(5 * a.DK + 2 * a.DV + (a.R > 0 ? a.R : 1)) * 4 +
-                      16 + (size_t)a.R * (a.DK + a.DV) * sizeof(TIn);
-  if (smem > 48 * 1024) {
-    cudaError_t e = cudaSuccess;
-    if (a.DK <= 64)
-      e = cudaFuncSetAttribute(decode_kernel<TIn, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    else if (a.DK <= 128)
-      e = cudaFuncSetAttribute(decode_kernel<TIn, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    else
-      e = cudaFuncSetAttribute(decode_kernel<TIn, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
-  const dim3 grid(a.B * a.H), block(kDecThreads);
-  if (a.DK <= 64)
-    decode_kernel<TIn, 2><<<grid, block, smem, st>>>(a);
-  else if (a.DK <= 128)
-    decode_kernel<TIn, 4><<<grid, block, smem, st>>>(a);
-  else
-    decode_kernel<TIn, 8><<<grid, block, smem, st>>>(a);
-  return cudaGetLastError();
+                      16 + (size_t)a.R * (a.DK + a.DV) * sizeof(TIn) +
+                      (size_t)(4 * a.DK + a.DV) * sizeof(TIn) + (size_t)a.DV * 4;
+  if ((long long)a.B * a.H * kSplit > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (a.DK <= 64) return launch_nj<TIn, 2>(a, smem, st);
+  if (a.DK <= 128) return launch_nj<TIn, 4>(a, smem, st);
+  return launch_nj<TIn, 8>(a, smem, st);
 }
 
 }  // namespace
