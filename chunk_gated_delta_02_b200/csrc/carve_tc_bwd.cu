@@ -153,6 +153,9 @@ struct BwdTcArgs {
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or key
 // channels 32 qd .. 32 qd + 31) and column group gp = w / 4, so every
 // element-wise phase is split four ways along the TMEM columns.
+// ACT: the instance for raw decay logits (decay_scale > 0); the other one
+// has no activation code at all
+template <bool ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_tc_kernel(const BwdTcArgs args,
                   const __grid_constant__ CUtensorMap tm_q,
@@ -400,7 +403,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      warps 0-7 by named barrier 7, then W = w V and dO = d_o + dm / L);
     //      s_x is cleared: it accumulates dlog gamma next
     if (warp < 8) {
-      tc::transform_block<8>(sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB,
+      tc::transform_block<8, ACT>(sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB,
                              sm + R_DSB + 16384, s_gam,
                              reinterpret_cast<float*>(sm + R_MP), 3, 16384, 7,
                              kThreads, a.dscale, kBlk);
@@ -773,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         float gsum = 0.f;
 #pragma unroll
         for (int e = 0; e < 16; ++e) gv[e] = ldbf(sm + R_RO + sw128_off(tb + e, jj, 64));
-        if (a.dscale > 0.f) {  // raw decay logits (uniform branch)
+        if constexpr (ACT) {  // raw decay logits
           decay_act8(gv, a.dscale, true);
           decay_act8(gv + 8, a.dscale, true);
         }
@@ -866,19 +869,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         acc += s_lq[g2 * 128 + jj] + (g2 < 3 ? s_qf[(g2 + 1) * 128 + jj] : dlg);
       // with raw decay logits a (decay_scale s > 0) the output is dL/da =
       // dL/dg * s expm1(g / s), formed from the log-decay itself
-      const float dsc = a.dscale;
-      if (dsc > 0.f) {  // uniform branch: dL/dg -> dL/da needs s expm1(g / s)
+      if constexpr (ACT) {  // dL/dg -> dL/da needs s expm1(g / s)
 #pragma unroll
-        for (int i = 0; i < 16; ++i) gv[i] = decay_act_grad(gv[i], dsc);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) gv[i] = 1.f;
+        for (int i = 0; i < 16; ++i) gv[i] = decay_act_grad(gv[i], a.dscale);
       }
       float hg = 0.f;  // the odd token's suffix sum
 #pragma unroll
       for (int i = 15; i >= 0; --i) {
         acc += dGv[i];
-        const float out = acc * gv[i];
+        const float out = ACT ? acc * gv[i] : acc;
         if (i & 1)
           hg = out;
         else
@@ -1088,12 +1087,12 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
       !make_map(&mv, a.v, kDV, a.H, rows) || !make_map(&mg, a.g, kDK, a.H, rows) ||
       !make_map(&mb, a.bx, kDK, a.H, rows) || !make_map(&mdo, a.d_o, kDV, a.H, rows))
     return cudaErrorInvalidValue;
+  auto kern = a.dscale > 0.f ? bwd_tc_kernel<true> : bwd_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(
-      bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   BwdTcArgs args{a, a.scratch};  // gate records live in the scratch area
-  bwd_tc_kernel<<<a.B * a.H, kThreads, kSmemBytes, st>>>(args, mq, mk, mv, mg,
-                                                         mb, mdo);
+  kern<<<a.B * a.H, kThreads, kSmemBytes, st>>>(args, mq, mk, mv, mg, mb, mdo);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.R > 0) {

@@ -124,17 +124,21 @@ constexpr uint32_t ID_BMN_NA = idesc_bf16_neg(128, 128, false, true, true, false
 // Key side of one block's transform by warps 8-15 (one out-of-line copy of
 // the unrolled code serves the prologue and the block loop): K~, Q~ in place
 // in X, K^ straight into rows 0..63 of its operand slot in KHP.
+template <bool ACT>
 static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* kh,
                                             const uint8_t* rg, float* gam,
                                             float* red, float dscale,
                                             int nvalid, float* nrm) {
-  tc::transform_keys<8>(x, kh, rg, gam, red, 3, 16384, 8, dscale, nvalid, nrm);
+  tc::transform_keys<8, ACT>(x, kh, rg, gam, red, 3, 16384, 8, dscale, nvalid, nrm);
 }
 
 // 16 warps in three groups (see the block loop): warp w serves TMEM lane
 // quadrant qd = w % 4 (value rows or Gram rows 32 qd .. 32 qd + 31).  Thread
 // 0 issues MMAs 3a, 3b, 4; thread 128 D1 and MMA 2; thread 256 the copies,
 // S += W^T K^ and the Grams.
+// ACT: the instance for raw decay logits (decay_scale > 0); the other one
+// has no activation code at all
+template <bool ACT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -395,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       bar_named(5, 256);
     }
-    keys_w8(sm + OFF_X, sm + OFF_KHP, sm + OFF_RG, (nb & 1) ? s_gam1 : s_gam0,
+    keys_w8<ACT>(sm + OFF_X, sm + OFF_KHP, sm + OFF_RG, (nb & 1) ? s_gam1 : s_gam0,
             s_red, a.dscale, cb, a.qknorm ? s_red : nullptr);
   };
 
@@ -990,11 +994,12 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
       !make_map(&mv, a.v, a.DV, a.H, rows, C) || !make_map(&mg, a.g, kDK, a.H, rows, C) ||
       !make_map(&mb, a.bx, kDK, a.H, rows, C) || !make_map(&mo, a.o, a.DV, a.H, rows, C))
     return cudaErrorInvalidValue;
+  auto kern = a.dscale > 0.f ? fwd_tc_kernel<true> : fwd_tc_kernel<false>;
   cudaError_t e = cudaFuncSetAttribute(
-      fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+      kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
   if (!dv2) {
-    fwd_tc_kernel<<<a.B * a.H, kThreads, kSmemBytes, st>>>(a, mq, mk, mv, mg, mb, mo);
+    kern<<<a.B * a.H, kThreads, kSmemBytes, st>>>(a, mq, mk, mv, mg, mb, mo);
     return cudaGetLastError();
   }
   // dv = 256: clusters of two CTAs, one per value half
@@ -1010,7 +1015,7 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, fwd_tc_kernel, a, mq, mk, mv, mg, mb, mo);
+  e = cudaLaunchKernelEx(&cfg, kern, a, mq, mk, mv, mg, mb, mo);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

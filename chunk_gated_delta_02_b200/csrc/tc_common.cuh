@@ -102,7 +102,7 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* p, float* x) {
 // The log-decay prefix over the token groups is a shuffle scan inside each
 // warp plus the totals of the preceding warps (named barriers bar_id,
 // bar_id + 1 for the two column blocks).
-template <int NW>
+template <int NW, bool ACT = false>
 __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
                                                 uint8_t* kp,
                                                 const uint8_t* graw,
@@ -132,9 +132,9 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
   for (int i = 0; i < TPT; ++i) {
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
-    // raw decay logits -> log-decay (dscale > 0; rows past the block's
-    // nvalid tokens: 0).  A uniform branch around an out-of-line helper.
-    if (dscale > 0.f) decay_act8(gv, dscale, TPT * tg + i < nvalid);
+    // raw decay logits -> log-decay (ACT: the kernel instance for dscale >
+    // 0; rows past the block's nvalid tokens: 0)
+    if constexpr (ACT) decay_act8(gv, dscale, TPT * tg + i < nvalid);
 #pragma unroll
     for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
   }
@@ -203,7 +203,7 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
 // wbase .. wbase + NW - 1.  With khs = 8192, K^ may overwrite the raw g
 // tile in place (kh == graw): each thread reads all its g chunks before it
 // writes K^ to the same offsets, and no other thread touches them.
-template <int NW>
+template <int NW, bool ACT = false>
 __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
                                                const uint8_t* graw,
                                                float* s_gam, float* red,
@@ -276,9 +276,9 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
   for (int i = 0; i < TPT; ++i) {
     float gv[8];
     ld_chunk(graw + off64(TPT * tg + i), gv);
-    // raw decay logits -> log-decay (dscale > 0; rows past the block's
-    // nvalid tokens: 0).  A uniform branch around an out-of-line helper.
-    if (dscale > 0.f) decay_act8(gv, dscale, TPT * tg + i < nvalid);
+    // raw decay logits -> log-decay (ACT: the kernel instance for dscale >
+    // 0; rows past the block's nvalid tokens: 0)
+    if constexpr (ACT) decay_act8(gv, dscale, TPT * tg + i < nvalid);
 #pragma unroll
     for (int e = 0; e < 8; ++e) gl[i][e] = (i ? gl[i - 1][e] : 0.f) + gv[e];
   }
