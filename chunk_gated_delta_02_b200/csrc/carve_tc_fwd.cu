@@ -637,27 +637,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(bars + B_M4);
         mark(B_M4);
       }
-      if (rec) {
-        // E [t][v] (K-major, the backward's operand layout) -> the A buffer
-        // (T was read from it) -> the record, while MMAs 3b and 4 run
-        if (row < 64) {
-#pragma unroll 1
-          for (int pc = 0; pc < 4; ++pc) {
-            float vals[32];
-            tmem_ld32(tl + TM_E + pc * 32, vals);
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8)
-              st_chunk(sm + OFF_AF + sw128_chunk(row, pc >> 1, (pc & 1) * 4 + c8, 64),
-                       vals + c8 * 8);
-          }
-        }
-        fence_async_smem();
-        bar_named(2, 128);
-        if (tid == 0) {
-          bulk_store(rec + kTcRecE, sm + OFF_AF, 16384);
-          bulk_commit();
-        }
-      }
       wait(B_M4, 8);
       tc_fence_after();
       // ---- S5. outputs o_t (a value row per thread, 64 tokens).  A whole
@@ -719,9 +698,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ================= R: warps 4-7 =================
       // ---- R1. D1 = S [K~; Q~]^T, issued after the Grams (the chain's
       //      next step) have run; [M; P_k] (strictly lower) -> bf16 operand
-      //      in MY (free once the previous block's MMA 3a read T); MMA 2
-      //      (after D1, and once W is formed)
-      if (ib > 0) wait(B_M3, 17);
+      //      in MY (the previous block's MMA 3a, waited for there, read T);
+      //      MMA 2 (after D1, and once W is formed)
       wait(B_GK, 3);
       tc_fence_after();
       if (tid == 128 && !*s_abort) issue_d1();
@@ -785,6 +763,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       bar_arrive_named(11, 256);  // R^T, u -> warps 0-3
       bar_arrive_named(12, 512);  // c_O -> warps 8-15
+      wait(B_M3, 17);  // MMA 3a: MY free for the next block; E formed
+      if (a.tc_rec) {
+        // training: E [t][v] (K-major, the backward's operand layout) ->
+        // the A buffer (T was read from it before MMA 3a) -> the record
+        // (lanes 0-63 of TMEM hold E: warps 4 and 5)
+        if (row < 64) {
+          tc_fence_after();
+#pragma unroll 1
+          for (int pc = 0; pc < 4; ++pc) {
+            float vals[32];
+            tmem_ld32(tl + TM_E + pc * 32, vals);
+#pragma unroll
+            for (int c8 = 0; c8 < 4; ++c8)
+              st_chunk(sm + OFF_AF + sw128_chunk(row, pc >> 1, (pc & 1) * 4 + c8, 64),
+                       vals + c8 * 8);
+          }
+        }
+        fence_async_smem();
+        bar_named(1, 128);
+        if (tid == 128) {
+          bulk_store(a.tc_rec + ((size_t)pair * NB + ib) * kTcRecBytes + kTcRecE,
+                     sm + OFF_AF, 16384);
+          bulk_commit();
+        }
+      }
       // ---- R3. S <- S Diag(gamma) (a value row per thread), its bf16
       //      operand (SB was read by this block's D1) and, in training, the
       //      next block's state record; the final state
@@ -838,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           bulk_commit();
         }
       }
-      if (tid == 128 && a.tc_rec) bulk_wait_read_all();  // SB is rewritten next block
+      if (tid == 128 && a.tc_rec) bulk_wait_read_all();  // SB, the A buffer are rewritten next block
     } else {
       // ================= K: warps 8-15 =================
       const int u = tid - 256;
