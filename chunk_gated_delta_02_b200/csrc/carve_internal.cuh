@@ -36,11 +36,11 @@ constexpr size_t kTcRecT = 49152;      // T    [t 64][s 64]   bf16   8 KB
 constexpr size_t kTcRecBytes = 57344;
 
 // Tensor-core kernels: bf16, DK = DV = 128, L % 64 == 0, R <= 32, T > 0
-// (the training forward, whose records this describes, and the backward).
+// (the training forward, whose records this describes, and the backward;
+// both with or without the fused per-token q / k normalisation).
 inline bool tc_shape(const carve_shape& s) {
   return s.dtype == CARVE_BF16 && s.DK == 128 && s.DV == 128 &&
-         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0 && !s.qk_l2norm &&
-         !s.erase_form;
+         s.L % kMaxBlock == 0 && s.R <= 32 && s.T > 0 && !s.erase_form;
 }
 // The tensor-core forward also runs, without training, DV = 256 (two CTAs
 // per pair) and chunks of 16, 32 or 48 tokens (one chunk per block, the

@@ -68,8 +68,9 @@ constexpr uint32_t SM_DW = 2304;     // dw sums | dh        64 f32
 constexpr uint32_t SM_BAR = 2560;    // kNumBars mbarriers
 constexpr uint32_t SM_TMEM = 2664;
 constexpr uint32_t SM_ABORT = 2668;
+constexpr uint32_t SM_QN = 2688;     // fused q / k norm: inverse norms [t][k, q] fp16, 256 B
 constexpr uint32_t kSmemBytes = 232448;
-static_assert(R_SM + 2688 <= kSmemBytes, "small region");
+static_assert(R_SM + SM_QN + 256 <= kSmemBytes, "small region");
 static_assert(R_PQ == R_MP + 16384 && R_TT == R_PQ + 8192, "G2 blocks");
 
 // mbarriers (index into the small region's array)
@@ -153,9 +154,10 @@ struct BwdTcArgs {
 // 16 warps: warp w serves TMEM lane quadrant qd = w % 4 (value rows or key
 // channels 32 qd .. 32 qd + 31) and column group gp = w / 4, so every
 // element-wise phase is split four ways along the TMEM columns.
-// ACT: the instance for raw decay logits (decay_scale > 0); the other one
-// has no activation code at all
-template <bool ACT>
+// ACT: the instance for raw decay logits (decay_scale > 0); QKN: the one
+// for the fused q / k normalisation.  Instances without them carry none of
+// their code.
+template <bool ACT, bool QKN>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_tc_kernel(const BwdTcArgs args,
                   const __grid_constant__ CUtensorMap tm_q,
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const BwdArgs& a = args.a;
   extern __shared__ __align__(1024) uint8_t sm[];
   float* s_p = reinterpret_cast<float*>(sm + R_SM + SM_P);
+  __half* s_qn = reinterpret_cast<__half*>(sm + R_SM + SM_QN);
   float* s_dmn = reinterpret_cast<float*>(sm + R_SM + SM_DMN);
   float* s_x = reinterpret_cast<float*>(sm + R_SM + SM_X);
   float* s_gam = reinterpret_cast<float*>(sm + R_SM + SM_GAM);
@@ -403,10 +406,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     //      warps 0-7 by named barrier 7, then W = w V and dO = d_o + dm / L);
     //      s_x is cleared: it accumulates dlog gamma next
     if (warp < 8) {
-      tc::transform_block<8, ACT>(sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB,
-                             sm + R_DSB + 16384, s_gam,
-                             reinterpret_cast<float*>(sm + R_MP), 3, 16384, 7,
-                             kThreads, a.dscale, kBlk);
+      tc::transform_block<8, ACT, QKN>(
+          sm + R_X, sm + R_KHP, sm + R_KHP + 8192, sm + R_DSB, sm + R_DSB + 16384,
+          s_gam, reinterpret_cast<float*>(sm + R_MP), 3, 16384, 7, kThreads,
+          a.dscale, kBlk, reinterpret_cast<float*>(sm + R_MP) + 1024, s_qn, 12);
       if (tid < 128) s_x[tid] = 0.f;
     } else {
       const int u = tid - 256;
@@ -807,8 +810,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             base + xp + (size_t)(t_even + (odd ? 1 : 0)) * tstride) = pr;
       };
       float hq = 0.f, hk = 0.f, hz = 0.f;  // the even token's values
+      float igprev = 0.f;                   // 1 / Gamma_{t-1} (QKN only)
+      if constexpr (QKN) igprev = __expf(-G);
 #pragma unroll
       for (int sub = 0; sub < 2; ++sub) {
+        float vq8[8], vk8[8], qh8[8], kh8[8];  // QKN: this sub-block's tokens
         float dd[32];  // dK~ | dQ~ | -dkap^ | dK^ of 8 tokens
         const int tsub = tb + 8 * sub;
         tmem_ld8x4(tl + T_G + tsub, tl + T_G + 64 + tsub, tl + T_D8 + tsub,
@@ -829,11 +835,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float vq = dQt * gprev;
           const float vk = fmaf(dKt, gam, fmaf(dKp, bb, dKh) * igam);
           const float dz = dKp * kh * bb * (1.f - bb);
+          if constexpr (QKN) {
+            // the gradients of the unit q^, k^ (q^ = Q~ / Gamma_{t-1},
+            // k^ = K^ Gamma_t), projected once the block's dots are known
+            vq8[e] = vq;
+            vk8[e] = vk;
+            qh8[e] = qt * igprev;
+            kh8[e] = kh * gam;
+          }
           if ((e & 1) == 0) {
             hq = vq; hk = vk; hz = dz;
           } else {
-            st_pair(dq, t - 1, hq, vq);
-            st_pair(dk, t - 1, hk, vk);
+            if constexpr (!QKN) {
+              st_pair(dq, t - 1, hq, vq);
+              st_pair(dk, t - 1, hk, vk);
+            }
             st_pair(dbx, t - 1, hz, dz);
           }
           dp_acc += dz;
@@ -844,6 +860,41 @@ __global__ void __launch_bounds__(kThreads, 1)
           else
             qfirst = qp;
           gprev = gam;
+          if constexpr (QKN) igprev = igam;
+        }
+        if constexpr (QKN) {
+          // dq = (dq^ - q^ (q^ . dq^)) / |q| and the same for k: the dots
+          // over the 128 channels of each token live on the four warps of
+          // this token quarter (warps 4 gp .. 4 gp + 3, named barrier 8 + gp)
+          float pr[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            pr[e] = vq8[e] * qh8[e];
+            pr[8 + e] = vk8[e] * kh8[e];
+          }
+          const float wsum = warp_reduce_scatter16(pr, lane);
+          float* s_part = s_scr + 1536;  // [4 quarters][4 warps][16]
+          float* s_fin = s_scr + 1792;   // [4 quarters][16]
+          if (lane < 16) s_part[(gp * 4 + qd) * 16 + lane] = wsum;
+          bar_named(8 + gp, 128);
+          if (qd == 0 && lane < 16)
+            s_fin[gp * 16 + lane] =
+                (s_part[(gp * 4) * 16 + lane] + s_part[(gp * 4 + 1) * 16 + lane]) +
+                (s_part[(gp * 4 + 2) * 16 + lane] + s_part[(gp * 4 + 3) * 16 + lane]);
+          bar_named(8 + gp, 128);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int t = tsub + e;
+            const float ink = __half2float(s_qn[t * 2]), inq = __half2float(s_qn[t * 2 + 1]);
+            const float dqr = inq * fmaf(-qh8[e], s_fin[gp * 16 + e], vq8[e]);
+            const float dkr = ink * fmaf(-kh8[e], s_fin[gp * 16 + 8 + e], vk8[e]);
+            if ((e & 1) == 0) {
+              hq = dqr; hk = dkr;
+            } else {
+              st_pair(dq, t - 1, hq, dqr);
+              st_pair(dk, t - 1, hk, dkr);
+            }
+          }
         }
       }
       float lsum = 0.f;
@@ -1087,7 +1138,8 @@ cudaError_t launch_bwd_tc(const BwdArgs& a, cudaStream_t st) {
       !make_map(&mv, a.v, kDV, a.H, rows) || !make_map(&mg, a.g, kDK, a.H, rows) ||
       !make_map(&mb, a.bx, kDK, a.H, rows) || !make_map(&mdo, a.d_o, kDV, a.H, rows))
     return cudaErrorInvalidValue;
-  auto kern = a.dscale > 0.f ? bwd_tc_kernel<true> : bwd_tc_kernel<false>;
+  auto kern = a.dscale > 0.f ? (a.qknorm ? bwd_tc_kernel<true, true> : bwd_tc_kernel<true, false>)
+                             : (a.qknorm ? bwd_tc_kernel<false, true> : bwd_tc_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;

@@ -102,7 +102,12 @@ __device__ __forceinline__ void ld_chunk(const uint8_t* p, float* x) {
 // The log-decay prefix over the token groups is a shuffle scan inside each
 // warp plus the totals of the preceding warps (named barriers bar_id,
 // bar_id + 1 for the two column blocks).
-template <int NW, bool ACT = false>
+// QKN: q and k are first divided by their per-token L2 norms (sums of
+// squares over each thread's 8 channels, reduced over the 8 lanes of a
+// token and exchanged between the two column blocks through `nrm`, 1 KB,
+// across named barrier bar_n of the NW warps); the inverse norms go to
+// qn_out as fp16 pairs [t][k, q] (zero rows get 0).
+template <int NW, bool ACT = false, bool QKN = false>
 __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
                                                 uint8_t* kp,
                                                 const uint8_t* graw,
@@ -110,7 +115,10 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
                                                 float* s_gam, float* red,
                                                 int bar_id, uint32_t khs,
                                                 int bar_b, int n_b,
-                                                float dscale, int nvalid) {
+                                                float dscale, int nvalid,
+                                                float* nrm = nullptr,
+                                                __half* qn_out = nullptr,
+                                                int bar_n = 0) {
   constexpr int WPB = NW / 2;         // warps per column block
   constexpr int TPT = 64 / (4 * WPB); // tokens per thread
   constexpr int NG = 64 / TPT;        // token groups
@@ -127,6 +135,47 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
   auto offk = [&](int t) {
     return (uint32_t)(blk * khs + t * 128 + ((ch ^ (t & 7)) << 4));
   };
+  float ink[TPT], inq[TPT];
+#pragma unroll
+  for (int i = 0; i < TPT; ++i) ink[i] = inq[i] = 1.f;
+  if constexpr (QKN) {
+    float sk[TPT], sq[TPT];
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+      const int t = TPT * tg + i;
+      float kv[8], qv[8];
+      ld_chunk(x + off128(t), kv);
+      ld_chunk(x + off128(64 + t), qv);
+      sk[i] = sq[i] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sk[i] = fmaf(kv[e], kv[e], sk[i]);
+        sq[i] = fmaf(qv[e], qv[e], sq[i]);
+      }
+#pragma unroll
+      for (int o = 1; o < 8; o <<= 1) {
+        sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], o);
+        sq[i] += __shfl_xor_sync(0xffffffffu, sq[i], o);
+      }
+      if (ch == 0) {
+        nrm[(blk * 64 + t) * 2] = sk[i];
+        nrm[(blk * 64 + t) * 2 + 1] = sq[i];
+      }
+    }
+    bar_named(bar_n, NW * 32);
+#pragma unroll
+    for (int i = 0; i < TPT; ++i) {
+      const int t = TPT * tg + i;
+      const float tk = nrm[t * 2] + nrm[(64 + t) * 2];
+      const float tq = nrm[t * 2 + 1] + nrm[(64 + t) * 2 + 1];
+      ink[i] = tk > 0.f ? 1.0f / sqrtf(tk) : 0.f;
+      inq[i] = tq > 0.f ? 1.0f / sqrtf(tq) : 0.f;
+      if (blk == 0 && ch == 0) {
+        qn_out[t * 2] = __float2half_rn(ink[i]);
+        qn_out[t * 2 + 1] = __float2half_rn(inq[i]);
+      }
+    }
+  }
   float gl[TPT][8];  // inclusive log-decay sums inside the token group
 #pragma unroll
   for (int i = 0; i < TPT; ++i) {
@@ -175,6 +224,13 @@ __device__ __forceinline__ void transform_block(uint8_t* x, uint8_t* kh,
     ld_chunk(x + off128(t), kv);
     ld_chunk(x + off128(64 + t), qv);
     ld_chunk_h(bsm + off64(t), bv);
+    if constexpr (QKN) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        kv[e] *= ink[i];
+        qv[e] *= inq[i];
+      }
+    }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const float gam = __expf(ex[e] + gl[i][e]);

@@ -83,8 +83,7 @@ typedef struct {
                        * and k by their Euclidean norms over DK themselves
                        * (a fused prologue) and the backward returns the
                        * gradients of the raw q and k.  Other values:
-                       * CARVE_ERR_INVALID_ARG.  Training with 1 runs on
-                       * the generic kernels. */
+                       * CARVE_ERR_INVALID_ARG. */
   int32_t erase_form; /* 0: S' (I - k (b (.) k)^T) as above; 1: the other
                        * erase that acts on the key axis only,
                        * S' (I - (b (.) k) k^T) (the gated key reads the

@@ -78,7 +78,7 @@ def test_decay_scale_validation(lib):
     assert ws_bytes(lib, shape(qk_l2norm=1), 1) > 0
     for bad in (2, -1):
         assert call_fwd(lib, shape(qk_l2norm=bad), FAKE, 1 << 20) == 1, bad
-    # it runs the tensor-core forward, and trains on the generic kernels
+    # it runs (and trains) on the tensor-core kernels
     path = lambda **kw: lib.carve_fwd_path(ctypes.byref(shape(**kw))).decode()
     tc = dict(DK=128, DV=128, R=32, L=64, T=128, dtype=carve.CARVE_BF16)
     assert path(**dict(tc, qk_l2norm=1)) == "tc"
@@ -86,10 +86,10 @@ def test_decay_scale_validation(lib):
     assert path(**dict(tc, erase_form=1)) == "generic"
     for bad in (2, -1):
         assert call_fwd(lib, shape(erase_form=bad), FAKE, 1 << 20) == 1, bad
+    # the tensor-core backward normalises again from the raw rows: training
+    # with the flag keeps the same workspace as without it
     n_tc = ws_bytes(lib, shape(**tc), 1)
-    n_norm = ws_bytes(lib, shape(**dict(tc, qk_l2norm=1)), 1)
-    assert n_norm - ws_bytes(lib, shape(**dict(tc, qk_l2norm=1)), 0) >= \
-        2 * 3 * (128 // 64 + 1) * 128 * 128 * 4 and n_norm != n_tc
+    assert ws_bytes(lib, shape(**dict(tc, qk_l2norm=1)), 1) == n_tc
 
 
 def test_status_strings_and_path(lib):

@@ -39,7 +39,8 @@ CASES = [
     (1, 2, 128, 64, 64, 8, 64, "bf16"),
     (1, 2, 128, 64, 64, 8, 64, "fp32"),
     (2, 1, 96, 32, 48, 4, 16, "fp32"),
-    (1, 2, 192, 128, 128, 32, 64, "bf16"),   # tc forward; trains on generic
+    (1, 2, 192, 128, 128, 32, 64, "bf16"),   # tensor-core forward and backward
+    (2, 2, 256, 128, 128, 16, 128, "bf16"),  # the same, two blocks per chunk
 ]
 
 
@@ -47,6 +48,9 @@ CASES = [
 def test_fused_normalisation_fwd_bwd(case):
     B, H, T, DK, DV, R, L, dt = case
     cfg = dict(B=B, H=H, T=T, DK=DK, DV=DV, R=R, L=L)
+    if DK == DV == 128 and dt == "bf16":
+        assert carve.fwd_path(carve.make_shape(B, T, H, DK, DV, R, L, torch.bfloat16,
+                                               0.0, True)) == "tc"
     inp = _raw_qk(cfg, 141, DT[dt])
     tol = TOL[DT[dt]]
     assert_within(fwd_errors(inp, L, qk_l2norm=True), tol,
