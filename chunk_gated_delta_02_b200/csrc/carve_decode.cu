@@ -15,12 +15,12 @@
 // row of S is independent once the key-side vectors (q, exp g, k, b k) are
 // known, so a (sequence, head) pair runs as a cluster of kSplit CTAs, each
 // owning a quarter of the value rows: every CTA forms the key-side vectors
-// and the gate itself (they are small), and its warps stream their rows: a
-// warp holds a batch of rows in registers (each row read as coalesced
-// 128-byte segments), reduces S q and S' k with butterfly shuffles, and
-// writes the new row back.  The gate of every CTA reads all of m_c, which a
-// chunk's last token rewrites row by row, so the CTAs of a cluster meet
-// once after staging m_c and before any of them can write it.
+// and the gate itself (they are small) while its rows of S arrive in shared
+// memory by asynchronous copies (requested first, and holding no register
+// while in flight), then its warps take a row each in turn, reduce S q and
+// S' k with butterfly shuffles, and write the new row back.  The gate of every CTA reads all of m_c, which a
+// chunk's last token rewrites row by row, so at that token the CTAs of a
+// cluster meet once after staging m_c and before any of them can write it.
 #include <cuda_bf16.h>
 
 #include "carve_internal.cuh"
@@ -32,7 +32,6 @@ namespace {
 constexpr int kDecThreads = 128;   // 4 warps per CTA
 constexpr int kSplit = 4;          // CTAs (a cluster) per (sequence, head)
 constexpr int kDecWarps = kDecThreads / 32;
-constexpr int kRows = 8;           // value rows a warp holds at once (DK <= 128)
 
 __device__ __forceinline__ float allsum(float x) {
 #pragma unroll
@@ -92,27 +91,16 @@ __global__ void __launch_bounds__(kDecThreads)
   const int bseq = pair / a.H, h = pair - bseq * a.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   float* S = a.S + (size_t)pair * DV * DK;
-  constexpr int RW = NJ > 4 ? kRows / 2 : kRows;  // rows per batch in registers
-  // this CTA's value rows [rlo, rhi)
-  const int rq = (DV + kSplit - 1) / kSplit;
-  const int rlo = part * rq, rhi = min(DV, rlo + rq);
-
-  // the first batch of this warp's state rows: requested before anything
-  // else, so that the gate below runs while they are in flight
-  float sv[RW][NJ];
-  float osv = 0.f;  // lane r < RW: the running output sum of row r0 + r
+  // this CTA's value rows rlo .. rlo + nrow - 1 (DV is a multiple of 16,
+  // so rq is a multiple of 4 and each CTA's rows start on a 16-byte
+  // boundary of the output sums too)
+  const int rq = DV / kSplit;
+  const int rlo = part * rq, nrow = rq;
+  // the CTA's rows of S [nrow][DK] and of the running output sum [nrow],
+  // fp32, after m_c
+  float* s_S = s_mraw + DV;
+  float* s_os = s_S + (size_t)rq * DK;
   float* osum = a.osum + (size_t)pair * DV;
-  auto load_rows = [&](int r0) {
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-#pragma unroll
-      for (int c = 0; c < NJ; ++c) {
-        const int j = lane + 32 * c;
-        sv[r][c] = (r0 + r < rhi && j < DK) ? S[(size_t)(r0 + r) * DK + j] : 0.f;
-      }
-    osv = (lane < RW && r0 + lane < rhi) ? osum[r0 + lane] : 0.f;
-  };
-  load_rows(rlo + warp * RW);
 
   const TIn* q = static_cast<const TIn*>(a.q) + (size_t)pair * DK;
   const TIn* k = static_cast<const TIn*>(a.k) + (size_t)pair * DK;
@@ -154,7 +142,16 @@ __global__ void __launch_bounds__(kDecThreads)
     }
     ptx::cp_async_commit();
   }
-  ptx::cp_async_wait_all();
+  {  // then the state rows and their output sums (the newest group): they
+     // land while the gate is formed
+    const float* Sg = S + (size_t)rlo * DK;
+    const int ns = nrow * DK / 4;
+    for (int i = tid; i < ns; i += kDecThreads) ptx::cp_async16(s_S + 4 * i, Sg + 4 * i);
+    for (int i = tid; i < nrow / 4; i += kDecThreads)
+      ptx::cp_async16(s_os + 4 * i, osum + rlo + 4 * i);
+    ptx::cp_async_commit();
+  }
+  ptx::cp_async_wait_but_newest();
   __syncthreads();
   for (int j = tid; j < DK; j += kDecThreads) {
     s_q[j] = ldf(s_raw, j);
@@ -168,7 +165,9 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   __syncthreads();
   // every CTA of the pair has m_c: a chunk's last token may now rewrite it
-  ptx::cluster_sync();
+  // (only that token writes m, and chunk_end is the same for the whole
+  // cluster, so the other tokens skip the barrier)
+  if (chunk_end) ptx::cluster_sync();
   if (a.qknorm) {  // fused normalisation: q / |q|, k / |k| (warp 0 reduces)
     if (warp == 0) {
       float sq = 0.f, sk = 0.f;
@@ -261,31 +260,39 @@ __global__ void __launch_bounds__(kDecThreads)
     ewj[c] = a.erase ? kj[c] : kpj[c];
   }
   const float invL = 1.0f / (float)a.L;
-  for (int r0 = rlo + warp * RW; r0 < rhi; r0 += kDecWarps * RW) {
-    if (r0 != rlo + warp * RW) load_rows(r0);
+  ptx::cp_async_wait_all();  // this thread's state copies
+  __syncthreads();           // and everyone's
+  // warp w takes batches of RW consecutive local rows (w RW, then
+  // w RW + 4 RW, ...), a batch unrolled so that its rows' reductions
+  // overlap; lane r writes the per-row scalars of the batch's row r
+  constexpr int RW = NJ > 4 ? 4 : 8;
+  for (int rl0 = warp * RW; rl0 < nrow; rl0 += kDecWarps * RW) {
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
-      const int row = r0 + r;
-      float ov = 0.f, ev = 0.f;
+      const int rl = rl0 + r;
+      if (rl < nrow) {  // (warp-uniform)
+        const int row = rlo + rl;
+        float sv[NJ];
+        float ov = 0.f, ev = 0.f;
 #pragma unroll
-      for (int c = 0; c < NJ; ++c) {
-        ov = fmaf(sv[r][c], qj[c], ov);
-        sv[r][c] *= alj[c];  // S' = S Diag(exp g)
-        ev = fmaf(sv[r][c], erj[c], ev);
-      }
-      ov = allsum(ov);
-      ev = allsum(ev);
-      if (row < rhi) {
+        for (int c = 0; c < NJ; ++c) {
+          const int j = lane + 32 * c;
+          sv[c] = j < DK ? s_S[(size_t)rl * DK + j] : 0.f;
+          ov = fmaf(sv[c], qj[c], ov);
+          sv[c] *= alj[c];  // S' = S Diag(exp g)
+          ev = fmaf(sv[c], erj[c], ev);
+        }
+        ov = allsum(ov);
+        ev = allsum(ev);
         const float wv = w * s_v[row];
 #pragma unroll
         for (int c = 0; c < NJ; ++c) {
           const int j = lane + 32 * c;
-          if (j < DK)
-            S[(size_t)row * DK + j] = fmaf(-ev, ewj[c], fmaf(wv, kj[c], sv[r][c]));
+          if (j < DK) S[(size_t)row * DK + j] = fmaf(-ev, ewj[c], fmaf(wv, kj[c], sv[c]));
         }
-        if (lane == r) {  // spread the per-row scalars over the warp's lanes
+        if (lane == r) {
           stf(o, row, ov);
-          const float os = osv + ov;
+          const float os = s_os[rl] + ov;
           if (chunk_end) {
             m[row] = os * invL;
             osum[row] = 0.f;
@@ -326,7 +333,8 @@ template <typename TIn>
 cudaError_t launch_typed(const DecArgs& a, cudaStream_t st) {
   const size_t smem = (size_t)(5 * a.DK + 2 * a.DV + (a.R > 0 ? a.R : 1)) * 4 +
                       16 + (size_t)a.R * (a.DK + a.DV) * sizeof(TIn) +
-                      (size_t)(4 * a.DK + a.DV) * sizeof(TIn) + (size_t)a.DV * 4;
+                      (size_t)(4 * a.DK + a.DV) * sizeof(TIn) + (size_t)a.DV * 4 +
+                      (size_t)(a.DV / kSplit) * (a.DK + 1) * 4;
   if ((long long)a.B * a.H * kSplit > 0x7fffffffLL) return cudaErrorInvalidValue;
   if (a.DK <= 64) return launch_nj<TIn, 2>(a, smem, st);
   if (a.DK <= 128) return launch_nj<TIn, 4>(a, smem, st);
