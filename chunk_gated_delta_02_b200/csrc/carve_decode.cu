@@ -16,9 +16,9 @@
 // known, so a (sequence, head) pair runs as a cluster of kSplit CTAs, each
 // owning a quarter of the value rows: every CTA forms the key-side vectors
 // and the gate itself (they are small) while its rows of S arrive in shared
-// memory by asynchronous copies (requested first, and holding no register
-// while in flight), then its warps take a row each in turn, reduce S q and
-// S' k with butterfly shuffles, and write the new row back.  The gate of every CTA reads all of m_c, which a
+// memory by bulk copies (requested first, on the copy engine), then its
+// warps take batches of rows, reduce S q and S' k of a batch together by
+// shuffles, and write the new rows back.  The gate of every CTA reads all of m_c, which a
 // chunk's last token rewrites row by row, so at that token the CTAs of a
 // cluster meet once after staging m_c and before any of them can write it.
 #include <cuda_bf16.h>
@@ -32,10 +32,33 @@ namespace {
 constexpr int kDecThreads = 128;   // 4 warps per CTA
 constexpr int kSplit = 4;          // CTAs (a cluster) per (sequence, head)
 constexpr int kDecWarps = kDecThreads / 32;
+constexpr long long kDecWaitCycles = 1ll << 31;  // a copy wait gives up (~1 s)
 
 __device__ __forceinline__ float allsum(float x) {
 #pragma unroll
   for (int k = 16; k >= 1; k >>= 1) x += __shfl_xor_sync(0xffffffffu, x, k);
+  return x;
+}
+
+// Warp sums of N values at once (N = 8 or 16): lane l ends with the sum over
+// the warp of v[l % N] (N - 1 + log2(32 / N) shuffles instead of 5 N).  At
+// the step for bit k a lane keeps the half of its values whose index has
+// bit k equal to its own lane bit k, adding its partner's copy of them.
+template <int N>
+__device__ __forceinline__ float reduce_scatter(float* v, int lane) {
+#pragma unroll
+  for (int k = N / 2; k >= 1; k >>= 1) {
+    const bool up = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const float send = up ? v[i] : v[i + k];
+      const float keep = up ? v[i + k] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+    }
+  }
+  float x = v[0];
+#pragma unroll
+  for (int k = N; k < 32; k <<= 1) x += __shfl_xor_sync(0xffffffffu, x, k);
   return x;
 }
 
@@ -112,62 +135,74 @@ __global__ void __launch_bounds__(kDecThreads)
   const float w = ldf(static_cast<const TIn*>(a.w), pair);
   const bool chunk_end = (a.pos[bseq] + 1) % a.L == 0;
 
-  // the head's U_b factors -> shared memory by asynchronous 16-byte copies
-  // (R * DV and DK * R elements fill whole 16-byte chunks: DK, DV are
-  // multiples of 16), in flight with the state rows; then the token's
-  // vectors and m_c
-  if (R > 0) {
-    const uint8_t* udg = reinterpret_cast<const uint8_t*>(
-        static_cast<const TIn*>(a.u_down) + (size_t)h * R * DV);
-    const uint8_t* uug = reinterpret_cast<const uint8_t*>(
-        static_cast<const TIn*>(a.u_up) + (size_t)h * DK * R);
-    const int nd = R * DV * (int)sizeof(TIn) / 16, nu = DK * R * (int)sizeof(TIn) / 16;
-    for (int i = tid; i < nd; i += kDecThreads)
-      ptx::cp_async16(reinterpret_cast<uint8_t*>(s_ud) + 16 * i, udg + 16 * i);
-    for (int i = tid; i < nu; i += kDecThreads)
-      ptx::cp_async16(reinterpret_cast<uint8_t*>(s_uu) + 16 * i, uug + 16 * i);
+  // Everything the CTA reads comes in by bulk copies that thread 0 issues
+  // at once (the copy engine, not the load/store pipe the gate uses): the
+  // head's U_b factors, the token's vectors and m_c on mbarrier 0, then
+  // the CTA's rows of S and of the output sum on mbarrier 1, which land
+  // while the gate is formed.  Each barrier completes once (parity 0); a
+  // wait gives up after kDecWaitCycles, and a CTA whose copies did not
+  // land leaves S, m and the sums as they were and writes NaN to its o.
+  __shared__ __align__(8) uint64_t s_bar[2];
+  if (tid == 0) {
+    ptx::mbar_init(&s_bar[0], 1);
+    ptx::mbar_init(&s_bar[1], 1);
+    ptx::mbar_init_fence();
   }
-  {  // every 16-byte chunk of the vectors and of m_c in one batch of copies
-    const int cv = DK * (int)sizeof(TIn) / 16, cw = DV * (int)sizeof(TIn) / 16;
-    const int nc = 4 * cv + cw + DV / 4;
-    for (int i = tid; i < nc; i += kDecThreads) {
-      const int which = i < 4 * cv ? i / cv : (i < 4 * cv + cw ? 4 : 5);
-      const int ci = which < 4 ? i - which * cv : (which == 4 ? i - 4 * cv : i - 4 * cv - cw);
-      const void* src = which == 0 ? (const void*)q : which == 1 ? (const void*)k
-                      : which == 2 ? (const void*)g : which == 3 ? (const void*)bx
-                      : which == 4 ? (const void*)v : (const void*)m;
-      uint8_t* dst = which < 5 ? reinterpret_cast<uint8_t*>(s_raw + which * DK)
-                               : reinterpret_cast<uint8_t*>(s_mraw);
-      ptx::cp_async16(dst + 16 * ci, static_cast<const uint8_t*>(src) + 16 * ci);
-    }
-    ptx::cp_async_commit();
-  }
-  {  // then the state rows and their output sums (the newest group): they
-     // land while the gate is formed
-    const float* Sg = S + (size_t)rlo * DK;
-    const int ns = nrow * DK / 4;
-    for (int i = tid; i < ns; i += kDecThreads) ptx::cp_async16(s_S + 4 * i, Sg + 4 * i);
-    for (int i = tid; i < nrow / 4; i += kDecThreads)
-      ptx::cp_async16(s_os + 4 * i, osum + rlo + 4 * i);
-    ptx::cp_async_commit();
-  }
-  ptx::cp_async_wait_but_newest();
   __syncthreads();
-  for (int j = tid; j < DK; j += kDecThreads) {
-    s_q[j] = ldf(s_raw, j);
-    s_k[j] = ldf(s_raw + DK, j);
-    s_al[j] = ldf(s_raw + 2 * DK, j);
-    s_bx[j] = ldf(s_raw + 3 * DK, j);
+  if (tid == 0) {
+    constexpr uint32_t sz = sizeof(TIn);
+    ptx::mbar_expect_tx(&s_bar[0], (uint32_t)(R * (DV + DK) + 4 * DK + DV) * sz +
+                                       (uint32_t)DV * 4u);
+    if (R > 0) {
+      ptx::bulk_load(s_ud, static_cast<const TIn*>(a.u_down) + (size_t)h * R * DV,
+                     (uint32_t)(R * DV) * sz, &s_bar[0]);
+      ptx::bulk_load(s_uu, static_cast<const TIn*>(a.u_up) + (size_t)h * DK * R,
+                     (uint32_t)(DK * R) * sz, &s_bar[0]);
+    }
+    ptx::bulk_load(s_raw, q, (uint32_t)DK * sz, &s_bar[0]);
+    ptx::bulk_load(s_raw + DK, k, (uint32_t)DK * sz, &s_bar[0]);
+    ptx::bulk_load(s_raw + 2 * DK, g, (uint32_t)DK * sz, &s_bar[0]);
+    ptx::bulk_load(s_raw + 3 * DK, bx, (uint32_t)DK * sz, &s_bar[0]);
+    ptx::bulk_load(s_raw + 4 * DK, v, (uint32_t)DV * sz, &s_bar[0]);
+    ptx::bulk_load(s_mraw, m, (uint32_t)DV * 4u, &s_bar[0]);
+    ptx::mbar_expect_tx(&s_bar[1], (uint32_t)(nrow * DK + nrow) * 4u);
+    ptx::bulk_load(s_S, S + (size_t)rlo * DK, (uint32_t)(nrow * DK) * 4u, &s_bar[1]);
+    ptx::bulk_load(s_os, osum + rlo, (uint32_t)nrow * 4u, &s_bar[1]);
   }
-  for (int i = tid; i < DV; i += kDecThreads) {
-    s_v[i] = ldf(s_raw + 4 * DK, i);
-    s_m[i] = s_mraw[i];
+  // every thread waits on the barrier itself (measured: faster than one
+  // warp waiting while the others sit at the CTA barrier after it)
+  auto mwait = [&](uint64_t* bar) {
+    const long long t0 = clock64();
+    while (!ptx::mbar_try_wait(bar, 0))
+      if (clock64() - t0 > kDecWaitCycles) return false;
+    return true;
+  };
+  auto give_up = [&]() {  // after the last cluster barrier only
+    mwait(&s_bar[1]);  // the state copies land before the CTA leaves
+    for (int rl = tid; rl < nrow; rl += kDecThreads) stf(o, rlo + rl, __int_as_float(0x7fc00000));
+  };
+  const bool bad = __syncthreads_or(!mwait(&s_bar[0]));
+  if (!bad) {
+    for (int j = tid; j < DK; j += kDecThreads) {
+      s_q[j] = ldf(s_raw, j);
+      s_k[j] = ldf(s_raw + DK, j);
+      s_al[j] = ldf(s_raw + 2 * DK, j);
+      s_bx[j] = ldf(s_raw + 3 * DK, j);
+    }
+    for (int i = tid; i < DV; i += kDecThreads) {
+      s_v[i] = ldf(s_raw + 4 * DK, i);
+      s_m[i] = s_mraw[i];
+    }
   }
   __syncthreads();
   // every CTA of the pair has m_c: a chunk's last token may now rewrite it
   // (only that token writes m, and chunk_end is the same for the whole
-  // cluster, so the other tokens skip the barrier)
+  // cluster, so the other tokens skip the barrier; every CTA takes it)
   if (chunk_end) ptx::cluster_sync();
+  if (bad) {
+    give_up();
+    return;
+  }
   if (a.qknorm) {  // fused normalisation: q / |q|, k / |k| (warp 0 reduces)
     if (warp == 0) {
       float sq = 0.f, sk = 0.f;
@@ -192,51 +227,95 @@ __global__ void __launch_bounds__(kDecThreads)
   }
   for (int j = tid; j < DK; j += kDecThreads)
     s_al[j] = expf(decay_act(s_al[j], a.dscale));
-  // h = U_down m_c: four threads per rank, each over a quarter of the
-  // values (every thread takes every pass, so that the whole warp meets the
-  // shuffles; ranks past R add nothing)
-  for (int base = 0; base < R; base += kDecThreads / 4) {
-    const int r = base + (tid >> 2), q4 = tid & 3;
-    float acc = 0.f;
-    if (r < R) {  // a contiguous quarter of the row, 16-byte vectors
-      constexpr int VN = Vec<TIn>::N;
-      const int i0 = q4 * (DV / 4), i1 = i0 + DV / 4;
-      float a4[4] = {0.f, 0.f, 0.f, 0.f};
-      if ((DV / 4) % VN == 0) {
-        for (int i = i0; i < i1; i += VN) {
-          float u[VN];
-          Vec<TIn>::load(s_ud + (size_t)r * DV + i, u);
+  // h = U_down m_c and p = U_up h.  Where a factor's rows are a power of
+  // two (<= 32) of 16-byte chunks, a warp instruction reads 32 consecutive
+  // chunks (512 contiguous bytes: whole rows side by side, no bank
+  // conflict), each lane takes the dot product of its chunk, and the lanes
+  // of a row sum by shuffles; otherwise four threads per rank (h) and a
+  // thread per key channel (p).  Every lane of a warp takes every pass, so
+  // the whole warp meets the shuffles; rows past R (or DK) add nothing.
+  constexpr int VN = Vec<TIn>::N;
+  auto pow2 = [](int x) { return x >= 1 && x <= 32 && (x & (x - 1)) == 0; };
+  const int cpr_d = DV / VN, cpr_u = R / VN;  // 16-byte chunks per row
+  if (pow2(cpr_d)) {
+    const int sub = lane / cpr_d, ch = lane % cpr_d, rpi = 32 / cpr_d;
+    float mv[VN];
 #pragma unroll
-          for (int e = 0; e < VN; ++e) a4[e & 3] = fmaf(u[e], s_m[i + e], a4[e & 3]);
-        }
-      } else {
-        for (int i = i0; i < i1; ++i) a4[0] = fmaf(ldf(s_ud, r * DV + i), s_m[i], a4[0]);
+    for (int e = 0; e < VN; ++e) mv[e] = s_m[ch * VN + e];
+    for (int r0 = warp * rpi; r0 < R; r0 += kDecWarps * rpi) {
+      const int r = r0 + sub;
+      float acc = 0.f;
+      if (r < R) {
+        float u[VN];
+        Vec<TIn>::load(s_ud + (size_t)r * DV + ch * VN, u);
+#pragma unroll
+        for (int e = 0; e < VN; ++e) acc = fmaf(u[e], mv[e], acc);
       }
-      acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      for (int k = 1; k < cpr_d; k <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, k);
+      if (ch == 0 && r < R) s_h[r] = acc;
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (q4 == 0 && r < R) s_h[r] = acc;
+  } else {
+    for (int base = 0; base < R; base += kDecThreads / 4) {
+      const int r = base + (tid >> 2), q4 = tid & 3;
+      float acc = 0.f;
+      if (r < R) {  // a contiguous quarter of the row
+        const int i0 = q4 * (DV / 4), i1 = i0 + DV / 4;
+        float a4[4] = {0.f, 0.f, 0.f, 0.f};
+        if ((DV / 4) % VN == 0) {
+          for (int i = i0; i < i1; i += VN) {
+            float u[VN];
+            Vec<TIn>::load(s_ud + (size_t)r * DV + i, u);
+#pragma unroll
+            for (int e = 0; e < VN; ++e) a4[e & 3] = fmaf(u[e], s_m[i + e], a4[e & 3]);
+          }
+        } else {
+          for (int i = i0; i < i1; ++i) a4[0] = fmaf(ldf(s_ud, r * DV + i), s_m[i], a4[0]);
+        }
+        acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (q4 == 0 && r < R) s_h[r] = acc;
+    }
   }
   __syncthreads();
-  // p = U_up h (a thread per key channel, its row of U_up read as 16-byte
-  // vectors when the row fills whole ones), b = sigmoid(b_x + p), b k
-  constexpr int VN = Vec<TIn>::N;
-  for (int j = tid; j < DK; j += kDecThreads) {
-    float p4[4] = {0.f, 0.f, 0.f, 0.f};
-    if (R % VN == 0) {
-      for (int r = 0; r < R; r += VN) {
-        float u[VN];
-        Vec<TIn>::load(s_uu + (size_t)j * R + r, u);
-#pragma unroll
-        for (int e = 0; e < VN; ++e) p4[e & 3] = fmaf(u[e], s_h[r + e], p4[e & 3]);
-      }
-    } else {
-      for (int r = 0; r < R; ++r) p4[0] = fmaf(ldf(s_uu, j * R + r), s_h[r], p4[0]);
-    }
-    const float p = (p4[0] + p4[1]) + (p4[2] + p4[3]);
+  // b = sigmoid(b_x + p), b k
+  auto gate_j = [&](int j, float p) {
     const float bj = 1.0f / (1.0f + expf(-(s_bx[j] + p)));
     s_kp[j] = bj * s_k[j];
+  };
+  if (R % VN == 0 && pow2(cpr_u)) {
+    const int sub = lane / cpr_u, ch = lane % cpr_u, rpi = 32 / cpr_u;
+    float hv[VN];
+#pragma unroll
+    for (int e = 0; e < VN; ++e) hv[e] = s_h[ch * VN + e];
+    for (int j0 = warp * rpi; j0 < DK; j0 += kDecWarps * rpi) {
+      const int j = j0 + sub;
+      float acc = 0.f;
+      if (j < DK) {
+        float u[VN];
+        Vec<TIn>::load(s_uu + (size_t)j * R + ch * VN, u);
+#pragma unroll
+        for (int e = 0; e < VN; ++e) acc = fmaf(u[e], hv[e], acc);
+      }
+      for (int k = 1; k < cpr_u; k <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, k);
+      if (ch == 0 && j < DK) gate_j(j, acc);
+    }
+  } else {
+    for (int j = tid; j < DK; j += kDecThreads) {
+      float p4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (R % VN == 0) {
+        for (int r = 0; r < R; r += VN) {
+          float u[VN];
+          Vec<TIn>::load(s_uu + (size_t)j * R + r, u);
+#pragma unroll
+          for (int e = 0; e < VN; ++e) p4[e & 3] = fmaf(u[e], s_h[r + e], p4[e & 3]);
+        }
+      } else {
+        for (int r = 0; r < R; ++r) p4[0] = fmaf(ldf(s_uu, j * R + r), s_h[r], p4[0]);
+      }
+      gate_j(j, (p4[0] + p4[1]) + (p4[2] + p4[3]));
+    }
   }
   __syncthreads();
 
@@ -260,39 +339,50 @@ __global__ void __launch_bounds__(kDecThreads)
     ewj[c] = a.erase ? kj[c] : kpj[c];
   }
   const float invL = 1.0f / (float)a.L;
-  ptx::cp_async_wait_all();  // this thread's state copies
-  __syncthreads();           // and everyone's
+  if (__syncthreads_or(!mwait(&s_bar[1]))) {  // the state rows
+    give_up();
+    return;
+  }
   // warp w takes batches of RW consecutive local rows (w RW, then
-  // w RW + 4 RW, ...), a batch unrolled so that its rows' reductions
-  // overlap; lane r writes the per-row scalars of the batch's row r
+  // w RW + 4 RW, ...); the batch's 2 RW partial sums (S q and S' k of each
+  // row) are reduced together, lane i ending with sum i % (2 RW); lane r
+  // writes the per-row scalars of the batch's row r
   constexpr int RW = NJ > 4 ? 4 : 8;
   for (int rl0 = warp * RW; rl0 < nrow; rl0 += kDecWarps * RW) {
+    float red[2 * RW];
+    float sv[RW][NJ];
 #pragma unroll
     for (int r = 0; r < RW; ++r) {
       const int rl = rl0 + r;
+      float ov = 0.f, ev = 0.f;
+#pragma unroll
+      for (int c = 0; c < NJ; ++c) {
+        const int j = lane + 32 * c;
+        float x = (rl < nrow && j < DK) ? s_S[(size_t)rl * DK + j] : 0.f;
+        ov = fmaf(x, qj[c], ov);
+        x *= alj[c];  // S' = S Diag(exp g)
+        ev = fmaf(x, erj[c], ev);
+        sv[r][c] = x;
+      }
+      red[r] = ov;
+      red[RW + r] = ev;
+    }
+    const float tot = reduce_scatter<2 * RW>(red, lane);
+#pragma unroll
+    for (int r = 0; r < RW; ++r) {
+      const int rl = rl0 + r;
+      const float ev = __shfl_sync(0xffffffffu, tot, RW + r);
       if (rl < nrow) {  // (warp-uniform)
         const int row = rlo + rl;
-        float sv[NJ];
-        float ov = 0.f, ev = 0.f;
-#pragma unroll
-        for (int c = 0; c < NJ; ++c) {
-          const int j = lane + 32 * c;
-          sv[c] = j < DK ? s_S[(size_t)rl * DK + j] : 0.f;
-          ov = fmaf(sv[c], qj[c], ov);
-          sv[c] *= alj[c];  // S' = S Diag(exp g)
-          ev = fmaf(sv[c], erj[c], ev);
-        }
-        ov = allsum(ov);
-        ev = allsum(ev);
         const float wv = w * s_v[row];
 #pragma unroll
         for (int c = 0; c < NJ; ++c) {
           const int j = lane + 32 * c;
-          if (j < DK) S[(size_t)row * DK + j] = fmaf(-ev, ewj[c], fmaf(wv, kj[c], sv[c]));
+          if (j < DK) S[(size_t)row * DK + j] = fmaf(-ev, ewj[c], fmaf(wv, kj[c], sv[r][c]));
         }
-        if (lane == r) {
-          stf(o, row, ov);
-          const float os = s_os[rl] + ov;
+        if (lane == r) {  // tot is S q of row r here
+          stf(o, row, tot);
+          const float os = s_os[rl] + tot;
           if (chunk_end) {
             m[row] = os * invL;
             osum[row] = 0.f;

@@ -86,10 +86,6 @@ __device__ __forceinline__ void cp_async_commit() {
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
-// Wait until at most the newest group of this thread's copies is pending.
-__device__ __forceinline__ void cp_async_wait_but_newest() {
-  asm volatile("cp.async.wait_group 1;" ::: "memory");
-}
 
 // Untiled bulk copies (addresses 16-byte aligned, size a multiple of 16).
 // Global -> shared, completion counted on `bar` like the tiled loads.
