@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kDecThreads)
     }
   }
   for (int j = tid; j < DK; j += kDecThreads)
-    s_al[j] = expf(decay_act(s_al[j], a.dscale));
+    s_al[j] = __expf(decay_act(s_al[j], a.dscale));
   // h = U_down m_c and p = U_up h.  Where a factor's rows are a power of
   // two (<= 32) of 16-byte chunks, a warp instruction reads 32 consecutive
   // chunks (512 contiguous bytes: whole rows side by side, no bank
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kDecThreads)
   __syncthreads();
   // b = sigmoid(b_x + p), b k
   auto gate_j = [&](int j, float p) {
-    const float bj = 1.0f / (1.0f + expf(-(s_bx[j] + p)));
+    const float bj = 1.0f / (1.0f + __expf(-(s_bx[j] + p)));
     s_kp[j] = bj * s_k[j];
   };
   if (R % VN == 0 && pow2(cpr_u)) {
