@@ -140,8 +140,9 @@ carve_status carve_chunk_fwd(const carve_shape* shape,
 
 /*
  * Forward without training over packed sequences of different lengths
- * (variable-length batches; survey item NEXT-4, the chunk-0 rule of the
- * pages applying to each sequence from its own start).
+ * (variable-length batches: the chunk-0 rule of the CARVE technical
+ * summary, gist.science, section 5 (acknowledged limitation), applies to
+ * each sequence from its own start).
  *
  *   shape        : B = number of sequences, T = total packed tokens (any
  *                  T >= 0), the other fields as for carve_chunk_fwd
