@@ -39,7 +39,9 @@ carve_status check_shape(const carve_shape* s) {
 // normal use): CARVE_TEST_WAIT_CYCLES lowers the cycles a device-side wait
 // spins before it gives up; CARVE_TEST_STALL_BLOCK makes CTA 0 of the
 // tensor-core kernels redirect the MMA commit of that block to a barrier
-// nobody waits on, so that a wait runs out and the timeout path runs.
+// nobody waits on, so that a wait runs out and the timeout path runs (in
+// the decode step, any value >= 0 makes CTA 0 issue none of its first
+// group of copies).
 void test_knobs(long long* spin, int* stall_block) {
   *spin = kSpinCycles;
   *stall_block = -1;
@@ -282,6 +284,9 @@ carve_status carve_decode_step(const carve_shape* shape, const void* q,
   a.dscale = s.decay_scale;
   a.qknorm = s.qk_l2norm;
   a.erase = s.erase_form;
+  int stall_block = -1;
+  test_knobs(&a.wait_cycles, &stall_block);
+  a.stall = stall_block >= 0 ? 1 : 0;
   return launch_decode(a, s.dtype, (cudaStream_t)stream) == cudaSuccess
              ? CARVE_OK
              : CARVE_ERR_CUDA;

@@ -140,8 +140,9 @@ __global__ void __launch_bounds__(kDecThreads)
   // head's U_b factors, the token's vectors and m_c on mbarrier 0, then
   // the CTA's rows of S and of the output sum on mbarrier 1, which land
   // while the gate is formed.  Each barrier completes once (parity 0); a
-  // wait gives up after kDecWaitCycles, and a CTA whose copies did not
-  // land leaves S, m and the sums as they were and writes NaN to its o.
+  // wait gives up after a.wait_cycles (normally kDecWaitCycles), and a CTA
+  // whose copies did not land leaves S, m and the sums as they were and
+  // writes NaN to its o.
   __shared__ __align__(8) uint64_t s_bar[2];
   if (tid == 0) {
     ptx::mbar_init(&s_bar[0], 1);
@@ -149,10 +150,17 @@ __global__ void __launch_bounds__(kDecThreads)
     ptx::mbar_init_fence();
   }
   __syncthreads();
+  // (test only, a.stall: CTA 0 announces its first group's bytes but
+  // issues none of its copies, so that group never completes and the wait
+  // for it gives up; nothing of it is in flight when the CTA leaves)
+  const bool issue0 = !(a.stall && blockIdx.x == 0);
   if (tid == 0) {
     constexpr uint32_t sz = sizeof(TIn);
     ptx::mbar_expect_tx(&s_bar[0], (uint32_t)(R * (DV + DK) + 4 * DK + DV) * sz +
                                        (uint32_t)DV * 4u);
+  }
+  if (tid == 0 && issue0) {
+    constexpr uint32_t sz = sizeof(TIn);
     if (R > 0) {
       ptx::bulk_load(s_ud, static_cast<const TIn*>(a.u_down) + (size_t)h * R * DV,
                      (uint32_t)(R * DV) * sz, &s_bar[0]);
@@ -165,23 +173,26 @@ __global__ void __launch_bounds__(kDecThreads)
     ptx::bulk_load(s_raw + 3 * DK, bx, (uint32_t)DK * sz, &s_bar[0]);
     ptx::bulk_load(s_raw + 4 * DK, v, (uint32_t)DV * sz, &s_bar[0]);
     ptx::bulk_load(s_mraw, m, (uint32_t)DV * 4u, &s_bar[0]);
+  }
+  if (tid == 0) {
     ptx::mbar_expect_tx(&s_bar[1], (uint32_t)(nrow * DK + nrow) * 4u);
     ptx::bulk_load(s_S, S + (size_t)rlo * DK, (uint32_t)(nrow * DK) * 4u, &s_bar[1]);
     ptx::bulk_load(s_os, osum + rlo, (uint32_t)nrow * 4u, &s_bar[1]);
   }
   // every thread waits on the barrier itself (measured: faster than one
   // warp waiting while the others sit at the CTA barrier after it)
-  auto mwait = [&](uint64_t* bar) {
+  auto mwait = [&](uint64_t* bar, long long limit) {
     const long long t0 = clock64();
     while (!ptx::mbar_try_wait(bar, 0))
-      if (clock64() - t0 > kDecWaitCycles) return false;
+      if (clock64() - t0 > limit) return false;
     return true;
   };
   auto give_up = [&]() {  // after the last cluster barrier only
-    mwait(&s_bar[1]);  // the state copies land before the CTA leaves
+    // the state copies land before the CTA leaves (on the full limit)
+    mwait(&s_bar[1], kDecWaitCycles);
     for (int rl = tid; rl < nrow; rl += kDecThreads) stf(o, rlo + rl, __int_as_float(0x7fc00000));
   };
-  const bool bad = __syncthreads_or(!mwait(&s_bar[0]));
+  const bool bad = __syncthreads_or(!mwait(&s_bar[0], a.wait_cycles));
   if (!bad) {
     for (int j = tid; j < DK; j += kDecThreads) {
       s_q[j] = ldf(s_raw, j);
@@ -339,7 +350,7 @@ __global__ void __launch_bounds__(kDecThreads)
     ewj[c] = a.erase ? kj[c] : kpj[c];
   }
   const float invL = 1.0f / (float)a.L;
-  if (__syncthreads_or(!mwait(&s_bar[1]))) {  // the state rows
+  if (__syncthreads_or(!mwait(&s_bar[1], a.wait_cycles))) {  // the state rows
     give_up();
     return;
   }

@@ -227,6 +227,8 @@ struct DecArgs {
   float dscale;         // decay activation scale (0: g is the log-decay)
   int qknorm;           // 1: q, k are normalised inside the kernel
   int erase;            // 1: the other erase form S' (I - (b k) k^T)
+  long long wait_cycles;  // a copy wait gives up after this many cycles
+  int stall;            // test only: CTA 0 issues none of its first copies
 };
 cudaError_t launch_decode(const DecArgs& a, int dtype, cudaStream_t st);
 

@@ -271,9 +271,15 @@ carve_status carve_chunk_fwd_noalloc(const carve_shape* shape,
  * S' = S Diag(exp g), S = S' - (S' k)(b k)^T + w v k^T, osum += o, and when
  * (pos + 1) % L == 0: m = osum / L, osum = 0.  A sequence processed by
  * carve_chunk_fwd (T a multiple of L, final S_T and m_T) continues here with
- * S = S_T, m = m_T, osum = 0, pos = T.  One CTA per (sequence, head); no
- * workspace; asynchronous on `stream`.  Errors: INVALID_ARG, UNSUPPORTED,
- * CUDA (launch failure).
+ * S = S_T, m = m_T, osum = 0, pos = T.  A cluster of four CTAs per
+ * (sequence, head), each owning a quarter of the value rows; no workspace;
+ * asynchronous on `stream`.  Errors: INVALID_ARG, UNSUPPORTED, CUDA (launch
+ * failure).  With no workspace there is no status word: a CTA whose input
+ * copies have not landed after about 1 s (2^31 cycles) leaves its rows of
+ * S, m and osum as they were and writes NaN to its rows of o.  The test
+ * knobs of carve_get_status apply: CARVE_TEST_WAIT_CYCLES lowers that
+ * limit, and CARVE_TEST_STALL_BLOCK (any value >= 0) makes the first CTA
+ * (pair 0, rows 0 .. DV/4 - 1) issue none of its first group of copies.
  */
 carve_status carve_decode_step(const carve_shape* shape,
                                const void* q, const void* k, const void* v,

@@ -137,3 +137,52 @@ def test_decode_continues_the_chunk_forward():
     assert rel(S.cpu(), S_all.cpu()) < 1e-2
     assert rel(m.cpu(), m_all.cpu()) < 1e-2
     assert float(osum.abs().max()) == 0.0
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp32"])
+def test_decode_copy_wait_gives_up(dt, monkeypatch):
+    # Test-only knobs: CTA 0 (pair (0, 0), value rows 0 .. dv/4 - 1)
+    # announces its first group of copies but issues none, so its bounded
+    # wait (lowered to 2e5 cycles) gives up.  That CTA writes NaN to its
+    # rows of o and leaves its rows of S, m and the output sums as they
+    # were; every other output equals a normal step's bit for bit, and a
+    # normal step afterwards does too.  Sequence 0 is at a chunk's last
+    # token, so the CTA that gave up still meets its cluster's barrier.
+    B, H, DK, DV, R, L = 2, 2, 128, 128, 16, 4
+    dtype = DT[dt]
+    tok, ud, uu = _tokens(B, H, 1, DK, DV, R, 91, dtype)
+    gen = torch.Generator().manual_seed(92)
+    S0 = (torch.randn((B, H, DV, DK), generator=gen) * 0.3).cuda()
+    m0 = (torch.randn((B, H, DV), generator=gen) * 0.3).cuda()
+    os0 = (torch.randn((B, H, DV), generator=gen) * 0.3).cuda()
+    pos = torch.tensor([L - 1, 1], dtype=torch.int32, device="cuda")
+    x = [tok[n][0].cuda() for n in ("q", "k", "v", "g", "bx", "w")]
+    udd, uud = ud.cuda(), uu.cuda()
+
+    def step():
+        S, m, osum = S0.clone(), m0.clone(), os0.clone()
+        o = carve.decode_step(*x, udd, uud, L, pos, S, m, osum)
+        torch.cuda.synchronize()
+        return o.float(), S, m, osum
+
+    o_r, S_r, m_r, s_r = step()
+    monkeypatch.setenv("CARVE_TEST_WAIT_CYCLES", "200000")
+    monkeypatch.setenv("CARVE_TEST_STALL_BLOCK", "0")
+    o_s, S_s, m_s, s_s = step()
+    monkeypatch.delenv("CARVE_TEST_WAIT_CYCLES")
+    monkeypatch.delenv("CARVE_TEST_STALL_BLOCK")
+    rq = DV // 4
+    assert bool(torch.isnan(o_s[0, 0, :rq]).all())
+    keep = torch.ones_like(o_r, dtype=torch.bool)
+    keep[0, 0, :rq] = False
+    assert torch.equal(o_s[keep], o_r[keep])
+    assert not bool(torch.isnan(o_r).any())
+    for got, ref, before in ((S_s, S_r, S0), (m_s, m_r, m0), (s_s, s_r, os0)):
+        assert torch.equal(got[0, 0, :rq], before[0, 0, :rq])
+        assert not torch.equal(ref[0, 0, :rq], before[0, 0, :rq])
+        k2 = torch.ones(got.shape[:3], dtype=torch.bool, device=got.device)
+        k2[0, 0, :rq] = False
+        assert torch.equal(got[k2], ref[k2])
+    o_n, S_n, m_n, s_n = step()
+    assert torch.equal(o_n, o_r) and torch.equal(S_n, S_r)
+    assert torch.equal(m_n, m_r) and torch.equal(s_n, s_r)
