@@ -1,13 +1,14 @@
 """Benchmark of the CARVE chunk-parallel recurrent core on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--mode train|fwd]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--mode train|fwd|decode]
                     [--workload layer_1p3b|long_context|tiny] [--impl carve|reference]
                     [--chunk L] [--seq-len T] [--no-extras]
 
 One step = one pass of the whole hot path over one batch: the training-mode
 forward (chunk walk, gate, WY solve, state update, checkpoints) plus the
 backward (reverse chunk walk and the U_b gradient reduction) -- or the
-forward alone with --mode fwd.  Inputs are synthetic (seeded, the
+forward alone with --mode fwd, or the single-token decode step alone with
+--mode decode (its own line: the `decode` entry below).  Inputs are synthetic (seeded, the
 distributions of chunk_gated_delta_02_b200/inputs.py) and resident in HBM
 when the timed region starts; they are larger than the 126 MB L2.
 
@@ -18,6 +19,9 @@ launch stream, the same warm-up, clocks sampled throughout):
   sweep         that forward at chunk lengths 16, 32, 64, 128: tokens/s,
                 roofline fraction, kernel family and the oracle error on one
                 (sequence, head) pair per length
+  decode        the decode step of all 128 (sequence, head) pairs: back to
+                back in a CUDA graph over states evicted from L2, and single
+                steps after an L2 flush
   long_context  the B=1, H=16, T=65536, dv=256 forward, with the bound its
                 sequential chunk chain sets (--no-extras skips all three;
                 --seq-len / --chunk change the main workload for profiling)
@@ -357,6 +361,85 @@ def pair_error(carve, host, d, L, bh):
     return {"o": rel(o[b, :, h, :], oo), "S_T": rel(S_T[b, h], SS)}
 
 
+def decode_bench(carve, d, cfg, it, warmup, pk, stream):
+    """The decode step at the shape of `cfg` (one new token per (sequence,
+    head), the fp32 state read and written once): back to back in a CUDA
+    graph over cold states, and single steps after an L2 flush."""
+    B, H, DK, DV = (cfg[n] for n in ("B", "H", "DK", "DV"))
+    dev = d["q"].device
+    L = cfg["L"]
+    tok = {n: d[n][:, 0].contiguous() for n in ("q", "k", "v", "g", "bx", "w")}
+    Sd = torch.randn((B, H, DV, DK), device=dev) * 0.1
+    md = torch.zeros((B, H, DV), device=dev)
+    od = torch.zeros((B, H, DV), device=dev)
+    pos = torch.full((B,), 5, dtype=torch.int32, device=dev)
+    outd = torch.empty((B, H, DV), dtype=d["q"].dtype, device=dev)
+    step = lambda: carve.decode_step(tok["q"], tok["k"], tok["v"], tok["g"],
+                                     tok["bx"], tok["w"], d["u_down"],
+                                     d["u_up"], L, pos, Sd, md, od, o=outd)
+    # the state (B H DV DK fp32 = 8 MiB here) fits in L2: write a buffer
+    # larger than L2 between timed steps so that each reads S from HBM
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(it)]
+    for _ in range(warmup):
+        step()
+    for e0, e1 in evs:
+        flush.fill_(1)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    msd = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
+    del flush
+    # back to back: steps over 20 separate states (160 MiB, more than L2),
+    # each step reading a state the 19 before it evicted, captured in one
+    # CUDA graph (as a serving loop would run them, without a Python call
+    # per step); the average per step is the kernel's launch-to-launch time
+    n_st = 20
+    states = [torch.randn((B, H, DV, DK), device=dev) * 0.1 for _ in range(n_st)]
+    bstep = lambda i: carve.decode_step(tok["q"], tok["k"], tok["v"], tok["g"],
+                                        tok["bx"], tok["w"], d["u_down"],
+                                        d["u_up"], L, pos, states[i % n_st],
+                                        md, od, o=outd)
+    n_b = 4 * n_st
+    for i in range(n_st):
+        bstep(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(n_b):
+            bstep(i)
+    for _ in range(2):
+        graph.replay()
+    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    reps = 3
+    b0.record()
+    for _ in range(reps):
+        graph.replay()
+    b1.record()
+    torch.cuda.synchronize()
+    msb = b0.elapsed_time(b1) / (reps * n_b)
+    del graph, states
+    pairs = B * H
+    dec_bytes = pairs * (2 * DV * DK * 4 + 2 * (4 * DK + 2 * DV + 1)
+                         + 4 * DV * 4)
+    dec_flops = pairs * (6 * DV * DK + 2 * DV * DK)
+    rdec = roof_obj("carve_decode_step", dec_flops, dec_bytes, msb, pk)
+    return {
+        "workload": "layer_1p3b decode step (B=8, H=16, dk=dv=128, r=32, "
+                    "L=64; one token per sequence)",
+        "ms": msb, "tokens_per_s": B / (msb * 1e-3), "roofline": rdec,
+        "timing": "%d steps back to back in one CUDA graph over %d states "
+                  "(%.0f MiB, above L2), average per step" % (
+                      n_b, n_st, n_st * B * H * DV * DK * 4 / 2**20),
+        "single_step_ms": msd,
+        "single_step_timing": "median of %d single steps, L2 flushed before "
+                              "each (includes the launch)" % it,
+        "bytes_per_pair_step": dec_bytes / pairs}
+
+
 def extras(carve, args, pk, host, d, stream, fwd_ms_train):
     """Inference forward, chunk-length sweep and long-context forward at
     their full sizes (one GPU), each timed like the main step."""
@@ -409,80 +492,7 @@ def extras(carve, args, pk, host, d, stream, fwd_ms_train):
         del wsl
     out["sweep"] = sweep
 
-    # decode: one new token per (sequence, head) at the 1.3B-layer shape,
-    # fp32 state S read and written once per step
-    dev = d["q"].device
-    L = cfg["L"]
-    tok = {n: d[n][:, 0].contiguous() for n in ("q", "k", "v", "g", "bx", "w")}
-    Sd = torch.randn((B, H, DV, DK), device=dev) * 0.1
-    md = torch.zeros((B, H, DV), device=dev)
-    od = torch.zeros((B, H, DV), device=dev)
-    pos = torch.full((B,), 5, dtype=torch.int32, device=dev)
-    outd = torch.empty((B, H, DV), dtype=d["q"].dtype, device=dev)
-    step = lambda: carve.decode_step(tok["q"], tok["k"], tok["v"], tok["g"],
-                                     tok["bx"], tok["w"], d["u_down"],
-                                     d["u_up"], L, pos, Sd, md, od, o=outd)
-    # the state (B H DV DK fp32 = 8 MiB here) fits in L2: write a buffer
-    # larger than L2 between timed steps so that each reads S from HBM
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    evs = [(torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(it)]
-    for _ in range(args.warmup):
-        step()
-    for e0, e1 in evs:
-        flush.fill_(1)
-        e0.record(stream)
-        step()
-        e1.record(stream)
-    torch.cuda.synchronize()
-    msd = statistics.median(e0.elapsed_time(e1) for e0, e1 in evs)
-    del flush
-    # back to back: steps over 20 separate states (160 MiB, more than L2),
-    # each step reading a state the 19 before it evicted, captured in one
-    # CUDA graph (as a serving loop would run them, without a Python call
-    # per step); the average per step is the kernel's launch-to-launch time
-    n_st = 20
-    states = [torch.randn((B, H, DV, DK), device=dev) * 0.1 for _ in range(n_st)]
-    bstep = lambda i: carve.decode_step(tok["q"], tok["k"], tok["v"], tok["g"],
-                                        tok["bx"], tok["w"], d["u_down"],
-                                        d["u_up"], L, pos, states[i % n_st],
-                                        md, od, o=outd)
-    n_b = 4 * n_st
-    for i in range(n_st):
-        bstep(i)
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for i in range(n_b):
-            bstep(i)
-    for _ in range(2):
-        graph.replay()
-    b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    reps = 3
-    b0.record()
-    for _ in range(reps):
-        graph.replay()
-    b1.record()
-    torch.cuda.synchronize()
-    msb = b0.elapsed_time(b1) / (reps * n_b)
-    del graph, states
-    pairs = B * H
-    dec_bytes = pairs * (2 * DV * DK * 4 + 2 * (4 * DK + 2 * DV + 1)
-                         + 4 * DV * 4)
-    dec_flops = pairs * (6 * DV * DK + 2 * DV * DK)
-    rdec = roof_obj("carve_decode_step", dec_flops, dec_bytes, msb, pk)
-    out["decode"] = {
-        "workload": "layer_1p3b decode step (B=8, H=16, dk=dv=128, r=32, "
-                    "L=64; one token per sequence)",
-        "ms": msb, "tokens_per_s": B / (msb * 1e-3), "roofline": rdec,
-        "timing": "%d steps back to back in one CUDA graph over %d states "
-                  "(%.0f MiB, above L2), average per step" % (
-                      n_b, n_st, n_st * B * H * DV * DK * 4 / 2**20),
-        "single_step_ms": msd,
-        "single_step_timing": "median of %d single steps, L2 flushed before "
-                              "each (includes the launch)" % it,
-        "bytes_per_pair_step": dec_bytes / pairs}
+    out["decode"] = decode_bench(carve, d, cfg, it, args.warmup, pk, stream)
 
     # long_context: config 3 (dv = 256, S0 != 0), forward
     lc = WORKLOADS["long_context"]
@@ -525,7 +535,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--mode", choices=["train", "fwd"], default="train")
+    ap.add_argument("--mode", choices=["train", "fwd", "decode"], default="train",
+                    help="decode: the single-token decode step alone")
     ap.add_argument("--workload", default="layer_1p3b", choices=list(WORKLOADS))
     ap.add_argument("--impl", choices=["carve", "reference"], default="carve")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -555,6 +566,19 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     dtype = torch.bfloat16
+    if args.mode == "decode":
+        # the decode step reads one token per sequence: inputs of 64 tokens
+        host = rank_batch(dict(cfg, T=64), rank, dtype)
+        dd = {k: v.to(dev) for k, v in host.items()}
+        res = decode_bench(carve, dd, cfg, max(5, args.steps), args.warmup,
+                           peaks(), torch.cuda.current_stream(dev))
+        if rank == 0:
+            print(json.dumps({
+                "metric": "decode tokens/s (one new token per sequence)",
+                "value": res["tokens_per_s"], "unit": "tokens/s", "n_gpus": ws,
+                "mode": "decode", "higher_is_better": True, "data": "synthetic",
+                "dtype": "bf16", "decode": res}), flush=True)
+        return
     B, T, H, DK, DV, R, L = (cfg[n] for n in ("B", "T", "H", "DK", "DV", "R",
                                               "L"))
     host = rank_batch(cfg, rank, dtype)
