@@ -285,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* s_co = reinterpret_cast<float*>(sm + OFF_MY + 8192);
   float* s_eu = s_co + 128;
   float* s_u2 = s_co + 256;
+  float* s_eu2 = s_co + 384;  // E^T u over the block's tokens 32..63
   auto gate = [&](int c) {
     const int u = tid - 256;
     bar_named(6, 256);  // s_m visible to all of warps 8-15
@@ -600,26 +601,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       wait(B_M3, 7);
       tc_fence_after();
-      {  // E^T -> bf16 operand (negated by the MMAs that use it); E^T u
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
-          float vals[32];
-          tmem_ld32(tl + TM_D1 + part * 32, vals);
-          float eu = 0.f;
+      {  // E^T columns 0..31 -> bf16 operand (negated by the MMAs that use
+         // it) and their share of E^T u; warps 4-7 take columns 32..63
+        float vals[32];
+        tmem_ld32(tl + TM_D1, vals);
+        float eu = 0.f;
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            eu = fmaf(vals[e], s_u2[part * 32 + e] + s_u2[64 + part * 32 + e], eu);
-          if (part == 0) s_eu[row] = eu; else s_eu[row] += eu;
+        for (int e = 0; e < 32; ++e) eu = fmaf(vals[e], s_u2[e] + s_u2[64 + e], eu);
+        s_eu[row] = eu;
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8)
-            st_chunk(sm + OFF_RE + sw128_chunk(row, 0, part * 4 + c8, 128),
-                     vals + c8 * 8);
-        }
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_RE + sw128_chunk(row, 0, c8, 128), vals + c8 * 8);
       }
       fence_async_smem();
       tc_fence_before();
-      bar_named(2, 128);          // -E^T complete
-      bar_arrive_named(12, 512);  // E^T u -> warps 8-15
+      bar_arrive_named(12, 512);  // E^T u (first half) -> warps 8-15
+      bar_named(13, 256);         // -E^T complete (warps 4-7 wrote the rest)
       // ---- S4. MMA 3b: O^T -= E^T P_kap^T; MMA 4: S -= E^T kap^ (after
       //      S += W^T K^)
       wait(B_WK, 11);
@@ -762,8 +759,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_async_smem();
       tc_fence_before();
       bar_arrive_named(11, 256);  // R^T, u -> warps 0-3
-      bar_arrive_named(12, 512);  // c_O -> warps 8-15
       wait(B_M3, 17);  // MMA 3a: MY free for the next block; E formed
+      tc_fence_after();
+      {  // E^T columns 32..63 -> bf16 operand and their share of E^T u
+        float vals[32];
+        tmem_ld32(tl + TM_D1 + 32, vals);
+        float eu = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) eu = fmaf(vals[e], s_u2[32 + e] + s_u2[96 + e], eu);
+        s_eu2[row] = eu;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8)
+          st_chunk(sm + OFF_RE + sw128_chunk(row, 0, 4 + c8, 128), vals + c8 * 8);
+      }
+      fence_async_smem();
+      tc_fence_before();
+      bar_arrive_named(13, 256);  // -E^T second half -> warps 0-3
+      bar_arrive_named(12, 512);  // c_O, E^T u (second half) -> warps 8-15
       if (a.tc_rec) {
         // training: E [t][v] (K-major, the backward's operand layout) ->
         // the A buffer (T was read from it before MMA 3a) -> the record
@@ -915,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       //      m_{c+1} and the next chunk's gate p = U_up U_down m_{c+1}
       bar_named(12, 512);  // c_O (warps 4-7), E^T u (warps 0-3)
       if (u < 128) {
-        const float bs = s_co[u] - s_eu[u];
+        const float bs = s_co[u] - (s_eu[u] + s_eu2[u]);
         const float acc = (ib % bpc == 0) ? bs : s_m[u] + bs;
         s_m[u] = chunk_end ? acc * invL : acc;
       }
