@@ -128,3 +128,32 @@ def test_fused_normalisation_decode(dt):
     errs = {n: rel(np.concatenate(g_), np.concatenate(r_))
             for n, (g_, r_) in acc.items()}
     assert_within(errs, TOL[DT[dt]], "fused qk norm decode " + dt)
+
+
+@pytest.mark.parametrize("case", [(1, 2, 192, 128, 128, 32, 64),
+                                  (2, 2, 128, 64, 64, 8, 64)],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_fused_normalisation_with_fused_activation(case):
+    # both fused prologues at once: raw q, k and raw decay logits (the
+    # tensor-core kernels' instances with both at dk = dv = 128, the generic
+    # kernels at 64); the oracle applies the activation and the
+    # normalisation as separate steps before the recurrence
+    from chunk_gated_delta_02_b200.inputs import DECAY_SCALE
+    B, H, T, DK, DV, R, L = case
+    cfg = dict(B=B, H=H, T=T, DK=DK, DV=DV, R=R, L=L)
+    if DK == DV == 128:
+        assert carve.fwd_path(carve.make_shape(B, T, H, DK, DV, R, L, torch.bfloat16,
+                                               DECAY_SCALE, True)) == "tc"
+    inp = inputs(cfg, 151, torch.bfloat16, raw_decay=True)
+    gen = torch.Generator().manual_seed(152)
+    for n in ("q", "k"):
+        f = 0.5 + 1.5 * torch.rand(inp[n].shape[:-1] + (1,), generator=gen)
+        inp[n] = (inp[n].double() * f).to(torch.bfloat16)
+    for n in ("u_down", "u_up"):
+        inp[n] = (inp[n].float() * 25.0).to(torch.bfloat16)
+    assert_within(fwd_errors(inp, L, decay_scale=DECAY_SCALE, qk_l2norm=True),
+                  1e-2, "fused qk norm + decay fwd %s" % (case,))
+    gro = grad_outputs(cfg, 153, torch.bfloat16)
+    assert_within(bwd_errors(inp, L, gro, du_heads=range(H), decay_scale=DECAY_SCALE,
+                             qk_l2norm=True),
+                  1e-2, "fused qk norm + decay bwd %s" % (case,))
