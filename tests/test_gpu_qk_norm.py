@@ -157,3 +157,21 @@ def test_fused_normalisation_with_fused_activation(case):
     assert_within(bwd_errors(inp, L, gro, du_heads=range(H), decay_scale=DECAY_SCALE,
                              qk_l2norm=True),
                   1e-2, "fused qk norm + decay bwd %s" % (case,))
+
+
+def test_fused_normalisation_layer_1p3b_training():
+    # the 1.3B-layer shape (B = 8, H = 16, T = 4096) with raw q, k and the
+    # fused normalisation, trained on the tensor cores: the oracle checks
+    # two sampled pairs (the corners) and the dU of head 3 over the batch
+    from chunk_gated_delta_02_b200.inputs import WORKLOADS, sample_pairs
+    cfg = WORKLOADS["layer_1p3b"]
+    inp = inputs(cfg, 161, torch.bfloat16)
+    gen = torch.Generator().manual_seed(162)
+    for n in ("q", "k"):
+        f = 0.5 + 1.5 * torch.rand(inp[n].shape[:-1] + (1,), generator=gen)
+        inp[n] = (inp[n].double() * f).to(torch.bfloat16)
+    gro = grad_outputs(cfg, 163, torch.bfloat16)
+    pairs = sample_pairs(cfg["B"], cfg["H"], 2, seed=161)
+    assert_within(bwd_errors(inp, cfg["L"], gro, pairs=pairs, du_heads=[3],
+                             qk_l2norm=True), 1e-2,
+                  "fused qk norm 1.3B-layer fwd+bwd")
