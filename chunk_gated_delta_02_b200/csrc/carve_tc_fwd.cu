@@ -137,8 +137,10 @@ static __device__ __noinline__ void keys_w8(uint8_t* x, uint8_t* kh,
 // 0 issues MMAs 3a, 3b, 4; thread 128 D1 and MMA 2; thread 256 the copies,
 // S += W^T K^ and the Grams.
 // ACT: the instance for raw decay logits (decay_scale > 0); the other one
-// has no activation code at all
-template <bool ACT>
+// has no activation code at all.  SHORT: the instance for blocks shorter
+// than 64 tokens (chunks of 16, 32, 48), which forms kap^ for the block's
+// rows only; the full-block instance keeps its 64-row loop
+template <bool ACT, bool SHORT>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_tc_kernel(const FwdArgs a, const __grid_constant__ CUtensorMap tm_q,
                   const __grid_constant__ CUtensorMap tm_k,
@@ -222,6 +224,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint4 z = make_uint4(0u, 0u, 0u, 0u);
     for (int i = tid; i < 32768 / 16; i += kThreads)
       *reinterpret_cast<uint4*>(sm + OFF_X + 16 * i) = z;
+    // [K^; kap^] too: kap^ is formed for rows 0..C-1 only, its other rows
+    // stay zero
+    for (int i = tid; i < 32768 / 16; i += kThreads)
+      *reinterpret_cast<uint4*>(sm + OFF_KHP + 16 * i) = z;
     for (int i = tid; i < 49152 / 16; i += kThreads)
       *reinterpret_cast<uint4*>(sm + OFF_RV + 16 * i) = z;  // RV, RG, RB
     fence_async_smem();
@@ -452,7 +458,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // block nb next to K^, then (thread 256) both Grams in one product,
   // G = [K~; Q~] [K^; kap^]^T -> [M; P_k | A; P_kap]
   auto kappa_g = [&](int nb, int kid, int nthr) {
-    tc::kappa_in_place(sm + OFF_KHP, sm + OFF_RB, s_p, 16384, kid, nthr);
+    // short blocks: kap^ only for the block's C rows (the rest of its slot
+    // was zeroed at entry); full blocks keep the 64-row loop
+    tc::kappa_in_place(sm + OFF_KHP, sm + OFF_RB, s_p, 16384, kid, nthr, SHORT ? C : kBlk);
     fence_async_smem();
     bar_named(9, nthr);
     if (tid == 256 && !*s_abort) {
@@ -1009,7 +1017,11 @@ cudaError_t launch_fwd_tc(const FwdArgs& a, cudaStream_t st) {
       !make_map(&mv, a.v, a.DV, a.H, rows, C) || !make_map(&mg, a.g, kDK, a.H, rows, C) ||
       !make_map(&mb, a.bx, kDK, a.H, rows, C) || !make_map(&mo, a.o, a.DV, a.H, rows, C))
     return cudaErrorInvalidValue;
-  auto kern = a.dscale > 0.f ? fwd_tc_kernel<true> : fwd_tc_kernel<false>;
+  // instances: the fused decay activation or not, and blocks shorter than
+  // 64 tokens (chunks of 16, 32, 48) or not, chosen here
+  const bool act = a.dscale > 0.f, sh = C < kBlk;
+  auto kern = act ? (sh ? fwd_tc_kernel<true, true> : fwd_tc_kernel<true, false>)
+                  : (sh ? fwd_tc_kernel<false, true> : fwd_tc_kernel<false, false>);
   cudaError_t e = cudaFuncSetAttribute(
       kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;

@@ -403,12 +403,13 @@ __device__ __forceinline__ void transform_keys(uint8_t* x, uint8_t* kh,
 // slot: `kh` holds K^ in rows 0..63 of each 128-row column block (blocks
 // `khs` bytes apart) and kap^ goes to rows 64..127 of the same blocks.
 // Thread t_id of n_thr takes 16-byte chunks t_id, t_id + n_thr, ... of the
-// 64 x 128 tile; the 8 threads of a quarter-warp take the 8 chunks of one
+// first `nrows` token rows of the 64 x 128 tile (the caller keeps the rows
+// past them zero); the 8 threads of a quarter-warp take the 8 chunks of one
 // row (conflict-free under the swizzle).
 __device__ __forceinline__ void kappa_in_place(uint8_t* kh, const uint8_t* braw,
                                                const float* s_p, uint32_t khs,
-                                               int t_id, int n_thr) {
-  for (int c = t_id; c < 1024; c += n_thr) {
+                                               int t_id, int n_thr, int nrows = 64) {
+  for (int c = t_id; c < 16 * nrows; c += n_thr) {
     const int t = c >> 4, blk = (c >> 3) & 1, ch = c & 7;
     const uint32_t sw = (uint32_t)(t * 128 + ((ch ^ (t & 7)) << 4));
     float kv[8], bv[8], o[8];
